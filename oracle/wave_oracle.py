@@ -1,0 +1,386 @@
+"""Wave-index oracle: a plain, slow, fp64 restatement of the method.
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, the package-level smoke check and the
+bench's CPU-baseline leg may import this module.  It shares no code with the
+CUDA path (no kernels, helpers, tables or pre/post-processing) and imports
+nothing from it.
+
+Sources (page title, section):
+  [RI]  "RetroInfer: A Vector Storage Engine for Scalable Long-Context LLM
+        Inference" (technical summary), section 2.A "Wave Index": item 1
+        Steady Zone, item 2 Retrieval Zone, item 3 Estimation Zone, and the
+        Segmented Clustering paragraph.
+  [VX]  "Vortex - Servizio di Attention Sparsa Efficiente e Programmabile per
+        Agenti AI", section 2.A (two-phase forward_cache / forward_indexer;
+        primitives GeMM, Softmax, Top-K, Gather) and 2.B (vTensor layout).
+  [IC]  "IceCache: Memory-Efficient KV-cache Management for Long-Sequence
+        LLMs" (catalog summary): attention sinks and the decoded tail stay
+        resident; pages are filled by similarity, not position.
+
+Readings where the pages are silent (each is listed in the design doc):
+  R-1 k-means distance is squared Euclidean on the raw keys.
+  R-2 a segment of n tokens gets ceil(n/cs) centroids, centroid j starts as the
+      key at segment position j*cs; `iters` rounds of (assign, update); an
+      empty cluster keeps its centroid; the stored centroid is the mean of the
+      final assignment.
+  R-3 every token is counted once: steady tokens are removed from the clusters
+      they belong to, both when a cluster is retrieved (they are skipped) and
+      when it is estimated (count and value sum are reduced); clusters left
+      with no non-steady token are neither candidates nor estimated.
+  R-4 GQA: q head h reads KV head floor(h/G); a cluster's selection score for a
+      KV head is the max over the group's q heads; each q head estimates with
+      its own score.
+  R-5 k per (sequence, KV head) = topk_clusters, or ceil(fraction * NC).
+  R-6 ties (top-k and argmin) go to the lower index.
+  R-7 centroids and value sums are stored in the KV dtype (round to nearest
+      even from the exact mean / sum); decode reads the stored values.
+  R-8 softmax scale 1/sqrt(d); no causal mask at decode.
+
+Parity pins for every function here live in tests/test_oracle_pins.py.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import List, Optional, Tuple
+
+import numpy as np
+
+
+# ---------------------------------------------------------------------------
+# Rounding to the stored dtype (reading R-7)
+# ---------------------------------------------------------------------------
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bfloat16 (ties to even), returned as fp64.
+
+    bfloat16 keeps 8 significant bits and fp32's exponent range; below 2^-126
+    the spacing stays 2^-133 (subnormals).  Overflow goes to +-inf.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    nz = (x != 0) & np.isfinite(x)
+    _, e = np.frexp(x[nz])                       # x = m * 2^e, 0.5 <= |m| < 1
+    quantum = np.ldexp(1.0, np.maximum(e - 1, -126) - 7)
+    out[nz] = np.rint(x[nz] / quantum) * quantum  # np.rint rounds half to even
+    out[~nz] = x[~nz]
+    big = np.abs(out) > 3.3895313892515355e38     # largest finite bfloat16
+    out[big] = np.sign(out[big]) * np.inf
+    return out
+
+
+def round_stored(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Round to the KV storage dtype ('bf16' or 'f32'), kept as fp64 values."""
+    if dtype == "bf16":
+        return round_bf16(x)
+    if dtype == "f32":
+        return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+    raise ValueError(dtype)
+
+
+# ---------------------------------------------------------------------------
+# Segmented clustering ([RI] 2.A, Segmented Clustering paragraph)
+# ---------------------------------------------------------------------------
+
+def segment_spans(T: int, seg_len: int) -> List[Tuple[int, int]]:
+    """The sequence is cut into consecutive segments of seg_len tokens; the last
+    one may be shorter.  Returns (start, length) pairs."""
+    return [(s, min(seg_len, T - s)) for s in range(0, T, seg_len)]
+
+
+def clusters_in_segment(length: int, cluster_size: int) -> int:
+    """R-2: ceil(length / cluster_size) centroids per segment."""
+    return -(-length // cluster_size)
+
+
+def n_clusters(T: int, seg_len: int, cluster_size: int) -> int:
+    return sum(clusters_in_segment(n, cluster_size) for _, n in segment_spans(T, seg_len))
+
+
+def kmeans_init(X: np.ndarray, cluster_size: int) -> np.ndarray:
+    """R-2: centroid j starts as the key at segment position j*cluster_size."""
+    m = clusters_in_segment(len(X), cluster_size)
+    return X[np.arange(m) * cluster_size].astype(np.float64).copy()
+
+
+def kmeans_assign(X: np.ndarray, C: np.ndarray) -> np.ndarray:
+    """Assignment step: each key goes to argmin_j ||x - c_j||^2 (R-1), the
+    lowest j on ties (R-6).  The squared distance is expanded as
+    ||x||^2 - 2 x.c + ||c||^2 and evaluated with an fp64 matrix product."""
+    X = np.asarray(X, dtype=np.float64)
+    C = np.asarray(C, dtype=np.float64)
+    dist = (X * X).sum(1)[:, None] - 2.0 * (X @ C.T) + (C * C).sum(1)[None, :]
+    return np.argmin(dist, axis=1)               # argmin returns the first minimum
+
+
+def kmeans_distances(X: np.ndarray, C: np.ndarray) -> np.ndarray:
+    """||x_i - c_j||^2 for all pairs (fp64), used by near-tie checks."""
+    X = np.asarray(X, dtype=np.float64)
+    C = np.asarray(C, dtype=np.float64)
+    return (X * X).sum(1)[:, None] - 2.0 * (X @ C.T) + (C * C).sum(1)[None, :]
+
+
+def kmeans_update(X: np.ndarray, labels: np.ndarray, C_prev: np.ndarray) -> np.ndarray:
+    """Update step: each centroid becomes the mean of its members; a centroid
+    with no member keeps its previous value (R-2)."""
+    X = np.asarray(X, dtype=np.float64)
+    m = len(C_prev)
+    counts = np.bincount(labels, minlength=m)
+    sums = np.zeros_like(C_prev, dtype=np.float64)
+    np.add.at(sums, labels, X)
+    C = np.array(C_prev, dtype=np.float64, copy=True)
+    nz = counts > 0
+    C[nz] = sums[nz] / counts[nz, None]
+    return C
+
+
+def kmeans_objective(X: np.ndarray, labels: np.ndarray, C: np.ndarray) -> float:
+    """Sum of squared distances of each key to its assigned centroid."""
+    diff = np.asarray(X, dtype=np.float64) - np.asarray(C, dtype=np.float64)[labels]
+    return float((diff * diff).sum())
+
+
+def kmeans_segment(X: np.ndarray, cluster_size: int, iters: int, C0: Optional[np.ndarray] = None):
+    """Lloyd iterations on one segment: `iters` rounds of (assign, update).
+
+    Returns (labels of the last assignment, centroids = means of that
+    assignment, objective after every assign and every update)."""
+    if iters < 1:
+        raise ValueError("iters must be >= 1")
+    C = kmeans_init(X, cluster_size) if C0 is None else np.array(C0, dtype=np.float64)
+    history = []
+    labels = None
+    for _ in range(iters):
+        labels = kmeans_assign(X, C)
+        history.append(kmeans_objective(X, labels, C))
+        C = kmeans_update(X, labels, C)
+        history.append(kmeans_objective(X, labels, C))
+    return labels, C, history
+
+
+@dataclass
+class UnitIndex:
+    """The wave index of one (sequence, KV head): the query-independent phase
+    ([VX] 2.A forward_cache) of the method."""
+    centroids: np.ndarray      # [NC][d] stored dtype values (fp64 array)
+    value_sums: np.ndarray     # [NC][d] stored dtype values
+    offsets: np.ndarray        # [NC+1] int64, slot range of each cluster
+    perm: np.ndarray           # [T] slot -> original position
+    invperm: np.ndarray        # [T] original position -> slot
+    k_perm: np.ndarray         # [T][d] keys in slot order
+    v_perm: np.ndarray         # [T][d] values in slot order
+    labels: np.ndarray         # [T] global cluster id of each original position
+    centroids_exact: np.ndarray  # [NC][d] fp64 means before rounding
+    value_sums_exact: np.ndarray  # [NC][d] fp64 sums before rounding
+
+
+def build_unit(K: np.ndarray, V: np.ndarray, seg_len: int, cluster_size: int, iters: int,
+               store: str, kmeans_iters_hook=None) -> UnitIndex:
+    """Index build for one (sequence, KV head): segmented k-means ([RI] 2.A),
+    then the cluster-permuted layout the retrieval zone reads.
+
+    Cluster ids are global: the clusters of segment s follow those of s-1.
+    Slots are cluster-major; inside a cluster, members keep ascending original
+    position.  Because clusters never cross a segment, segment s occupies the
+    same slot range as its position range.
+    """
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    T, d = K.shape
+    labels = np.empty(T, dtype=np.int64)
+    cents = []
+    base = 0
+    for start, n in segment_spans(T, seg_len):
+        lab, C, _ = kmeans_segment(K[start:start + n], cluster_size, iters)
+        labels[start:start + n] = lab + base
+        cents.append(C)
+        base += len(C)
+    NC = base
+    C = np.concatenate(cents, 0) if cents else np.zeros((0, d))
+    counts = np.bincount(labels, minlength=NC)
+    offsets = np.zeros(NC + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    perm = np.argsort(labels, kind="stable")     # cluster-major, positions ascending
+    invperm = np.empty(T, dtype=np.int64)
+    invperm[perm] = np.arange(T)
+    vsum = np.zeros((NC, d))
+    np.add.at(vsum, labels, V)
+    return UnitIndex(centroids=round_stored(C, store), value_sums=round_stored(vsum, store),
+                     offsets=offsets, perm=perm, invperm=invperm, k_perm=K[perm], v_perm=V[perm],
+                     labels=labels, centroids_exact=C, value_sums_exact=vsum)
+
+
+# ---------------------------------------------------------------------------
+# Decode: steady, retrieval and estimation zones ([RI] 2.A items 1-3)
+# ---------------------------------------------------------------------------
+
+def steady_positions(T: int, n_sink: int, window: int) -> np.ndarray:
+    """Steady zone ([RI] 2.A item 1; [IC] sinks and tail resident): the first
+    n_sink positions and the last `window` positions, each counted once."""
+    pos = set(range(min(n_sink, T))) | set(range(max(T - window, 0), T))
+    return np.array(sorted(pos), dtype=np.int64)
+
+
+def k_for(NC: int, topk_clusters: int, topk_fraction: float) -> int:
+    """R-5: a fixed k, or ceil(fraction * NC) computed in double precision."""
+    if topk_clusters >= 0:
+        return int(topk_clusters)
+    return int(math.ceil(float(topk_fraction) * NC))
+
+
+def select_topk(a: np.ndarray, candidate: np.ndarray, k: int) -> np.ndarray:
+    """Retrieval zone selection ([RI] 2.A item 2; [VX] 2.A Top-K): the k
+    candidates with the largest score, lower index first on equal scores
+    (R-6).  k is clamped to the number of candidates.  Returned ascending."""
+    idx = [c for c in range(len(a)) if candidate[c]]
+    idx.sort(key=lambda c: (-a[c], c))
+    return np.array(sorted(idx[:k]), dtype=np.int64)
+
+
+def zone_stats(scores: np.ndarray, weights: np.ndarray, values: np.ndarray):
+    """One softmax part: m = max score, l = sum_i w_i e^(s_i - m),
+    o = sum_i e^(s_i - m) value_i.  An empty part is (-inf, 0, 0)."""
+    G = scores.shape[0]
+    d = values.shape[1]
+    if scores.shape[1] == 0:
+        return np.full(G, -np.inf), np.zeros(G), np.zeros((G, d))
+    m = scores.max(1)
+    e = np.exp(scores - m[:, None])
+    return m, (e * weights[None, :]).sum(1), e @ values
+
+
+def lse_merge(parts):
+    """Log-sum-exp combine of softmax parts (m_i, l_i, o_i): with m = max m_i,
+    out = sum e^(m_i-m) o_i / sum e^(m_i-m) l_i and lse = m + ln(denominator)."""
+    ms = np.stack([p[0] for p in parts])         # [P][G]
+    m = ms.max(0)
+    G = m.shape[0]
+    d = parts[0][2].shape[1]
+    num = np.zeros((G, d))
+    den = np.zeros(G)
+    for (mi, li, oi) in parts:
+        f = np.where(np.isfinite(mi), np.exp(mi - np.where(np.isfinite(m), m, 0.0)), 0.0)
+        num += f[:, None] * oi
+        den += f * li
+    with np.errstate(divide="ignore", invalid="ignore"):
+        out = np.where(den[:, None] > 0, num / np.where(den > 0, den, 1.0)[:, None], 0.0)
+        lse = np.where(den > 0, m + np.log(np.where(den > 0, den, 1.0)), -np.inf)
+    return out, lse
+
+
+@dataclass
+class DecodeTrace:
+    out: np.ndarray          # [G][d]
+    lse: np.ndarray          # [G]
+    selected: np.ndarray     # ascending cluster ids
+    scores: np.ndarray       # [G][NC] q.kbar / sqrt(d)
+    sel_score: np.ndarray    # [NC] max over the group
+    candidate: np.ndarray    # [NC] bool
+    k: int
+    exact: tuple             # (m, l, o) of the exact part
+    estimate: tuple          # (m, l, o) of the estimation part
+
+
+def decode_unit(q: np.ndarray, ix: UnitIndex, n_sink: int, window: int, k: int,
+                selected: Optional[np.ndarray] = None) -> DecodeTrace:
+    """One decode step of one KV head's query group ([VX] 2.A forward_indexer).
+
+    q: [G][d] query heads of the group (values as fed to the kernel).
+    (a) score every centroid: s[h,c] = q_h . kbar_c / sqrt(d);
+    (b) select the top-k clusters on max_h s[h,c] among candidates (R-3, R-4);
+    (c) exact attention over the steady zone plus the non-steady members of the
+        selected clusters ([RI] item 1 and item 2);
+    (d) every other candidate cluster c contributes cnt'_c * e^(s[h,c]) with
+        value sum Vsum'_c ([RI] item 3: the cluster counted |C| times at its
+        centroid score, times its mean value);
+    (e) the two parts are combined by log-sum-exp.
+    `selected` overrides step (b) (used to compare downstream steps on a given set).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    G, d = q.shape
+    T = len(ix.perm)
+    NC = len(ix.centroids)
+    scale = 1.0 / math.sqrt(d)
+
+    steady_pos = steady_positions(T, n_sink, window)
+    is_steady_pos = np.zeros(T, dtype=bool)
+    is_steady_pos[steady_pos] = True
+    steady_slots = ix.invperm[steady_pos]
+    cl_of_slot = np.searchsorted(ix.offsets, steady_slots, side="right") - 1
+    dcnt = np.bincount(cl_of_slot, minlength=NC) if NC else np.zeros(0, dtype=np.int64)
+    dv = np.zeros((NC, d))
+    np.add.at(dv, cl_of_slot, ix.v_perm[steady_slots])
+    cnt = np.diff(ix.offsets)
+    cnt_p = cnt - dcnt
+    vsum_p = ix.value_sums - dv
+    candidate = cnt_p > 0
+
+    s = (q @ ix.centroids.T) * scale             # [G][NC]
+    a = s.max(0) if NC else np.zeros(0)
+    if selected is None:
+        sel = select_topk(a, candidate, k)
+    else:
+        sel = np.asarray(selected, dtype=np.int64)
+    is_sel = np.zeros(NC, dtype=bool)
+    is_sel[sel] = True
+
+    # exact part: selected clusters' non-steady slots, then the steady slots
+    ex = []
+    for c in sel:
+        for slot in range(ix.offsets[c], ix.offsets[c + 1]):
+            if not is_steady_pos[ix.perm[slot]]:
+                ex.append(slot)
+    ex = np.array(ex + list(steady_slots), dtype=np.int64)
+    s_ex = (q @ ix.k_perm[ex].T) * scale
+    exact = zone_stats(s_ex, np.ones(len(ex)), ix.v_perm[ex])
+
+    # estimation part: candidates not selected
+    X = np.nonzero(candidate & ~is_sel)[0]
+    estimate = zone_stats(s[:, X], cnt_p[X].astype(np.float64), vsum_p[X])
+
+    out, lse = lse_merge([exact, estimate])
+    return DecodeTrace(out=out, lse=lse, selected=sel, scores=s, sel_score=a,
+                       candidate=candidate, k=k, exact=exact, estimate=estimate)
+
+
+def dense_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray):
+    """Full softmax attention of q [G][d] over all T tokens (no mask)."""
+    q = np.asarray(q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    s = (q @ K.T) / math.sqrt(q.shape[1])
+    m = s.max(1)
+    e = np.exp(s - m[:, None])
+    l = e.sum(1)
+    return (e @ V) / l[:, None], m + np.log(l)
+
+
+# ---------------------------------------------------------------------------
+# Batched helpers: (sequence, KV head) units of a workload
+# ---------------------------------------------------------------------------
+
+def build_all(keys, values, seg_len, cluster_size, iters, store) -> List[List[UnitIndex]]:
+    """keys[b], values[b]: [Hkv][T_b][d].  Returns index[b][hkv]."""
+    return [[build_unit(kb[h], vb[h], seg_len, cluster_size, iters, store)
+             for h in range(kb.shape[0])] for kb, vb in zip(keys, values)]
+
+
+def decode_all(q: np.ndarray, index, n_sink, window, topk_clusters, topk_fraction):
+    """q: [B][Hq][d].  Returns out [B][Hq][d], lse [B][Hq], traces[b][hkv]."""
+    B, Hq, d = q.shape
+    Hkv = len(index[0])
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, d))
+    lse = np.zeros((B, Hq))
+    traces = []
+    for b in range(B):
+        tb = []
+        for h in range(Hkv):
+            ix = index[b][h]
+            k = k_for(len(ix.centroids), topk_clusters, topk_fraction)
+            tr = decode_unit(q[b, h * G:(h + 1) * G], ix, n_sink, window, k)
+            out[b, h * G:(h + 1) * G] = tr.out
+            lse[b, h * G:(h + 1) * G] = tr.lse
+            tb.append(tr)
+        traces.append(tb)
+    return out, lse, traces

@@ -1,0 +1,437 @@
+"""Wave-index sparse decode benchmark (one decode step of one layer = one step).
+
+Default workload: one Llama-3-8B-shaped layer, bf16 KV, batch 1, 32 q / 8 KV
+heads, head_dim 128, 131072 tokens of context, segments of 8192, 16 tokens per
+cluster (8192 clusters per KV head), 10 k-means rounds, steady zone 4 sinks +
+64 recent tokens, top 1.8% of clusters retrieved (148 per KV head), page 16.
+
+The index is built once on the GPU (timed separately, reported under
+"build"), then cloned into R layer replicas; timed steps rotate through the
+replicas so each step's ~44 MB working set was evicted from the 126 MB L2 by
+the steps in between (R * step bytes > 2 * L2).
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--impl wave|reference]
+Multi-GPU: one process per GPU under torch.distributed.run; every rank runs
+its own independent replica workload (no collective on the data path), the
+step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-decode µs/step/layer + achieved HBM GB/s (% of roofline), 128K–1M ctx"
+UNIT = "us/step/layer"
+FALLBACK_HBM_GBS = 6650.0
+# FP32 CUDA-core peak for the build's assignment (148 SMs x 128 lanes x 2 flop x 1.965 GHz)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def workload_args(cfg: int):
+    import wave_inputs as WI
+    names = {1: "tiny fp32, T=4096, d=64, 1 q / 1 KV head",
+             2: "Llama-3-8B-shaped layer, bf16, B=1, T=131072, 32q/8kv, d=128",
+             3: "batched decode, bf16, B=16 x T=32768, 32q/8kv, d=128",
+             4: "long context, bf16, B=1, T=1048576, 32q/8kv, d=128",
+             5: "ragged paged batch, bf16, 8 seqs log-uniform in [4096, 262144]"}
+    return names[cfg]
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}",
+                                          f"--query-gpu={self.QUERY}", "--format=csv,noheader",
+                                          "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1].split()[0]))
+                mx = float(parts[2].split()[0])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- helpers
+
+def algorithmic_bytes(index, params, info: np.ndarray, n_st_per_seq):
+    """Bytes the method must move in one decode step (centroids, value sums,
+    offsets, retrieved K/V rows + perm, steady K/V rows + invperm, q, out, lse)."""
+    e = 2 if index.dtype == torch.bfloat16 else 4
+    d = index.head_dim
+    H = index.n_kv_heads
+    per_stage = {"score": 0, "estimate": 0, "attend": 0}
+    total = 0
+    for b, T in enumerate(index.seq_lens):
+        NC = index.nc[b]
+        cent = H * NC * d * e
+        vs = H * NC * d * e
+        offs = H * (NC + 1) * 4
+        sel_tok = int(sum(info[b * H + h, 3] for h in range(H)))
+        dense = bool(info[b * H, 6])
+        st = T if dense else n_st_per_seq[b]
+        retr = sel_tok * (2 * d * e + 4)
+        steady = H * st * (2 * d * e + 4)
+        qo = params.n_q_heads * d * e + params.n_q_heads * (d + 1) * 4
+        per_stage["score"] += cent + offs + params.n_q_heads * d * e
+        per_stage["estimate"] += vs + offs
+        per_stage["attend"] += retr + steady
+        total += cent + vs + offs + retr + steady + qo
+    return total, per_stage
+
+
+def steady_count(T, n_sink, window):
+    ns = min(n_sink, T)
+    ws = max(T - window, ns)
+    return ns + (T - ws)
+
+
+def clone_index(wx):
+    import copy
+    c = copy.copy(wx)
+    for name in ["centroids", "value_sums", "offsets", "perm", "invperm", "k_pool", "v_pool"]:
+        setattr(c, name, getattr(wx, name).clone())
+    return c
+
+
+# ----------------------------------------------------------------- wave arm
+
+def run_wave(args, rank, world, local_rank):
+    import retrieval_sparse_attention_wave_b200 as W
+    import wave_inputs as WI
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = WI.config(args.config, device=dev, seed=None if rank == 0 else 1000 * rank + args.config)
+    # paged input cache, contiguous block table
+    bt, n_pages = WI.make_block_table(wl.seq_lens, wl.page_size,
+                                      shuffle_seed=(5 if args.config == 5 else None))
+    kv = W.KVCache(WI.to_pages(wl.keys, bt, n_pages, wl.page_size),
+                   WI.to_pages(wl.values, bt, n_pages, wl.page_size),
+                   torch.as_tensor(bt, device=dev), list(wl.seq_lens))
+    wl.keys = wl.values = None
+    bt_out, n_out = WI.make_block_table(wl.seq_lens, wl.page_size,
+                                        shuffle_seed=(6 if args.config == 5 else None))
+    bt_out = torch.as_tensor(bt_out, device=dev)
+
+    # build (cold, once), timed with events
+    W.build_index(kv, wl.seg_len, wl.cluster_size, 1, block_table=bt_out, n_pages=n_out)  # warm
+    torch.cuda.synchronize()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record()
+    wx = W.build_index(kv, wl.seg_len, wl.cluster_size, wl.iters, block_table=bt_out,
+                       n_pages=n_out)
+    b1.record()
+    torch.cuda.synchronize()
+    build_ms = b0.elapsed_time(b1)
+    assert W.read_device_status(wx._build_ws) == 0
+    del kv
+    torch.cuda.empty_cache()
+
+    params = W.DecodeParams(n_q_heads=wl.n_q_heads, n_sink=wl.n_sink, window=wl.window,
+                            topk_clusters=wl.topk_clusters, topk_fraction=wl.topk_fraction)
+    q = wl.q.to(dev)
+    ws = W.decode_workspace(wx, params)
+    lay = W.decode_layout(wx, params)
+    n_units = wl.batch * wl.n_kv_heads
+
+    # per-step bytes; replicas so that R * step bytes > 2 * L2
+    W.decode(q, wx, params, ws=ws)
+    torch.cuda.synchronize()
+    info = W.unit_info(ws, lay, n_units).cpu().numpy()
+    n_st = [steady_count(T, wl.n_sink, wl.window) for T in wl.seq_lens]
+    step_bytes, stage_bytes = algorithmic_bytes(wx, params, info, n_st)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = max(2, math.ceil(2 * l2 / step_bytes) + 2) if args.replicas <= 0 else args.replicas
+    reps = [wx] + [clone_index(wx) for _ in range(R - 1)]
+    outs = [torch.empty(wl.batch, wl.n_q_heads, wl.head_dim, dtype=torch.float32, device=dev)
+            for _ in range(R)]
+    lses = [torch.empty(wl.batch, wl.n_q_heads, dtype=torch.float32, device=dev)
+            for _ in range(R)]
+
+    stream = torch.cuda.Stream(device=dev)
+    graphs = []
+    with torch.cuda.stream(stream):
+        for r in range(R):                      # warm every replica before capture
+            W.decode(q, reps[r], params, out=outs[r], lse=lses[r], ws=ws, stream=stream)
+        stream.synchronize()
+        if not args.no_graph:
+            for r in range(R):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    W.decode(q, reps[r], params, out=outs[r], lse=lses[r], ws=ws, stream=stream)
+                graphs.append(g)
+
+    def step(i):
+        r = i % R
+        if graphs:
+            graphs[r].replay()
+        else:
+            W.decode(q, reps[r], params, out=outs[r], lse=lses[r], ws=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+
+    dist = world > 1
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+    stream.synchronize()
+    clk = clocks.stop()
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    us_per_step = ms * 1e3 / args.steps
+
+    # per-stage device time (ungraphed launches, events on the launching stream)
+    nst = W.lib().wi_decode_stage_count()
+    names = W.stage_names()
+    acc = np.zeros(nst)
+    n_prof = max(20, min(200, args.steps))
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
+    with torch.cuda.stream(stream):
+        for i in range(n_prof):
+            r = i % R
+            W.decode(q, reps[r], params, out=outs[r], lse=lses[r], ws=ws, stream=stream,
+                     stage_events=evs)
+            evs[-1].synchronize()
+            acc += [evs[j].elapsed_time(evs[j + 1]) for j in range(nst)]
+    stage_us = {names[j]: acc[j] * 1e3 / n_prof for j in range(nst)}
+
+    # end to end through the public API with host buffers
+    q_h = wl.q.cpu().pin_memory()
+    out_h = torch.empty(wl.batch, wl.n_q_heads, wl.head_dim, dtype=torch.float32).pin_memory()
+    lse_h = torch.empty(wl.batch, wl.n_q_heads, dtype=torch.float32).pin_memory()
+    n_e2e = max(10, min(args.steps, 200))
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            W.decode_host(q_h, reps[i % R], params, out_h, lse_h, ws, stream=stream)
+        stream.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(n_e2e):
+            W.decode_host(q_h, reps[i % R], params, out_h, lse_h, ws, stream=stream)
+            stream.synchronize()                 # the host reads this step's result
+        f1.record(stream)
+        stream.synchronize()
+    e2e_us = f0.elapsed_time(f1) * 1e3 / n_e2e
+    assert np.isfinite(out_h.numpy()).all()
+    assert W.read_device_status(ws, stream) == 0
+
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    dom = max(("score", "estimate", "attend"), key=lambda k: stage_us[k])
+    dom_gbs = stage_bytes[dom] / (stage_us[dom] * 1e-6) / 1e9
+    step_gbs = step_bytes / (us_per_step * 1e-6) / 1e9
+    tokens = sum(wl.seq_lens)
+    assign_flop = 2.0 * sum(wl.seq_lens) * wl.n_kv_heads * (wl.seg_len // wl.cluster_size) \
+        * wl.head_dim * wl.iters
+    result = {
+        "metric": METRIC,
+        "value": us_per_step / world,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": us_per_step / 1e3,
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded Gaussian-mixture keys, N(0,1) values)",
+        "config": {"workload": workload_args(args.config), "batch": wl.batch,
+                   "context": wl.seq_lens if wl.batch > 1 else wl.seq_lens[0],
+                   "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads,
+                   "head_dim": wl.head_dim, "seg_len": wl.seg_len,
+                   "cluster_size": wl.cluster_size, "topk_fraction": wl.topk_fraction,
+                   "n_sink": wl.n_sink, "window": wl.window,
+                   "l2": f"rotate {R} layer replicas ({R * step_bytes / 1e6:.0f} MB per cycle > 2x L2)",
+                   "cuda_graph": not args.no_graph, "parallelism": f"replicas{world}"},
+        "tokens_per_s": tokens * world / (us_per_step * 1e-6),
+        "hbm_gbs": step_gbs,
+        "step_bytes": step_bytes,
+        "roofline_step": {"achieved": step_gbs, "peak": hbm, "unit": "GB/s",
+                          "frac": step_gbs / hbm, "peak_kind": peak_kind},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": dom_gbs, "peak": hbm,
+                     "unit": "GB/s", "frac": dom_gbs / hbm, "traffic": None,
+                     "bytes_per_launch": stage_bytes[dom], "us_per_launch": stage_us[dom],
+                     "peak_kind": peak_kind},
+        "stage_us": stage_us,
+        "gpu_launches": nst * args.steps,
+        "e2e": {"value": e2e_us, "unit": UNIT,
+                "h2d_bytes_per_step": int(q_h.numel() * q_h.element_size()),
+                "d2h_bytes_per_step": int(out_h.numel() * 4 + lse_h.numel() * 4)},
+        "build": {"ms": build_ms, "iters": wl.iters, "assign_tflop": assign_flop / 1e12,
+                  "assign_tflops_achieved": assign_flop / (build_ms * 1e-3) / 1e12,
+                  "bound": "alu", "peak_tflops": FP32_ALU_TFLOPS},
+        "clocks": clk,
+    }
+    return result, wx, wl
+
+
+# ----------------------------------------------------------------- oracle arm
+
+def oracle_timing(cfg: int, budget_s: float):
+    """Time the fp64 oracle decode on host cores on a bounded sample: the index
+    of one (sequence, KV head) unit built by the oracle, then decode steps of
+    that unit until the budget is spent; scaled to a whole layer step."""
+    import oracle as O
+    import wave_inputs as WI
+    wl = WI.config(cfg, device="cpu")
+    G = wl.n_q_heads // wl.n_kv_heads
+    b, h = 0, 0
+    K = wl.keys[b][h].to(torch.float64).numpy()
+    V = wl.values[b][h].to(torch.float64).numpy()
+    store = "bf16" if wl.dtype == torch.bfloat16 else "f32"
+    t0 = time.perf_counter()
+    ix = O.build_unit(K, V, wl.seg_len, wl.cluster_size, wl.iters, store)
+    build_s = time.perf_counter() - t0
+    qg = wl.q[b, h * G:(h + 1) * G].to(torch.float64).numpy()
+    k = O.k_for(len(ix.centroids), wl.topk_clusters, wl.topk_fraction)
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        O.decode_unit(qg, ix, wl.n_sink, wl.window, k)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    units = wl.batch * wl.n_kv_heads
+    us_step = el / n * units * 1e6
+    cores = len(os.sched_getaffinity(0))
+    return {"value": us_step, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"unit (b=0, kv head 0) of {units}; oracle-built index "
+                      f"({wl.iters} rounds, {build_s:.1f} s); {n} decode steps in {el:.1f} s, "
+                      f"x{units} units per layer step",
+            "build_s_per_unit": build_s}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--impl", default="wave", choices=["wave", "reference"])
+    ap.add_argument("--replicas", type=int, default=0)
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        # the oracle arm: rank 0 alone times the fp64 oracle on host cores
+        if rank != 0:
+            return
+        steps = max(1, args.steps)
+        cb = oracle_timing(args.config, budget_s=min(args.cpu_budget, 60.0))
+        res = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT,
+               "n_gpus": world, "steps": steps, "warmup": args.warmup,
+               "ms_per_step": cb["value"] / 1e3, "higher_is_better": False,
+               "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+               "data": "synthetic (seeded Gaussian-mixture keys, N(0,1) values)",
+               "config": {"workload": workload_args(args.config)},
+               "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+               "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                       "d2h_bytes_per_step": 0}}
+        print(json.dumps(res))
+        return
+
+    if world > 1:
+        from datetime import timedelta
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        res, _, _ = run_wave(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                cb = oracle_timing(args.config, budget_s=args.cpu_budget)
+                res["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind",
+                                                          "sample")}
+            print(json.dumps(res))
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

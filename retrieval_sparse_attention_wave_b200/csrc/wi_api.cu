@@ -1,0 +1,435 @@
+// C ABI of libwi.so: argument validation, launch plans, workspace layout.
+// Every argument error is detected here, on the host, before any CUDA call.
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <algorithm>
+#include <mutex>
+
+#include "wi.h"
+#include "wi_common.cuh"
+#include "wi_plan.h"
+
+namespace wi {
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+wi_status cuda_fail(cudaError_t e) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return WI_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+int ilog2(int x) { int r = 0; while ((1 << r) < x) ++r; return r; }
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int64_t clusters_of(int64_t T, int S, int cs) {
+  const int64_t full = T / S, rem = T % S;
+  return full * (S / cs) + cdiv(rem, cs);
+}
+
+int esize(wi_dtype d) { return d == WI_BF16 ? 2 : 4; }
+
+// Common geometry checks for a paged pool description.
+wi_status check_common(wi_dtype dtype, int batch, int hkv, int d, int page, int64_t n_pages,
+                       const void* kp, const void* vp, const int32_t* bt, int max_pages,
+                       const int32_t* seq_lens) {
+  if (dtype != WI_F32 && dtype != WI_BF16) return WI_ERR_INVALID_ARG;
+  if (batch < 1 || hkv < 1 || d < 1 || page < 1 || n_pages < 1 || max_pages < 1)
+    return WI_ERR_INVALID_ARG;
+  if (batch > kMaxBatch) return WI_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return WI_ERR_UNSUPPORTED;
+  if (!pow2(page) || page > 1024) return WI_ERR_INVALID_ARG;
+  if (!kp || !vp || !bt || !seq_lens) return WI_ERR_INVALID_ARG;
+  if (!aligned(kp, 16) || !aligned(vp, 16) || !aligned(bt, 4)) return WI_ERR_INVALID_ARG;
+  int64_t tot = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t T = seq_lens[b];
+    if (T < 1) return WI_ERR_INVALID_ARG;
+    if (cdiv(T, page) > max_pages) return WI_ERR_INVALID_ARG;
+    tot += T;
+  }
+  if (tot * hkv > INT32_MAX) return WI_ERR_UNSUPPORTED;
+  return WI_OK;
+}
+
+wi_status check_seg(int S, int cs) {
+  if (S < 1 || cs < 1 || S % cs != 0) return WI_ERR_INVALID_ARG;
+  if (S > WI_MAX_SEG_LEN) return WI_ERR_UNSUPPORTED;
+  return WI_OK;
+}
+
+void fill_geo(Geo& g, int batch, int hkv, int d, const int32_t* seq_lens, int S, int cs) {
+  std::memset(&g, 0, sizeof(g));
+  g.batch = batch; g.hkv = hkv; g.d = d;
+  for (int b = 0; b < batch; ++b) {
+    g.tok_base[b + 1] = g.tok_base[b] + seq_lens[b];
+    g.cl_base[b + 1] = g.cl_base[b] + (int32_t)clusters_of(seq_lens[b], S, cs);
+  }
+}
+
+int64_t n_steady(int64_t T, int64_t n_sink, int64_t window) {
+  const int64_t ns = std::min(n_sink, T);
+  const int64_t ws = std::max(T - window, ns);
+  return ns + (T - ws);
+}
+
+int rows_per_warp(int dtype, int D) {
+  const int epl = 16 / esize((wi_dtype)dtype);
+  return 32 / (D / epl);
+}
+
+wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, DecodePlan& pl) {
+  if (!ix || !p) return WI_ERR_INVALID_ARG;
+  wi_status st = check_common(ix->dtype, ix->batch, ix->n_kv_heads, ix->head_dim, ix->page_size,
+                              ix->n_pages, ix->k_pool, ix->v_pool, ix->block_table,
+                              ix->max_pages, ix->seq_lens);
+  if (st != WI_OK) return st;
+  if ((st = check_seg(ix->seg_len, ix->cluster_size)) != WI_OK) return st;
+  if (!ix->centroids || !ix->value_sums || !ix->offsets || !ix->perm || !ix->invperm)
+    return WI_ERR_INVALID_ARG;
+  if (!aligned(ix->centroids, 16) || !aligned(ix->value_sums, 16) || !aligned(ix->offsets, 4) ||
+      !aligned(ix->perm, 4) || !aligned(ix->invperm, 4))
+    return WI_ERR_INVALID_ARG;
+  if (p->n_q_heads < 1 || p->n_q_heads % ix->n_kv_heads != 0) return WI_ERR_INVALID_ARG;
+  const int G = p->n_q_heads / ix->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return WI_ERR_UNSUPPORTED;
+  if (p->n_sink < 0 || p->window < 0) return WI_ERR_INVALID_ARG;
+  if (p->topk_clusters < 0 && !(p->topk_fraction >= 0.0 && p->topk_fraction <= 1.0))
+    return WI_ERR_INVALID_ARG;
+
+  std::memset(&pl, 0, sizeof(pl));
+  fill_geo(pl.geo, ix->batch, ix->n_kv_heads, ix->head_dim, ix->seq_lens, ix->seg_len,
+           ix->cluster_size);
+  pl.dtype = ix->dtype; pl.D = ix->head_dim; pl.G = G; pl.Hq = p->n_q_heads;
+  pl.U = ix->batch * ix->n_kv_heads;
+  pl.n_sink = p->n_sink; pl.window = p->window;
+  pl.topk_clusters = p->topk_clusters; pl.topk_fraction = p->topk_fraction;
+  pl.scale = 1.0f / std::sqrt((float)ix->head_dim);
+
+  int max_nc = 0, cap = 1;
+  int64_t max_tok = 1;
+  for (int b = 0; b < ix->batch; ++b) {
+    const int T = ix->seq_lens[b];
+    const int nc = pl.geo.NC(b);
+    max_nc = std::max(max_nc, nc);
+    const int64_t nst = n_steady(T, p->n_sink, p->window);
+    int64_t k = p->topk_clusters >= 0 ? p->topk_clusters
+                                      : (int64_t)std::ceil(p->topk_fraction * (double)nc);
+    k = std::min<int64_t>(k, nc);
+    if (nst >= T) {
+      max_tok = std::max<int64_t>(max_tok, T);
+    } else {
+      if (nst > WI_MAX_STEADY) return WI_ERR_UNSUPPORTED;
+      cap = std::max<int>(cap, (int)nst);
+      max_tok = std::max<int64_t>(max_tok, std::min<int64_t>(T, k * ix->cluster_size + nst));
+    }
+  }
+  pl.max_nc = max_nc;
+  pl.cap = cap;
+  pl.sort_pow2 = 1;
+  while (pl.sort_pow2 < cap) pl.sort_pow2 <<= 1;
+
+  // score: ~8 CTAs of 256 threads per SM
+  const int rows_it = 8 * rows_per_warp(pl.dtype, pl.D) * 4;
+  const int64_t total_rows = (int64_t)max_nc * pl.U;
+  const int64_t iters = std::max<int64_t>(1, cdiv(total_rows, (int64_t)rows_it * kNumSMs * 8));
+  pl.score_chunk = (int)(rows_it * iters);
+  pl.n_score_blocks = (int)cdiv(max_nc, pl.score_chunk);
+  // exact attention: ~2 CTAs per SM overall, at least ~128 tokens per CTA
+  int ns = (int)cdiv(2 * kNumSMs, pl.U);
+  ns = (int)std::min<int64_t>(ns, cdiv(max_tok, 128));
+  ns = (int)std::max<int64_t>(ns, cdiv(max_tok, 4096));
+  pl.n_splits = std::max(1, std::min(ns, 1024));
+  // estimation: ~2 CTAs per SM overall, 256..2048 clusters each
+  int64_t ec = cdiv(total_rows, 2 * kNumSMs);
+  ec = std::max<int64_t>(256, std::min<int64_t>(2048, cdiv(ec, 256) * 256));
+  pl.echunk = (int)ec;
+  pl.n_est = (int)cdiv(max_nc, pl.echunk);
+  pl.n_parts = pl.n_splits + pl.n_est;
+
+  const int64_t ncl = (int64_t)pl.geo.cl_base[ix->batch] * ix->n_kv_heads;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t r = o; o = align_up(o + bytes, 256); return r; };
+  pl.off_status = take(256);
+  pl.off_scores = take((size_t)ncl * G * 4);
+  pl.off_keys = take((size_t)ncl * 4);
+  pl.off_sel = take((size_t)ncl * 4);
+  pl.off_seltok = take((size_t)(ncl + pl.U) * 4);
+  pl.off_info = take((size_t)pl.U * kInfoInts * 4);
+  pl.off_st_slot = take((size_t)pl.U * cap * 4);
+  pl.off_st_cl = take((size_t)pl.U * cap * 4);
+  pl.off_aff_cl = take((size_t)pl.U * cap * 4);
+  pl.off_aff_start = take((size_t)pl.U * (cap + 1) * 4);
+  pl.off_partials = take((size_t)pl.U * pl.n_parts * G * (pl.D + 2) * 4);
+  const size_t nq = (size_t)ix->batch * p->n_q_heads;
+  pl.off_q = take(nq * pl.D * esize(ix->dtype));
+  pl.off_out = take(nq * pl.D * 4);
+  pl.off_lse = take(nq * 4);
+  pl.total = o;
+  return WI_OK;
+}
+
+wi_status check_ws(const void* ws, size_t have, size_t need) {
+  if (!ws || !aligned(ws, 256) || have < need) return WI_ERR_WORKSPACE;
+  return WI_OK;
+}
+
+wi_status make_build_plan(const wi_kv_cache* kv, int S, int cs, BuildPlan& pl) {
+  if (!kv) return WI_ERR_INVALID_ARG;
+  wi_status st = check_common(kv->dtype, kv->batch, kv->n_kv_heads, kv->head_dim, kv->page_size,
+                              kv->n_pages, kv->k_pool, kv->v_pool, kv->block_table,
+                              kv->max_pages, kv->seq_lens);
+  if (st != WI_OK) return st;
+  if ((st = check_seg(S, cs)) != WI_OK) return st;
+  std::memset(&pl, 0, sizeof(pl));
+  fill_geo(pl.geo, kv->batch, kv->n_kv_heads, kv->head_dim, kv->seq_lens, S, cs);
+  pl.dtype = kv->dtype; pl.D = kv->head_dim; pl.U = kv->batch * kv->n_kv_heads;
+  pl.S = S; pl.cs = cs;
+  int max_nseg = 0;
+  for (int b = 0; b < kv->batch; ++b) max_nseg = std::max<int>(max_nseg, (int)cdiv(kv->seq_lens[b], S));
+  pl.max_nseg = max_nseg;
+  pl.max_ncl_seg = S / cs;
+  pl.update_smem = (size_t)(2 * pl.max_ncl_seg + 1 + 32) * 4 + (size_t)S * 2 * 2;
+  const int64_t ncl = (int64_t)pl.geo.cl_base[kv->batch] * kv->n_kv_heads;
+  const int64_t ntok = (int64_t)pl.geo.tok_base[kv->batch] * kv->n_kv_heads;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t r = o; o = align_up(o + bytes, 256); return r; };
+  pl.off_status = take(256);
+  pl.off_cent32 = take((size_t)ncl * pl.D * 4);
+  pl.off_assign = take((size_t)ntok * 4);
+  pl.total = o;
+  return WI_OK;
+}
+
+Pool make_pool(const void* base, const int32_t* bt, int64_t n_pages, int max_pages, int page) {
+  return Pool{base, bt, n_pages, max_pages, ilog2(page)};
+}
+
+wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params* p, float* out,
+                      float* lse, void* ws, size_t ws_bytes, cudaStream_t s, const void* q_host,
+                      float* out_host, float* lse_host) {
+  DecodePlan pl;
+  wi_status st = make_decode_plan(ix, p, pl);
+  if (st != WI_OK) return st;
+  const bool host = q_host != nullptr || out_host != nullptr;
+  if (host) {
+    if (!q_host || !out_host) return WI_ERR_INVALID_ARG;
+  } else {
+    if (!q || !out || !aligned(q, 16) || !aligned(out, 4) || (lse && !aligned(lse, 4)))
+      return WI_ERR_INVALID_ARG;
+  }
+  if ((st = check_ws(ws, ws_bytes, pl.total)) != WI_OK) return st;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  const size_t nq = (size_t)ix->batch * p->n_q_heads;
+  if (host) {
+    q = w + pl.off_q;
+    out = reinterpret_cast<float*>(w + pl.off_out);
+    lse = lse_host ? reinterpret_cast<float*>(w + pl.off_lse) : nullptr;
+    cudaError_t e = cudaMemcpyAsync(const_cast<void*>(q), q_host, nq * pl.D * esize(ix->dtype),
+                                    cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  DecodeArgs a{};
+  a.q = q;
+  a.centroids = ix->centroids;
+  a.value_sums = ix->value_sums;
+  a.offsets = ix->offsets;
+  a.perm = ix->perm;
+  a.invperm = ix->invperm;
+  a.kp = make_pool(ix->k_pool, ix->block_table, ix->n_pages, ix->max_pages, ix->page_size);
+  a.vp = make_pool(ix->v_pool, ix->block_table, ix->n_pages, ix->max_pages, ix->page_size);
+  a.out = out;
+  a.lse = lse;
+  a.ws = w;
+  a.stage_events = reinterpret_cast<cudaEvent_t*>(p->stage_events);
+  cudaError_t e = launch_decode(pl, a, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (host) {
+    e = cudaMemcpyAsync(out_host, out, nq * pl.D * 4, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess && lse_host) e = cudaMemcpyAsync(lse_host, lse, nq * 4, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return WI_OK;
+}
+
+}  // namespace
+}  // namespace wi
+
+using namespace wi;
+
+extern "C" {
+
+wi_status wi_index_clusters(int32_t batch, const int32_t* seq_lens, int32_t seg_len,
+                            int32_t cluster_size, int32_t* nc_out, int64_t* nc_total) {
+  if (batch < 1 || !seq_lens || !nc_total) return WI_ERR_INVALID_ARG;
+  wi_status st = check_seg(seg_len, cluster_size);
+  if (st != WI_OK) return st;
+  int64_t tot = 0;
+  for (int b = 0; b < batch; ++b) {
+    if (seq_lens[b] < 1) return WI_ERR_INVALID_ARG;
+    const int64_t nc = clusters_of(seq_lens[b], seg_len, cluster_size);
+    if (nc_out) nc_out[b] = (int32_t)nc;
+    tot += nc;
+  }
+  *nc_total = tot;
+  return WI_OK;
+}
+
+wi_status wi_build_workspace_size(const wi_kv_cache* kv, int32_t seg_len, int32_t cluster_size,
+                                  size_t* bytes) {
+  if (!bytes) return WI_ERR_INVALID_ARG;
+  BuildPlan pl;
+  wi_status st = make_build_plan(kv, seg_len, cluster_size, pl);
+  if (st != WI_OK) return st;
+  *bytes = pl.total;
+  return WI_OK;
+}
+
+wi_status wi_build_index(const wi_kv_cache* kv, int32_t seg_len, int32_t cluster_size,
+                         int32_t iters, const wi_index* out, void* ws, size_t ws_bytes,
+                         wi_stream_t stream) {
+  BuildPlan pl;
+  wi_status st = make_build_plan(kv, seg_len, cluster_size, pl);
+  if (st != WI_OK) return st;
+  if (iters < 1 || !out) return WI_ERR_INVALID_ARG;
+  if (out->dtype != kv->dtype || out->batch != kv->batch || out->n_kv_heads != kv->n_kv_heads ||
+      out->head_dim != kv->head_dim || out->page_size != kv->page_size ||
+      out->seg_len != seg_len || out->cluster_size != cluster_size || !out->seq_lens)
+    return WI_ERR_INVALID_ARG;
+  for (int b = 0; b < kv->batch; ++b)
+    if (out->seq_lens[b] != kv->seq_lens[b]) return WI_ERR_INVALID_ARG;
+  st = check_common(out->dtype, out->batch, out->n_kv_heads, out->head_dim, out->page_size,
+                    out->n_pages, out->k_pool, out->v_pool, out->block_table, out->max_pages,
+                    out->seq_lens);
+  if (st != WI_OK) return st;
+  if (!out->centroids || !out->value_sums || !out->offsets || !out->perm || !out->invperm)
+    return WI_ERR_INVALID_ARG;
+  if (!aligned(out->centroids, 16) || !aligned(out->value_sums, 16) || !aligned(out->offsets, 4) ||
+      !aligned(out->perm, 4) || !aligned(out->invperm, 4))
+    return WI_ERR_INVALID_ARG;
+  if (out->k_pool == kv->k_pool || out->v_pool == kv->v_pool || out->k_pool == kv->v_pool ||
+      out->v_pool == kv->k_pool)
+    return WI_ERR_INVALID_ARG;
+  pl.iters = iters;
+  if ((st = check_ws(ws, ws_bytes, pl.total)) != WI_OK) return st;
+  BuildArgs a{};
+  a.kin = make_pool(kv->k_pool, kv->block_table, kv->n_pages, kv->max_pages, kv->page_size);
+  a.vin = make_pool(kv->v_pool, kv->block_table, kv->n_pages, kv->max_pages, kv->page_size);
+  a.centroids = out->centroids;
+  a.value_sums = out->value_sums;
+  a.offsets = out->offsets;
+  a.perm = out->perm;
+  a.invperm = out->invperm;
+  a.kout = out->k_pool;
+  a.vout = out->v_pool;
+  a.bt_out = out->block_table;
+  a.n_pages_out = out->n_pages;
+  a.max_pages_out = out->max_pages;
+  a.page_shift_out = ilog2(out->page_size);
+  a.ws = static_cast<unsigned char*>(ws);
+  const cudaError_t e = launch_build(pl, a, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WI_OK : cuda_fail(e);
+}
+
+wi_status wi_kmeans_assign(const wi_kv_cache* kv, int32_t seg_len, int32_t cluster_size,
+                           const float* centroids, int32_t* assign, void* ws, size_t ws_bytes,
+                           wi_stream_t stream) {
+  BuildPlan pl;
+  wi_status st = make_build_plan(kv, seg_len, cluster_size, pl);
+  if (st != WI_OK) return st;
+  if (!centroids || !assign || !aligned(centroids, 16) || !aligned(assign, 4))
+    return WI_ERR_INVALID_ARG;
+  if ((st = check_ws(ws, ws_bytes, pl.total)) != WI_OK) return st;
+  BuildArgs a{};
+  a.kin = make_pool(kv->k_pool, kv->block_table, kv->n_pages, kv->max_pages, kv->page_size);
+  a.vin = make_pool(kv->v_pool, kv->block_table, kv->n_pages, kv->max_pages, kv->page_size);
+  a.ws = static_cast<unsigned char*>(ws);
+  const cudaError_t e =
+      launch_assign_only(pl, a, centroids, assign, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WI_OK : cuda_fail(e);
+}
+
+wi_status wi_decode_workspace_size(const wi_index* idx, const wi_decode_params* p, size_t* bytes) {
+  if (!bytes) return WI_ERR_INVALID_ARG;
+  DecodePlan pl;
+  const wi_status st = make_decode_plan(idx, p, pl);
+  if (st != WI_OK) return st;
+  *bytes = pl.total;
+  return WI_OK;
+}
+
+wi_status wi_decode_workspace_layout(const wi_index* idx, const wi_decode_params* p,
+                                     wi_decode_layout* layout) {
+  if (!layout) return WI_ERR_INVALID_ARG;
+  DecodePlan pl;
+  const wi_status st = make_decode_plan(idx, p, pl);
+  if (st != WI_OK) return st;
+  layout->total_bytes = pl.total;
+  layout->status = pl.off_status;
+  layout->scores = pl.off_scores;
+  layout->keys = pl.off_keys;
+  layout->selected = pl.off_sel;
+  layout->unit_info = pl.off_info;
+  layout->n_splits = pl.n_splits;
+  layout->n_est_chunks = pl.n_est;
+  return WI_OK;
+}
+
+wi_status wi_decode(const void* q, const wi_index* idx, const wi_decode_params* p, float* out,
+                    float* lse, void* ws, size_t ws_bytes, wi_stream_t stream) {
+  return decode_impl(q, idx, p, out, lse, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
+                     nullptr, nullptr, nullptr);
+}
+
+wi_status wi_decode_host(const void* q_host, const wi_index* idx, const wi_decode_params* p,
+                         float* out_host, float* lse_host, void* ws, size_t ws_bytes,
+                         wi_stream_t stream) {
+  if (!q_host || !out_host) return WI_ERR_INVALID_ARG;
+  return decode_impl(nullptr, idx, p, nullptr, nullptr, ws, ws_bytes,
+                     reinterpret_cast<cudaStream_t>(stream), q_host, out_host, lse_host);
+}
+
+int32_t wi_decode_stage_count(void) { return kDecodeStages; }
+
+const char* wi_decode_stage_name(int32_t i) {
+  return (i >= 0 && i < kDecodeStages) ? kDecodeStageNames[i] : nullptr;
+}
+
+wi_status wi_read_device_status(const void* ws, wi_stream_t stream, uint32_t* flags, int clear) {
+  if (!ws || !flags || !aligned(ws, 256)) return WI_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  uint32_t v = 0;
+  e = cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (clear && v) {
+    e = cudaMemsetAsync(const_cast<void*>(ws), 0, sizeof(v), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  *flags = v;
+  return v ? WI_ERR_DEVICE_CHECK : WI_OK;
+}
+
+const char* wi_status_string(wi_status s) {
+  switch (s) {
+    case WI_OK: return "ok";
+    case WI_ERR_INVALID_ARG: return "invalid argument";
+    case WI_ERR_UNSUPPORTED: return "unsupported configuration";
+    case WI_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case WI_ERR_CUDA: return "CUDA error";
+    case WI_ERR_DEVICE_CHECK: return "device-side index check failed";
+  }
+  return "unknown status";
+}
+
+const char* wi_last_error_string(void) { return g_last_error; }
+
+}  // extern "C"

@@ -1,0 +1,372 @@
+// Index-build kernels of the wave index (sm_100a): segmented k-means and the
+// cluster-permuted paged KV scatter (RetroInfer technical summary, section
+// 2.A, Segmented Clustering paragraph and item 2 Retrieval Zone; Vortex
+// summary, section 2.A forward_cache).
+//
+//   init    centroid j of a segment = key at segment position j*cs
+//   assign  argmin_j sum_e (k_e - c_je)^2 in fp32 (direct form, no
+//           ||k||^2 - 2k.c + ||c||^2 cancellation), ties to the lower j;
+//           64 tokens x 64 centroids per tile, 4x4 outputs per thread
+//   update  per (unit, segment): stable counting sort of the tokens by
+//           cluster, fp32 sums in ascending position, mean = sum / count;
+//           on the last round it also writes offsets, perm, invperm, the
+//           rounded centroids and value sums, and copies the K/V rows to the
+//           permuted pools (one pass over K and V).
+#include <cfloat>
+#include <climits>
+
+#include "wi_common.cuh"
+#include "wi_plan.h"
+
+namespace wi {
+namespace {
+
+template <typename T, int D>
+struct BRow {
+  static constexpr int EPL = Elem<T>::kPerVec;
+  static constexpr int LPR = D / EPL;
+  static constexpr int RPW = 32 / LPR;
+};
+
+// ------------------------------------------------------------------- init
+template <typename T, int D>
+__global__ void __launch_bounds__(kStreamThreads)
+kmeans_init_kernel(const Geo geo, const Pool kin, int S, int cs, float* __restrict__ cent32,
+                   uint32_t* status) {
+  using R = BRow<T, D>;
+  const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
+  const int T_ = geo.T(b);
+  const int seg = blockIdx.x, start = seg * S;
+  if (start >= T_) return;
+  const int len = min(S, T_ - start);
+  const int ncl = (len + cs - 1) / cs;
+  const int64_t crow = geo.cl_row(b, h) + (int64_t)seg * (S / cs);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane % R::LPR, rsub = lane / R::LPR;
+  const int groups = (blockDim.x >> 5) * R::RPW;
+  for (int j = warp * R::RPW + rsub; j < ncl; j += groups) {
+    const int64_t ro = pool_row(kin, geo.hkv, D, b, h, start + j * cs, status);
+    float x[R::EPL];
+    if (ro >= 0) {
+      const uint4 raw = ld_stream(reinterpret_cast<const T*>(kin.base) + ro + sub * R::EPL);
+      Elem<T>::unpack(raw, x);
+    } else {
+#pragma unroll
+      for (int e = 0; e < R::EPL; ++e) x[e] = 0.f;
+    }
+    float* dst = cent32 + (crow + j) * D + sub * R::EPL;
+#pragma unroll
+    for (int e = 0; e < R::EPL; ++e) dst[e] = x[e];
+  }
+}
+
+// ----------------------------------------------------------------- assign
+constexpr int kTok = 64, kCen = 64, kPad = 4;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+kmeans_assign_kernel(const Geo geo, const Pool kin, int S, int cs, const float* __restrict__ cent32,
+                     int32_t* __restrict__ assign, uint32_t* status) {
+  using R = BRow<T, D>;
+  extern __shared__ float4 sh_assign4[];
+  float* sk = reinterpret_cast<float*>(sh_assign4);      // [D][kTok + kPad]
+  float* sc = sk + D * (kTok + kPad);                    // [D][kCen + kPad]
+  const int u = blockIdx.z, b = u / geo.hkv, h = u - b * geo.hkv;
+  const int T_ = geo.T(b);
+  const int seg = blockIdx.y, start = seg * S;
+  if (start >= T_) return;
+  const int len = min(S, T_ - start);
+  const int t0 = blockIdx.x * kTok;
+  if (t0 >= len) return;
+  const int ntok = min(kTok, len - t0);
+  const int ncl = (len + cs - 1) / cs;
+  const int64_t crow = geo.cl_row(b, h) + (int64_t)seg * (S / cs);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int sub = lane % R::LPR, rsub = lane / R::LPR;
+  constexpr int LD = kTok + kPad;
+
+  // keys of the tile, transposed into shared memory as fp32
+  for (int r = warp * R::RPW + rsub; r < kTok; r += 8 * R::RPW) {
+    float x[R::EPL];
+#pragma unroll
+    for (int e = 0; e < R::EPL; ++e) x[e] = 0.f;
+    if (r < ntok) {
+      const int64_t ro = pool_row(kin, geo.hkv, D, b, h, start + t0 + r, status);
+      if (ro >= 0) {
+        const uint4 raw = ld_stream(reinterpret_cast<const T*>(kin.base) + ro + sub * R::EPL);
+        Elem<T>::unpack(raw, x);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < R::EPL; ++e) sk[(sub * R::EPL + e) * LD + r] = x[e];
+  }
+
+  float best[4];
+  int besti[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) { best[i] = INFINITY; besti[i] = 0; }
+
+  for (int cb = 0; cb < ncl; cb += kCen) {
+    __syncthreads();
+    // centroid tile, transposed (fp32 rows of D floats, 4 per lane per step)
+    for (int idx = tid; idx < kCen * (D / 4); idx += blockDim.x) {
+      const int j = idx / (D / 4), e4 = idx - j * (D / 4);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (cb + j < ncl) v = *reinterpret_cast<const float4*>(cent32 + (crow + cb + j) * D + e4 * 4);
+      sc[(e4 * 4 + 0) * LD + j] = v.x;
+      sc[(e4 * 4 + 1) * LD + j] = v.y;
+      sc[(e4 * 4 + 2) * LD + j] = v.z;
+      sc[(e4 * 4 + 3) * LD + j] = v.w;
+    }
+    __syncthreads();
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+    for (int e = 0; e < D; ++e) {
+      const float4 a = *reinterpret_cast<const float4*>(sk + e * LD + ty * 4);
+      const float4 c = *reinterpret_cast<const float4*>(sc + e * LD + tx * 4);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float cv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float df = av[i] - cv[j];
+          acc[i][j] = fmaf(df, df, acc[i][j]);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int cj = cb + tx * 4 + j;
+      if (cj < ncl) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (acc[i][j] < best[i]) { best[i] = acc[i][j]; besti[i] = cj; }
+      }
+    }
+  }
+  // reduce over the 16 threads that share the same tokens (same ty)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best[i], o);
+      const int oi = __shfl_xor_sync(0xffffffffu, besti[i], o);
+      if (ob < best[i] || (ob == best[i] && oi < besti[i])) { best[i] = ob; besti[i] = oi; }
+    }
+  }
+  if (tx == 0) {
+    int32_t* dst = assign + geo.tok_row(b, h) + start + t0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (ty * 4 + i < ntok) dst[ty * 4 + i] = besti[i];
+  }
+}
+
+// ----------------------------------------------------------------- update
+constexpr int kUpdThreads = 512;
+
+struct FinalOut {
+  void* centroids;
+  void* value_sums;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* invperm;
+  void* kout;
+  void* vout;
+  Pool pout;   // block table / geometry of the permuted pools
+  Pool vin;
+  int enabled;
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kUpdThreads)
+kmeans_update_kernel(const Geo geo, const Pool kin, int S, int cs, float* __restrict__ cent32,
+                     const int32_t* __restrict__ assign, const FinalOut fo, uint32_t* status) {
+  using R = BRow<T, D>;
+  extern __shared__ int32_t sh_upd[];
+  const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
+  const int T_ = geo.T(b);
+  const int seg = blockIdx.x, start = seg * S;
+  if (start >= T_) return;
+  const int len = min(S, T_ - start);
+  const int ncl = (len + cs - 1) / cs;
+  const int ncl_max = (S + cs - 1) / cs;
+  int32_t* s_cur = sh_upd;                                      // [ncl_max] cursor
+  int32_t* s_start = s_cur + ncl_max;                           // [ncl_max + 1]
+  int32_t* s_scan = s_start + ncl_max + 1;                      // [32]
+  uint16_t* s_asg = reinterpret_cast<uint16_t*>(s_scan + 32);   // [S]
+  uint16_t* s_mem = s_asg + S;                                  // [S]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  const int64_t trow = geo.tok_row(b, h);
+  const int64_t crow = geo.cl_row(b, h) + (int64_t)seg * (S / cs);
+
+  for (int j = tid; j < ncl; j += blockDim.x) s_cur[j] = 0;
+  __syncthreads();
+  for (int i = tid; i < len; i += blockDim.x) {
+    int a = assign[trow + start + i];
+    if (a < 0 || a >= ncl) { flag_error(status, WI_DEV_BAD_CLUSTER); a = 0; }
+    s_asg[i] = (uint16_t)a;
+    atomicAdd(&s_cur[a], 1);
+  }
+  __syncthreads();
+  // exclusive scan of the counts
+  int run = 0;
+  for (int base = 0; base < ncl; base += blockDim.x) {
+    const int j = base + tid;
+    const int c = j < ncl ? s_cur[j] : 0;
+    int tot;
+    const int incl = block_inclusive_scan(c, s_scan, &tot);
+    if (j < ncl) s_start[j] = run + incl - c;
+    run += tot;
+  }
+  if (tid == 0) s_start[ncl] = len;
+  __syncthreads();
+  for (int j = tid; j < ncl; j += blockDim.x) s_cur[j] = s_start[j];
+  __syncthreads();
+  // stable scatter: tokens in ascending order, warps in turn within a round
+  for (int base = 0; base < len; base += blockDim.x) {
+    const int t = base + tid;
+    const unsigned act = __ballot_sync(0xffffffffu, t < len);
+    for (int w = 0; w < nw; ++w) {
+      if (warp == w && t < len) {
+        const int bin = s_asg[t];
+        const unsigned peers = __match_any_sync(act, bin);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        const int leader = __ffs(peers) - 1;
+        int pos = 0;
+        if (lane == leader) { pos = s_cur[bin]; s_cur[bin] = pos + __popc(peers); }
+        pos = __shfl_sync(peers, pos, leader);
+        s_mem[pos + rank] = (uint16_t)t;
+      }
+      __syncthreads();
+    }
+  }
+  // means (fixed ascending-position order per cluster), final layout
+  const int sub = lane % R::LPR, rsub = lane / R::LPR;
+  const int groups = nw * R::RPW;
+  const T* kb = reinterpret_cast<const T*>(kin.base) + sub * R::EPL;
+  for (int j = warp * R::RPW + rsub; j < ncl; j += groups) {
+    const int m0 = s_start[j], m1 = s_start[j + 1];
+    float ks[R::EPL], vs[R::EPL];
+#pragma unroll
+    for (int e = 0; e < R::EPL; ++e) { ks[e] = 0.f; vs[e] = 0.f; }
+    for (int m = m0; m < m1; ++m) {
+      const int p = start + s_mem[m];
+      const int64_t ro = pool_row(kin, geo.hkv, D, b, h, p, status);
+      if (ro < 0) continue;
+      const uint4 kraw = ld_stream(kb + ro);
+      float x[R::EPL];
+      Elem<T>::unpack(kraw, x);
+#pragma unroll
+      for (int e = 0; e < R::EPL; ++e) ks[e] += x[e];
+      if (fo.enabled) {
+        const int slot = start + m;
+        const int64_t vo = pool_row(fo.vin, geo.hkv, D, b, h, p, status);
+        const int64_t oo = pool_row(fo.pout, geo.hkv, D, b, h, slot, status);
+        uint4 vraw = make_uint4(0, 0, 0, 0);
+        if (vo >= 0) vraw = ld_stream(reinterpret_cast<const T*>(fo.vin.base) + vo + sub * R::EPL);
+        Elem<T>::unpack(vraw, x);
+#pragma unroll
+        for (int e = 0; e < R::EPL; ++e) vs[e] += x[e];
+        if (oo >= 0) {
+          *reinterpret_cast<uint4*>(reinterpret_cast<T*>(fo.kout) + oo + sub * R::EPL) = kraw;
+          *reinterpret_cast<uint4*>(reinterpret_cast<T*>(fo.vout) + oo + sub * R::EPL) = vraw;
+        }
+        if (sub == 0) {
+          fo.perm[trow + slot] = p;
+          fo.invperm[trow + p] = slot;
+        }
+      }
+    }
+    const int cnt = m1 - m0;
+    float* c32 = cent32 + (crow + j) * D + sub * R::EPL;
+    if (cnt > 0) {
+#pragma unroll
+      for (int e = 0; e < R::EPL; ++e) c32[e] = ks[e] / (float)cnt;
+    }
+    if (fo.enabled) {
+      T* cdst = reinterpret_cast<T*>(fo.centroids) + (crow + j) * D + sub * R::EPL;
+      T* vdst = reinterpret_cast<T*>(fo.value_sums) + (crow + j) * D + sub * R::EPL;
+#pragma unroll
+      for (int e = 0; e < R::EPL; ++e) {
+        store_elem(cdst + e, c32[e]);
+        store_elem(vdst + e, vs[e]);
+      }
+      if (sub == 0) fo.offsets[geo.off_row(b, h) + seg * (S / cs) + j] = start + m0;
+    }
+  }
+  if (fo.enabled && tid == 0 && start + len == T_) fo.offsets[geo.off_row(b, h) + geo.NC(b)] = T_;
+}
+
+template <typename F>
+cudaError_t with_build_types(int dtype, int D, F&& f) {
+  if (dtype == WI_BF16) {
+    if (D == 128) return f.template operator()<__nv_bfloat16, 128>();
+    if (D == 64) return f.template operator()<__nv_bfloat16, 64>();
+  } else {
+    if (D == 128) return f.template operator()<float, 128>();
+    if (D == 64) return f.template operator()<float, 64>();
+  }
+  return cudaErrorInvalidValue;
+}
+
+size_t assign_smem(int D) { return (size_t)D * ((kTok + kPad) + (kCen + kPad)) * sizeof(float); }
+
+}  // namespace
+
+cudaError_t launch_assign_only(const BuildPlan& p, const BuildArgs& a, const float* cent32,
+                               int32_t* assign, cudaStream_t s) {
+  uint32_t* status = reinterpret_cast<uint32_t*>(a.ws + p.off_status);
+  return with_build_types(p.dtype, p.D, [&]<typename T, int D>() -> cudaError_t {
+    const size_t smem = assign_smem(D);
+    cudaFuncSetAttribute(kmeans_assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    const dim3 grid((p.S + kTok - 1) / kTok, p.max_nseg, p.U);
+    kmeans_assign_kernel<T, D><<<grid, 256, smem, s>>>(p.geo, a.kin, p.S, p.cs, cent32, assign,
+                                                       status);
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s) {
+  uint32_t* status = reinterpret_cast<uint32_t*>(a.ws + p.off_status);
+  float* cent32 = reinterpret_cast<float*>(a.ws + p.off_cent32);
+  int32_t* assign = reinterpret_cast<int32_t*>(a.ws + p.off_assign);
+  return with_build_types(p.dtype, p.D, [&]<typename T, int D>() -> cudaError_t {
+    const size_t smem = assign_smem(D);
+    cudaFuncSetAttribute(kmeans_assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    cudaFuncSetAttribute(kmeans_update_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)p.update_smem);
+    kmeans_init_kernel<T, D><<<dim3(p.max_nseg, p.U), kStreamThreads, 0, s>>>(
+        p.geo, a.kin, p.S, p.cs, cent32, status);
+    FinalOut none{};
+    none.enabled = 0;
+    FinalOut fin{};
+    fin.centroids = a.centroids;
+    fin.value_sums = a.value_sums;
+    fin.offsets = a.offsets;
+    fin.perm = a.perm;
+    fin.invperm = a.invperm;
+    fin.kout = a.kout;
+    fin.vout = a.vout;
+    fin.pout = Pool{a.kout, a.bt_out, a.n_pages_out, a.max_pages_out, a.page_shift_out};
+    fin.vin = a.vin;
+    fin.enabled = 1;
+    const dim3 agrid((p.S + kTok - 1) / kTok, p.max_nseg, p.U);
+    for (int it = 0; it < p.iters; ++it) {
+      kmeans_assign_kernel<T, D><<<agrid, 256, smem, s>>>(p.geo, a.kin, p.S, p.cs, cent32, assign,
+                                                          status);
+      kmeans_update_kernel<T, D><<<dim3(p.max_nseg, p.U), kUpdThreads, p.update_smem, s>>>(
+          p.geo, a.kin, p.S, p.cs, cent32, assign, it == p.iters - 1 ? fin : none, status);
+    }
+    return cudaGetLastError();
+  });
+}
+
+}  // namespace wi

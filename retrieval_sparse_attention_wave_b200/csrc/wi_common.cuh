@@ -1,0 +1,187 @@
+// Shared device helpers for the wave-index kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "wi.h"
+
+namespace wi {
+
+constexpr int kMaxBatch = WI_MAX_BATCH;
+constexpr int kWarp = 32;
+
+// Ragged per-call geometry, passed to kernels by value (about 2 KB).
+struct Geo {
+  int32_t batch, hkv, d;
+  int32_t tok_base[kMaxBatch + 1];  // prefix sums of T_b
+  int32_t cl_base[kMaxBatch + 1];   // prefix sums of NC_b
+
+  __host__ __device__ __forceinline__ int T(int b) const { return tok_base[b + 1] - tok_base[b]; }
+  __host__ __device__ __forceinline__ int NC(int b) const { return cl_base[b + 1] - cl_base[b]; }
+  // first cluster row of unit (b,h) in centroid / score / key arrays
+  __host__ __device__ __forceinline__ int64_t cl_row(int b, int h) const {
+    return (int64_t)cl_base[b] * hkv + (int64_t)h * NC(b);
+  }
+  // first entry of unit (b,h) in the offsets array (NC_b + 1 entries per unit)
+  __host__ __device__ __forceinline__ int64_t off_row(int b, int h) const {
+    return ((int64_t)cl_base[b] + b) * hkv + (int64_t)h * (NC(b) + 1);
+  }
+  // first entry of unit (b,h) in token-indexed arrays (perm, invperm, assign)
+  __host__ __device__ __forceinline__ int64_t tok_row(int b, int h) const {
+    return (int64_t)tok_base[b] * hkv + (int64_t)h * T(b);
+  }
+};
+
+// A paged pool [n_pages][hkv][page][d] addressed through a block table.
+struct Pool {
+  const void* base;
+  const int32_t* bt;
+  int64_t n_pages;
+  int32_t max_pages;
+  int32_t page_shift;  // log2(page_size)
+};
+
+// Status word in the first bytes of every workspace.
+__device__ __forceinline__ void flag_error(uint32_t* status, uint32_t bit) {
+  atomicOr(status, bit);
+}
+
+// Element offset of row `slot` of unit (b,h) in a pool, or -1 (and a status
+// bit) when the block table points outside the pool.
+__device__ __forceinline__ int64_t pool_row(const Pool& p, int hkv, int d, int b, int h, int slot,
+                                            uint32_t* status) {
+  const int lp = slot >> p.page_shift;
+  if (slot < 0 || lp >= p.max_pages) {
+    flag_error(status, WI_DEV_BAD_SLOT);
+    return -1;
+  }
+  const int pg = __ldg(p.bt + (int64_t)b * p.max_pages + lp);
+  if (pg < 0 || (int64_t)pg >= p.n_pages) {
+    flag_error(status, WI_DEV_BAD_PAGE);
+    return -1;
+  }
+  const int row = slot & ((1 << p.page_shift) - 1);
+  return ((((int64_t)pg * hkv + h) << p.page_shift) + row) * d;
+}
+
+// 16-byte streaming load (read-only path, no L1 allocation).
+__device__ __forceinline__ uint4 ld_stream(const void* ptr) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(ptr));
+  return r;
+}
+
+// Element traits: how a 16-byte vector unpacks into floats.
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static constexpr int kPerVec = 4;
+  __device__ __forceinline__ static void unpack(const uint4& v, float* x) {
+    x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
+    x[2] = __uint_as_float(v.z); x[3] = __uint_as_float(v.w);
+  }
+  __device__ __forceinline__ static float from_float(float f) { return f; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static constexpr int kPerVec = 8;
+  __device__ __forceinline__ static void unpack(const uint4& v, float* x) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
+
+__device__ __forceinline__ void store_elem(float* p, float v) { *p = v; }
+__device__ __forceinline__ void store_elem(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+// Order-preserving map of a float to uint32 (larger float -> larger key).
+// Key 0 is reserved for "not a candidate".
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return k == 0u ? 1u : k;
+}
+
+// Sum N values across groups of L consecutive lanes (N <= L, both powers of
+// two) with log2(L) shuffle rounds and N-1+log2(L/N) shuffles in total: each
+// round halves the values a lane keeps (it keeps the half selected by its
+// lane bit and receives the partner's copy of that half).  Afterwards v[0] of
+// every lane holds the group's full sum of value index j = (lane % L) / (L / N).
+template <int N, int O>
+struct GroupReduce {
+  __device__ __forceinline__ static void run(float* v, int lane) {
+    if constexpr (O >= 1) {
+      const bool hi = (lane & O) != 0;
+      if constexpr (N > 1) {
+#pragma unroll
+        for (int i = 0; i < N / 2; ++i) {
+          const float keep = hi ? v[i + N / 2] : v[i];
+          const float send = hi ? v[i] : v[i + N / 2];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+        }
+        GroupReduce<N / 2, O / 2>::run(v, lane);
+      } else {
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+        GroupReduce<1, O / 2>::run(v, lane);
+      }
+    }
+  }
+};
+
+template <int N, int L>
+__device__ __forceinline__ void group_reduce_multi(float (&v)[N], int lane) {
+  static_assert(N >= 1 && N <= L && L <= 32, "bad reduce shape");
+  GroupReduce<N, L / 2>::run(v, lane);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Inclusive scan of one int per thread over the block (blockDim.x multiple of
+// 32, <= 1024).  `sh` needs 32 ints.  Returns the inclusive prefix; *total
+// receives the block sum.  Contains __syncthreads.
+__device__ __forceinline__ int block_inclusive_scan(int x, int* sh, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int s = lane < nw ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    sh[lane] = s;
+  }
+  __syncthreads();
+  const int r = x + (w > 0 ? sh[w - 1] : 0);
+  *total = sh[nw - 1];
+  __syncthreads();
+  return r;
+}
+
+}  // namespace wi

@@ -1,0 +1,87 @@
+// Host-side launch plans for the wave-index kernels: the geometry of one call,
+// the launch shapes, and where each workspace region lives.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "wi_common.cuh"
+
+namespace wi {
+
+constexpr int kStreamThreads = 256;   // streaming kernels: 8 warps
+constexpr int kTopkThreads = 1024;    // one CTA per unit
+constexpr int kAttendTile = 64;       // tokens per exact-attention tile
+constexpr int kInfoInts = 8;          // per-unit info record (see wi_decode_layout)
+constexpr int kNumSMs = 148;          // B200
+
+struct DecodePlan {
+  Geo geo;
+  int dtype, D, G, Hq, U;
+  int n_sink, window, topk_clusters;
+  double topk_fraction;
+  int max_nc;
+  int score_chunk, n_score_blocks;
+  int cap;                 // steady-list capacity per unit (>= 1)
+  int sort_pow2;           // shared-memory sort size for the steady list
+  int n_splits;            // exact-attention CTAs per unit
+  int echunk, n_est;       // estimation clusters per CTA, CTAs per unit
+  int n_parts;             // n_splits + n_est softmax parts per (unit, head)
+  float scale;             // 1/sqrt(d)
+  // workspace byte offsets
+  size_t off_status, off_scores, off_keys, off_sel, off_seltok, off_info;
+  size_t off_st_slot, off_st_cl, off_aff_cl, off_aff_start, off_partials;
+  size_t off_q, off_out, off_lse;
+  size_t total;
+};
+
+struct BuildPlan {
+  Geo geo;
+  int dtype, D, U, S, cs, iters;
+  int max_nseg, max_ncl_seg;
+  size_t update_smem;
+  size_t off_status, off_cent32, off_assign;
+  size_t total;
+};
+
+// Pointers of one decode call.
+struct DecodeArgs {
+  const void* q;
+  const void* centroids;
+  const void* value_sums;
+  const int32_t* offsets;
+  const int32_t* perm;
+  const int32_t* invperm;
+  Pool kp, vp;
+  float* out;
+  float* lse;
+  unsigned char* ws;
+  cudaEvent_t* stage_events;
+};
+
+struct BuildArgs {
+  Pool kin, vin;
+  // outputs (index); null pointers for the assign-only entry
+  void* centroids;
+  void* value_sums;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* invperm;
+  void* kout;
+  void* vout;
+  const int32_t* bt_out;
+  int64_t n_pages_out;
+  int32_t max_pages_out;
+  int32_t page_shift_out;
+  unsigned char* ws;
+};
+
+constexpr int kDecodeStages = 6;
+extern const char* const kDecodeStageNames[kDecodeStages];
+
+cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s);
+cudaError_t launch_assign_only(const BuildPlan& p, const BuildArgs& a, const float* cent32,
+                               int32_t* assign, cudaStream_t s);
+
+}  // namespace wi

@@ -10,3 +10,11 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_sessionstart(session):
+    # The C-ABI library is a build artefact (not committed); build it in-tree
+    # when it is missing or older than its sources.  nvcc cross-compiles for
+    # sm_100a without a GPU.
+    from retrieval_sparse_attention_wave_b200 import build as _build
+    _build.build()

@@ -1,0 +1,195 @@
+"""The C-ABI boundary on the host: the library loads, exports every symbol
+include/wi.h declares, and rejects bad arguments with status codes before any
+CUDA call (so these run without a GPU)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import retrieval_sparse_attention_wave_b200 as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x7f0000000000          # 256-byte aligned, never dereferenced
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "wi.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(wi_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(W.lib(), n), n
+    assert sorted(names) == sorted(W.EXPORTED)
+
+
+def test_stage_names():
+    assert W.stage_names() == ["steady", "score", "topk", "attend", "estimate", "merge"]
+    assert W.lib().wi_decode_stage_name(99) is None
+
+
+def test_index_clusters_counts():
+    assert W.clusters_per_sequence([131072], 8192, 16) == [8192]
+    assert W.clusters_per_sequence([4196, 1, 17], 1024, 16) == [263, 1, 2]
+    tot = C.c_int64()
+    arr = (C.c_int32 * 1)(100)
+    assert W.lib().wi_index_clusters(1, arr, 30, 16, None, C.byref(tot)) == W.WI_ERR_INVALID_ARG
+    assert W.lib().wi_index_clusters(1, arr, 32768, 16, None, C.byref(tot)) == W.WI_ERR_UNSUPPORTED
+
+
+def kv_struct(**over):
+    seq = over.pop("seq", [4096])
+    s = W.WiKVCache()
+    s.dtype = W.WI_BF16
+    s.batch = len(seq)
+    s.n_kv_heads, s.head_dim, s.page_size = 8, 128, 16
+    s.n_pages = 4096
+    s.k_pool = FAKE
+    s.v_pool = FAKE + 0x10000000
+    s.block_table = FAKE + 0x20000000
+    s.max_pages = 4096
+    s._seq = (C.c_int32 * len(seq))(*seq)
+    s.seq_lens = C.cast(s._seq, C.POINTER(C.c_int32))
+    for k, v in over.items():
+        setattr(s, k, v)
+    return s
+
+
+def index_struct(**over):
+    seq = over.pop("seq", [4096])
+    s = W.WiIndex()
+    s.dtype = W.WI_BF16
+    s.batch = len(seq)
+    s.n_kv_heads, s.head_dim, s.page_size, s.seg_len, s.cluster_size = 8, 128, 16, 1024, 16
+    s._seq = (C.c_int32 * len(seq))(*seq)
+    s.seq_lens = C.cast(s._seq, C.POINTER(C.c_int32))
+    for i, f in enumerate(["centroids", "value_sums", "offsets", "perm", "invperm", "k_pool",
+                           "v_pool", "block_table"]):
+        setattr(s, f, FAKE + (i + 1) * 0x1000000)
+    s.n_pages = 4096
+    s.max_pages = 4096
+    for k, v in over.items():
+        setattr(s, k, v)
+    return s
+
+
+def params(**over):
+    p = W.WiDecodeParams()
+    p.n_q_heads, p.n_sink, p.window, p.topk_clusters, p.topk_fraction = 32, 4, 64, -1, 0.018
+    for k, v in over.items():
+        setattr(p, k, v)
+    return p
+
+
+def ws_size(ix, p):
+    n = C.c_size_t()
+    st = W.lib().wi_decode_workspace_size(C.byref(ix), C.byref(p), C.byref(n))
+    return st, n.value
+
+
+def test_decode_workspace_size_and_layout():
+    st, n = ws_size(index_struct(), params())
+    assert st == W.WI_OK and n > 0 and n % 256 == 0
+    lay = W.WiDecodeLayout()
+    assert W.lib().wi_decode_workspace_layout(C.byref(index_struct()), C.byref(params()),
+                                              C.byref(lay)) == W.WI_OK
+    assert lay.total_bytes == n and lay.status == 0
+    assert 0 < lay.scores < lay.keys < lay.selected < lay.unit_info < n
+    assert lay.n_splits >= 1 and lay.n_est_chunks >= 1
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(n_q_heads=0), W.WI_ERR_INVALID_ARG),
+    (dict(n_q_heads=31), W.WI_ERR_INVALID_ARG),       # not a multiple of Hkv
+    (dict(n_q_heads=8 * 16), W.WI_ERR_UNSUPPORTED),   # G = 16
+    (dict(n_q_heads=8 * 3), W.WI_ERR_UNSUPPORTED),    # G = 3
+    (dict(n_sink=-1), W.WI_ERR_INVALID_ARG),
+    (dict(window=-5), W.WI_ERR_INVALID_ARG),
+    (dict(topk_clusters=-1, topk_fraction=1.5), W.WI_ERR_INVALID_ARG),
+    (dict(n_sink=5000, window=5000), W.WI_OK),        # all steady (dense) is legal
+    (dict(n_sink=8000, window=192), W.WI_OK),         # exactly WI_MAX_STEADY
+])
+def test_decode_param_validation(over, expect):
+    st, _ = ws_size(index_struct(seq=[10000]), params(**over))
+    assert st == expect
+
+
+def test_steady_limit_is_reported():
+    st, _ = ws_size(index_struct(seq=[100000], max_pages=8192), params(n_sink=5000, window=5000))
+    assert st == W.WI_ERR_UNSUPPORTED
+    st, _ = ws_size(index_struct(seq=[10000]), params(n_sink=8000, window=193))
+    assert st == W.WI_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(head_dim=96), W.WI_ERR_UNSUPPORTED),
+    (dict(head_dim=0), W.WI_ERR_INVALID_ARG),
+    (dict(page_size=12), W.WI_ERR_INVALID_ARG),
+    (dict(dtype=7), W.WI_ERR_INVALID_ARG),
+    (dict(centroids=None), W.WI_ERR_INVALID_ARG),
+    (dict(perm=FAKE + 2), W.WI_ERR_INVALID_ARG),       # misaligned
+    (dict(k_pool=FAKE + 8), W.WI_ERR_INVALID_ARG),     # not 16-byte aligned
+    (dict(seg_len=1000), W.WI_ERR_INVALID_ARG),        # not a multiple of cluster_size
+    (dict(seg_len=32768), W.WI_ERR_UNSUPPORTED),
+    (dict(max_pages=10), W.WI_ERR_INVALID_ARG),        # 4096 tokens need 256 pages
+    (dict(seq=[0]), W.WI_ERR_INVALID_ARG),
+    (dict(seq=[16] * 300), W.WI_ERR_UNSUPPORTED),      # batch > WI_MAX_BATCH
+])
+def test_index_validation(over, expect):
+    st, _ = ws_size(index_struct(**over), params())
+    assert st == expect
+
+
+def test_decode_rejects_before_any_cuda_call():
+    ix, p = index_struct(), params()
+    lib = W.lib()
+    # null q / out
+    assert lib.wi_decode(None, C.byref(ix), C.byref(p), FAKE, None, FAKE, 1 << 30, None) \
+        == W.WI_ERR_INVALID_ARG
+    assert lib.wi_decode(FAKE, C.byref(ix), C.byref(p), None, None, FAKE, 1 << 30, None) \
+        == W.WI_ERR_INVALID_ARG
+    # workspace missing, too small, misaligned
+    _, need = ws_size(ix, p)
+    assert lib.wi_decode(FAKE, C.byref(ix), C.byref(p), FAKE, None, None, need, None) \
+        == W.WI_ERR_WORKSPACE
+    assert lib.wi_decode(FAKE, C.byref(ix), C.byref(p), FAKE, None, FAKE, need - 1, None) \
+        == W.WI_ERR_WORKSPACE
+    assert lib.wi_decode(FAKE, C.byref(ix), C.byref(p), FAKE, None, FAKE + 16, need, None) \
+        == W.WI_ERR_WORKSPACE
+    assert lib.wi_decode_host(None, C.byref(ix), C.byref(p), FAKE, None, FAKE, need, None) \
+        == W.WI_ERR_INVALID_ARG
+
+
+def test_build_validation():
+    lib = W.lib()
+    kv = kv_struct()
+    n = C.c_size_t()
+    assert lib.wi_build_workspace_size(C.byref(kv), 1024, 16, C.byref(n)) == W.WI_OK
+    assert n.value >= 8 * 4096 * 4
+    out = index_struct()
+    # iters < 1
+    assert lib.wi_build_index(C.byref(kv), 1024, 16, 0, C.byref(out), FAKE, n.value, None) \
+        == W.WI_ERR_INVALID_ARG
+    # geometry mismatch between input and output
+    assert lib.wi_build_index(C.byref(kv), 512, 16, 3, C.byref(out), FAKE, n.value, None) \
+        == W.WI_ERR_INVALID_ARG
+    # output pools aliasing the input pools
+    alias = index_struct(k_pool=kv.k_pool)
+    assert lib.wi_build_index(C.byref(kv), 1024, 16, 3, C.byref(alias), FAKE, n.value, None) \
+        == W.WI_ERR_INVALID_ARG
+    # workspace too small
+    assert lib.wi_build_index(C.byref(kv), 1024, 16, 3, C.byref(out), FAKE, 1024, None) \
+        == W.WI_ERR_WORKSPACE
+    assert lib.wi_kmeans_assign(C.byref(kv), 1024, 16, None, FAKE, FAKE, n.value, None) \
+        == W.WI_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    lib = W.lib()
+    for s in range(6):
+        assert lib.wi_status_string(s)
+    assert lib.wi_read_device_status(None, None, None, 0) == W.WI_ERR_INVALID_ARG

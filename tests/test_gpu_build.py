@@ -1,0 +1,205 @@
+"""Build parity: segmented k-means and the cluster-permuted scatter on the GPU
+against the fp64 oracle (RetroInfer technical summary, section 2.A,
+Segmented Clustering).
+
+* Assignment from identical centroids is bit-exact except near-ties: a token
+  may pick another centroid only if its fp64 distance is within 1e-5
+  relative of the best one.
+* With one round from the (exact) initial centroids the whole index equals
+  the oracle's: offsets and perm exactly, centroids and value sums within one
+  unit in the last place of the KV dtype, permuted rows bit-exact.
+* After ten rounds, the GPU index is valid on its own terms (a bijective
+  perm, slot ranges, ascending members, rows copied bit-exactly, stored
+  centroid / value sum = rounded mean / sum of its members) and its k-means
+  objective is close to the oracle's.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import retrieval_sparse_attention_wave_b200 as W
+import wave_inputs as WI
+from tests import wave_harness as H
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def wl_small(dtype=torch.bfloat16, d=128, seq_lens=(3000, 1100), Hkv=2, seg=1024, cs=16, seed=21):
+    return WI.mixture_workload("build", seq_lens=list(seq_lens), n_q_heads=Hkv * 2,
+                               n_kv_heads=Hkv, head_dim=d, n_centers=40, dtype=dtype,
+                               seg_len=seg, cluster_size=cs, iters=10, seed=seed, device=DEV)
+
+
+def ulp(x: np.ndarray, dtype) -> np.ndarray:
+    bits = 8 if dtype == torch.bfloat16 else 24
+    ax = np.maximum(np.abs(x), 1e-30)
+    return np.ldexp(1.0, np.floor(np.log2(ax)).astype(int) - (bits - 1))
+
+
+def segment_views(wl, b, h, keys):
+    X = keys[b][h]
+    return [(s, X[s:s + n]) for s, n in O.segment_spans(len(X), wl.seg_len)]
+
+
+def assign_check(wl, cents_by_unit):
+    """Run the GPU assignment with the given fp32 centroids and compare."""
+    kv = H.paged_kv(wl, DEV, shuffle_seed=9)
+    nc = W.clusters_per_sequence(wl.seq_lens, wl.seg_len, wl.cluster_size)
+    Hkv = wl.n_kv_heads
+    C32 = torch.zeros(Hkv * sum(nc), wl.head_dim, dtype=torch.float32)
+    for (b, h), C in cents_by_unit.items():
+        r = Hkv * sum(nc[:b]) + h * nc[b]
+        C32[r:r + len(C)] = torch.as_tensor(C, dtype=torch.float32)
+    assign = W.kmeans_assign(kv, wl.seg_len, wl.cluster_size, C32.to(DEV).contiguous())
+    torch.cuda.synchronize()
+    assign = assign.cpu().numpy()
+    keys, _ = H.host_rows(wl)
+    flips = 0
+    for (b, h), C in cents_by_unit.items():
+        C = np.asarray(C, dtype=np.float32).astype(np.float64)
+        t = Hkv * sum(wl.seq_lens[:b]) + h * wl.seq_lens[b]
+        base = 0
+        for s, X in segment_views(wl, b, h, keys):
+            m = O.clusters_in_segment(len(X), wl.cluster_size)
+            Cs = C[base:base + m]
+            ref = O.kmeans_assign(X, Cs)
+            got = assign[t + s:t + s + len(X)]
+            assert got.min() >= 0 and got.max() < m
+            bad = np.nonzero(got != ref)[0]
+            if len(bad):
+                D = O.kmeans_distances(X[bad], Cs)
+                dg = D[np.arange(len(bad)), got[bad]]
+                dr = D[np.arange(len(bad)), ref[bad]]
+                assert np.all(dg <= dr * (1 + 1e-5)), "assignment differs beyond near-ties"
+                flips += len(bad)
+            base += m
+    return flips
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64),
+                                     (torch.bfloat16, 64), (torch.float32, 128)])
+def test_assign_from_initial_centroids(dtype, d):
+    wl = wl_small(dtype=dtype, d=d)
+    keys, _ = H.host_rows(wl)
+    cents = {}
+    for b in range(wl.batch):
+        for h in range(wl.n_kv_heads):
+            cents[(b, h)] = np.concatenate([O.kmeans_init(X, wl.cluster_size)
+                                            for _, X in segment_views(wl, b, h, keys)])
+    flips = assign_check(wl, cents)
+    assert flips <= 2
+
+
+def test_assign_from_later_centroids():
+    wl = wl_small()
+    keys, _ = H.host_rows(wl)
+    cents = {}
+    for b in range(wl.batch):
+        for h in range(wl.n_kv_heads):
+            parts = []
+            for _, X in segment_views(wl, b, h, keys):
+                _, C, _ = O.kmeans_segment(X, wl.cluster_size, 3)
+                parts.append(C)
+            cents[(b, h)] = np.concatenate(parts)
+    flips = assign_check(wl, cents)
+    assert flips <= 5
+
+
+def gpu_build(wl, iters, shuffle_in=9, shuffle_out=4):
+    kv = H.paged_kv(wl, DEV, shuffle_seed=shuffle_in)
+    bt, n_pages = H.out_block_table(wl, DEV, shuffle_seed=shuffle_out)
+    wx = W.build_index(kv, wl.seg_len, wl.cluster_size, iters, block_table=bt, n_pages=n_pages)
+    torch.cuda.synchronize()
+    assert W.read_device_status(wx._build_ws) == 0
+    return wx
+
+
+def check_valid(wl, wx, b, h, keys, vals):
+    g = H.download_unit(wx, b, h)
+    T = wl.seq_lens[b]
+    NC = O.n_clusters(T, wl.seg_len, wl.cluster_size)
+    off, perm, inv = g["offsets"], g["perm"], g["invperm"]
+    assert len(off) == NC + 1 and off[0] == 0 and off[-1] == T and np.all(np.diff(off) >= 0)
+    assert np.array_equal(np.sort(perm), np.arange(T))
+    assert np.array_equal(inv[perm], np.arange(T))
+    for s, n in O.segment_spans(T, wl.seg_len):       # clusters stay inside segments
+        assert set(perm[s:s + n].tolist()) == set(range(s, s + n))
+    cl = np.repeat(np.arange(NC), np.diff(off))
+    same = cl[1:] == cl[:-1]
+    assert np.all(perm[1:][same] > perm[:-1][same])   # ascending inside a cluster
+    np.testing.assert_array_equal(g["k_perm"], keys[b][h][perm])
+    np.testing.assert_array_equal(g["v_perm"], vals[b][h][perm])
+    cnt = np.diff(off)
+    nz = cnt > 0
+    ksum = np.zeros((NC, wl.head_dim))
+    vsum = np.zeros((NC, wl.head_dim))
+    np.add.at(ksum, cl, keys[b][h][perm])
+    np.add.at(vsum, cl, vals[b][h][perm])
+    mean = ksum[nz] / cnt[nz, None]
+    assert np.all(np.abs(g["centroids"][nz] - mean) <= ulp(mean, wl.dtype) + 1e-30)
+    assert np.all(np.abs(g["value_sums"] - vsum) <= ulp(vsum, wl.dtype) + 1e-30)
+    assert np.all(g["value_sums"][~nz] == 0)
+    return g
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_one_round_build_equals_oracle(dtype, d):
+    wl = wl_small(dtype=dtype, d=d)
+    wx = gpu_build(wl, iters=1)
+    ref = H.oracle_build(wl, iters=1)
+    keys, vals = H.host_rows(wl)
+    for (b, h), ix in ref.items():
+        g = check_valid(wl, wx, b, h, keys, vals)
+        if np.array_equal(g["offsets"], ix.offsets) and np.array_equal(g["perm"], ix.perm):
+            assert np.all(np.abs(g["centroids"] - ix.centroids) <= ulp(ix.centroids, dtype))
+            assert np.all(np.abs(g["value_sums"] - ix.value_sums) <= ulp(ix.value_sums, dtype))
+        else:  # a near-tie flipped a token: the index is still valid; count the difference
+            lab_g = np.repeat(np.arange(len(ix.offsets) - 1), np.diff(g["offsets"]))
+            lab_o = np.repeat(np.arange(len(ix.offsets) - 1), np.diff(ix.offsets))
+            pos_g = np.empty_like(lab_g); pos_g[g["perm"]] = lab_g
+            pos_o = np.empty_like(lab_o); pos_o[ix.perm] = lab_o
+            assert np.count_nonzero(pos_g != pos_o) <= 2
+
+
+def test_full_build_valid_and_objective_close():
+    wl = wl_small(seq_lens=(2500, 4097))
+    wx = gpu_build(wl, iters=10)
+    ref = H.oracle_build(wl, iters=10)
+    keys, vals = H.host_rows(wl)
+    for (b, h), ix in ref.items():
+        g = check_valid(wl, wx, b, h, keys, vals)
+        T = wl.seq_lens[b]
+        lab_g = np.empty(T, dtype=np.int64)
+        lab_g[g["perm"]] = np.repeat(np.arange(len(g["offsets"]) - 1), np.diff(g["offsets"]))
+        obj_g = sum(np.sum((keys[b][h] - g["centroids"][lab_g]) ** 2, axis=1))
+        obj_o = sum(np.sum((keys[b][h] - ix.centroids[ix.labels]) ** 2, axis=1))
+        assert abs(obj_g - obj_o) <= 0.02 * obj_o, (obj_g, obj_o)
+
+
+def test_build_then_decode_all_retrieved_is_dense():
+    """End to end on the GPU-built index: retrieving every cluster must give
+    full attention over the original keys and values (any index does)."""
+    wl = wl_small(seq_lens=(3000, 1100))
+    wx = gpu_build(wl, iters=4)
+    p = W.DecodeParams(n_q_heads=wl.n_q_heads, n_sink=4, window=64, topk_clusters=1 << 30)
+    out, lse = W.decode(wl.q.to(DEV), wx, p)
+    out = out.cpu().numpy().astype(np.float64)
+    keys, vals = H.host_rows(wl)
+    qh = H.q_host(wl)
+    G = wl.n_q_heads // wl.n_kv_heads
+    for b in range(wl.batch):
+        for h in range(wl.n_kv_heads):
+            dense, _ = O.dense_attention(qh[b, h * G:(h + 1) * G], keys[b][h], vals[b][h])
+            assert H.rel_err(out[b, h * G:(h + 1) * G], dense, wl.dtype) <= 2e-4
+
+
+def test_build_repeat_is_bit_identical():
+    wl = wl_small(seq_lens=(2100,))
+    a = gpu_build(wl, iters=3)
+    b = gpu_build(wl, iters=3)
+    for name in ["centroids", "value_sums", "offsets", "perm", "invperm", "k_pool", "v_pool"]:
+        assert torch.equal(getattr(a, name), getattr(b, name)), name

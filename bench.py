@@ -116,11 +116,13 @@ class ClockSampler:
 
 def algorithmic_bytes(index, params, info: np.ndarray, n_st_per_seq):
     """Bytes the method must move in one decode step (centroids, value sums,
-    offsets, retrieved K/V rows + perm, steady K/V rows + invperm, q, out, lse)."""
+    offsets, retrieved K/V rows, steady K/V rows + invperm, q, out, lse), and
+    the share each launch moves: score reads centroids + offsets + q;
+    attend_estimate reads value sums + offsets + retrieved and steady rows."""
     e = 2 if index.dtype == torch.bfloat16 else 4
     d = index.head_dim
     H = index.n_kv_heads
-    per_stage = {"score": 0, "estimate": 0, "attend": 0}
+    per_stage = {"score": 0, "topk": 0, "attend_estimate": 0}
     total = 0
     for b, T in enumerate(index.seq_lens):
         NC = index.nc[b]
@@ -130,12 +132,11 @@ def algorithmic_bytes(index, params, info: np.ndarray, n_st_per_seq):
         sel_tok = int(sum(info[b * H + h, 3] for h in range(H)))
         dense = bool(info[b * H, 6])
         st = T if dense else n_st_per_seq[b]
-        retr = sel_tok * (2 * d * e + 4)
+        retr = sel_tok * 2 * d * e
         steady = H * st * (2 * d * e + 4)
         qo = params.n_q_heads * d * e + params.n_q_heads * (d + 1) * 4
         per_stage["score"] += cent + offs + params.n_q_heads * d * e
-        per_stage["estimate"] += vs + offs
-        per_stage["attend"] += retr + steady
+        per_stage["attend_estimate"] += vs + offs + retr + steady + params.n_q_heads * (d + 1) * 4
         total += cent + vs + offs + retr + steady + qo
     return total, per_stage
 
@@ -149,7 +150,8 @@ def steady_count(T, n_sink, window):
 def clone_index(wx):
     import copy
     c = copy.copy(wx)
-    for name in ["centroids", "value_sums", "offsets", "perm", "invperm", "k_pool", "v_pool"]:
+    for name in ["centroids", "value_sums", "offsets", "perm", "invperm", "labels", "k_pool",
+                 "v_pool"]:
         setattr(c, name, getattr(wx, name).clone())
     return c
 
@@ -295,7 +297,7 @@ def run_wave(args, rank, world, local_rank):
 
     peaks, peak_kind = measured_peaks()
     hbm = float(peaks["hbm_gbs"])
-    dom = max(("score", "estimate", "attend"), key=lambda k: stage_us[k])
+    dom = max(("score", "attend_estimate"), key=lambda k: stage_us[k])
     dom_gbs = stage_bytes[dom] / (stage_us[dom] * 1e-6) / 1e9
     step_gbs = step_bytes / (us_per_step * 1e-6) / 1e9
     tokens = sum(wl.seq_lens)

@@ -75,6 +75,8 @@ typedef enum wi_dtype { WI_F32 = 0, WI_BF16 = 1 } wi_dtype;
 #define WI_DEV_BAD_PAGE    0x1u  /* block-table entry outside [0, n_pages)      */
 #define WI_DEV_BAD_SLOT    0x2u  /* perm / invperm value outside [0, T_b)       */
 #define WI_DEV_BAD_CLUSTER 0x4u  /* offsets not monotone or cluster out of range */
+#define WI_DEV_BAD_HIST    0x8u  /* stale selection histogram (workspace reused
+                                    after a failed call); recomputed, result valid */
 
 /*
  * Paged KV cache in original token order (the build input).
@@ -117,6 +119,8 @@ typedef struct wi_index {
                                   NC_b+1 entries per unit, last = T_b           */
   int32_t *perm;               /* [Hkv*sum T_b]  slot -> original position      */
   int32_t *invperm;            /* [Hkv*sum T_b]  original position -> slot      */
+  int32_t *labels;             /* [Hkv*sum T_b]  original position -> cluster id
+                                  (0..NC_b-1, unit-local)                       */
   void *k_pool;                /* [n_pages][Hkv][P][d]  keys in slot order      */
   void *v_pool;                /* [n_pages][Hkv][P][d]  values in slot order    */
   int64_t n_pages;
@@ -147,6 +151,11 @@ typedef struct wi_decode_layout {
                           in ascending id, sel_count[u] of them                   */
   size_t unit_info;    /* int32 [B*Hkv][8]: {sel_count, thr_key, thr_idx,
                           sel_tokens, steady, n_affected, dense, k}              */
+  size_t gather;       /* int32 [B*Hkv][gather_stride]: per unit, the pool row of
+                          each exactly attended token (retrieved clusters in id
+                          order, -1 for their steady members, then the steady
+                          slots); sel_tokens + steady entries are valid          */
+  int64_t gather_stride;
   int32_t n_splits;    /* exact-attention splits per unit                        */
   int32_t n_est_chunks;/* estimation chunks per unit                             */
 } wi_decode_layout;
@@ -171,10 +180,11 @@ wi_status wi_build_workspace_size(const wi_kv_cache *kv, int32_t seg_len,
  * positions 0, cs, 2cs, ...; then `iters` rounds of
  *   assign: each key to the centroid at least squared Euclidean distance
  *           (fp32, direct form sum (k-c)^2; ties to the lower index),
- *   update: each centroid to the fp32 mean of its members summed in
- *           ascending position; an empty cluster keeps its centroid.
+ *   update: each centroid to the mean of its members (fp64 sum in
+ *           ascending position, kept as fp32 for the next assignment); an
+ *           empty cluster keeps its centroid.
  * Then writes `out`: centroids (the final means) and value sums rounded to
- * the KV dtype (round-to-nearest-even), offsets, perm, invperm, and the K/V
+ * the KV dtype (round-to-nearest-even), offsets, perm, invperm, labels, and the K/V
  * rows scattered into out->k_pool/v_pool in slot order through
  * out->block_table.  Requires seg_len % cluster_size == 0, seg_len <=
  * WI_MAX_SEG_LEN, iters >= 1, and `out` geometry equal to `kv`'s.

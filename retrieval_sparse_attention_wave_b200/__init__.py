@@ -39,7 +39,7 @@ WI_F32, WI_BF16 = 0, 1
 WI_MAX_BATCH = 256
 WI_MAX_SEG_LEN = 16384
 WI_MAX_STEADY = 8192
-WI_DEV_BAD_PAGE, WI_DEV_BAD_SLOT, WI_DEV_BAD_CLUSTER = 0x1, 0x2, 0x4
+WI_DEV_BAD_PAGE, WI_DEV_BAD_SLOT, WI_DEV_BAD_CLUSTER, WI_DEV_BAD_HIST = 0x1, 0x2, 0x4, 0x8
 
 EXPORTED = [
     "wi_index_clusters", "wi_build_workspace_size", "wi_build_index", "wi_kmeans_assign",
@@ -61,7 +61,8 @@ class WiIndex(C.Structure):
                 ("head_dim", C.c_int32), ("page_size", C.c_int32), ("seg_len", C.c_int32),
                 ("cluster_size", C.c_int32), ("seq_lens", C.POINTER(C.c_int32)),
                 ("centroids", C.c_void_p), ("value_sums", C.c_void_p), ("offsets", C.c_void_p),
-                ("perm", C.c_void_p), ("invperm", C.c_void_p), ("k_pool", C.c_void_p),
+                ("perm", C.c_void_p), ("invperm", C.c_void_p), ("labels", C.c_void_p),
+                ("k_pool", C.c_void_p),
                 ("v_pool", C.c_void_p), ("n_pages", C.c_int64), ("block_table", C.c_void_p),
                 ("max_pages", C.c_int32)]
 
@@ -75,6 +76,7 @@ class WiDecodeParams(C.Structure):
 class WiDecodeLayout(C.Structure):
     _fields_ = [("total_bytes", C.c_size_t), ("status", C.c_size_t), ("scores", C.c_size_t),
                 ("keys", C.c_size_t), ("selected", C.c_size_t), ("unit_info", C.c_size_t),
+                ("gather", C.c_size_t), ("gather_stride", C.c_int64),
                 ("n_splits", C.c_int32), ("n_est_chunks", C.c_int32)]
 
 
@@ -241,6 +243,7 @@ class WaveIndex:
         self.offsets = torch.zeros(H * (sum(self.nc) + B), dtype=torch.int32, device=dev)
         self.perm = torch.zeros(ntok, dtype=torch.int32, device=dev)
         self.invperm = torch.zeros(ntok, dtype=torch.int32, device=dev)
+        self.labels = torch.zeros(ntok, dtype=torch.int32, device=dev)
         if block_table is None:
             block_table = contiguous_block_table(self.seq_lens, page_size, dev)
         if n_pages is None:
@@ -275,6 +278,7 @@ class WaveIndex:
         s.offsets = self.offsets.data_ptr()
         s.perm = self.perm.data_ptr()
         s.invperm = self.invperm.data_ptr()
+        s.labels = self.labels.data_ptr()
         s.k_pool = self.k_pool.data_ptr()
         s.v_pool = self.v_pool.data_ptr()
         s.n_pages = self.k_pool.shape[0]
@@ -349,6 +353,9 @@ class DecodeParams:
         p.n_q_heads, p.n_sink, p.window = self.n_q_heads, self.n_sink, self.window
         p.topk_clusters, p.topk_fraction = self.topk_clusters, self.topk_fraction
         if events is not None:
+            for e in events:
+                if not e.cuda_event:      # torch creates the CUDA event on first record
+                    e.record()
             arr = (C.c_void_p * len(events))(*[e.cuda_event for e in events])
             p.stage_events = C.cast(arr, C.POINTER(C.c_void_p))
             p._keep = arr
@@ -420,6 +427,12 @@ def selected_clusters(ws: torch.Tensor, layout: WiDecodeLayout, index: WaveIndex
                       b: int, h: int, count: int) -> torch.Tensor:
     row = index.cl_row(b, h)
     return ws[layout.selected:].view(torch.int32)[row:row + count]
+
+
+def gather_rows(ws: torch.Tensor, layout: WiDecodeLayout, u: int, count: int) -> torch.Tensor:
+    """Pool row indices of unit u's exactly attended tokens (-1 = skipped)."""
+    base = u * layout.gather_stride
+    return ws[layout.gather:].view(torch.int32)[base:base + count]
 
 
 def centroid_scores(ws: torch.Tensor, layout: WiDecodeLayout, index: WaveIndex, G: int,

@@ -79,10 +79,6 @@ int64_t n_steady(int64_t T, int64_t n_sink, int64_t window) {
   return ns + (T - ws);
 }
 
-int rows_per_warp(int dtype, int D) {
-  const int epl = 16 / esize((wi_dtype)dtype);
-  return 32 / (D / epl);
-}
 
 wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, DecodePlan& pl) {
   if (!ix || !p) return WI_ERR_INVALID_ARG;
@@ -91,12 +87,14 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
                               ix->max_pages, ix->seq_lens);
   if (st != WI_OK) return st;
   if ((st = check_seg(ix->seg_len, ix->cluster_size)) != WI_OK) return st;
-  if (!ix->centroids || !ix->value_sums || !ix->offsets || !ix->perm || !ix->invperm)
+  if (!ix->centroids || !ix->value_sums || !ix->offsets || !ix->perm || !ix->invperm ||
+      !ix->labels)
     return WI_ERR_INVALID_ARG;
   if (!aligned(ix->centroids, 16) || !aligned(ix->value_sums, 16) || !aligned(ix->offsets, 4) ||
-      !aligned(ix->perm, 4) || !aligned(ix->invperm, 4))
+      !aligned(ix->perm, 4) || !aligned(ix->invperm, 4) || !aligned(ix->labels, 4))
     return WI_ERR_INVALID_ARG;
   if (p->n_q_heads < 1 || p->n_q_heads % ix->n_kv_heads != 0) return WI_ERR_INVALID_ARG;
+  if (ix->n_pages * ix->n_kv_heads * ix->page_size >= INT32_MAX) return WI_ERR_UNSUPPORTED;
   const int G = p->n_q_heads / ix->n_kv_heads;
   if (G != 1 && G != 2 && G != 4 && G != 8) return WI_ERR_UNSUPPORTED;
   if (p->n_sink < 0 || p->window < 0) return WI_ERR_INVALID_ARG;
@@ -135,38 +133,49 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   pl.sort_pow2 = 1;
   while (pl.sort_pow2 < cap) pl.sort_pow2 <<= 1;
 
-  // score: ~8 CTAs of 256 threads per SM
-  const int rows_it = 8 * rows_per_warp(pl.dtype, pl.D) * 4;
-  const int64_t total_rows = (int64_t)max_nc * pl.U;
-  const int64_t iters = std::max<int64_t>(1, cdiv(total_rows, (int64_t)rows_it * kNumSMs * 8));
-  pl.score_chunk = (int)(rows_it * iters);
+  pl.seg_len = ix->seg_len;
+  pl.seg_clusters = ix->seg_len / ix->cluster_size;
+  // score: one CTA per 64 KB of centroid rows
+  pl.score_chunk = 65536 / (pl.D * esize(ix->dtype));
   pl.n_score_blocks = (int)cdiv(max_nc, pl.score_chunk);
-  // exact attention: ~2 CTAs per SM overall, at least ~128 tokens per CTA
-  int ns = (int)cdiv(2 * kNumSMs, pl.U);
-  ns = (int)std::min<int64_t>(ns, cdiv(max_tok, 128));
-  ns = (int)std::max<int64_t>(ns, cdiv(max_tok, 4096));
-  pl.n_splits = std::max(1, std::min(ns, 1024));
-  // estimation: ~2 CTAs per SM overall, 256..2048 clusters each
-  int64_t ec = cdiv(total_rows, 2 * kNumSMs);
-  ec = std::max<int64_t>(256, std::min<int64_t>(2048, cdiv(ec, 256) * 256));
-  pl.echunk = (int)ec;
+  pl.topk_smem_keys = (int)cdiv(max_nc, kTopkCluster);
+  if (pl.topk_smem_keys > 20480) return WI_ERR_UNSUPPORTED;   // > 163,840 clusters per sequence
+  // exact attention: about two 16 KB tiles of rows per CTA
+  const int row_bytes = pl.D * esize(ix->dtype);
+  const int tile_rows = 16384 / row_bytes;
+  int ns = (int)cdiv(max_tok, 2 * tile_rows);
+  pl.n_splits = std::max(1, std::min(ns, 4096));
+  // estimation: 512 clusters per CTA (4 prefetched tiles + the rest streamed)
+  pl.echunk = 512;
   pl.n_est = (int)cdiv(max_nc, pl.echunk);
   pl.n_parts = pl.n_splits + pl.n_est;
+  pl.wcap = std::max(pl.echunk, pl.n_parts);
+  if (decode_attend_smem(pl.dtype, pl.D, G, pl.wcap, pl.echunk, cap) > 200 * 1024)
+    return WI_ERR_UNSUPPORTED;
 
   const int64_t ncl = (int64_t)pl.geo.cl_base[ix->batch] * ix->n_kv_heads;
   size_t o = 0;
   auto take = [&](size_t bytes) { const size_t r = o; o = align_up(o + bytes, 256); return r; };
   pl.off_status = take(256);
+  pl.off_counters = take((size_t)pl.U * 4);
+  pl.off_hist = take((size_t)pl.U * 2048 * 4);   // zeroed after use by the top-k kernel
   pl.off_scores = take((size_t)ncl * G * 4);
   pl.off_keys = take((size_t)ncl * 4);
   pl.off_sel = take((size_t)ncl * 4);
+  pl.off_sel_slot0 = take((size_t)ncl * 4);
   pl.off_seltok = take((size_t)(ncl + pl.U) * 4);
+  pl.off_split = take((size_t)pl.U * (pl.n_splits + 1) * 4);
   pl.off_info = take((size_t)pl.U * kInfoInts * 4);
   pl.off_st_slot = take((size_t)pl.U * cap * 4);
   pl.off_st_cl = take((size_t)pl.U * cap * 4);
   pl.off_aff_cl = take((size_t)pl.U * cap * 4);
   pl.off_aff_start = take((size_t)pl.U * (cap + 1) * 4);
-  pl.off_partials = take((size_t)pl.U * pl.n_parts * G * (pl.D + 2) * 4);
+  pl.off_partials = take((size_t)pl.U * pl.n_parts * G * (pl.D + 4) * 4);
+  int64_t tmax = 0;
+  for (int b = 0; b < ix->batch; ++b) tmax = std::max<int64_t>(tmax, ix->seq_lens[b]);
+  pl.gather_stride = tmax + cap;   // retrieved slots (steady members as -1) + steady slots
+  pl.off_gather = take((size_t)pl.U * pl.gather_stride * 4);
+  pl.off_dv = take((size_t)pl.U * cap * pl.D * 4);
   const size_t nq = (size_t)ix->batch * p->n_q_heads;
   pl.off_q = take(nq * pl.D * esize(ix->dtype));
   pl.off_out = take(nq * pl.D * 4);
@@ -242,6 +251,7 @@ wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params*
   a.offsets = ix->offsets;
   a.perm = ix->perm;
   a.invperm = ix->invperm;
+  a.labels = ix->labels;
   a.kp = make_pool(ix->k_pool, ix->block_table, ix->n_pages, ix->max_pages, ix->page_size);
   a.vp = make_pool(ix->v_pool, ix->block_table, ix->n_pages, ix->max_pages, ix->page_size);
   a.out = out;
@@ -308,10 +318,11 @@ wi_status wi_build_index(const wi_kv_cache* kv, int32_t seg_len, int32_t cluster
                     out->n_pages, out->k_pool, out->v_pool, out->block_table, out->max_pages,
                     out->seq_lens);
   if (st != WI_OK) return st;
-  if (!out->centroids || !out->value_sums || !out->offsets || !out->perm || !out->invperm)
+  if (!out->centroids || !out->value_sums || !out->offsets || !out->perm || !out->invperm ||
+      !out->labels)
     return WI_ERR_INVALID_ARG;
   if (!aligned(out->centroids, 16) || !aligned(out->value_sums, 16) || !aligned(out->offsets, 4) ||
-      !aligned(out->perm, 4) || !aligned(out->invperm, 4))
+      !aligned(out->perm, 4) || !aligned(out->invperm, 4) || !aligned(out->labels, 4))
     return WI_ERR_INVALID_ARG;
   if (out->k_pool == kv->k_pool || out->v_pool == kv->v_pool || out->k_pool == kv->v_pool ||
       out->v_pool == kv->k_pool)
@@ -326,6 +337,7 @@ wi_status wi_build_index(const wi_kv_cache* kv, int32_t seg_len, int32_t cluster
   a.offsets = out->offsets;
   a.perm = out->perm;
   a.invperm = out->invperm;
+  a.labels = out->labels;
   a.kout = out->k_pool;
   a.vout = out->v_pool;
   a.bt_out = out->block_table;
@@ -376,6 +388,8 @@ wi_status wi_decode_workspace_layout(const wi_index* idx, const wi_decode_params
   layout->keys = pl.off_keys;
   layout->selected = pl.off_sel;
   layout->unit_info = pl.off_info;
+  layout->gather = pl.off_gather;
+  layout->gather_stride = pl.gather_stride;
   layout->n_splits = pl.n_splits;
   layout->n_est_chunks = pl.n_est;
   return WI_OK;

@@ -8,8 +8,8 @@
 //           ||k||^2 - 2k.c + ||c||^2 cancellation), ties to the lower j;
 //           64 tokens x 64 centroids per tile, 4x4 outputs per thread
 //   update  per (unit, segment): stable counting sort of the tokens by
-//           cluster, fp32 sums in ascending position, mean = sum / count;
-//           on the last round it also writes offsets, perm, invperm, the
+//           cluster, fp64 sums in ascending position, mean = sum / count;
+//           on the last round it also writes offsets, perm, invperm, labels, the
 //           rounded centroids and value sums, and copies the K/V rows to the
 //           permuted pools (one pass over K and V).
 #include <cfloat>
@@ -176,6 +176,7 @@ struct FinalOut {
   int32_t* offsets;
   int32_t* perm;
   int32_t* invperm;
+  int32_t* labels;
   void* kout;
   void* vout;
   Pool pout;   // block table / geometry of the permuted pools
@@ -252,9 +253,11 @@ kmeans_update_kernel(const Geo geo, const Pool kin, int S, int cs, float* __rest
   const T* kb = reinterpret_cast<const T*>(kin.base) + sub * R::EPL;
   for (int j = warp * R::RPW + rsub; j < ncl; j += groups) {
     const int m0 = s_start[j], m1 = s_start[j + 1];
-    float ks[R::EPL], vs[R::EPL];
+    // member sums in fp64: the stored mean / sum is then the correctly rounded
+    // value of the exact one (the fp32 working centroid too)
+    double ks[R::EPL], vs[R::EPL];
 #pragma unroll
-    for (int e = 0; e < R::EPL; ++e) { ks[e] = 0.f; vs[e] = 0.f; }
+    for (int e = 0; e < R::EPL; ++e) { ks[e] = 0.0; vs[e] = 0.0; }
     for (int m = m0; m < m1; ++m) {
       const int p = start + s_mem[m];
       const int64_t ro = pool_row(kin, geo.hkv, D, b, h, p, status);
@@ -263,7 +266,7 @@ kmeans_update_kernel(const Geo geo, const Pool kin, int S, int cs, float* __rest
       float x[R::EPL];
       Elem<T>::unpack(kraw, x);
 #pragma unroll
-      for (int e = 0; e < R::EPL; ++e) ks[e] += x[e];
+      for (int e = 0; e < R::EPL; ++e) ks[e] += (double)x[e];
       if (fo.enabled) {
         const int slot = start + m;
         const int64_t vo = pool_row(fo.vin, geo.hkv, D, b, h, p, status);
@@ -272,7 +275,7 @@ kmeans_update_kernel(const Geo geo, const Pool kin, int S, int cs, float* __rest
         if (vo >= 0) vraw = ld_stream(reinterpret_cast<const T*>(fo.vin.base) + vo + sub * R::EPL);
         Elem<T>::unpack(vraw, x);
 #pragma unroll
-        for (int e = 0; e < R::EPL; ++e) vs[e] += x[e];
+        for (int e = 0; e < R::EPL; ++e) vs[e] += (double)x[e];
         if (oo >= 0) {
           *reinterpret_cast<uint4*>(reinterpret_cast<T*>(fo.kout) + oo + sub * R::EPL) = kraw;
           *reinterpret_cast<uint4*>(reinterpret_cast<T*>(fo.vout) + oo + sub * R::EPL) = vraw;
@@ -280,21 +283,25 @@ kmeans_update_kernel(const Geo geo, const Pool kin, int S, int cs, float* __rest
         if (sub == 0) {
           fo.perm[trow + slot] = p;
           fo.invperm[trow + p] = slot;
+          fo.labels[trow + p] = seg * (S / cs) + j;
         }
       }
     }
     const int cnt = m1 - m0;
     float* c32 = cent32 + (crow + j) * D + sub * R::EPL;
+    double mean[R::EPL];
+#pragma unroll
+    for (int e = 0; e < R::EPL; ++e) mean[e] = cnt > 0 ? ks[e] / (double)cnt : (double)c32[e];
     if (cnt > 0) {
 #pragma unroll
-      for (int e = 0; e < R::EPL; ++e) c32[e] = ks[e] / (float)cnt;
+      for (int e = 0; e < R::EPL; ++e) c32[e] = __double2float_rn(mean[e]);
     }
     if (fo.enabled) {
       T* cdst = reinterpret_cast<T*>(fo.centroids) + (crow + j) * D + sub * R::EPL;
       T* vdst = reinterpret_cast<T*>(fo.value_sums) + (crow + j) * D + sub * R::EPL;
 #pragma unroll
       for (int e = 0; e < R::EPL; ++e) {
-        store_elem(cdst + e, c32[e]);
+        store_elem(cdst + e, mean[e]);
         store_elem(vdst + e, vs[e]);
       }
       if (sub == 0) fo.offsets[geo.off_row(b, h) + seg * (S / cs) + j] = start + m0;
@@ -353,6 +360,7 @@ cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s)
     fin.offsets = a.offsets;
     fin.perm = a.perm;
     fin.invperm = a.invperm;
+    fin.labels = a.labels;
     fin.kout = a.kout;
     fin.vout = a.vout;
     fin.pout = Pool{a.kout, a.bt_out, a.n_pages_out, a.max_pages_out, a.page_shift_out};

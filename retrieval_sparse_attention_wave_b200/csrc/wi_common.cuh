@@ -99,6 +99,9 @@ template <> struct Elem<__nv_bfloat16> {
 
 __device__ __forceinline__ void store_elem(float* p, float v) { *p = v; }
 __device__ __forceinline__ void store_elem(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+// Round-to-nearest-even from double straight to the storage type (no double rounding).
+__device__ __forceinline__ void store_elem(float* p, double v) { *p = __double2float_rn(v); }
+__device__ __forceinline__ void store_elem(__nv_bfloat16* p, double v) { *p = __double2bfloat16(v); }
 
 // Order-preserving map of a float to uint32 (larger float -> larger key).
 // Key 0 is reserved for "not a candidate".
@@ -154,6 +157,97 @@ __device__ __forceinline__ int warp_sum_int(int v) {
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
+}
+
+// Programmatic dependent launch: let the next kernel in the stream start its
+// prologue now / wait until the previous kernel's results are visible.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// 16-byte asynchronous global -> shared copy (L2 only) and its group fences.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Wait until at most n of this thread's cp.async groups are pending (n <= 7).
+__device__ __forceinline__ void cp_async_wait_dyn(int n) {
+  switch (n) {
+    case 0: cp_async_wait<0>(); break;
+    case 1: cp_async_wait<1>(); break;
+    case 2: cp_async_wait<2>(); break;
+    case 3: cp_async_wait<3>(); break;
+    case 4: cp_async_wait<4>(); break;
+    case 5: cp_async_wait<5>(); break;
+    case 6: cp_async_wait<6>(); break;
+    default: cp_async_wait<7>(); break;
+  }
+}
+
+// Dot products of one 16-byte vector (EPL elements, already fp32) with G
+// query slices, two lanes of packed fp32 FMA (sm_100 FFMA2) at a time.
+template <int G, int EPL>
+__device__ __forceinline__ void dot_g(const float (&qv)[G][EPL], const float (&x)[EPL],
+                                      float (&acc)[G]) {
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int e = 0; e < EPL; e += 2)
+      a = __ffma2_rn(make_float2(qv[g][e], qv[g][e + 1]), make_float2(x[e], x[e + 1]), a);
+    acc[g] = a.x + a.y;
+  }
+}
+
+// acc[g][e] += w[g] * x[e] with packed fp32 FMA.
+template <int G, int EPL>
+__device__ __forceinline__ void axpy_g(const float (&w)[G], const float (&x)[EPL],
+                                       float (&acc)[G][EPL]) {
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < EPL; e += 2) {
+      const float2 r = __ffma2_rn(make_float2(w[g], w[g]), make_float2(x[e], x[e + 1]),
+                                  make_float2(acc[g][e], acc[g][e + 1]));
+      acc[g][e] = r.x;
+      acc[g][e + 1] = r.y;
+    }
+}
+
+// Inclusive scan of two ints per thread over the block (as block_inclusive_scan).
+// `sh` needs 64 ints.
+__device__ __forceinline__ int2 block_inclusive_scan2(int2 x, int* sh, int2* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ya = __shfl_up_sync(0xffffffffu, x.x, o);
+    const int yb = __shfl_up_sync(0xffffffffu, x.y, o);
+    if (lane >= o) { x.x += ya; x.y += yb; }
+  }
+  if (lane == 31) { sh[w] = x.x; sh[32 + w] = x.y; }
+  __syncthreads();
+  if (w == 0) {
+    int a = lane < nw ? sh[lane] : 0, c = lane < nw ? sh[32 + lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ya = __shfl_up_sync(0xffffffffu, a, o);
+      const int yc = __shfl_up_sync(0xffffffffu, c, o);
+      if (lane >= o) { a += ya; c += yc; }
+    }
+    sh[lane] = a; sh[32 + lane] = c;
+  }
+  __syncthreads();
+  const int2 r = make_int2(x.x + (w > 0 ? sh[w - 1] : 0), x.y + (w > 0 ? sh[32 + w - 1] : 0));
+  *total = make_int2(sh[nw - 1], sh[32 + nw - 1]);
+  __syncthreads();
+  return r;
 }
 
 // Inclusive scan of one int per thread over the block (blockDim.x multiple of

@@ -1,34 +1,44 @@
 // Decode-step kernels of the wave index (sm_100a).
 //
-// One decode step is the query-dependent phase of the method
-// (RetroInfer technical summary, section 2.A, items 1-3; Vortex summary,
-// section 2.A forward_indexer):
-//   steady    resolve the steady zone (sinks + recent window) to slots and
-//             clusters (query-independent; item 1 Steady Zone)
-//   score     q . centroid / sqrt(d) for every cluster, per q head, and the
-//             group-max selection key (item 2, the index lookup)
-//   topk      exact radix select of the k best candidate clusters per KV head
-//             (item 2; Vortex 2.C Top-K), ties to the lower cluster id
-//   attend    gather the retrieved clusters' rows plus the steady rows from the
-//             cluster-permuted paged layout and run split-K exact attention
-//             (items 1 and 2)
-//   estimate  every other candidate cluster as cnt' * e^s with value sum
-//             Vsum' (item 3 Estimation Zone)
-//   merge     log-sum-exp combine of all partial softmax parts
-// All streaming kernels read 16-byte vectors with the row of one cluster or
-// token spread over LPR = d*sizeof(T)/16 lanes; the score / estimate GEMVs
-// have M = G <= 8 rows, so they run on the CUDA cores (FFMA), not tensor cores.
+// One decode step is the query-dependent phase of the method (RetroInfer
+// technical summary, section 2.A, items 1-3; Vortex summary, section 2.A
+// forward_indexer).  Three launches, chained with programmatic dependent
+// launch so each one's prologue overlaps the previous one's tail:
+//
+//  K_A score    q . centroid / sqrt(d) for every cluster and q head, and the
+//               group-max selection key (item 2, the index lookup).  U extra
+//               CTAs resolve the steady zone (item 1): sink and window
+//               positions -> slots -> clusters, run-length encoded.
+//  K_B topk     exact radix select (11+11+10-bit digits) of the k best
+//               candidate clusters per KV head, ties to the lower id (Vortex
+//               2.C Top-K), and the gather plan (slot starts, token prefix,
+//               split boundaries).
+//  K_C attend + estimate
+//               attend CTAs: gather the retrieved clusters' rows and the
+//               steady rows from the cluster-permuted paged layout into
+//               shared memory (16-byte cp.async) and run split-K exact
+//               attention (items 1 and 2);
+//               estimate CTAs: prefetch their value-sum rows into a shared
+//               memory ring before waiting on K_B, then add every other
+//               candidate cluster as cnt' * e^s with value sum Vsum'
+//               (item 3 Estimation Zone);
+//               the last CTA of each unit merges all parts by log-sum-exp.
+//
+// The score / estimate GEMVs have M = G <= 8 rows, so they run on the CUDA
+// cores (FFMA); every row is spread over LPR = d*sizeof(T)/16 lanes.
 #include <cfloat>
 #include <climits>
+#include <algorithm>
 #include <cmath>
+
+#include <cooperative_groups.h>
 
 #include "wi_common.cuh"
 #include "wi_plan.h"
 
 namespace wi {
 
-const char* const kDecodeStageNames[kDecodeStages] = {"steady", "score", "topk",
-                                                      "attend", "estimate", "merge"};
+const char* const kDecodeStageNames[kDecodeStages] = {"score", "topk", "attend_estimate"};
 
 namespace {
 
@@ -37,6 +47,8 @@ struct RowShape {
   static constexpr int EPL = Elem<T>::kPerVec;  // elements per lane (one 16-B vector)
   static constexpr int LPR = D / EPL;           // lanes per row
   static constexpr int RPW = 32 / LPR;          // rows per warp step
+  static constexpr int ROWB = D * (int)sizeof(T);
+  static constexpr int TILE = 16384 / ROWB;     // rows per 16 KB shared-memory tile
 };
 
 template <typename T, int D, int G>
@@ -53,40 +65,58 @@ __device__ __forceinline__ void load_q(const T* q, int n_q_heads, int b, int h, 
   }
 }
 
-// ------------------------------------------------------------------ steady
-// One CTA per unit.  Maps the steady positions to slots (invperm), sorts the
-// slots (bitonic, shared memory), finds each slot's cluster (binary search in
-// offsets) and run-length encodes the clusters ("affected" clusters with
-// their steady-member ranges).
-__global__ void __launch_bounds__(kStreamThreads)
-wave_steady_kernel(const Geo geo, const int32_t* __restrict__ invperm,
-                   const int32_t* __restrict__ offsets, int n_sink, int window, int cap,
-                   int sort_pow2, int32_t* __restrict__ st_slot, int32_t* __restrict__ st_cl,
-                   int32_t* __restrict__ aff_cl, int32_t* __restrict__ aff_start,
-                   int32_t* __restrict__ info, uint32_t* status) {
-  extern __shared__ int32_t sh_sort[];
-  const int u = blockIdx.x, b = u / geo.hkv, h = u - b * geo.hkv;
-  const int T = geo.T(b), NC = geo.NC(b);
-  const int ns = min(n_sink, T);
-  const int wstart = max(T - window, ns);
-  const int n_st = ns + (T - wstart);
-  int32_t* I = info + (int64_t)u * kInfoInts;
-  if (n_st >= T) {  // all steady: attended densely, nothing retrieved or estimated
-    if (threadIdx.x == 0) { I[4] = T; I[5] = 0; I[6] = 1; }
+// Binary search in a sorted shared-memory array: index of x or -1.
+__device__ __forceinline__ int find_sorted(const int32_t* a, int n, int x) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] < x) lo = mid + 1; else hi = mid;
+  }
+  return (lo < n && a[lo] == x) ? lo : -1;
+}
+
+struct SteadyArgs {
+  const int32_t* invperm;
+  const int32_t* labels;
+  Pool vp;
+  int n_sink, window, cap, sort_pow2;
+  int32_t *st_slot, *st_cl, *aff_cl, *aff_start, *info;
+  float* dv;  // [U][cap][D] fp32: sum of the steady members' values per affected cluster
+};
+
+// Steady zone of unit u: positions -> (slot, cluster) through invperm and
+// labels (one round of independent loads), sorted by slot (which also
+// groups them by cluster, clusters being slot ranges), then run-length
+// encoded into (affected cluster, first steady index), and the value rows
+// of each affected cluster's steady members summed in slot order (dV).
+template <typename T, int D>
+__device__ void steady_role(const Geo& geo, int u, const SteadyArgs& a, uint32_t* status,
+                            unsigned long long* sh_sort) {
+  const int b = u / geo.hkv, h = u - b * geo.hkv;
+  const int Tb = geo.T(b), NC = geo.NC(b);
+  const int ns = min(a.n_sink, Tb);
+  const int wstart = max(Tb - a.window, ns);
+  const int n_st = ns + (Tb - wstart);
+  int32_t* I = a.info + (int64_t)u * kInfoInts;
+  if (n_st >= Tb) {  // all steady: attended densely, nothing retrieved or estimated
+    if (threadIdx.x == 0) { I[4] = Tb; I[5] = 0; I[6] = 1; }
     return;
   }
   int npow = 1;
   while (npow < n_st) npow <<= 1;
-  if (npow > sort_pow2) npow = sort_pow2;  // host guarantees n_st <= cap <= sort_pow2
-  const int32_t* inv = invperm + geo.tok_row(b, h);
+  npow = min(npow, a.sort_pow2);
+  const int32_t* inv = a.invperm + geo.tok_row(b, h);
+  const int32_t* lab = a.labels + geo.tok_row(b, h);
   for (int i = threadIdx.x; i < npow; i += blockDim.x) {
-    int32_t s = INT_MAX;
+    unsigned long long kv = ~0ull;
     if (i < n_st) {
       const int pos = i < ns ? i : wstart + (i - ns);
-      s = inv[pos];
-      if (s < 0 || s >= T) { flag_error(status, WI_DEV_BAD_SLOT); s = INT_MAX; }
+      int s = __ldg(inv + pos), c = __ldg(lab + pos);
+      if (s < 0 || s >= Tb) { flag_error(status, WI_DEV_BAD_SLOT); s = 0x7fffffff; }
+      if (c < 0 || c >= NC) { flag_error(status, WI_DEV_BAD_CLUSTER); c = 0; }
+      kv = ((unsigned long long)(uint32_t)s << 32) | (uint32_t)c;
     }
-    sh_sort[i] = s;
+    sh_sort[i] = kv;
   }
   __syncthreads();
   for (int k = 2; k <= npow; k <<= 1) {
@@ -95,38 +125,29 @@ wave_steady_kernel(const Geo geo, const int32_t* __restrict__ invperm,
         const int ixj = i ^ j;
         if (ixj > i) {
           const bool up = (i & k) == 0;
-          const int32_t a = sh_sort[i], c = sh_sort[ixj];
-          if ((a > c) == up) { sh_sort[i] = c; sh_sort[ixj] = a; }
+          const unsigned long long x = sh_sort[i], y = sh_sort[ixj];
+          if ((x > y) == up) { sh_sort[i] = y; sh_sort[ixj] = x; }
         }
       }
       __syncthreads();
     }
   }
-  const int32_t* off = offsets + geo.off_row(b, h);
-  int32_t* slots = st_slot + (int64_t)u * cap;
-  int32_t* cls = st_cl + (int64_t)u * cap;
+  int32_t* slots = a.st_slot + (int64_t)u * a.cap;
+  int32_t* cls = a.st_cl + (int64_t)u * a.cap;
   for (int i = threadIdx.x; i < n_st; i += blockDim.x) {
-    const int32_t s = sh_sort[i];
-    // largest c with off[c] <= s
-    int lo = 0, hi = NC;  // answer in [0, NC)
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (off[mid] <= s) lo = mid; else hi = mid - 1;
-    }
-    if (s != INT_MAX && (off[lo] > s || off[lo + 1] <= s)) flag_error(status, WI_DEV_BAD_CLUSTER);
-    slots[i] = s;
-    cls[i] = lo;
+    slots[i] = (int32_t)(sh_sort[i] >> 32);
+    cls[i] = (int32_t)(sh_sort[i] & 0xffffffffu);
   }
-  __syncthreads();
+  __shared__ int s_naff;
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
-    int32_t* acl = aff_cl + (int64_t)u * cap;
-    int32_t* ast = aff_start + (int64_t)u * (cap + 1);
+    int32_t* acl = a.aff_cl + (int64_t)u * a.cap;
+    int32_t* ast = a.aff_start + (int64_t)u * (a.cap + 1);
     int n_aff = 0;
     for (int base = 0; base < n_st; base += 32) {
       const int i = base + lane;
-      const int c = i < n_st ? cls[i] : -1;
-      const bool head = i < n_st && (i == 0 || cls[i - 1] != c);
+      const int c = i < n_st ? (int)(sh_sort[i] & 0xffffffffu) : -1;
+      const bool head = i < n_st && (i == 0 || (int)(sh_sort[i - 1] & 0xffffffffu) != c);
       const unsigned bal = __ballot_sync(0xffffffffu, head);
       if (head) {
         const int r = __popc(bal & ((1u << lane) - 1u));
@@ -138,395 +159,520 @@ wave_steady_kernel(const Geo geo, const int32_t* __restrict__ invperm,
     if (lane == 0) {
       ast[n_aff] = n_st;
       I[4] = n_st; I[5] = n_aff; I[6] = 0;
+      s_naff = n_aff;
     }
+  }
+  __syncthreads();
+  // dV: one group of LPR lanes per affected cluster, members in slot order
+  constexpr int EPL = Elem<T>::kPerVec, LPR = D / EPL, GPB = kStreamThreads / LPR;
+  const int lane = threadIdx.x & 31, sub = lane % LPR, grp = threadIdx.x / LPR;
+  const int n_aff = s_naff;
+  const int32_t* ast = a.aff_start + (int64_t)u * (a.cap + 1);
+  const T* vb = reinterpret_cast<const T*>(a.vp.base) + sub * EPL;
+  for (int j = grp; j < n_aff; j += GPB) {
+    float acc[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+    int i0 = 0, i1 = 0;  // steady index range of cluster j (recomputed from the sorted list)
+    {
+      // the j-th run head: count heads until j (runs are short; ast was written above)
+      i0 = ast[j];
+      i1 = ast[j + 1];
+    }
+    for (int i = i0; i < i1; ++i) {
+      const int slot = (int)(sh_sort[i] >> 32);
+      const int64_t ro = pool_row(a.vp, geo.hkv, D, b, h, slot, status);
+      if (ro >= 0) {
+        float x[EPL];
+        Elem<T>::unpack(ld_stream(vb + ro), x);
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] += x[e];
+      }
+    }
+    float* dst = a.dv + ((int64_t)u * a.cap + j) * D + sub * EPL;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) dst[e] = acc[e];
   }
 }
 
-// ------------------------------------------------------------------- score
+// ---------------------------------------------------------------- K_A score
+// Each CTA stages its chunk of centroid rows (64 KB) in shared memory with
+// 16-byte cp.async, scores it, writes the per-head scores and the
+// order-preserving group-max keys, and adds its keys' top 11 bits to the
+// unit's selection histogram (the first radix digit of the top-k).
+constexpr int kHistBins = 2048;
+constexpr int kHistShift = 21;
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kStreamThreads)
 wave_score_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const T* __restrict__ cent,
                   const int32_t* __restrict__ offsets, float* __restrict__ scores,
-                  uint32_t* __restrict__ keys, float scale, int chunk) {
+                  uint32_t* __restrict__ keys, int32_t* __restrict__ hist_g, float scale,
+                  int n_score_blocks, const SteadyArgs sa, uint32_t* status) {
   using RS = RowShape<T, D>;
-  constexpr int EPL = RS::EPL, LPR = RS::LPR, RPW = RS::RPW, UNR = 4;
+  constexpr int EPL = RS::EPL, LPR = RS::LPR, RPW = RS::RPW;
   constexpr int NW = kStreamThreads / 32;
+  constexpr int CROWS = 65536 / RS::ROWB;   // rows per CTA
   static_assert(G <= LPR, "group larger than lanes per row");
-  const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
+  extern __shared__ __align__(16) unsigned char sh_dyn[];
+  pdl_launch_dependents();
+  const int u = blockIdx.y;
+  if (blockIdx.x == n_score_blocks) {
+    steady_role<T, D>(geo, u, sa, status, reinterpret_cast<unsigned long long*>(sh_dyn));
+    return;
+  }
+  const int b = u / geo.hkv, h = u - b * geo.hkv;
   const int NC = geo.NC(b);
-  const int c0 = blockIdx.x * chunk;
+  const int c0 = blockIdx.x * CROWS;
   if (c0 >= NC) return;
-  const int c1 = min(NC, c0 + chunk);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c1 = min(NC, c0 + CROWS);
+  const int nrows = c1 - c0;
+  T* rows = reinterpret_cast<T*>(sh_dyn);
+  int* hist = reinterpret_cast<int*>(sh_dyn + 65536);
+  int* s_off = hist + kHistBins;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tid = threadIdx.x;
   const int sub = lane % LPR, rsub = lane / LPR;
+  const int64_t row0 = geo.cl_row(b, h);
+  const T* src = cent + (row0 + c0) * D;
+  constexpr int TR = RS::TILE, NT = CROWS / TR;  // 4 tiles of 16 KB, one cp.async group each
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int r0 = t * TR, nr = min(TR, nrows - r0);
+    for (int i = tid; i < nr * LPR; i += blockDim.x)
+      cp_async16(rows + (r0 * LPR + i) * EPL, src + (r0 * LPR + i) * EPL);
+    cp_async_commit();
+  }
+  const int32_t* off = offsets + geo.off_row(b, h) + c0;
+  for (int i = tid; i <= nrows; i += blockDim.x) s_off[i] = __ldg(off + i);
+  for (int i = tid; i < kHistBins; i += blockDim.x) hist[i] = 0;
   float qv[G][EPL];
   load_q<T, D, G>(q, n_q_heads, b, h, sub, scale, qv);
-  const int64_t row0 = geo.cl_row(b, h);
-  const T* cb = cent + row0 * D + sub * EPL;
-  const int32_t* off = offsets + geo.off_row(b, h);
   const int j = sub / (LPR / G);
-  for (int base = c0 + warp * RPW * UNR; base < c1; base += NW * RPW * UNR) {
-    uint4 raw[UNR];
 #pragma unroll
-    for (int i = 0; i < UNR; ++i) {
-      const int c = base + i * RPW + rsub;
-      raw[i] = c < c1 ? ld_stream(cb + (int64_t)c * D) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int i = 0; i < UNR; ++i) {
-      const int c = base + i * RPW + rsub;
+  for (int t = 0; t < NT; ++t) {
+    cp_async_wait_dyn(NT - 1 - t);  // tile t has landed; later tiles still in flight
+    __syncthreads();
+    const int r1 = min(nrows, (t + 1) * TR);
+    for (int rb = t * TR + warp * RPW; rb < r1; rb += NW * RPW) {
+      const int r = rb + rsub;
+      const bool ok = r < r1;
       float x[EPL];
-      Elem<T>::unpack(raw[i], x);
-      float acc[G];
+      if (ok) {
+        Elem<T>::unpack(*reinterpret_cast<const uint4*>(rows + r * D + sub * EPL), x);
+      } else {
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        acc[g] = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[g] = fmaf(qv[g][e], x[e], acc[g]);
+        for (int e = 0; e < EPL; ++e) x[e] = 0.f;
       }
+      float acc[G];
+      dot_g<G, EPL>(qv, x, acc);
       group_reduce_multi<G, LPR>(acc, lane);
       float m = acc[0];
 #pragma unroll
       for (int o = LPR / 2; o >= LPR / G; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (c < c1) {
-        if (sub % (LPR / G) == 0) scores[(row0 + c) * G + j] = acc[0];
+      if (ok) {
+        if (sub % (LPR / G) == 0) scores[(row0 + c0 + r) * G + j] = acc[0];
         if (sub == 0) {
-          const int cnt = off[c + 1] - off[c];
-          keys[row0 + c] = cnt > 0 ? ordered_key(m) : 0u;
+          const uint32_t key = (s_off[r + 1] - s_off[r]) > 0 ? ordered_key(m) : 0u;
+          keys[row0 + c0 + r] = key;
+          if (key) atomicAdd(&hist[key >> kHistShift], 1);
         }
       }
     }
   }
+  __syncthreads();
+  int* hg = hist_g + (int64_t)u * kHistBins;
+  for (int i = tid; i < kHistBins; i += blockDim.x)
+    if (hist[i]) atomicAdd(hg + i, hist[i]);
 }
 
-// -------------------------------------------------------------------- topk
-// One CTA per unit: drop clusters with no non-steady member, then an exact
-// 4-pass MSB radix select (8-bit digits) of the k-th largest key, then an
-// ordered compaction of the selected ids and a prefix sum of their sizes.
+// ----------------------------------------------------------------- K_B topk
+// A thread-block cluster of kTopkCluster CTAs per unit; CTA r owns the
+// contiguous cluster-id range [r*chunk, (r+1)*chunk) with its keys in shared
+// memory.  The first radix digit comes from K_A's histogram (identical in
+// every CTA; zeroed after use so the workspace is clean for the next call,
+// and rebuilt if its total disagrees with the candidate count).  The next
+// two digits merge per-CTA histograms through distributed shared memory.
+// The ordered selection and its token prefix use per-CTA counts exchanged
+// the same way.  Five cluster barriers in all.
+__device__ __forceinline__ int suffix_digit(const int* hist, int nbins, int krem, int* scan_sh,
+                                            int* bc) {
+  // thread t owns bins nbins-1-8t .. nbins-8-8t (descending)
+  const int tid = threadIdx.x;
+  int c[8], s8 = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int bin = nbins - 1 - 8 * tid - i;
+    c[i] = bin >= 0 ? hist[bin] : 0;
+    s8 += c[i];
+  }
+  int tot;
+  const int incl = block_inclusive_scan(s8, scan_sh, &tot);
+  int acc = incl - s8;
+  if (acc < krem && incl >= krem) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (acc + c[i] >= krem) { bc[0] = nbins - 1 - 8 * tid - i; bc[1] = acc; break; }
+      acc += c[i];
+    }
+  }
+  __syncthreads();
+  return bc[0];
+}
+
 __global__ void __launch_bounds__(kTopkThreads)
-wave_topk_kernel(const Geo geo, uint32_t* __restrict__ keys, const int32_t* __restrict__ offsets,
+wave_topk_kernel(const Geo geo, const uint32_t* __restrict__ keys,
+                 const int32_t* __restrict__ offsets, int32_t* __restrict__ hist_g,
                  const int32_t* __restrict__ aff_cl, const int32_t* __restrict__ aff_start, int cap,
-                 int topk_clusters, double topk_fraction, int32_t* __restrict__ sel,
-                 int32_t* __restrict__ sel_tok, int32_t* __restrict__ info) {
-  __shared__ int hist[256];
-  __shared__ int scan_sh[32];
-  __shared__ int bcast[4];
-  const int u = blockIdx.x, b = u / geo.hkv, h = u - b * geo.hkv;
+                 int topk_clusters, double topk_fraction, int n_splits, int smem_keys,
+                 int32_t* __restrict__ sel, int32_t* __restrict__ sel_slot0,
+                 int32_t* __restrict__ sel_tok, int32_t* __restrict__ split_first,
+                 int32_t* __restrict__ info, const int32_t* __restrict__ st_slot, const Pool kp,
+                 int32_t* __restrict__ gather, int64_t gather_stride, uint32_t* status) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  // shared: keys [smem_keys + 1] | offsets [smem_keys + 1] | excluded bitmask
+  //         [smem_keys/32 + 1] | affected list (cluster, steady count) [2 * cap]
+  //         | steady slots [cap]; keys and offsets later hold the gather-list chunk
+  extern __shared__ uint32_t sk[];
+  int32_t* so = reinterpret_cast<int32_t*>(sk + smem_keys + 1);
+  uint32_t* sx = reinterpret_cast<uint32_t*>(so + smem_keys + 1);
+  int32_t* sa = reinterpret_cast<int32_t*>(sx + smem_keys / 32 + 1);
+  int32_t* ss = sa + 2 * cap;
+  __shared__ int hist[kHistBins];                // digit 1 (all CTAs identical)
+  __shared__ int mh[2][kHistBins];               // merged histograms of digits 2 and 3
+  __shared__ int scan_sh[64];
+  __shared__ int bc[4];
+  __shared__ int x_cnt[4];                       // values the other CTAs read
+  __shared__ int s_wgt[32], s_weq[32], s_wgt2[32], s_weq2[32];
+  __shared__ int s_info[8];
+  pdl_launch_dependents();
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+  const int rank = (int)cluster.block_rank();
+  const int R = kTopkCluster;
+  const int u = blockIdx.x / R, b = u / geo.hkv, h = u - b * geo.hkv;
   const int NC = geo.NC(b);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int chunk = (NC + R - 1) / R;
+  const int c_lo = min(NC, rank * chunk), c_hi = min(NC, c_lo + chunk), nk = c_hi - c_lo;
+  for (int i = tid; i < 2 * kHistBins; i += nt) (&mh[0][0])[i] = 0;
+  for (int i = tid; i <= nk / 32; i += nt) sx[i] = 0u;
+  pdl_wait();
   int32_t* I = info + (int64_t)u * kInfoInts;
   const int64_t row0 = geo.cl_row(b, h);
   int32_t* pre = sel_tok + row0 + u;
-  const int k_req = topk_clusters >= 0 ? topk_clusters
-                                       : (int)ceil(topk_fraction * (double)NC);
-  if (I[6]) {  // dense unit
-    if (tid == 0) {
-      I[0] = 0; I[1] = (int32_t)0xFFFFFFFFu; I[2] = -1; I[3] = 0; I[7] = k_req;
-      pre[0] = 0;
-    }
-    return;
-  }
-  uint32_t* kk = keys + row0;
+  int32_t* split = split_first + (int64_t)u * (n_splits + 1);
+  int* hg = hist_g + (int64_t)u * kHistBins;
+  const int k_req = topk_clusters >= 0 ? topk_clusters : (int)ceil(topk_fraction * (double)NC);
+  const uint32_t* kk = keys + row0;
   const int32_t* off = offsets + geo.off_row(b, h);
-  const int n_aff = I[5];
-  for (int jj = tid; jj < n_aff; jj += blockDim.x) {
-    const int c = aff_cl[(int64_t)u * cap + jj];
-    const int dc = aff_start[(int64_t)u * (cap + 1) + jj + 1] - aff_start[(int64_t)u * (cap + 1) + jj];
-    if (c >= 0 && c < NC && off[c + 1] - off[c] - dc <= 0) kk[c] = 0u;
+  // one round of independent loads: unit record, histogram, keys, offsets, steady lists
+  if (tid < 8) s_info[tid] = I[tid];
+  for (int i = tid; i < kHistBins; i += nt) hist[i] = hg[i];
+  for (int i = tid; i < nk; i += nt) sk[i] = kk[c_lo + i];
+  for (int i = tid; i <= nk; i += nt) so[i] = off[c_lo + i];
+  for (int i = tid; i < cap; i += nt) {  // unconditional: no wait on the unit record
+    sa[2 * i] = aff_cl[(int64_t)u * cap + i];
+    sa[2 * i + 1] = aff_start[(int64_t)u * (cap + 1) + i + 1] - aff_start[(int64_t)u * (cap + 1) + i];
+    ss[i] = st_slot[(int64_t)u * cap + i];
   }
   __syncthreads();
-
-  uint32_t prefix = 0, pmask = 0;
-  int krem = 0, ncand = 0, ksel = 0;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    int mine = 0;
-    for (int c = tid; c < NC; c += blockDim.x) {
-      const uint32_t key = kk[c];
-      if (key == 0u) continue;
-      ++mine;
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+  const int n_st = s_info[4];
+  const int dense = s_info[6];
+  const int n_aff = dense ? 0 : min(cap, s_info[5]);
+  const int Tb = geo.T(b);
+  int32_t* gat = gather + (int64_t)u * gather_stride;
+  // pool row index of slot s of this unit (-1 if the block table is out of range)
+  auto row_of = [&](int slot) -> int32_t {
+    const int64_t ro = pool_row(kp, geo.hkv, 1, b, h, slot, status);
+    return ro < 0 ? -1 : (int32_t)ro;
+  };
+  // clusters of this CTA's range left without a non-steady member are not candidates
+  for (int jj = tid; jj < n_aff; jj += nt) {
+    const int c = sa[2 * jj];
+    if (c >= c_lo && c < c_hi && so[c - c_lo + 1] - so[c - c_lo] - sa[2 * jj + 1] <= 0)
+      atomicOr(&sx[(c - c_lo) >> 5], 1u << ((c - c_lo) & 31));
+  }
+  __syncthreads();
+  auto key_of = [&](int i) -> uint32_t {  // local index; 0 if not a candidate
+    return ((sx[i >> 5] >> (i & 31)) & 1u) ? 0u : sk[i];
+  };
+  int mine = 0;
+  for (int i = tid; i < nk; i += nt) mine += key_of(i) != 0u;
+  int nc_local;
+  block_inclusive_scan(mine, scan_sh, &nc_local);
+  if (tid == 0) x_cnt[0] = nc_local;
+  cluster.sync();                                            // barrier 1
+  if (rank == 0)
+    for (int i = tid; i < kHistBins; i += nt) hg[i] = 0;    // every CTA has its copy
+  int ncand = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) ncand += *cluster.map_shared_rank(&x_cnt[0], r);
+  if (dense) {  // the attend CTAs take all slots in order
+    for (int t = rank * nt + tid; t < Tb; t += R * nt) gat[t] = row_of(t);
+    if (rank == 0) {
+      if (tid == 0) {
+        I[0] = 0; I[1] = (int32_t)0xFFFFFFFFu; I[2] = -1; I[3] = 0; I[7] = k_req;
+        pre[0] = 0;
+      }
+      for (int j = tid; j <= n_splits; j += nt) split[j] = 0;
     }
-    if (pass == 0) {
-      int tot;
-      block_inclusive_scan(mine, scan_sh, &tot);
-      ncand = tot;
-      ksel = min(max(k_req, 0), ncand);
-      krem = ksel;
-      if (ksel == 0 || ksel == ncand) break;
-    } else {
+    cluster.sync();
+    return;
+  }
+  // remove the excluded clusters (any range) from this CTA's digit-1 histogram
+  for (int jj = tid; jj < n_aff; jj += nt) {
+    const int c = sa[2 * jj];
+    if (c < 0 || c >= NC) continue;
+    const int r = min(R - 1, c / max(chunk, 1));
+    const int li = c - r * chunk;
+    const int32_t* ro = cluster.map_shared_rank(so, r);
+    if (ro[li + 1] - ro[li] - sa[2 * jj + 1] <= 0) {
+      const uint32_t key = *cluster.map_shared_rank(sk + li, r);
+      if (key) atomicSub(&hist[key >> kHistShift], 1);
+    }
+  }
+  __syncthreads();
+  {  // a stale digit-1 histogram (workspace reused after a failed call) is rebuilt
+    int hs = 0;
+    for (int i = tid; i < kHistBins; i += nt) hs += hist[i];
+    int tot;
+    block_inclusive_scan(hs, scan_sh, &tot);
+    if (tot != ncand) {
+      if (tid == 0 && rank == 0) flag_error(status, WI_DEV_BAD_HIST);
+      for (int i = tid; i < kHistBins; i += nt) hist[i] = 0;
+      __syncthreads();
+      for (int r = 0; r < R; ++r) {
+        const int lo = min(NC, r * chunk), n = min(NC, lo + chunk) - lo;
+        const uint32_t* rk = cluster.map_shared_rank(sk, r);
+        const uint32_t* rx = cluster.map_shared_rank(sx, r);
+        for (int i = tid; i < n; i += nt) {
+          const uint32_t key = ((rx[i >> 5] >> (i & 31)) & 1u) ? 0u : rk[i];
+          if (key) atomicAdd(&hist[key >> kHistShift], 1);
+        }
+      }
       __syncthreads();
     }
-    if (warp == 0) {
-      int cnt[8], sum = 0;
+  }
+  const int ksel = min(max(k_req, 0), ncand);
+  int krem = ksel;
+  uint32_t prefix = 0, pmask = 0;
+  const bool radix = ksel > 0 && ksel < ncand;
+  if (radix) {
+    const int d = suffix_digit(hist, kHistBins, krem, scan_sh, bc);
+    krem -= bc[1];
+    prefix = (uint32_t)d << 21;
+    pmask = 0x7FFu << 21;
+  }
+#pragma unroll 1
+  for (int pass = 1; pass < 3; ++pass) {       // barriers 2 and 3 (taken by every CTA)
+    const int bits = pass == 2 ? 10 : 11;
+    const int shift = pass == 1 ? 10 : 0;
+    const int nbins = 1 << bits;
+    int* loc = hist;                             // digit-1 histogram no longer needed
+    if (radix) {
+      for (int i = tid; i < nbins; i += nt) loc[i] = 0;
+      __syncthreads();
+      for (int i = tid; i < nk; i += nt) {
+        const uint32_t key = key_of(i);
+        if (key != 0u && (key & pmask) == prefix) atomicAdd(&loc[(key >> shift) & (nbins - 1)], 1);
+      }
+      __syncthreads();
+      for (int i = tid; i < nbins; i += nt) {
+        const int v = loc[i];
+        if (v)
 #pragma unroll
-      for (int t = 0; t < 8; ++t) { cnt[t] = hist[255 - 8 * lane - t]; sum += cnt[t]; }
-      int incl = sum;
+          for (int r = 0; r < R; ++r) atomicAdd(cluster.map_shared_rank(&mh[pass - 1][i], r), v);
+      }
+    }
+    cluster.sync();
+    if (radix) {
+      const int d = suffix_digit(mh[pass - 1], nbins, krem, scan_sh, bc);
+      krem -= bc[1];
+      prefix |= (uint32_t)d << shift;
+      pmask |= (uint32_t)(nbins - 1) << shift;
+    }
+  }
+  uint32_t kstar;
+  int eq_take;  // how many keys equal to kstar are selected (lowest ids first)
+  if (ksel == 0) { kstar = 0xFFFFFFFFu; eq_take = 0; }
+  else if (ksel == ncand) { kstar = 1u; eq_take = INT_MAX; }
+  else { kstar = prefix; eq_take = krem; }
+
+  // ordered selection: warp w of this CTA owns [wb, we) of its range
+  const unsigned lt = (1u << lane) - 1u;
+  const int B = (((nk + nw - 1) / nw) + 31) & ~31;
+  const int wb = min(nk, warp * B), we = min(nk, wb + B);
+  int gt_w = 0, eq_w = 0, tk_w = 0;
+  for (int base = wb; base < we; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < we ? key_of(i) : 0u;
+    gt_w += __popc(__ballot_sync(0xffffffffu, key != 0u && key > kstar));
+    eq_w += __popc(__ballot_sync(0xffffffffu, key != 0u && key == kstar));
+  }
+  if (lane == 0) { s_wgt[warp] = gt_w; s_weq[warp] = eq_w; s_wgt2[warp] = gt_w; s_weq2[warp] = eq_w; }
+  __syncthreads();
+  if (tid == 0) {
+    int g = 0, q = 0;
+    for (int w = 0; w < nw; ++w) { g += s_wgt[w]; q += s_weq[w]; }
+    x_cnt[1] = g; x_cnt[2] = q;
+  }
+  cluster.sync();                                            // barrier 4
+  int eq_before = 0, sel_before = 0;
+  for (int r = 0; r < rank; ++r) {
+    const int g = *cluster.map_shared_rank(&x_cnt[1], r);
+    const int q = *cluster.map_shared_rank(&x_cnt[2], r);
+    sel_before += g + min(max(eq_take - eq_before, 0), q);
+    eq_before += q;
+  }
+  const int cta_first = sel_before;
+  const int eq_cta0 = eq_before;  // equal keys before this CTA
+  for (int w = 0; w < warp; ++w) {
+    sel_before += s_wgt[w] + min(max(eq_take - eq_before, 0), s_weq[w]);
+    eq_before += s_weq[w];
+  }
+  // first walk: token count of this warp's selection (offsets are in shared memory)
+  {
+    int run_eq = eq_before;
+    for (int base = wb; base < we; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = i < we ? key_of(i) : 0u;
+      const bool isgt = key != 0u && key > kstar;
+      const bool iseq = key != 0u && key == kstar;
+      const unsigned beq = __ballot_sync(0xffffffffu, iseq);
+      const bool take = isgt || (iseq && run_eq + __popc(beq & lt) < eq_take);
+      tk_w += take ? so[i + 1] - so[i] : 0;
+      run_eq += __popc(beq);
+    }
+    tk_w = warp_sum_int(tk_w);
+  }
+  __syncthreads();
+  if (lane == 0) s_wgt[warp] = tk_w;
+  __syncthreads();
+  if (tid == 0) {
+    int t = 0;
+    for (int w = 0; w < nw; ++w) t += s_wgt[w];
+    x_cnt[3] = t;
+  }
+  cluster.sync();                                            // barrier 5
+  int tok_before = 0, total_tok = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int t = *cluster.map_shared_rank(&x_cnt[3], r);
+    if (r < rank) tok_before += t;
+    total_tok += t;
+  }
+  const int tok_cta_end = tok_before + x_cnt[3];
+  for (int w = 0; w < warp; ++w) tok_before += s_wgt[w];
+  const int n_tok = total_tok + n_st;
+  const int split_len = (n_tok + n_splits - 1) / n_splits;
+  // second walk: write the selection, its slot starts, token prefix and split starts
+  {
+    int run_eq = eq_before, pos = sel_before, tok = tok_before;
+    for (int base = wb; base < we; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = i < we ? key_of(i) : 0u;
+      const bool isgt = key != 0u && key > kstar;
+      const bool iseq = key != 0u && key == kstar;
+      const unsigned beq = __ballot_sync(0xffffffffu, iseq);
+      const int eqrank = run_eq + __popc(beq & lt);
+      const bool take = isgt || (iseq && eqrank < eq_take);
+      if (iseq && eqrank == eq_take - 1) I[2] = c_lo + i;   // last selected key equal to kstar
+      const unsigned bs = __ballot_sync(0xffffffffu, take);
+      const int n = take ? so[i + 1] - so[i] : 0;
+      int incl = n;  // inclusive warp scan of token counts
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      const unsigned bal = __ballot_sync(0xffffffffu, incl >= krem);
-      const int first = __ffs(bal) - 1;
-      if (lane == first) {
-        int acc = incl - sum;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          if (acc + cnt[t] >= krem) { bcast[0] = 255 - 8 * lane - t; bcast[1] = acc; break; }
-          acc += cnt[t];
+      if (take) {
+        const int si = pos + __popc(bs & lt), st = tok + incl - n;
+        sel[row0 + si] = c_lo + i;
+        sel_slot0[row0 + si] = so[i];
+        pre[si] = st;
+        if (split_len > 0)  // splits whose first token falls inside this cluster start at it
+          for (int j = (st + split_len - 1) / split_len; j * split_len < st + n && j < n_splits; ++j)
+            split[j] = si;
+      }
+      pos += __popc(bs);
+      tok += __shfl_sync(0xffffffffu, incl, 31);
+      run_eq += __popc(beq);
+    }
+  }
+  // gather list of this CTA's selection: tokens expanded CTA-wide from a
+  // shared-memory copy of (token start, slot start) of its selected clusters
+  __syncthreads();
+  {
+    int32_t* lst = reinterpret_cast<int32_t*>(sk);       // keys are no longer read
+    int32_t* lso = so;                                   // nor are the offsets
+    const int cap_list = smem_keys;                      // entries per chunk (+1 end mark)
+    const int my_first = cta_first;
+    int my_sel = 0;
+    {  // clusters this CTA selected = end of its last warp's run - cta_first
+      int g = 0, q = 0;
+      for (int w = 0; w < nw; ++w) { g += s_wgt2[w]; q += s_weq2[w]; }
+      my_sel = g + min(max(eq_take - eq_cta0, 0), q);
+    }
+    for (int j0 = 0; j0 < my_sel; j0 += cap_list) {
+      const int nj = min(cap_list, my_sel - j0);
+      __syncthreads();
+      for (int k = tid; k <= nj; k += nt) {
+        const int si = my_first + j0 + k;
+        lst[k] = (k < nj) ? pre[si] : ((j0 + nj < my_sel) ? pre[si] : tok_cta_end);
+        if (k < nj) lso[k] = sel_slot0[row0 + si];
+      }
+      __syncthreads();
+      const int q0 = lst[0], q1 = lst[nj];
+      for (int qq = q0 + tid; qq < q1; qq += nt) {
+        int lo = 0, hi = nj - 1;  // largest k with lst[k] <= qq
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (lst[mid] <= qq) lo = mid; else hi = mid - 1;
         }
+        const int slot = lso[lo] + (qq - lst[lo]);
+        gat[qq] = find_sorted(ss, n_st, slot) >= 0 ? -1 : row_of(slot);
       }
     }
-    __syncthreads();
-    krem -= bcast[1];
-    prefix |= (uint32_t)bcast[0] << shift;
-    pmask |= 255u << shift;
-    __syncthreads();
   }
-
-  uint32_t kstar;
-  int thr;
-  if (ksel == 0) {
-    kstar = 0xFFFFFFFFu; thr = -1;
-  } else if (ksel == ncand) {
-    kstar = 1u; thr = NC;
-  } else {
-    kstar = prefix;
-    // index of the krem-th key equal to kstar, in ascending cluster id
-    int running = 0;
-    if (tid == 0) bcast[2] = -1;
-    __syncthreads();
-    for (int base = 0; base < NC; base += blockDim.x) {
-      const int c = base + tid;
-      const int f = (c < NC && kk[c] == kstar) ? 1 : 0;
-      int tot;
-      const int incl = block_inclusive_scan(f, scan_sh, &tot);
-      if (f && running + incl == krem) bcast[2] = c;
-      running += tot;
-      __syncthreads();
-      if (bcast[2] >= 0) break;
-    }
-    thr = bcast[2];
+  for (int j = rank * nt + tid; j < n_st; j += R * nt) gat[total_tok + j] = row_of(ss[j]);
+  if (rank == 0 && tid == 0) {
+    (void)cta_first;
+    pre[ksel] = total_tok;
+    const int j0 = split_len > 0 ? (total_tok + split_len - 1) / split_len : 0;
+    for (int j = j0; j <= n_splits; ++j) split[j] = ksel;
+    if (ksel == 0) I[2] = -1;
+    else if (ksel == ncand) I[2] = NC;
+    I[0] = ksel; I[1] = (int32_t)kstar; I[3] = total_tok; I[7] = k_req;
   }
-  // ordered compaction of the selection
-  int running = 0;
-  for (int base = 0; base < NC; base += blockDim.x) {
-    const int c = base + tid;
-    int f = 0;
-    if (c < NC) {
-      const uint32_t key = kk[c];
-      f = key != 0u && (key > kstar || (key == kstar && c <= thr));
-    }
-    int tot;
-    const int incl = block_inclusive_scan(f, scan_sh, &tot);
-    if (f) sel[row0 + running + incl - 1] = c;
-    running += tot;
-  }
-  __syncthreads();
-  // token prefix over the selected clusters (all slots, steady ones included)
-  int tok = 0;
-  for (int base = 0; base < ksel; base += blockDim.x) {
-    const int i = base + tid;
-    int cnt = 0;
-    if (i < ksel) {
-      const int c = sel[row0 + i];
-      cnt = (c >= 0 && c < NC) ? off[c + 1] - off[c] : 0;
-    }
-    int tot;
-    const int incl = block_inclusive_scan(cnt, scan_sh, &tot);
-    if (i < ksel) pre[i + 1] = tok + incl;
-    tok += tot;
-  }
-  if (tid == 0) {
-    pre[0] = 0;
-    I[0] = ksel; I[1] = (int32_t)kstar; I[2] = thr; I[3] = tok; I[7] = k_req;
-  }
+  cluster.sync();  // keep every CTA's shared memory alive until all remote reads are done
 }
 
-// ------------------------------------------------------------------ attend
-// Split-K exact attention over the retrieved clusters' non-steady rows
-// followed by the steady rows.  CTA (split, unit) takes an equal share of
-// the unit's token list; the list is resolved tile by tile through the
-// prefix sums of the selected cluster sizes.
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kStreamThreads)
-wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const Pool kp,
-                   const Pool vp, const int32_t* __restrict__ perm,
-                   const int32_t* __restrict__ offsets, const int32_t* __restrict__ sel,
-                   const int32_t* __restrict__ sel_tok, const int32_t* __restrict__ st_slot,
-                   const int32_t* __restrict__ info, int n_sink, int window, int cap,
-                   int n_splits, int n_parts, float* __restrict__ partials, float scale,
-                   uint32_t* status) {
-  using RS = RowShape<T, D>;
-  constexpr int EPL = RS::EPL, LPR = RS::LPR, RPW = RS::RPW;
+// -------------------------------------------------- K_C attend + estimate
+struct AttendArgs {
+  const int32_t *gather, *aff_cl, *aff_start;
+  const float* dv;
+  int64_t gather_stride;
+  const int32_t* info;
+  const float* scores;
+  const uint32_t* keys;
+  int n_sink, window, cap, n_splits, n_est, echunk, n_parts, wcap;
+  float* partials;
+  int32_t* counters;
+  float* out;
+  float* lse;
+  float scale;
+};
+
+// A softmax part of one (unit, q head): {m, l, -, -, o[D]}; o starts 16-byte aligned.
+template <int D>
+struct Part {
+  static constexpr int kStride = D + 4;
+  static constexpr int kO = 4;
+};
+
+template <int G, int EPL, int LPR, int D>
+__device__ __forceinline__ void reduce_and_store(float (&acc)[G][EPL], float* s_red, int warp,
+                                                 int sub, int rsub, float* part) {
   constexpr int NW = kStreamThreads / 32;
-  constexpr int TILE = kAttendTile;
-  static_assert(TILE % (NW * RPW) == 0, "tile must be a multiple of rows per CTA step");
-  __shared__ int64_t s_row[TILE];
-  __shared__ float s_sc[TILE][G];
-  __shared__ int s_pre[TILE + 2];
-  __shared__ int s_coff[TILE + 1];
-  __shared__ int s_cursor;
-  __shared__ float s_red[NW][G][D];
-
-  const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
-  const int Tb = geo.T(b), NC = geo.NC(b);
-  const int ns = min(n_sink, Tb);
-  const int wstart = max(Tb - window, ns);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tid = threadIdx.x;
-  const int sub = lane % LPR, rsub = lane / LPR;
-  const int32_t* I = info + (int64_t)u * kInfoInts;
-  const int dense = I[6];
-  const int ksel = dense ? 0 : I[0];
-  const int nsel_tok = dense ? 0 : I[3];
-  const int n_st = I[4];
-  const int n_tok = nsel_tok + n_st;
-  const int per = (n_tok + n_splits - 1) / n_splits;
-  const int t0 = blockIdx.x * per;
-  const int t1 = min(n_tok, t0 + per);
-
-  float qv[G][EPL];
-  load_q<T, D, G>(q, n_q_heads, b, h, sub, scale, qv);
-  const int64_t row0 = geo.cl_row(b, h);
-  const int32_t* pre = sel_tok + row0 + u;
-  const int32_t* selu = sel + row0;
-  const int32_t* off = offsets + geo.off_row(b, h);
-  const int32_t* permu = perm + geo.tok_row(b, h);
-  const T* kbase = reinterpret_cast<const T*>(kp.base) + sub * EPL;
-  const T* vbase = reinterpret_cast<const T*>(vp.base) + sub * EPL;
-  const int jh = sub / (LPR / G);
-
-  float m_run[G], l_run[G], acc[G][EPL];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m_run[g] = -INFINITY; l_run[g] = 0.f;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[g][e] = 0.f;
-  }
-
-  if (tid == 0) {
-    int cur = ksel;
-    if (t0 < nsel_tok) {  // largest i < ksel with pre[i] <= t0
-      int lo = 0, hi = ksel - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (pre[mid] <= t0) lo = mid; else hi = mid - 1;
-      }
-      cur = lo;
-    }
-    s_cursor = cur;
-  }
-  __syncthreads();
-
-  for (int tb = t0; tb < t1; tb += TILE) {
-    const int n = min(TILE, t1 - tb);
-    const int cur = s_cursor;
-    if (tb < nsel_tok) {
-      for (int i = tid; i < TILE + 2; i += blockDim.x) {
-        const int idx = cur + i;
-        s_pre[i] = idx <= ksel ? pre[idx] : INT_MAX;
-      }
-      for (int i = tid; i < TILE + 1; i += blockDim.x) {
-        const int idx = cur + i;
-        int o = 0;
-        if (idx < ksel) {
-          const int c = selu[idx];
-          if (c >= 0 && c < NC) o = off[c]; else flag_error(status, WI_DEV_BAD_CLUSTER);
-        }
-        s_coff[i] = o;
-      }
-    }
-    __syncthreads();
-    if (tid < TILE) {
-      int64_t rowoff = -1;
-      if (tid < n) {
-        const int tok = tb + tid;
-        int slot;
-        bool valid = true;
-        if (tok < nsel_tok) {
-          int lo = 0, hi = TILE;  // largest i with s_pre[i] <= tok
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (s_pre[mid] <= tok) lo = mid; else hi = mid - 1;
-          }
-          slot = s_coff[lo] + (tok - s_pre[lo]);
-          if (slot < 0 || slot >= Tb) {
-            flag_error(status, WI_DEV_BAD_SLOT);
-            valid = false;
-          } else {
-            const int pos = permu[slot];
-            valid = !(pos < ns || pos >= wstart);
-          }
-          if (tid == n - 1) s_cursor = cur + lo;
-        } else {
-          const int js = tok - nsel_tok;
-          slot = dense ? js : st_slot[(int64_t)u * cap + js];
-        }
-        if (valid) rowoff = pool_row(kp, geo.hkv, D, b, h, slot, status);
-      }
-      s_row[tid] = rowoff;
-    }
-    __syncthreads();
-    // scores of the tile
-#pragma unroll
-    for (int rb = warp * RPW; rb < TILE; rb += NW * RPW) {
-      const int r = rb + rsub;
-      const int64_t ro = s_row[r];
-      const uint4 raw = ro >= 0 ? ld_stream(kbase + ro) : make_uint4(0, 0, 0, 0);
-      float x[EPL];
-      Elem<T>::unpack(raw, x);
-      float a[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        a[g] = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) a[g] = fmaf(qv[g][e], x[e], a[g]);
-      }
-      group_reduce_multi<G, LPR>(a, lane);
-      if (sub % (LPR / G) == 0) s_sc[r][jh] = ro >= 0 ? a[0] : -INFINITY;
-    }
-    __syncthreads();
-    // running max / sum update (identical in every warp)
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float mt = -INFINITY;
-      for (int r = lane; r < TILE; r += 32) mt = fmaxf(mt, s_sc[r][g]);
-      mt = warp_max(mt);
-      const float mnew = fmaxf(m_run[g], mt);
-      const float corr = mnew == -INFINITY ? 1.f : __expf(m_run[g] - mnew);
-      float ps = 0.f;
-      for (int r = lane; r < TILE; r += 32) {
-        const float sv = s_sc[r][g];
-        ps += sv == -INFINITY ? 0.f : __expf(sv - mnew);
-      }
-      ps = warp_sum(ps);
-      l_run[g] = l_run[g] * corr + ps;
-      m_run[g] = mnew;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) acc[g][e] *= corr;
-    }
-    // weighted value sum
-#pragma unroll
-    for (int rb = warp * RPW; rb < TILE; rb += NW * RPW) {
-      const int r = rb + rsub;
-      const int64_t ro = s_row[r];
-      const uint4 raw = ro >= 0 ? ld_stream(vbase + ro) : make_uint4(0, 0, 0, 0);
-      float x[EPL];
-      Elem<T>::unpack(raw, x);
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float sv = s_sc[r][g];
-        const float p = sv == -INFINITY ? 0.f : __expf(sv - m_run[g]);
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[g][e] = fmaf(p, x[e], acc[g][e]);
-      }
-    }
-    __syncthreads();
-  }
-  // reduce the value accumulators over row groups and warps
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
@@ -537,265 +683,415 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
 #pragma unroll
     for (int g = 0; g < G; ++g)
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) s_red[warp][g][sub * EPL + e] = acc[g][e];
+      for (int e = 0; e < EPL; ++e) s_red[(warp * G + g) * D + sub * EPL + e] = acc[g][e];
   }
   __syncthreads();
-  float* part = partials + ((int64_t)u * n_parts + blockIdx.x) * G * (D + 2);
-  for (int i = tid; i < G * D; i += blockDim.x) {
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
     const int g = i / D, e = i - g * D;
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) v += s_red[w][g][e];
-    part[g * (D + 2) + 2 + e] = v;
-  }
-  if (tid == 0) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) { part[g * (D + 2)] = m_run[g]; part[g * (D + 2) + 1] = l_run[g]; }
+    for (int w = 0; w < NW; ++w) v += s_red[(w * G + g) * D + e];
+    part[g * Part<D>::kStride + Part<D>::kO + e] = v;
   }
 }
 
-// ---------------------------------------------------------------- estimate
-// CTA (chunk, unit) estimates the candidate clusters of its chunk that were
-// not retrieved: weights w = e^(s - m) from the stored scores, denominator
-// sum cnt' * w, numerator sum w * Vsum, then minus w * v for each steady
-// member of an affected cluster (Vsum' = Vsum - sum of steady values).
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kStreamThreads)
-wave_estimate_kernel(const Geo geo, const T* __restrict__ vsum, const int32_t* __restrict__ offsets,
-                     const float* __restrict__ scores, const uint32_t* __restrict__ keys,
-                     const int32_t* __restrict__ info, const int32_t* __restrict__ aff_cl,
-                     const int32_t* __restrict__ aff_start, const int32_t* __restrict__ st_slot,
-                     const int32_t* __restrict__ st_cl, const Pool vp, int cap, int echunk,
-                     int n_splits, int n_parts, float* __restrict__ partials, uint32_t* status) {
+wave_attend_estimate_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const Pool kp,
+                            const Pool vp, const T* __restrict__ vsum,
+                            const int32_t* __restrict__ offsets, const AttendArgs A,
+                            uint32_t* status) {
   using RS = RowShape<T, D>;
-  constexpr int EPL = RS::EPL, LPR = RS::LPR, RPW = RS::RPW, UNR = 4;
+  constexpr int EPL = RS::EPL, LPR = RS::LPR, RPW = RS::RPW, TR = RS::TILE;
   constexpr int NW = kStreamThreads / 32;
-  extern __shared__ float sh_est[];
-  float* s_w = sh_est;                                   // [echunk][G]
-  int* s_cnt = reinterpret_cast<int*>(sh_est + echunk * G);  // [echunk]
-  __shared__ float s_red[NW][G][D];
-  __shared__ float s_part[NW][G];
-  __shared__ float s_m[G], s_l[G];
-  __shared__ int s_arange[2];
+  constexpr int NST = 4;                    // estimate ring stages (TR rows each)
+  static_assert(TR % (NW * RPW) == 0, "tile must be a multiple of rows per CTA step");
+  extern __shared__ __align__(16) unsigned char sh[];
+  // shared layout: [ring: 4 tiles of TR rows (attend: K x2, V x2); the final
+  //                 cross-warp reduction reuses it] [s_w wcap*G f32]
+  //                [s_cnt echunk i32] [steady / affected lists 2*cap+2 i32]
+  T* ring = reinterpret_cast<T*>(sh);
+  float* s_red = reinterpret_cast<float*>(sh);
+  float* s_w = reinterpret_cast<float*>(sh + NST * TR * RS::ROWB);
+  int* s_cnt = reinterpret_cast<int*>(s_w + A.wcap * G);
+  int32_t* s_list = s_cnt + A.echunk;
+  __shared__ int64_t s_row[2][TR];
+  __shared__ float s_sc[TR][G];
+  __shared__ int s_last;
+  __shared__ float s_m[G], s_l[G], s_part[NW][G];
+  __shared__ int s_info[kInfoInts];
 
   const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
-  const int NC = geo.NC(b);
+  const int Tb = geo.T(b), NC = geo.NC(b);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tid = threadIdx.x;
   const int sub = lane % LPR, rsub = lane / LPR;
-  const int32_t* I = info + (int64_t)u * kInfoInts;
-  const int c0 = blockIdx.x * echunk;
-  const int c1 = min(NC, c0 + echunk);
-  float* part = partials + ((int64_t)u * n_parts + n_splits + blockIdx.x) * G * (D + 2);
-  if (I[6] || c0 >= NC) {
-    for (int i = tid; i < G * (D + 2); i += blockDim.x) {
-      const int e = i % (D + 2);
-      part[i] = e == 0 ? -INFINITY : 0.f;
-    }
-    return;
-  }
-  const uint32_t kstar = (uint32_t)I[1];
-  const int thr = I[2];
-  const int n_aff = I[5];
+  const int jh = sub / (LPR / G);
   const int64_t row0 = geo.cl_row(b, h);
   const int32_t* off = offsets + geo.off_row(b, h);
-  const int32_t* acl = aff_cl + (int64_t)u * cap;
-  const int32_t* ast = aff_start + (int64_t)u * (cap + 1);
-  if (tid < 2) {  // affected clusters inside [c0, c1): lower_bound of c0 and c1
-    const int key = tid == 0 ? c0 : c1;
-    int lo = 0, hi = n_aff;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (acl[mid] < key) lo = mid + 1; else hi = mid;
-    }
-    s_arange[tid] = lo;
-  }
-  __syncthreads();
-  const int a0 = s_arange[0], a1 = s_arange[1];
+  const bool role_est = (int)blockIdx.x >= A.n_splits;
+  constexpr int PS = Part<D>::kStride;
+  float* part = A.partials + ((int64_t)u * A.n_parts + blockIdx.x) * G * PS;
 
-  // phase 1: contribution mask, reduced counts, scores
-  float mloc[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) mloc[g] = -INFINITY;
-  for (int i = tid; i < c1 - c0; i += blockDim.x) {
-    const int c = c0 + i;
-    const uint32_t key = keys[row0 + c];
-    const bool picked = key > kstar || (key == kstar && c <= thr);
-    int cntp = off[c + 1] - off[c];
-    bool contrib = key != 0u && !picked;
-    if (contrib && a1 > a0) {
-      int lo = a0, hi = a1;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (acl[mid] < c) lo = mid + 1; else hi = mid;
-      }
-      if (lo < a1 && acl[lo] == c) cntp -= ast[lo + 1] - ast[lo];
-    }
-    contrib = contrib && cntp > 0;
-    s_cnt[i] = contrib ? cntp : 0;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float sv = contrib ? scores[(row0 + c) * G + g] : -INFINITY;
-      s_w[i * G + g] = sv;
-      mloc[g] = fmaxf(mloc[g], sv);
-    }
-  }
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float v = warp_max(mloc[g]);
-    if (lane == 0) s_part[warp][g] = v;
-  }
-  __syncthreads();
-  if (tid < G) {
-    float v = -INFINITY;
-    for (int w = 0; w < NW; ++w) v = fmaxf(v, s_part[w][tid]);
-    s_m[tid] = v;
-  }
-  __syncthreads();
-  // phase 2: weights and denominator
-  float lloc[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) lloc[g] = 0.f;
-  for (int i = tid; i < c1 - c0; i += blockDim.x) {
-    const int cnt = s_cnt[i];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float w = cnt > 0 ? __expf(s_w[i * G + g] - s_m[g]) : 0.f;
-      s_w[i * G + g] = w;
-      lloc[g] += (float)cnt * w;
-    }
-  }
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float v = warp_sum(lloc[g]);
-    if (lane == 0) s_part[warp][g] = v;
-  }
-  __syncthreads();
-  if (tid < G) {
-    float v = 0.f;
-    for (int w = 0; w < NW; ++w) v += s_part[w][tid];
-    s_l[tid] = v;
-  }
-  // phase 3: numerator over the value sums
   float acc[G][EPL];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int e = 0; e < EPL; ++e) acc[g][e] = 0.f;
-  const T* vb = vsum + row0 * D + sub * EPL;
-  for (int base = c0 + warp * RPW * UNR; base < c1; base += NW * RPW * UNR) {
-    uint4 raw[UNR];
+
+  if (role_est) {
+    // ------------------------------------------------------------ estimate
+    const int c0 = (blockIdx.x - A.n_splits) * A.echunk;
+    const int c1 = min(NC, c0 + A.echunk);
+    const int ntile = c0 < c1 ? (c1 - c0 + TR - 1) / TR : 0;
+    const T* vrow = vsum + row0 * D;
+    auto issue = [&](int t) {
+      if (t < ntile) {
+        T* dst = ring + (size_t)(t % NST) * TR * D;
+        const int r0 = c0 + t * TR, nr = min(TR, c1 - r0);
+        for (int i = tid; i < nr * LPR; i += blockDim.x) {
+          const int r = i / LPR, ch = i - r * LPR;
+          cp_async16(dst + r * D + ch * EPL, vrow + (int64_t)(r0 + r) * D + ch * EPL);
+        }
+      }
+      cp_async_commit();
+    };
 #pragma unroll
-    for (int i = 0; i < UNR; ++i) {
-      const int c = base + i * RPW + rsub;
-      raw[i] = (c < c1 && s_cnt[c - c0] > 0) ? ld_stream(vb + (int64_t)c * D)
-                                             : make_uint4(0, 0, 0, 0);
+    for (int t = 0; t < NST; ++t) issue(t);  // value sums do not depend on the selection
+    pdl_wait();
+    // one round of independent loads: unit record, affected list, and the
+    // chunk's keys, offsets and scores (kept in registers across the barrier)
+    constexpr int EPT = 2;                       // clusters per thread (echunk <= 512)
+    const int32_t* I = A.info + (int64_t)u * kInfoInts;
+    if (tid < kInfoInts) s_info[tid] = I[tid];
+    int32_t* s_acl = s_list;
+    int32_t* s_ast = s_list + A.cap;
+    for (int i = tid; i < A.cap; i += blockDim.x) {
+      s_acl[i] = A.aff_cl[(int64_t)u * A.cap + i];
+      s_ast[i] = A.aff_start[(int64_t)u * (A.cap + 1) + i];
     }
+    if (tid == 0) s_ast[A.cap] = A.aff_start[(int64_t)u * (A.cap + 1) + A.cap];
+    uint32_t kv[EPT];
+    int cv[EPT];
+    float sv[EPT][G];
 #pragma unroll
-    for (int i = 0; i < UNR; ++i) {
-      const int c = base + i * RPW + rsub;
-      if (c < c1 && s_cnt[c - c0] > 0) {
-        float x[EPL];
-        Elem<T>::unpack(raw[i], x);
+    for (int k = 0; k < EPT; ++k) {
+      const int c = c0 + tid + k * kStreamThreads;
+      kv[k] = 0u; cv[k] = 0;
+      if (c < c1) {
+        kv[k] = A.keys[row0 + c];
+        cv[k] = __ldg(off + c + 1) - __ldg(off + c);
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) sv[k][g] = c < c1 ? A.scores[(row0 + c) * G + g] : -INFINITY;
+    }
+    __syncthreads();
+    const bool skip = s_info[6] || c0 >= c1;
+    const int n_aff = s_info[6] ? 0 : min(A.cap, s_info[5]);
+    if (!skip) {
+      const uint32_t kstar = (uint32_t)s_info[1];
+      const int thr = s_info[2];
+      float m_loc[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) m_loc[g] = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < EPT; ++k) {
+        const int i = tid + k * kStreamThreads;
+        if (i >= c1 - c0) continue;
+        const int c = c0 + i;
+        const uint32_t key = kv[k];
+        const bool picked = key > kstar || (key == kstar && c <= thr);
+        int cntp = cv[k];
+        bool contrib = key != 0u && !picked;
+        if (contrib && n_aff > 0) {
+          const int f = find_sorted(s_acl, n_aff, c);
+          if (f >= 0) cntp -= s_ast[f + 1] - s_ast[f];
+        }
+        contrib = contrib && cntp > 0;
+        s_cnt[i] = contrib ? cntp : 0;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const float w = s_w[(c - c0) * G + g];
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) acc[g][e] = fmaf(w, x[e], acc[g][e]);
+          const float v = contrib ? sv[k][g] : -INFINITY;
+          s_w[i * G + g] = v;
+          m_loc[g] = fmaxf(m_loc[g], v);
         }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float v = warp_max(m_loc[g]);
+        if (lane == 0) s_part[warp][g] = v;
+      }
+      __syncthreads();
+      if (tid < G) {
+        float v = -INFINITY;
+        for (int w = 0; w < NW; ++w) v = fmaxf(v, s_part[w][tid]);
+        s_m[tid] = v;
+      }
+      __syncthreads();
+      float l_loc[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) l_loc[g] = 0.f;
+      for (int i = tid; i < c1 - c0; i += blockDim.x) {
+        const int cnt = s_cnt[i];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float w = cnt > 0 ? __expf(s_w[i * G + g] - s_m[g]) : 0.f;
+          s_w[i * G + g] = w;
+          l_loc[g] += (float)cnt * w;
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float v = warp_sum(l_loc[g]);
+        if (lane == 0) s_part[warp][g] = v;
+      }
+      __syncthreads();
+      if (tid < G) {
+        float v = 0.f;
+        for (int w = 0; w < NW; ++w) v += s_part[w][tid];
+        s_l[tid] = v;
       }
     }
-  }
-  // phase 4: remove the steady members of estimated clusters
-  if (a1 > a0) {
-    const int s_begin = ast[a0], s_end = ast[a1];
-    const int32_t* slots = st_slot + (int64_t)u * cap;
-    const int32_t* cls = st_cl + (int64_t)u * cap;
-    const T* vpb = reinterpret_cast<const T*>(vp.base) + sub * EPL;
-    for (int base = s_begin + warp * RPW; base < s_end; base += NW * RPW) {
-      const int i = base + rsub;
-      bool ok = false;
-      int64_t ro = -1;
-      int ci = 0;
-      if (i < s_end) {
-        ci = cls[i] - c0;
-        ok = ci >= 0 && ci < c1 - c0 && s_cnt[ci] > 0;
-        if (ok) {
-          ro = pool_row(vp, geo.hkv, D, b, h, slots[i], status);
-          ok = ro >= 0;
+    // stream the value sums through the ring
+    for (int t = 0; t < ntile; ++t) {
+      cp_async_wait<NST - 1>();
+      __syncthreads();
+      if (!skip) {
+        const T* tile = ring + (size_t)(t % NST) * TR * D;
+        const int r0 = t * TR, nr = min(TR, c1 - c0 - r0);
+        for (int rb = warp * RPW; rb < nr; rb += NW * RPW) {
+          const int r = rb + rsub;
+          if (r < nr && s_cnt[r0 + r] > 0) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(tile + r * D + sub * EPL);
+            float x[EPL];
+            Elem<T>::unpack(raw, x);
+            float wv[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) wv[g] = s_w[(r0 + r) * G + g];
+            axpy_g<G, EPL>(wv, x, acc);
+          }
         }
       }
-      if (ok) {
-        const uint4 raw = ld_stream(vpb + ro);
+      __syncthreads();
+      issue(t + NST);
+    }
+    cp_async_wait<0>();
+    if (!skip) {
+      // Vsum' = Vsum - (values of the cluster's steady members)
+      int a0, a1;
+      {  // affected clusters inside [c0, c1)
+        int lo = 0, hi = n_aff;
+        while (lo < hi) { const int mid = (lo + hi) >> 1; if (s_acl[mid] < c0) lo = mid + 1; else hi = mid; }
+        a0 = lo;
+        hi = n_aff;
+        while (lo < hi) { const int mid = (lo + hi) >> 1; if (s_acl[mid] < c1) lo = mid + 1; else hi = mid; }
+        a1 = lo;
+      }
+      // each affected cluster of the chunk that is estimated: subtract w * dV
+      for (int base = a0 + warp * RPW; base < a1; base += NW * RPW) {
+        const int j = base + rsub;
+        if (j >= a1) continue;
+        const int ci = s_acl[j] - c0;
+        if (ci < 0 || ci >= c1 - c0 || s_cnt[ci] <= 0) continue;
+        const float* dvr = A.dv + ((int64_t)u * A.cap + j) * D + sub * EPL;
+        float x[EPL];
+#pragma unroll
+        for (int e4 = 0; e4 < EPL; e4 += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(dvr + e4);
+          x[e4] = v.x; x[e4 + 1] = v.y; x[e4 + 2] = v.z; x[e4 + 3] = v.w;
+        }
+        float wv[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) wv[g] = -s_w[ci * G + g];
+        axpy_g<G, EPL>(wv, x, acc);
+      }
+      reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part);
+      if (tid < G) { part[tid * PS] = s_m[tid]; part[tid * PS + 1] = s_l[tid]; }
+    } else {
+      for (int i = tid; i < G * PS; i += blockDim.x) part[i] = (i % PS) == 0 ? -INFINITY : 0.f;
+    }
+  } else {
+    // -------------------------------------------------------------- attend
+    float qv[G][EPL];
+    load_q<T, D, G>(q, n_q_heads, b, h, sub, A.scale, qv);
+    pdl_wait();
+    const int32_t* I = A.info + (int64_t)u * kInfoInts;
+    const int dense = I[6];
+    const int n_tok = (dense ? 0 : I[3]) + I[4];
+    const int per = (n_tok + A.n_splits - 1) / A.n_splits;
+    const int t0 = min(n_tok, (int)blockIdx.x * per);
+    const int t1 = min(n_tok, t0 + per);
+    const int32_t* gat = A.gather + (int64_t)u * A.gather_stride;
+    T* const kt0 = ring;
+    T* const vt0 = ring + (size_t)2 * TR * D;
+    const T* kbase = reinterpret_cast<const T*>(kp.base);
+    const T* vbase = reinterpret_cast<const T*>(vp.base);
+    const int ntile = t0 < t1 ? (t1 - t0 + TR - 1) / TR : 0;
+
+    // tile t: pool rows from the gather list, then 16-byte copies of K and V
+    auto stage = [&](int t) {
+      const int bi = t & 1;
+      const int tb = t0 + t * TR, n = min(TR, t1 - tb);
+      if (tid < TR) {
+        const int32_t ri = tid < n ? gat[tb + tid] : -1;
+        s_row[bi][tid] = ri >= 0 ? (int64_t)ri * D : -1;
+      }
+      __syncthreads();
+      T* kt = kt0 + (size_t)bi * TR * D;
+      T* vt = vt0 + (size_t)bi * TR * D;
+      for (int i = tid; i < n * LPR; i += blockDim.x) {
+        const int r = i / LPR, ch = i - r * LPR;
+        const int64_t ro = s_row[bi][r];
+        if (ro >= 0) {
+          cp_async16(kt + r * D + ch * EPL, kbase + ro + ch * EPL);
+          cp_async16(vt + r * D + ch * EPL, vbase + ro + ch * EPL);
+        }
+      }
+      cp_async_commit();
+    };
+
+    float m_run[G], l_run[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) { m_run[g] = -INFINITY; l_run[g] = 0.f; }
+    if (ntile > 0) stage(0);
+    for (int t = 0; t < ntile; ++t) {
+      const int bi = t & 1;
+      if (t + 1 < ntile) { stage(t + 1); cp_async_wait<1>(); } else { cp_async_wait<0>(); }
+      __syncthreads();
+      const T* kt = kt0 + (size_t)bi * TR * D;
+      const T* vt = vt0 + (size_t)bi * TR * D;
+      for (int rb = warp * RPW; rb < TR; rb += NW * RPW) {
+        const int r = rb + rsub;
+        const int64_t ro = s_row[bi][r];
+        float x[EPL];
+        if (ro >= 0) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(kt + r * D + sub * EPL);
+          Elem<T>::unpack(raw, x);
+        } else {
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) x[e] = 0.f;
+        }
+        float a[G];
+        dot_g<G, EPL>(qv, x, a);
+        group_reduce_multi<G, LPR>(a, lane);
+        if (sub % (LPR / G) == 0) s_sc[r][jh] = ro >= 0 ? a[0] : -INFINITY;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float mt = -INFINITY;
+        for (int r = lane; r < TR; r += 32) mt = fmaxf(mt, s_sc[r][g]);
+        mt = warp_max(mt);
+        const float mnew = fmaxf(m_run[g], mt);
+        const float corr = mnew == -INFINITY ? 1.f : __expf(m_run[g] - mnew);
+        float ps = 0.f;
+        for (int r = lane; r < TR; r += 32) {
+          const float sv = s_sc[r][g];
+          ps += sv == -INFINITY ? 0.f : __expf(sv - mnew);
+        }
+        ps = warp_sum(ps);
+        l_run[g] = l_run[g] * corr + ps;
+        m_run[g] = mnew;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[g][e] *= corr;
+      }
+      for (int rb = warp * RPW; rb < TR; rb += NW * RPW) {
+        const int r = rb + rsub;
+        if (s_row[bi][r] < 0) continue;
+        const uint4 raw = *reinterpret_cast<const uint4*>(vt + r * D + sub * EPL);
         float x[EPL];
         Elem<T>::unpack(raw, x);
+        float pw[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float w = s_w[ci * G + g];
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) acc[g][e] = fmaf(-w, x[e], acc[g][e]);
-        }
+        for (int g = 0; g < G; ++g) pw[g] = __expf(s_sc[r][g] - m_run[g]);
+        axpy_g<G, EPL>(pw, x, acc);
       }
+      __syncthreads();
+    }
+    reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part);
+    if (tid == 0) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) { part[g * PS] = m_run[g]; part[g * PS + 1] = l_run[g]; }
     }
   }
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int e = 0; e < EPL; ++e)
-#pragma unroll
-      for (int o = LPR; o < 32; o <<= 1) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], o);
-  if (rsub == 0) {
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) s_red[warp][g][sub * EPL + e] = acc[g][e];
+
+  // ---------------------------------------- last CTA of the unit merges
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(A.counters + u, 1) == A.n_parts - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // stage every part's (m, l) in shared memory with one round of loads
+  float* f = s_w;                                   // [n_parts][G] rescale factors
+  float* lp = reinterpret_cast<float*>(ring);       // [n_parts][G] part denominators
+  const float* pbase = A.partials + (int64_t)u * A.n_parts * G * PS;
+  for (int i = tid; i < A.n_parts * G; i += blockDim.x) {
+    f[i] = __ldcg(pbase + (int64_t)i * PS);
+    lp[i] = __ldcg(pbase + (int64_t)i * PS + 1);
   }
   __syncthreads();
-  for (int i = tid; i < G * D; i += blockDim.x) {
-    const int g = i / D, e = i - g * D;
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) v += s_red[w][g][e];
-    part[g * (D + 2) + 2 + e] = v;
+  if (warp < G) {
+    float M = -INFINITY;
+    for (int p = lane; p < A.n_parts; p += 32) M = fmaxf(M, f[p * G + warp]);
+    M = warp_max(M);
+    float l = 0.f;
+    for (int p = lane; p < A.n_parts; p += 32) {
+      const float mp = f[p * G + warp];
+      l += mp == -INFINITY ? 0.f : expf(mp - M) * lp[p * G + warp];
+    }
+    l = warp_sum(l);
+    if (lane == 0) { s_m[warp] = M; s_l[warp] = l; }
   }
-  if (tid < G) {
-    part[tid * (D + 2)] = s_m[tid];
-    part[tid * (D + 2) + 1] = s_l[tid];
+  __syncthreads();
+  for (int i = tid; i < A.n_parts * G; i += blockDim.x) {
+    const float mp = f[i];
+    f[i] = mp == -INFINITY ? 0.f : expf(mp - s_m[i % G]);
   }
-}
-
-// ------------------------------------------------------------------- merge
-// One CTA per (unit, q head): log-sum-exp combine of all parts.
-template <int D, int G>
-__global__ void __launch_bounds__(128)
-wave_merge_kernel(const Geo geo, const float* __restrict__ partials, int n_parts, int n_q_heads,
-                  float* __restrict__ out, float* __restrict__ lse) {
-  const int u = blockIdx.x / G, g = blockIdx.x % G;
-  const int b = u / geo.hkv, h = u - b * geo.hkv;
-  const float* base = partials + ((int64_t)u * n_parts * G + g) * (D + 2);
-  const int64_t stride = (int64_t)G * (D + 2);
-  float M = -INFINITY;
-  for (int p = 0; p < n_parts; ++p) M = fmaxf(M, base[p * stride]);
-  float l = 0.f;
-  float o[(D + 127) / 128];
+  __syncthreads();
+  {
+    // thread t sums float4 chunk (t % NCH) over parts p = t / NCH, t / NCH + PP, ...
+    constexpr int NCH = G * D / 4;                  // float4 chunks of one part's outputs
+    constexpr int PP = kStreamThreads / NCH > 0 ? kStreamThreads / NCH : 1;
+    float4* red4 = reinterpret_cast<float4*>(lp + ((A.n_parts * G + 3) & ~3));
+    for (int ch = tid % NCH; ch < NCH; ch += kStreamThreads) {
+      const int g = (ch * 4) / D, e = (ch * 4) - g * D;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      int p = tid / NCH;
+      for (; p + 3 * PP < A.n_parts; p += 4 * PP) {  // four independent loads in flight
+        float4 v[4];
 #pragma unroll
-  for (int i = 0; i < (D + 127) / 128; ++i) o[i] = 0.f;
-  for (int p = 0; p < n_parts; ++p) {
-    const float mp = base[p * stride];
-    const float f = mp == -INFINITY ? 0.f : expf(mp - M);
-    l += f * base[p * stride + 1];
+        for (int k = 0; k < 4; ++k)
+          v[k] = __ldcg(reinterpret_cast<const float4*>(pbase + ((int64_t)(p + k * PP) * G + g) * PS + Part<D>::kO + e));
 #pragma unroll
-    for (int i = 0; i < (D + 127) / 128; ++i) {
-      const int e = threadIdx.x + 128 * i;
-      if (e < D) o[i] += f * base[p * stride + 2 + e];
+        for (int k = 0; k < 4; ++k) {
+          const float w = f[(p + k * PP) * G + g];
+          o.x += w * v[k].x; o.y += w * v[k].y; o.z += w * v[k].z; o.w += w * v[k].w;
+        }
+      }
+      for (; p < A.n_parts; p += PP) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(pbase + ((int64_t)p * G + g) * PS + Part<D>::kO + e));
+        const float w = f[p * G + g];
+        o.x += w * v.x; o.y += w * v.y; o.z += w * v.z; o.w += w * v.w;
+      }
+      if (tid < NCH * PP) red4[tid] = o;
+    }
+    __syncthreads();
+    for (int ch = tid; ch < NCH; ch += blockDim.x) {
+      float4 o = red4[ch];
+      for (int k = 1; k < PP; ++k) {
+        const float4 v = red4[ch + k * NCH];
+        o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
+      }
+      const int g = (ch * 4) / D, e = (ch * 4) - g * D;
+      const float l = s_l[g];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int64_t qh = (int64_t)b * n_q_heads + (int64_t)h * G + g;
+      *reinterpret_cast<float4*>(A.out + qh * D + e) =
+          make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+      if (e == 0 && A.lse != nullptr) A.lse[qh] = l > 0.f ? s_m[g] + logf(l) : -INFINITY;
     }
   }
-  const int64_t qh = (int64_t)b * n_q_heads + (int64_t)h * G + g;
-#pragma unroll
-  for (int i = 0; i < (D + 127) / 128; ++i) {
-    const int e = threadIdx.x + 128 * i;
-    if (e < D) out[qh * D + e] = l > 0.f ? o[i] / l : 0.f;
-  }
-  if (lse != nullptr && threadIdx.x == 0) lse[qh] = l > 0.f ? M + logf(l) : -INFINITY;
+  if (tid == 0) A.counters[u] = 0;
 }
 
 template <typename F>
@@ -819,7 +1115,49 @@ cudaError_t with_types(int dtype, int D, int G, F&& f) {
   return cudaErrorInvalidValue;
 }
 
+template <typename Kern, typename... Args>
+cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                      Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+template <typename... Args>
+cudaError_t launch_topk(dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                        Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kTopkCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, wave_topk_kernel, args...);
+}
+
 }  // namespace
+
+size_t decode_attend_smem(int dtype, int D, int G, int wcap, int echunk, int cap) {
+  (void)dtype;
+  const size_t ring = 4 * 16384;  // also holds the NW*G*D fp32 reduction (<= 32 KB)
+  return ring + (size_t)wcap * G * 4 + (size_t)echunk * 4 + (size_t)(2 * cap + 2) * 4;
+}
 
 cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
   unsigned char* ws = a.ws;
@@ -827,46 +1165,62 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
   float* scores = reinterpret_cast<float*>(ws + p.off_scores);
   uint32_t* keys = reinterpret_cast<uint32_t*>(ws + p.off_keys);
   int32_t* sel = reinterpret_cast<int32_t*>(ws + p.off_sel);
+  int32_t* sel_slot0 = reinterpret_cast<int32_t*>(ws + p.off_sel_slot0);
   int32_t* seltok = reinterpret_cast<int32_t*>(ws + p.off_seltok);
+  int32_t* split_first = reinterpret_cast<int32_t*>(ws + p.off_split);
   int32_t* info = reinterpret_cast<int32_t*>(ws + p.off_info);
+  int32_t* counters = reinterpret_cast<int32_t*>(ws + p.off_counters);
+  int32_t* hist = reinterpret_cast<int32_t*>(ws + p.off_hist);
   int32_t* st_slot = reinterpret_cast<int32_t*>(ws + p.off_st_slot);
   int32_t* st_cl = reinterpret_cast<int32_t*>(ws + p.off_st_cl);
   int32_t* aff_cl = reinterpret_cast<int32_t*>(ws + p.off_aff_cl);
   int32_t* aff_start = reinterpret_cast<int32_t*>(ws + p.off_aff_start);
   float* partials = reinterpret_cast<float*>(ws + p.off_partials);
+  int32_t* gather = reinterpret_cast<int32_t*>(ws + p.off_gather);
+  float* dv = reinterpret_cast<float*>(ws + p.off_dv);
   cudaEvent_t* ev = a.stage_events;
+  const bool pdl = ev == nullptr;  // stage timing serialises the launches
   auto mark = [&](int i) { if (ev) cudaEventRecord(ev[i], s); };
 
   return with_types(p.dtype, p.D, p.G, [&]<typename T, int D, int G>() -> cudaError_t {
     const T* q = reinterpret_cast<const T*>(a.q);
+    SteadyArgs sa{a.invperm, a.labels, a.vp, p.n_sink, p.window, p.cap, p.sort_pow2, st_slot,
+                  st_cl, aff_cl, aff_start, info, dv};
+    cudaError_t e;
     mark(0);
-    wave_steady_kernel<<<p.U, kStreamThreads, p.sort_pow2 * sizeof(int32_t), s>>>(
-        p.geo, a.invperm, a.offsets, p.n_sink, p.window, p.cap, p.sort_pow2, st_slot, st_cl,
-        aff_cl, aff_start, info, status);
+    const size_t score_smem = std::max<size_t>(65536 + (kHistBins + 1) * 4 +
+                                                   (size_t)(65536 / (D * sizeof(T)) + 1) * 4,
+                                               (size_t)p.sort_pow2 * 8);
+    cudaFuncSetAttribute(wave_score_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)score_smem);
+    e = launch_ex(wave_score_kernel<T, D, G>, dim3(p.n_score_blocks + 1, p.U),
+                  dim3(kStreamThreads), score_smem, s, false, p.geo, q, p.Hq,
+                  reinterpret_cast<const T*>(a.centroids), a.offsets, scores, keys, hist, p.scale,
+                  p.n_score_blocks, sa, status);
+    if (e != cudaSuccess) return e;
     mark(1);
-    wave_score_kernel<T, D, G><<<dim3(p.n_score_blocks, p.U), kStreamThreads, 0, s>>>(
-        p.geo, q, p.Hq, reinterpret_cast<const T*>(a.centroids), a.offsets, scores, keys,
-        p.scale, p.score_chunk);
+    const size_t topk_smem = ((size_t)p.topk_smem_keys * 2 + 3 + p.topk_smem_keys / 32 + 1 +
+                              3 * (size_t)p.cap) * sizeof(uint32_t);
+    cudaFuncSetAttribute(wave_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)topk_smem);
+    e = launch_topk(dim3(p.U * kTopkCluster), dim3(kTopkThreads), topk_smem, s, pdl, p.geo,
+                    (const uint32_t*)keys, a.offsets, hist, (const int32_t*)aff_cl,
+                    (const int32_t*)aff_start, p.cap, p.topk_clusters, p.topk_fraction,
+                    p.n_splits, p.topk_smem_keys, sel, sel_slot0, seltok, split_first, info,
+                    (const int32_t*)st_slot, a.kp, gather, (int64_t)p.gather_stride, status);
+    if (e != cudaSuccess) return e;
     mark(2);
-    wave_topk_kernel<<<p.U, kTopkThreads, 0, s>>>(p.geo, keys, a.offsets, aff_cl, aff_start,
-                                                  p.cap, p.topk_clusters, p.topk_fraction, sel,
-                                                  seltok, info);
+    AttendArgs A{gather, aff_cl, aff_start, dv, (int64_t)p.gather_stride, info, scores, keys,
+                 p.n_sink, p.window, p.cap, p.n_splits, p.n_est, p.echunk, p.n_parts, p.wcap,
+                 partials, counters, a.out, a.lse, p.scale};
+    const size_t smem = decode_attend_smem(p.dtype, D, G, p.wcap, p.echunk, p.cap);
+    cudaFuncSetAttribute(wave_attend_estimate_kernel<T, D, G>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = launch_ex(wave_attend_estimate_kernel<T, D, G>, dim3(p.n_splits + p.n_est, p.U),
+                  dim3(kStreamThreads), smem, s, pdl, p.geo, q, p.Hq, a.kp, a.vp,
+                  reinterpret_cast<const T*>(a.value_sums), a.offsets, A, status);
+    if (e != cudaSuccess) return e;
     mark(3);
-    wave_attend_kernel<T, D, G><<<dim3(p.n_splits, p.U), kStreamThreads, 0, s>>>(
-        p.geo, q, p.Hq, a.kp, a.vp, a.perm, a.offsets, sel, seltok, st_slot, info, p.n_sink,
-        p.window, p.cap, p.n_splits, p.n_parts, partials, p.scale, status);
-    mark(4);
-    const size_t est_smem = (size_t)p.echunk * (G + 1) * sizeof(float);
-    cudaFuncSetAttribute(wave_estimate_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)est_smem);
-    wave_estimate_kernel<T, D, G><<<dim3(p.n_est, p.U), kStreamThreads, est_smem, s>>>(
-        p.geo, reinterpret_cast<const T*>(a.value_sums), a.offsets, scores, keys, info, aff_cl,
-        aff_start, st_slot, st_cl, a.vp, p.cap, p.echunk, p.n_splits, p.n_parts, partials,
-        status);
-    mark(5);
-    wave_merge_kernel<D, G><<<p.U * G, 128, 0, s>>>(p.geo, partials, p.n_parts, p.Hq, a.out,
-                                                    a.lse);
-    mark(6);
     return cudaGetLastError();
   });
 }

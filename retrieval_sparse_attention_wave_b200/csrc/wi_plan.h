@@ -10,7 +10,8 @@
 namespace wi {
 
 constexpr int kStreamThreads = 256;   // streaming kernels: 8 warps
-constexpr int kTopkThreads = 1024;    // one CTA per unit
+constexpr int kTopkThreads = 256;     // per CTA of a top-k cluster
+constexpr int kTopkCluster = 8;       // CTAs per unit in the top-k cluster
 constexpr int kAttendTile = 64;       // tokens per exact-attention tile
 constexpr int kInfoInts = 8;          // per-unit info record (see wi_decode_layout)
 constexpr int kNumSMs = 148;          // B200
@@ -21,16 +22,22 @@ struct DecodePlan {
   int n_sink, window, topk_clusters;
   double topk_fraction;
   int max_nc;
+  int seg_len, seg_clusters;  // segment length and clusters per full segment
   int score_chunk, n_score_blocks;
+  int topk_smem_keys;      // keys per top-k CTA (ceil(NC / kTopkCluster)) held in shared memory
   int cap;                 // steady-list capacity per unit (>= 1)
   int sort_pow2;           // shared-memory sort size for the steady list
   int n_splits;            // exact-attention CTAs per unit
   int echunk, n_est;       // estimation clusters per CTA, CTAs per unit
   int n_parts;             // n_splits + n_est softmax parts per (unit, head)
+  int wcap;                // max(echunk, n_parts): weight / merge-factor rows
   float scale;             // 1/sqrt(d)
   // workspace byte offsets
-  size_t off_status, off_scores, off_keys, off_sel, off_seltok, off_info;
+  size_t off_status, off_counters, off_hist, off_scores, off_keys, off_sel, off_sel_slot0, off_seltok;
+  size_t off_split, off_info;
   size_t off_st_slot, off_st_cl, off_aff_cl, off_aff_start, off_partials;
+  size_t off_gather, off_dv;
+  int64_t gather_stride;   // gather-list entries per unit (max T_b)
   size_t off_q, off_out, off_lse;
   size_t total;
 };
@@ -52,6 +59,7 @@ struct DecodeArgs {
   const int32_t* offsets;
   const int32_t* perm;
   const int32_t* invperm;
+  const int32_t* labels;
   Pool kp, vp;
   float* out;
   float* lse;
@@ -67,6 +75,7 @@ struct BuildArgs {
   int32_t* offsets;
   int32_t* perm;
   int32_t* invperm;
+  int32_t* labels;
   void* kout;
   void* vout;
   const int32_t* bt_out;
@@ -76,10 +85,11 @@ struct BuildArgs {
   unsigned char* ws;
 };
 
-constexpr int kDecodeStages = 6;
+constexpr int kDecodeStages = 3;
 extern const char* const kDecodeStageNames[kDecodeStages];
 
 cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
+size_t decode_attend_smem(int dtype, int D, int G, int wcap, int echunk, int cap);
 cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s);
 cudaError_t launch_assign_only(const BuildPlan& p, const BuildArgs& a, const float* cent32,
                                int32_t* assign, cudaStream_t s);

@@ -28,7 +28,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_stage_names():
-    assert W.stage_names() == ["steady", "score", "topk", "attend", "estimate", "merge"]
+    assert W.stage_names() == ["score", "topk", "attend_estimate"]
     assert W.lib().wi_decode_stage_name(99) is None
 
 
@@ -67,8 +67,8 @@ def index_struct(**over):
     s.n_kv_heads, s.head_dim, s.page_size, s.seg_len, s.cluster_size = 8, 128, 16, 1024, 16
     s._seq = (C.c_int32 * len(seq))(*seq)
     s.seq_lens = C.cast(s._seq, C.POINTER(C.c_int32))
-    for i, f in enumerate(["centroids", "value_sums", "offsets", "perm", "invperm", "k_pool",
-                           "v_pool", "block_table"]):
+    for i, f in enumerate(["centroids", "value_sums", "offsets", "perm", "invperm", "labels",
+                           "k_pool", "v_pool", "block_table"]):
         setattr(s, f, FAKE + (i + 1) * 0x1000000)
     s.n_pages = 4096
     s.max_pages = 4096

@@ -131,6 +131,7 @@ def check_valid(wl, wx, b, h, keys, vals):
     cl = np.repeat(np.arange(NC), np.diff(off))
     same = cl[1:] == cl[:-1]
     assert np.all(perm[1:][same] > perm[:-1][same])   # ascending inside a cluster
+    assert np.array_equal(g["labels"][perm], cl)        # labels name each position's cluster
     np.testing.assert_array_equal(g["k_perm"], keys[b][h][perm])
     np.testing.assert_array_equal(g["v_perm"], vals[b][h][perm])
     cnt = np.diff(off)

@@ -84,6 +84,9 @@ def upload_unit(wx: W.WaveIndex, b: int, h: int, ix: O.UnitIndex):
     t = wx.tok_row(b, h)
     wx.perm[t:t + T] = torch.as_tensor(ix.perm.astype(np.int32), device=dev)
     wx.invperm[t:t + T] = torch.as_tensor(ix.invperm.astype(np.int32), device=dev)
+    lab = np.empty(T, dtype=np.int64)                 # cluster of each position
+    lab[ix.perm] = np.repeat(np.arange(NC), np.diff(ix.offsets))
+    wx.labels[t:t + T] = torch.as_tensor(lab.astype(np.int32), device=dev)
     pages, rows = _slot_addr(wx, b, T)
     wx.k_pool[pages, h, rows] = torch.as_tensor(ix.k_perm, device=dev).to(wx.dtype)
     wx.v_pool[pages, h, rows] = torch.as_tensor(ix.v_perm, device=dev).to(wx.dtype)
@@ -105,13 +108,14 @@ def download_unit(wx: W.WaveIndex, b: int, h: int) -> dict:
         offsets=wx.offsets[o:o + NC + 1].cpu().numpy().astype(np.int64),
         perm=wx.perm[t:t + T].cpu().numpy().astype(np.int64),
         invperm=wx.invperm[t:t + T].cpu().numpy().astype(np.int64),
+        labels=wx.labels[t:t + T].cpu().numpy().astype(np.int64),
         k_perm=f(wx.k_pool[pages, h, rows]), v_perm=f(wx.v_pool[pages, h, rows]))
 
 
 def as_unit_index(d: dict) -> O.UnitIndex:
     return O.UnitIndex(centroids=d["centroids"], value_sums=d["value_sums"],
                        offsets=d["offsets"], perm=d["perm"], invperm=d["invperm"],
-                       k_perm=d["k_perm"], v_perm=d["v_perm"], labels=None,
+                       k_perm=d["k_perm"], v_perm=d["v_perm"], labels=d["labels"],
                        centroids_exact=None, value_sums_exact=None)
 
 

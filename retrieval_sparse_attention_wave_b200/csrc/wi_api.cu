@@ -138,8 +138,9 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   // score: one CTA per 64 KB of centroid rows
   pl.score_chunk = 65536 / (pl.D * esize(ix->dtype));
   pl.n_score_blocks = (int)cdiv(max_nc, pl.score_chunk);
-  pl.topk_smem_keys = (int)cdiv(max_nc, kTopkCluster);
-  if (pl.topk_smem_keys > 20480) return WI_ERR_UNSUPPORTED;   // > 163,840 clusters per sequence
+  // top-k shared memory: exclusion bitmask, steady lists, one round's list
+  if ((size_t)(max_nc + 31) / 32 * 4 + 8 * (size_t)cap + 8 * 8192 + 8 > 200 * 1024)
+    return WI_ERR_UNSUPPORTED;
   // exact attention: about two 16 KB tiles of rows per CTA
   const int row_bytes = pl.D * esize(ix->dtype);
   const int tile_rows = 16384 / row_bytes;

@@ -31,8 +31,6 @@
 #include <algorithm>
 #include <cmath>
 
-#include <cooperative_groups.h>
-
 #include "wi_common.cuh"
 #include "wi_plan.h"
 
@@ -286,75 +284,54 @@ wave_score_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const T
 }
 
 // ----------------------------------------------------------------- K_B topk
-// A thread-block cluster of kTopkCluster CTAs per unit; CTA r owns the
-// contiguous cluster-id range [r*chunk, (r+1)*chunk) with its keys in shared
-// memory.  The first radix digit comes from K_A's histogram (identical in
-// every CTA; zeroed after use so the workspace is clean for the next call,
-// and rebuilt if its total disagrees with the candidate count).  The next
-// two digits merge per-CTA histograms through distributed shared memory.
-// The ordered selection and its token prefix use per-CTA counts exchanged
-// the same way.  Five cluster barriers in all.
-__device__ __forceinline__ int suffix_digit(const int* hist, int nbins, int krem, int* scan_sh,
-                                            int* bc) {
-  // thread t owns bins nbins-1-8t .. nbins-8-8t (descending)
-  const int tid = threadIdx.x;
-  int c[8], s8 = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int bin = nbins - 1 - 8 * tid - i;
-    c[i] = bin >= 0 ? hist[bin] : 0;
-    s8 += c[i];
-  }
-  int tot;
-  const int incl = block_inclusive_scan(s8, scan_sh, &tot);
-  int acc = incl - s8;
-  if (acc < krem && incl >= krem) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (acc + c[i] >= krem) { bc[0] = nbins - 1 - 8 * tid - i; bc[1] = acc; break; }
-      acc += c[i];
-    }
-  }
-  __syncthreads();
-  return bc[0];
-}
+// One CTA per unit.  Keys are walked in rounds of kTopkThreads*16: warp w
+// owns a contiguous id range of 512 per round, lane-interleaved (coalesced
+// loads, ballot-based ranking, no shared-memory bank conflicts).
+//  1. the first radix digit's histogram comes from K_A (zeroed after use, so
+//     the workspace is clean for the next call; a histogram whose total
+//     disagrees with the candidate count is rebuilt and flagged);
+//  2. the keys in the threshold bin (1-2% of them) are gathered and ranked
+//     exactly by (key desc, id asc); more than kTopkCand of them fall back
+//     to two further radix digits over all keys;
+//  3. an ordered compaction writes the selection, its slot starts, the token
+//     prefix, the split starts and the gather list (pool rows of the
+//     retrieved clusters' tokens, -1 for their steady members).
+constexpr int kTopkPerLane = 16;
+constexpr int kTopkRound = kTopkThreads * kTopkPerLane;   // 8192 ids per round
+constexpr int kTopkCand = 1024;
 
 __global__ void __launch_bounds__(kTopkThreads)
 wave_topk_kernel(const Geo geo, const uint32_t* __restrict__ keys,
                  const int32_t* __restrict__ offsets, int32_t* __restrict__ hist_g,
                  const int32_t* __restrict__ aff_cl, const int32_t* __restrict__ aff_start, int cap,
-                 int topk_clusters, double topk_fraction, int n_splits, int smem_keys,
+                 int topk_clusters, double topk_fraction, int n_splits,
                  int32_t* __restrict__ sel, int32_t* __restrict__ sel_slot0,
                  int32_t* __restrict__ sel_tok, int32_t* __restrict__ split_first,
                  int32_t* __restrict__ info, const int32_t* __restrict__ st_slot, const Pool kp,
                  int32_t* __restrict__ gather, int64_t gather_stride, uint32_t* status) {
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
-  // shared: keys [smem_keys + 1] | offsets [smem_keys + 1] | excluded bitmask
-  //         [smem_keys/32 + 1] | affected list (cluster, steady count) [2 * cap]
-  //         | steady slots [cap]; keys and offsets later hold the gather-list chunk
-  extern __shared__ uint32_t sk[];
-  int32_t* so = reinterpret_cast<int32_t*>(sk + smem_keys + 1);
-  uint32_t* sx = reinterpret_cast<uint32_t*>(so + smem_keys + 1);
-  int32_t* sa = reinterpret_cast<int32_t*>(sx + smem_keys / 32 + 1);
-  int32_t* ss = sa + 2 * cap;
-  __shared__ int hist[kHistBins];                // digit 1 (all CTAs identical)
-  __shared__ int mh[2][kHistBins];               // merged histograms of digits 2 and 3
+  // dynamic shared: excluded bitmask [ceil(NCmax/32)] | steady slots [cap]
+  //                 | affected list [cap] | round list (token start, slot start) [2 * kTopkRound + 2]
+  extern __shared__ int32_t sdyn[];
+  __shared__ int hist[kHistBins];
+  __shared__ unsigned long long cand[kTopkCand];
   __shared__ int scan_sh[64];
-  __shared__ int bc[4];
-  __shared__ int x_cnt[4];                       // values the other CTAs read
-  __shared__ int s_wgt[32], s_weq[32], s_wgt2[32], s_weq2[32];
-  __shared__ int s_info[8];
+  __shared__ int s_info[kInfoInts];
+  __shared__ int s_w[2][32];
+  __shared__ int s_ctl[8];
   pdl_launch_dependents();
-  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
-  const int rank = (int)cluster.block_rank();
-  const int R = kTopkCluster;
-  const int u = blockIdx.x / R, b = u / geo.hkv, h = u - b * geo.hkv;
-  const int NC = geo.NC(b);
-  const int chunk = (NC + R - 1) / R;
-  const int c_lo = min(NC, rank * chunk), c_hi = min(NC, c_lo + chunk), nk = c_hi - c_lo;
-  for (int i = tid; i < 2 * kHistBins; i += nt) (&mh[0][0])[i] = 0;
-  for (int i = tid; i <= nk / 32; i += nt) sx[i] = 0u;
+  const int tid = threadIdx.x, nt = kTopkThreads, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = kTopkThreads / 32;
+  const unsigned lt = (1u << lane) - 1u;
+  const int u = blockIdx.x, b = u / geo.hkv, h = u - b * geo.hkv;
+  const int NC = geo.NC(b), Tb = geo.T(b);
+  const int nmask = (NC + 31) >> 5;
+  uint32_t* sx = reinterpret_cast<uint32_t*>(sdyn);
+  int32_t* ss = sdyn + nmask;
+  int32_t* sa = ss + cap;
+  int32_t* lst = sa + cap;                         // [kTopkRound + 1] token starts
+  int32_t* lso = lst + kTopkRound + 1;             // [kTopkRound] slot starts
+  for (int i = tid; i < nmask; i += nt) sx[i] = 0u;
+  if (tid == 0) s_ctl[0] = 0;
   pdl_wait();
   int32_t* I = info + (int64_t)u * kInfoInts;
   const int64_t row0 = geo.cl_row(b, h);
@@ -364,286 +341,263 @@ wave_topk_kernel(const Geo geo, const uint32_t* __restrict__ keys,
   const int k_req = topk_clusters >= 0 ? topk_clusters : (int)ceil(topk_fraction * (double)NC);
   const uint32_t* kk = keys + row0;
   const int32_t* off = offsets + geo.off_row(b, h);
-  // one round of independent loads: unit record, histogram, keys, offsets, steady lists
-  if (tid < 8) s_info[tid] = I[tid];
-  for (int i = tid; i < kHistBins; i += nt) hist[i] = hg[i];
-  for (int i = tid; i < nk; i += nt) sk[i] = kk[c_lo + i];
-  for (int i = tid; i <= nk; i += nt) so[i] = off[c_lo + i];
-  for (int i = tid; i < cap; i += nt) {  // unconditional: no wait on the unit record
-    sa[2 * i] = aff_cl[(int64_t)u * cap + i];
-    sa[2 * i + 1] = aff_start[(int64_t)u * (cap + 1) + i + 1] - aff_start[(int64_t)u * (cap + 1) + i];
+  int32_t* gat = gather + (int64_t)u * gather_stride;
+  // one round of independent loads
+  if (tid < kInfoInts) s_info[tid] = I[tid];
+  for (int i = tid; i < kHistBins; i += nt) { hist[i] = hg[i]; hg[i] = 0; }
+  for (int i = tid; i < cap; i += nt) {
+    sa[i] = aff_cl[(int64_t)u * cap + i];
     ss[i] = st_slot[(int64_t)u * cap + i];
   }
   __syncthreads();
   const int n_st = s_info[4];
   const int dense = s_info[6];
   const int n_aff = dense ? 0 : min(cap, s_info[5]);
-  const int Tb = geo.T(b);
-  int32_t* gat = gather + (int64_t)u * gather_stride;
-  // pool row index of slot s of this unit (-1 if the block table is out of range)
   auto row_of = [&](int slot) -> int32_t {
     const int64_t ro = pool_row(kp, geo.hkv, 1, b, h, slot, status);
     return ro < 0 ? -1 : (int32_t)ro;
   };
-  // clusters of this CTA's range left without a non-steady member are not candidates
-  for (int jj = tid; jj < n_aff; jj += nt) {
-    const int c = sa[2 * jj];
-    if (c >= c_lo && c < c_hi && so[c - c_lo + 1] - so[c - c_lo] - sa[2 * jj + 1] <= 0)
-      atomicOr(&sx[(c - c_lo) >> 5], 1u << ((c - c_lo) & 31));
-  }
-  __syncthreads();
-  auto key_of = [&](int i) -> uint32_t {  // local index; 0 if not a candidate
-    return ((sx[i >> 5] >> (i & 31)) & 1u) ? 0u : sk[i];
-  };
-  int mine = 0;
-  for (int i = tid; i < nk; i += nt) mine += key_of(i) != 0u;
-  int nc_local;
-  block_inclusive_scan(mine, scan_sh, &nc_local);
-  if (tid == 0) x_cnt[0] = nc_local;
-  cluster.sync();                                            // barrier 1
-  if (rank == 0)
-    for (int i = tid; i < kHistBins; i += nt) hg[i] = 0;    // every CTA has its copy
-  int ncand = 0;
-#pragma unroll
-  for (int r = 0; r < R; ++r) ncand += *cluster.map_shared_rank(&x_cnt[0], r);
   if (dense) {  // the attend CTAs take all slots in order
-    for (int t = rank * nt + tid; t < Tb; t += R * nt) gat[t] = row_of(t);
-    if (rank == 0) {
-      if (tid == 0) {
-        I[0] = 0; I[1] = (int32_t)0xFFFFFFFFu; I[2] = -1; I[3] = 0; I[7] = k_req;
-        pre[0] = 0;
-      }
-      for (int j = tid; j <= n_splits; j += nt) split[j] = 0;
+    for (int t = tid; t < Tb; t += nt) gat[t] = row_of(t);
+    if (tid == 0) {
+      I[0] = 0; I[1] = (int32_t)0xFFFFFFFFu; I[2] = -1; I[3] = 0; I[7] = k_req;
+      pre[0] = 0;
     }
-    cluster.sync();
+    for (int j = tid; j <= n_splits; j += nt) split[j] = 0;
     return;
   }
-  // remove the excluded clusters (any range) from this CTA's digit-1 histogram
-  for (int jj = tid; jj < n_aff; jj += nt) {
-    const int c = sa[2 * jj];
-    if (c < 0 || c >= NC) continue;
-    const int r = min(R - 1, c / max(chunk, 1));
-    const int li = c - r * chunk;
-    const int32_t* ro = cluster.map_shared_rank(so, r);
-    if (ro[li + 1] - ro[li] - sa[2 * jj + 1] <= 0) {
-      const uint32_t key = *cluster.map_shared_rank(sk + li, r);
+  // clusters left without a non-steady member are not candidates
+  for (int j = tid; j < n_aff; j += nt) {
+    const int c = sa[j];
+    const int dc = aff_start[(int64_t)u * (cap + 1) + j + 1] - aff_start[(int64_t)u * (cap + 1) + j];
+    if (c >= 0 && c < NC && __ldg(off + c + 1) - __ldg(off + c) - dc <= 0) {
+      atomicOr(&sx[c >> 5], 1u << (c & 31));
+      const uint32_t key = kk[c];
       if (key) atomicSub(&hist[key >> kHistShift], 1);
     }
   }
   __syncthreads();
-  {  // a stale digit-1 histogram (workspace reused after a failed call) is rebuilt
-    int hs = 0;
-    for (int i = tid; i < kHistBins; i += nt) hs += hist[i];
+  auto cand_key = [&](int c, uint32_t key) -> uint32_t {
+    return ((sx[c >> 5] >> (c & 31)) & 1u) ? 0u : key;
+  };
+  const int n_rounds = (NC + kTopkRound - 1) / kTopkRound;
+  const int wbase = warp * (kTopkRound / NW);       // warp's offset inside a round
+
+  // histogram total -> threshold bin of the first digit (valid if consistent)
+  int hs = 0;
+  for (int i = tid; i < kHistBins; i += nt) hs += hist[i];
+  int hist_total;
+  block_inclusive_scan(hs, scan_sh, &hist_total);
+  int ksel = min(max(k_req, 0), hist_total);
+  auto first_digit = [&](int krem, int* above) -> int {
+    // thread t owns bins 2047-4t .. 2044-4t (descending)
+    int c4[4], s4 = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { c4[i] = hist[kHistBins - 1 - 4 * tid - i]; s4 += c4[i]; }
     int tot;
-    block_inclusive_scan(hs, scan_sh, &tot);
-    if (tot != ncand) {
-      if (tid == 0 && rank == 0) flag_error(status, WI_DEV_BAD_HIST);
+    const int incl = block_inclusive_scan(s4, scan_sh, &tot);
+    int acc = incl - s4;
+    if (acc < krem && incl >= krem) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (acc + c4[i] >= krem) { s_ctl[1] = kHistBins - 1 - 4 * tid - i; s_ctl[2] = acc; break; }
+        acc += c4[i];
+      }
+    }
+    __syncthreads();
+    *above = s_ctl[2];
+    return s_ctl[1];
+  };
+  int bin1 = -1, above1 = 0;
+  if (ksel > 0 && ksel < hist_total) bin1 = first_digit(ksel, &above1);
+
+  // the round's keys / offsets in registers: all loads issued before any use
+  uint32_t kr[kTopkPerLane];
+  int o0r[kTopkPerLane], o1r[kTopkPerLane];
+  auto load_round = [&](int r, bool with_off) {
+#pragma unroll
+    for (int i = 0; i < kTopkPerLane; ++i) {
+      const int c = r * kTopkRound + wbase + i * 32 + lane;
+      kr[i] = c < NC ? kk[c] : 0u;
+      if (with_off) {
+        o0r[i] = c < NC ? __ldg(off + c) : 0;
+        o1r[i] = c < NC ? __ldg(off + c + 1) : 0;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kTopkPerLane; ++i) {
+      const int c = r * kTopkRound + wbase + i * 32 + lane;
+      kr[i] = c < NC ? cand_key(c, kr[i]) : 0u;
+    }
+  };
+  // pass A: candidate count, and the keys of the threshold bin
+  int mine = 0;
+  for (int r = 0; r < n_rounds; ++r) {
+    load_round(r, true);
+#pragma unroll
+    for (int i = 0; i < kTopkPerLane; ++i) {
+      const uint32_t key = kr[i];
+      if (key == 0u) continue;
+      ++mine;
+      if ((int)(key >> kHistShift) == bin1) {
+        const int c = r * kTopkRound + wbase + i * 32 + lane;
+        const int slot = atomicAdd(&s_ctl[0], 1);
+        if (slot < kTopkCand)
+          cand[slot] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)c);
+      }
+    }
+  }
+  int ncand;
+  block_inclusive_scan(mine, scan_sh, &ncand);
+  const int nbin = s_ctl[0];
+  const bool hist_ok = ncand == hist_total;
+  if (!hist_ok && tid == 0) flag_error(status, WI_DEV_BAD_HIST);
+  ksel = min(max(k_req, 0), ncand);
+  uint32_t kstar;
+  int thr;
+  if (ksel == 0) { kstar = 0xFFFFFFFFu; thr = -1; }
+  else if (ksel == ncand) { kstar = 1u; thr = NC; }
+  else if (hist_ok && nbin <= kTopkCand) {
+    // exact rank inside the threshold bin: the (ksel - above1)-th largest
+    const int want = ksel - above1 - 1;
+    for (int i = tid; i < nbin; i += nt) {
+      const unsigned long long x = cand[i];
+      int rank = 0;
+      for (int j = 0; j < nbin; ++j) rank += cand[j] > x;
+      if (rank == want) { s_ctl[3] = (int)(x >> 32); s_ctl[4] = (int)(0xFFFFFFFFu - (uint32_t)x); }
+    }
+    __syncthreads();
+    kstar = (uint32_t)s_ctl[3];
+    thr = s_ctl[4];
+  } else {
+    // fallback: a full radix select over all keys (stale histogram or a
+    // crowded threshold bin), 11 + 11 + 10 bit digits
+    uint32_t prefix = 0, pmask = 0;
+    int krem = ksel;
+    for (int pass = 0; pass < 3; ++pass) {
+      const int bits = pass == 2 ? 10 : 11;
+      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+      const int nbins = 1 << bits;
       for (int i = tid; i < kHistBins; i += nt) hist[i] = 0;
       __syncthreads();
-      for (int r = 0; r < R; ++r) {
-        const int lo = min(NC, r * chunk), n = min(NC, lo + chunk) - lo;
-        const uint32_t* rk = cluster.map_shared_rank(sk, r);
-        const uint32_t* rx = cluster.map_shared_rank(sx, r);
-        for (int i = tid; i < n; i += nt) {
-          const uint32_t key = ((rx[i >> 5] >> (i & 31)) & 1u) ? 0u : rk[i];
-          if (key) atomicAdd(&hist[key >> kHistShift], 1);
-        }
+      for (int c = tid; c < NC; c += nt) {
+        const uint32_t key = cand_key(c, kk[c]);
+        if (key != 0u && (key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nbins - 1)], 1);
       }
       __syncthreads();
-    }
-  }
-  const int ksel = min(max(k_req, 0), ncand);
-  int krem = ksel;
-  uint32_t prefix = 0, pmask = 0;
-  const bool radix = ksel > 0 && ksel < ncand;
-  if (radix) {
-    const int d = suffix_digit(hist, kHistBins, krem, scan_sh, bc);
-    krem -= bc[1];
-    prefix = (uint32_t)d << 21;
-    pmask = 0x7FFu << 21;
-  }
-#pragma unroll 1
-  for (int pass = 1; pass < 3; ++pass) {       // barriers 2 and 3 (taken by every CTA)
-    const int bits = pass == 2 ? 10 : 11;
-    const int shift = pass == 1 ? 10 : 0;
-    const int nbins = 1 << bits;
-    int* loc = hist;                             // digit-1 histogram no longer needed
-    if (radix) {
-      for (int i = tid; i < nbins; i += nt) loc[i] = 0;
-      __syncthreads();
-      for (int i = tid; i < nk; i += nt) {
-        const uint32_t key = key_of(i);
-        if (key != 0u && (key & pmask) == prefix) atomicAdd(&loc[(key >> shift) & (nbins - 1)], 1);
-      }
-      __syncthreads();
-      for (int i = tid; i < nbins; i += nt) {
-        const int v = loc[i];
-        if (v)
-#pragma unroll
-          for (int r = 0; r < R; ++r) atomicAdd(cluster.map_shared_rank(&mh[pass - 1][i], r), v);
-      }
-    }
-    cluster.sync();
-    if (radix) {
-      const int d = suffix_digit(mh[pass - 1], nbins, krem, scan_sh, bc);
-      krem -= bc[1];
+      int ab;
+      const int d = first_digit(krem, &ab) & (nbins - 1);
+      krem -= ab;
       prefix |= (uint32_t)d << shift;
       pmask |= (uint32_t)(nbins - 1) << shift;
+      __syncthreads();
     }
+    kstar = prefix;
+    // the krem-th key equal to kstar in ascending id order
+    if (tid == 0) s_ctl[4] = -1;
+    __syncthreads();
+    int run = 0;
+    for (int base = 0; base < NC && s_ctl[4] < 0; base += nt) {
+      const int c = base + tid;
+      const int f = (c < NC && cand_key(c, kk[c]) == kstar) ? 1 : 0;
+      int tot;
+      const int incl = block_inclusive_scan(f, scan_sh, &tot);
+      if (f && run + incl == krem) s_ctl[4] = c;
+      run += tot;
+      __syncthreads();
+    }
+    thr = s_ctl[4];
   }
-  uint32_t kstar;
-  int eq_take;  // how many keys equal to kstar are selected (lowest ids first)
-  if (ksel == 0) { kstar = 0xFFFFFFFFu; eq_take = 0; }
-  else if (ksel == ncand) { kstar = 1u; eq_take = INT_MAX; }
-  else { kstar = prefix; eq_take = krem; }
+  auto picked = [&](int c, uint32_t key) -> bool {  // key: candidate key or 0
+    return key != 0u && (key > kstar || (key == kstar && c <= thr));
+  };
 
-  // ordered selection: warp w of this CTA owns [wb, we) of its range
-  const unsigned lt = (1u << lane) - 1u;
-  const int B = (((nk + nw - 1) / nw) + 31) & ~31;
-  const int wb = min(nk, warp * B), we = min(nk, wb + B);
-  int gt_w = 0, eq_w = 0, tk_w = 0;
-  for (int base = wb; base < we; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < we ? key_of(i) : 0u;
-    gt_w += __popc(__ballot_sync(0xffffffffu, key != 0u && key > kstar));
-    eq_w += __popc(__ballot_sync(0xffffffffu, key != 0u && key == kstar));
-  }
-  if (lane == 0) { s_wgt[warp] = gt_w; s_weq[warp] = eq_w; s_wgt2[warp] = gt_w; s_weq2[warp] = eq_w; }
-  __syncthreads();
-  if (tid == 0) {
-    int g = 0, q = 0;
-    for (int w = 0; w < nw; ++w) { g += s_wgt[w]; q += s_weq[w]; }
-    x_cnt[1] = g; x_cnt[2] = q;
-  }
-  cluster.sync();                                            // barrier 4
-  int eq_before = 0, sel_before = 0;
-  for (int r = 0; r < rank; ++r) {
-    const int g = *cluster.map_shared_rank(&x_cnt[1], r);
-    const int q = *cluster.map_shared_rank(&x_cnt[2], r);
-    sel_before += g + min(max(eq_take - eq_before, 0), q);
-    eq_before += q;
-  }
-  const int cta_first = sel_before;
-  const int eq_cta0 = eq_before;  // equal keys before this CTA
-  for (int w = 0; w < warp; ++w) {
-    sel_before += s_wgt[w] + min(max(eq_take - eq_before, 0), s_weq[w]);
-    eq_before += s_weq[w];
-  }
-  // first walk: token count of this warp's selection (offsets are in shared memory)
-  {
-    int run_eq = eq_before;
-    for (int base = wb; base < we; base += 32) {
-      const int i = base + lane;
-      const uint32_t key = i < we ? key_of(i) : 0u;
-      const bool isgt = key != 0u && key > kstar;
-      const bool iseq = key != 0u && key == kstar;
-      const unsigned beq = __ballot_sync(0xffffffffu, iseq);
-      const bool take = isgt || (iseq && run_eq + __popc(beq & lt) < eq_take);
-      tk_w += take ? so[i + 1] - so[i] : 0;
-      run_eq += __popc(beq);
-    }
-    tk_w = warp_sum_int(tk_w);
-  }
-  __syncthreads();
-  if (lane == 0) s_wgt[warp] = tk_w;
-  __syncthreads();
-  if (tid == 0) {
-    int t = 0;
-    for (int w = 0; w < nw; ++w) t += s_wgt[w];
-    x_cnt[3] = t;
-  }
-  cluster.sync();                                            // barrier 5
-  int tok_before = 0, total_tok = 0;
+  // pass B: ordered compaction, round by round
+  int sel_run = 0, tok_run = 0;   // totals of earlier rounds
+  int total_tok = 0;
+  {  // token total first: the split length depends on it
+    int tk = 0;
+    for (int r = 0; r < n_rounds; ++r) {
+      if (n_rounds > 1) load_round(r, true);
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int t = *cluster.map_shared_rank(&x_cnt[3], r);
-    if (r < rank) tok_before += t;
-    total_tok += t;
+      for (int i = 0; i < kTopkPerLane; ++i) {
+        const int c = r * kTopkRound + wbase + i * 32 + lane;
+        if (picked(c, kr[i])) tk += o1r[i] - o0r[i];
+      }
+    }
+    block_inclusive_scan(tk, scan_sh, &total_tok);
   }
-  const int tok_cta_end = tok_before + x_cnt[3];
-  for (int w = 0; w < warp; ++w) tok_before += s_wgt[w];
   const int n_tok = total_tok + n_st;
   const int split_len = (n_tok + n_splits - 1) / n_splits;
-  // second walk: write the selection, its slot starts, token prefix and split starts
-  {
-    int run_eq = eq_before, pos = sel_before, tok = tok_before;
-    for (int base = wb; base < we; base += 32) {
-      const int i = base + lane;
-      const uint32_t key = i < we ? key_of(i) : 0u;
-      const bool isgt = key != 0u && key > kstar;
-      const bool iseq = key != 0u && key == kstar;
-      const unsigned beq = __ballot_sync(0xffffffffu, iseq);
-      const int eqrank = run_eq + __popc(beq & lt);
-      const bool take = isgt || (iseq && eqrank < eq_take);
-      if (iseq && eqrank == eq_take - 1) I[2] = c_lo + i;   // last selected key equal to kstar
-      const unsigned bs = __ballot_sync(0xffffffffu, take);
-      const int n = take ? so[i + 1] - so[i] : 0;
-      int incl = n;  // inclusive warp scan of token counts
+  for (int r = 0; r < n_rounds; ++r) {
+    if (n_rounds > 1) load_round(r, true);
+    int cnt = 0, tk = 0;
+#pragma unroll
+    for (int i = 0; i < kTopkPerLane; ++i) {
+      const int c = r * kTopkRound + wbase + i * 32 + lane;
+      const bool p = picked(c, kr[i]);
+      cnt += __popc(__ballot_sync(0xffffffffu, p));
+      tk += p ? o1r[i] - o0r[i] : 0;
+    }
+    tk = warp_sum_int(tk);
+    if (lane == 0) { s_w[0][warp] = cnt; s_w[1][warp] = tk; }
+    __syncthreads();
+    int sb = sel_run, tb = tok_run, rs = 0, rt = 0;
+    for (int w = 0; w < NW; ++w) {
+      if (w < warp) { sb += s_w[0][w]; tb += s_w[1][w]; }
+      rs += s_w[0][w]; rt += s_w[1][w];
+    }
+    // write this warp's selection in id order
+#pragma unroll
+    for (int i = 0; i < kTopkPerLane; ++i) {
+      const int c = r * kTopkRound + wbase + i * 32 + lane;
+      const bool p = picked(c, kr[i]);
+      const int o0 = o0r[i];
+      const int n = p ? o1r[i] - o0 : 0;
+      const unsigned bs = __ballot_sync(0xffffffffu, p);
+      int incl = n;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      if (take) {
-        const int si = pos + __popc(bs & lt), st = tok + incl - n;
-        sel[row0 + si] = c_lo + i;
-        sel_slot0[row0 + si] = so[i];
+      if (p) {
+        const int si = sb + __popc(bs & lt), st = tb + incl - n;
+        sel[row0 + si] = c;
+        sel_slot0[row0 + si] = o0;
         pre[si] = st;
+        lst[si - sel_run] = st;
+        lso[si - sel_run] = o0;
         if (split_len > 0)  // splits whose first token falls inside this cluster start at it
           for (int j = (st + split_len - 1) / split_len; j * split_len < st + n && j < n_splits; ++j)
             split[j] = si;
       }
-      pos += __popc(bs);
-      tok += __shfl_sync(0xffffffffu, incl, 31);
-      run_eq += __popc(beq);
+      sb += __popc(bs);
+      tb += __shfl_sync(0xffffffffu, incl, 31);
     }
-  }
-  // gather list of this CTA's selection: tokens expanded CTA-wide from a
-  // shared-memory copy of (token start, slot start) of its selected clusters
-  __syncthreads();
-  {
-    int32_t* lst = reinterpret_cast<int32_t*>(sk);       // keys are no longer read
-    int32_t* lso = so;                                   // nor are the offsets
-    const int cap_list = smem_keys;                      // entries per chunk (+1 end mark)
-    const int my_first = cta_first;
-    int my_sel = 0;
-    {  // clusters this CTA selected = end of its last warp's run - cta_first
-      int g = 0, q = 0;
-      for (int w = 0; w < nw; ++w) { g += s_wgt2[w]; q += s_weq2[w]; }
-      my_sel = g + min(max(eq_take - eq_cta0, 0), q);
-    }
-    for (int j0 = 0; j0 < my_sel; j0 += cap_list) {
-      const int nj = min(cap_list, my_sel - j0);
-      __syncthreads();
-      for (int k = tid; k <= nj; k += nt) {
-        const int si = my_first + j0 + k;
-        lst[k] = (k < nj) ? pre[si] : ((j0 + nj < my_sel) ? pre[si] : tok_cta_end);
-        if (k < nj) lso[k] = sel_slot0[row0 + si];
+    if (tid == 0) lst[rs] = tok_run + rt;
+    __syncthreads();
+    // gather list: the round's tokens expanded CTA-wide
+    for (int qq = tok_run + tid; qq < tok_run + rt; qq += nt) {
+      int lo = 0, hi = rs - 1;  // largest k with lst[k] <= qq
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (lst[mid] <= qq) lo = mid; else hi = mid - 1;
       }
-      __syncthreads();
-      const int q0 = lst[0], q1 = lst[nj];
-      for (int qq = q0 + tid; qq < q1; qq += nt) {
-        int lo = 0, hi = nj - 1;  // largest k with lst[k] <= qq
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (lst[mid] <= qq) lo = mid; else hi = mid - 1;
-        }
-        const int slot = lso[lo] + (qq - lst[lo]);
-        gat[qq] = find_sorted(ss, n_st, slot) >= 0 ? -1 : row_of(slot);
-      }
+      const int slot = lso[lo] + (qq - lst[lo]);
+      gat[qq] = find_sorted(ss, n_st, slot) >= 0 ? -1 : row_of(slot);
     }
+    sel_run += rs;
+    tok_run += rt;
+    __syncthreads();
   }
-  for (int j = rank * nt + tid; j < n_st; j += R * nt) gat[total_tok + j] = row_of(ss[j]);
-  if (rank == 0 && tid == 0) {
-    (void)cta_first;
+  for (int j = tid; j < n_st; j += nt) gat[total_tok + j] = row_of(ss[j]);
+  if (tid == 0) {
     pre[ksel] = total_tok;
     const int j0 = split_len > 0 ? (total_tok + split_len - 1) / split_len : 0;
     for (int j = j0; j <= n_splits; ++j) split[j] = ksel;
-    if (ksel == 0) I[2] = -1;
-    else if (ksel == ncand) I[2] = NC;
-    I[0] = ksel; I[1] = (int32_t)kstar; I[3] = total_tok; I[7] = k_req;
+    I[0] = ksel; I[1] = (int32_t)kstar; I[2] = thr; I[3] = total_tok; I[7] = k_req;
   }
-  cluster.sync();  // keep every CTA's shared memory alive until all remote reads are done
 }
 
 // -------------------------------------------------- K_C attend + estimate
@@ -1131,26 +1085,6 @@ cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <typename... Args>
-cudaError_t launch_topk(dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
-                        Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kTopkCluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, wave_topk_kernel, args...);
-}
-
 }  // namespace
 
 size_t decode_attend_smem(int dtype, int D, int G, int wcap, int echunk, int cap) {
@@ -1199,15 +1133,15 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
                   p.n_score_blocks, sa, status);
     if (e != cudaSuccess) return e;
     mark(1);
-    const size_t topk_smem = ((size_t)p.topk_smem_keys * 2 + 3 + p.topk_smem_keys / 32 + 1 +
-                              3 * (size_t)p.cap) * sizeof(uint32_t);
+    const size_t topk_smem = ((size_t)(p.max_nc + 31) / 32 + 2 * (size_t)p.cap +
+                              2 * (size_t)kTopkRound + 2) * sizeof(int32_t);
     cudaFuncSetAttribute(wave_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)topk_smem);
-    e = launch_topk(dim3(p.U * kTopkCluster), dim3(kTopkThreads), topk_smem, s, pdl, p.geo,
-                    (const uint32_t*)keys, a.offsets, hist, (const int32_t*)aff_cl,
-                    (const int32_t*)aff_start, p.cap, p.topk_clusters, p.topk_fraction,
-                    p.n_splits, p.topk_smem_keys, sel, sel_slot0, seltok, split_first, info,
-                    (const int32_t*)st_slot, a.kp, gather, (int64_t)p.gather_stride, status);
+    e = launch_ex(wave_topk_kernel, dim3(p.U), dim3(kTopkThreads), topk_smem, s, pdl, p.geo,
+                  (const uint32_t*)keys, a.offsets, hist, (const int32_t*)aff_cl,
+                  (const int32_t*)aff_start, p.cap, p.topk_clusters, p.topk_fraction, p.n_splits,
+                  sel, sel_slot0, seltok, split_first, info, (const int32_t*)st_slot, a.kp, gather,
+                  (int64_t)p.gather_stride, status);
     if (e != cudaSuccess) return e;
     mark(2);
     AttendArgs A{gather, aff_cl, aff_start, dv, (int64_t)p.gather_stride, info, scores, keys,

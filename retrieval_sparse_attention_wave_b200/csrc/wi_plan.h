@@ -10,8 +10,7 @@
 namespace wi {
 
 constexpr int kStreamThreads = 256;   // streaming kernels: 8 warps
-constexpr int kTopkThreads = 256;     // per CTA of a top-k cluster
-constexpr int kTopkCluster = 8;       // CTAs per unit in the top-k cluster
+constexpr int kTopkThreads = 512;     // one CTA per unit
 constexpr int kAttendTile = 64;       // tokens per exact-attention tile
 constexpr int kInfoInts = 8;          // per-unit info record (see wi_decode_layout)
 constexpr int kNumSMs = 148;          // B200
@@ -24,7 +23,6 @@ struct DecodePlan {
   int max_nc;
   int seg_len, seg_clusters;  // segment length and clusters per full segment
   int score_chunk, n_score_blocks;
-  int topk_smem_keys;      // keys per top-k CTA (ceil(NC / kTopkCluster)) held in shared memory
   int cap;                 // steady-list capacity per unit (>= 1)
   int sort_pow2;           // shared-memory sort size for the steady list
   int n_splits;            // exact-attention CTAs per unit

@@ -1,6 +1,7 @@
 """Compile libwi.so (the wave-index C ABI and its sm_100a kernels) in-tree.
 
-Usage: python -m retrieval_sparse_attention_wave_b200.build [--force] [-v]
+Usage: python retrieval_sparse_attention_wave_b200/build.py [--force] [-v] [--ptxas-v]
+(run it by path: importing the package loads the library this script builds)
 """
 from __future__ import annotations
 

@@ -16,5 +16,9 @@ def pytest_sessionstart(session):
     # The C-ABI library is a build artefact (not committed); build it in-tree
     # when it is missing or older than its sources.  nvcc cross-compiles for
     # sm_100a without a GPU.
-    from retrieval_sparse_attention_wave_b200 import build as _build
-    _build.build()
+    import importlib.util
+    path = os.path.join(ROOT, "retrieval_sparse_attention_wave_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_wi_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()

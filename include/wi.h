@@ -248,6 +248,29 @@ wi_status wi_decode_host(const void *q_host, const wi_index *idx, const wi_decod
                          float *out_host, float *lse_host, void *ws, size_t ws_bytes,
                          wi_stream_t stream);
 
+/*
+ * wi_decode with no allocation and no caller workspace.  The method has no
+ * counterpart of this call; it exists for callers that cannot allocate device
+ * memory where they decode: code inside a CUDA stream capture (cudaMalloc
+ * cannot be captured), serving loops whose device memory is all owned by a
+ * fixed arena, and C callers embedded in runtimes without a device allocator.
+ *
+ * The workspace is a fixed array of WI_NOALLOC_SCRATCH_MIB MiB in the
+ * library's device memory, held by every GPU that loads the library until
+ * the process exits.  A decode whose workspace (wi_decode_workspace_size)
+ * exceeds it returns WI_ERR_WORKSPACE before touching the GPU.  Each call
+ * clears the part of the scratch that must start at zero, then runs exactly
+ * what wi_decode runs.  All calls share the one array, so calls that overlap
+ * on the GPU (other streams, other host threads) race; serialise them.  The
+ * first call on a device looks up the array's device address, so make it
+ * before any stream capture on that device.  Device-side index checks still
+ * skip bad accesses, but their status bits are not readable through this
+ * entry point.  q, out, lse: as for wi_decode.
+ */
+#define WI_NOALLOC_SCRATCH_MIB 32
+wi_status wi_decode_noalloc(const void *q, const wi_index *idx, const wi_decode_params *p,
+                            float *out, float *lse, wi_stream_t stream);
+
 /* Number of kernels one wi_decode call launches, and its stage names. */
 int32_t wi_decode_stage_count(void);
 const char *wi_decode_stage_name(int32_t i);

@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(_HERE, "libwi.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"{LIB_PATH} is missing; build it with "
-        "`python -m retrieval_sparse_attention_wave_b200.build` (needs nvcc)")
+        "`python retrieval_sparse_attention_wave_b200/build.py` (needs nvcc)")
 _lib = C.CDLL(LIB_PATH)
 
 # ---------------------------------------------------------------- C types
@@ -45,7 +45,7 @@ EXPORTED = [
     "wi_index_clusters", "wi_build_workspace_size", "wi_build_index", "wi_kmeans_assign",
     "wi_decode_workspace_size", "wi_decode_workspace_layout", "wi_decode", "wi_decode_host",
     "wi_decode_stage_count", "wi_decode_stage_name", "wi_read_device_status",
-    "wi_status_string", "wi_last_error_string",
+    "wi_status_string", "wi_last_error_string", "wi_decode_noalloc",
 ]
 
 
@@ -98,6 +98,8 @@ _sig = {
                             C.c_size_t, _P]),
     "wi_decode_host": (C.c_int, [_P, C.POINTER(WiIndex), C.POINTER(WiDecodeParams), _P, _P, _P,
                                  C.c_size_t, _P]),
+    "wi_decode_noalloc": (C.c_int, [_P, C.POINTER(WiIndex), C.POINTER(WiDecodeParams), _P, _P,
+                                    _P]),
     "wi_decode_stage_count": (C.c_int32, []),
     "wi_decode_stage_name": (C.c_char_p, [C.c_int32]),
     "wi_read_device_status": (C.c_int, [_P, _P, C.POINTER(C.c_uint32), C.c_int]),
@@ -404,6 +406,31 @@ def decode_host(q_host: torch.Tensor, index: WaveIndex, params: DecodeParams,
     _check(_lib.wi_decode_host(_ptr(q_host), C.byref(ix), C.byref(p), _ptr(out_host),
                                _ptr(lse_host), _ptr(ws), ws.numel(), _stream_ptr(stream)),
            "wi_decode_host")
+
+
+NOALLOC_SCRATCH_MIB = 32
+
+
+def decode_noalloc(q: torch.Tensor, index: WaveIndex, params: DecodeParams,
+                   out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                   stream=None):
+    """Decode with the library's fixed device scratch instead of a workspace.
+
+    For callers that cannot allocate device memory where they decode (inside a
+    stream capture, under a fixed memory arena, or from a runtime without an
+    allocator).  Pass preallocated out / lse to allocate nothing at all.  Calls
+    share one scratch array: do not overlap them on the GPU.  The first call on
+    a device looks up the scratch address; make it before any stream capture.
+    """
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    ix, p = index.c_struct(), params.c_struct()
+    _check(_lib.wi_decode_noalloc(_ptr(q), C.byref(ix), C.byref(p), _ptr(out), _ptr(lse),
+                                  _stream_ptr(stream)), "wi_decode_noalloc")
+    return out, lse
 
 
 def read_device_status(ws: torch.Tensor, stream=None, clear: bool = True) -> int:

@@ -270,6 +270,20 @@ wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params*
 }
 
 }  // namespace
+
+// Total workspace bytes of a decode call and the length of its leading
+// region that must be zero when a call starts (status word, merge counters,
+// selection histogram).  Host only.
+wi_status decode_workspace_extent(const wi_index* idx, const wi_decode_params* p, size_t* total,
+                                  size_t* zero_prefix) {
+  DecodePlan pl;
+  const wi_status st = make_decode_plan(idx, p, pl);
+  if (st != WI_OK) return st;
+  *total = pl.total;
+  *zero_prefix = pl.off_scores;
+  return WI_OK;
+}
+
 }  // namespace wi
 
 using namespace wi;

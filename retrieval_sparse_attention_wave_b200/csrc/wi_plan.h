@@ -87,6 +87,8 @@ constexpr int kDecodeStages = 3;
 extern const char* const kDecodeStageNames[kDecodeStages];
 
 cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
+wi_status decode_workspace_extent(const wi_index* idx, const wi_decode_params* p, size_t* total,
+                                  size_t* zero_prefix);
 size_t decode_attend_smem(int dtype, int D, int G, int wcap, int echunk, int cap);
 cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s);
 cudaError_t launch_assign_only(const BuildPlan& p, const BuildArgs& a, const float* cent32,

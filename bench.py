@@ -117,12 +117,14 @@ class ClockSampler:
 def algorithmic_bytes(index, params, info: np.ndarray, n_st_per_seq):
     """Bytes the method must move in one decode step (centroids, value sums,
     offsets, retrieved K/V rows, steady K/V rows + invperm, q, out, lse), and
-    the share each launch moves: score reads centroids + offsets + q;
-    attend_estimate reads value sums + offsets + retrieved and steady rows."""
+    the share each launch moves: score_estimate reads centroids + value sums +
+    offsets + q; attend reads the retrieved and steady rows and writes out and
+    lse.  Work partials and the correction's re-read of the retrieved
+    clusters' value sums are not counted (they are not the method's bytes)."""
     e = 2 if index.dtype == torch.bfloat16 else 4
     d = index.head_dim
     H = index.n_kv_heads
-    per_stage = {"score": 0, "topk": 0, "attend_estimate": 0}
+    per_stage = {"score_estimate": 0, "topk": 0, "attend": 0}
     total = 0
     for b, T in enumerate(index.seq_lens):
         NC = index.nc[b]
@@ -135,8 +137,8 @@ def algorithmic_bytes(index, params, info: np.ndarray, n_st_per_seq):
         retr = sel_tok * 2 * d * e
         steady = H * st * (2 * d * e + 4)
         qo = params.n_q_heads * d * e + params.n_q_heads * (d + 1) * 4
-        per_stage["score"] += cent + offs + params.n_q_heads * d * e
-        per_stage["attend_estimate"] += vs + offs + retr + steady + params.n_q_heads * (d + 1) * 4
+        per_stage["score_estimate"] += cent + vs + offs + params.n_q_heads * d * e
+        per_stage["attend"] += retr + steady + params.n_q_heads * (d + 1) * 4
         total += cent + vs + offs + retr + steady + qo
     return total, per_stage
 
@@ -297,7 +299,7 @@ def run_wave(args, rank, world, local_rank):
 
     peaks, peak_kind = measured_peaks()
     hbm = float(peaks["hbm_gbs"])
-    dom = max(("score", "attend_estimate"), key=lambda k: stage_us[k])
+    dom = max(("score_estimate", "attend"), key=lambda k: stage_us[k])
     dom_gbs = stage_bytes[dom] / (stage_us[dom] * 1e-6) / 1e9
     step_gbs = step_bytes / (us_per_step * 1e-6) / 1e9
     tokens = sum(wl.seq_lens)

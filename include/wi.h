@@ -150,14 +150,14 @@ typedef struct wi_decode_layout {
   size_t selected;     /* int32 [Hkv*sum NC_b]: per unit, the retrieved clusters
                           in ascending id, sel_count[u] of them                   */
   size_t unit_info;    /* int32 [B*Hkv][8]: {sel_count, thr_key, thr_idx,
-                          sel_tokens, steady, n_affected, dense, k}              */
+                          sel_tokens, steady, n_affected, dense, candidates}     */
   size_t gather;       /* int32 [B*Hkv][gather_stride]: per unit, the pool row of
                           each exactly attended token (retrieved clusters in id
                           order, -1 for their steady members, then the steady
                           slots); sel_tokens + steady entries are valid          */
   int64_t gather_stride;
   int32_t n_splits;    /* exact-attention splits per unit                        */
-  int32_t n_est_chunks;/* estimation chunks per unit                             */
+  int32_t n_est_chunks;/* score + estimation chunks (CTAs) per unit             */
 } wi_decode_layout;
 
 /* ------------------------------------------------------------------ sizes */

@@ -446,7 +446,7 @@ def read_device_status(ws: torch.Tensor, stream=None, clear: bool = True) -> int
 
 def unit_info(ws: torch.Tensor, layout: WiDecodeLayout, n_units: int) -> torch.Tensor:
     """Per-unit record {sel_count, thr_key, thr_idx, sel_tokens, steady,
-    n_affected, dense, k} from a decode workspace (int32 [U][8])."""
+    n_affected, dense, candidates} from a decode workspace (int32 [U][8])."""
     return ws[layout.unit_info:layout.unit_info + n_units * 32].view(torch.int32).view(n_units, 8)
 
 

@@ -111,7 +111,7 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   pl.scale = 1.0f / std::sqrt((float)ix->head_dim);
 
   int max_nc = 0, cap = 1;
-  int64_t max_tok = 1;
+  int64_t max_tok = 1, max_k = 0;
   for (int b = 0; b < ix->batch; ++b) {
     const int T = ix->seq_lens[b];
     const int nc = pl.geo.NC(b);
@@ -120,6 +120,7 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
     int64_t k = p->topk_clusters >= 0 ? p->topk_clusters
                                       : (int64_t)std::ceil(p->topk_fraction * (double)nc);
     k = std::min<int64_t>(k, nc);
+    max_k = std::max<int64_t>(max_k, k);
     if (nst >= T) {
       max_tok = std::max<int64_t>(max_tok, T);
     } else {
@@ -135,24 +136,27 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
 
   pl.seg_len = ix->seg_len;
   pl.seg_clusters = ix->seg_len / ix->cluster_size;
-  // score: one CTA per 64 KB of centroid rows
-  pl.score_chunk = 65536 / (pl.D * esize(ix->dtype));
+  // score + estimate: one CTA per 32 KB of centroid rows (and their value sums)
+  pl.score_chunk = kScoreChunkBytes / (pl.D * esize(ix->dtype));
   pl.n_score_blocks = (int)cdiv(max_nc, pl.score_chunk);
-  // top-k shared memory: exclusion bitmask, steady lists, one round's list
-  if ((size_t)(max_nc + 31) / 32 * 4 + 8 * (size_t)cap + 8 * 8192 + 8 > 200 * 1024)
-    return WI_ERR_UNSUPPORTED;
+  if (decode_score_smem(pl.dtype, pl.D, pl.sort_pow2, cap) > 200 * 1024) return WI_ERR_UNSUPPORTED;
+  // top-k shared memory: exclusion bitmask, steady lists, one round's lists,
+  // and the block-table row when it fits
+  pl.bt_cap = std::min<int>(ix->max_pages, kTopkBtCap);
+  if (decode_topk_smem(max_nc, cap, 0) + 24 * 1024 > 200 * 1024) return WI_ERR_UNSUPPORTED;
+  while (pl.bt_cap > 0 && decode_topk_smem(max_nc, cap, pl.bt_cap) + 24 * 1024 > 200 * 1024)
+    pl.bt_cap >>= 1;
   // exact attention: about two 16 KB tiles of rows per CTA
   const int row_bytes = pl.D * esize(ix->dtype);
   const int tile_rows = 16384 / row_bytes;
   int ns = (int)cdiv(max_tok, 2 * tile_rows);
   pl.n_splits = std::max(1, std::min(ns, 4096));
-  // estimation: 512 clusters per CTA (4 prefetched tiles + the rest streamed)
-  pl.echunk = 512;
-  pl.n_est = (int)cdiv(max_nc, pl.echunk);
-  pl.n_parts = pl.n_splits + pl.n_est;
-  pl.wcap = std::max(pl.echunk, pl.n_parts);
-  if (decode_attend_smem(pl.dtype, pl.D, G, pl.wcap, pl.echunk, cap) > 200 * 1024)
-    return WI_ERR_UNSUPPORTED;
+  // estimation correction: retrieved + affected clusters, kNegRows per CTA
+  pl.n_neg = std::max<int>(1, (int)cdiv(max_k + cap, kNegRows));
+  pl.n_fold = std::max<int>(1, (int)cdiv(pl.n_score_blocks, kFold));
+  pl.n_parts = pl.n_splits + pl.n_neg + pl.n_fold;
+  pl.wcap = std::max(kNegRows, pl.n_parts);
+  if (decode_attend_smem(pl.dtype, pl.D, G, pl.wcap) > 200 * 1024) return WI_ERR_UNSUPPORTED;
 
   const int64_t ncl = (int64_t)pl.geo.cl_base[ix->batch] * ix->n_kv_heads;
   size_t o = 0;
@@ -163,9 +167,7 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   pl.off_scores = take((size_t)ncl * G * 4);
   pl.off_keys = take((size_t)ncl * 4);
   pl.off_sel = take((size_t)ncl * 4);
-  pl.off_sel_slot0 = take((size_t)ncl * 4);
   pl.off_seltok = take((size_t)(ncl + pl.U) * 4);
-  pl.off_split = take((size_t)pl.U * (pl.n_splits + 1) * 4);
   pl.off_info = take((size_t)pl.U * kInfoInts * 4);
   pl.off_st_slot = take((size_t)pl.U * cap * 4);
   pl.off_st_cl = take((size_t)pl.U * cap * 4);
@@ -177,6 +179,8 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   pl.gather_stride = tmax + cap;   // retrieved slots (steady members as -1) + steady slots
   pl.off_gather = take((size_t)pl.U * pl.gather_stride * 4);
   pl.off_dv = take((size_t)pl.U * cap * pl.D * 4);
+  pl.off_est = take((size_t)pl.U * pl.n_score_blocks * G * (pl.D + 4) * 4);
+  pl.off_nonc = take((size_t)pl.U * (cap + 1) * 4);
   const size_t nq = (size_t)ix->batch * p->n_q_heads;
   pl.off_q = take(nq * pl.D * esize(ix->dtype));
   pl.off_out = take(nq * pl.D * 4);
@@ -406,7 +410,7 @@ wi_status wi_decode_workspace_layout(const wi_index* idx, const wi_decode_params
   layout->gather = pl.off_gather;
   layout->gather_stride = pl.gather_stride;
   layout->n_splits = pl.n_splits;
-  layout->n_est_chunks = pl.n_est;
+  layout->n_est_chunks = pl.n_score_blocks;
   return WI_OK;
 }
 

@@ -149,6 +149,30 @@ def steady_count(T, n_sink, window):
     return ns + (T - ws)
 
 
+def rank_seed(cfg: int, rank: int):
+    """Seed of rank r's synthetic workload: rank 0 uses the workload's own
+    seed, every other rank a distinct one, so the ranks' replicas differ."""
+    return None if rank == 0 else 1000 * rank + cfg
+
+
+def max_over_ranks(x: float, device) -> float:
+    """The largest x over all ranks (a MAX all-reduce); x itself alone."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(ms_total_max: float, steps: int, world: int):
+    """(device time per step on the slowest rank in us, whole-job value): with
+    every rank decoding its own replica layer per step, the job advances
+    `world` layer steps per step time, so the time per layer step is the
+    slowest rank's step time divided by the number of ranks."""
+    us_per_step = ms_total_max * 1e3 / steps
+    return us_per_step, us_per_step / world
+
+
 def clone_index(wx):
     import copy
     c = copy.copy(wx)
@@ -166,7 +190,7 @@ def run_wave(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = WI.config(args.config, device=dev, seed=None if rank == 0 else 1000 * rank + args.config)
+    wl = WI.config(args.config, device=dev, seed=rank_seed(args.config, rank))
     # paged input cache, contiguous block table
     bt, n_pages = WI.make_block_table(wl.seq_lens, wl.page_size,
                                       shuffle_seed=(5 if args.config == 5 else None))
@@ -255,12 +279,8 @@ def run_wave(args, rank, world, local_rank):
     if dist:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    us_per_step = ms * 1e3 / args.steps
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    us_per_step, job_us = job_value(ms, args.steps, world)
 
     # per-stage device time (ungraphed launches, events on the launching stream)
     nst = W.lib().wi_decode_stage_count()
@@ -307,7 +327,7 @@ def run_wave(args, rank, world, local_rank):
         * wl.head_dim * wl.iters
     result = {
         "metric": METRIC,
-        "value": us_per_step / world,
+        "value": job_us,
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,

@@ -77,6 +77,8 @@ typedef enum wi_dtype { WI_F32 = 0, WI_BF16 = 1 } wi_dtype;
 #define WI_DEV_BAD_CLUSTER 0x4u  /* offsets not monotone or cluster out of range */
 #define WI_DEV_BAD_HIST    0x8u  /* stale selection histogram (workspace reused
                                     after a failed call); recomputed, result valid */
+#define WI_DEV_TIMEOUT     0x10u /* a bounded wait for an asynchronous copy gave
+                                    up; the call's results are not valid        */
 
 /*
  * Paged KV cache in original token order (the build input).
@@ -147,17 +149,13 @@ typedef struct wi_decode_layout {
   size_t scores;       /* float [Hkv*sum NC_b][G]: q_h . centroid / sqrt(d)      */
   size_t keys;         /* uint32 [Hkv*sum NC_b]: order-preserving key of the
                           group-max score; 0 = not a candidate                   */
-  size_t selected;     /* int32 [Hkv*sum NC_b]: per unit, the retrieved clusters
-                          in ascending id, sel_count[u] of them                   */
+  size_t selected;     /* int32 [Hkv*sum NC_b]: per unit (at its centroid row), the
+                          retrieved clusters in no particular order, sel_count
+                          of them                                                 */
   size_t unit_info;    /* int32 [B*Hkv][8]: {sel_count, thr_key, thr_idx,
                           sel_tokens, steady, n_affected, dense, candidates}     */
-  size_t gather;       /* int32 [B*Hkv][gather_stride]: per unit, the pool row of
-                          each exactly attended token (retrieved clusters in id
-                          order, -1 for their steady members, then the steady
-                          slots); sel_tokens + steady entries are valid          */
-  int64_t gather_stride;
-  int32_t n_splits;    /* exact-attention splits per unit                        */
-  int32_t n_est_chunks;/* score + estimation chunks (CTAs) per unit             */
+  int32_t n_attend_ctas; /* exact-attention CTAs per unit                         */
+  int32_t n_score_ctas;  /* score + estimation chunks (CTAs) per unit             */
 } wi_decode_layout;
 
 /* ------------------------------------------------------------------ sizes */

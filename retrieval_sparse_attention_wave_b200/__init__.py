@@ -76,8 +76,7 @@ class WiDecodeParams(C.Structure):
 class WiDecodeLayout(C.Structure):
     _fields_ = [("total_bytes", C.c_size_t), ("status", C.c_size_t), ("scores", C.c_size_t),
                 ("keys", C.c_size_t), ("selected", C.c_size_t), ("unit_info", C.c_size_t),
-                ("gather", C.c_size_t), ("gather_stride", C.c_int64),
-                ("n_splits", C.c_int32), ("n_est_chunks", C.c_int32)]
+                ("n_attend_ctas", C.c_int32), ("n_score_ctas", C.c_int32)]
 
 
 _P = C.c_void_p
@@ -452,14 +451,10 @@ def unit_info(ws: torch.Tensor, layout: WiDecodeLayout, n_units: int) -> torch.T
 
 def selected_clusters(ws: torch.Tensor, layout: WiDecodeLayout, index: WaveIndex,
                       b: int, h: int, count: int) -> torch.Tensor:
+    """The retrieved clusters of unit (b, h), ascending (the workspace holds
+    them in no particular order)."""
     row = index.cl_row(b, h)
-    return ws[layout.selected:].view(torch.int32)[row:row + count]
-
-
-def gather_rows(ws: torch.Tensor, layout: WiDecodeLayout, u: int, count: int) -> torch.Tensor:
-    """Pool row indices of unit u's exactly attended tokens (-1 = skipped)."""
-    base = u * layout.gather_stride
-    return ws[layout.gather:].view(torch.int32)[base:base + count]
+    return torch.sort(ws[layout.selected:].view(torch.int32)[row:row + count]).values
 
 
 def centroid_scores(ws: torch.Tensor, layout: WiDecodeLayout, index: WaveIndex, G: int,

@@ -111,22 +111,13 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   pl.scale = 1.0f / std::sqrt((float)ix->head_dim);
 
   int max_nc = 0, cap = 1;
-  int64_t max_tok = 1, max_k = 0;
   for (int b = 0; b < ix->batch; ++b) {
     const int T = ix->seq_lens[b];
-    const int nc = pl.geo.NC(b);
-    max_nc = std::max(max_nc, nc);
+    max_nc = std::max(max_nc, pl.geo.NC(b));
     const int64_t nst = n_steady(T, p->n_sink, p->window);
-    int64_t k = p->topk_clusters >= 0 ? p->topk_clusters
-                                      : (int64_t)std::ceil(p->topk_fraction * (double)nc);
-    k = std::min<int64_t>(k, nc);
-    max_k = std::max<int64_t>(max_k, k);
-    if (nst >= T) {
-      max_tok = std::max<int64_t>(max_tok, T);
-    } else {
+    if (nst < T) {  // not attended densely: its steady list is kept
       if (nst > WI_MAX_STEADY) return WI_ERR_UNSUPPORTED;
       cap = std::max<int>(cap, (int)nst);
-      max_tok = std::max<int64_t>(max_tok, std::min<int64_t>(T, k * ix->cluster_size + nst));
     }
   }
   pl.max_nc = max_nc;
@@ -139,45 +130,38 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   // score + estimate: one CTA per 32 KB of centroid rows (and their value sums)
   pl.score_chunk = kScoreChunkBytes / (pl.D * esize(ix->dtype));
   pl.n_score_blocks = (int)cdiv(max_nc, pl.score_chunk);
-  if (decode_score_smem(pl.dtype, pl.D, pl.sort_pow2, cap) > 200 * 1024) return WI_ERR_UNSUPPORTED;
-  // top-k shared memory: exclusion bitmask, steady lists, one round's lists,
-  // and the block-table row when it fits
-  pl.bt_cap = std::min<int>(ix->max_pages, kTopkBtCap);
-  if (decode_topk_smem(max_nc, cap, 0) + 24 * 1024 > 200 * 1024) return WI_ERR_UNSUPPORTED;
-  while (pl.bt_cap > 0 && decode_topk_smem(max_nc, cap, pl.bt_cap) + 24 * 1024 > 200 * 1024)
-    pl.bt_cap >>= 1;
-  // exact attention: about two 16 KB tiles of rows per CTA
+  if (decode_score_smem(pl.dtype, pl.D, G, pl.sort_pow2, cap) > 200 * 1024) return WI_ERR_UNSUPPORTED;
+  // top-k shared memory: exclusion bitmask and the non-candidate list
+  if (decode_topk_smem(max_nc, cap) + 24 * 1024 > 200 * 1024) return WI_ERR_UNSUPPORTED;
+  // attend: range CTAs of kRangeClusters ids, steady CTAs of two 16 KB tiles
+  // of rows
   const int row_bytes = pl.D * esize(ix->dtype);
   const int tile_rows = 16384 / row_bytes;
-  int ns = (int)cdiv(max_tok, 2 * tile_rows);
-  pl.n_splits = std::max(1, std::min(ns, 4096));
-  // estimation correction: retrieved + affected clusters, kNegRows per CTA
-  pl.n_neg = std::max<int>(1, (int)cdiv(max_k + cap, kNegRows));
+  pl.n_rng = std::max<int>(1, (int)cdiv(max_nc, kRangeClusters));
+  pl.n_sc = std::max<int>(1, (int)cdiv(cap, 2 * tile_rows));
   pl.n_fold = std::max<int>(1, (int)cdiv(pl.n_score_blocks, kFold));
-  pl.n_parts = pl.n_splits + pl.n_neg + pl.n_fold;
-  pl.wcap = std::max(kNegRows, pl.n_parts);
-  if (decode_attend_smem(pl.dtype, pl.D, G, pl.wcap) > 200 * 1024) return WI_ERR_UNSUPPORTED;
+  pl.n_parts = pl.n_rng + pl.n_sc + pl.n_fold;
+  if (decode_attend_smem(pl.dtype, pl.D, G, pl.n_parts) + 24 * 1024 > 200 * 1024)
+    return WI_ERR_UNSUPPORTED;
 
   const int64_t ncl = (int64_t)pl.geo.cl_base[ix->batch] * ix->n_kv_heads;
+  pl.ncl = ncl;
   size_t o = 0;
   auto take = [&](size_t bytes) { const size_t r = o; o = align_up(o + bytes, 256); return r; };
   pl.off_status = take(256);
   pl.off_counters = take((size_t)pl.U * 4);
-  pl.off_hist = take((size_t)pl.U * 2048 * 4);   // zeroed after use by the top-k kernel
+  pl.off_hist = take((size_t)pl.U * 2048 * 4);      // zeroed after use by the top-k kernel
+  pl.off_aff_of = take((size_t)pl.U * max_nc * 4);  // reset after use by the attend kernel
   pl.off_scores = take((size_t)ncl * G * 4);
   pl.off_keys = take((size_t)ncl * 4);
   pl.off_sel = take((size_t)ncl * 4);
-  pl.off_seltok = take((size_t)(ncl + pl.U) * 4);
+  pl.off_sel_n = take((size_t)pl.U * 4);
   pl.off_info = take((size_t)pl.U * kInfoInts * 4);
   pl.off_st_slot = take((size_t)pl.U * cap * 4);
   pl.off_st_cl = take((size_t)pl.U * cap * 4);
   pl.off_aff_cl = take((size_t)pl.U * cap * 4);
   pl.off_aff_start = take((size_t)pl.U * (cap + 1) * 4);
   pl.off_partials = take((size_t)pl.U * pl.n_parts * G * (pl.D + 4) * 4);
-  int64_t tmax = 0;
-  for (int b = 0; b < ix->batch; ++b) tmax = std::max<int64_t>(tmax, ix->seq_lens[b]);
-  pl.gather_stride = tmax + cap;   // retrieved slots (steady members as -1) + steady slots
-  pl.off_gather = take((size_t)pl.U * pl.gather_stride * 4);
   pl.off_dv = take((size_t)pl.U * cap * pl.D * 4);
   pl.off_est = take((size_t)pl.U * pl.n_score_blocks * G * (pl.D + 4) * 4);
   pl.off_nonc = take((size_t)pl.U * (cap + 1) * 4);
@@ -407,10 +391,8 @@ wi_status wi_decode_workspace_layout(const wi_index* idx, const wi_decode_params
   layout->keys = pl.off_keys;
   layout->selected = pl.off_sel;
   layout->unit_info = pl.off_info;
-  layout->gather = pl.off_gather;
-  layout->gather_stride = pl.gather_stride;
-  layout->n_splits = pl.n_splits;
-  layout->n_est_chunks = pl.n_score_blocks;
+  layout->n_attend_ctas = pl.n_rng + pl.n_sc;
+  layout->n_score_ctas = pl.n_score_blocks;
   return WI_OK;
 }
 

@@ -30,6 +30,11 @@
 #include <climits>
 #include <algorithm>
 #include <cmath>
+#include <mutex>
+#include <type_traits>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
 #include "wi_common.cuh"
 #include "wi_plan.h"
@@ -49,6 +54,38 @@ struct RowShape {
   static constexpr int TILE = 16384 / ROWB;     // rows per 16 KB shared-memory tile
 };
 
+// G consecutive floats of shared memory (16-byte aligned rows when G >= 4)
+template <int G>
+__device__ __forceinline__ void load_row(const float* p, float (&v)[G]) {
+  if constexpr (G % 4 == 0) {
+#pragma unroll
+    for (int g = 0; g < G; g += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(p + g);
+      v[g] = x.x; v[g + 1] = x.y; v[g + 2] = x.z; v[g + 3] = x.w;
+    }
+  } else if constexpr (G == 2) {
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    v[0] = x.x; v[1] = x.y;
+  } else {
+#pragma unroll
+    for (int g = 0; g < G; ++g) v[g] = p[g];
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void store_row(float* p, const float (&v)[G]) {
+  if constexpr (G % 4 == 0) {
+#pragma unroll
+    for (int g = 0; g < G; g += 4)
+      *reinterpret_cast<float4*>(p + g) = make_float4(v[g], v[g + 1], v[g + 2], v[g + 3]);
+  } else if constexpr (G == 2) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  } else {
+#pragma unroll
+    for (int g = 0; g < G; ++g) p[g] = v[g];
+  }
+}
+
 template <typename T, int D, int G>
 __device__ __forceinline__ void load_q(const T* q, int n_q_heads, int b, int h, int sub, float scale,
                                        float (&qv)[G][Elem<T>::kPerVec]) {
@@ -63,16 +100,6 @@ __device__ __forceinline__ void load_q(const T* q, int n_q_heads, int b, int h, 
   }
 }
 
-// Binary search in a sorted shared-memory array: index of x or -1.
-__device__ __forceinline__ int find_sorted(const int32_t* a, int n, int x) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (a[mid] < x) lo = mid + 1; else hi = mid;
-  }
-  return (lo < n && a[lo] == x) ? lo : -1;
-}
-
 struct SteadyArgs {
   const int32_t* invperm;
   const int32_t* labels;
@@ -80,7 +107,9 @@ struct SteadyArgs {
   Pool vp;
   int n_sink, window, cap, sort_pow2;
   int32_t *st_slot, *st_cl, *aff_cl, *aff_start, *nonc, *info;
-  float* dv;  // [U][cap][D] fp32: sum of the steady members' values per affected cluster
+  float* dv;       // [U][cap][D] fp32: sum of the steady members' values per affected cluster
+  int32_t* aff_of; // [U][max_nc]: +(j+1) for affected cluster j, -(j+1) if not a candidate
+  int max_nc;
 };
 
 constexpr int kSteadyRank = 256;   // steady lists up to this size are rank-sorted in one step
@@ -204,7 +233,9 @@ __device__ void steady_role(const Geo& geo, int u, const SteadyArgs& a, uint32_t
     if (i < n_aff) {
       const int c = s_acl[i];
       const int full = __ldg(off + c + 1) - __ldg(off + c);
-      if (full - (s_ast[i + 1] - s_ast[i]) <= 0) nonc[1 + atomicAdd(&s_nnc, 1)] = c;
+      const bool none_left = full - (s_ast[i + 1] - s_ast[i]) <= 0;
+      if (none_left) nonc[1 + atomicAdd(&s_nnc, 1)] = c;
+      a.aff_of[(int64_t)u * a.max_nc + c] = none_left ? -(i + 1) : i + 1;
     }
     if (staged) s_ro[i] = pool_row(a.vp, geo.hkv, D, b, h, (int)(srt[i] >> 32), status);
   }
@@ -301,169 +332,542 @@ __device__ __forceinline__ void empty_part(float* part, int G, int PS) {
   for (int i = threadIdx.x; i < G * PS; i += blockDim.x) part[i] = (i % PS) == 0 ? -INFINITY : 0.f;
 }
 
+// Shared-memory layout of a K_A stream CTA (bytes).
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kStreamThreads, G >= 8 ? 2 : 3)
+struct ScoreSmem {
+  static constexpr int ROWB = D * (int)sizeof(T);
+  static constexpr int CROWS = kScoreChunkBytes / ROWB;          // clusters per chunk
+  static constexpr int TR = 16384 / ROWB;                         // rows per 16 KB tile
+  static constexpr size_t kRing = 4 * 16384;                      // 4 tiles in flight
+  static constexpr size_t kRed = (size_t)(kStreamThreads / 32) * G * D * 4;
+  static constexpr size_t kHist = (size_t)kHistBins / 2 * 4;
+  static constexpr size_t kOff = (size_t)2 * (CROWS + 4) * 4;    // offsets, double-buffered
+  static constexpr size_t kW = (size_t)CROWS * G * 4;
+  static constexpr size_t kQ = (size_t)2 * G * D * sizeof(T);    // q, double-buffered
+  static constexpr size_t oRed = kRing, oHist = oRed + kRed, oOff = oHist + kHist,
+                          oW = oOff + kOff, oQ = oW + kW, kTotal = oQ + kQ;
+};
+
+// K_A.  blockIdx.x < U: the steady role of unit blockIdx.x.  The other
+// n_stream CTAs are persistent: CTA s takes chunks [s n / n_stream,
+// (s+1) n / n_stream) of the n = U * n_chunks chunks (unit-major) and streams
+// each chunk's two centroid tiles and two value-sum tiles through a ring of
+// four 16 KB slots (one cp.async group per tile; a slot is refilled with the
+// tile four places ahead as soon as it is consumed, so the next chunk loads
+// while this one computes).  The chunk's offsets and q ride in the group of
+// its first tile.
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kStreamThreads, G >= 8 ? 1 : 2)
 wave_score_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const T* __restrict__ cent,
                   const T* __restrict__ vsum, const int32_t* __restrict__ offsets,
                   float* __restrict__ scores, uint32_t* __restrict__ keys,
                   int32_t* __restrict__ hist_g, float* __restrict__ est_parts, float scale,
-                  int n_score_blocks, const SteadyArgs sa, uint32_t* status) {
+                  int n_chunks, int n_stream, const SteadyArgs sa, uint32_t* status) {
   using RS = RowShape<T, D>;
+  using SM = ScoreSmem<T, D, G>;
   constexpr int EPL = RS::EPL, LPR = RS::LPR, RPW = RS::RPW, TR = RS::TILE;
   constexpr int NW = kStreamThreads / 32;
-  constexpr int CROWS = kScoreChunkBytes / RS::ROWB;  // clusters per CTA
-  constexpr int NT = CROWS / TR;                      // 16 KB tiles per matrix
+  constexpr int CROWS = SM::CROWS;
   constexpr int PS = Part<D>::kStride;
+  constexpr int ITR = TR / (NW * RPW);
   static_assert(G <= LPR && G <= NW, "group larger than lanes per row or warps");
-  static_assert(NT == 2, "two tiles per matrix");
+  static_assert(CROWS == 2 * TR, "two tiles per matrix per chunk");
   extern __shared__ __align__(16) unsigned char sh_dyn[];
   __shared__ float s_m[G], s_l[G];
   pdl_launch_dependents();
-  const int u = blockIdx.y;
-  if (blockIdx.x == n_score_blocks) {
-    steady_role<T, D>(geo, u, sa, status, sh_dyn);
+  const int U = geo.batch * geo.hkv;
+  if ((int)blockIdx.x < U) {
+    steady_role<T, D>(geo, blockIdx.x, sa, status, sh_dyn);
     return;
   }
-  const int b = u / geo.hkv, h = u - b * geo.hkv;
-  const int NC = geo.NC(b);
-  const int c0 = blockIdx.x * CROWS;
-  float* part = est_parts + ((int64_t)u * n_score_blocks + blockIdx.x) * G * PS;
-  const int tid = threadIdx.x;
-  if (c0 >= NC) {  // past this sequence's clusters: an empty part
-    empty_part(part, G, PS);
-    return;
-  }
-  const int nrows = min(NC - c0, CROWS);
-  // shared: centroid rows [CROWS][D] | value-sum rows [CROWS][D] | histogram,
-  //         two 16-bit counts per word [kHistBins/2] | offsets [CROWS+1 (+3)]
-  //         | scores, then weights [CROWS][G]
-  T* crow = reinterpret_cast<T*>(sh_dyn);
-  T* vrow = crow + CROWS * D;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(vrow + CROWS * D);
-  int* s_off = reinterpret_cast<int*>(hist + kHistBins / 2);
-  float* s_w = reinterpret_cast<float*>(s_off + CROWS + 4);
-  const int lane = tid & 31, warp = tid >> 5;
+  const int sidx = blockIdx.x - U;
+  const int n_tot = U * n_chunks;
+  const int k0 = (int)((int64_t)sidx * n_tot / n_stream);
+  const int k1 = (int)((int64_t)(sidx + 1) * n_tot / n_stream);
+  const int nk = k1 - k0;
+  T* ring = reinterpret_cast<T*>(sh_dyn);
+  float* s_red = reinterpret_cast<float*>(sh_dyn + SM::oRed);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sh_dyn + SM::oHist);
+  int* s_offb = reinterpret_cast<int*>(sh_dyn + SM::oOff);
+  float* s_w = reinterpret_cast<float*>(sh_dyn + SM::oW);
+  T* s_q = reinterpret_cast<T*>(sh_dyn + SM::oQ);
+  __shared__ __align__(8) uint64_t s_bar[4];         // one per ring slot
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int sub = lane % LPR, rsub = lane / LPR;
-  const int64_t row0 = geo.cl_row(b, h);
-#pragma unroll
-  for (int t = 0; t < 2 * NT; ++t) {
-    const T* src = (t < NT ? cent : vsum) + (row0 + c0) * D;
-    T* dst = t < NT ? crow : vrow;
-    const int r0 = (t % NT) * TR, nr = min(TR, nrows - r0);
-    for (int i = tid; i < nr * LPR; i += blockDim.x)
-      cp_async16(dst + (r0 * LPR + i) * EPL, src + (r0 * LPR + i) * EPL);
-    cp_async_commit();
-  }
-  const int32_t* off = offsets + geo.off_row(b, h) + c0;
-  for (int i = tid; i <= nrows; i += blockDim.x) s_off[i] = __ldg(off + i);
-  for (int i = tid; i < kHistBins / 2; i += blockDim.x) hist[i] = 0u;
-  float qv[G][EPL];
-  load_q<T, D, G>(q, n_q_heads, b, h, sub, scale, qv);
   const int j = sub / (LPR / G);
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    cp_async_wait_dyn(2 * NT - 1 - t);  // centroid tile t has landed
-    __syncthreads();
-    const int r1 = min(nrows, (t + 1) * TR);
-    for (int rb = t * TR + warp * RPW; rb < r1; rb += NW * RPW) {
-      const int r = rb + rsub;
-      const bool ok = r < r1;
-      float x[EPL];
-      if (ok) {
-        Elem<T>::unpack(*reinterpret_cast<const uint4*>(crow + r * D + sub * EPL), x);
-      } else {
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) x[e] = 0.f;
-      }
-      float acc[G];
-      dot_g<G, EPL>(qv, x, acc);
-      group_reduce_multi<G, LPR>(acc, lane);
-      float m = acc[0];
-#pragma unroll
-      for (int o = LPR / 2; o >= LPR / G; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (ok) {
-        if (sub % (LPR / G) == 0) {
-          scores[(row0 + c0 + r) * G + j] = acc[0];
-          s_w[r * G + j] = acc[0];
-        }
-        if (sub == 0) {
-          const uint32_t key = (s_off[r + 1] - s_off[r]) > 0 ? ordered_key(m) : 0u;
-          keys[row0 + c0 + r] = key;
-          if (key) atomicAdd(&hist[key >> (kHistShift + 1)], 1u << (16 * ((key >> kHistShift) & 1u)));
-        }
+  struct Chunk { int u, b, h, c0, nrows; int64_t row0; };
+  auto chunk = [&](int k) -> Chunk {
+    Chunk c;
+    c.u = k / n_chunks;
+    c.b = c.u / geo.hkv;
+    c.h = c.u - c.b * geo.hkv;
+    c.c0 = (k - c.u * n_chunks) * CROWS;
+    c.nrows = max(0, min(geo.NC(c.b) - c.c0, CROWS));
+    c.row0 = geo.cl_row(c.b, c.h);
+    return c;
+  };
+  // thread 0: tile i of this CTA (chunk i / 4; centroid rows 0..TR-1,
+  // TR..2TR-1, then value-sum rows likewise) into ring slot i % 4 as one bulk
+  // copy completing on the slot's barrier (a plain arrive for an empty tile)
+  auto issue_tile = [&](int i) {
+    if (i >= 4 * nk) return;
+    const int part = i & 3;
+    const Chunk c = chunk(k0 + (i >> 2));
+    const int r0 = (part & 1) * TR, nr = min(TR, c.nrows - r0);
+    uint64_t* bar = &s_bar[i & 3];
+    if (nr <= 0) { mbar_arrive(bar); return; }
+    const T* src = (part < 2 ? cent : vsum) + (c.row0 + c.c0 + r0) * D;
+    fence_proxy_async();
+    mbar_arrive_expect(bar, (uint32_t)(nr * SM::ROWB));
+    bulk_load(ring + (size_t)(i & 3) * TR * D, src, (uint32_t)(nr * SM::ROWB), bar);
+  };
+  // all threads: chunk kk's offsets and q (double-buffered), one cp.async group
+  auto issue_meta = [&](int kk) {
+    if (kk < nk) {
+      const Chunk c = chunk(k0 + kk);
+      if (c.nrows > 0) {
+        int* so = s_offb + (kk & 1) * (CROWS + 4);
+        const int32_t* off = offsets + geo.off_row(c.b, c.h) + c.c0;
+        for (int x = tid; x <= c.nrows; x += blockDim.x) cp_async4(so + x, off + x);
+        T* sq = s_q + (size_t)(kk & 1) * G * D;
+        const T* qs = q + ((int64_t)c.b * n_q_heads + (int64_t)c.h * G) * D;
+        for (int x = tid; x < G * LPR; x += blockDim.x) cp_async16(sq + x * EPL, qs + x * EPL);
       }
     }
+    cp_async_commit();
+  };
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mbar_init(&s_bar[i], 1);
+    mbar_init_fence();
   }
+  for (int i = tid; i < kHistBins / 2; i += blockDim.x) hist[i] = 0u;
   __syncthreads();
-  {
-    int* hg = hist_g + (int64_t)u * kHistBins;
-    for (int i = tid; i < kHistBins / 2; i += blockDim.x) {
-      const uint32_t w = hist[i];
-      if (w & 0xffffu) atomicAdd(hg + 2 * i, (int)(w & 0xffffu));
-      if (w >> 16) atomicAdd(hg + 2 * i + 1, (int)(w >> 16));
-    }
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) issue_tile(i);
   }
-  // the chunk's max, weights and denominator per head (warp g: head g)
-  if (warp < G) {
-    float m = -INFINITY;
-    for (int r = lane; r < nrows; r += 32) m = fmaxf(m, s_w[r * G + warp]);
-    m = warp_max(m);
-    float l = 0.f;
-    for (int r = lane; r < nrows; r += 32) {
-      const int cnt = s_off[r + 1] - s_off[r];
-      const float w = cnt > 0 ? __expf(s_w[r * G + warp] - m) : 0.f;
-      s_w[r * G + warp] = w;
-      l += (float)cnt * w;
-    }
-    l = warp_sum(l);
-    if (lane == 0) { s_m[warp] = m; s_l[warp] = l; }
-  }
-  __syncthreads();
-  float acc[G][EPL];
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[g][e] = 0.f;
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    cp_async_wait_dyn(NT - 1 - t);  // value-sum tile t has landed
+  issue_meta(0);
+  issue_meta(1);
+
+  for (int kk = 0; kk < nk; ++kk) {
+    const Chunk c = chunk(k0 + kk);
+    float* part = est_parts + ((int64_t)(k0 + kk)) * G * PS;   // [u][chunk] = k
+    const int* s_off = s_offb + (kk & 1) * (CROWS + 4);
+    const uint32_t par = kk & 1;                                 // each slot: one phase per chunk
+    cp_async_wait<1>();  // this chunk's offsets and q (the next chunk's may be in flight)
     __syncthreads();
-    const int r1 = min(nrows, (t + 1) * TR);
-    for (int rb = t * TR + warp * RPW; rb < r1; rb += NW * RPW) {
-      const int r = rb + rsub;
-      if (r < r1) {
-        float x[EPL];
-        Elem<T>::unpack(*reinterpret_cast<const uint4*>(vrow + r * D + sub * EPL), x);
-        float wv[G];
+    float qv[G][EPL];
+    if (c.nrows > 0) {
+      const T* sq = s_q + (size_t)(kk & 1) * G * D;
 #pragma unroll
-        for (int g = 0; g < G; ++g) wv[g] = s_w[r * G + g];
-        axpy_g<G, EPL>(wv, x, acc);
+      for (int g = 0; g < G; ++g) {
+        Elem<T>::unpack(*reinterpret_cast<const uint4*>(sq + g * D + sub * EPL), qv[g]);
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) qv[g][e] *= scale;
       }
     }
+    // ---- scores over the two centroid tiles
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      mbar_wait(&s_bar[(4 * kk + t) & 3], par, status);
+      const T* tile = ring + (size_t)((4 * kk + t) & 3) * TR * D;
+      if (c.nrows > t * TR) {
+#pragma unroll
+        for (int it = 0; it < ITR; ++it) {
+          const int rl = (it * NW + warp) * RPW + rsub;
+          const int r = t * TR + rl;
+          const bool ok = r < c.nrows;
+          float x[EPL];
+          if (ok) {
+            Elem<T>::unpack(*reinterpret_cast<const uint4*>(tile + rl * D + sub * EPL), x);
+          } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) x[e] = 0.f;
+          }
+          float acc[G];
+          dot_g<G, EPL>(qv, x, acc);
+          group_reduce_multi<G, LPR>(acc, lane);
+          float m = acc[0];
+#pragma unroll
+          for (int o = LPR / 2; o >= LPR / G; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          if (ok) {
+            if (sub % (LPR / G) == 0) {
+              scores[(c.row0 + c.c0 + r) * G + j] = acc[0];
+              s_w[r * G + j] = acc[0];
+            }
+            if (sub == 0) {
+              const uint32_t key = (s_off[r + 1] - s_off[r]) > 0 ? ordered_key(m) : 0u;
+              keys[c.row0 + c.c0 + r] = key;
+              if (key) atomicAdd(&hist[key >> (kHistShift + 1)], 1u << (16 * ((key >> kHistShift) & 1u)));
+            }
+          }
+        }
+      }
+      __syncthreads();
+      if (tid == 0) issue_tile(4 * kk + t + 4);
+    }
+    if (c.nrows == 0) {
+      // past this sequence's clusters: an empty part; consume the value-sum tiles
+      empty_part(part, G, PS);
+#pragma unroll
+      for (int t = 2; t < 4; ++t) {
+        mbar_wait(&s_bar[(4 * kk + t) & 3], par, status);
+        __syncthreads();
+        if (tid == 0) issue_tile(4 * kk + t + 4);
+      }
+      issue_meta(kk + 2);
+      continue;
+    }
+    // ---- histogram flush (two 16-bit counts per word), chunk statistics
+    {
+      int* hg = hist_g + (int64_t)c.u * kHistBins;
+      for (int i = tid; i < kHistBins / 2; i += blockDim.x) {
+        const uint32_t w = hist[i];
+        if (w) {
+          if (w & 0xffffu) atomicAdd(hg + 2 * i, (int)(w & 0xffffu));
+          if (w >> 16) atomicAdd(hg + 2 * i + 1, (int)(w >> 16));
+          hist[i] = 0u;
+        }
+      }
+    }
+    if (warp < G) {  // warp g: head g's max, weights and denominator
+      float m = -INFINITY;
+      for (int r = lane; r < c.nrows; r += 32) m = fmaxf(m, s_w[r * G + warp]);
+      m = warp_max(m);
+      float l = 0.f;
+      for (int r = lane; r < c.nrows; r += 32) {
+        const int cnt = s_off[r + 1] - s_off[r];
+        const float w = cnt > 0 ? __expf(s_w[r * G + warp] - m) : 0.f;
+        s_w[r * G + warp] = w;
+        l += (float)cnt * w;
+      }
+      l = warp_sum(l);
+      if (lane == 0) { s_m[warp] = m; s_l[warp] = l; }
+    }
+    __syncthreads();
+    // ---- weighted value sums over the two value-sum tiles
+    float acc[G][EPL];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) acc[g][e] = 0.f;
+#pragma unroll
+    for (int t = 2; t < 4; ++t) {
+      mbar_wait(&s_bar[(4 * kk + t) & 3], par, status);
+      const T* tile = ring + (size_t)((4 * kk + t) & 3) * TR * D;
+#pragma unroll
+      for (int it = 0; it < ITR; ++it) {
+        const int rl = (it * NW + warp) * RPW + rsub;
+        const int r = (t - 2) * TR + rl;
+        if (r < c.nrows) {
+          float x[EPL];
+          Elem<T>::unpack(*reinterpret_cast<const uint4*>(tile + rl * D + sub * EPL), x);
+          float wv[G];
+          load_row<G>(s_w + r * G, wv);
+          axpy_g<G, EPL>(wv, x, acc);
+        }
+      }
+      __syncthreads();
+      if (tid == 0) issue_tile(4 * kk + t + 4);
+    }
+    reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part);
+    if (tid < G) { part[tid * PS] = s_m[tid]; part[tid * PS + 1] = s_l[tid]; }
+    issue_meta(kk + 2);
   }
-  // the cross-warp reduction reuses the centroid rows (<= 32 KB, read long ago)
-  reduce_and_store<G, EPL, LPR, D>(acc, reinterpret_cast<float*>(sh_dyn), warp, sub, rsub, part);
-  if (tid < G) { part[tid * PS] = s_m[tid]; part[tid * PS + 1] = s_l[tid]; }
+  cp_async_wait<0>();
+  // every tile issued was waited for above; should a bounded wait have given
+  // up, wait (bounded again) for each slot's last copy before leaving
+  if (nk > 0) {
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) mbar_wait(&s_bar[sl], (uint32_t)((nk - 1) & 1), status);
+  }
+}
+
+// K_A on the tensor cores (bf16, d = 128).  Same chunking, ring and
+// pipeline as wave_score_kernel, with the two tiny contractions on mma.sync
+// m16n8k16 (bf16 in, fp32 accumulate): the CUDA-core form of this kernel is
+// issue-bound, not memory-bound, at G <= 8 query rows.
+//  scores:  S^T[g][r] = sum_d q[g][d] c[r][d]  (A = q, heads padded to 16 rows;
+//           B = centroid rows through ldmatrix), scaled by 1/sqrt(d) after;
+//  weights: o[g][d] = sum_r w[g][r] Vsum[r][d] (A = w split into two bf16
+//           terms, w = hi + lo to ~2^-17; B = value-sum rows through
+//           ldmatrix.trans).  Each warp owns 16 output columns, so no
+//           cross-warp reduction.
+// Tiles arrive by 2-D tensor copies (two 64-column boxes per 16 KB tile)
+// with the 128-byte swizzle, which makes every ldmatrix conflict-free.
+template <int G>
+struct MmaSmem {
+  static constexpr int D = 128, CROWS = kScoreChunkBytes / (D * 2), TR = 64;
+  static constexpr size_t kRing = 4 * 16384;
+  static constexpr size_t kHist = (size_t)kHistBins / 2 * 4;
+  static constexpr size_t kOff = (size_t)2 * (CROWS + 4) * 4;
+  static constexpr size_t kW = (size_t)G * CROWS * 4;
+  static constexpr size_t kQ = (size_t)2 * G * D * 2;
+  static constexpr size_t oHist = kRing, oOff = oHist + kHist, oW = oOff + kOff, oQ = oW + kW,
+                          kTotal = oQ + kQ + 1024;   // + 1 KB to align the ring to 1024 B
+};
+
+template <int G>
+__global__ void __launch_bounds__(kStreamThreads, 2)
+wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_q_heads,
+                      const __grid_constant__ CUtensorMap tm_cent,
+                      const __grid_constant__ CUtensorMap tm_vsum,
+                      const int32_t* __restrict__ offsets, float* __restrict__ scores,
+                      uint32_t* __restrict__ keys, int32_t* __restrict__ hist_g,
+                      float* __restrict__ est_parts, float scale, int n_chunks, int n_stream,
+                      const SteadyArgs sa, uint32_t* status) {
+  using T = __nv_bfloat16;
+  using SM = MmaSmem<G>;
+  constexpr int D = SM::D, CROWS = SM::CROWS, TR = SM::TR;
+  constexpr int PS = Part<D>::kStride;
+  static_assert(G <= 8, "at most 8 query heads per KV head (MMA rows 0..7)");
+  extern __shared__ __align__(16) unsigned char sh_raw[];
+  __shared__ float s_m[G], s_l[G];
+  __shared__ __align__(8) uint64_t s_bar[4];
+  pdl_launch_dependents();
+  const int U = geo.batch * geo.hkv;
+  if ((int)blockIdx.x < U) {
+    steady_role<T, D>(geo, blockIdx.x, sa, status, sh_raw);
+    return;
+  }
+  unsigned char* sh = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(sh_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* ring = sh;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sh + SM::oHist);
+  int* s_offb = reinterpret_cast<int*>(sh + SM::oOff);
+  float* s_w = reinterpret_cast<float*>(sh + SM::oW);          // [G][CROWS]
+  T* s_q = reinterpret_cast<T*>(sh + SM::oQ);
+  const int sidx = blockIdx.x - U;
+  const int n_tot = U * n_chunks;
+  const int k0 = (int)((int64_t)sidx * n_tot / n_stream);
+  const int k1 = (int)((int64_t)(sidx + 1) * n_tot / n_stream);
+  const int nk = k1 - k0;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tq = lane & 3;    // MMA fragment row (head) and column pair
+  struct Chunk { int u, b, h, c0, nrows; int64_t row0; };
+  auto chunk = [&](int k) -> Chunk {
+    Chunk c;
+    c.u = k / n_chunks;
+    c.b = c.u / geo.hkv;
+    c.h = c.u - c.b * geo.hkv;
+    c.c0 = (k - c.u * n_chunks) * CROWS;
+    c.nrows = max(0, min(geo.NC(c.b) - c.c0, CROWS));
+    c.row0 = geo.cl_row(c.b, c.h);
+    return c;
+  };
+  auto issue_tile = [&](int i) {   // thread 0
+    if (i >= 4 * nk) return;
+    const int part = i & 3;
+    const Chunk c = chunk(k0 + (i >> 2));
+    const int r0 = (part & 1) * TR;
+    uint64_t* bar = &s_bar[i & 3];
+    if (c.nrows - r0 <= 0) { mbar_arrive(bar); return; }
+    const CUtensorMap* tm = part < 2 ? &tm_cent : &tm_vsum;
+    unsigned char* dst = ring + (size_t)(i & 3) * 16384;
+    const int y = (int)(c.row0 + c.c0 + r0);
+    fence_proxy_async();
+    mbar_arrive_expect(bar, 16384u);
+    tensor_load_2d(dst, tm, 0, y, bar);
+    tensor_load_2d(dst + 8192, tm, 64, y, bar);
+  };
+  auto issue_meta = [&](int kk) {   // all threads
+    if (kk < nk) {
+      const Chunk c = chunk(k0 + kk);
+      if (c.nrows > 0) {
+        int* so = s_offb + (kk & 1) * (CROWS + 4);
+        const int32_t* off = offsets + geo.off_row(c.b, c.h) + c.c0;
+        for (int x = tid; x <= c.nrows; x += blockDim.x) cp_async4(so + x, off + x);
+        T* sq = s_q + (size_t)(kk & 1) * G * D;
+        const T* qs = q + ((int64_t)c.b * n_q_heads + (int64_t)c.h * G) * D;
+        for (int x = tid; x < G * D / 8; x += blockDim.x) cp_async16(sq + x * 8, qs + x * 8);
+      }
+    }
+    cp_async_commit();
+  };
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mbar_init(&s_bar[i], 1);
+    mbar_init_fence();
+  }
+  for (int i = tid; i < kHistBins / 2; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) issue_tile(i);
+  }
+  issue_meta(0);
+  issue_meta(1);
+
+  for (int kk = 0; kk < nk; ++kk) {
+    const Chunk c = chunk(k0 + kk);
+    float* part = est_parts + ((int64_t)(k0 + kk)) * G * PS;
+    const int* s_off = s_offb + (kk & 1) * (CROWS + 4);
+    const uint32_t par = kk & 1;
+    cp_async_wait<1>();
+    __syncthreads();
+    // q as A fragments (rows = heads; heads >= G and rows 8..15 are zero)
+    uint32_t qa0[D / 16], qa2[D / 16];
+    {
+      const uint32_t* qw = reinterpret_cast<const uint32_t*>(s_q + (size_t)(kk & 1) * G * D + g * D);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        qa0[ks] = (g < G && c.nrows > 0) ? qw[8 * ks + tq] : 0u;
+        qa2[ks] = (g < G && c.nrows > 0) ? qw[8 * ks + 4 + tq] : 0u;
+      }
+    }
+    // ---- scores: warp w takes the tile's rows 8w .. 8w + 7
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      mbar_wait(&s_bar[t], par, status);
+      const unsigned char* slot = ring + (size_t)t * 16384;
+      if (c.nrows > t * TR) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const int n0 = 8 * warp;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ks += 2) {
+          const int ch = 2 * ks + (lane >> 3);                     // 16-byte column chunk
+          uint32_t bm[4];
+          ldsm_x4(bm, slot + (ch >> 3) * 8192 + swz128(n0 + (lane & 7), ch & 7));
+          mma_bf16(acc, qa0[ks], qa2[ks], bm[0], bm[1]);
+          mma_bf16(acc, qa0[ks + 1], qa2[ks + 1], bm[2], bm[3]);
+        }
+        const int rl = t * TR + n0 + 2 * tq;                       // rows rl, rl + 1 of the chunk
+        const float s0 = acc[0] * scale, s1 = acc[1] * scale;
+        const bool ok0 = rl < c.nrows, ok1 = rl + 1 < c.nrows;
+        if (g < G) {
+          if (ok0) scores[(c.row0 + c.c0 + rl) * G + g] = s0;
+          if (ok1) scores[(c.row0 + c.c0 + rl + 1) * G + g] = s1;
+          *reinterpret_cast<float2*>(s_w + g * CROWS + rl) = make_float2(s0, s1);
+        }
+        float m0 = g < G ? s0 : -INFINITY, m1 = g < G ? s1 : -INFINITY;
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+          m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+        }
+        if (g == 0) {
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int r = rl + k;
+            if (r < c.nrows) {
+              const uint32_t key = (s_off[r + 1] - s_off[r]) > 0 ? ordered_key(k ? m1 : m0) : 0u;
+              keys[c.row0 + c.c0 + r] = key;
+              if (key) atomicAdd(&hist[key >> (kHistShift + 1)], 1u << (16 * ((key >> kHistShift) & 1u)));
+            }
+          }
+        }
+      }
+      __syncthreads();
+      if (tid == 0) issue_tile(4 * kk + t + 4);
+    }
+    if (c.nrows == 0) {
+      empty_part(part, G, PS);
+#pragma unroll
+      for (int t = 2; t < 4; ++t) {
+        mbar_wait(&s_bar[t], par, status);
+        __syncthreads();
+        if (tid == 0) issue_tile(4 * kk + t + 4);
+      }
+      issue_meta(kk + 2);
+      continue;
+    }
+    // ---- histogram flush, chunk statistics (warp g: head g); weights of
+    // rows past the chunk's clusters are zero
+    {
+      int* hg = hist_g + (int64_t)c.u * kHistBins;
+      for (int i = tid; i < kHistBins / 2; i += blockDim.x) {
+        const uint32_t w = hist[i];
+        if (w) {
+          if (w & 0xffffu) atomicAdd(hg + 2 * i, (int)(w & 0xffffu));
+          if (w >> 16) atomicAdd(hg + 2 * i + 1, (int)(w >> 16));
+          hist[i] = 0u;
+        }
+      }
+    }
+    if (warp < G) {
+      float* wr = s_w + warp * CROWS;
+      float m = -INFINITY;
+      for (int r = lane; r < c.nrows; r += 32) m = fmaxf(m, wr[r]);
+      m = warp_max(m);
+      float l = 0.f;
+      for (int r = lane; r < CROWS; r += 32) {
+        const int cnt = r < c.nrows ? s_off[r + 1] - s_off[r] : 0;
+        const float w = cnt > 0 ? __expf(wr[r] - m) : 0.f;
+        wr[r] = w;
+        l += (float)cnt * w;
+      }
+      l = warp_sum(l);
+      if (lane == 0) { s_m[warp] = m; s_l[warp] = l; }
+    }
+    __syncthreads();
+    // ---- weighted value sums: warp w owns output columns 16w .. 16w + 15
+    float oacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int t = 2; t < 4; ++t) {
+      mbar_wait(&s_bar[t], par, status);
+      const unsigned char* slot = ring + (size_t)t * 16384;
+      const int kb = (t - 2) * TR;
+      // a tile past the chunk's rows was never loaded (its slot holds older
+      // data, or none): skip it; in a loaded tile the rows past the chunk
+      // are real rows (or zero fill) with zero weight
+#pragma unroll
+      for (int ks = 0; ks < TR / 16; ++ks) {
+        if (c.nrows <= kb) break;
+        uint32_t ah0 = 0u, al0 = 0u, ah2 = 0u, al2 = 0u;
+        if (g < G) {
+          const float* wr = s_w + g * CROWS + kb + 16 * ks + 2 * tq;
+          const float2 w01 = *reinterpret_cast<const float2*>(wr);
+          const float2 w23 = *reinterpret_cast<const float2*>(wr + 8);
+          split_bf16(w01.x, w01.y, ah0, al0);
+          split_bf16(w23.x, w23.y, ah2, al2);
+        }
+        const int row = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int ch = 2 * warp + (lane >> 4);
+        uint32_t bm[4];
+        ldsm_x4_t(bm, slot + (ch >> 3) * 8192 + swz128(row, ch & 7));
+        mma_bf16(oacc[0], ah0, ah2, bm[0], bm[1]);
+        mma_bf16(oacc[0], al0, al2, bm[0], bm[1]);
+        mma_bf16(oacc[1], ah0, ah2, bm[2], bm[3]);
+        mma_bf16(oacc[1], al0, al2, bm[2], bm[3]);
+      }
+      __syncthreads();
+      if (tid == 0) issue_tile(4 * kk + t + 4);
+    }
+    if (g < G) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int d = 16 * warp + 8 * nt + 2 * tq;
+        *reinterpret_cast<float2*>(part + g * PS + Part<D>::kO + d) = make_float2(oacc[nt][0], oacc[nt][1]);
+      }
+    }
+    if (tid < G) { part[tid * PS] = s_m[tid]; part[tid * PS + 1] = s_l[tid]; }
+    issue_meta(kk + 2);
+  }
+  cp_async_wait<0>();
+  if (nk > 0) {
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) mbar_wait(&s_bar[sl], (uint32_t)((nk - 1) & 1), status);
+  }
 }
 
 // ----------------------------------------------------------------- K_B topk
-// One CTA per unit.  Every global read it needs is issued in one round at
-// the start (unit record, first-digit histogram, non-candidate, steady and
-// affected lists, the sequence's block-table row, and the first kTopkRound
-// keys and offsets into registers, 16 consecutive cluster ids per thread);
-// all later steps work in shared memory and registers:
+// One CTA per unit finds the selection threshold: the k-th best candidate
+// key kstar and the largest id thr taken at that key, so that cluster c is
+// retrieved iff key_c > kstar or (key_c == kstar and c <= thr) (Vortex 2.C
+// Top-K: exact, ties to the lower id).  Every global read is issued in one
+// round at the start (unit record, first-digit histogram, non-candidate
+// list, and the keys, kTopkPerLane per thread, lane-interleaved so each warp
+// load is one 128-byte line); then
 //  1. the first radix digit's histogram comes from K_A (zeroed after use, so
 //     the workspace is clean for the next call), minus the non-candidates; a
 //     histogram whose total disagrees with the candidate count is flagged
 //     and the select falls back to a full radix select over all keys;
 //  2. the keys of the threshold bin (1-2% of them) get a second 11-bit digit
 //     histogram, and the few keys of its threshold bin are ranked exactly by
-//     (key desc, id asc) (Vortex 2.C Top-K: exact, ties to the lower id);
-//  3. one block scan orders the selection: each thread writes its selected
-//     clusters (ascending ids) with their token starts; then each warp
-//     expands its threads' selected clusters into the gather list (pool rows
-//     of their tokens, -1 for steady members), and the steady slots' rows
-//     follow.
+//     (key desc, id asc).
+// The retrieved clusters themselves are picked by the attend kernel's CTAs,
+// each over its own range of cluster ids.
 constexpr int kTopkPerLane = 16;
 constexpr int kTopkRound = kTopkThreads * kTopkPerLane;   // 8192 ids per round
 constexpr int kTopkCand = 1024;
@@ -513,27 +917,18 @@ __device__ void fold_role(const FoldArgs& f, int u, int j) {
 
 struct TopkArgs {
   const uint32_t* keys;
-  const int32_t* offsets;
   int32_t* hist_g;
   const int32_t* nonc;       // [U][cap+1]: count, then the non-candidate clusters
-  const int32_t* st_slot;    // [U][cap]: steady slots, ascending
-  const int32_t* aff_cl;     // [U][cap]: affected clusters, ascending
-  const int32_t* aff_start;  // [U][cap+1]: their first steady index
   int cap;
   int topk_clusters;
   double topk_fraction;
-  int32_t *sel, *sel_tok, *info;
-  Pool kp;
-  int32_t* gather;
-  int64_t gather_stride;
-  int bt_cap;                // block-table entries staged in shared memory
+  int32_t* info;
+  int32_t* sel_n;            // [U]: selection-list counter of the attend kernel (zeroed here)
 };
 
 __global__ void __launch_bounds__(kTopkThreads)
 wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* status) {
   // dynamic shared: excluded bitmask [ceil(NCmax/32)] | non-candidates [cap+1]
-  //   | steady slots [cap] | affected clusters [cap] | their starts [cap+1]
-  //   | block-table row [bt_cap]
   extern __shared__ __align__(16) int32_t sdyn[];
   __shared__ __align__(16) int hist[kHistBins];
   __shared__ unsigned long long cand[kTopkCand];
@@ -548,45 +943,33 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* s
     return;
   }
   constexpr int PT = kTopkPerLane;
+  constexpr int NW = kTopkThreads / 32;
   const int tid = threadIdx.x, nt = kTopkThreads, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
   const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
-  const int NC = geo.NC(b), Tb = geo.T(b);
+  const int NC = geo.NC(b);
   const int nmask = (NC + 31) >> 5;
   const int cap = A.cap;
   uint32_t* sx = reinterpret_cast<uint32_t*>(sdyn);
   int32_t* snc = sdyn + nmask;
-  int32_t* ss = snc + cap + 1;
-  int32_t* sacl = ss + cap;
-  int32_t* sast = sacl + cap;
-  int32_t* sbt = sast + cap + 1;
-  const int page_shift = A.kp.page_shift;
-  const int n_bt = (Tb + (1 << page_shift) - 1) >> page_shift;
-  const bool bt_sh = n_bt <= A.bt_cap && n_bt <= A.kp.max_pages;
   for (int i = tid; i < nmask; i += nt) sx[i] = 0u;
   if (tid == 0) { s_ctl[0] = 0; s_ctl[5] = 0; }
   int32_t* I = A.info + (int64_t)u * kInfoInts;
   const int64_t row0 = geo.cl_row(b, h);
-  int32_t* pre = A.sel_tok + row0 + u;
   int* hg = A.hist_g + (int64_t)u * kHistBins;
   const int k_req = A.topk_clusters >= 0 ? A.topk_clusters
                                          : (int)ceil(A.topk_fraction * (double)NC);
   const uint32_t* kk = A.keys + row0;
-  const int32_t* off = A.offsets + geo.off_row(b, h);
-  int32_t* gat = A.gather + (int64_t)u * A.gather_stride;
   const int n_rounds = (NC + kTopkRound - 1) / kTopkRound;
+  const int wbase = warp * (kTopkRound / NW);       // warp's offset inside a round
   uint32_t kr[PT];
-  int ofs[PT + 1];
-  auto cid = [&](int r, int i) { return r * kTopkRound + tid * PT + i; };
-  auto load_round = [&](int r) {                    // raw keys and offsets of round r
+  auto cid = [&](int r, int i) { return r * kTopkRound + wbase + i * 32 + lane; };
+  auto load_round = [&](int r) {
 #pragma unroll
     for (int i = 0; i < PT; ++i) {
       const int c = cid(r, i);
       kr[i] = c < NC ? kk[c] : 0u;
-      ofs[i] = c <= NC ? __ldg(off + c) : 0;
     }
-    const int c = cid(r, PT);
-    ofs[PT] = c <= NC ? __ldg(off + c) : 0;
   };
   auto masked = [&](int c) -> bool { return ((sx[c >> 5] >> (c & 31)) & 1u) != 0u; };
   auto mask_round = [&](int r) {
@@ -601,43 +984,15 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* s
   // ---- the one round of loads
   if (tid < kInfoInts) cp_async4(&s_info[tid], I + tid);
   for (int i = tid; i < kHistBins / 4; i += nt) cp_async16(&hist[4 * i], hg + 4 * i);
-  for (int i = tid; i <= cap; i += nt) {
-    cp_async4(snc + i, A.nonc + (int64_t)u * (cap + 1) + i);
-    cp_async4(sast + i, A.aff_start + (int64_t)u * (cap + 1) + i);
-    if (i < cap) {
-      cp_async4(ss + i, A.st_slot + (int64_t)u * cap + i);
-      cp_async4(sacl + i, A.aff_cl + (int64_t)u * cap + i);
-    }
-  }
-  if (bt_sh)
-    for (int i = tid; i < n_bt; i += nt) cp_async4(sbt + i, A.kp.bt + (int64_t)b * A.kp.max_pages + i);
+  for (int i = tid; i <= cap; i += nt) cp_async4(snc + i, A.nonc + (int64_t)u * (cap + 1) + i);
   cp_async_commit();
   load_round(0);
   cp_async_wait<0>();
   __syncthreads();
   for (int i = tid; i < kHistBins; i += nt) hg[i] = 0;   // clean for the next call
-  const int n_st = s_info[4];
-  const int dense = s_info[6];
-  const int n_aff = dense ? 0 : min(max(s_info[5], 0), cap);
-  auto row_of = [&](int slot) -> int32_t {
-    if (bt_sh) {
-      const int lp = slot >> page_shift;
-      const int pg = (slot >= 0 && lp < n_bt) ? sbt[lp] : -1;
-      if (pg < 0 || (int64_t)pg >= A.kp.n_pages) {
-        flag_error(status, slot < 0 || lp >= n_bt ? WI_DEV_BAD_SLOT : WI_DEV_BAD_PAGE);
-        return -1;
-      }
-      return (((int32_t)pg * geo.hkv + h) << page_shift) + (slot & ((1 << page_shift) - 1));
-    }
-    const int64_t ro = pool_row(A.kp, geo.hkv, 1, b, h, slot, status);
-    return ro < 0 ? -1 : (int32_t)ro;
-  };
-  if (dense) {  // the attend CTAs take all slots in order
-    for (int t = tid; t < Tb; t += nt) gat[t] = row_of(t);
-    if (tid == 0) {
-      I[0] = 0; I[1] = (int32_t)0xFFFFFFFFu; I[2] = -1; I[3] = 0; I[7] = 0;
-      pre[0] = 0;
-    }
+  if (tid == 0) { A.sel_n[u] = 0; I[3] = 0; }
+  if (s_info[6]) {  // dense unit: every token is attended, nothing is selected
+    if (tid == 0) { I[0] = 0; I[1] = (int32_t)0xFFFFFFFFu; I[2] = -1; I[7] = 0; }
     return;
   }
   // clusters left without a non-steady member are not candidates
@@ -663,23 +1018,20 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* s
   }
   __syncthreads();
 
-  // histogram total -> threshold bin of the first digit (valid if consistent)
-  int hs = 0;
-  for (int i = tid; i < kHistBins; i += nt) hs += hist[i];
-  int hist_total;
-  block_inclusive_scan(hs, scan_sh, &hist_total);
-  int ksel = min(max(k_req, 0), hist_total);
-  // bin holding the krem-th largest of the histogram (bins scanned downwards);
-  // *above: count in the bins above it
-  auto first_digit = [&](int krem, int* above) -> int {
+  // bin holding the krem-th largest of the histogram (bins scanned
+  // downwards); *above: the count in the bins above it; *total: all
+  auto first_digit = [&](int krem, int* above, int* total) -> int {
     // thread t owns bins 2047-4t .. 2044-4t (descending)
     int c4[4], s4 = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) { c4[i] = hist[kHistBins - 1 - 4 * tid - i]; s4 += c4[i]; }
     int tot;
     const int incl = block_inclusive_scan(s4, scan_sh, &tot);
+    if (krem < 0) krem = min(max(k_req, 0), tot);   // the first digit: k clamped to the total
     int acc = incl - s4;
-    if (acc < krem && incl >= krem) {
+    if (tid == 0) { s_ctl[1] = -1; s_ctl[2] = 0; }
+    __syncthreads();
+    if (krem > 0 && acc < krem && incl >= krem) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         if (acc + c4[i] >= krem) { s_ctl[1] = kHistBins - 1 - 4 * tid - i; s_ctl[2] = acc; break; }
@@ -688,10 +1040,9 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* s
     }
     __syncthreads();
     *above = s_ctl[2];
+    if (total) *total = tot;
     return s_ctl[1];
   };
-  int bin1 = -1, above1 = 0;
-  if (ksel > 0 && ksel < hist_total) bin1 = first_digit(ksel, &above1);
   // ballot-aggregated append of x to list[cap_] through counter *ctr
   auto append = [&](bool in, unsigned long long x, unsigned long long* list, int cap_, int* ctr) {
     const unsigned bal = __ballot_sync(0xffffffffu, in);
@@ -703,6 +1054,9 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* s
       if (in && slot < cap_) list[slot] = x;
     }
   };
+  int above1 = 0, hist_total = 0;
+  int bin1 = first_digit(-1, &above1, &hist_total);
+  if (min(max(k_req, 0), hist_total) >= hist_total) bin1 = -1;   // all or none: no threshold bin
 
   // pass A: candidate count, and the keys of the threshold bin
   int mine = 0;
@@ -722,9 +1076,9 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* s
   const int nbin = s_ctl[0];
   const bool hist_ok = ncand == hist_total;
   if (!hist_ok && tid == 0) flag_error(status, WI_DEV_BAD_HIST);
-  ksel = min(max(k_req, 0), ncand);
-  uint32_t kstar;
-  int thr;
+  const int ksel = min(max(k_req, 0), ncand);
+  uint32_t kstar = 0;
+  int thr = 0;
   bool found = false;
   if (ksel == 0) { kstar = 0xFFFFFFFFu; thr = -1; found = true; }
   else if (ksel == ncand) { kstar = 1u; thr = NC; found = true; }
@@ -737,7 +1091,7 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* s
       atomicAdd(&hist[(int)(cand[i] >> 42) & (kHistBins - 1)], 1);
     __syncthreads();
     int above2;
-    const int bin2 = first_digit(krem, &above2);
+    const int bin2 = first_digit(krem, &above2, nullptr);
     krem -= above2;
     for (int i0 = 0; i0 < nbin; i0 += nt) {
       const int i = i0 + tid;
@@ -779,7 +1133,7 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* s
       }
       __syncthreads();
       int ab;
-      const int d = first_digit(krem, &ab) & (nbins - 1);
+      const int d = first_digit(krem, &ab, nullptr) & (nbins - 1);
       krem -= ab;
       prefix |= (uint32_t)d << shift;
       pmask |= (uint32_t)(nbins - 1) << shift;
@@ -801,91 +1155,42 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* s
     }
     thr = s_ctl[4];
   }
-  auto picked = [&](int c, uint32_t key) -> bool {  // key: candidate key or 0
-    return key != 0u && (key > kstar || (key == kstar && c <= thr));
-  };
-
-  // ordered compaction and gather list, round by round
-  int sel_run = 0, tok_run = 0;   // totals of earlier rounds
-  for (int r = 0; r < n_rounds; ++r) {
-    if (n_rounds > 1) { load_round(r); mask_round(r); }
-    int cnt = 0, tk = 0;
-#pragma unroll
-    for (int i = 0; i < PT; ++i) {
-      const bool p = picked(cid(r, i), kr[i]);
-      cnt += p;
-      tk += p ? ofs[i + 1] - ofs[i] : 0;
-    }
-    int2 tot;
-    const int2 incl = block_inclusive_scan2(make_int2(cnt, tk), scan_sh, &tot);
-    int si = sel_run + incl.x - cnt, st = tok_run + incl.y - tk;
-    // this thread's selected clusters: list entries, and per cluster the
-    // token start and the range of its steady members (affected clusters)
-    unsigned pmask = 0u;
-    int tst[PT], aj[PT];
-#pragma unroll
-    for (int i = 0; i < PT; ++i) {
-      const int c = cid(r, i);
-      tst[i] = st;
-      aj[i] = -1;
-      if (picked(c, kr[i])) {
-        pmask |= 1u << i;
-        A.sel[row0 + si] = c;
-        pre[si] = st;
-        aj[i] = n_aff ? find_sorted(sacl, n_aff, c) : -1;
-        ++si;
-        st += ofs[i + 1] - ofs[i];
-      }
-    }
-    // the warp expands its lanes' selected clusters, one cluster at a time
-#pragma unroll
-    for (int i = 0; i < PT; ++i) {
-      unsigned bal = __ballot_sync(0xffffffffu, (pmask >> i) & 1u);
-      while (bal) {
-        const int src = __ffs(bal) - 1;
-        bal &= bal - 1u;
-        const int o0 = __shfl_sync(0xffffffffu, ofs[i], src);
-        const int n = __shfl_sync(0xffffffffu, ofs[i + 1], src) - o0;
-        const int t0 = __shfl_sync(0xffffffffu, tst[i], src);
-        const int j = __shfl_sync(0xffffffffu, aj[i], src);
-        const int s0 = j >= 0 ? sast[j] : 0, s1 = j >= 0 ? sast[j + 1] : 0;
-        for (int t = lane; t < n; t += 32) {
-          const int slot = o0 + t;
-          bool steady = false;
-          for (int k = s0; k < s1; ++k) steady |= ss[k] == slot;
-          gat[t0 + t] = steady ? -1 : row_of(slot);
-        }
-      }
-    }
-    sel_run += tot.x;
-    tok_run += tot.y;
-  }
-  const int total_tok = tok_run;
-  for (int j = tid; j < n_st; j += nt) gat[total_tok + j] = row_of(ss[j]);
-  if (tid == 0) {
-    pre[ksel] = total_tok;
-    I[0] = ksel; I[1] = (int32_t)kstar; I[2] = thr; I[3] = total_tok; I[7] = ncand;
-  }
+  if (tid == 0) { I[0] = ksel; I[1] = (int32_t)kstar; I[2] = thr; I[7] = ncand; }
 }
 
-// --------------------------------------------------- K_C attend + correct
-// attend CTAs: split-K exact attention over the gather list (retrieved
-// clusters' non-steady rows, then the steady rows);
-// correction CTAs: the part -(what K_A's chunk parts counted that the
-// estimation zone leaves out), kNegChunk clusters per CTA, their rows staged
-// in shared memory by one round of cp.async;
-// the last CTA of each unit merges the attend parts, the correction parts and
-// K_B's folded estimation parts by log-sum-exp.
-constexpr int kNegChunk = kNegRows;
+// ----------------------------------------------------------------- K_C attend
+// range CTAs (kRangeW cluster ids each): pick the retrieved clusters of the
+// range against K_B's threshold, append them to the unit's (unordered)
+// selection list, resolve their tokens' pool rows (skipping steady members)
+// and run exact attention over them; in the same part, take back out of
+// the estimate what K_A's chunk parts counted that the estimation zone
+// leaves out: every retrieved cluster and every cluster left without a
+// non-steady member in full (cnt, Vsum), and the steady members (their
+// count, dV) of the other affected clusters;
+// steady CTAs (two tiles of steady slots each): exact attention over the
+// steady zone;
+// the last CTA of each unit merges these parts and K_B's folded estimation
+// parts by log-sum-exp.
+constexpr int kRangeW = kRangeClusters;    // clusters per range CTA, one per thread
+static_assert(kRangeW == kStreamThreads, "one cluster per thread");
+constexpr int kCorrRows = 32;              // correction rows staged per pass
+constexpr int kRowCap = 512;               // tokens resolved per pass of a range CTA
 
 struct AttendArgs {
-  const int32_t *gather, *aff_cl, *aff_start, *sel;
-  const float* dv;
-  int64_t gather_stride;
-  const int32_t* info;
-  const float* scores;
   const uint32_t* keys;
-  int cap, n_splits, n_neg, n_parts, wcap;
+  const float* scores;
+  const int32_t* info;
+  int32_t* aff_of;           // [U][max_nc]: +(j+1) affected, -(j+1) non-candidate; reset here
+  int max_nc;
+  const int32_t* aff_start;  // [U][cap+1]
+  const int32_t* st_slot;    // [U][cap]
+  const float* dv;           // [U][cap][D]
+  int cap;
+  const int32_t* perm;       // slot -> position
+  int n_sink, window;
+  int32_t* sel;              // per unit, the retrieved clusters (unordered)
+  int32_t* sel_n;            // [U] its counter
+  int n_rng, n_sc, n_parts;
   float* partials;
   int32_t* counters;
   float* out;
@@ -894,306 +1199,410 @@ struct AttendArgs {
 };
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kStreamThreads)
-wave_attend_estimate_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const Pool kp,
-                            const Pool vp, const T* __restrict__ vsum,
-                            const int32_t* __restrict__ offsets, const AttendArgs A,
-                            uint32_t* status) {
+__global__ void __launch_bounds__(kStreamThreads, G * Elem<T>::kPerVec >= 64 ? 1 : 2)
+wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const Pool kp,
+                   const Pool vp, const T* __restrict__ vsum,
+                   const int32_t* __restrict__ offsets, const AttendArgs A, uint32_t* status) {
   using RS = RowShape<T, D>;
   constexpr int EPL = RS::EPL, LPR = RS::LPR, RPW = RS::RPW, TR = RS::TILE;
   constexpr int NW = kStreamThreads / 32;
+  constexpr int PS = Part<D>::kStride;
   static_assert(TR % (NW * RPW) == 0, "tile must be a multiple of rows per CTA step");
-  static_assert(kNegChunk * D * 4 <= 4 * 16384, "correction rows must fit the ring");
+  static_assert(2 * TR <= kStreamThreads, "one thread per token of a chunk");
   extern __shared__ __align__(16) unsigned char sh[];
-  // shared layout: [ring 64 KB: attend K x2, V x2 tiles | correction rows,
-  //                 kNegChunk slots of D fp32; the final cross-warp reduction
-  //                 and the merge reuse it] [s_w wcap*G f32] [s_cnt, s_ent kNegChunk i32]
+  // dynamic: [ring 64 KB: K x2, V x2 tiles; the cross-warp reduction and the
+  //           merge reuse it] [correction rows kCorrRows x D fp32] [merge factors]
   T* ring = reinterpret_cast<T*>(sh);
   float* s_red = reinterpret_cast<float*>(sh);
-  float* s_w = reinterpret_cast<float*>(sh + 4 * 16384);
-  int* s_cnt = reinterpret_cast<int*>(s_w + A.wcap * G);
-  int* s_ent = s_cnt + kNegChunk;
-  __shared__ int64_t s_row[2][TR];
-  __shared__ float s_sc[TR][G];
-  __shared__ int s_last;
-  __shared__ float s_m[G], s_l[G], s_part[NW][G];
-  __shared__ int s_info[kInfoInts];
+  unsigned char* s_crow = sh + 4 * 16384;
+  float* s_f = reinterpret_cast<float*>(s_crow + kCorrRows * D * 4);
+  __shared__ int32_t s_row[kRowCap];                 // pool rows of the tokens (-1 = skip)
+  __shared__ __align__(16) float s_sc[TR][G];
+  __shared__ int s_pkc[kRangeW], s_pkt[kRangeW], s_pko[kRangeW];   // picked: id, token start, slot start
+  __shared__ int s_cec[kRangeW], s_cew[kRangeW];                   // correction: row selector, count
+  __shared__ float s_ces[kRangeW * G];                              // correction: scores -> weights
+  __shared__ int scan_sh[64];
+  __shared__ int s_info[kInfoInts], s_base, s_last;
+  __shared__ float s_m[G], s_l[G];
 
   const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
-  const int NC = geo.NC(b);
+  const int NC = geo.NC(b), Tb = geo.T(b);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tid = threadIdx.x;
   const int sub = lane % LPR, rsub = lane / LPR;
   const int jh = sub / (LPR / G);
   const int64_t row0 = geo.cl_row(b, h);
   const int32_t* off = offsets + geo.off_row(b, h);
-  const bool role_neg = (int)blockIdx.x >= A.n_splits;
-  constexpr int PS = Part<D>::kStride;
+  const bool role_range = (int)blockIdx.x < A.n_rng;
   float* part = A.partials + ((int64_t)u * A.n_parts + blockIdx.x) * G * PS;
+  const int ns = min(A.n_sink, Tb), wstart = max(Tb - A.window, ns);
 
+  float qv[G][EPL];
+  load_q<T, D, G>(q, n_q_heads, b, h, sub, A.scale, qv);
   float acc[G][EPL];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int e = 0; e < EPL; ++e) acc[g][e] = 0.f;
+  float m_run[G], l_run[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) { m_run[g] = -INFINITY; l_run[g] = 0.f; }
 
-  if (role_neg) {
-    // ---------------------------------------------------------- correction
-    // entries e0 .. e0+ne-1 of [retrieved clusters (ascending) | affected
-    // clusters]: a retrieved cluster or an affected one left without a
-    // non-steady member counts in full (cnt, Vsum); another affected one
-    // that is estimated counts its steady members (their count, dV); an
-    // affected one that is also retrieved was counted with the retrieved.
-    pdl_wait();
-    if (tid < kInfoInts) s_info[tid] = A.info[(int64_t)u * kInfoInts + tid];
-    __syncthreads();
-    const int ksel = s_info[0];
-    const int n_aff = min(A.cap, s_info[5]);
-    const bool est = !s_info[6] && ksel < s_info[7] && NC > 0;
-    const int e0 = (blockIdx.x - A.n_splits) * kNegChunk;
-    const int ne = est ? max(0, min(kNegChunk, ksel + n_aff - e0)) : 0;
-    const uint32_t kstar = (uint32_t)s_info[1];
-    const int thr = s_info[2];
-    float m_loc[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) m_loc[g] = -INFINITY;
-    for (int i = tid; i < ne; i += blockDim.x) {
-      const int e = e0 + i;
-      int c, cnt, ent;
-      if (e < ksel) {
-        c = min(max(A.sel[row0 + e], 0), NC - 1);
-        cnt = __ldg(off + c + 1) - __ldg(off + c);
-        ent = c;
-      } else {
-        const int jj = e - ksel;
-        c = min(max(A.aff_cl[(int64_t)u * A.cap + jj], 0), NC - 1);
-        const int32_t* as = A.aff_start + (int64_t)u * (A.cap + 1) + jj;
-        const int dc = as[1] - as[0];
-        const int full = __ldg(off + c + 1) - __ldg(off + c);
-        const uint32_t key = A.keys[row0 + c];
-        if (full - dc <= 0) { cnt = full; ent = c; }
-        else if (key > kstar || (key == kstar && c <= thr)) { cnt = 0; ent = c; }
-        else { cnt = dc; ent = ~jj; }
-      }
-      s_cnt[i] = cnt;
-      s_ent[i] = ent;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float v = cnt > 0 ? A.scores[(row0 + c) * G + g] : -INFINITY;
-        s_w[i * G + g] = v;
-        m_loc[g] = fmaxf(m_loc[g], v);
-      }
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float v = warp_max(m_loc[g]);
-      if (lane == 0) s_part[warp][g] = v;
-    }
-    __syncthreads();
-    // stage the rows: slot i holds D fp32 (dV) or D elements of T (Vsum)
-    constexpr int CHF = D * 4 / 16, CHT = RS::ROWB / 16;
-    for (int k = tid; k < ne * CHF; k += blockDim.x) {
-      const int i = k / CHF, ch = k - i * CHF;
-      if (s_cnt[i] <= 0) continue;
-      const int ent = s_ent[i];
-      unsigned char* slot = sh + (size_t)i * D * 4;
-      if (ent >= 0) {
-        if (ch < CHT)
-          cp_async16(slot + ch * 16, reinterpret_cast<const unsigned char*>(vsum + (row0 + ent) * D) + ch * 16);
-      } else {
-        cp_async16(slot + ch * 16,
-                   reinterpret_cast<const unsigned char*>(A.dv + ((int64_t)u * A.cap + ~ent) * D) + ch * 16);
-      }
-    }
-    cp_async_commit();
-    if (tid < G) {
-      float v = -INFINITY;
-      for (int w = 0; w < NW; ++w) v = fmaxf(v, s_part[w][tid]);
-      s_m[tid] = v;
-    }
-    __syncthreads();
-    float l_loc[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) l_loc[g] = 0.f;
-    for (int i = tid; i < ne; i += blockDim.x) {
-      const int cnt = s_cnt[i];
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float w = cnt > 0 ? __expf(s_w[i * G + g] - s_m[g]) : 0.f;
-        s_w[i * G + g] = w;
-        l_loc[g] += (float)cnt * w;
-      }
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float v = warp_sum(l_loc[g]);
-      if (lane == 0) s_part[warp][g] = v;
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-    if (tid < G) {
-      float v = 0.f;
-      for (int w = 0; w < NW; ++w) v += s_part[w][tid];
-      s_l[tid] = v;
-    }
-    for (int rb = warp * RPW; rb < ne; rb += NW * RPW) {
-      const int i = rb + rsub;
-      if (i >= ne || s_cnt[i] <= 0) continue;
-      const unsigned char* slot = sh + (size_t)i * D * 4;
-      float x[EPL];
-      if (s_ent[i] >= 0) {
-        Elem<T>::unpack(*reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(slot) + sub * EPL), x);
-      } else {
-        const float* fr = reinterpret_cast<const float*>(slot) + sub * EPL;
-#pragma unroll
-        for (int e4 = 0; e4 < EPL; e4 += 4) {
-          const float4 v = *reinterpret_cast<const float4*>(fr + e4);
-          x[e4] = v.x; x[e4 + 1] = v.y; x[e4 + 2] = v.z; x[e4 + 3] = v.w;
-        }
-      }
-      float wv[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) wv[g] = -s_w[i * G + g];
-      axpy_g<G, EPL>(wv, x, acc);
-    }
-    __syncthreads();  // the staged rows are read before the reduction reuses them
-    reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part);
-    if (tid < G) { part[tid * PS] = s_m[tid]; part[tid * PS + 1] = -s_l[tid]; }
-  } else {
-    // -------------------------------------------------------------- attend
-    // chunks of 2 TR tokens of the unit's gather list: chunk x, then (when
-    // the clusters hold more tokens than the plan expected) x + n_splits,
-    // x + 2 n_splits, ...; the first chunk's list entries are read in the
-    // same round as the unit record, then the K and V rows of both tiles of
-    // a chunk are issued together
-    float qv[G][EPL];
-    load_q<T, D, G>(q, n_q_heads, b, h, sub, A.scale, qv);
-    pdl_wait();
-    const int32_t* gat = A.gather + (int64_t)u * A.gather_stride;
-    int32_t ge = -1;
-    {
-      const int t = (int)blockIdx.x * 2 * TR + tid;
-      if (tid < 2 * TR && t < A.gather_stride) ge = gat[t];  // valid below n_tok
-    }
-    if (tid < kInfoInts) s_info[tid] = A.info[(int64_t)u * kInfoInts + tid];
-    __syncthreads();
-    const int n_tok = (s_info[6] ? 0 : s_info[3]) + s_info[4];
-    T* const kt0 = ring;
-    T* const vt0 = ring + (size_t)2 * TR * D;
+  // exact attention over the tokens in s_row[0 .. n) (pool rows, -1 = skip):
+  // tiles of TR tokens stream through two ring slots (K and V tiles each),
+  // tile t + 2 issued as soon as tile t is consumed; online softmax carried
+  // in m_run / l_run / acc
+  auto attend_tokens = [&](int n) {
     const T* kbase = reinterpret_cast<const T*>(kp.base);
     const T* vbase = reinterpret_cast<const T*>(vp.base);
-    float m_run[G], l_run[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) { m_run[g] = -INFINITY; l_run[g] = 0.f; }
-    for (int ck = blockIdx.x; ck * 2 * TR < n_tok; ck += A.n_splits) {
-      const int t0 = ck * 2 * TR;
-      if (ck != (int)blockIdx.x) ge = (tid < 2 * TR && t0 + tid < n_tok) ? gat[t0 + tid] : -1;
-      if (tid < 2 * TR) s_row[tid / TR][tid % TR] = (t0 + tid < n_tok && ge >= 0) ? (int64_t)ge * D : -1;
-      __syncthreads();
-      const int ntile = (min(2 * TR, n_tok - t0) + TR - 1) / TR;
-      for (int bi = 0; bi < ntile; ++bi) {
-        T* kt = kt0 + (size_t)bi * TR * D;
-        T* vt = vt0 + (size_t)bi * TR * D;
+    const int ntile = (n + TR - 1) / TR;
+    auto issue = [&](int t) {
+      if (t < ntile) {
+        T* kt = ring + (size_t)(t & 1) * TR * D;
+        T* vt = ring + (size_t)(2 + (t & 1)) * TR * D;
         for (int i = tid; i < TR * LPR; i += blockDim.x) {
           const int r = i / LPR, ch = i - r * LPR;
-          const int64_t ro = s_row[bi][r];
-          if (ro >= 0) {
-            cp_async16(kt + r * D + ch * EPL, kbase + ro + ch * EPL);
-            cp_async16(vt + r * D + ch * EPL, vbase + ro + ch * EPL);
+          const int rr = t * TR + r;
+          const int32_t ri = rr < n ? s_row[rr] : -1;
+          if (ri >= 0) {
+            cp_async16(kt + r * D + ch * EPL, kbase + (int64_t)ri * D + ch * EPL);
+            cp_async16(vt + r * D + ch * EPL, vbase + (int64_t)ri * D + ch * EPL);
+          }
+        }
+      }
+      cp_async_commit();
+    };
+    issue(0);
+    issue(1);
+    constexpr int ITR = TR / (NW * RPW);   // row steps of a warp per tile
+    static_assert(TR % 32 == 0, "tile rows a multiple of the warp size");
+    for (int t = 0; t < ntile; ++t) {
+      cp_async_wait<1>();
+      __syncthreads();
+      const T* kt = ring + (size_t)(t & 1) * TR * D;
+      const T* vt = ring + (size_t)(2 + (t & 1)) * TR * D;
+      // scores: the warp's ITR row steps are independent (unrolled)
+#pragma unroll
+      for (int it = 0; it < ITR; ++it) {
+        const int r = (it * NW + warp) * RPW + rsub;
+        const int rr = t * TR + r;
+        const bool ok = rr < n && s_row[rr] >= 0;
+        float x[EPL];
+        if (ok) {
+          Elem<T>::unpack(*reinterpret_cast<const uint4*>(kt + r * D + sub * EPL), x);
+        } else {
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) x[e] = 0.f;
+        }
+        float a[G];
+        dot_g<G, EPL>(qv, x, a);
+        group_reduce_multi<G, LPR>(a, lane);
+        if (sub % (LPR / G) == 0) s_sc[r][jh] = ok ? a[0] : -INFINITY;
+      }
+      __syncthreads();
+      // softmax statistics of the tile for all heads at once (each warp
+      // redundantly, no barrier): lane holds rows lane, lane + 32, ...
+      float sv[TR / 32][G];
+#pragma unroll
+      for (int k = 0; k < TR / 32; ++k) load_row<G>(&s_sc[lane + 32 * k][0], sv[k]);
+      float mt[G], ps[G], corr[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        mt[g] = sv[0][g];
+#pragma unroll
+        for (int k = 1; k < TR / 32; ++k) mt[g] = fmaxf(mt[g], sv[k][g]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int g = 0; g < G; ++g) mt[g] = fmaxf(mt[g], __shfl_xor_sync(0xffffffffu, mt[g], o));
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float mnew = fmaxf(m_run[g], mt[g]);
+        corr[g] = mnew == -INFINITY ? 1.f : __expf(m_run[g] - mnew);
+        m_run[g] = mnew;
+        ps[g] = 0.f;
+#pragma unroll
+        for (int k = 0; k < TR / 32; ++k) {
+          sv[k][g] = sv[k][g] == -INFINITY ? 0.f : __expf(sv[k][g] - mnew);
+          ps[g] += sv[k][g];
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int g = 0; g < G; ++g) ps[g] += __shfl_xor_sync(0xffffffffu, ps[g], o);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        l_run[g] = l_run[g] * corr[g] + ps[g];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[g][e] *= corr[g];
+      }
+      __syncthreads();  // every warp has read the scores
+      if (warp == 0) {  // the weights e^(s - m) replace the scores
+#pragma unroll
+        for (int k = 0; k < TR / 32; ++k) store_row<G>(&s_sc[lane + 32 * k][0], sv[k]);
+      }
+      __syncthreads();
+#pragma unroll
+      for (int it = 0; it < ITR; ++it) {
+        const int r = (it * NW + warp) * RPW + rsub;
+        const int rr = t * TR + r;
+        if (!(rr < n && s_row[rr] >= 0)) continue;
+        float x[EPL];
+        Elem<T>::unpack(*reinterpret_cast<const uint4*>(vt + r * D + sub * EPL), x);
+        float pw[G];
+        load_row<G>(&s_sc[r][0], pw);
+        axpy_g<G, EPL>(pw, x, acc);
+      }
+      __syncthreads();  // slot t & 1 and s_sc are read before they are refilled
+      issue(t + 2);
+    }
+    cp_async_wait<0>();
+  };
+
+  pdl_wait();
+  if (role_range) {
+    // ---------------------------------------------------------- range CTA
+    const int c = (int)blockIdx.x * kRangeW + tid;
+    const bool inr = c < NC;
+    // one round: unit record, and this thread's cluster: key, affected
+    // index, offsets, scores
+    uint32_t key = 0u;
+    int af = 0, o0 = 0, o1 = 0;
+    float scv[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) scv[g] = 0.f;
+    int32_t* afp = A.aff_of + (int64_t)u * A.max_nc + c;
+    if (inr) {
+      key = A.keys[row0 + c];
+      af = *afp;
+      o0 = __ldg(off + c);
+      o1 = __ldg(off + c + 1);
+#pragma unroll
+      for (int g = 0; g < G; ++g) scv[g] = A.scores[(row0 + c) * G + g];
+    }
+    if (tid < kInfoInts) s_info[tid] = A.info[(int64_t)u * kInfoInts + tid];
+    __syncthreads();
+    if (af != 0) *afp = 0;  // consumed: clean for the next call
+    const bool dense = s_info[6] != 0;
+    const bool est = !dense && s_info[0] < s_info[7] && NC > 0;
+    const uint32_t kstar = (uint32_t)s_info[1];
+    const int thr = s_info[2];
+    const int cnt = o1 - o0;
+    const bool pk = inr && cnt > 0 &&
+                    (dense || (key != 0u && af >= 0 && (key > kstar || (key == kstar && c <= thr))));
+    int cw = 0, csel = 0;  // correction: count (-1: steady members, read below), row selector
+    if (est && inr && cnt > 0) {
+      if (pk || af < 0) { cw = cnt; csel = c; }
+      else if (af > 0 && key != 0u) { cw = -1; csel = ~(af - 1); }
+    }
+    int2 tot;
+    const int2 incl = block_inclusive_scan2(make_int2((pk ? 1 : 0) | ((cw != 0 ? 1 : 0) << 16), pk ? cnt : 0),
+                                            scan_sh, &tot);
+    const int n_pk = tot.x & 0xffff, n_ce = tot.x >> 16, n_tk = tot.y;
+    if (pk) {
+      const int i = (incl.x & 0xffff) - 1;
+      s_pkc[i] = af > 0 ? ~c : c;             // marked when it has steady members
+      s_pkt[i] = incl.y - cnt;
+      s_pko[i] = o0;
+    }
+    if (cw != 0) {
+      const int i = (incl.x >> 16) - 1;
+      s_cec[i] = csel;
+      s_cew[i] = cw;
+#pragma unroll
+      for (int g = 0; g < G; ++g) s_ces[i * G + g] = scv[g];
+    }
+    if (tid == 0 && !dense && n_pk > 0) {
+      s_base = atomicAdd(A.sel_n + u, n_pk);
+      atomicAdd(const_cast<int32_t*>(A.info) + (int64_t)u * kInfoInts + 3, n_tk);
+    }
+    __syncthreads();
+    if (pk && !dense) A.sel[row0 + s_base + (incl.x & 0xffff) - 1] = c;
+    // correction entries: the steady members' counts (loaded now, used after
+    // the exact part)
+    int as0 = 0, as1 = 0;
+    const bool need_dc = tid < n_ce && s_cew[tid] < 0;
+    if (need_dc) {
+      const int32_t* as = A.aff_start + (int64_t)u * (A.cap + 1) + ~s_cec[tid];
+      as0 = as[0];
+      as1 = as[1];
+    }
+    // exact part: the picked clusters' tokens, kRowCap per pass; each
+    // thread resolves two tokens with their loads (position, page) in flight
+    // together
+    const int32_t* pm = A.perm + geo.tok_row(b, h);
+    for (int p0 = 0; p0 < n_tk; p0 += kRowCap) {
+      const int np_ = min(kRowCap, n_tk - p0);
+      int slot2[2], cl2[2];
+      bool st2[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int t = p0 + tid + k * kStreamThreads;
+        slot2[k] = -1;
+        cl2[k] = 0;
+        st2[k] = false;
+        if (t < p0 + np_) {
+          int lo = 0, hi = n_pk - 1;  // largest i with s_pkt[i] <= t
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_pkt[mid] <= t) lo = mid; else hi = mid - 1;
+          }
+          slot2[k] = s_pko[lo] + (t - s_pkt[lo]);
+          cl2[k] = s_pkc[lo];
+        }
+      }
+      int pos2[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k)   // an affected cluster's tokens: steady?
+        pos2[k] = (slot2[k] >= 0 && cl2[k] < 0 && !dense) ? __ldg(pm + slot2[k]) : -1;
+      int32_t ro2[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int64_t ro = slot2[k] >= 0 ? pool_row(kp, geo.hkv, 1, b, h, slot2[k], status) : -1;
+        ro2[k] = (int32_t)ro;
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int t = tid + k * kStreamThreads;
+        if (t < np_) {
+          st2[k] = pos2[k] >= 0 && (pos2[k] < ns || pos2[k] >= wstart);
+          s_row[t] = st2[k] ? -1 : ro2[k];
+        }
+      }
+      __syncthreads();
+      attend_tokens(np_);
+      __syncthreads();
+    }
+    // correction part: -(cnt e^(s - mc) , e^(s - mc) row), kCorrRows rows per pass
+    float mc[G], lc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) { mc[g] = -INFINITY; lc[g] = 0.f; }
+    float cacc[G][EPL];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) cacc[g][e] = 0.f;
+    if (need_dc) s_cew[tid] = as1 - as0;
+    if (n_ce > 0) {
+      __syncthreads();  // the steady-member counts are written
+      if (warp < G) {   // per head: max, weights and denominator over the entries
+        float m = -INFINITY;
+        for (int i = lane; i < n_ce; i += 32) m = fmaxf(m, s_ces[i * G + warp]);
+        m = warp_max(m);
+        float l = 0.f;
+        for (int i = lane; i < n_ce; i += 32) {
+          const float w = __expf(s_ces[i * G + warp] - m);
+          s_ces[i * G + warp] = w;
+          l += (float)s_cew[i] * w;
+        }
+        l = warp_sum(l);
+        if (lane == 0) { s_m[warp] = m; s_l[warp] = l; }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int g = 0; g < G; ++g) { mc[g] = s_m[g]; lc[g] = s_l[g]; }
+      constexpr int CHF = D * 4 / 16, CHT = RS::ROWB / 16;
+      for (int p0 = 0; p0 < n_ce; p0 += kCorrRows) {
+        const int np_ = min(kCorrRows, n_ce - p0);
+        for (int k = tid; k < np_ * CHF; k += blockDim.x) {
+          const int i = k / CHF, ch = k - i * CHF;
+          const int sel_ = s_cec[p0 + i];
+          unsigned char* slot = s_crow + (size_t)i * D * 4;
+          if (sel_ >= 0) {
+            if (ch < CHT)
+              cp_async16(slot + ch * 16, reinterpret_cast<const unsigned char*>(vsum + (row0 + sel_) * D) + ch * 16);
+          } else {
+            cp_async16(slot + ch * 16,
+                       reinterpret_cast<const unsigned char*>(A.dv + ((int64_t)u * A.cap + ~sel_) * D) + ch * 16);
           }
         }
         cp_async_commit();
-      }
-      for (int bi = 0; bi < ntile; ++bi) {
-        if (bi == 0 && ntile > 1) cp_async_wait<1>(); else cp_async_wait<0>();
+        cp_async_wait<0>();
         __syncthreads();
-        const T* kt = kt0 + (size_t)bi * TR * D;
-        const T* vt = vt0 + (size_t)bi * TR * D;
-        for (int rb = warp * RPW; rb < TR; rb += NW * RPW) {
-          const int r = rb + rsub;
-          const int64_t ro = s_row[bi][r];
+        for (int rb = warp * RPW; rb < np_; rb += NW * RPW) {
+          const int i = rb + rsub;
+          if (i >= np_) continue;
+          const unsigned char* slot = s_crow + (size_t)i * D * 4;
           float x[EPL];
-          if (ro >= 0) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(kt + r * D + sub * EPL);
-            Elem<T>::unpack(raw, x);
+          if (s_cec[p0 + i] >= 0) {
+            Elem<T>::unpack(*reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(slot) + sub * EPL), x);
           } else {
+            const float* fr = reinterpret_cast<const float*>(slot) + sub * EPL;
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) x[e] = 0.f;
+            for (int e4 = 0; e4 < EPL; e4 += 4) {
+              const float4 v = *reinterpret_cast<const float4*>(fr + e4);
+              x[e4] = v.x; x[e4 + 1] = v.y; x[e4 + 2] = v.z; x[e4 + 3] = v.w;
+            }
           }
-          float a[G];
-          dot_g<G, EPL>(qv, x, a);
-          group_reduce_multi<G, LPR>(a, lane);
-          if (sub % (LPR / G) == 0) s_sc[r][jh] = ro >= 0 ? a[0] : -INFINITY;
+          float wv[G];
+#pragma unroll
+          for (int g = 0; g < G; ++g) wv[g] = s_ces[(p0 + i) * G + g];
+          axpy_g<G, EPL>(wv, x, cacc);
         }
         __syncthreads();
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          float mt = -INFINITY;
-          for (int r = lane; r < TR; r += 32) mt = fmaxf(mt, s_sc[r][g]);
-          mt = warp_max(mt);
-          const float mnew = fmaxf(m_run[g], mt);
-          const float corr = mnew == -INFINITY ? 1.f : __expf(m_run[g] - mnew);
-          float ps = 0.f;
-          for (int r = lane; r < TR; r += 32) {
-            const float sv = s_sc[r][g];
-            ps += sv == -INFINITY ? 0.f : __expf(sv - mnew);
-          }
-          ps = warp_sum(ps);
-          l_run[g] = l_run[g] * corr + ps;
-          m_run[g] = mnew;
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) acc[g][e] *= corr;
-        }
-        for (int rb = warp * RPW; rb < TR; rb += NW * RPW) {
-          const int r = rb + rsub;
-          if (s_row[bi][r] < 0) continue;
-          const uint4 raw = *reinterpret_cast<const uint4*>(vt + r * D + sub * EPL);
-          float x[EPL];
-          Elem<T>::unpack(raw, x);
-          float pw[G];
-#pragma unroll
-          for (int g = 0; g < G; ++g) pw[g] = __expf(s_sc[r][g] - m_run[g]);
-          axpy_g<G, EPL>(pw, x, acc);
-        }
       }
-      __syncthreads();  // this chunk's tiles and rows are read before the next chunk reuses them
     }
-    reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part);
-    if (tid == 0) {
+    // one part: exact minus correction at a common max
 #pragma unroll
-      for (int g = 0; g < G; ++g) { part[g * PS] = m_run[g]; part[g * PS + 1] = l_run[g]; }
+    for (int g = 0; g < G; ++g) {
+      const float M = fmaxf(m_run[g], mc[g]);
+      const float f1 = m_run[g] == -INFINITY ? 0.f : expf(m_run[g] - M);
+      const float f2 = mc[g] == -INFINITY ? 0.f : expf(mc[g] - M);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) acc[g][e] = acc[g][e] * f1 - cacc[g][e] * f2;
+      l_run[g] = l_run[g] * f1 - lc[g] * f2;
+      m_run[g] = M;
     }
+  } else {
+    // --------------------------------------------------------- steady CTA
+    // steady slots j0 .. j0 + 2 TR - 1 of the unit's (slot-sorted) steady list
+    const int j0 = ((int)blockIdx.x - A.n_rng) * 2 * TR;
+    if (tid < kInfoInts) s_info[tid] = A.info[(int64_t)u * kInfoInts + tid];
+    int32_t sl = -1;
+    if (tid < 2 * TR && j0 + tid < A.cap) sl = A.st_slot[(int64_t)u * A.cap + j0 + tid];
+    __syncthreads();
+    const int n_here = max(0, min(2 * TR, (s_info[6] ? 0 : s_info[4]) - j0));
+    if (tid < 2 * TR) s_row[tid] = tid < n_here ? (int32_t)pool_row(kp, geo.hkv, 1, b, h, sl, status) : -1;
+    __syncthreads();
+    if (n_here > 0) attend_tokens(n_here);
+  }
+  __syncthreads();
+  reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part);
+  if (tid == 0) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) { part[g * PS] = m_run[g]; part[g * PS + 1] = l_run[g]; }
   }
 
   // ---------------------------------------- last CTA of the unit merges
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(A.counters + u, 1) == A.n_splits + A.n_neg - 1;
+  if (tid == 0) s_last = atomicAdd(A.counters + u, 1) == A.n_rng + A.n_sc - 1;
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // parts: [attend splits | corrections | folded estimation parts]; a unit
-  // with nothing estimated (dense, or every candidate retrieved) merges the
-  // attend parts alone
+  // parts: [range CTAs | steady CTAs | folded estimation parts]; a unit with
+  // nothing estimated (dense, or every candidate retrieved) merges the
+  // first two groups alone
   const int32_t* I = A.info + (int64_t)u * kInfoInts;
-  const int np = (!I[6] && I[0] < I[7] && NC > 0) ? A.n_parts : A.n_splits;
-  // one round of loads: every part's (m, l) into shared memory, and this
-  // thread's first MB parts of its float4 output chunk into registers
-  constexpr int NCH = G * D / 4;                  // float4 chunks of one part's outputs
-  constexpr int PP = kStreamThreads / NCH > 0 ? kStreamThreads / NCH : 1;
-  constexpr int MB = 16;
-  float* f = s_w;                                   // [np][G] rescale factors
-  float* lp = reinterpret_cast<float*>(ring);       // [np][G] part denominators
-  const float* pbase = A.partials + (int64_t)u * A.n_parts * G * PS;
-  const int ch0 = tid % NCH, g0 = (ch0 * 4) / D, e0 = (ch0 * 4) - g0 * D;
-  const int pb = tid / NCH;
-  float4 v[MB];
-#pragma unroll
-  for (int k = 0; k < MB; ++k) {
-    const int p = pb + k * PP;
-    v[k] = (tid < NCH * PP && p < np)
-               ? __ldcg(reinterpret_cast<const float4*>(pbase + ((int64_t)p * G + g0) * PS + Part<D>::kO + e0))
-               : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+  const int np = (!I[6] && I[0] < I[7] && NC > 0) ? A.n_parts : A.n_rng + A.n_sc;
+  // the parts stream through the ring and the correction rows (contiguous)
+  // in batches: one cp.async round per batch, the first batch issued
+  // together with the loads of every part's (m, l)
+  constexpr int PFL = G * PS;                       // floats per part
+  const int bcap = max(1, (int)((4 * 16384 + kCorrRows * D * 4) / (PFL * 4)));
+  float* stage = reinterpret_cast<float*>(sh);
+  float* f = s_f;                                   // [np][G] rescale factors
+  float* lp = s_f + A.n_parts * G;                  // [np][G] part denominators
+  const float* pbase = A.partials + (int64_t)u * A.n_parts * PFL;
+  auto stage_batch = [&](int p0) {
+    const int nb = min(bcap, np - p0);
+    const float4* src = reinterpret_cast<const float4*>(pbase + (int64_t)p0 * PFL);
+    for (int i = tid; i < nb * PFL / 4; i += blockDim.x)
+      cp_async16(reinterpret_cast<float4*>(stage) + i, src + i);
+    cp_async_commit();
+  };
+  stage_batch(0);
   for (int i = tid; i < np * G; i += blockDim.x) {
     f[i] = __ldcg(pbase + (int64_t)i * PS);
     lp[i] = __ldcg(pbase + (int64_t)i * PS + 1);
@@ -1216,41 +1625,38 @@ wave_attend_estimate_kernel(const Geo geo, const T* __restrict__ q, int n_q_head
     const float mp = f[i];
     f[i] = mp == -INFINITY ? 0.f : expf(mp - s_m[i % G]);
   }
-  __syncthreads();
-  {
-    // thread t sums float4 chunk (t % NCH) over parts p = t / NCH, t / NCH + PP, ...
-    float4* red4 = reinterpret_cast<float4*>(lp + ((np * G + 3) & ~3));
-    for (int ch = ch0; ch < NCH; ch += kStreamThreads) {
-      const int g = (ch * 4) / D, e = (ch * 4) - g * D;
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (ch == ch0) {
+  // each thread: outputs tid, tid + 256, ... of the G x D block
+  constexpr int OPT = (G * D + kStreamThreads - 1) / kStreamThreads;
+  float o[OPT];
 #pragma unroll
-        for (int k = 0; k < MB; ++k) {
-          const int p = pb + k * PP;
-          const float w = p < np ? f[p * G + g] : 0.f;
-          o.x += w * v[k].x; o.y += w * v[k].y; o.z += w * v[k].z; o.w += w * v[k].w;
-        }
-      }
-      for (int p = (ch == ch0 ? pb + MB * PP : pb); p < np; p += PP) {
-        const float4 x = __ldcg(reinterpret_cast<const float4*>(pbase + ((int64_t)p * G + g) * PS + Part<D>::kO + e));
-        const float w = f[p * G + g];
-        o.x += w * x.x; o.y += w * x.y; o.z += w * x.z; o.w += w * x.w;
-      }
-      if (tid < NCH * PP) red4[tid] = o;
+  for (int k = 0; k < OPT; ++k) o[k] = 0.f;
+  for (int p0 = 0; p0 < np; p0 += bcap) {
+    if (p0 > 0) {
+      __syncthreads();  // the previous batch is consumed
+      stage_batch(p0);
     }
+    cp_async_wait<0>();
     __syncthreads();
-    for (int ch = tid; ch < NCH; ch += blockDim.x) {
-      float4 o = red4[ch];
-      for (int k = 1; k < PP; ++k) {
-        const float4 v = red4[ch + k * NCH];
-        o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
+    const int nb = min(bcap, np - p0);
+#pragma unroll
+    for (int k = 0; k < OPT; ++k) {
+      const int i = tid + k * kStreamThreads;
+      if (i < G * D) {
+        const int g = i / D, e = i - g * D;
+        float acc_o = o[k];
+        for (int p = 0; p < nb; ++p) acc_o += f[(p0 + p) * G + g] * stage[p * PFL + g * PS + Part<D>::kO + e];
+        o[k] = acc_o;
       }
-      const int g = (ch * 4) / D, e = (ch * 4) - g * D;
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < OPT; ++k) {
+    const int i = tid + k * kStreamThreads;
+    if (i < G * D) {
+      const int g = i / D, e = i - g * D;
       const float l = s_l[g];
-      const float inv = l > 0.f ? 1.f / l : 0.f;
       const int64_t qh = (int64_t)b * n_q_heads + (int64_t)h * G + g;
-      *reinterpret_cast<float4*>(A.out + qh * D + e) =
-          make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+      A.out[qh * D + e] = l > 0.f ? o[k] / l : 0.f;
       if (e == 0 && A.lse != nullptr) A.lse[qh] = l > 0.f ? s_m[g] + logf(l) : -INFINITY;
     }
   }
@@ -1296,21 +1702,23 @@ cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_
 
 }  // namespace
 
-size_t decode_attend_smem(int dtype, int D, int G, int wcap) {
-  (void)dtype; (void)D;
-  const size_t ring = 4 * 16384;  // also holds the correction rows and the reductions
-  return ring + (size_t)wcap * G * 4 + 2 * (size_t)kNegChunk * 4;
+size_t decode_attend_smem(int dtype, int D, int G, int n_parts) {
+  (void)dtype;
+  // ring (also the merge staging) | correction rows | merge factors and denominators
+  return 4 * 16384 + (size_t)kCorrRows * D * 4 + 2 * (size_t)n_parts * G * 4;
 }
 
-size_t decode_topk_smem(int max_nc, int cap, int bt_cap) {
-  return ((size_t)(max_nc + 31) / 32 + 4 * (size_t)cap + 2 + (size_t)bt_cap) * sizeof(int32_t);
+size_t decode_topk_smem(int max_nc, int cap) {
+  return ((size_t)(max_nc + 31) / 32 + (size_t)cap + 1) * sizeof(int32_t);
 }
 
-size_t decode_score_smem(int dtype, int D, int sort_pow2, int cap) {
+size_t decode_score_smem(int dtype, int D, int G, int sort_pow2, int cap) {
   const int rowb = D * (dtype == WI_BF16 ? 2 : 4);
-  const int crows = kScoreChunkBytes / rowb;
-  const size_t chunk = 2 * (size_t)kScoreChunkBytes + (size_t)kHistBins / 2 * 4 +
-                       (size_t)(crows + 4) * 4 + (size_t)crows * 8 * 4;
+  // stream CTA: ring | reduction | histogram | offsets | weights | q
+  const size_t chunk = 4 * 16384 + (size_t)(kStreamThreads / 32) * G * D * 4 +
+                       (size_t)kHistBins / 2 * 4 + (size_t)2 * (kScoreChunkBytes / rowb + 4) * 4 +
+                       (size_t)(kScoreChunkBytes / rowb) * G * 4 +
+                       (size_t)2 * G * D * (dtype == WI_BF16 ? 2 : 4);
   // steady role: sort keys (twice for the rank sort) | affected lists |
   // staged pool rows (offsets + rows, lists of up to kSteadyStage)
   const size_t steady = (size_t)8 * sort_pow2 * (sort_pow2 <= kSteadyRank ? 2 : 1) +
@@ -1319,23 +1727,61 @@ size_t decode_score_smem(int dtype, int D, int sort_pow2, int cap) {
   return std::max(chunk, steady);
 }
 
+namespace {
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library); null when unavailable
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// rows x 128 bf16 matrix, boxes of 64 rows x 64 columns, 128-byte swizzle
+bool encode_rows128(CUtensorMap* tm, const void* base, int64_t rows) {
+  auto fn = encode_fn();
+  if (!fn || rows <= 0) return false;
+  const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {128 * 2};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = kNumSMs;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+}  // namespace
+
 cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
   unsigned char* ws = a.ws;
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + p.off_status);
   float* scores = reinterpret_cast<float*>(ws + p.off_scores);
   uint32_t* keys = reinterpret_cast<uint32_t*>(ws + p.off_keys);
   int32_t* sel = reinterpret_cast<int32_t*>(ws + p.off_sel);
-  int32_t* seltok = reinterpret_cast<int32_t*>(ws + p.off_seltok);
+  int32_t* sel_n = reinterpret_cast<int32_t*>(ws + p.off_sel_n);
   int32_t* info = reinterpret_cast<int32_t*>(ws + p.off_info);
   int32_t* counters = reinterpret_cast<int32_t*>(ws + p.off_counters);
   int32_t* hist = reinterpret_cast<int32_t*>(ws + p.off_hist);
+  int32_t* aff_of = reinterpret_cast<int32_t*>(ws + p.off_aff_of);
   int32_t* st_slot = reinterpret_cast<int32_t*>(ws + p.off_st_slot);
   int32_t* st_cl = reinterpret_cast<int32_t*>(ws + p.off_st_cl);
   int32_t* aff_cl = reinterpret_cast<int32_t*>(ws + p.off_aff_cl);
   int32_t* aff_start = reinterpret_cast<int32_t*>(ws + p.off_aff_start);
   float* partials = reinterpret_cast<float*>(ws + p.off_partials);
   float* est_parts = reinterpret_cast<float*>(ws + p.off_est);
-  int32_t* gather = reinterpret_cast<int32_t*>(ws + p.off_gather);
   float* dv = reinterpret_cast<float*>(ws + p.off_dv);
   int32_t* nonc = reinterpret_cast<int32_t*>(ws + p.off_nonc);
   cudaEvent_t* ev = a.stage_events;
@@ -1345,36 +1791,61 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
   return with_types(p.dtype, p.D, p.G, [&]<typename T, int D, int G>() -> cudaError_t {
     const T* q = reinterpret_cast<const T*>(a.q);
     SteadyArgs sa{a.invperm, a.labels, a.offsets, a.vp, p.n_sink, p.window, p.cap, p.sort_pow2,
-                  st_slot, st_cl, aff_cl, aff_start, nonc, info, dv};
+                  st_slot, st_cl, aff_cl, aff_start, nonc, info, dv, aff_of, p.max_nc};
     cudaError_t e;
     mark(0);
-    const size_t score_smem = decode_score_smem(p.dtype, D, p.sort_pow2, p.cap);
-    cudaFuncSetAttribute(wave_score_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)score_smem);
-    e = launch_ex(wave_score_kernel<T, D, G>, dim3(p.n_score_blocks + 1, p.U),
-                  dim3(kStreamThreads), score_smem, s, false, p.geo, q, p.Hq,
-                  reinterpret_cast<const T*>(a.centroids), reinterpret_cast<const T*>(a.value_sums),
-                  a.offsets, scores, keys, hist, est_parts, p.scale, p.n_score_blocks, sa, status);
+    const size_t steady_smem = decode_score_smem(p.dtype, D, G, p.sort_pow2, p.cap);
+    const int n_tot = p.U * p.n_score_blocks;
+    e = cudaErrorInvalidValue;
+    bool done = false;
+    if constexpr (std::is_same_v<T, __nv_bfloat16> && D == 128) {
+      CUtensorMap tmc, tmv;
+      if (encode_rows128(&tmc, a.centroids, p.ncl) && encode_rows128(&tmv, a.value_sums, p.ncl)) {
+        const size_t smem = std::max(MmaSmem<G>::kTotal, steady_smem);
+        cudaFuncSetAttribute(wave_score_mma_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        int per_sm = 0;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, wave_score_mma_kernel<G>,
+                                                      kStreamThreads, smem);
+        const int n_stream = std::max(1, std::min(n_tot, std::max(1, per_sm) * sm_count() - p.U));
+        e = launch_ex(wave_score_mma_kernel<G>, dim3(p.U + n_stream), dim3(kStreamThreads), smem, s,
+                      false, p.geo, q, p.Hq, tmc, tmv, a.offsets, scores, keys, hist, est_parts,
+                      p.scale, p.n_score_blocks, n_stream, sa, status);
+        done = true;
+      }
+    }
+    if (!done) {
+      const size_t score_smem = steady_smem;
+      cudaFuncSetAttribute(wave_score_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)score_smem);
+      int per_sm = 0;
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, wave_score_kernel<T, D, G>,
+                                                    kStreamThreads, score_smem);
+      const int n_stream = std::max(1, std::min(n_tot, std::max(1, per_sm) * sm_count() - p.U));
+      e = launch_ex(wave_score_kernel<T, D, G>, dim3(p.U + n_stream), dim3(kStreamThreads),
+                    score_smem, s, false, p.geo, q, p.Hq, reinterpret_cast<const T*>(a.centroids),
+                    reinterpret_cast<const T*>(a.value_sums), a.offsets, scores, keys, hist,
+                    est_parts, p.scale, p.n_score_blocks, n_stream, sa, status);
+    }
     if (e != cudaSuccess) return e;
     mark(1);
-    const size_t topk_smem = decode_topk_smem(p.max_nc, p.cap, p.bt_cap);
+    const size_t topk_smem = decode_topk_smem(p.max_nc, p.cap);
     cudaFuncSetAttribute(wave_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)topk_smem);
-    FoldArgs fa{est_parts, p.n_score_blocks, partials, p.n_parts, p.n_splits + p.n_neg, G, D};
-    TopkArgs ta{keys, a.offsets, hist, nonc, st_slot, aff_cl, aff_start, p.cap, p.topk_clusters,
-                p.topk_fraction, sel, seltok, info, a.kp, gather, (int64_t)p.gather_stride, p.bt_cap};
+    FoldArgs fa{est_parts, p.n_score_blocks, partials, p.n_parts, p.n_rng + p.n_sc, G, D};
+    TopkArgs ta{keys, hist, nonc, p.cap, p.topk_clusters, p.topk_fraction, info, sel_n};
     e = launch_ex(wave_topk_kernel, dim3(1 + p.n_fold, p.U), dim3(kTopkThreads), topk_smem, s,
                   pdl, p.geo, ta, fa, status);
     if (e != cudaSuccess) return e;
     mark(2);
-    AttendArgs A{gather, aff_cl, aff_start, sel, dv, (int64_t)p.gather_stride, info, scores,
-                 keys, p.cap, p.n_splits, p.n_neg, p.n_parts, p.wcap, partials, counters,
+    AttendArgs A{keys, scores, info, aff_of, p.max_nc, aff_start, st_slot, dv, p.cap, a.perm,
+                 p.n_sink, p.window, sel, sel_n, p.n_rng, p.n_sc, p.n_parts, partials, counters,
                  a.out, a.lse, p.scale};
-    const size_t smem = decode_attend_smem(p.dtype, D, G, p.wcap);
-    cudaFuncSetAttribute(wave_attend_estimate_kernel<T, D, G>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    e = launch_ex(wave_attend_estimate_kernel<T, D, G>, dim3(p.n_splits + p.n_neg, p.U),
-                  dim3(kStreamThreads), smem, s, pdl, p.geo, q, p.Hq, a.kp, a.vp,
+    const size_t smem = decode_attend_smem(p.dtype, D, G, p.n_parts);
+    cudaFuncSetAttribute(wave_attend_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    e = launch_ex(wave_attend_kernel<T, D, G>, dim3(p.n_rng + p.n_sc, p.U), dim3(kStreamThreads),
+                  smem, s, pdl, p.geo, q, p.Hq, a.kp, a.vp,
                   reinterpret_cast<const T*>(a.value_sums), a.offsets, A, status);
     if (e != cudaSuccess) return e;
     mark(3);

@@ -16,8 +16,7 @@ constexpr int kInfoInts = 8;          // per-unit info record (see wi_decode_lay
 constexpr int kNumSMs = 148;          // B200
 constexpr int kScoreChunkBytes = 32768;  // centroid bytes (and as many value-sum bytes) per score CTA
 constexpr int kFold = 16;             // score-chunk parts folded into one by a K_B fold CTA
-constexpr int kNegRows = 128;         // clusters per correction CTA
-constexpr int kTopkBtCap = 16384;     // block-table entries the top-k may stage (64 KB)
+constexpr int kRangeClusters = 256;   // cluster ids per attend range CTA (one per thread)
 
 struct DecodePlan {
   Geo geo;
@@ -25,23 +24,21 @@ struct DecodePlan {
   int n_sink, window, topk_clusters;
   double topk_fraction;
   int max_nc;
+  int64_t ncl;               // centroid rows of the index (Hkv * sum NC_b)
   int seg_len, seg_clusters;  // segment length and clusters per full segment
   int score_chunk, n_score_blocks;   // clusters per score CTA, score CTAs per unit
   int cap;                 // steady-list capacity per unit (>= 1)
   int sort_pow2;           // shared-memory sort size for the steady list
-  int n_splits;            // exact-attention CTAs per unit
-  int n_neg;               // estimation-correction CTAs per unit
+  int n_rng;               // attend range CTAs per unit (kRangeW cluster ids each)
+  int n_sc;                // attend steady CTAs per unit (two tiles of steady slots each)
   int n_fold;              // fold CTAs per unit (kFold score parts each)
-  int n_parts;             // n_splits + n_neg + n_fold softmax parts per (unit, head)
-  int wcap;                // max(kNegRows, n_parts): weight / merge-factor rows
-  int bt_cap;              // block-table entries the top-k stages in shared memory
+  int n_parts;             // n_rng + n_sc + n_fold softmax parts per (unit, head)
   float scale;             // 1/sqrt(d)
-  // workspace byte offsets
-  size_t off_status, off_counters, off_hist, off_scores, off_keys, off_sel, off_seltok;
-  size_t off_info;
+  // workspace byte offsets; [0, off_scores) must be zero before the first call
+  size_t off_status, off_counters, off_hist, off_aff_of;
+  size_t off_scores, off_keys, off_sel, off_sel_n, off_info;
   size_t off_st_slot, off_st_cl, off_aff_cl, off_aff_start, off_partials;
-  size_t off_gather, off_dv, off_est, off_nonc;
-  int64_t gather_stride;   // gather-list entries per unit (max T_b)
+  size_t off_dv, off_est, off_nonc;
   size_t off_q, off_out, off_lse;
   size_t total;
 };
@@ -95,9 +92,9 @@ extern const char* const kDecodeStageNames[kDecodeStages];
 cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 wi_status decode_workspace_extent(const wi_index* idx, const wi_decode_params* p, size_t* total,
                                   size_t* zero_prefix);
-size_t decode_attend_smem(int dtype, int D, int G, int wcap);
-size_t decode_score_smem(int dtype, int D, int sort_pow2, int cap);
-size_t decode_topk_smem(int max_nc, int cap, int bt_cap);
+size_t decode_attend_smem(int dtype, int D, int G, int n_parts);
+size_t decode_score_smem(int dtype, int D, int G, int sort_pow2, int cap);
+size_t decode_topk_smem(int max_nc, int cap);
 cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s);
 cudaError_t launch_assign_only(const BuildPlan& p, const BuildArgs& a, const float* cent32,
                                int32_t* assign, cudaStream_t s);

@@ -99,7 +99,7 @@ def test_decode_workspace_size_and_layout():
                                               C.byref(lay)) == W.WI_OK
     assert lay.total_bytes == n and lay.status == 0
     assert 0 < lay.scores < lay.keys < lay.selected < lay.unit_info < n
-    assert lay.n_splits >= 1 and lay.n_est_chunks >= 1
+    assert lay.n_attend_ctas >= 2 and lay.n_score_ctas >= 1
 
 
 @pytest.mark.parametrize("over,expect", [

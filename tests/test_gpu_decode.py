@@ -65,26 +65,11 @@ def check_decode(wl, units, params, *, shuffle_seed=None, page_size=None, ref_de
             assert np.all(np.abs(tr.sel_score[diff] - kth) <= 1e-5 * abs(kth)), \
                 f"unit {(b, h)}: sets differ beyond near-ties"
             tr = O.decode_unit(qg, ix, params.n_sink, params.window, k, selected=gsel)
-        # gather plan: retrieved clusters' slots in id order (-1 for steady
-        # members), then the steady slots, as pool row indices
-        n_tok = int(info[u, 3]) + int(info[u, 4])
-        got_rows = W.gather_rows(ws, lay, u, n_tok).cpu().numpy().astype(np.int64)
-        T = len(ix.perm)
-        st_pos = O.steady_positions(T, params.n_sink, params.window)
-        st_slots = np.sort(ix.invperm[st_pos])
+        # the retrieved clusters' tokens, counted once each
         if info[u, 6]:
-            want_slots = np.arange(T)
+            assert int(info[u, 3]) == 0
         else:
-            parts = [np.arange(ix.offsets[c], ix.offsets[c + 1]) for c in gsel]
-            sel_slots = np.concatenate(parts) if parts else np.zeros(0, np.int64)
-            want_slots = np.concatenate([sel_slots, st_slots])
-            steady_in_sel = np.isin(sel_slots, st_slots)
-        bt = wx.block_table[b].cpu().numpy().astype(np.int64)
-        P = wx.page_size
-        want_rows = (bt[want_slots // P] * wl.n_kv_heads + h) * P + want_slots % P
-        if not info[u, 6]:
-            want_rows[:len(sel_slots)][steady_in_sel] = -1
-        assert np.array_equal(got_rows, want_rows), f"gather list of unit {(b, h)}"
+            assert int(info[u, 3]) == int(sum(ix.offsets[c + 1] - ix.offsets[c] for c in gsel))
         # (a3-a6) output and lse
         og = out_g[b, h * G:(h + 1) * G]
         err = H.rel_err(og, tr.out, wl.dtype)

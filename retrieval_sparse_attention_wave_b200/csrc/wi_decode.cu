@@ -301,9 +301,12 @@ struct Part {  // one softmax part of one (unit, q head): {m, l, -, -, o[D]}
   static constexpr int kO = 4;
 };
 
+// part.o[g][e] = sum over the CTA of acc (+ extra[g][e] * fac[g] when extra)
 template <int G, int EPL, int LPR, int D>
 __device__ __forceinline__ void reduce_and_store(float (&acc)[G][EPL], float* s_red, int warp,
-                                                 int sub, int rsub, float* part) {
+                                                 int sub, int rsub, float* part,
+                                                 const float* extra = nullptr,
+                                                 const float* fac = nullptr) {
   constexpr int NW = kStreamThreads / 32;
 #pragma unroll
   for (int g = 0; g < G; ++g)
@@ -320,7 +323,7 @@ __device__ __forceinline__ void reduce_and_store(float (&acc)[G][EPL], float* s_
   __syncthreads();
   for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
     const int g = i / D, e = i - g * D;
-    float v = 0.f;
+    float v = extra ? extra[g * D + e] * fac[g] : 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) v += s_red[(w * G + g) * D + e];
     part[g * Part<D>::kStride + Part<D>::kO + e] = v;
@@ -691,13 +694,13 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
     mbar_init_fence();
   }
   for (int i = tid; i < kHistBins / 2; i += blockDim.x) hist[i] = 0u;
+  issue_meta(0);   // the small loads first, ahead of the tiles
+  issue_meta(1);
   __syncthreads();
   if (tid == 0) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) issue_tile(i);
   }
-  issue_meta(0);
-  issue_meta(1);
 
   for (int kk = 0; kk < nk; ++kk) {
     const Chunk c = chunk(k0 + kk);
@@ -1224,6 +1227,13 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   __shared__ int scan_sh[64];
   __shared__ int s_info[kInfoInts], s_base, s_last;
   __shared__ float s_m[G], s_l[G];
+  // tensor-core exact attention (bf16, d = 128): tile weights, per-warp tile
+  // max / sum, the exact part's output and running (m, l)
+  constexpr bool kMma = std::is_same_v<T, __nv_bfloat16> && D == 128;
+  __shared__ __align__(16) float s_p[kMma ? G : 1][kMma ? 64 : 1];
+  __shared__ float s_wmax[NW][G], s_wsum[NW][G];
+  __shared__ __align__(16) float s_o[kMma ? G * D : 1];
+  __shared__ float s_em[G], s_el[G], s_f1[G];
 
   const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
   const int NC = geo.NC(b), Tb = geo.T(b);
@@ -1246,12 +1256,135 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   float m_run[G], l_run[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) { m_run[g] = -INFINITY; l_run[g] = 0.f; }
+  // MMA-path state: this lane's head gm = lane / 4 (valid below G), its
+  // column pair tq, q as A fragments, running (mr, lr) of head gm, and the
+  // output columns 16 warp .. 16 warp + 15 of head gm
+  const int gm = lane >> 2, tq = lane & 3;
+  uint32_t qa0[kMma ? 8 : 1], qa2[kMma ? 8 : 1];
+  float mr = -INFINITY, lr = 0.f;
+  float oacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  if constexpr (kMma) {
+    const uint32_t* qw = reinterpret_cast<const uint32_t*>(
+        q + ((int64_t)b * n_q_heads + (int64_t)h * G + (gm < G ? gm : 0)) * D);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      qa0[ks] = gm < G ? qw[8 * ks + tq] : 0u;
+      qa2[ks] = gm < G ? qw[8 * ks + 4 + tq] : 0u;
+    }
+    // rows no copy writes keep finite contents (zero weight times a finite row)
+    for (int i = tid; i < 4 * 16384 / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(sh)[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
 
   // exact attention over the tokens in s_row[0 .. n) (pool rows, -1 = skip):
   // tiles of TR tokens stream through two ring slots (K and V tiles each),
   // tile t + 2 issued as soon as tile t is consumed; online softmax carried
   // in m_run / l_run / acc
+  auto attend_tokens_mma = [&](int n) {
+    // tiles of 64 tokens: K rows into ring slot t & 1, V rows into slot
+    // 2 + (t & 1), each 16 KB slot two 128-byte-swizzled halves of 64 rows
+    const unsigned char* kb8 = reinterpret_cast<const unsigned char*>(kp.base);
+    const unsigned char* vb8 = reinterpret_cast<const unsigned char*>(vp.base);
+    unsigned char* r8 = reinterpret_cast<unsigned char*>(ring);
+    const int ntile = (n + 63) / 64;
+    auto issue = [&](int t) {
+      if (t < ntile) {
+        unsigned char* ks_ = r8 + (size_t)(t & 1) * 16384;
+        unsigned char* vs_ = r8 + (size_t)(2 + (t & 1)) * 16384;
+        for (int i = tid; i < 64 * 16; i += blockDim.x) {
+          const int r = i >> 4, ch = i & 15;
+          const int rr = t * 64 + r;
+          const int32_t ri = rr < n ? s_row[rr] : -1;
+          if (ri >= 0) {
+            const int o = (ch >> 3) * 8192 + swz128(r, ch & 7);
+            cp_async16(ks_ + o, kb8 + (int64_t)ri * 256 + ch * 16);
+            cp_async16(vs_ + o, vb8 + (int64_t)ri * 256 + ch * 16);
+          }
+        }
+      }
+      cp_async_commit();
+    };
+    issue(0);
+    issue(1);
+    for (int t = 0; t < ntile; ++t) {
+      cp_async_wait<1>();
+      __syncthreads();
+      const unsigned char* ks_ = r8 + (size_t)(t & 1) * 16384;
+      const unsigned char* vs_ = r8 + (size_t)(2 + (t & 1)) * 16384;
+      // scores of rows 8 warp .. 8 warp + 7
+      float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+      const int n0 = 8 * warp;
+#pragma unroll
+      for (int ks = 0; ks < 8; ks += 2) {
+        const int ch = 2 * ks + (lane >> 3);
+        uint32_t bm[4];
+        ldsm_x4(bm, ks_ + (ch >> 3) * 8192 + swz128(n0 + (lane & 7), ch & 7));
+        mma_bf16(sacc, qa0[ks], qa2[ks], bm[0], bm[1]);
+        mma_bf16(sacc, qa0[ks + 1], qa2[ks + 1], bm[2], bm[3]);
+      }
+      const int r0 = n0 + 2 * tq;
+      const bool v0 = t * 64 + r0 < n && s_row[t * 64 + r0] >= 0;
+      const bool v1 = t * 64 + r0 + 1 < n && s_row[t * 64 + r0 + 1] >= 0;
+      const float sc0 = v0 ? sacc[0] * A.scale : -INFINITY;
+      const float sc1 = v1 ? sacc[1] * A.scale : -INFINITY;
+      float mx = fmaxf(sc0, sc1);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      if (tq == 0 && gm < G) s_wmax[warp][gm] = mx;
+      __syncthreads();
+      float mt = -INFINITY;
+      if (gm < G) {
+#pragma unroll
+        for (int w = 0; w < NW; ++w) mt = fmaxf(mt, s_wmax[w][gm]);
+      }
+      const float mnew = fmaxf(mr, mt);
+      const float corr = mnew == -INFINITY ? 1.f : __expf(mr - mnew);
+      const float p0 = sc0 == -INFINITY ? 0.f : __expf(sc0 - mnew);
+      const float p1 = sc1 == -INFINITY ? 0.f : __expf(sc1 - mnew);
+      if (gm < G) *reinterpret_cast<float2*>(&s_p[gm][r0]) = make_float2(p0, p1);
+      float ps = p0 + p1;
+      ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+      ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+      if (tq == 0 && gm < G) s_wsum[warp][gm] = ps;
+      __syncthreads();
+      float lt = 0.f;
+      if (gm < G) {
+#pragma unroll
+        for (int w = 0; w < NW; ++w) lt += s_wsum[w][gm];
+      }
+      lr = lr * corr + lt;
+      mr = mnew;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oacc[nt][e] *= corr;
+      // P V for output columns 16 warp .. 16 warp + 15
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        uint32_t ah0 = 0u, al0 = 0u, ah2 = 0u, al2 = 0u;
+        if (gm < G) {
+          const float2 w01 = *reinterpret_cast<const float2*>(&s_p[gm][16 * ks + 2 * tq]);
+          const float2 w23 = *reinterpret_cast<const float2*>(&s_p[gm][16 * ks + 8 + 2 * tq]);
+          split_bf16(w01.x, w01.y, ah0, al0);
+          split_bf16(w23.x, w23.y, ah2, al2);
+        }
+        const int row = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int ch = 2 * warp + (lane >> 4);
+        uint32_t bm[4];
+        ldsm_x4_t(bm, vs_ + (ch >> 3) * 8192 + swz128(row, ch & 7));
+        mma_bf16(oacc[0], ah0, ah2, bm[0], bm[1]);
+        mma_bf16(oacc[0], al0, al2, bm[0], bm[1]);
+        mma_bf16(oacc[1], ah0, ah2, bm[2], bm[3]);
+        mma_bf16(oacc[1], al0, al2, bm[2], bm[3]);
+      }
+      __syncthreads();  // slots, s_p and the per-warp stats are read before reuse
+      issue(t + 2);
+    }
+    cp_async_wait<0>();
+  };
+
   auto attend_tokens = [&](int n) {
+    if constexpr (kMma) { attend_tokens_mma(n); return; }
     const T* kbase = reinterpret_cast<const T*>(kp.base);
     const T* vbase = reinterpret_cast<const T*>(vp.base);
     const int ntile = (n + TR - 1) / TR;
@@ -1358,6 +1491,24 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       issue(t + 2);
     }
     cp_async_wait<0>();
+  };
+
+  // MMA path: the exact part's output and (m, l) into shared memory, (m, l)
+  // into every thread's m_run / l_run
+  auto exact_to_shared = [&]() {
+    if constexpr (kMma) {
+      if (gm < G) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int d = 16 * warp + 8 * nt + 2 * tq;
+          *reinterpret_cast<float2*>(&s_o[gm * D + d]) = make_float2(oacc[nt][0], oacc[nt][1]);
+        }
+        if (warp == 0 && tq == 0) { s_em[gm] = mr; s_el[gm] = lr; }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int g = 0; g < G; ++g) { m_run[g] = s_em[g]; l_run[g] = s_el[g]; }
+    }
   };
 
   pdl_wait();
@@ -1474,6 +1625,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       attend_tokens(np_);
       __syncthreads();
     }
+    exact_to_shared();
     // correction part: -(cnt e^(s - mc) , e^(s - mc) row), kCorrRows rows per pass
     float mc[G], lc[G];
 #pragma unroll
@@ -1553,6 +1705,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       for (int e = 0; e < EPL; ++e) acc[g][e] = acc[g][e] * f1 - cacc[g][e] * f2;
       l_run[g] = l_run[g] * f1 - lc[g] * f2;
       m_run[g] = M;
+      if (tid == 0) s_f1[g] = f1;
     }
   } else {
     // --------------------------------------------------------- steady CTA
@@ -1566,9 +1719,12 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     if (tid < 2 * TR) s_row[tid] = tid < n_here ? (int32_t)pool_row(kp, geo.hkv, 1, b, h, sl, status) : -1;
     __syncthreads();
     if (n_here > 0) attend_tokens(n_here);
+    exact_to_shared();
+    if (tid < G) s_f1[tid] = 1.f;
   }
   __syncthreads();
-  reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part);
+  reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part, kMma ? s_o : nullptr,
+                                   kMma ? s_f1 : nullptr);
   if (tid == 0) {
 #pragma unroll
     for (int g = 0; g < G; ++g) { part[g * PS] = m_run[g]; part[g * PS + 1] = l_run[g]; }

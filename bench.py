@@ -48,6 +48,32 @@ def measured_peaks():
     return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
 
 
+def kernel_source_sha256() -> str:
+    """Hash of the CUDA sources (csrc/*.cu, *.cuh, *.h) in file-name order."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "retrieval_sparse_attention_wave_b200", "csrc", "*"))):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(f, "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(cfg: int, kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary of this
+    workload, or None when there is none or the kernels changed since."""
+    p = os.path.join(ROOT, "profiles", f"traffic_config{cfg}.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("kernel_source_sha256") != kernel_source_sha256():
+        return None
+    v = d.get("dram_bytes_per_launch", {}).get(kernel)
+    return float(v) if v is not None else None
+
+
 def workload_args(cfg: int):
     import wave_inputs as WI
     names = {1: "tiny fp32, T=4096, d=64, 1 q / 1 KV head",
@@ -352,7 +378,8 @@ def run_wave(args, rank, world, local_rank):
         "roofline_step": {"achieved": step_gbs, "peak": hbm, "unit": "GB/s",
                           "frac": step_gbs / hbm, "peak_kind": peak_kind},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": dom_gbs, "peak": hbm,
-                     "unit": "GB/s", "frac": dom_gbs / hbm, "traffic": None,
+                     "unit": "GB/s", "frac": dom_gbs / hbm,
+                     "traffic": measured_traffic(args.config, dom),
                      "bytes_per_launch": stage_bytes[dom], "us_per_launch": stage_us[dom],
                      "peak_kind": peak_kind},
         "stage_us": stage_us,

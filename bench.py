@@ -263,8 +263,12 @@ def run_wave(args, rank, world, local_rank):
     lses = [torch.empty(wl.batch, wl.n_q_heads, dtype=torch.float32, device=dev)
             for _ in range(R)]
 
+    # CUDA graphs: one per replica, and one with all R replicas back to back
+    # (the layers of one model step, as a serving engine captures them); the
+    # decode's first kernel is a plain launch, so layers never overlap
     stream = torch.cuda.Stream(device=dev)
     graphs = []
+    full = None
     with torch.cuda.stream(stream):
         for r in range(R):                      # warm every replica before capture
             W.decode(q, reps[r], params, out=outs[r], lse=lses[r], ws=ws, stream=stream)
@@ -275,17 +279,31 @@ def run_wave(args, rank, world, local_rank):
                 with torch.cuda.graph(g, stream=stream):
                     W.decode(q, reps[r], params, out=outs[r], lse=lses[r], ws=ws, stream=stream)
                 graphs.append(g)
+            full = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(full, stream=stream):
+                for r in range(R):
+                    W.decode(q, reps[r], params, out=outs[r], lse=lses[r], ws=ws, stream=stream)
 
-    def step(i):
-        r = i % R
-        if graphs:
+    def steps(n, per_layer_graphs=False):
+        """Exactly n decode steps (layer r of step i is replica i % R)."""
+        if not graphs:
+            for i in range(n):
+                r = i % R
+                W.decode(q, reps[r], params, out=outs[r], lse=lses[r], ws=ws, stream=stream)
+            return
+        if per_layer_graphs:
+            for i in range(n):
+                graphs[i % R].replay()
+            return
+        whole, rest = divmod(n, R)
+        for _ in range(whole):
+            full.replay()
+        for r in range(rest):
             graphs[r].replay()
-        else:
-            W.decode(q, reps[r], params, out=outs[r], lse=lses[r], ws=ws, stream=stream)
 
     with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            step(i)
+        steps(args.warmup)
+        steps(args.warmup, per_layer_graphs=True)
     stream.synchronize()
 
     dist = world > 1
@@ -297,11 +315,18 @@ def run_wave(args, rank, world, local_rank):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for i in range(args.steps):
-            step(i)
+        steps(args.steps)
         e1.record(stream)
     stream.synchronize()
     clk = clocks.stop()
+    # the same steps with one graph launch per layer decode (reported beside)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g0.record(stream)
+        steps(args.steps, per_layer_graphs=True)
+        g1.record(stream)
+    stream.synchronize()
+    per_layer_graph_us = max_over_ranks(g0.elapsed_time(g1), dev) * 1e3 / args.steps
     if dist:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -371,7 +396,9 @@ def run_wave(args, rank, world, local_rank):
                    "cluster_size": wl.cluster_size, "topk_fraction": wl.topk_fraction,
                    "n_sink": wl.n_sink, "window": wl.window,
                    "l2": f"rotate {R} layer replicas ({R * step_bytes / 1e6:.0f} MB per cycle > 2x L2)",
-                   "cuda_graph": not args.no_graph, "parallelism": f"replicas{world}"},
+                   "cuda_graph": (f"{R} layer decodes per graph" if not args.no_graph else False),
+                   "parallelism": f"replicas{world}"},
+        "us_per_step_one_graph_per_layer": per_layer_graph_us,
         "tokens_per_s": tokens * world / (us_per_step * 1e-6),
         "hbm_gbs": step_gbs,
         "step_bytes": step_bytes,

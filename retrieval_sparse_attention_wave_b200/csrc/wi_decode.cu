@@ -602,7 +602,8 @@ wave_score_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const T
 template <int G>
 struct MmaSmem {
   static constexpr int D = 128, CROWS = kScoreChunkBytes / (D * 2), TR = 64;
-  static constexpr size_t kRing = 4 * 16384;
+  static constexpr int kSlots = 6;                     // tiles in flight per CTA
+  static constexpr size_t kRing = (size_t)kSlots * 16384;
   static constexpr size_t kHist = (size_t)kHistBins / 2 * 4;
   static constexpr size_t kOff = (size_t)2 * (CROWS + 4) * 4;
   static constexpr size_t kW = (size_t)G * CROWS * 4;
@@ -627,7 +628,8 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
   static_assert(G <= 8, "at most 8 query heads per KV head (MMA rows 0..7)");
   extern __shared__ __align__(16) unsigned char sh_raw[];
   __shared__ float s_m[G], s_l[G];
-  __shared__ __align__(8) uint64_t s_bar[4];
+  constexpr int NS = SM::kSlots;
+  __shared__ __align__(8) uint64_t s_bar[SM::kSlots];
   pdl_launch_dependents();
   const int U = geo.batch * geo.hkv;
   if ((int)blockIdx.x < U) {
@@ -664,10 +666,10 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
     const int part = i & 3;
     const Chunk c = chunk(k0 + (i >> 2));
     const int r0 = (part & 1) * TR;
-    uint64_t* bar = &s_bar[i & 3];
+    uint64_t* bar = &s_bar[i % NS];
     if (c.nrows - r0 <= 0) { mbar_arrive(bar); return; }
     const CUtensorMap* tm = part < 2 ? &tm_cent : &tm_vsum;
-    unsigned char* dst = ring + (size_t)(i & 3) * 16384;
+    unsigned char* dst = ring + (size_t)(i % NS) * 16384;
     const int y = (int)(c.row0 + c.c0 + r0);
     fence_proxy_async();
     mbar_arrive_expect(bar, 16384u);
@@ -690,7 +692,7 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
   };
   if (tid == 0) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) mbar_init(&s_bar[i], 1);
+    for (int i = 0; i < NS; ++i) mbar_init(&s_bar[i], 1);
     mbar_init_fence();
   }
   for (int i = tid; i < kHistBins / 2; i += blockDim.x) hist[i] = 0u;
@@ -699,14 +701,16 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
   __syncthreads();
   if (tid == 0) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) issue_tile(i);
+    for (int i = 0; i < NS; ++i) issue_tile(i);
   }
+  // tile i sits in slot i % NS and completes phase (i / NS) & 1 of its barrier
+  auto tile_wait = [&](int i) { mbar_wait(&s_bar[i % NS], (uint32_t)((i / NS) & 1), status); };
+  auto tile_ptr = [&](int i) -> const unsigned char* { return ring + (size_t)(i % NS) * 16384; };
 
   for (int kk = 0; kk < nk; ++kk) {
     const Chunk c = chunk(k0 + kk);
     float* part = est_parts + ((int64_t)(k0 + kk)) * G * PS;
     const int* s_off = s_offb + (kk & 1) * (CROWS + 4);
-    const uint32_t par = kk & 1;
     cp_async_wait<1>();
     __syncthreads();
     // q as A fragments (rows = heads; heads >= G and rows 8..15 are zero)
@@ -722,8 +726,8 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
     // ---- scores: warp w takes the tile's rows 8w .. 8w + 7
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-      mbar_wait(&s_bar[t], par, status);
-      const unsigned char* slot = ring + (size_t)t * 16384;
+      tile_wait(4 * kk + t);
+      const unsigned char* slot = tile_ptr(4 * kk + t);
       if (c.nrows > t * TR) {
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         const int n0 = 8 * warp;
@@ -762,15 +766,15 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
         }
       }
       __syncthreads();
-      if (tid == 0) issue_tile(4 * kk + t + 4);
+      if (tid == 0) issue_tile(4 * kk + t + NS);
     }
     if (c.nrows == 0) {
       empty_part(part, G, PS);
 #pragma unroll
       for (int t = 2; t < 4; ++t) {
-        mbar_wait(&s_bar[t], par, status);
+        tile_wait(4 * kk + t);
         __syncthreads();
-        if (tid == 0) issue_tile(4 * kk + t + 4);
+        if (tid == 0) issue_tile(4 * kk + t + NS);
       }
       issue_meta(kk + 2);
       continue;
@@ -808,8 +812,8 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
     float oacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int t = 2; t < 4; ++t) {
-      mbar_wait(&s_bar[t], par, status);
-      const unsigned char* slot = ring + (size_t)t * 16384;
+      tile_wait(4 * kk + t);
+      const unsigned char* slot = tile_ptr(4 * kk + t);
       const int kb = (t - 2) * TR;
       // a tile past the chunk's rows was never loaded (its slot holds older
       // data, or none): skip it; in a loaded tile the rows past the chunk
@@ -835,7 +839,7 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
         mma_bf16(oacc[1], al0, al2, bm[2], bm[3]);
       }
       __syncthreads();
-      if (tid == 0) issue_tile(4 * kk + t + 4);
+      if (tid == 0) issue_tile(4 * kk + t + NS);
     }
     if (g < G) {
 #pragma unroll
@@ -848,10 +852,8 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
     issue_meta(kk + 2);
   }
   cp_async_wait<0>();
-  if (nk > 0) {
-#pragma unroll
-    for (int sl = 0; sl < 4; ++sl) mbar_wait(&s_bar[sl], (uint32_t)((nk - 1) & 1), status);
-  }
+  // the last tile of each slot (waited above; again, bounded, in case a wait gave up)
+  for (int i = max(0, 4 * nk - NS); i < 4 * nk; ++i) tile_wait(i);
 }
 
 // ----------------------------------------------------------------- K_B topk
@@ -1582,6 +1584,26 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     // exact part: the picked clusters' tokens, kRowCap per pass; each
     // thread resolves two tokens with their loads (position, page) in flight
     // together
+    // correction rows, first kCorrRows of them: staged now, in flight with the
+    // exact part's tiles (their group completes before the first tile's)
+    constexpr int CHF = D * 4 / 16, CHT = RS::ROWB / 16;
+    auto issue_corr = [&](int p0) {
+      const int np_ = min(kCorrRows, n_ce - p0);
+      for (int k = tid; k < np_ * CHF; k += blockDim.x) {
+        const int i = k / CHF, ch = k - i * CHF;
+        const int sel_ = s_cec[p0 + i];
+        unsigned char* slot = s_crow + (size_t)i * D * 4;
+        if (sel_ >= 0) {
+          if (ch < CHT)
+            cp_async16(slot + ch * 16, reinterpret_cast<const unsigned char*>(vsum + (row0 + sel_) * D) + ch * 16);
+        } else {
+          cp_async16(slot + ch * 16,
+                     reinterpret_cast<const unsigned char*>(A.dv + ((int64_t)u * A.cap + ~sel_) * D) + ch * 16);
+        }
+      }
+      cp_async_commit();
+    };
+    if (n_ce > 0) issue_corr(0);
     const int32_t* pm = A.perm + geo.tok_row(b, h);
     for (int p0 = 0; p0 < n_tk; p0 += kRowCap) {
       const int np_ = min(kRowCap, n_tk - p0);
@@ -1654,22 +1676,9 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       __syncthreads();
 #pragma unroll
       for (int g = 0; g < G; ++g) { mc[g] = s_m[g]; lc[g] = s_l[g]; }
-      constexpr int CHF = D * 4 / 16, CHT = RS::ROWB / 16;
       for (int p0 = 0; p0 < n_ce; p0 += kCorrRows) {
         const int np_ = min(kCorrRows, n_ce - p0);
-        for (int k = tid; k < np_ * CHF; k += blockDim.x) {
-          const int i = k / CHF, ch = k - i * CHF;
-          const int sel_ = s_cec[p0 + i];
-          unsigned char* slot = s_crow + (size_t)i * D * 4;
-          if (sel_ >= 0) {
-            if (ch < CHT)
-              cp_async16(slot + ch * 16, reinterpret_cast<const unsigned char*>(vsum + (row0 + sel_) * D) + ch * 16);
-          } else {
-            cp_async16(slot + ch * 16,
-                       reinterpret_cast<const unsigned char*>(A.dv + ((int64_t)u * A.cap + ~sel_) * D) + ch * 16);
-          }
-        }
-        cp_async_commit();
+        if (p0 > 0) issue_corr(p0);
         cp_async_wait<0>();
         __syncthreads();
         for (int rb = warp * RPW; rb < np_; rb += NW * RPW) {

@@ -234,6 +234,10 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* smem) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(smem_addr(smem)));
 }
+__device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], const void* smem) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1]) : "r"(smem_addr(smem)));
+}
 // d += a * b with a = {a0, 0, a2, 0} (rows 8..15 of A are zero)
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
   asm volatile(

@@ -41,7 +41,7 @@
 
 namespace wi {
 
-const char* const kDecodeStageNames[kDecodeStages] = {"score_estimate", "topk", "attend"};
+const char* const kDecodeStageNames[kDecodeStages] = {"score", "topk_estimate", "attend"};
 
 namespace {
 
@@ -587,18 +587,14 @@ wave_score_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const T
   }
 }
 
-// K_A on the tensor cores (bf16, d = 128).  Same chunking, ring and
-// pipeline as wave_score_kernel, with the two tiny contractions on mma.sync
-// m16n8k16 (bf16 in, fp32 accumulate): the CUDA-core form of this kernel is
-// issue-bound, not memory-bound, at G <= 8 query rows.
-//  scores:  S^T[g][r] = sum_d q[g][d] c[r][d]  (A = q, heads padded to 16 rows;
-//           B = centroid rows through ldmatrix), scaled by 1/sqrt(d) after;
-//  weights: o[g][d] = sum_r w[g][r] Vsum[r][d] (A = w split into two bf16
-//           terms, w = hi + lo to ~2^-17; B = value-sum rows through
-//           ldmatrix.trans).  Each warp owns 16 output columns, so no
-//           cross-warp reduction.
-// Tiles arrive by 2-D tensor copies (two 64-column boxes per 16 KB tile)
-// with the 128-byte swizzle, which makes every ldmatrix conflict-free.
+// K_A on the tensor cores (bf16, d = 128): the centroids alone.  Same
+// chunking as wave_score_kernel (128 clusters per chunk); a chunk's two
+// centroid tiles stream through a ring of NS 16 KB slots filled by 2-D tensor
+// copies (two 64-column boxes per tile, 128-byte swizzle, so ldmatrix is
+// conflict-free); scores S^T[g][r] = sum_d q[g][d] c[r][d] on mma.sync
+// m16n8k16 (A = q with the heads padded to 16 rows, B = centroid rows),
+// scaled by 1/sqrt(d) after.  The value sums stream in K_B's estimate CTAs,
+// beside the top-k.
 template <int G>
 struct MmaSmem {
   static constexpr int D = 128, CROWS = kScoreChunkBytes / (D * 2), TR = 64;
@@ -606,9 +602,8 @@ struct MmaSmem {
   static constexpr size_t kRing = (size_t)kSlots * 16384;
   static constexpr size_t kHist = (size_t)kHistBins / 2 * 4;
   static constexpr size_t kOff = (size_t)2 * (CROWS + 4) * 4;
-  static constexpr size_t kW = (size_t)G * CROWS * 4;
   static constexpr size_t kQ = (size_t)2 * G * D * 2;
-  static constexpr size_t oHist = kRing, oOff = oHist + kHist, oW = oOff + kOff, oQ = oW + kW,
+  static constexpr size_t oHist = kRing, oOff = oHist + kHist, oQ = oOff + kOff,
                           kTotal = oQ + kQ + 1024;   // + 1 KB to align the ring to 1024 B
 };
 
@@ -616,19 +611,14 @@ template <int G>
 __global__ void __launch_bounds__(kStreamThreads, 2)
 wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_q_heads,
                       const __grid_constant__ CUtensorMap tm_cent,
-                      const __grid_constant__ CUtensorMap tm_vsum,
                       const int32_t* __restrict__ offsets, float* __restrict__ scores,
-                      uint32_t* __restrict__ keys, int32_t* __restrict__ hist_g,
-                      float* __restrict__ est_parts, float scale, int n_chunks, int n_stream,
-                      const SteadyArgs sa, uint32_t* status) {
+                      uint32_t* __restrict__ keys, int32_t* __restrict__ hist_g, float scale,
+                      int n_chunks, int n_stream, const SteadyArgs sa, uint32_t* status) {
   using T = __nv_bfloat16;
   using SM = MmaSmem<G>;
-  constexpr int D = SM::D, CROWS = SM::CROWS, TR = SM::TR;
-  constexpr int PS = Part<D>::kStride;
+  constexpr int D = SM::D, CROWS = SM::CROWS, TR = SM::TR, NS = SM::kSlots;
   static_assert(G <= 8, "at most 8 query heads per KV head (MMA rows 0..7)");
   extern __shared__ __align__(16) unsigned char sh_raw[];
-  __shared__ float s_m[G], s_l[G];
-  constexpr int NS = SM::kSlots;
   __shared__ __align__(8) uint64_t s_bar[SM::kSlots];
   pdl_launch_dependents();
   const int U = geo.batch * geo.hkv;
@@ -641,7 +631,6 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
   unsigned char* ring = sh;
   uint32_t* hist = reinterpret_cast<uint32_t*>(sh + SM::oHist);
   int* s_offb = reinterpret_cast<int*>(sh + SM::oOff);
-  float* s_w = reinterpret_cast<float*>(sh + SM::oW);          // [G][CROWS]
   T* s_q = reinterpret_cast<T*>(sh + SM::oQ);
   const int sidx = blockIdx.x - U;
   const int n_tot = U * n_chunks;
@@ -661,22 +650,21 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
     c.row0 = geo.cl_row(c.b, c.h);
     return c;
   };
-  auto issue_tile = [&](int i) {   // thread 0
-    if (i >= 4 * nk) return;
-    const int part = i & 3;
-    const Chunk c = chunk(k0 + (i >> 2));
-    const int r0 = (part & 1) * TR;
+  // thread 0: tile i (chunk i / 2, centroid rows (i % 2) * TR ..) into slot i % NS
+  auto issue_tile = [&](int i) {
+    if (i >= 2 * nk) return;
+    const Chunk c = chunk(k0 + (i >> 1));
+    const int r0 = (i & 1) * TR;
     uint64_t* bar = &s_bar[i % NS];
     if (c.nrows - r0 <= 0) { mbar_arrive(bar); return; }
-    const CUtensorMap* tm = part < 2 ? &tm_cent : &tm_vsum;
     unsigned char* dst = ring + (size_t)(i % NS) * 16384;
     const int y = (int)(c.row0 + c.c0 + r0);
-    fence_proxy_async();
+    if (i >= NS) fence_proxy_async();   // the slot was read by the generic proxy
     mbar_arrive_expect(bar, 16384u);
-    tensor_load_2d(dst, tm, 0, y, bar);
-    tensor_load_2d(dst + 8192, tm, 64, y, bar);
+    tensor_load_2d(dst, &tm_cent, 0, y, bar);
+    tensor_load_2d(dst + 8192, &tm_cent, 64, y, bar);
   };
-  auto issue_meta = [&](int kk) {   // all threads
+  auto issue_meta = [&](int kk) {   // all threads: chunk kk's offsets and q
     if (kk < nk) {
       const Chunk c = chunk(k0 + kk);
       if (c.nrows > 0) {
@@ -705,29 +693,27 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
   }
   // tile i sits in slot i % NS and completes phase (i / NS) & 1 of its barrier
   auto tile_wait = [&](int i) { mbar_wait(&s_bar[i % NS], (uint32_t)((i / NS) & 1), status); };
-  auto tile_ptr = [&](int i) -> const unsigned char* { return ring + (size_t)(i % NS) * 16384; };
 
   for (int kk = 0; kk < nk; ++kk) {
     const Chunk c = chunk(k0 + kk);
-    float* part = est_parts + ((int64_t)(k0 + kk)) * G * PS;
     const int* s_off = s_offb + (kk & 1) * (CROWS + 4);
     cp_async_wait<1>();
     __syncthreads();
     // q as A fragments (rows = heads; heads >= G and rows 8..15 are zero)
     uint32_t qa0[D / 16], qa2[D / 16];
     {
-      const uint32_t* qw = reinterpret_cast<const uint32_t*>(s_q + (size_t)(kk & 1) * G * D + g * D);
+      const uint32_t* qw = reinterpret_cast<const uint32_t*>(s_q + (size_t)(kk & 1) * G * D + (g < G ? g : 0) * D);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         qa0[ks] = (g < G && c.nrows > 0) ? qw[8 * ks + tq] : 0u;
         qa2[ks] = (g < G && c.nrows > 0) ? qw[8 * ks + 4 + tq] : 0u;
       }
     }
-    // ---- scores: warp w takes the tile's rows 8w .. 8w + 7
+    // scores: warp w takes the tile's rows 8w .. 8w + 7
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-      tile_wait(4 * kk + t);
-      const unsigned char* slot = tile_ptr(4 * kk + t);
+      tile_wait(2 * kk + t);
+      const unsigned char* slot = ring + (size_t)((2 * kk + t) % NS) * 16384;
       if (c.nrows > t * TR) {
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         const int n0 = 8 * warp;
@@ -745,7 +731,6 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
         if (g < G) {
           if (ok0) scores[(c.row0 + c.c0 + rl) * G + g] = s0;
           if (ok1) scores[(c.row0 + c.c0 + rl + 1) * G + g] = s1;
-          *reinterpret_cast<float2*>(s_w + g * CROWS + rl) = make_float2(s0, s1);
         }
         float m0 = g < G ? s0 : -INFINITY, m1 = g < G ? s1 : -INFINITY;
 #pragma unroll
@@ -766,22 +751,9 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
         }
       }
       __syncthreads();
-      if (tid == 0) issue_tile(4 * kk + t + NS);
+      if (tid == 0) issue_tile(2 * kk + t + NS);
     }
-    if (c.nrows == 0) {
-      empty_part(part, G, PS);
-#pragma unroll
-      for (int t = 2; t < 4; ++t) {
-        tile_wait(4 * kk + t);
-        __syncthreads();
-        if (tid == 0) issue_tile(4 * kk + t + NS);
-      }
-      issue_meta(kk + 2);
-      continue;
-    }
-    // ---- histogram flush, chunk statistics (warp g: head g); weights of
-    // rows past the chunk's clusters are zero
-    {
+    if (c.nrows > 0) {  // histogram flush (two 16-bit counts per word)
       int* hg = hist_g + (int64_t)c.u * kHistBins;
       for (int i = tid; i < kHistBins / 2; i += blockDim.x) {
         const uint32_t w = hist[i];
@@ -792,68 +764,11 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
         }
       }
     }
-    if (warp < G) {
-      float* wr = s_w + warp * CROWS;
-      float m = -INFINITY;
-      for (int r = lane; r < c.nrows; r += 32) m = fmaxf(m, wr[r]);
-      m = warp_max(m);
-      float l = 0.f;
-      for (int r = lane; r < CROWS; r += 32) {
-        const int cnt = r < c.nrows ? s_off[r + 1] - s_off[r] : 0;
-        const float w = cnt > 0 ? __expf(wr[r] - m) : 0.f;
-        wr[r] = w;
-        l += (float)cnt * w;
-      }
-      l = warp_sum(l);
-      if (lane == 0) { s_m[warp] = m; s_l[warp] = l; }
-    }
-    __syncthreads();
-    // ---- weighted value sums: warp w owns output columns 16w .. 16w + 15
-    float oacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-    for (int t = 2; t < 4; ++t) {
-      tile_wait(4 * kk + t);
-      const unsigned char* slot = tile_ptr(4 * kk + t);
-      const int kb = (t - 2) * TR;
-      // a tile past the chunk's rows was never loaded (its slot holds older
-      // data, or none): skip it; in a loaded tile the rows past the chunk
-      // are real rows (or zero fill) with zero weight
-#pragma unroll
-      for (int ks = 0; ks < TR / 16; ++ks) {
-        if (c.nrows <= kb) break;
-        uint32_t ah0 = 0u, al0 = 0u, ah2 = 0u, al2 = 0u;
-        if (g < G) {
-          const float* wr = s_w + g * CROWS + kb + 16 * ks + 2 * tq;
-          const float2 w01 = *reinterpret_cast<const float2*>(wr);
-          const float2 w23 = *reinterpret_cast<const float2*>(wr + 8);
-          split_bf16(w01.x, w01.y, ah0, al0);
-          split_bf16(w23.x, w23.y, ah2, al2);
-        }
-        const int row = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
-        const int ch = 2 * warp + (lane >> 4);
-        uint32_t bm[4];
-        ldsm_x4_t(bm, slot + (ch >> 3) * 8192 + swz128(row, ch & 7));
-        mma_bf16(oacc[0], ah0, ah2, bm[0], bm[1]);
-        mma_bf16(oacc[0], al0, al2, bm[0], bm[1]);
-        mma_bf16(oacc[1], ah0, ah2, bm[2], bm[3]);
-        mma_bf16(oacc[1], al0, al2, bm[2], bm[3]);
-      }
-      __syncthreads();
-      if (tid == 0) issue_tile(4 * kk + t + NS);
-    }
-    if (g < G) {
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int d = 16 * warp + 8 * nt + 2 * tq;
-        *reinterpret_cast<float2*>(part + g * PS + Part<D>::kO + d) = make_float2(oacc[nt][0], oacc[nt][1]);
-      }
-    }
-    if (tid < G) { part[tid * PS] = s_m[tid]; part[tid * PS + 1] = s_l[tid]; }
     issue_meta(kk + 2);
   }
   cp_async_wait<0>();
   // the last tile of each slot (waited above; again, bounded, in case a wait gave up)
-  for (int i = max(0, 4 * nk - NS); i < 4 * nk; ++i) tile_wait(i);
+  for (int i = max(0, 2 * nk - NS); i < 2 * nk; ++i) tile_wait(i);
 }
 
 // ----------------------------------------------------------------- K_B topk
@@ -920,6 +835,155 @@ __device__ void fold_role(const FoldArgs& f, int u, int j) {
   }
 }
 
+// Estimate CTAs of K_B (blockIdx.x >= 1 on the tensor-core path): the
+// estimation parts of K_A's chunks, beside the top-k.  CTA x of unit u takes
+// chunks [x n / n_ev, (x+1) n / n_ev) of the unit's n chunks; a chunk's two
+// value-sum tiles stream through a ring of 2-D tensor copies issued before
+// the grid-dependency wait (the index does not depend on K_A), the chunk's
+// scores and offsets after it; per head: m = max s, w = cnt e^(s - m)
+// weights, l = sum cnt e^(s - m); o[g][d] = sum_r e^(s - m) Vsum[r][d] on
+// mma.sync (A = the weights split into two bf16 terms, B = value-sum rows
+// through ldmatrix.trans; warp w owns output columns 8w .. 8w + 7).
+struct EstArgs {
+  CUtensorMap tm_vsum;       // value sums: rows x 128 bf16, 64 x 64 boxes, 128-byte swizzle
+  const float* scores;       // [ncl][G]
+  const int32_t* offsets;
+  float* est_parts;          // [U][n_chunks][G][D+4]
+  int n_ev;                  // estimate CTAs per unit (0: K_A wrote the parts)
+  int n_chunks;              // score chunks per unit
+  int G;
+};
+constexpr int kEvSlots = 4;
+constexpr size_t kEvSmem = (size_t)kEvSlots * 16384 + 1024 + (size_t)8 * 128 * 4 +
+                           (size_t)2 * (128 + 4) * 4 + (size_t)2 * 128 * 8 * 4;
+
+__device__ void estimate_role(const Geo& geo, const EstArgs& ea, int u, int x, unsigned char* sh_raw,
+                              uint64_t* bars, uint32_t* status) {
+  constexpr int D = 128, CROWS = 128, TR = 64, NS = kEvSlots;
+  constexpr int PS = Part<D>::kStride;
+  __shared__ float s_m[8], s_l[8];
+  const int G = ea.G;
+  unsigned char* sh = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(sh_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* ring = sh;
+  float* s_w = reinterpret_cast<float*>(sh + (size_t)NS * 16384);        // [8][CROWS]
+  int* s_offb = reinterpret_cast<int*>(s_w + 8 * CROWS);                  // [2][CROWS + 4]
+  float* s_scb = reinterpret_cast<float*>(s_offb + 2 * (CROWS + 4));      // [2][CROWS][8]
+  const int b = u / geo.hkv, h = u - b * geo.hkv;
+  const int NC = geo.NC(b);
+  const int64_t row0 = geo.cl_row(b, h);
+  const int k0 = (int)((int64_t)x * ea.n_chunks / ea.n_ev);
+  const int k1 = (int)((int64_t)(x + 1) * ea.n_chunks / ea.n_ev);
+  const int nk = k1 - k0;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tq = lane & 3;
+  auto nrows_of = [&](int c) { return max(0, min(NC - c * CROWS, CROWS)); };
+  auto issue_tile = [&](int i) {   // thread 0: tile i = chunk k0 + i / 2, value rows (i % 2) * TR ..
+    if (i >= 2 * nk) return;
+    const int c = k0 + (i >> 1), r0 = (i & 1) * TR;
+    uint64_t* bar = &bars[i % NS];
+    if (nrows_of(c) - r0 <= 0) { mbar_arrive(bar); return; }
+    unsigned char* dst = ring + (size_t)(i % NS) * 16384;
+    const int y = (int)(row0 + (int64_t)c * CROWS + r0);
+    if (i >= NS) fence_proxy_async();   // the slot was read by the generic proxy
+    mbar_arrive_expect(bar, 16384u);
+    tensor_load_2d(dst, &ea.tm_vsum, 0, y, bar);
+    tensor_load_2d(dst + 8192, &ea.tm_vsum, 64, y, bar);
+  };
+  auto issue_meta = [&](int kk) {  // all threads: chunk kk's scores and offsets
+    if (kk < nk) {
+      const int c = k0 + kk, nr = nrows_of(c);
+      if (nr > 0) {
+        float* ss = s_scb + (size_t)(kk & 1) * CROWS * 8;
+        const float* sc = ea.scores + (row0 + (int64_t)c * CROWS) * G;
+        for (int i = tid; i < nr * G; i += blockDim.x) cp_async4(ss + i, sc + i);
+        int* so = s_offb + (kk & 1) * (CROWS + 4);
+        const int32_t* off = ea.offsets + geo.off_row(b, h) + c * CROWS;
+        for (int i = tid; i <= nr; i += blockDim.x) cp_async4(so + i, off + i);
+      }
+    }
+    cp_async_commit();
+  };
+  auto tile_wait = [&](int i) { mbar_wait(&bars[i % NS], (uint32_t)((i / NS) & 1), status); };
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int i = 0; i < 2; ++i) issue_tile(i);    // the index does not depend on K_A
+  pdl_wait();                                       // the scores do
+  issue_meta(0);                                    // small loads ahead of more tiles
+  issue_meta(1);
+  if (tid == 0)
+    for (int i = 2; i < NS; ++i) issue_tile(i);
+  for (int kk = 0; kk < nk; ++kk) {
+    const int c = k0 + kk, nr = nrows_of(c);
+    float* part = ea.est_parts + ((int64_t)u * ea.n_chunks + c) * G * PS;
+    const float* ss = s_scb + (size_t)(kk & 1) * CROWS * 8;
+    const int* so = s_offb + (kk & 1) * (CROWS + 4);
+    cp_async_wait<1>();
+    __syncthreads();
+    if (nr == 0) {
+      empty_part(part, G, PS);
+      for (int t = 0; t < 2; ++t) {
+        tile_wait(2 * kk + t);
+        __syncthreads();
+        if (tid == 0) issue_tile(2 * kk + t + NS);
+      }
+      issue_meta(kk + 2);
+      continue;
+    }
+    if (warp < G) {  // warp g: head g's max, weights and denominator
+      float* wr = s_w + warp * CROWS;
+      float m = -INFINITY;
+      for (int r = lane; r < nr; r += 32) m = fmaxf(m, ss[r * G + warp]);
+      m = warp_max(m);
+      float l = 0.f;
+      for (int r = lane; r < CROWS; r += 32) {
+        const int cnt = r < nr ? so[r + 1] - so[r] : 0;
+        const float w = cnt > 0 ? __expf(ss[r * G + warp] - m) : 0.f;
+        wr[r] = w;
+        l += (float)cnt * w;
+      }
+      l = warp_sum(l);
+      if (lane == 0) { s_m[warp] = m; s_l[warp] = l; }
+    }
+    __syncthreads();
+    float oacc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int t = 0; t < 2; ++t) {
+      tile_wait(2 * kk + t);
+      const unsigned char* slot = ring + (size_t)((2 * kk + t) % NS) * 16384;
+      if (nr > t * TR) {
+#pragma unroll
+        for (int ks = 0; ks < TR / 16; ++ks) {
+          uint32_t ah0 = 0u, al0 = 0u, ah2 = 0u, al2 = 0u;
+          if (g < G) {
+            const float* wr = s_w + g * CROWS + t * TR + 16 * ks + 2 * tq;
+            const float2 w01 = *reinterpret_cast<const float2*>(wr);
+            const float2 w23 = *reinterpret_cast<const float2*>(wr + 8);
+            split_bf16(w01.x, w01.y, ah0, al0);
+            split_bf16(w23.x, w23.y, ah2, al2);
+          }
+          const int row = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
+          uint32_t bm[2];
+          ldsm_x2_t(bm, slot + (warp >> 3) * 8192 + swz128(row, warp & 7));
+          mma_bf16(oacc, ah0, ah2, bm[0], bm[1]);
+          mma_bf16(oacc, al0, al2, bm[0], bm[1]);
+        }
+      }
+      __syncthreads();
+      if (tid == 0) issue_tile(2 * kk + t + NS);
+    }
+    if (g < G)
+      *reinterpret_cast<float2*>(part + g * PS + Part<D>::kO + 8 * warp + 2 * tq) = make_float2(oacc[0], oacc[1]);
+    if (tid < G) { part[tid * PS] = s_m[tid]; part[tid * PS + 1] = s_l[tid]; }
+    issue_meta(kk + 2);
+  }
+  cp_async_wait<0>();
+  for (int i = max(0, 2 * nk - NS); i < 2 * nk; ++i) tile_wait(i);
+}
+
 struct TopkArgs {
   const uint32_t* keys;
   int32_t* hist_g;
@@ -932,7 +996,7 @@ struct TopkArgs {
 };
 
 __global__ void __launch_bounds__(kTopkThreads)
-wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* status) {
+wave_topk_kernel(const Geo geo, const TopkArgs A, const __grid_constant__ EstArgs ea, uint32_t* status) {
   // dynamic shared: excluded bitmask [ceil(NCmax/32)] | non-candidates [cap+1]
   extern __shared__ __align__(16) int32_t sdyn[];
   __shared__ __align__(16) int hist[kHistBins];
@@ -941,10 +1005,11 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* s
   __shared__ int scan_sh[64];
   __shared__ int s_info[kInfoInts];
   __shared__ int s_ctl[8];
+  __shared__ __align__(8) uint64_t s_bars[kEvSlots];
   pdl_launch_dependents();
   if (blockIdx.x > 0) {
-    pdl_wait();
-    fold_role(fa, blockIdx.y, blockIdx.x - 1);
+    estimate_role(geo, ea, blockIdx.y, blockIdx.x - 1, reinterpret_cast<unsigned char*>(sdyn), s_bars,
+                  status);
     return;
   }
   constexpr int PT = kTopkPerLane;
@@ -994,9 +1059,9 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* s
   load_round(0);
   cp_async_wait<0>();
   __syncthreads();
-  for (int i = tid; i < kHistBins; i += nt) hg[i] = 0;   // clean for the next call
   if (tid == 0) { A.sel_n[u] = 0; I[3] = 0; }
   if (s_info[6]) {  // dense unit: every token is attended, nothing is selected
+    for (int i = tid; i < kHistBins; i += nt) hg[i] = 0;   // clean for the next call
     if (tid == 0) { I[0] = 0; I[1] = (int32_t)0xFFFFFFFFu; I[2] = -1; I[7] = 0; }
     return;
   }
@@ -1161,6 +1226,7 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const FoldArgs fa, uint32_t* s
     thr = s_ctl[4];
   }
   if (tid == 0) { I[0] = ksel; I[1] = (int32_t)kstar; I[2] = thr; I[7] = ncand; }
+  for (int i = tid; i < kHistBins; i += nt) hg[i] = 0;   // clean for the next call
 }
 
 // ----------------------------------------------------------------- K_C attend
@@ -1195,7 +1261,9 @@ struct AttendArgs {
   int n_sink, window;
   int32_t* sel;              // per unit, the retrieved clusters (unordered)
   int32_t* sel_n;            // [U] its counter
-  int n_rng, n_sc, n_parts;
+  const float* est_parts;    // [U][n_chunks][G][D+4], folded by the fold CTAs
+  int n_chunks;
+  int n_rng, n_sc, n_fold, n_parts;
   float* partials;
   int32_t* counters;
   float* out;
@@ -1245,6 +1313,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   const int64_t row0 = geo.cl_row(b, h);
   const int32_t* off = offsets + geo.off_row(b, h);
   const bool role_range = (int)blockIdx.x < A.n_rng;
+  const bool role_fold = (int)blockIdx.x >= A.n_rng + A.n_sc;
   float* part = A.partials + ((int64_t)u * A.n_parts + blockIdx.x) * G * PS;
   const int ns = min(A.n_sink, Tb), wstart = max(Tb - A.window, ns);
 
@@ -1514,7 +1583,10 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   };
 
   pdl_wait();
-  if (role_range) {
+  if (role_fold) {
+    FoldArgs fa{A.est_parts, A.n_chunks, A.partials, A.n_parts, A.n_rng + A.n_sc, G, D};
+    fold_role(fa, u, (int)blockIdx.x - A.n_rng - A.n_sc);
+  } else if (role_range) {
     // ---------------------------------------------------------- range CTA
     const int c = (int)blockIdx.x * kRangeW + tid;
     const bool inr = c < NC;
@@ -1731,18 +1803,20 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     exact_to_shared();
     if (tid < G) s_f1[tid] = 1.f;
   }
-  __syncthreads();
-  reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part, kMma ? s_o : nullptr,
-                                   kMma ? s_f1 : nullptr);
-  if (tid == 0) {
+  if (!role_fold) {
+    __syncthreads();
+    reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part, kMma ? s_o : nullptr,
+                                     kMma ? s_f1 : nullptr);
+    if (tid == 0) {
 #pragma unroll
-    for (int g = 0; g < G; ++g) { part[g * PS] = m_run[g]; part[g * PS + 1] = l_run[g]; }
+      for (int g = 0; g < G; ++g) { part[g * PS] = m_run[g]; part[g * PS + 1] = l_run[g]; }
+    }
   }
 
   // ---------------------------------------- last CTA of the unit merges
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(A.counters + u, 1) == A.n_rng + A.n_sc - 1;
+  if (tid == 0) s_last = atomicAdd(A.counters + u, 1) == A.n_rng + A.n_sc + A.n_fold - 1;
   __syncthreads();
   if (!s_last) return;
   __threadfence();
@@ -1962,10 +2036,18 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
     const size_t steady_smem = decode_score_smem(p.dtype, D, G, p.sort_pow2, p.cap);
     const int n_tot = p.U * p.n_score_blocks;
     e = cudaErrorInvalidValue;
+    // tensor-core path: K_A scores only, K_B's estimate CTAs stream the value sums
+    EstArgs ea{};
+    ea.scores = scores;
+    ea.offsets = a.offsets;
+    ea.est_parts = est_parts;
+    ea.n_chunks = p.n_score_blocks;
+    ea.G = G;
+    ea.n_ev = 0;
     bool done = false;
     if constexpr (std::is_same_v<T, __nv_bfloat16> && D == 128) {
-      CUtensorMap tmc, tmv;
-      if (encode_rows128(&tmc, a.centroids, p.ncl) && encode_rows128(&tmv, a.value_sums, p.ncl)) {
+      CUtensorMap tmc;
+      if (encode_rows128(&tmc, a.centroids, p.ncl) && encode_rows128(&ea.tm_vsum, a.value_sums, p.ncl)) {
         const size_t smem = std::max(MmaSmem<G>::kTotal, steady_smem);
         cudaFuncSetAttribute(wave_score_mma_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
@@ -1974,8 +2056,12 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
                                                       kStreamThreads, smem);
         const int n_stream = std::max(1, std::min(n_tot, std::max(1, per_sm) * sm_count() - p.U));
         e = launch_ex(wave_score_mma_kernel<G>, dim3(p.U + n_stream), dim3(kStreamThreads), smem, s,
-                      false, p.geo, q, p.Hq, tmc, tmv, a.offsets, scores, keys, hist, est_parts,
-                      p.scale, p.n_score_blocks, n_stream, sa, status);
+                      false, p.geo, q, p.Hq, tmc, a.offsets, scores, keys, hist, p.scale,
+                      p.n_score_blocks, n_stream, sa, status);
+        // two CTAs per SM in all (the top-k CTAs included), and at most four
+        // chunks per estimate CTA when there are many units
+        ea.n_ev = std::max(1, std::min(p.n_score_blocks,
+                                       std::max((2 * sm_count()) / p.U - 1, (p.n_score_blocks + 3) / 4)));
         done = true;
       }
     }
@@ -1994,22 +2080,21 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
     }
     if (e != cudaSuccess) return e;
     mark(1);
-    const size_t topk_smem = decode_topk_smem(p.max_nc, p.cap);
+    const size_t topk_smem = std::max(decode_topk_smem(p.max_nc, p.cap), ea.n_ev > 0 ? kEvSmem : 0);
     cudaFuncSetAttribute(wave_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)topk_smem);
-    FoldArgs fa{est_parts, p.n_score_blocks, partials, p.n_parts, p.n_rng + p.n_sc, G, D};
     TopkArgs ta{keys, hist, nonc, p.cap, p.topk_clusters, p.topk_fraction, info, sel_n};
-    e = launch_ex(wave_topk_kernel, dim3(1 + p.n_fold, p.U), dim3(kTopkThreads), topk_smem, s,
-                  pdl, p.geo, ta, fa, status);
+    e = launch_ex(wave_topk_kernel, dim3(1 + ea.n_ev, p.U), dim3(kTopkThreads), topk_smem, s,
+                  pdl, p.geo, ta, ea, status);
     if (e != cudaSuccess) return e;
     mark(2);
     AttendArgs A{keys, scores, info, aff_of, p.max_nc, aff_start, st_slot, dv, p.cap, a.perm,
-                 p.n_sink, p.window, sel, sel_n, p.n_rng, p.n_sc, p.n_parts, partials, counters,
-                 a.out, a.lse, p.scale};
+                 p.n_sink, p.window, sel, sel_n, est_parts, p.n_score_blocks, p.n_rng, p.n_sc,
+                 p.n_fold, p.n_parts, partials, counters, a.out, a.lse, p.scale};
     const size_t smem = decode_attend_smem(p.dtype, D, G, p.n_parts);
     cudaFuncSetAttribute(wave_attend_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    e = launch_ex(wave_attend_kernel<T, D, G>, dim3(p.n_rng + p.n_sc, p.U), dim3(kStreamThreads),
+    e = launch_ex(wave_attend_kernel<T, D, G>, dim3(p.n_rng + p.n_sc + p.n_fold, p.U), dim3(kStreamThreads),
                   smem, s, pdl, p.geo, q, p.Hq, a.kp, a.vp,
                   reinterpret_cast<const T*>(a.value_sums), a.offsets, A, status);
     if (e != cudaSuccess) return e;

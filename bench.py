@@ -144,16 +144,17 @@ def algorithmic_bytes(index, params, info: np.ndarray, n_st_per_seq):
     """Bytes the method must move in one decode step (centroids, value sums,
     offsets, retrieved K/V rows, steady K/V rows + invperm, q, out, lse), and
     the share each launch moves.  On the tensor-core path (bf16, d = 128) the
-    score launch reads centroids + offsets + q and the top-k launch's estimate
+    score launch reads centroids + offsets + q and the attend launch's range
     CTAs read the value sums; otherwise the score launch reads both.  The
     attend launch reads the retrieved and steady rows and writes out and lse.
-    Work partials and the correction's re-read of the retrieved clusters'
-    value sums are not counted (they are not the method's bytes)."""
+    Work partials, the steady members' dV rows and re-reads (offsets, scores,
+    keys between launches) are not counted: they are not the method's
+    bytes."""
     e = 2 if index.dtype == torch.bfloat16 else 4
     d = index.head_dim
     H = index.n_kv_heads
     tensor_path = index.dtype == torch.bfloat16 and d == 128
-    per_stage = {"score": 0, "topk_estimate": 0, "attend": 0}
+    per_stage = {"score": 0, "topk": 0, "attend": 0}
     total = 0
     for b, T in enumerate(index.seq_lens):
         NC = index.nc[b]
@@ -167,8 +168,7 @@ def algorithmic_bytes(index, params, info: np.ndarray, n_st_per_seq):
         steady = H * st * (2 * d * e + 4)
         qo = params.n_q_heads * d * e + params.n_q_heads * (d + 1) * 4
         per_stage["score"] += cent + offs + params.n_q_heads * d * e + (0 if tensor_path else vs)
-        per_stage["topk_estimate"] += vs if tensor_path else 0
-        per_stage["attend"] += retr + steady + params.n_q_heads * (d + 1) * 4
+        per_stage["attend"] += retr + steady + params.n_q_heads * (d + 1) * 4 + (vs if tensor_path else 0)
         total += cent + vs + offs + retr + steady + qo
     return total, per_stage
 
@@ -374,7 +374,7 @@ def run_wave(args, rank, world, local_rank):
 
     peaks, peak_kind = measured_peaks()
     hbm = float(peaks["hbm_gbs"])
-    dom = max(("score", "topk_estimate", "attend"), key=lambda k: stage_us[k])
+    dom = max(("score", "topk", "attend"), key=lambda k: stage_us[k])
     dom_gbs = stage_bytes[dom] / (stage_us[dom] * 1e-6) / 1e9
     step_gbs = step_bytes / (us_per_step * 1e-6) / 1e9
     tokens = sum(wl.seq_lens)

@@ -139,7 +139,10 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   const int tile_rows = 16384 / row_bytes;
   pl.n_rng = std::max<int>(1, (int)cdiv(max_nc, kRangeClusters));
   pl.n_sc = std::max<int>(1, (int)cdiv(cap, 2 * tile_rows));
-  pl.n_fold = std::max<int>(1, (int)cdiv(pl.n_score_blocks, kFold));
+  // the tensor-core path (bf16, d = 128) estimates inside the range CTAs;
+  // the CUDA-core path folds the score kernel's chunk parts
+  const bool mma = ix->dtype == WI_BF16 && pl.D == 128;
+  pl.n_fold = mma ? 0 : std::max<int>(1, (int)cdiv(pl.n_score_blocks, kFold));
   pl.n_parts = pl.n_rng + pl.n_sc + pl.n_fold;
   if (decode_attend_smem(pl.dtype, pl.D, G, pl.n_parts) + 24 * 1024 > 200 * 1024)
     return WI_ERR_UNSUPPORTED;
@@ -163,7 +166,7 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   pl.off_aff_start = take((size_t)pl.U * (cap + 1) * 4);
   pl.off_partials = take((size_t)pl.U * pl.n_parts * G * (pl.D + 4) * 4);
   pl.off_dv = take((size_t)pl.U * cap * pl.D * 4);
-  pl.off_est = take((size_t)pl.U * pl.n_score_blocks * G * (pl.D + 4) * 4);
+  pl.off_est = take(mma ? 0 : (size_t)pl.U * pl.n_score_blocks * G * (pl.D + 4) * 4);
   pl.off_nonc = take((size_t)pl.U * (cap + 1) * 4);
   const size_t nq = (size_t)ix->batch * p->n_q_heads;
   pl.off_q = take(nq * pl.D * esize(ix->dtype));

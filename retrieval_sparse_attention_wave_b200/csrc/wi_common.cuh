@@ -66,6 +66,23 @@ __device__ __forceinline__ int64_t pool_row(const Pool& p, int hkv, int d, int b
   return ((((int64_t)pg * hkv + h) << p.page_shift) + row) * d;
 }
 
+// pool_row with the page lookup supplied: `pg` is the block-table entry of
+// the slot's logical page (read earlier, e.g. staged in shared memory)
+__device__ __forceinline__ int64_t pool_row_pg(const Pool& p, int hkv, int d, int h, int slot, int pg,
+                                               uint32_t* status) {
+  const int lp = slot >> p.page_shift;
+  if (slot < 0 || lp >= p.max_pages) {
+    flag_error(status, WI_DEV_BAD_SLOT);
+    return -1;
+  }
+  if (pg < 0 || (int64_t)pg >= p.n_pages) {
+    flag_error(status, WI_DEV_BAD_PAGE);
+    return -1;
+  }
+  const int row = slot & ((1 << p.page_shift) - 1);
+  return ((((int64_t)pg * hkv + h) << p.page_shift) + row) * d;
+}
+
 // 16-byte streaming load (read-only path, no L1 allocation).
 __device__ __forceinline__ uint4 ld_stream(const void* ptr) {
   uint4 r;
@@ -245,6 +262,16 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a2
       " {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+// d += a * b with all four A registers: a0 / a2 rows 0..7, a1 / a3 rows
+// 8..15 (k 0..7 / 8..15 of each)
+__device__ __forceinline__ void mma_bf16_4(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                           uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9},"
+      " {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 // two floats as a bf16 pair (round to nearest even), low element first
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

@@ -5,31 +5,33 @@
 // forward_indexer).  Three launches, chained with programmatic dependent
 // launch so each one's prologue overlaps the previous one's tail:
 //
-//  K_A score    q . centroid / sqrt(d) for every cluster and q head, and the
-//               group-max selection key (item 2, the index lookup).  U extra
-//               CTAs resolve the steady zone (item 1): sink and window
-//               positions -> slots -> clusters, run-length encoded.
-//  K_B topk     exact radix select (11+11+10-bit digits) of the k best
-//               candidate clusters per KV head, ties to the lower id (Vortex
-//               2.C Top-K), and the gather plan (slot starts, token prefix,
-//               split boundaries).
-//  K_C attend + estimate
-//               attend CTAs: gather the retrieved clusters' rows and the
-//               steady rows from the cluster-permuted paged layout into
-//               shared memory (16-byte cp.async) and run split-K exact
-//               attention (items 1 and 2);
-//               estimate CTAs: prefetch their value-sum rows into a shared
-//               memory ring before waiting on K_B, then add every other
-//               candidate cluster as cnt' * e^s with value sum Vsum'
-//               (item 3 Estimation Zone);
-//               the last CTA of each unit merges all parts by log-sum-exp.
+//  K_A score    q . centroid / sqrt(d) for every cluster and q head, the
+//               group-max selection key and its first radix digit's
+//               histogram (item 2, the index lookup).  U extra CTAs resolve
+//               the steady zone (item 1): sink and window positions -> slots
+//               -> clusters, run-length encoded, and the steady members'
+//               value sums dV.  bf16 with d = 128: centroid tiles by 2-D
+//               tensor copies, scores on mma.sync.  Other shapes: FFMA over
+//               16-byte cp.async tiles, with every cluster's estimation term
+//               folded in during the same pass over the value sums.
+//  K_B topk     exact radix select of the k best candidate clusters per KV
+//               head (a threshold key and id), ties to the lower id (Vortex
+//               2.C Top-K).
+//  K_C attend   range CTAs pick their range's retrieved clusters against the
+//               threshold, resolve the tokens' pool rows and run exact
+//               attention over them (items 1 and 2) together with the
+//               range's estimation zone (item 3); steady CTAs attend the
+//               steady zone; the last CTA of each unit merges every part by
+//               log-sum-exp.
 //
-// The score / estimate GEMVs have M = G <= 8 rows, so they run on the CUDA
-// cores (FFMA); every row is spread over LPR = d*sizeof(T)/16 lanes.
+// The score and estimation contractions have M = G <= 8 rows: on the tensor
+// cores the heads are padded to the 16 rows of an m16n8k16 tile; on the CUDA
+// cores every row is spread over LPR = d*sizeof(T)/16 lanes.
 #include <cfloat>
 #include <climits>
 #include <algorithm>
 #include <cmath>
+#include <cstring>
 #include <mutex>
 #include <type_traits>
 
@@ -41,7 +43,7 @@
 
 namespace wi {
 
-const char* const kDecodeStageNames[kDecodeStages] = {"score", "topk_estimate", "attend"};
+const char* const kDecodeStageNames[kDecodeStages] = {"score", "topk", "attend"};
 
 namespace {
 
@@ -108,7 +110,8 @@ struct SteadyArgs {
   int n_sink, window, cap, sort_pow2;
   int32_t *st_slot, *st_cl, *aff_cl, *aff_start, *nonc, *info;
   float* dv;       // [U][cap][D] fp32: sum of the steady members' values per affected cluster
-  int32_t* aff_of; // [U][max_nc]: +(j+1) for affected cluster j, -(j+1) if not a candidate
+  int32_t* aff_of; // [U][max_nc]: affected cluster j: (j+1) | (its steady members << 16),
+                   // or -(j+1) when none of its members is left (not a candidate)
   int max_nc;
 };
 
@@ -235,7 +238,8 @@ __device__ void steady_role(const Geo& geo, int u, const SteadyArgs& a, uint32_t
       const int full = __ldg(off + c + 1) - __ldg(off + c);
       const bool none_left = full - (s_ast[i + 1] - s_ast[i]) <= 0;
       if (none_left) nonc[1 + atomicAdd(&s_nnc, 1)] = c;
-      a.aff_of[(int64_t)u * a.max_nc + c] = none_left ? -(i + 1) : i + 1;
+      a.aff_of[(int64_t)u * a.max_nc + c] =
+          none_left ? -(i + 1) : (i + 1) | ((s_ast[i + 1] - s_ast[i]) << 16);
     }
     if (staged) s_ro[i] = pool_row(a.vp, geo.hkv, D, b, h, (int)(srt[i] >> 32), status);
   }
@@ -301,7 +305,8 @@ struct Part {  // one softmax part of one (unit, q head): {m, l, -, -, o[D]}
   static constexpr int kO = 4;
 };
 
-// part.o[g][e] = sum over the CTA of acc (+ extra[g][e] * fac[g] when extra)
+// part.o[g][e] = sum over the CTA of acc (+ extra[g][e] * fac[g] when extra;
+// fac null: 1)
 template <int G, int EPL, int LPR, int D>
 __device__ __forceinline__ void reduce_and_store(float (&acc)[G][EPL], float* s_red, int warp,
                                                  int sub, int rsub, float* part,
@@ -323,7 +328,7 @@ __device__ __forceinline__ void reduce_and_store(float (&acc)[G][EPL], float* s_
   __syncthreads();
   for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
     const int g = i / D, e = i - g * D;
-    float v = extra ? extra[g * D + e] * fac[g] : 0.f;
+    float v = extra ? extra[g * D + e] * (fac ? fac[g] : 1.f) : 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) v += s_red[(w * G + g) * D + e];
     part[g * Part<D>::kStride + Part<D>::kO + e] = v;
@@ -593,8 +598,8 @@ wave_score_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const T
 // copies (two 64-column boxes per tile, 128-byte swizzle, so ldmatrix is
 // conflict-free); scores S^T[g][r] = sum_d q[g][d] c[r][d] on mma.sync
 // m16n8k16 (A = q with the heads padded to 16 rows, B = centroid rows),
-// scaled by 1/sqrt(d) after.  The value sums stream in K_B's estimate CTAs,
-// beside the top-k.
+// scaled by 1/sqrt(d) after.  The value sums are read by the attend
+// kernel's range CTAs, which estimate their own clusters.
 template <int G>
 struct MmaSmem {
   static constexpr int D = 128, CROWS = kScoreChunkBytes / (D * 2), TR = 64;
@@ -793,10 +798,11 @@ constexpr int kTopkRound = kTopkThreads * kTopkPerLane;   // 8192 ids per round
 constexpr int kTopkCand = 1024;
 constexpr int kTopkCand2 = 256;
 
-// Fold CTAs of K_B (blockIdx.x >= 1, beside the unit's top-k CTA): each
-// log-sum-exp combines kFold consecutive chunk parts of K_A into one part of
-// the unit's final merge, so the merge reads a few parts instead of one per
-// 32 KB chunk.  All loads of a fold are issued before the first use.
+// Fold CTAs of the attend kernel (CUDA-core path, where K_A writes one
+// estimation part per 32 KB chunk): each log-sum-exp combines kFold
+// consecutive chunk parts into one part of the unit's final merge, so the
+// merge reads a few parts instead of one per chunk.  All loads of a fold are
+// issued before the first use.
 struct FoldArgs {
   const float* est_parts;   // [U][n_chunks][G][D+4]
   int n_chunks;
@@ -835,155 +841,6 @@ __device__ void fold_role(const FoldArgs& f, int u, int j) {
   }
 }
 
-// Estimate CTAs of K_B (blockIdx.x >= 1 on the tensor-core path): the
-// estimation parts of K_A's chunks, beside the top-k.  CTA x of unit u takes
-// chunks [x n / n_ev, (x+1) n / n_ev) of the unit's n chunks; a chunk's two
-// value-sum tiles stream through a ring of 2-D tensor copies issued before
-// the grid-dependency wait (the index does not depend on K_A), the chunk's
-// scores and offsets after it; per head: m = max s, w = cnt e^(s - m)
-// weights, l = sum cnt e^(s - m); o[g][d] = sum_r e^(s - m) Vsum[r][d] on
-// mma.sync (A = the weights split into two bf16 terms, B = value-sum rows
-// through ldmatrix.trans; warp w owns output columns 8w .. 8w + 7).
-struct EstArgs {
-  CUtensorMap tm_vsum;       // value sums: rows x 128 bf16, 64 x 64 boxes, 128-byte swizzle
-  const float* scores;       // [ncl][G]
-  const int32_t* offsets;
-  float* est_parts;          // [U][n_chunks][G][D+4]
-  int n_ev;                  // estimate CTAs per unit (0: K_A wrote the parts)
-  int n_chunks;              // score chunks per unit
-  int G;
-};
-constexpr int kEvSlots = 4;
-constexpr size_t kEvSmem = (size_t)kEvSlots * 16384 + 1024 + (size_t)8 * 128 * 4 +
-                           (size_t)2 * (128 + 4) * 4 + (size_t)2 * 128 * 8 * 4;
-
-__device__ void estimate_role(const Geo& geo, const EstArgs& ea, int u, int x, unsigned char* sh_raw,
-                              uint64_t* bars, uint32_t* status) {
-  constexpr int D = 128, CROWS = 128, TR = 64, NS = kEvSlots;
-  constexpr int PS = Part<D>::kStride;
-  __shared__ float s_m[8], s_l[8];
-  const int G = ea.G;
-  unsigned char* sh = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(sh_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* ring = sh;
-  float* s_w = reinterpret_cast<float*>(sh + (size_t)NS * 16384);        // [8][CROWS]
-  int* s_offb = reinterpret_cast<int*>(s_w + 8 * CROWS);                  // [2][CROWS + 4]
-  float* s_scb = reinterpret_cast<float*>(s_offb + 2 * (CROWS + 4));      // [2][CROWS][8]
-  const int b = u / geo.hkv, h = u - b * geo.hkv;
-  const int NC = geo.NC(b);
-  const int64_t row0 = geo.cl_row(b, h);
-  const int k0 = (int)((int64_t)x * ea.n_chunks / ea.n_ev);
-  const int k1 = (int)((int64_t)(x + 1) * ea.n_chunks / ea.n_ev);
-  const int nk = k1 - k0;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, tq = lane & 3;
-  auto nrows_of = [&](int c) { return max(0, min(NC - c * CROWS, CROWS)); };
-  auto issue_tile = [&](int i) {   // thread 0: tile i = chunk k0 + i / 2, value rows (i % 2) * TR ..
-    if (i >= 2 * nk) return;
-    const int c = k0 + (i >> 1), r0 = (i & 1) * TR;
-    uint64_t* bar = &bars[i % NS];
-    if (nrows_of(c) - r0 <= 0) { mbar_arrive(bar); return; }
-    unsigned char* dst = ring + (size_t)(i % NS) * 16384;
-    const int y = (int)(row0 + (int64_t)c * CROWS + r0);
-    if (i >= NS) fence_proxy_async();   // the slot was read by the generic proxy
-    mbar_arrive_expect(bar, 16384u);
-    tensor_load_2d(dst, &ea.tm_vsum, 0, y, bar);
-    tensor_load_2d(dst + 8192, &ea.tm_vsum, 64, y, bar);
-  };
-  auto issue_meta = [&](int kk) {  // all threads: chunk kk's scores and offsets
-    if (kk < nk) {
-      const int c = k0 + kk, nr = nrows_of(c);
-      if (nr > 0) {
-        float* ss = s_scb + (size_t)(kk & 1) * CROWS * 8;
-        const float* sc = ea.scores + (row0 + (int64_t)c * CROWS) * G;
-        for (int i = tid; i < nr * G; i += blockDim.x) cp_async4(ss + i, sc + i);
-        int* so = s_offb + (kk & 1) * (CROWS + 4);
-        const int32_t* off = ea.offsets + geo.off_row(b, h) + c * CROWS;
-        for (int i = tid; i <= nr; i += blockDim.x) cp_async4(so + i, off + i);
-      }
-    }
-    cp_async_commit();
-  };
-  auto tile_wait = [&](int i) { mbar_wait(&bars[i % NS], (uint32_t)((i / NS) & 1), status); };
-  if (tid == 0) {
-    for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
-    mbar_init_fence();
-  }
-  __syncthreads();
-  if (tid == 0)
-    for (int i = 0; i < 2; ++i) issue_tile(i);    // the index does not depend on K_A
-  pdl_wait();                                       // the scores do
-  issue_meta(0);                                    // small loads ahead of more tiles
-  issue_meta(1);
-  if (tid == 0)
-    for (int i = 2; i < NS; ++i) issue_tile(i);
-  for (int kk = 0; kk < nk; ++kk) {
-    const int c = k0 + kk, nr = nrows_of(c);
-    float* part = ea.est_parts + ((int64_t)u * ea.n_chunks + c) * G * PS;
-    const float* ss = s_scb + (size_t)(kk & 1) * CROWS * 8;
-    const int* so = s_offb + (kk & 1) * (CROWS + 4);
-    cp_async_wait<1>();
-    __syncthreads();
-    if (nr == 0) {
-      empty_part(part, G, PS);
-      for (int t = 0; t < 2; ++t) {
-        tile_wait(2 * kk + t);
-        __syncthreads();
-        if (tid == 0) issue_tile(2 * kk + t + NS);
-      }
-      issue_meta(kk + 2);
-      continue;
-    }
-    if (warp < G) {  // warp g: head g's max, weights and denominator
-      float* wr = s_w + warp * CROWS;
-      float m = -INFINITY;
-      for (int r = lane; r < nr; r += 32) m = fmaxf(m, ss[r * G + warp]);
-      m = warp_max(m);
-      float l = 0.f;
-      for (int r = lane; r < CROWS; r += 32) {
-        const int cnt = r < nr ? so[r + 1] - so[r] : 0;
-        const float w = cnt > 0 ? __expf(ss[r * G + warp] - m) : 0.f;
-        wr[r] = w;
-        l += (float)cnt * w;
-      }
-      l = warp_sum(l);
-      if (lane == 0) { s_m[warp] = m; s_l[warp] = l; }
-    }
-    __syncthreads();
-    float oacc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int t = 0; t < 2; ++t) {
-      tile_wait(2 * kk + t);
-      const unsigned char* slot = ring + (size_t)((2 * kk + t) % NS) * 16384;
-      if (nr > t * TR) {
-#pragma unroll
-        for (int ks = 0; ks < TR / 16; ++ks) {
-          uint32_t ah0 = 0u, al0 = 0u, ah2 = 0u, al2 = 0u;
-          if (g < G) {
-            const float* wr = s_w + g * CROWS + t * TR + 16 * ks + 2 * tq;
-            const float2 w01 = *reinterpret_cast<const float2*>(wr);
-            const float2 w23 = *reinterpret_cast<const float2*>(wr + 8);
-            split_bf16(w01.x, w01.y, ah0, al0);
-            split_bf16(w23.x, w23.y, ah2, al2);
-          }
-          const int row = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
-          uint32_t bm[2];
-          ldsm_x2_t(bm, slot + (warp >> 3) * 8192 + swz128(row, warp & 7));
-          mma_bf16(oacc, ah0, ah2, bm[0], bm[1]);
-          mma_bf16(oacc, al0, al2, bm[0], bm[1]);
-        }
-      }
-      __syncthreads();
-      if (tid == 0) issue_tile(2 * kk + t + NS);
-    }
-    if (g < G)
-      *reinterpret_cast<float2*>(part + g * PS + Part<D>::kO + 8 * warp + 2 * tq) = make_float2(oacc[0], oacc[1]);
-    if (tid < G) { part[tid * PS] = s_m[tid]; part[tid * PS + 1] = s_l[tid]; }
-    issue_meta(kk + 2);
-  }
-  cp_async_wait<0>();
-  for (int i = max(0, 2 * nk - NS); i < 2 * nk; ++i) tile_wait(i);
-}
-
 struct TopkArgs {
   const uint32_t* keys;
   int32_t* hist_g;
@@ -996,7 +853,7 @@ struct TopkArgs {
 };
 
 __global__ void __launch_bounds__(kTopkThreads)
-wave_topk_kernel(const Geo geo, const TopkArgs A, const __grid_constant__ EstArgs ea, uint32_t* status) {
+wave_topk_kernel(const Geo geo, const TopkArgs A, uint32_t* status) {
   // dynamic shared: excluded bitmask [ceil(NCmax/32)] | non-candidates [cap+1]
   extern __shared__ __align__(16) int32_t sdyn[];
   __shared__ __align__(16) int hist[kHistBins];
@@ -1005,18 +862,12 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const __grid_constant__ EstArg
   __shared__ int scan_sh[64];
   __shared__ int s_info[kInfoInts];
   __shared__ int s_ctl[8];
-  __shared__ __align__(8) uint64_t s_bars[kEvSlots];
   pdl_launch_dependents();
-  if (blockIdx.x > 0) {
-    estimate_role(geo, ea, blockIdx.y, blockIdx.x - 1, reinterpret_cast<unsigned char*>(sdyn), s_bars,
-                  status);
-    return;
-  }
   constexpr int PT = kTopkPerLane;
   constexpr int NW = kTopkThreads / 32;
   const int tid = threadIdx.x, nt = kTopkThreads, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
-  const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
+  const int u = blockIdx.x, b = u / geo.hkv, h = u - b * geo.hkv;
   const int NC = geo.NC(b);
   const int nmask = (NC + 31) >> 5;
   const int cap = A.cap;
@@ -1233,25 +1084,34 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, const __grid_constant__ EstArg
 // range CTAs (kRangeW cluster ids each): pick the retrieved clusters of the
 // range against K_B's threshold, append them to the unit's (unordered)
 // selection list, resolve their tokens' pool rows (skipping steady members)
-// and run exact attention over them; in the same part, take back out of
-// the estimate what K_A's chunk parts counted that the estimation zone
-// leaves out: every retrieved cluster and every cluster left without a
-// non-steady member in full (cnt, Vsum), and the steady members (their
-// count, dV) of the other affected clusters;
+// and run exact attention over them.  The estimation zone of the range goes
+// into the same part:
+//  - tensor-core path (bf16, d = 128): the range's value sums (64 KB) are
+//    brought into shared memory by 2-D tensor copies issued before the
+//    grid-dependency wait, so they land while the top-k runs; after the
+//    picks, o_e = sum over the zone of e^(s - m_e) Vsum on mma.sync and
+//    l_e = sum of (cnt - steady members) e^(s - m_e); the steady members'
+//    value sums dV of the zone's affected clusters are taken back out;
+//  - CUDA-core path: K_A's chunk parts counted every cluster, so the range
+//    CTA takes back out what the zone leaves out: every retrieved cluster and
+//    every cluster left without a non-steady member in full (cnt, Vsum), and
+//    the steady members (their count, dV) of the other affected clusters;
+//    fold CTAs combine K_A's chunk parts into a few merge parts;
 // steady CTAs (two tiles of steady slots each): exact attention over the
 // steady zone;
-// the last CTA of each unit merges these parts and K_B's folded estimation
-// parts by log-sum-exp.
+// the last CTA of each unit merges the parts by log-sum-exp.
 constexpr int kRangeW = kRangeClusters;    // clusters per range CTA, one per thread
 static_assert(kRangeW == kStreamThreads, "one cluster per thread");
 constexpr int kCorrRows = 32;              // correction rows staged per pass
 constexpr int kRowCap = 512;               // tokens resolved per pass of a range CTA
+constexpr int kBtStage = 2 * kRangeW;      // block-table entries a range CTA stages
 
 struct AttendArgs {
   const uint32_t* keys;
   const float* scores;
   const int32_t* info;
-  int32_t* aff_of;           // [U][max_nc]: +(j+1) affected, -(j+1) non-candidate; reset here
+  int32_t* aff_of;           // [U][max_nc]: (j+1) | (steady members << 16) affected,
+                             // -(j+1) non-candidate; reset here
   int max_nc;
   const int32_t* aff_start;  // [U][cap+1]
   const int32_t* st_slot;    // [U][cap]
@@ -1275,16 +1135,21 @@ template <typename T, int D, int G>
 __global__ void __launch_bounds__(kStreamThreads, G * Elem<T>::kPerVec >= 64 ? 1 : 2)
 wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const Pool kp,
                    const Pool vp, const T* __restrict__ vsum,
-                   const int32_t* __restrict__ offsets, const AttendArgs A, uint32_t* status) {
+                   const int32_t* __restrict__ offsets, const AttendArgs A,
+                   const __grid_constant__ CUtensorMap tm_vsum, uint32_t* status) {
   using RS = RowShape<T, D>;
   constexpr int EPL = RS::EPL, LPR = RS::LPR, RPW = RS::RPW, TR = RS::TILE;
   constexpr int NW = kStreamThreads / 32;
   constexpr int PS = Part<D>::kStride;
   static_assert(TR % (NW * RPW) == 0, "tile must be a multiple of rows per CTA step");
   static_assert(2 * TR <= kStreamThreads, "one thread per token of a chunk");
-  extern __shared__ __align__(16) unsigned char sh[];
-  // dynamic: [ring 64 KB: K x2, V x2 tiles; the cross-warp reduction and the
-  //           merge reuse it] [correction rows kCorrRows x D fp32] [merge factors]
+  extern __shared__ __align__(16) unsigned char sh_raw[];
+  // dynamic, from the first 1024-byte boundary (the tensor copies' swizzle
+  // repeats every 1024 bytes of address): [ring 64 KB: K x2, V x2 tiles, or
+  // the range's value sums; the cross-warp reduction and the merge reuse it]
+  // [correction rows kCorrRows x D fp32] [merge factors]
+  unsigned char* sh = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(sh_raw) + 1023) & ~uintptr_t(1023));
   T* ring = reinterpret_cast<T*>(sh);
   float* s_red = reinterpret_cast<float*>(sh);
   unsigned char* s_crow = sh + 4 * 16384;
@@ -1293,17 +1158,24 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   __shared__ __align__(16) float s_sc[TR][G];
   __shared__ int s_pkc[kRangeW], s_pkt[kRangeW], s_pko[kRangeW];   // picked: id, token start, slot start
   __shared__ int s_cec[kRangeW], s_cew[kRangeW];                   // correction: row selector, count
-  __shared__ float s_ces[kRangeW * G];                              // correction: scores -> weights
   __shared__ int scan_sh[64];
-  __shared__ int s_info[kInfoInts], s_base, s_last;
+  __shared__ int s_info[kInfoInts], s_base, s_last, s_lp0;
   __shared__ float s_m[G], s_l[G];
   // tensor-core exact attention (bf16, d = 128): tile weights, per-warp tile
   // max / sum, the exact part's output and running (m, l)
   constexpr bool kMma = std::is_same_v<T, __nv_bfloat16> && D == 128;
-  __shared__ __align__(16) float s_p[kMma ? G : 1][kMma ? 64 : 1];
+  __shared__ int32_t s_bt[kMma ? kBtStage : 1];      // block-table window of a range CTA
+  __shared__ __align__(16) float s_ces[kMma ? 1 : kRangeW * G];   // correction: scores -> weights
+  // MMA A operands in bf16, high terms in rows 0..7 (head g = row g), low
+  // terms in rows 8..15, rows of heads >= G zero; padded rows (144 / 528
+  // bytes) keep ldmatrix conflict-free: a tile's weights, and a range CTA's
+  // estimation weights
+  __shared__ __align__(16) __nv_bfloat16 s_P[kMma ? 16 : 1][kMma ? 72 : 1];
+  __shared__ __align__(16) __nv_bfloat16 s_W[kMma ? 16 : 1][kMma ? kRangeW + 8 : 1];
   __shared__ float s_wmax[NW][G], s_wsum[NW][G];
   __shared__ __align__(16) float s_o[kMma ? G * D : 1];
   __shared__ float s_em[G], s_el[G], s_f1[G];
+  __shared__ __align__(8) uint64_t s_vbar;          // the range's value sums have landed
 
   const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
   const int NC = geo.NC(b), Tb = geo.T(b);
@@ -1329,7 +1201,9 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   for (int g = 0; g < G; ++g) { m_run[g] = -INFINITY; l_run[g] = 0.f; }
   // MMA-path state: this lane's head gm = lane / 4 (valid below G), its
   // column pair tq, q as A fragments, running (mr, lr) of head gm, and the
-  // output columns 16 warp .. 16 warp + 15 of head gm
+  // output columns 16 warp .. 16 warp + 15 of head gm: in oacc[nt][0..1]
+  // the products of the weights' high bf16 terms (A rows 0..7), in
+  // oacc[nt][2..3] those of their low terms (A rows 8..15), summed at the end
   const int gm = lane >> 2, tq = lane & 3;
   uint32_t qa0[kMma ? 8 : 1], qa2[kMma ? 8 : 1];
   float mr = -INFINITY, lr = 0.f;
@@ -1342,9 +1216,32 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       qa0[ks] = gm < G ? qw[8 * ks + tq] : 0u;
       qa2[ks] = gm < G ? qw[8 * ks + 4 + tq] : 0u;
     }
-    // rows no copy writes keep finite contents (zero weight times a finite row)
-    for (int i = tid; i < 4 * 16384 / 16; i += blockDim.x)
-      reinterpret_cast<uint4*>(sh)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (role_range) {
+      // the range's 256 value-sum rows (index data, independent of the
+      // previous kernels): four 64-row tiles, each two 64-column boxes, fill
+      // the ring (rows past the last cluster row are zero-filled)
+      if (tid == 0) {
+        mbar_init(&s_vbar, 1);
+        mbar_init_fence();
+        mbar_arrive_expect(&s_vbar, 4u * 16384u);
+        const int y0 = (int)(row0 + (int64_t)blockIdx.x * kRangeW);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          tensor_load_2d(sh + t * 16384, &tm_vsum, 0, y0 + 64 * t, &s_vbar);
+          tensor_load_2d(sh + t * 16384 + 8192, &tm_vsum, 64, y0 + 64 * t, &s_vbar);
+        }
+      }
+    } else {
+      // rows no copy writes keep finite contents (zero weight times a finite row)
+      for (int i = tid; i < 4 * 16384 / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(sh)[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    // the A operands' rows that no head writes stay zero
+    for (int i = tid; i < (int)(sizeof(s_P) / 16); i += blockDim.x)
+      reinterpret_cast<uint4*>(&s_P[0][0])[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (role_range)
+      for (int i = tid; i < (int)(sizeof(s_W) / 16); i += blockDim.x)
+        reinterpret_cast<uint4*>(&s_W[0][0])[i] = make_uint4(0u, 0u, 0u, 0u);
   }
 
   // exact attention over the tokens in s_row[0 .. n) (pool rows, -1 = skip):
@@ -1412,7 +1309,12 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       const float corr = mnew == -INFINITY ? 1.f : __expf(mr - mnew);
       const float p0 = sc0 == -INFINITY ? 0.f : __expf(sc0 - mnew);
       const float p1 = sc1 == -INFINITY ? 0.f : __expf(sc1 - mnew);
-      if (gm < G) *reinterpret_cast<float2*>(&s_p[gm][r0]) = make_float2(p0, p1);
+      if (gm < G) {
+        uint32_t hi, lo;
+        split_bf16(p0, p1, hi, lo);
+        *reinterpret_cast<uint32_t*>(&s_P[gm][r0]) = hi;
+        *reinterpret_cast<uint32_t*>(&s_P[8 + gm][r0]) = lo;
+      }
       float ps = p0 + p1;
       ps += __shfl_xor_sync(0xffffffffu, ps, 1);
       ps += __shfl_xor_sync(0xffffffffu, ps, 2);
@@ -1429,26 +1331,20 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) oacc[nt][e] *= corr;
-      // P V for output columns 16 warp .. 16 warp + 15
+      // P V for output columns 16 warp .. 16 warp + 15 (one MMA takes both
+      // bf16 terms of the weights: high in rows 0..7, low in rows 8..15)
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        uint32_t ah0 = 0u, al0 = 0u, ah2 = 0u, al2 = 0u;
-        if (gm < G) {
-          const float2 w01 = *reinterpret_cast<const float2*>(&s_p[gm][16 * ks + 2 * tq]);
-          const float2 w23 = *reinterpret_cast<const float2*>(&s_p[gm][16 * ks + 8 + 2 * tq]);
-          split_bf16(w01.x, w01.y, ah0, al0);
-          split_bf16(w23.x, w23.y, ah2, al2);
-        }
+        uint32_t a[4];
+        ldsm_x4(a, &s_P[(lane & 7) + 8 * ((lane >> 3) & 1)][16 * ks + 8 * (lane >> 4)]);
         const int row = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
         const int ch = 2 * warp + (lane >> 4);
         uint32_t bm[4];
         ldsm_x4_t(bm, vs_ + (ch >> 3) * 8192 + swz128(row, ch & 7));
-        mma_bf16(oacc[0], ah0, ah2, bm[0], bm[1]);
-        mma_bf16(oacc[0], al0, al2, bm[0], bm[1]);
-        mma_bf16(oacc[1], ah0, ah2, bm[2], bm[3]);
-        mma_bf16(oacc[1], al0, al2, bm[2], bm[3]);
+        mma_bf16_4(oacc[0], a[0], a[1], a[2], a[3], bm[0], bm[1]);
+        mma_bf16_4(oacc[1], a[0], a[1], a[2], a[3], bm[2], bm[3]);
       }
-      __syncthreads();  // slots, s_p and the per-warp stats are read before reuse
+      __syncthreads();  // slots, s_P and the per-warp stats are read before reuse
       issue(t + 2);
     }
     cp_async_wait<0>();
@@ -1572,7 +1468,8 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           const int d = 16 * warp + 8 * nt + 2 * tq;
-          *reinterpret_cast<float2*>(&s_o[gm * D + d]) = make_float2(oacc[nt][0], oacc[nt][1]);
+          *reinterpret_cast<float2*>(&s_o[gm * D + d]) =
+              make_float2(oacc[nt][0] + oacc[nt][2], oacc[nt][1] + oacc[nt][3]);
         }
         if (warp == 0 && tq == 0) { s_em[gm] = mr; s_el[gm] = lr; }
       }
@@ -1582,100 +1479,13 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     }
   };
 
-  pdl_wait();
-  if (role_fold) {
-    FoldArgs fa{A.est_parts, A.n_chunks, A.partials, A.n_parts, A.n_rng + A.n_sc, G, D};
-    fold_role(fa, u, (int)blockIdx.x - A.n_rng - A.n_sc);
-  } else if (role_range) {
-    // ---------------------------------------------------------- range CTA
-    const int c = (int)blockIdx.x * kRangeW + tid;
-    const bool inr = c < NC;
-    // one round: unit record, and this thread's cluster: key, affected
-    // index, offsets, scores
-    uint32_t key = 0u;
-    int af = 0, o0 = 0, o1 = 0;
-    float scv[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) scv[g] = 0.f;
-    int32_t* afp = A.aff_of + (int64_t)u * A.max_nc + c;
-    if (inr) {
-      key = A.keys[row0 + c];
-      af = *afp;
-      o0 = __ldg(off + c);
-      o1 = __ldg(off + c + 1);
-#pragma unroll
-      for (int g = 0; g < G; ++g) scv[g] = A.scores[(row0 + c) * G + g];
-    }
-    if (tid < kInfoInts) s_info[tid] = A.info[(int64_t)u * kInfoInts + tid];
-    __syncthreads();
-    if (af != 0) *afp = 0;  // consumed: clean for the next call
-    const bool dense = s_info[6] != 0;
-    const bool est = !dense && s_info[0] < s_info[7] && NC > 0;
-    const uint32_t kstar = (uint32_t)s_info[1];
-    const int thr = s_info[2];
-    const int cnt = o1 - o0;
-    const bool pk = inr && cnt > 0 &&
-                    (dense || (key != 0u && af >= 0 && (key > kstar || (key == kstar && c <= thr))));
-    int cw = 0, csel = 0;  // correction: count (-1: steady members, read below), row selector
-    if (est && inr && cnt > 0) {
-      if (pk || af < 0) { cw = cnt; csel = c; }
-      else if (af > 0 && key != 0u) { cw = -1; csel = ~(af - 1); }
-    }
-    int2 tot;
-    const int2 incl = block_inclusive_scan2(make_int2((pk ? 1 : 0) | ((cw != 0 ? 1 : 0) << 16), pk ? cnt : 0),
-                                            scan_sh, &tot);
-    const int n_pk = tot.x & 0xffff, n_ce = tot.x >> 16, n_tk = tot.y;
-    if (pk) {
-      const int i = (incl.x & 0xffff) - 1;
-      s_pkc[i] = af > 0 ? ~c : c;             // marked when it has steady members
-      s_pkt[i] = incl.y - cnt;
-      s_pko[i] = o0;
-    }
-    if (cw != 0) {
-      const int i = (incl.x >> 16) - 1;
-      s_cec[i] = csel;
-      s_cew[i] = cw;
-#pragma unroll
-      for (int g = 0; g < G; ++g) s_ces[i * G + g] = scv[g];
-    }
-    if (tid == 0 && !dense && n_pk > 0) {
-      s_base = atomicAdd(A.sel_n + u, n_pk);
-      atomicAdd(const_cast<int32_t*>(A.info) + (int64_t)u * kInfoInts + 3, n_tk);
-    }
-    __syncthreads();
-    if (pk && !dense) A.sel[row0 + s_base + (incl.x & 0xffff) - 1] = c;
-    // correction entries: the steady members' counts (loaded now, used after
-    // the exact part)
-    int as0 = 0, as1 = 0;
-    const bool need_dc = tid < n_ce && s_cew[tid] < 0;
-    if (need_dc) {
-      const int32_t* as = A.aff_start + (int64_t)u * (A.cap + 1) + ~s_cec[tid];
-      as0 = as[0];
-      as1 = as[1];
-    }
-    // exact part: the picked clusters' tokens, kRowCap per pass; each
-    // thread resolves two tokens with their loads (position, page) in flight
-    // together
-    // correction rows, first kCorrRows of them: staged now, in flight with the
-    // exact part's tiles (their group completes before the first tile's)
-    constexpr int CHF = D * 4 / 16, CHT = RS::ROWB / 16;
-    auto issue_corr = [&](int p0) {
-      const int np_ = min(kCorrRows, n_ce - p0);
-      for (int k = tid; k < np_ * CHF; k += blockDim.x) {
-        const int i = k / CHF, ch = k - i * CHF;
-        const int sel_ = s_cec[p0 + i];
-        unsigned char* slot = s_crow + (size_t)i * D * 4;
-        if (sel_ >= 0) {
-          if (ch < CHT)
-            cp_async16(slot + ch * 16, reinterpret_cast<const unsigned char*>(vsum + (row0 + sel_) * D) + ch * 16);
-        } else {
-          cp_async16(slot + ch * 16,
-                     reinterpret_cast<const unsigned char*>(A.dv + ((int64_t)u * A.cap + ~sel_) * D) + ch * 16);
-        }
-      }
-      cp_async_commit();
-    };
-    if (n_ce > 0) issue_corr(0);
+  // exact attention over the picked clusters' tokens (lists s_pkc / s_pkt /
+  // s_pko of n_pk clusters, n_tk tokens), kRowCap tokens per pass; each
+  // thread resolves two tokens with their loads (position, page) in flight
+  // together; an affected cluster's steady members are skipped.  Pages
+  // lp0 .. lp0 + kBtStage - 1 of the block table are read from s_bt when
+  // lp0 >= 0 (staged by the caller), the others from global memory.
+  auto exact_over_picked = [&](int n_pk, int n_tk, bool dense, int lp0) {
     const int32_t* pm = A.perm + geo.tok_row(b, h);
     for (int p0 = 0; p0 < n_tk; p0 += kRowCap) {
       const int np_ = min(kRowCap, n_tk - p0);
@@ -1704,7 +1514,13 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       int32_t ro2[2];
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        const int64_t ro = slot2[k] >= 0 ? pool_row(kp, geo.hkv, 1, b, h, slot2[k], status) : -1;
+        int64_t ro = -1;
+        if (slot2[k] >= 0) {
+          const int li = (slot2[k] >> kp.page_shift) - lp0;
+          ro = lp0 >= 0 && li >= 0 && li < kBtStage
+                   ? pool_row_pg(kp, geo.hkv, 1, h, slot2[k], s_bt[li], status)
+                   : pool_row(kp, geo.hkv, 1, b, h, slot2[k], status);
+        }
         ro2[k] = (int32_t)ro;
       }
 #pragma unroll
@@ -1719,6 +1535,299 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       attend_tokens(np_);
       __syncthreads();
     }
+  };
+
+  pdl_wait();
+  if (role_fold) {
+    FoldArgs fa{A.est_parts, A.n_chunks, A.partials, A.n_parts, A.n_rng + A.n_sc, G, D};
+    fold_role(fa, u, (int)blockIdx.x - A.n_rng - A.n_sc);
+  } else if (role_range) {
+   if constexpr (kMma) {
+    // ------------------------------------ range CTA, tensor-core estimate
+    const int c = (int)blockIdx.x * kRangeW + tid;
+    const bool inr = c < NC;
+    uint32_t key = 0u;
+    int af = 0, o0 = 0, o1 = 0;
+    float scv[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) scv[g] = 0.f;
+    int32_t* afp = A.aff_of + (int64_t)u * A.max_nc + c;
+    if (inr) {
+      key = A.keys[row0 + c];
+      af = *afp;
+      o0 = __ldg(off + c);
+      o1 = __ldg(off + c + 1);
+#pragma unroll
+      for (int g = 0; g < G; ++g) scv[g] = A.scores[(row0 + c) * G + g];
+    }
+    if (tid < kInfoInts) s_info[tid] = A.info[(int64_t)u * kInfoInts + tid];
+    if (tid == 0) s_lp0 = inr ? o0 >> kp.page_shift : -1;   // the range's first page
+    __syncthreads();
+    if (af != 0) *afp = 0;  // consumed: clean for the next call
+    // the block-table entries of the range's pages, in flight until the
+    // exact part resolves its rows
+    const int lp0 = s_lp0;
+    if (lp0 >= 0) {
+      for (int i = tid; i < kBtStage; i += blockDim.x)
+        if (lp0 + i < kp.max_pages) cp_async4(&s_bt[i], kp.bt + (int64_t)b * kp.max_pages + lp0 + i);
+      cp_async_commit();
+    }
+    const bool dense = s_info[6] != 0;
+    const bool est = !dense && s_info[0] < s_info[7] && NC > 0;
+    const uint32_t kstar = (uint32_t)s_info[1];
+    const int thr = s_info[2];
+    const int cnt = o1 - o0;
+    const bool pk = inr && cnt > 0 &&
+                    (dense || (key != 0u && af >= 0 && (key > kstar || (key == kstar && c <= thr))));
+    // estimation zone: a candidate (it keeps a non-steady member) that is not
+    // retrieved; an affected one's steady members come back out (ce)
+    const bool ez = est && inr && cnt > 0 && !pk && af >= 0;
+    const bool ce = ez && af > 0;
+    const int dcnt = ce ? af >> 16 : 0;       // its steady members
+#pragma unroll
+    for (int g = 0; g < G; ++g) {   // per head: the zone's score max, per warp
+      const float mx = warp_max(ez ? scv[g] : -INFINITY);
+      if (lane == 0) s_wmax[warp][g] = mx;
+    }
+    int2 tot;
+    const int2 incl = block_inclusive_scan2(make_int2((pk ? 1 : 0) | ((ce ? 1 : 0) << 16), pk ? cnt : 0),
+                                            scan_sh, &tot);
+    const int n_pk = tot.x & 0xffff, n_ce = tot.x >> 16, n_tk = tot.y;
+    if (pk) {
+      const int i = (incl.x & 0xffff) - 1;
+      s_pkc[i] = af > 0 ? ~c : c;             // marked when it has steady members
+      s_pkt[i] = incl.y - cnt;
+      s_pko[i] = o0;
+    }
+    if (ce) {
+      const int i = (incl.x >> 16) - 1;
+      s_cec[i] = (af & 0xffff) - 1;           // its affected-list entry (dV row)
+      s_cew[i] = tid;                         // its weights' column
+    }
+    // weights w = e^(s - m_e) of the zone (zero elsewhere) by head, as two
+    // bf16 terms (the value the tensor cores use, also for the denominator
+    // terms (cnt - steady members) w and the dV correction)
+    float me0 = -INFINITY;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float me = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) me = fmaxf(me, s_wmax[w][g]);
+      if (g == 0) me0 = me;
+      const float wgt = ez ? __expf(scv[g] - me) : 0.f;
+      const __nv_bfloat16 whi = __float2bfloat16_rn(wgt);
+      const __nv_bfloat16 wlo = __float2bfloat16_rn(wgt - __bfloat162float(whi));
+      s_W[g][tid] = whi;
+      s_W[8 + g][tid] = wlo;
+      const float lz = warp_sum((__bfloat162float(whi) + __bfloat162float(wlo)) * (float)(cnt - dcnt));
+      if (lane == 0) s_wsum[warp][g] = lz;
+    }
+    // the selection list's slots: the atomic's result is used at the end, so
+    // its round trip overlaps the work below
+    int base_r = 0;
+    if (tid == 0 && !dense && n_pk > 0) {
+      base_r = atomicAdd(A.sel_n + u, n_pk);
+      atomicAdd(const_cast<int32_t*>(A.info) + (int64_t)u * kInfoInts + 3, n_tk);
+    }
+    const int sel_i = pk && !dense ? (incl.x & 0xffff) - 1 : -1;
+    __syncthreads();
+    // this lane's head gm: the zone's (m_e, l_e)
+    float me_r = -INFINITY, le_r = 0.f;
+    if (gm < G) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) { me_r = fmaxf(me_r, s_wmax[w][gm]); le_r += s_wsum[w][gm]; }
+    }
+    // dV rows of the zone's affected clusters, kCorrRows per pass: the first
+    // pass in flight with the exact part's tiles (its group completes first)
+    constexpr int CHF = D * 4 / 16;
+    auto issue_dv = [&](int p0) {
+      const int np_ = min(kCorrRows, n_ce - p0);
+      for (int k = tid; k < np_ * CHF; k += blockDim.x) {
+        const int i = k / CHF, ch = k - i * CHF;
+        cp_async16(s_crow + (size_t)i * D * 4 + ch * 16,
+                   reinterpret_cast<const unsigned char*>(A.dv + ((int64_t)u * A.cap + s_cec[p0 + i]) * D) +
+                       ch * 16);
+      }
+      cp_async_commit();
+    };
+    if (n_ce > 0) issue_dv(0);
+    // o_e = W Vsum on the tensor cores: A = the weights split into two bf16
+    // terms (high in rows 0..7, low in rows 8..15, heads below G), B = the
+    // value-sum rows of the ring (ldmatrix.trans); warp w owns output columns
+    // 16 w .. 16 w + 15
+    mbar_wait(&s_vbar, 0, status);
+    if (me0 != -INFINITY) {
+      float oe[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      const unsigned char* r8 = sh;
+#pragma unroll 4
+      for (int ks = 0; ks < kRangeW / 16; ++ks) {
+        uint32_t a[4];
+        ldsm_x4(a, &s_W[(lane & 7) + 8 * ((lane >> 3) & 1)][16 * ks + 8 * (lane >> 4)]);
+        const unsigned char* tile = r8 + (size_t)(ks >> 2) * 16384;
+        const int row = 16 * (ks & 3) + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int ch = 2 * warp + (lane >> 4);
+        uint32_t bm[4];
+        ldsm_x4_t(bm, tile + (ch >> 3) * 8192 + swz128(row, ch & 7));
+        mma_bf16_4(oe[0], a[0], a[1], a[2], a[3], bm[0], bm[1]);
+        mma_bf16_4(oe[1], a[0], a[1], a[2], a[3], bm[2], bm[3]);
+      }
+      if (gm < G) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int d = 16 * warp + 8 * nt + 2 * tq;
+          *reinterpret_cast<float2*>(&s_o[gm * D + d]) =
+              make_float2(oe[nt][0] + oe[nt][2], oe[nt][1] + oe[nt][3]);
+        }
+      }
+    } else if (gm < G) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int d = 16 * warp + 8 * nt + 2 * tq;
+        *reinterpret_cast<float2*>(&s_o[gm * D + d]) = make_float2(0.f, 0.f);
+      }
+    }
+    // the exact part; this barrier also orders the ring's reads above
+    // before the tiles' copies into it
+    if (lp0 >= 0) cp_async_wait_dyn(n_ce > 0 ? 1 : 0);   // the block-table window
+    __syncthreads();
+    exact_over_picked(n_pk, n_tk, dense, lp0);
+    // exact and zone parts of head gm at a common max, into s_o
+    if (gm < G) {
+      const float M = fmaxf(mr, me_r);
+      const float fx = mr == -INFINITY ? 0.f : expf(mr - M);
+      const float fe = me_r == -INFINITY ? 0.f : expf(me_r - M);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int d = 16 * warp + 8 * nt + 2 * tq;
+        float2* op = reinterpret_cast<float2*>(&s_o[gm * D + d]);
+        const float2 e = *op;
+        *op = make_float2((oacc[nt][0] + oacc[nt][2]) * fx + e.x * fe,
+                          (oacc[nt][1] + oacc[nt][3]) * fx + e.y * fe);
+      }
+      if (warp == 0 && tq == 0) { s_em[gm] = M; s_el[gm] = lr * fx + le_r * fe; s_f1[gm] = fe; }
+    }
+    // the steady members' dV, weighted like their clusters, come back out
+    float cacc[G][EPL];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) cacc[g][e] = 0.f;
+    for (int p0 = 0; p0 < n_ce; p0 += kCorrRows) {
+      const int np_ = min(kCorrRows, n_ce - p0);
+      if (p0 > 0) issue_dv(p0);
+      cp_async_wait<0>();
+      __syncthreads();
+      for (int rb = warp * RPW; rb < np_; rb += NW * RPW) {
+        const int i = rb + rsub;
+        if (i >= np_) continue;
+        const float* fr = reinterpret_cast<const float*>(s_crow + (size_t)i * D * 4) + sub * EPL;
+        float x[EPL];
+#pragma unroll
+        for (int e4 = 0; e4 < EPL; e4 += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(fr + e4);
+          x[e4] = v.x; x[e4 + 1] = v.y; x[e4 + 2] = v.z; x[e4 + 3] = v.w;
+        }
+        float wv[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          wv[g] = __bfloat162float(s_W[g][s_cew[p0 + i]]) + __bfloat162float(s_W[8 + g][s_cew[p0 + i]]);
+        axpy_g<G, EPL>(wv, x, cacc);
+      }
+      __syncthreads();
+    }
+    if (tid == 0) s_base = base_r;
+    __syncthreads();   // s_em / s_el / s_f1 / s_base are written
+    if (sel_i >= 0) A.sel[row0 + s_base + sel_i] = c;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      m_run[g] = s_em[g];
+      l_run[g] = s_el[g];
+      const float fe = s_f1[g];
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) acc[g][e] = -cacc[g][e] * fe;
+    }
+   } else {
+    // ------------------------------------------------- range CTA, CUDA cores
+    const int c = (int)blockIdx.x * kRangeW + tid;
+    const bool inr = c < NC;
+    // one round: unit record, and this thread's cluster: key, affected
+    // index, offsets, scores
+    uint32_t key = 0u;
+    int af = 0, o0 = 0, o1 = 0;
+    float scv[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) scv[g] = 0.f;
+    int32_t* afp = A.aff_of + (int64_t)u * A.max_nc + c;
+    if (inr) {
+      key = A.keys[row0 + c];
+      af = *afp;
+      o0 = __ldg(off + c);
+      o1 = __ldg(off + c + 1);
+#pragma unroll
+      for (int g = 0; g < G; ++g) scv[g] = A.scores[(row0 + c) * G + g];
+    }
+    if (tid < kInfoInts) s_info[tid] = A.info[(int64_t)u * kInfoInts + tid];
+    __syncthreads();
+    if (af != 0) *afp = 0;  // consumed: clean for the next call
+    const bool dense = s_info[6] != 0;
+    const bool est = !dense && s_info[0] < s_info[7] && NC > 0;
+    const uint32_t kstar = (uint32_t)s_info[1];
+    const int thr = s_info[2];
+    const int cnt = o1 - o0;
+    const bool pk = inr && cnt > 0 &&
+                    (dense || (key != 0u && af >= 0 && (key > kstar || (key == kstar && c <= thr))));
+    int cw = 0, csel = 0;  // correction: count, row selector
+    if (est && inr && cnt > 0) {
+      if (pk || af < 0) { cw = cnt; csel = c; }
+      else if (af > 0 && key != 0u) { cw = af >> 16; csel = ~((af & 0xffff) - 1); }
+    }
+    int2 tot;
+    const int2 incl = block_inclusive_scan2(make_int2((pk ? 1 : 0) | ((cw != 0 ? 1 : 0) << 16), pk ? cnt : 0),
+                                            scan_sh, &tot);
+    const int n_pk = tot.x & 0xffff, n_ce = tot.x >> 16, n_tk = tot.y;
+    if (pk) {
+      const int i = (incl.x & 0xffff) - 1;
+      s_pkc[i] = af > 0 ? ~c : c;             // marked when it has steady members
+      s_pkt[i] = incl.y - cnt;
+      s_pko[i] = o0;
+    }
+    if (cw != 0) {
+      const int i = (incl.x >> 16) - 1;
+      s_cec[i] = csel;
+      s_cew[i] = cw;
+#pragma unroll
+      for (int g = 0; g < G; ++g) s_ces[i * G + g] = scv[g];
+    }
+    if (tid == 0 && !dense && n_pk > 0) {
+      s_base = atomicAdd(A.sel_n + u, n_pk);
+      atomicAdd(const_cast<int32_t*>(A.info) + (int64_t)u * kInfoInts + 3, n_tk);
+    }
+    __syncthreads();
+    if (pk && !dense) A.sel[row0 + s_base + (incl.x & 0xffff) - 1] = c;
+    // exact part: the picked clusters' tokens, kRowCap per pass; each
+    // thread resolves two tokens with their loads (position, page) in flight
+    // together
+    // correction rows, first kCorrRows of them: staged now, in flight with the
+    // exact part's tiles (their group completes before the first tile's)
+    constexpr int CHF = D * 4 / 16, CHT = RS::ROWB / 16;
+    auto issue_corr = [&](int p0) {
+      const int np_ = min(kCorrRows, n_ce - p0);
+      for (int k = tid; k < np_ * CHF; k += blockDim.x) {
+        const int i = k / CHF, ch = k - i * CHF;
+        const int sel_ = s_cec[p0 + i];
+        unsigned char* slot = s_crow + (size_t)i * D * 4;
+        if (sel_ >= 0) {
+          if (ch < CHT)
+            cp_async16(slot + ch * 16, reinterpret_cast<const unsigned char*>(vsum + (row0 + sel_) * D) + ch * 16);
+        } else {
+          cp_async16(slot + ch * 16,
+                     reinterpret_cast<const unsigned char*>(A.dv + ((int64_t)u * A.cap + ~sel_) * D) + ch * 16);
+        }
+      }
+      cp_async_commit();
+    };
+    if (n_ce > 0) issue_corr(0);
+    exact_over_picked(n_pk, n_tk, dense, -1);
     exact_to_shared();
     // correction part: -(cnt e^(s - mc) , e^(s - mc) row), kCorrRows rows per pass
     float mc[G], lc[G];
@@ -1729,9 +1838,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     for (int g = 0; g < G; ++g)
 #pragma unroll
       for (int e = 0; e < EPL; ++e) cacc[g][e] = 0.f;
-    if (need_dc) s_cew[tid] = as1 - as0;
     if (n_ce > 0) {
-      __syncthreads();  // the steady-member counts are written
       if (warp < G) {   // per head: max, weights and denominator over the entries
         float m = -INFINITY;
         for (int i = lane; i < n_ce; i += 32) m = fmaxf(m, s_ces[i * G + warp]);
@@ -1788,6 +1895,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       m_run[g] = M;
       if (tid == 0) s_f1[g] = f1;
     }
+   }
   } else {
     // --------------------------------------------------------- steady CTA
     // steady slots j0 .. j0 + 2 TR - 1 of the unit's (slot-sorted) steady list
@@ -1801,12 +1909,10 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     __syncthreads();
     if (n_here > 0) attend_tokens(n_here);
     exact_to_shared();
-    if (tid < G) s_f1[tid] = 1.f;
   }
   if (!role_fold) {
     __syncthreads();
-    reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part, kMma ? s_o : nullptr,
-                                     kMma ? s_f1 : nullptr);
+    reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part, kMma ? s_o : nullptr);
     if (tid == 0) {
 #pragma unroll
       for (int g = 0; g < G; ++g) { part[g * PS] = m_run[g]; part[g * PS + 1] = l_run[g]; }
@@ -1943,8 +2049,9 @@ cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_
 
 size_t decode_attend_smem(int dtype, int D, int G, int n_parts) {
   (void)dtype;
-  // ring (also the merge staging) | correction rows | merge factors and denominators
-  return 4 * 16384 + (size_t)kCorrRows * D * 4 + 2 * (size_t)n_parts * G * 4;
+  // 1024-byte alignment | ring (also the merge staging) | correction rows |
+  // merge factors and denominators
+  return 1024 + 4 * 16384 + (size_t)kCorrRows * D * 4 + 2 * (size_t)n_parts * G * 4;
 }
 
 size_t decode_topk_smem(int max_nc, int cap) {
@@ -2036,34 +2143,26 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
     const size_t steady_smem = decode_score_smem(p.dtype, D, G, p.sort_pow2, p.cap);
     const int n_tot = p.U * p.n_score_blocks;
     e = cudaErrorInvalidValue;
-    // tensor-core path: K_A scores only, K_B's estimate CTAs stream the value sums
-    EstArgs ea{};
-    ea.scores = scores;
-    ea.offsets = a.offsets;
-    ea.est_parts = est_parts;
-    ea.n_chunks = p.n_score_blocks;
-    ea.G = G;
-    ea.n_ev = 0;
+    // tensor-core path (bf16, d = 128): K_A scores only; the attend kernel's
+    // range CTAs estimate from the value sums through their own tensor map
+    CUtensorMap tm_vsum;
+    std::memset(&tm_vsum, 0, sizeof(tm_vsum));
     bool done = false;
     if constexpr (std::is_same_v<T, __nv_bfloat16> && D == 128) {
       CUtensorMap tmc;
-      if (encode_rows128(&tmc, a.centroids, p.ncl) && encode_rows128(&ea.tm_vsum, a.value_sums, p.ncl)) {
-        const size_t smem = std::max(MmaSmem<G>::kTotal, steady_smem);
-        cudaFuncSetAttribute(wave_score_mma_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-        int per_sm = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, wave_score_mma_kernel<G>,
-                                                      kStreamThreads, smem);
-        const int n_stream = std::max(1, std::min(n_tot, std::max(1, per_sm) * sm_count() - p.U));
-        e = launch_ex(wave_score_mma_kernel<G>, dim3(p.U + n_stream), dim3(kStreamThreads), smem, s,
-                      false, p.geo, q, p.Hq, tmc, a.offsets, scores, keys, hist, p.scale,
-                      p.n_score_blocks, n_stream, sa, status);
-        // two CTAs per SM in all (the top-k CTAs included), and at most four
-        // chunks per estimate CTA when there are many units
-        ea.n_ev = std::max(1, std::min(p.n_score_blocks,
-                                       std::max((2 * sm_count()) / p.U - 1, (p.n_score_blocks + 3) / 4)));
-        done = true;
-      }
+      if (!encode_rows128(&tmc, a.centroids, p.ncl) || !encode_rows128(&tm_vsum, a.value_sums, p.ncl))
+        return cudaErrorInvalidValue;
+      const size_t smem = std::max(MmaSmem<G>::kTotal, steady_smem);
+      cudaFuncSetAttribute(wave_score_mma_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+      int per_sm = 0;
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, wave_score_mma_kernel<G>,
+                                                    kStreamThreads, smem);
+      const int n_stream = std::max(1, std::min(n_tot, std::max(1, per_sm) * sm_count() - p.U));
+      e = launch_ex(wave_score_mma_kernel<G>, dim3(p.U + n_stream), dim3(kStreamThreads), smem, s,
+                    false, p.geo, q, p.Hq, tmc, a.offsets, scores, keys, hist, p.scale,
+                    p.n_score_blocks, n_stream, sa, status);
+      done = true;
     }
     if (!done) {
       const size_t score_smem = steady_smem;
@@ -2080,12 +2179,12 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
     }
     if (e != cudaSuccess) return e;
     mark(1);
-    const size_t topk_smem = std::max(decode_topk_smem(p.max_nc, p.cap), ea.n_ev > 0 ? kEvSmem : 0);
+    const size_t topk_smem = decode_topk_smem(p.max_nc, p.cap);
     cudaFuncSetAttribute(wave_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)topk_smem);
     TopkArgs ta{keys, hist, nonc, p.cap, p.topk_clusters, p.topk_fraction, info, sel_n};
-    e = launch_ex(wave_topk_kernel, dim3(1 + ea.n_ev, p.U), dim3(kTopkThreads), topk_smem, s,
-                  pdl, p.geo, ta, ea, status);
+    e = launch_ex(wave_topk_kernel, dim3(p.U), dim3(kTopkThreads), topk_smem, s, pdl, p.geo, ta,
+                  status);
     if (e != cudaSuccess) return e;
     mark(2);
     AttendArgs A{keys, scores, info, aff_of, p.max_nc, aff_start, st_slot, dv, p.cap, a.perm,
@@ -2096,7 +2195,7 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
                          (int)smem);
     e = launch_ex(wave_attend_kernel<T, D, G>, dim3(p.n_rng + p.n_sc + p.n_fold, p.U), dim3(kStreamThreads),
                   smem, s, pdl, p.geo, q, p.Hq, a.kp, a.vp,
-                  reinterpret_cast<const T*>(a.value_sums), a.offsets, A, status);
+                  reinterpret_cast<const T*>(a.value_sums), a.offsets, A, tm_vsum, status);
     if (e != cudaSuccess) return e;
     mark(3);
     return cudaGetLastError();

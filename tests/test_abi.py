@@ -28,7 +28,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_stage_names():
-    assert W.stage_names() == ["score", "topk_estimate", "attend"]
+    assert W.stage_names() == ["score", "topk", "attend"]
     assert W.lib().wi_decode_stage_name(99) is None
 
 

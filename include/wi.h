@@ -149,13 +149,14 @@ typedef struct wi_decode_layout {
   size_t scores;       /* float [Hkv*sum NC_b][G]: q_h . centroid / sqrt(d)      */
   size_t keys;         /* uint32 [Hkv*sum NC_b]: order-preserving key of the
                           group-max score; 0 = not a candidate                   */
-  size_t selected;     /* int32 [Hkv*sum NC_b]: per unit (at its centroid row), the
-                          retrieved clusters in no particular order, sel_count
-                          of them                                                 */
+  size_t selected;     /* uint32 [B*Hkv][sel_words]: per unit, bit c % 32 of word
+                          c / 32 is set iff cluster c is retrieved (sel_count
+                          bits; none for a unit attended densely)                 */
   size_t unit_info;    /* int32 [B*Hkv][8]: {sel_count, thr_key, thr_idx,
                           sel_tokens, steady, n_affected, dense, candidates}     */
   int32_t n_attend_ctas; /* exact-attention CTAs per unit                         */
   int32_t n_score_ctas;  /* score + estimation chunks (CTAs) per unit             */
+  int32_t sel_words;     /* words of `selected` per unit                          */
 } wi_decode_layout;
 
 /* ------------------------------------------------------------------ sizes */

@@ -76,7 +76,8 @@ class WiDecodeParams(C.Structure):
 class WiDecodeLayout(C.Structure):
     _fields_ = [("total_bytes", C.c_size_t), ("status", C.c_size_t), ("scores", C.c_size_t),
                 ("keys", C.c_size_t), ("selected", C.c_size_t), ("unit_info", C.c_size_t),
-                ("n_attend_ctas", C.c_int32), ("n_score_ctas", C.c_int32)]
+                ("n_attend_ctas", C.c_int32), ("n_score_ctas", C.c_int32),
+                ("sel_words", C.c_int32)]
 
 
 _P = C.c_void_p
@@ -451,10 +452,15 @@ def unit_info(ws: torch.Tensor, layout: WiDecodeLayout, n_units: int) -> torch.T
 
 def selected_clusters(ws: torch.Tensor, layout: WiDecodeLayout, index: WaveIndex,
                       b: int, h: int, count: int) -> torch.Tensor:
-    """The retrieved clusters of unit (b, h), ascending (the workspace holds
-    them in no particular order)."""
-    row = index.cl_row(b, h)
-    return torch.sort(ws[layout.selected:].view(torch.int32)[row:row + count]).values
+    """The retrieved clusters of unit (b, h), ascending, read from the
+    workspace's selection bitmap (`count` of them)."""
+    u = b * index.n_kv_heads + h
+    words = ws[layout.selected:].view(torch.int32)[u * layout.sel_words:(u + 1) * layout.sel_words]
+    bits = (words.to(torch.int64).unsqueeze(1) >> torch.arange(32, device=words.device)) & 1
+    ids = torch.nonzero(bits.flatten()).flatten().to(torch.int32)
+    if len(ids) != count:
+        raise RuntimeError(f"selection bitmap holds {len(ids)} clusters, unit record says {count}")
+    return ids
 
 
 def centroid_scores(ws: torch.Tensor, layout: WiDecodeLayout, index: WaveIndex, G: int,

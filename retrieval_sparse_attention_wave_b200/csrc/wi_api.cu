@@ -157,8 +157,8 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   pl.off_aff_of = take((size_t)pl.U * max_nc * 4);  // reset after use by the attend kernel
   pl.off_scores = take((size_t)ncl * G * 4);
   pl.off_keys = take((size_t)ncl * 4);
-  pl.off_sel = take((size_t)ncl * 4);
-  pl.off_sel_n = take((size_t)pl.U * 4);
+  pl.sel_words = pl.n_rng * (kRangeClusters / 32);
+  pl.off_sel = take((size_t)pl.U * pl.sel_words * 4);
   pl.off_info = take((size_t)pl.U * kInfoInts * 4);
   pl.off_st_slot = take((size_t)pl.U * cap * 4);
   pl.off_st_cl = take((size_t)pl.U * cap * 4);
@@ -396,6 +396,7 @@ wi_status wi_decode_workspace_layout(const wi_index* idx, const wi_decode_params
   layout->unit_info = pl.off_info;
   layout->n_attend_ctas = pl.n_rng + pl.n_sc;
   layout->n_score_ctas = pl.n_score_blocks;
+  layout->sel_words = pl.sel_words;
   return WI_OK;
 }
 

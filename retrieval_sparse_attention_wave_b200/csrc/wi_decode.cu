@@ -849,7 +849,6 @@ struct TopkArgs {
   int topk_clusters;
   double topk_fraction;
   int32_t* info;
-  int32_t* sel_n;            // [U]: selection-list counter of the attend kernel (zeroed here)
 };
 
 __global__ void __launch_bounds__(kTopkThreads)
@@ -910,7 +909,6 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, uint32_t* status) {
   load_round(0);
   cp_async_wait<0>();
   __syncthreads();
-  if (tid == 0) { A.sel_n[u] = 0; I[3] = 0; }
   if (s_info[6]) {  // dense unit: every token is attended, nothing is selected
     for (int i = tid; i < kHistBins; i += nt) hg[i] = 0;   // clean for the next call
     if (tid == 0) { I[0] = 0; I[1] = (int32_t)0xFFFFFFFFu; I[2] = -1; I[7] = 0; }
@@ -1119,8 +1117,8 @@ struct AttendArgs {
   int cap;
   const int32_t* perm;       // slot -> position
   int n_sink, window;
-  int32_t* sel;              // per unit, the retrieved clusters (unordered)
-  int32_t* sel_n;            // [U] its counter
+  uint32_t* sel;             // [U][sel_words]: selection bitmap (bit c: cluster c retrieved)
+  int sel_words;
   const float* est_parts;    // [U][n_chunks][G][D+4], folded by the fold CTAs
   int n_chunks;
   int n_rng, n_sc, n_fold, n_parts;
@@ -1159,7 +1157,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   __shared__ int s_pkc[kRangeW], s_pkt[kRangeW], s_pko[kRangeW];   // picked: id, token start, slot start
   __shared__ int s_cec[kRangeW], s_cew[kRangeW];                   // correction: row selector, count
   __shared__ int scan_sh[64];
-  __shared__ int s_info[kInfoInts], s_base, s_last, s_lp0;
+  __shared__ int s_info[kInfoInts], s_last;
   __shared__ float s_m[G], s_l[G];
   // tensor-core exact attention (bf16, d = 128): tile weights, per-warp tile
   // max / sum, the exact part's output and running (m, l)
@@ -1208,6 +1206,10 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   uint32_t qa0[kMma ? 8 : 1], qa2[kMma ? 8 : 1];
   float mr = -INFINITY, lr = 0.f;
   float oacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  // range CTAs of the MMA path: their clusters' offsets and first page,
+  // read before the grid-dependency wait (index data: written before this
+  // call, never by the decode's kernels)
+  int r_o0 = 0, r_o1 = 0, r_lp0 = -1;
   if constexpr (kMma) {
     const uint32_t* qw = reinterpret_cast<const uint32_t*>(
         q + ((int64_t)b * n_q_heads + (int64_t)h * G + (gm < G ? gm : 0)) * D);
@@ -1231,6 +1233,19 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
           tensor_load_2d(sh + t * 16384 + 8192, &tm_vsum, 64, y0 + 64 * t, &s_vbar);
         }
       }
+      const int c0 = (int)blockIdx.x * kRangeW;
+      if (c0 + tid < NC) {
+        r_o0 = __ldg(off + c0 + tid);
+        r_o1 = __ldg(off + c0 + tid + 1);
+      }
+      r_lp0 = c0 < NC ? __ldg(off + c0) >> kp.page_shift : -1;
+      // the block-table entries of the range's pages, in flight until the
+      // exact part resolves its rows
+      if (r_lp0 >= 0) {
+        for (int i = tid; i < kBtStage; i += blockDim.x)
+          if (r_lp0 + i < kp.max_pages) cp_async4(&s_bt[i], kp.bt + (int64_t)b * kp.max_pages + r_lp0 + i);
+        cp_async_commit();
+      }
     } else {
       // rows no copy writes keep finite contents (zero weight times a finite row)
       for (int i = tid; i < 4 * 16384 / 16; i += blockDim.x)
@@ -1248,37 +1263,43 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   // tiles of TR tokens stream through two ring slots (K and V tiles each),
   // tile t + 2 issued as soon as tile t is consumed; online softmax carried
   // in m_run / l_run / acc
-  auto attend_tokens_mma = [&](int n) {
-    // tiles of 64 tokens: K rows into ring slot t & 1, V rows into slot
-    // 2 + (t & 1), each 16 KB slot two 128-byte-swizzled halves of 64 rows
+  // MMA path, tiles of 64 tokens: tile t's K rows into ring slot
+  // kv_slot(t), its V rows into the next slot (slots 2, 3 for even tiles,
+  // 0, 1 for odd ones), each 16 KB slot two 128-byte-swizzled halves of 64
+  // rows; one cp.async group per tile
+  auto kv_slot = [](int t) { return 2 * ((t + 1) & 1); };
+  auto issue_kv = [&](int t, int n) {
     const unsigned char* kb8 = reinterpret_cast<const unsigned char*>(kp.base);
     const unsigned char* vb8 = reinterpret_cast<const unsigned char*>(vp.base);
     unsigned char* r8 = reinterpret_cast<unsigned char*>(ring);
-    const int ntile = (n + 63) / 64;
-    auto issue = [&](int t) {
-      if (t < ntile) {
-        unsigned char* ks_ = r8 + (size_t)(t & 1) * 16384;
-        unsigned char* vs_ = r8 + (size_t)(2 + (t & 1)) * 16384;
-        for (int i = tid; i < 64 * 16; i += blockDim.x) {
-          const int r = i >> 4, ch = i & 15;
-          const int rr = t * 64 + r;
-          const int32_t ri = rr < n ? s_row[rr] : -1;
-          if (ri >= 0) {
-            const int o = (ch >> 3) * 8192 + swz128(r, ch & 7);
-            cp_async16(ks_ + o, kb8 + (int64_t)ri * 256 + ch * 16);
-            cp_async16(vs_ + o, vb8 + (int64_t)ri * 256 + ch * 16);
-          }
+    if (t < (n + 63) / 64) {
+      unsigned char* ks_ = r8 + (size_t)kv_slot(t) * 16384;
+      unsigned char* vs_ = ks_ + 16384;
+      for (int i = tid; i < 64 * 16; i += blockDim.x) {
+        const int r = i >> 4, ch = i & 15;
+        const int rr = t * 64 + r;
+        const int32_t ri = rr < n ? s_row[rr] : -1;
+        if (ri >= 0) {
+          const int o = (ch >> 3) * 8192 + swz128(r, ch & 7);
+          cp_async16(ks_ + o, kb8 + (int64_t)ri * 256 + ch * 16);
+          cp_async16(vs_ + o, vb8 + (int64_t)ri * 256 + ch * 16);
         }
       }
-      cp_async_commit();
-    };
-    issue(0);
-    issue(1);
+    }
+    cp_async_commit();
+  };
+  // exact attention over the tokens of s_row[0 .. n) on the tensor cores;
+  // tiles 0 .. issued - 1 were issued by the caller
+  auto attend_tokens_mma = [&](int n, int issued) {
+    unsigned char* r8 = reinterpret_cast<unsigned char*>(ring);
+    const int ntile = (n + 63) / 64;
+    auto issue = [&](int t) { issue_kv(t, n); };
+    for (int t = issued; t < 2; ++t) issue(t);
     for (int t = 0; t < ntile; ++t) {
       cp_async_wait<1>();
       __syncthreads();
-      const unsigned char* ks_ = r8 + (size_t)(t & 1) * 16384;
-      const unsigned char* vs_ = r8 + (size_t)(2 + (t & 1)) * 16384;
+      const unsigned char* ks_ = r8 + (size_t)kv_slot(t) * 16384;
+      const unsigned char* vs_ = ks_ + 16384;
       // scores of rows 8 warp .. 8 warp + 7
       float sacc[4] = {0.f, 0.f, 0.f, 0.f};
       const int n0 = 8 * warp;
@@ -1350,8 +1371,8 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     cp_async_wait<0>();
   };
 
-  auto attend_tokens = [&](int n) {
-    if constexpr (kMma) { attend_tokens_mma(n); return; }
+  auto attend_tokens = [&](int n, int issued) {
+    if constexpr (kMma) { attend_tokens_mma(n, issued); return; }
     const T* kbase = reinterpret_cast<const T*>(kp.base);
     const T* vbase = reinterpret_cast<const T*>(vp.base);
     const int ntile = (n + TR - 1) / TR;
@@ -1485,7 +1506,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   // together; an affected cluster's steady members are skipped.  Pages
   // lp0 .. lp0 + kBtStage - 1 of the block table are read from s_bt when
   // lp0 >= 0 (staged by the caller), the others from global memory.
-  auto exact_over_picked = [&](int n_pk, int n_tk, bool dense, int lp0) {
+  auto exact_over_picked = [&](int n_pk, int n_tk, bool dense, int lp0, auto&& first_pass) {
     const int32_t* pm = A.perm + geo.tok_row(b, h);
     for (int p0 = 0; p0 < n_tk; p0 += kRowCap) {
       const int np_ = min(kRowCap, n_tk - p0);
@@ -1532,7 +1553,8 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
         }
       }
       __syncthreads();
-      attend_tokens(np_);
+      // first_pass(np_) may issue the first tiles itself; it returns how many
+      attend_tokens(np_, p0 == 0 ? first_pass(np_) : 0);
       __syncthreads();
     }
   };
@@ -1547,7 +1569,8 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     const int c = (int)blockIdx.x * kRangeW + tid;
     const bool inr = c < NC;
     uint32_t key = 0u;
-    int af = 0, o0 = 0, o1 = 0;
+    int af = 0;
+    const int o0 = r_o0, o1 = r_o1, lp0 = r_lp0;
     float scv[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) scv[g] = 0.f;
@@ -1555,23 +1578,12 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     if (inr) {
       key = A.keys[row0 + c];
       af = *afp;
-      o0 = __ldg(off + c);
-      o1 = __ldg(off + c + 1);
 #pragma unroll
       for (int g = 0; g < G; ++g) scv[g] = A.scores[(row0 + c) * G + g];
     }
     if (tid < kInfoInts) s_info[tid] = A.info[(int64_t)u * kInfoInts + tid];
-    if (tid == 0) s_lp0 = inr ? o0 >> kp.page_shift : -1;   // the range's first page
     __syncthreads();
     if (af != 0) *afp = 0;  // consumed: clean for the next call
-    // the block-table entries of the range's pages, in flight until the
-    // exact part resolves its rows
-    const int lp0 = s_lp0;
-    if (lp0 >= 0) {
-      for (int i = tid; i < kBtStage; i += blockDim.x)
-        if (lp0 + i < kp.max_pages) cp_async4(&s_bt[i], kp.bt + (int64_t)b * kp.max_pages + lp0 + i);
-      cp_async_commit();
-    }
     const bool dense = s_info[6] != 0;
     const bool est = !dense && s_info[0] < s_info[7] && NC > 0;
     const uint32_t kstar = (uint32_t)s_info[1];
@@ -1622,14 +1634,12 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       const float lz = warp_sum((__bfloat162float(whi) + __bfloat162float(wlo)) * (float)(cnt - dcnt));
       if (lane == 0) s_wsum[warp][g] = lz;
     }
-    // the selection list's slots: the atomic's result is used at the end, so
-    // its round trip overlaps the work below
-    int base_r = 0;
-    if (tid == 0 && !dense && n_pk > 0) {
-      base_r = atomicAdd(A.sel_n + u, n_pk);
-      atomicAdd(const_cast<int32_t*>(A.info) + (int64_t)u * kInfoInts + 3, n_tk);
+    // the range's words of the selection bitmap (no atomics: a barrier after
+    // a global atomic would wait for its round trip)
+    {
+      const uint32_t bits = __ballot_sync(0xffffffffu, pk && !dense);
+      if (lane == 0) A.sel[(int64_t)u * A.sel_words + blockIdx.x * (kRangeW / 32) + warp] = bits;
     }
-    const int sel_i = pk && !dense ? (incl.x & 0xffff) - 1 : -1;
     __syncthreads();
     // this lane's head gm: the zone's (m_e, l_e)
     float me_r = -INFINITY, le_r = 0.f;
@@ -1654,13 +1664,13 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     // o_e = W Vsum on the tensor cores: A = the weights split into two bf16
     // terms (high in rows 0..7, low in rows 8..15, heads below G), B = the
     // value-sum rows of the ring (ldmatrix.trans); warp w owns output columns
-    // 16 w .. 16 w + 15
-    mbar_wait(&s_vbar, 0, status);
-    if (me0 != -INFINITY) {
-      float oe[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    // 16 w .. 16 w + 15.  k-steps 8..15 (ring slots 2, 3) run first, so the
+    // exact part's first tile can load into those slots while k-steps 0..7
+    // run; its second tile follows into slots 0, 1.
+    auto est_steps = [&](float (&oe)[2][4], int ks0, int ks1) {
       const unsigned char* r8 = sh;
 #pragma unroll 4
-      for (int ks = 0; ks < kRangeW / 16; ++ks) {
+      for (int ks = ks0; ks < ks1; ++ks) {
         uint32_t a[4];
         ldsm_x4(a, &s_W[(lane & 7) + 8 * ((lane >> 3) & 1)][16 * ks + 8 * (lane >> 4)]);
         const unsigned char* tile = r8 + (size_t)(ks >> 2) * 16384;
@@ -1671,6 +1681,14 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
         mma_bf16_4(oe[0], a[0], a[1], a[2], a[3], bm[0], bm[1]);
         mma_bf16_4(oe[1], a[0], a[1], a[2], a[3], bm[2], bm[3]);
       }
+    };
+    auto estimate = [&](int np_) -> int {
+      float oe[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      mbar_wait(&s_vbar, 0, status);
+      if (me0 != -INFINITY) est_steps(oe, kRangeW / 32, kRangeW / 16);
+      __syncthreads();              // slots 2, 3 are read
+      issue_kv(0, np_);
+      if (me0 != -INFINITY) est_steps(oe, 0, kRangeW / 32);
       if (gm < G) {
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -1679,18 +1697,15 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
               make_float2(oe[nt][0] + oe[nt][2], oe[nt][1] + oe[nt][3]);
         }
       }
-    } else if (gm < G) {
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int d = 16 * warp + 8 * nt + 2 * tq;
-        *reinterpret_cast<float2*>(&s_o[gm * D + d]) = make_float2(0.f, 0.f);
-      }
-    }
-    // the exact part; this barrier also orders the ring's reads above
-    // before the tiles' copies into it
+      __syncthreads();              // slots 0, 1 are read
+      issue_kv(1, np_);
+      return 2;
+    };
+    // the exact part, the estimate folded into its first pass
     if (lp0 >= 0) cp_async_wait_dyn(n_ce > 0 ? 1 : 0);   // the block-table window
     __syncthreads();
-    exact_over_picked(n_pk, n_tk, dense, lp0);
+    exact_over_picked(n_pk, n_tk, dense, lp0, estimate);
+    if (n_tk == 0) estimate(0);
     // exact and zone parts of head gm at a common max, into s_o
     if (gm < G) {
       const float M = fmaxf(mr, me_r);
@@ -1735,9 +1750,8 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       }
       __syncthreads();
     }
-    if (tid == 0) s_base = base_r;
-    __syncthreads();   // s_em / s_el / s_f1 / s_base are written
-    if (sel_i >= 0) A.sel[row0 + s_base + sel_i] = c;
+    __syncthreads();   // s_em / s_el / s_f1 are written
+    if (tid == 0) part[2] = dense ? 0.f : (float)n_tk;   // retrieved tokens, summed by the merge
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       m_run[g] = s_em[g];
@@ -1798,12 +1812,12 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
 #pragma unroll
       for (int g = 0; g < G; ++g) s_ces[i * G + g] = scv[g];
     }
-    if (tid == 0 && !dense && n_pk > 0) {
-      s_base = atomicAdd(A.sel_n + u, n_pk);
-      atomicAdd(const_cast<int32_t*>(A.info) + (int64_t)u * kInfoInts + 3, n_tk);
+    {
+      const uint32_t bits = __ballot_sync(0xffffffffu, pk && !dense);
+      if (lane == 0) A.sel[(int64_t)u * A.sel_words + blockIdx.x * (kRangeW / 32) + warp] = bits;
     }
+    if (tid == 0) part[2] = dense ? 0.f : (float)n_tk;   // retrieved tokens, summed by the merge
     __syncthreads();
-    if (pk && !dense) A.sel[row0 + s_base + (incl.x & 0xffff) - 1] = c;
     // exact part: the picked clusters' tokens, kRowCap per pass; each
     // thread resolves two tokens with their loads (position, page) in flight
     // together
@@ -1827,7 +1841,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       cp_async_commit();
     };
     if (n_ce > 0) issue_corr(0);
-    exact_over_picked(n_pk, n_tk, dense, -1);
+    exact_over_picked(n_pk, n_tk, dense, -1, [](int) { return 0; });
     exact_to_shared();
     // correction part: -(cnt e^(s - mc) , e^(s - mc) row), kCorrRows rows per pass
     float mc[G], lc[G];
@@ -1907,7 +1921,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     const int n_here = max(0, min(2 * TR, (s_info[6] ? 0 : s_info[4]) - j0));
     if (tid < 2 * TR) s_row[tid] = tid < n_here ? (int32_t)pool_row(kp, geo.hkv, 1, b, h, sl, status) : -1;
     __syncthreads();
-    if (n_here > 0) attend_tokens(n_here);
+    if (n_here > 0) attend_tokens(n_here, 0);
     exact_to_shared();
   }
   if (!role_fold) {
@@ -1951,6 +1965,12 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   for (int i = tid; i < np * G; i += blockDim.x) {
     f[i] = __ldcg(pbase + (int64_t)i * PS);
     lp[i] = __ldcg(pbase + (int64_t)i * PS + 1);
+  }
+  if (warp == NW - 1) {   // the unit's retrieved tokens: the range parts' counts
+    int st = 0;
+    for (int p = lane; p < A.n_rng; p += 32) st += (int)__ldcg(pbase + (int64_t)p * PFL + 2);
+    st = warp_sum_int(st);
+    if (lane == 0) const_cast<int32_t*>(I)[3] = st;
   }
   __syncthreads();
   if (warp < G) {
@@ -2116,8 +2136,7 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + p.off_status);
   float* scores = reinterpret_cast<float*>(ws + p.off_scores);
   uint32_t* keys = reinterpret_cast<uint32_t*>(ws + p.off_keys);
-  int32_t* sel = reinterpret_cast<int32_t*>(ws + p.off_sel);
-  int32_t* sel_n = reinterpret_cast<int32_t*>(ws + p.off_sel_n);
+  uint32_t* sel = reinterpret_cast<uint32_t*>(ws + p.off_sel);
   int32_t* info = reinterpret_cast<int32_t*>(ws + p.off_info);
   int32_t* counters = reinterpret_cast<int32_t*>(ws + p.off_counters);
   int32_t* hist = reinterpret_cast<int32_t*>(ws + p.off_hist);
@@ -2182,13 +2201,13 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
     const size_t topk_smem = decode_topk_smem(p.max_nc, p.cap);
     cudaFuncSetAttribute(wave_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)topk_smem);
-    TopkArgs ta{keys, hist, nonc, p.cap, p.topk_clusters, p.topk_fraction, info, sel_n};
+    TopkArgs ta{keys, hist, nonc, p.cap, p.topk_clusters, p.topk_fraction, info};
     e = launch_ex(wave_topk_kernel, dim3(p.U), dim3(kTopkThreads), topk_smem, s, pdl, p.geo, ta,
                   status);
     if (e != cudaSuccess) return e;
     mark(2);
     AttendArgs A{keys, scores, info, aff_of, p.max_nc, aff_start, st_slot, dv, p.cap, a.perm,
-                 p.n_sink, p.window, sel, sel_n, est_parts, p.n_score_blocks, p.n_rng, p.n_sc,
+                 p.n_sink, p.window, sel, p.sel_words, est_parts, p.n_score_blocks, p.n_rng, p.n_sc,
                  p.n_fold, p.n_parts, partials, counters, a.out, a.lse, p.scale};
     const size_t smem = decode_attend_smem(p.dtype, D, G, p.n_parts);
     cudaFuncSetAttribute(wave_attend_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,

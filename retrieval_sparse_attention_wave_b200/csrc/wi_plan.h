@@ -36,7 +36,8 @@ struct DecodePlan {
   float scale;             // 1/sqrt(d)
   // workspace byte offsets; [0, off_scores) must be zero before the first call
   size_t off_status, off_counters, off_hist, off_aff_of;
-  size_t off_scores, off_keys, off_sel, off_sel_n, off_info;
+  size_t off_scores, off_keys, off_sel, off_info;
+  int sel_words;           // selection bitmap words per unit (kRangeClusters / 32 per range CTA)
   size_t off_st_slot, off_st_cl, off_aff_cl, off_aff_start, off_partials;
   size_t off_dv, off_est, off_nonc;
   size_t off_q, off_out, off_lse;

@@ -100,6 +100,7 @@ def test_decode_workspace_size_and_layout():
     assert lay.total_bytes == n and lay.status == 0
     assert 0 < lay.scores < lay.keys < lay.selected < lay.unit_info < n
     assert lay.n_attend_ctas >= 2 and lay.n_score_ctas >= 1
+    assert lay.sel_words >= 8 and lay.sel_words % 8 == 0
 
 
 @pytest.mark.parametrize("over,expect", [

@@ -699,6 +699,7 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
   // tile i sits in slot i % NS and completes phase (i / NS) & 1 of its barrier
   auto tile_wait = [&](int i) { mbar_wait(&s_bar[i % NS], (uint32_t)((i / NS) & 1), status); };
 
+  int since_flush = 0;
   for (int kk = 0; kk < nk; ++kk) {
     const Chunk c = chunk(k0 + kk);
     const int* s_off = s_offb + (kk & 1) * (CROWS + 4);
@@ -758,7 +759,12 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
       __syncthreads();
       if (tid == 0) issue_tile(2 * kk + t + NS);
     }
-    if (c.nrows > 0) {  // histogram flush (two 16-bit counts per word)
+    // histogram flush (two 16-bit counts per word) when the next chunk is
+    // another unit's, after the last chunk, or before a count could reach
+    // 2^16; a barrier waits for the round trip of global atomics issued
+    // before it, so they are issued as rarely as possible
+    ++since_flush;
+    if (kk == nk - 1 || chunk(k0 + kk + 1).u != c.u || since_flush == 256) {
       int* hg = hist_g + (int64_t)c.u * kHistBins;
       for (int i = tid; i < kHistBins / 2; i += blockDim.x) {
         const uint32_t w = hist[i];
@@ -768,6 +774,7 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
           hist[i] = 0u;
         }
       }
+      since_flush = 0;
     }
     issue_meta(kk + 2);
   }
@@ -1559,6 +1566,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     }
   };
 
+  bool acc_used = !kMma;   // the CUDA-core accumulators hold part of the output
   pdl_wait();
   if (role_fold) {
     FoldArgs fa{A.est_parts, A.n_chunks, A.partials, A.n_parts, A.n_rng + A.n_sc, G, D};
@@ -1760,6 +1768,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
 #pragma unroll
       for (int e = 0; e < EPL; ++e) acc[g][e] = -cacc[g][e] * fe;
     }
+    acc_used = n_ce > 0;
    } else {
     // ------------------------------------------------- range CTA, CUDA cores
     const int c = (int)blockIdx.x * kRangeW + tid;
@@ -1926,7 +1935,14 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   }
   if (!role_fold) {
     __syncthreads();
-    reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part, kMma ? s_o : nullptr);
+    if (acc_used) {
+      reduce_and_store<G, EPL, LPR, D>(acc, s_red, warp, sub, rsub, part, kMma ? s_o : nullptr);
+    } else if constexpr (kMma) {   // nothing in acc: the part's output is s_o
+      for (int i = tid; i < G * D; i += blockDim.x) {
+        const int g = i / D;
+        part[g * PS + Part<D>::kO + (i - g * D)] = s_o[i];
+      }
+    }
     if (tid == 0) {
 #pragma unroll
       for (int g = 0; g < G; ++g) { part[g * PS] = m_run[g]; part[g * PS + 1] = l_run[g]; }
@@ -1934,17 +1950,22 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   }
 
   // ---------------------------------------- last CTA of the unit merges
-  __threadfence();
+  // (thread 0's acquire-release add orders the CTA's part writes, which the
+  // barrier ordered before it, ahead of the count; the last arrival acquires
+  // every other CTA's parts)
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(A.counters + u, 1) == A.n_rng + A.n_sc + A.n_fold - 1;
+  if (tid == 0) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(A.counters + u) : "memory");
+    s_last = old == A.n_rng + A.n_sc + A.n_fold - 1;
+  }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   // parts: [range CTAs | steady CTAs | folded estimation parts]; a unit with
   // nothing estimated (dense, or every candidate retrieved) merges the
   // first two groups alone
   const int32_t* I = A.info + (int64_t)u * kInfoInts;
-  const int np = (!I[6] && I[0] < I[7] && NC > 0) ? A.n_parts : A.n_rng + A.n_sc;
+  const int np = A.n_fold == 0 || (!I[6] && I[0] < I[7] && NC > 0) ? A.n_parts : A.n_rng + A.n_sc;
   // the parts stream through the ring and the correction rows (contiguous)
   // in batches: one cp.async round per batch, the first batch issued
   // together with the loads of every part's (m, l)
@@ -2123,6 +2144,17 @@ bool encode_rows128(CUtensorMap* tm, const void* base, int64_t rows) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Dynamic shared memory limit, and the full shared-memory carveout for every
+// decode kernel: kernels that run back to back (or overlap under
+// programmatic dependent launch) then never need the SM's L1 / shared split
+// reconfigured between them.
+template <typename Kern>
+void set_smem(Kern kern, size_t bytes) {
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                       (int)cudaSharedmemCarveoutMaxShared);
+}
+
 int sm_count() {
   int dev = 0, n = kNumSMs;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -2172,8 +2204,7 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
       if (!encode_rows128(&tmc, a.centroids, p.ncl) || !encode_rows128(&tm_vsum, a.value_sums, p.ncl))
         return cudaErrorInvalidValue;
       const size_t smem = std::max(MmaSmem<G>::kTotal, steady_smem);
-      cudaFuncSetAttribute(wave_score_mma_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
+      set_smem(wave_score_mma_kernel<G>, smem);
       int per_sm = 0;
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, wave_score_mma_kernel<G>,
                                                     kStreamThreads, smem);
@@ -2185,8 +2216,7 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
     }
     if (!done) {
       const size_t score_smem = steady_smem;
-      cudaFuncSetAttribute(wave_score_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)score_smem);
+      set_smem(wave_score_kernel<T, D, G>, score_smem);
       int per_sm = 0;
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, wave_score_kernel<T, D, G>,
                                                     kStreamThreads, score_smem);
@@ -2199,8 +2229,7 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
     if (e != cudaSuccess) return e;
     mark(1);
     const size_t topk_smem = decode_topk_smem(p.max_nc, p.cap);
-    cudaFuncSetAttribute(wave_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)topk_smem);
+    set_smem(wave_topk_kernel, topk_smem);
     TopkArgs ta{keys, hist, nonc, p.cap, p.topk_clusters, p.topk_fraction, info};
     e = launch_ex(wave_topk_kernel, dim3(p.U), dim3(kTopkThreads), topk_smem, s, pdl, p.geo, ta,
                   status);
@@ -2210,8 +2239,7 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
                  p.n_sink, p.window, sel, p.sel_words, est_parts, p.n_score_blocks, p.n_rng, p.n_sc,
                  p.n_fold, p.n_parts, partials, counters, a.out, a.lse, p.scale};
     const size_t smem = decode_attend_smem(p.dtype, D, G, p.n_parts);
-    cudaFuncSetAttribute(wave_attend_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
+    set_smem(wave_attend_kernel<T, D, G>, smem);
     e = launch_ex(wave_attend_kernel<T, D, G>, dim3(p.n_rng + p.n_sc + p.n_fold, p.U), dim3(kStreamThreads),
                   smem, s, pdl, p.geo, q, p.Hq, a.kp, a.vp,
                   reinterpret_cast<const T*>(a.value_sums), a.offsets, A, tm_vsum, status);

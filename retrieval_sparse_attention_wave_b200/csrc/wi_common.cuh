@@ -195,6 +195,15 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
+// The first 1024-byte boundary at or after p, a shared-memory pointer: the
+// offset is added to p itself (not computed through an integer round trip),
+// so the compiler keeps the shared address space and emits shared-memory
+// instructions for every access through the result.
+__device__ __forceinline__ unsigned char* align_smem_1024(unsigned char* p) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+  return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
 // ---- bulk (TMA) copies into shared memory, completed on an mbarrier
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);

@@ -631,8 +631,7 @@ wave_score_mma_kernel(const Geo geo, const __nv_bfloat16* __restrict__ q, int n_
     steady_role<T, D>(geo, blockIdx.x, sa, status, sh_raw);
     return;
   }
-  unsigned char* sh = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(sh_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sh = align_smem_1024(sh_raw);
   unsigned char* ring = sh;
   uint32_t* hist = reinterpret_cast<uint32_t*>(sh + SM::oHist);
   int* s_offb = reinterpret_cast<int*>(sh + SM::oOff);
@@ -1153,8 +1152,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   // repeats every 1024 bytes of address): [ring 64 KB: K x2, V x2 tiles, or
   // the range's value sums; the cross-warp reduction and the merge reuse it]
   // [correction rows kCorrRows x D fp32] [merge factors]
-  unsigned char* sh = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(sh_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sh = align_smem_1024(sh_raw);
   T* ring = reinterpret_cast<T*>(sh);
   float* s_red = reinterpret_cast<float*>(sh);
   unsigned char* s_crow = sh + 4 * 16384;
@@ -2011,11 +2009,12 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     const float mp = f[i];
     f[i] = mp == -INFINITY ? 0.f : expf(mp - s_m[i % G]);
   }
-  // each thread: outputs tid, tid + 256, ... of the G x D block
-  constexpr int OPT = (G * D + kStreamThreads - 1) / kStreamThreads;
-  float o[OPT];
+  // each thread: output pairs tid, tid + 256, ... of the G x D block, the
+  // parts taken two at a time into two accumulators (independent chains)
+  constexpr int OPT = (G * D / 2 + kStreamThreads - 1) / kStreamThreads;
+  float2 o[OPT];
 #pragma unroll
-  for (int k = 0; k < OPT; ++k) o[k] = 0.f;
+  for (int k = 0; k < OPT; ++k) o[k] = make_float2(0.f, 0.f);
   for (int p0 = 0; p0 < np; p0 += bcap) {
     if (p0 > 0) {
       __syncthreads();  // the previous batch is consumed
@@ -2026,23 +2025,39 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     const int nb = min(bcap, np - p0);
 #pragma unroll
     for (int k = 0; k < OPT; ++k) {
-      const int i = tid + k * kStreamThreads;
+      const int i = 2 * (tid + k * kStreamThreads);
       if (i < G * D) {
         const int g = i / D, e = i - g * D;
-        float acc_o = o[k];
-        for (int p = 0; p < nb; ++p) acc_o += f[(p0 + p) * G + g] * stage[p * PFL + g * PS + Part<D>::kO + e];
-        o[k] = acc_o;
+        const float* sp = stage + g * PS + Part<D>::kO + e;
+        const float* fp = f + p0 * G + g;
+        float2 a0 = o[k], a1 = make_float2(0.f, 0.f);
+        int p = 0;
+#pragma unroll 4
+        for (; p + 1 < nb; p += 2) {
+          const float2 v0 = *reinterpret_cast<const float2*>(sp + p * PFL);
+          const float2 v1 = *reinterpret_cast<const float2*>(sp + (p + 1) * PFL);
+          const float w0 = fp[p * G], w1 = fp[(p + 1) * G];
+          a0.x += w0 * v0.x; a0.y += w0 * v0.y;
+          a1.x += w1 * v1.x; a1.y += w1 * v1.y;
+        }
+        if (p < nb) {
+          const float2 v0 = *reinterpret_cast<const float2*>(sp + p * PFL);
+          const float w0 = fp[p * G];
+          a0.x += w0 * v0.x; a0.y += w0 * v0.y;
+        }
+        o[k] = make_float2(a0.x + a1.x, a0.y + a1.y);
       }
     }
   }
 #pragma unroll
   for (int k = 0; k < OPT; ++k) {
-    const int i = tid + k * kStreamThreads;
+    const int i = 2 * (tid + k * kStreamThreads);
     if (i < G * D) {
       const int g = i / D, e = i - g * D;
       const float l = s_l[g];
       const int64_t qh = (int64_t)b * n_q_heads + (int64_t)h * G + g;
-      A.out[qh * D + e] = l > 0.f ? o[k] / l : 0.f;
+      A.out[qh * D + e] = l > 0.f ? o[k].x / l : 0.f;   // (out is only 4-byte aligned)
+      A.out[qh * D + e + 1] = l > 0.f ? o[k].y / l : 0.f;
       if (e == 0 && A.lse != nullptr) A.lse[qh] = l > 0.f ? s_m[g] + logf(l) : -INFINITY;
     }
   }

@@ -194,6 +194,37 @@ wi_status wi_build_index(const wi_kv_cache *kv, int32_t seg_len, int32_t cluster
                          wi_stream_t stream);
 
 /*
+ * Extend a built index to longer sequences (RetroInfer 2.A, Segmented
+ * Clustering: the index is a sequence of independently clustered segments,
+ * so tokens appended while decoding join it segment by segment).
+ *
+ * old_ix  an index built (or extended) for lengths T_b = old_ix->seq_lens[b].
+ * kv      the KV cache in original token order, now of lengths
+ *         T'_b = kv->seq_lens[b] >= T_b.  Only positions from
+ *         s0_b = floor(T_b / seg_len) * seg_len on are read.
+ * out     the index for T'_b, with the seg_len and cluster_size of old_ix.
+ *         Its centroid, value-sum, offset, perm, invperm and label buffers
+ *         are new, sized for T'_b, and must not be old_ix's.  Its permuted
+ *         pools and block table must already hold old_ix's permuted rows for
+ *         every slot below s0_b (normally old_ix's own pools, with the block
+ *         table extended by pages for the new slots): those rows are not
+ *         read or written.
+ *
+ * The whole segments below s0_b are copied from old_ix. From s0_b on,
+ * segments are clustered anew and scattered: a partial last segment of
+ * old_ix is redone together with its new tokens. The result equals
+ * wi_build_index on the extended sequences with the same iters, bit for
+ * bit. Once its slots from s0_b on are rewritten, old_ix no longer matches
+ * a shared pool. Workspace: wi_build_workspace_size for kv.
+ *
+ * Errors are those of wi_build_index, plus WI_ERR_INVALID_ARG when old_ix's
+ * geometry differs from out's, when some T'_b < T_b, or when out reuses
+ * one of old_ix's index buffers.
+ */
+wi_status wi_extend_index(const wi_index *old_ix, const wi_kv_cache *kv, int32_t iters,
+                          const wi_index *out, void *ws, size_t ws_bytes, wi_stream_t stream);
+
+/*
  * One k-means assignment step with caller-given fp32 centroids
  * (RetroInfer 2.A, Segmented Clustering), the kernel wi_build_index uses.
  * centroids: device float [Hkv*sum NC_b][d] laid out like wi_index.centroids.

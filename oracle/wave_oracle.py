@@ -210,6 +210,53 @@ def build_unit(K: np.ndarray, V: np.ndarray, seg_len: int, cluster_size: int, it
                      labels=labels, centroids_exact=C, value_sums_exact=vsum)
 
 
+def extend_unit(old: UnitIndex, K: np.ndarray, V: np.ndarray, seg_len: int, cluster_size: int,
+                iters: int, store: str) -> UnitIndex:
+    """Grow the index `old` of a sequence's first T_old tokens to the longer
+    sequence K, V ([RI] 2.A, Segmented Clustering: segments are clustered
+    independently).  The segments of `old` that are whole are kept as they
+    are (their centroids, value sums, offsets, slots and labels); from the
+    first position they do not cover on, segments are clustered anew, a
+    partial last segment of `old` together with its new tokens."""
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    T, d = K.shape
+    T_old = len(old.perm)
+    assert T_old <= T
+    s0 = (T_old // seg_len) * seg_len                       # first position clustered anew
+    nc0 = (T_old // seg_len) * clusters_in_segment(seg_len, cluster_size)
+    labels = np.empty(T, dtype=np.int64)
+    labels[:s0] = old.labels[:s0]
+    cents, base = [], nc0
+    for start, n in segment_spans(T, seg_len):
+        if start < s0:
+            continue
+        lab, C, _ = kmeans_segment(K[start:start + n], cluster_size, iters)
+        labels[start:start + n] = lab + base
+        cents.append(C)
+        base += len(C)
+    NC = base
+    C_new = np.concatenate(cents, 0) if cents else np.zeros((0, d))
+    counts = np.bincount(labels[s0:] - nc0, minlength=NC - nc0)
+    offsets = np.zeros(NC + 1, dtype=np.int64)
+    offsets[:nc0 + 1] = old.offsets[:nc0 + 1]
+    offsets[nc0 + 1:] = s0 + np.cumsum(counts)
+    perm = np.concatenate([old.perm[:s0], s0 + np.argsort(labels[s0:], kind="stable")])
+    invperm = np.empty(T, dtype=np.int64)
+    invperm[perm] = np.arange(T)
+    vsum_new = np.zeros((NC - nc0, d))
+    np.add.at(vsum_new, labels[s0:] - nc0, V[s0:])
+    exact_c = exact_v = None
+    if old.centroids_exact is not None and old.value_sums_exact is not None:
+        exact_c = np.concatenate([old.centroids_exact[:nc0], C_new], 0)
+        exact_v = np.concatenate([old.value_sums_exact[:nc0], vsum_new], 0)
+    return UnitIndex(centroids=np.concatenate([old.centroids[:nc0], round_stored(C_new, store)], 0),
+                     value_sums=np.concatenate([old.value_sums[:nc0],
+                                                round_stored(vsum_new, store)], 0),
+                     offsets=offsets, perm=perm, invperm=invperm, k_perm=K[perm], v_perm=V[perm],
+                     labels=labels, centroids_exact=exact_c, value_sums_exact=exact_v)
+
+
 # ---------------------------------------------------------------------------
 # Decode: steady, retrieval and estimation zones ([RI] 2.A items 1-3)
 # ---------------------------------------------------------------------------

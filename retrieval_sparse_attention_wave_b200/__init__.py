@@ -42,7 +42,8 @@ WI_MAX_STEADY = 8192
 WI_DEV_BAD_PAGE, WI_DEV_BAD_SLOT, WI_DEV_BAD_CLUSTER, WI_DEV_BAD_HIST = 0x1, 0x2, 0x4, 0x8
 
 EXPORTED = [
-    "wi_index_clusters", "wi_build_workspace_size", "wi_build_index", "wi_kmeans_assign",
+    "wi_index_clusters", "wi_build_workspace_size", "wi_build_index", "wi_extend_index",
+    "wi_kmeans_assign",
     "wi_decode_workspace_size", "wi_decode_workspace_layout", "wi_decode", "wi_decode_host",
     "wi_decode_stage_count", "wi_decode_stage_name", "wi_read_device_status",
     "wi_status_string", "wi_last_error_string", "wi_decode_noalloc",
@@ -88,6 +89,8 @@ _sig = {
                                           C.POINTER(C.c_size_t)]),
     "wi_build_index": (C.c_int, [C.POINTER(WiKVCache), C.c_int32, C.c_int32, C.c_int32,
                                  C.POINTER(WiIndex), _P, C.c_size_t, _P]),
+    "wi_extend_index": (C.c_int, [C.POINTER(WiIndex), C.POINTER(WiKVCache), C.c_int32,
+                                  C.POINTER(WiIndex), _P, C.c_size_t, _P]),
     "wi_kmeans_assign": (C.c_int, [C.POINTER(WiKVCache), C.c_int32, C.c_int32, _P, _P, _P,
                                    C.c_size_t, _P]),
     "wi_decode_workspace_size": (C.c_int, [C.POINTER(WiIndex), C.POINTER(WiDecodeParams),
@@ -232,7 +235,7 @@ class WaveIndex:
 
     def __init__(self, seq_lens, n_kv_heads, head_dim, dtype, page_size, seg_len, cluster_size,
                  device, block_table: Optional[torch.Tensor] = None,
-                 n_pages: Optional[int] = None):
+                 n_pages: Optional[int] = None, pools=None):
         self.seq_lens = [int(t) for t in seq_lens]
         self.n_kv_heads, self.head_dim, self.dtype = n_kv_heads, head_dim, dtype
         self.page_size, self.seg_len, self.cluster_size = page_size, seg_len, cluster_size
@@ -251,8 +254,11 @@ class WaveIndex:
         if n_pages is None:
             n_pages = int(block_table.max().item()) + 1
         self.block_table = block_table.to(device=dev, dtype=torch.int32).contiguous()
-        self.k_pool = torch.zeros(n_pages, H, page_size, head_dim, dtype=dtype, device=dev)
-        self.v_pool = torch.zeros_like(self.k_pool)
+        if pools is not None:   # another index's permuted pools (an extension)
+            self.k_pool, self.v_pool = pools
+        else:
+            self.k_pool = torch.zeros(n_pages, H, page_size, head_dim, dtype=dtype, device=dev)
+            self.v_pool = torch.zeros_like(self.k_pool)
         self._seq = _i32_array(self.seq_lens)
 
     # unit (b, h) views ------------------------------------------------------
@@ -318,6 +324,25 @@ def build_index(kv: KVCache, seg_len: int, cluster_size: int, iters: int,
     s, o = kv.c_struct(), out.c_struct()
     _check(_lib.wi_build_index(C.byref(s), seg_len, cluster_size, iters, C.byref(o),
                                _ptr(ws), ws.numel(), _stream_ptr(stream)), "wi_build_index")
+    out._build_ws = ws
+    return out
+
+
+def extend_index(old: WaveIndex, kv: KVCache, iters: int, ws: Optional[torch.Tensor] = None,
+                 stream=None) -> WaveIndex:
+    """The index of the longer sequences in `kv`, grown from `old` segment by
+    segment (new centroid / value-sum / offset / perm / invperm / label
+    buffers; `old`'s permuted pools and block table are kept, so the block
+    table must already map pages for the new slots)."""
+    out = WaveIndex(kv.seq_lens, old.n_kv_heads, old.head_dim, old.dtype, old.page_size,
+                    old.seg_len, old.cluster_size, old.k_pool.device, old.block_table,
+                    old.k_pool.shape[0], pools=(old.k_pool, old.v_pool))
+    need = build_workspace_bytes(kv, old.seg_len, old.cluster_size)
+    if ws is None:
+        ws = workspace(need, kv.k_pool.device)
+    o_old, s, o = old.c_struct(), kv.c_struct(), out.c_struct()
+    _check(_lib.wi_extend_index(C.byref(o_old), C.byref(s), iters, C.byref(o), _ptr(ws),
+                                ws.numel(), _stream_ptr(stream)), "wi_extend_index")
     out._build_ws = ws
     return out
 

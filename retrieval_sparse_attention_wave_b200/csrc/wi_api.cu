@@ -195,6 +195,7 @@ wi_status make_build_plan(const wi_kv_cache* kv, int S, int cs, BuildPlan& pl) {
   int max_nseg = 0;
   for (int b = 0; b < kv->batch; ++b) max_nseg = std::max<int>(max_nseg, (int)cdiv(kv->seq_lens[b], S));
   pl.max_nseg = max_nseg;
+  pl.nseg_grid = max_nseg;   // every segment from the first (sf zero)
   pl.max_ncl_seg = S / cs;
   pl.update_smem = (size_t)(2 * pl.max_ncl_seg + 1 + 32) * 4 + (size_t)S * 2 * 2;
   const int64_t ncl = (int64_t)pl.geo.cl_base[kv->batch] * kv->n_kv_heads;
@@ -277,6 +278,57 @@ wi_status decode_workspace_extent(const wi_index* idx, const wi_decode_params* p
 
 }  // namespace wi
 
+namespace wi {
+namespace {
+// Checks of an index that a build writes, against the KV cache it is built from.
+wi_status check_build_out(const wi_kv_cache* kv, int32_t seg_len, int32_t cluster_size,
+                          const wi_index* out) {
+  if (!out) return WI_ERR_INVALID_ARG;
+  wi_status st;
+  if (out->dtype != kv->dtype || out->batch != kv->batch || out->n_kv_heads != kv->n_kv_heads ||
+      out->head_dim != kv->head_dim || out->page_size != kv->page_size ||
+      out->seg_len != seg_len || out->cluster_size != cluster_size || !out->seq_lens)
+    return WI_ERR_INVALID_ARG;
+  for (int b = 0; b < kv->batch; ++b)
+    if (out->seq_lens[b] != kv->seq_lens[b]) return WI_ERR_INVALID_ARG;
+  st = check_common(out->dtype, out->batch, out->n_kv_heads, out->head_dim, out->page_size,
+                    out->n_pages, out->k_pool, out->v_pool, out->block_table, out->max_pages,
+                    out->seq_lens);
+  if (st != WI_OK) return st;
+  if (!out->centroids || !out->value_sums || !out->offsets || !out->perm || !out->invperm ||
+      !out->labels)
+    return WI_ERR_INVALID_ARG;
+  if (!aligned(out->centroids, 16) || !aligned(out->value_sums, 16) || !aligned(out->offsets, 4) ||
+      !aligned(out->perm, 4) || !aligned(out->invperm, 4) || !aligned(out->labels, 4))
+    return WI_ERR_INVALID_ARG;
+  if (out->k_pool == kv->k_pool || out->v_pool == kv->v_pool || out->k_pool == kv->v_pool ||
+      out->v_pool == kv->k_pool)
+    return WI_ERR_INVALID_ARG;
+  return WI_OK;
+}
+
+BuildArgs build_args(const wi_kv_cache* kv, const wi_index* out, void* ws) {
+  BuildArgs a{};
+  a.kin = make_pool(kv->k_pool, kv->block_table, kv->n_pages, kv->max_pages, kv->page_size);
+  a.vin = make_pool(kv->v_pool, kv->block_table, kv->n_pages, kv->max_pages, kv->page_size);
+  a.centroids = out->centroids;
+  a.value_sums = out->value_sums;
+  a.offsets = out->offsets;
+  a.perm = out->perm;
+  a.invperm = out->invperm;
+  a.labels = out->labels;
+  a.kout = out->k_pool;
+  a.vout = out->v_pool;
+  a.bt_out = out->block_table;
+  a.n_pages_out = out->n_pages;
+  a.max_pages_out = out->max_pages;
+  a.page_shift_out = ilog2(out->page_size);
+  a.ws = static_cast<unsigned char*>(ws);
+  return a;
+}
+}  // namespace
+}  // namespace wi
+
 using namespace wi;
 
 extern "C" {
@@ -307,51 +359,68 @@ wi_status wi_build_workspace_size(const wi_kv_cache* kv, int32_t seg_len, int32_
   return WI_OK;
 }
 
+
 wi_status wi_build_index(const wi_kv_cache* kv, int32_t seg_len, int32_t cluster_size,
                          int32_t iters, const wi_index* out, void* ws, size_t ws_bytes,
                          wi_stream_t stream) {
   BuildPlan pl;
   wi_status st = make_build_plan(kv, seg_len, cluster_size, pl);
   if (st != WI_OK) return st;
-  if (iters < 1 || !out) return WI_ERR_INVALID_ARG;
-  if (out->dtype != kv->dtype || out->batch != kv->batch || out->n_kv_heads != kv->n_kv_heads ||
-      out->head_dim != kv->head_dim || out->page_size != kv->page_size ||
-      out->seg_len != seg_len || out->cluster_size != cluster_size || !out->seq_lens)
-    return WI_ERR_INVALID_ARG;
-  for (int b = 0; b < kv->batch; ++b)
-    if (out->seq_lens[b] != kv->seq_lens[b]) return WI_ERR_INVALID_ARG;
-  st = check_common(out->dtype, out->batch, out->n_kv_heads, out->head_dim, out->page_size,
-                    out->n_pages, out->k_pool, out->v_pool, out->block_table, out->max_pages,
-                    out->seq_lens);
-  if (st != WI_OK) return st;
-  if (!out->centroids || !out->value_sums || !out->offsets || !out->perm || !out->invperm ||
-      !out->labels)
-    return WI_ERR_INVALID_ARG;
-  if (!aligned(out->centroids, 16) || !aligned(out->value_sums, 16) || !aligned(out->offsets, 4) ||
-      !aligned(out->perm, 4) || !aligned(out->invperm, 4) || !aligned(out->labels, 4))
-    return WI_ERR_INVALID_ARG;
-  if (out->k_pool == kv->k_pool || out->v_pool == kv->v_pool || out->k_pool == kv->v_pool ||
-      out->v_pool == kv->k_pool)
-    return WI_ERR_INVALID_ARG;
+  if (iters < 1) return WI_ERR_INVALID_ARG;
+  if ((st = check_build_out(kv, seg_len, cluster_size, out)) != WI_OK) return st;
   pl.iters = iters;
   if ((st = check_ws(ws, ws_bytes, pl.total)) != WI_OK) return st;
-  BuildArgs a{};
-  a.kin = make_pool(kv->k_pool, kv->block_table, kv->n_pages, kv->max_pages, kv->page_size);
-  a.vin = make_pool(kv->v_pool, kv->block_table, kv->n_pages, kv->max_pages, kv->page_size);
-  a.centroids = out->centroids;
-  a.value_sums = out->value_sums;
-  a.offsets = out->offsets;
-  a.perm = out->perm;
-  a.invperm = out->invperm;
-  a.labels = out->labels;
-  a.kout = out->k_pool;
-  a.vout = out->v_pool;
-  a.bt_out = out->block_table;
-  a.n_pages_out = out->n_pages;
-  a.max_pages_out = out->max_pages;
-  a.page_shift_out = ilog2(out->page_size);
-  a.ws = static_cast<unsigned char*>(ws);
+  const BuildArgs a = build_args(kv, out, ws);
   const cudaError_t e = launch_build(pl, a, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WI_OK : cuda_fail(e);
+}
+
+wi_status wi_extend_index(const wi_index* old_ix, const wi_kv_cache* kv, int32_t iters,
+                          const wi_index* out, void* ws, size_t ws_bytes, wi_stream_t stream) {
+  if (!old_ix || !kv || !out) return WI_ERR_INVALID_ARG;
+  const int32_t S = out->seg_len, cs = out->cluster_size;
+  BuildPlan pl;
+  wi_status st = make_build_plan(kv, S, cs, pl);
+  if (st != WI_OK) return st;
+  if (iters < 1) return WI_ERR_INVALID_ARG;
+  if ((st = check_build_out(kv, S, cs, out)) != WI_OK) return st;
+  // the old index: same geometry, no sequence longer than now
+  if (old_ix->dtype != kv->dtype || old_ix->batch != kv->batch ||
+      old_ix->n_kv_heads != kv->n_kv_heads || old_ix->head_dim != kv->head_dim ||
+      old_ix->page_size != kv->page_size || old_ix->seg_len != S || old_ix->cluster_size != cs ||
+      !old_ix->seq_lens || !old_ix->centroids || !old_ix->value_sums || !old_ix->offsets ||
+      !old_ix->perm || !old_ix->invperm || !old_ix->labels)
+    return WI_ERR_INVALID_ARG;
+  if (!aligned(old_ix->centroids, 16) || !aligned(old_ix->value_sums, 16))
+    return WI_ERR_INVALID_ARG;
+  if (old_ix->centroids == out->centroids || old_ix->value_sums == out->value_sums ||
+      old_ix->offsets == out->offsets || old_ix->perm == out->perm ||
+      old_ix->invperm == out->invperm || old_ix->labels == out->labels)
+    return WI_ERR_INVALID_ARG;
+  for (int b = 0; b < kv->batch; ++b)
+    if (old_ix->seq_lens[b] < 1 || old_ix->seq_lens[b] > kv->seq_lens[b]) return WI_ERR_INVALID_ARG;
+  ExtendCopy c{};
+  fill_geo(c.gold, old_ix->batch, old_ix->n_kv_heads, old_ix->head_dim, old_ix->seq_lens, S, cs);
+  c.centroids = old_ix->centroids;
+  c.value_sums = old_ix->value_sums;
+  c.offsets = old_ix->offsets;
+  c.perm = old_ix->perm;
+  c.invperm = old_ix->invperm;
+  c.labels = old_ix->labels;
+  // whole segments of the old index are kept; from its first incomplete one
+  // (or the first new one) on, segments are clustered anew
+  int nseg_grid = 0;
+  for (int b = 0; b < kv->batch; ++b) {
+    pl.sf.s0[b] = old_ix->seq_lens[b] / S;
+    nseg_grid = std::max<int>(nseg_grid, (int)cdiv(kv->seq_lens[b], S) - pl.sf.s0[b]);
+  }
+  pl.nseg_grid = nseg_grid;
+  pl.iters = iters;
+  if ((st = check_ws(ws, ws_bytes, pl.total)) != WI_OK) return st;
+  const BuildArgs a = build_args(kv, out, ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_extend_copy(pl, c, a, s);
+  if (e == cudaSuccess) e = launch_build(pl, a, s);
   return e == cudaSuccess ? WI_OK : cuda_fail(e);
 }
 

@@ -31,12 +31,12 @@ struct BRow {
 // ------------------------------------------------------------------- init
 template <typename T, int D>
 __global__ void __launch_bounds__(kStreamThreads)
-kmeans_init_kernel(const Geo geo, const Pool kin, int S, int cs, float* __restrict__ cent32,
-                   uint32_t* status) {
+kmeans_init_kernel(const Geo geo, const Pool kin, int S, int cs, const SegFrom sf,
+                   float* __restrict__ cent32, uint32_t* status) {
   using R = BRow<T, D>;
   const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
   const int T_ = geo.T(b);
-  const int seg = blockIdx.x, start = seg * S;
+  const int seg = sf.s0[b] + (int)blockIdx.x, start = seg * S;
   if (start >= T_) return;
   const int len = min(S, T_ - start);
   const int ncl = (len + cs - 1) / cs;
@@ -65,15 +65,16 @@ constexpr int kTok = 64, kCen = 64, kPad = 4;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
-kmeans_assign_kernel(const Geo geo, const Pool kin, int S, int cs, const float* __restrict__ cent32,
-                     int32_t* __restrict__ assign, uint32_t* status) {
+kmeans_assign_kernel(const Geo geo, const Pool kin, int S, int cs, const SegFrom sf,
+                     const float* __restrict__ cent32, int32_t* __restrict__ assign,
+                     uint32_t* status) {
   using R = BRow<T, D>;
   extern __shared__ float4 sh_assign4[];
   float* sk = reinterpret_cast<float*>(sh_assign4);      // [D][kTok + kPad]
   float* sc = sk + D * (kTok + kPad);                    // [D][kCen + kPad]
   const int u = blockIdx.z, b = u / geo.hkv, h = u - b * geo.hkv;
   const int T_ = geo.T(b);
-  const int seg = blockIdx.y, start = seg * S;
+  const int seg = sf.s0[b] + (int)blockIdx.y, start = seg * S;
   if (start >= T_) return;
   const int len = min(S, T_ - start);
   const int t0 = blockIdx.x * kTok;
@@ -186,13 +187,14 @@ struct FinalOut {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kUpdThreads)
-kmeans_update_kernel(const Geo geo, const Pool kin, int S, int cs, float* __restrict__ cent32,
-                     const int32_t* __restrict__ assign, const FinalOut fo, uint32_t* status) {
+kmeans_update_kernel(const Geo geo, const Pool kin, int S, int cs, const SegFrom sf,
+                     float* __restrict__ cent32, const int32_t* __restrict__ assign,
+                     const FinalOut fo, uint32_t* status) {
   using R = BRow<T, D>;
   extern __shared__ int32_t sh_upd[];
   const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
   const int T_ = geo.T(b);
-  const int seg = blockIdx.x, start = seg * S;
+  const int seg = sf.s0[b] + (int)blockIdx.x, start = seg * S;
   if (start >= T_) return;
   const int len = min(S, T_ - start);
   const int ncl = (len + cs - 1) / cs;
@@ -310,6 +312,42 @@ kmeans_update_kernel(const Geo geo, const Pool kin, int S, int cs, float* __rest
   if (fo.enabled && tid == 0 && start + len == T_) fo.offsets[geo.off_row(b, h) + geo.NC(b)] = T_;
 }
 
+// ----------------------------------------------------------- extension copy
+// Unit blockIdx.y: the first s0 * S / cs clusters (centroid and value-sum
+// rows, their offsets and the offset after them) and the first s0 * S tokens
+// (perm, invperm, labels) of the old index, moved to the unit's rows of the
+// new index.  Those segments are whole in both, so their slots, clusters and
+// labels keep their numbers.
+template <typename T, int D>
+__global__ void __launch_bounds__(kStreamThreads)
+extend_copy_kernel(const Geo gnew, const Geo gold, int S, int cs, const SegFrom sf,
+                   const ExtendCopy c, void* __restrict__ centroids, void* __restrict__ value_sums,
+                   int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+                   int32_t* __restrict__ invperm, int32_t* __restrict__ labels) {
+  const int u = blockIdx.y, b = u / gnew.hkv, h = u - b * gnew.hkv;
+  const int ncc = sf.s0[b] * (S / cs);          // clusters kept
+  const int ntc = sf.s0[b] * S;                 // tokens kept
+  constexpr int V = 16 / (int)sizeof(T);        // elements per 16-byte vector
+  const int64_t ro = gold.cl_row(b, h) * D, rn = gnew.cl_row(b, h) * D;
+  const int nvec = ncc * D / V;
+  const int stride = gridDim.x * blockDim.x;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nvec; i += stride) {
+    reinterpret_cast<uint4*>(static_cast<T*>(centroids) + rn)[i] =
+        reinterpret_cast<const uint4*>(static_cast<const T*>(c.centroids) + ro)[i];
+    reinterpret_cast<uint4*>(static_cast<T*>(value_sums) + rn)[i] =
+        reinterpret_cast<const uint4*>(static_cast<const T*>(c.value_sums) + ro)[i];
+  }
+  const int64_t oo = gold.off_row(b, h), on = gnew.off_row(b, h);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= ncc; i += stride)
+    offsets[on + i] = c.offsets[oo + i];
+  const int64_t to = gold.tok_row(b, h), tn = gnew.tok_row(b, h);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < ntc; i += stride) {
+    perm[tn + i] = c.perm[to + i];
+    invperm[tn + i] = c.invperm[to + i];
+    labels[tn + i] = c.labels[to + i];
+  }
+}
+
 template <typename F>
 cudaError_t with_build_types(int dtype, int D, F&& f) {
   if (dtype == WI_BF16) {
@@ -333,9 +371,9 @@ cudaError_t launch_assign_only(const BuildPlan& p, const BuildArgs& a, const flo
     const size_t smem = assign_smem(D);
     cudaFuncSetAttribute(kmeans_assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    const dim3 grid((p.S + kTok - 1) / kTok, p.max_nseg, p.U);
-    kmeans_assign_kernel<T, D><<<grid, 256, smem, s>>>(p.geo, a.kin, p.S, p.cs, cent32, assign,
-                                                       status);
+    const dim3 grid((p.S + kTok - 1) / kTok, p.nseg_grid, p.U);
+    kmeans_assign_kernel<T, D><<<grid, 256, smem, s>>>(p.geo, a.kin, p.S, p.cs, p.sf, cent32,
+                                                       assign, status);
     return cudaGetLastError();
   });
 }
@@ -350,8 +388,9 @@ cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s)
                          (int)smem);
     cudaFuncSetAttribute(kmeans_update_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)p.update_smem);
-    kmeans_init_kernel<T, D><<<dim3(p.max_nseg, p.U), kStreamThreads, 0, s>>>(
-        p.geo, a.kin, p.S, p.cs, cent32, status);
+    if (p.nseg_grid < 1) return cudaSuccess;   // nothing new to cluster
+    kmeans_init_kernel<T, D><<<dim3(p.nseg_grid, p.U), kStreamThreads, 0, s>>>(
+        p.geo, a.kin, p.S, p.cs, p.sf, cent32, status);
     FinalOut none{};
     none.enabled = 0;
     FinalOut fin{};
@@ -366,13 +405,23 @@ cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s)
     fin.pout = Pool{a.kout, a.bt_out, a.n_pages_out, a.max_pages_out, a.page_shift_out};
     fin.vin = a.vin;
     fin.enabled = 1;
-    const dim3 agrid((p.S + kTok - 1) / kTok, p.max_nseg, p.U);
+    const dim3 agrid((p.S + kTok - 1) / kTok, p.nseg_grid, p.U);
     for (int it = 0; it < p.iters; ++it) {
-      kmeans_assign_kernel<T, D><<<agrid, 256, smem, s>>>(p.geo, a.kin, p.S, p.cs, cent32, assign,
-                                                          status);
-      kmeans_update_kernel<T, D><<<dim3(p.max_nseg, p.U), kUpdThreads, p.update_smem, s>>>(
-          p.geo, a.kin, p.S, p.cs, cent32, assign, it == p.iters - 1 ? fin : none, status);
+      kmeans_assign_kernel<T, D><<<agrid, 256, smem, s>>>(p.geo, a.kin, p.S, p.cs, p.sf, cent32,
+                                                          assign, status);
+      kmeans_update_kernel<T, D><<<dim3(p.nseg_grid, p.U), kUpdThreads, p.update_smem, s>>>(
+          p.geo, a.kin, p.S, p.cs, p.sf, cent32, assign, it == p.iters - 1 ? fin : none, status);
     }
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t launch_extend_copy(const BuildPlan& p, const ExtendCopy& c, const BuildArgs& a,
+                               cudaStream_t s) {
+  return with_build_types(p.dtype, p.D, [&]<typename T, int D>() -> cudaError_t {
+    extend_copy_kernel<T, D><<<dim3(16, p.U), kStreamThreads, 0, s>>>(
+        p.geo, c.gold, p.S, p.cs, p.sf, c, a.centroids, a.value_sums, a.offsets, a.perm,
+        a.invperm, a.labels);
     return cudaGetLastError();
   });
 }

@@ -44,10 +44,18 @@ struct DecodePlan {
   size_t total;
 };
 
+// First segment each sequence's build kernels process (all zero for a full
+// build; an index extension starts at the old index's first incomplete one).
+struct SegFrom {
+  int32_t s0[kMaxBatch];
+};
+
 struct BuildPlan {
   Geo geo;
   int dtype, D, U, S, cs, iters;
   int max_nseg, max_ncl_seg;
+  SegFrom sf;              // first segment per sequence
+  int nseg_grid;           // max over sequences of (segments - first segment)
   size_t update_smem;
   size_t off_status, off_cent32, off_assign;
   size_t total;
@@ -97,6 +105,20 @@ size_t decode_attend_smem(int dtype, int D, int G, int n_parts);
 size_t decode_score_smem(int dtype, int D, int G, int sort_pow2, int cap);
 size_t decode_topk_smem(int max_nc, int cap);
 cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s);
+// Copy the part of an old index that an extension keeps (segments below
+// p.sf.s0[b]) into the new index's buffers: centroid and value-sum rows,
+// offsets, perm, invperm and labels.
+struct ExtendCopy {
+  Geo gold;
+  const void* centroids;
+  const void* value_sums;
+  const int32_t* offsets;
+  const int32_t* perm;
+  const int32_t* invperm;
+  const int32_t* labels;
+};
+cudaError_t launch_extend_copy(const BuildPlan& p, const ExtendCopy& c, const BuildArgs& a,
+                               cudaStream_t s);
 cudaError_t launch_assign_only(const BuildPlan& p, const BuildArgs& a, const float* cent32,
                                int32_t* assign, cudaStream_t s);
 

@@ -189,6 +189,33 @@ def test_build_validation():
         == W.WI_ERR_INVALID_ARG
 
 
+def test_extend_validation():
+    """wi_extend_index checks every argument before any launch."""
+    lib = W.lib()
+    kv = kv_struct(seq=[4096])
+    n = C.c_size_t()
+    assert lib.wi_build_workspace_size(C.byref(kv), 1024, 16, C.byref(n)) == W.WI_OK
+    out = index_struct(seq=[4096])
+    old = index_struct(seq=[3000], **{f: FAKE + (20 + i) * 0x1000000 for i, f in enumerate(
+        ["centroids", "value_sums", "offsets", "perm", "invperm", "labels"])})
+    ext = lambda o, k, it, x, nb: lib.wi_extend_index(o, k, it, x, FAKE, nb, None)
+    assert ext(None, C.byref(kv), 3, C.byref(out), n.value) == W.WI_ERR_INVALID_ARG
+    assert ext(C.byref(old), C.byref(kv), 0, C.byref(out), n.value) == W.WI_ERR_INVALID_ARG
+    # the old index longer than the new sequences
+    longer = index_struct(seq=[5000], **{f: getattr(old, f) for f in ["centroids", "value_sums",
+                                                                      "offsets", "perm",
+                                                                      "invperm", "labels"]})
+    assert ext(C.byref(longer), C.byref(kv), 3, C.byref(out), n.value) == W.WI_ERR_INVALID_ARG
+    # the new index reusing one of the old index's buffers
+    reuse = index_struct(seq=[4096], perm=old.perm)
+    assert ext(C.byref(old), C.byref(kv), 3, C.byref(reuse), n.value) == W.WI_ERR_INVALID_ARG
+    # another segment length than the old index
+    other = index_struct(seq=[3000], seg_len=512)
+    assert ext(C.byref(other), C.byref(kv), 3, C.byref(out), n.value) == W.WI_ERR_INVALID_ARG
+    # workspace too small
+    assert ext(C.byref(old), C.byref(kv), 3, C.byref(out), 1024) == W.WI_ERR_WORKSPACE
+
+
 def test_status_strings():
     lib = W.lib()
     for s in range(6):

@@ -157,6 +157,25 @@ def test_build_layout_invariants():
         np.testing.assert_allclose(ix.value_sums_exact[c], V[members].sum(0), atol=1e-12)
 
 
+@pytest.mark.parametrize("T_old,T_new", [(1500, 2900), (1024, 2048), (700, 700), (2048, 2048),
+                                         (1, 1030)])
+def test_extension_equals_build_of_the_longer_sequence(T_old, T_new):
+    """Segments are clustered independently ([RI] 2.A, Segmented Clustering),
+    so growing the index of the first T_old tokens to T_new tokens equals
+    building it for T_new tokens: every field, exactly."""
+    rng = np.random.default_rng(11)
+    K, V, _ = mixture(rng, T_new, 8, n_centers=12)
+    for store in ("f32", "bf16"):
+        old = O.build_unit(K[:T_old], V[:T_old], seg_len=512, cluster_size=16, iters=3, store=store)
+        ext = O.extend_unit(old, K, V, seg_len=512, cluster_size=16, iters=3, store=store)
+        ref = O.build_unit(K, V, seg_len=512, cluster_size=16, iters=3, store=store)
+        for f in ("centroids", "value_sums", "offsets", "perm", "invperm", "labels", "k_perm",
+                  "v_perm", "centroids_exact"):
+            np.testing.assert_array_equal(getattr(ext, f), getattr(ref, f), err_msg=f)
+        # exact value sums agree to summation order (the kept ones are copied)
+        np.testing.assert_allclose(ext.value_sums_exact, ref.value_sums_exact, atol=1e-12)
+
+
 # --------------------------------------------------------------- decode pins
 
 def test_steady_positions():

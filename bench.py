@@ -243,7 +243,25 @@ def run_wave(args, rank, world, local_rank):
     torch.cuda.synchronize()
     build_ms = b0.elapsed_time(b1)
     assert W.read_device_status(wx._build_ws) == 0
-    del kv
+
+    # index extension: each sequence's last seg_len tokens arrive later (as a
+    # decode appends them); the index of the shorter sequences grows to the
+    # full ones, timed with events, and must equal the full build
+    old_lens = [max(1, T - wl.seg_len) for T in wl.seq_lens]
+    kv_old = W.KVCache(kv.k_pool, kv.v_pool, kv.block_table, old_lens)
+    old = W.build_index(kv_old, wl.seg_len, wl.cluster_size, wl.iters, block_table=bt_out,
+                        n_pages=n_out)
+    W.extend_index(old, kv, wl.iters)   # warm
+    torch.cuda.synchronize()
+    b0.record()
+    ext = W.extend_index(old, kv, wl.iters)
+    b1.record()
+    torch.cuda.synchronize()
+    extend_ms = b0.elapsed_time(b1)
+    assert W.read_device_status(ext._build_ws) == 0
+    assert torch.equal(ext.centroids, wx.centroids) and torch.equal(ext.perm, wx.perm)
+    extend_tokens = sum(T - t for T, t in zip(wl.seq_lens, old_lens))
+    del kv, kv_old, old, ext
     torch.cuda.empty_cache()
 
     params = W.DecodeParams(n_q_heads=wl.n_q_heads, n_sink=wl.n_sink, window=wl.window,
@@ -421,6 +439,9 @@ def run_wave(args, rank, world, local_rank):
         "build": {"ms": build_ms, "iters": wl.iters, "assign_tflop": assign_flop / 1e12,
                   "assign_tflops_achieved": assign_flop / (build_ms * 1e-3) / 1e12,
                   "bound": "alu", "peak_tflops": FP32_ALU_TFLOPS},
+        "extend": {"ms": extend_ms, "iters": wl.iters, "new_tokens": extend_tokens,
+                   "note": "index grown by the last seg_len tokens of every sequence; "
+                           "equals the full build"},
         "clocks": clk,
     }
     return result, wx, wl

@@ -987,13 +987,33 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, uint32_t* status) {
   int mine = 0;
   for (int r = 0; r < n_rounds; ++r) {
     if (r > 0) { load_round(r); mask_round(r); }
+    // the round's threshold-bin members: counted per thread, placed by one
+    // warp prefix and one shared-memory atomic per warp (the list is a set:
+    // its order does not matter)
+    int nm = 0;
 #pragma unroll
     for (int i = 0; i < PT; ++i) {
-      const uint32_t key = kr[i];
-      mine += key != 0u;
-      append(key != 0u && (int)(key >> kHistShift) == bin1,
-             ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)cid(r, i)), cand, kTopkCand,
-             &s_ctl[0]);
+      mine += kr[i] != 0u;
+      nm += kr[i] != 0u && (int)(kr[i] >> kHistShift) == bin1;
+    }
+    int incl = nm;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int wb = 0;
+    if (lane == 31 && incl > 0) wb = atomicAdd(&s_ctl[0], incl);
+    int pos = __shfl_sync(0xffffffffu, wb, 31) + incl - nm;
+    if (nm > 0) {
+#pragma unroll
+      for (int i = 0; i < PT; ++i) {
+        if (kr[i] != 0u && (int)(kr[i] >> kHistShift) == bin1) {
+          if (pos < kTopkCand)
+            cand[pos] = ((unsigned long long)kr[i] << 32) | (0xFFFFFFFFu - (uint32_t)cid(r, i));
+          ++pos;
+        }
+      }
     }
   }
   int ncand;

@@ -49,14 +49,21 @@ def measured_peaks():
 
 
 def kernel_source_sha256() -> str:
-    """Hash of the CUDA sources (csrc/*.cu, *.cuh, *.h) in file-name order."""
+    """Hash of the CUDA sources (csrc/*.cu, *.cuh, *.h) in file-name order,
+    comments and blank lines left out: a comment edit does not change the
+    compiled kernels, so it keeps the measured traffic valid."""
     import glob
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "retrieval_sparse_attention_wave_b200", "csrc", "*"))):
         if f.endswith((".cu", ".cuh", ".h")):
-            with open(f, "rb") as fh:
-                h.update(fh.read())
+            with open(f) as fh:
+                src = fh.read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            src = re.sub(r"//[^\n]*", "", src)
+            src = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+            h.update(src.encode())
     return h.hexdigest()
 
 

@@ -1106,8 +1106,8 @@ wave_topk_kernel(const Geo geo, const TopkArgs A, uint32_t* status) {
 
 // ----------------------------------------------------------------- K_C attend
 // range CTAs (kRangeW cluster ids each): pick the retrieved clusters of the
-// range against K_B's threshold, append them to the unit's (unordered)
-// selection list, resolve their tokens' pool rows (skipping steady members)
+// range against K_B's threshold, write the range's words of the unit's
+// selection bitmap, resolve their tokens' pool rows (skipping steady members)
 // and run exact attention over them.  The estimation zone of the range goes
 // into the same part:
 //  - tensor-core path (bf16, d = 128): the range's value sums (64 KB) are

@@ -15,7 +15,7 @@ constexpr int kAttendTile = 64;       // tokens per exact-attention tile
 constexpr int kInfoInts = 8;          // per-unit info record (see wi_decode_layout)
 constexpr int kNumSMs = 148;          // B200
 constexpr int kScoreChunkBytes = 32768;  // centroid bytes (and as many value-sum bytes) per score CTA
-constexpr int kFold = 16;             // score-chunk parts folded into one by a K_B fold CTA
+constexpr int kFold = 16;             // score-chunk parts folded into one by an attend fold CTA
 constexpr int kRangeClusters = 256;   // cluster ids per attend range CTA (one per thread)
 
 struct DecodePlan {

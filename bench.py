@@ -268,6 +268,10 @@ def run_wave(args, rank, world, local_rank):
     assert W.read_device_status(ext._build_ws) == 0
     assert torch.equal(ext.centroids, wx.centroids) and torch.equal(ext.perm, wx.perm)
     extend_tokens = sum(T - t for T, t in zip(wl.seq_lens, old_lens))
+    # the block top-k workload's index: position blocks of cluster_size tokens
+    bx = W.build_blocks(kv, wl.seg_len, wl.cluster_size, block_table=bt_out, n_pages=n_out)
+    torch.cuda.synchronize()
+    assert W.read_device_status(bx._build_ws) == 0
     del kv, kv_old, old, ext
     torch.cuda.empty_cache()
 
@@ -397,6 +401,42 @@ def run_wave(args, rank, world, local_rank):
     assert np.isfinite(out_h.numpy()).all()
     assert W.read_device_status(ws, stream) == 0
 
+    # block top-k workload (exact attention over the top 1.8% blocks and the
+    # steady zone, no estimation zone) on the block index, and the wave
+    # decode under the same protocol: one CUDA graph per step, L2 flushed by
+    # a 2 x L2 write outside each timed step
+    bparams = W.DecodeParams(n_q_heads=wl.n_q_heads, n_sink=wl.n_sink, window=wl.window,
+                             topk_clusters=wl.topk_clusters, topk_fraction=wl.topk_fraction,
+                             exact_only=True)
+    bws = W.decode_workspace(bx, bparams)
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+    def flushed_us(ix, prm, wsp, n=50):
+        o = torch.empty(wl.batch, wl.n_q_heads, wl.head_dim, dtype=torch.float32, device=dev)
+        lo = torch.empty(wl.batch, wl.n_q_heads, dtype=torch.float32, device=dev)
+        with torch.cuda.stream(stream):
+            W.decode(q, ix, prm, out=o, lse=lo, ws=wsp, stream=stream)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                W.decode(q, ix, prm, out=o, lse=lo, ws=wsp, stream=stream)
+            tot = 0.0
+            for _ in range(n + 3):
+                flush.fill_(1)
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record(stream)
+                g.replay()
+                a1.record(stream)
+                stream.synchronize()
+                tot += a0.elapsed_time(a1) if _ >= 3 else 0.0
+        assert W.read_device_status(wsp, stream) == 0 and torch.isfinite(o).all()
+        del g
+        return tot * 1e3 / n
+
+    block_us = flushed_us(bx, bparams, bws)
+    wave_flushed_us = flushed_us(wx, params, ws)
+    del bx, bws, flush
+
     peaks, peak_kind = measured_peaks()
     hbm = float(peaks["hbm_gbs"])
     dom = max(("score", "topk", "attend"), key=lambda k: stage_us[k])
@@ -446,6 +486,10 @@ def run_wave(args, rank, world, local_rank):
         "build": {"ms": build_ms, "iters": wl.iters, "assign_tflop": assign_flop / 1e12,
                   "assign_tflops_achieved": assign_flop / (build_ms * 1e-3) / 1e12,
                   "bound": "alu", "peak_tflops": FP32_ALU_TFLOPS},
+        "block_topk": {"us_per_step": block_us, "wave_us_per_step_same_protocol": wave_flushed_us,
+                       "note": "exact attention over the top blocks of cluster_size tokens "
+                               "and the steady zone, no estimation; one graph per step, "
+                               "L2 flushed between steps"},
         "extend": {"ms": extend_ms, "iters": wl.iters, "new_tokens": extend_tokens,
                    "note": "index grown by the last seg_len tokens of every sequence; "
                            "equals the full build"},

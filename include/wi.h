@@ -140,6 +140,10 @@ typedef struct wi_decode_params {
   double topk_fraction;        /* in [0, 1], used when topk_clusters < 0        */
   wi_event_t *stage_events;    /* optional: wi_decode_stage_count()+1 events,
                                   recorded before each stage and after the last */
+  int32_t exact_only;          /* nonzero: no estimation zone; the output is
+                                  attention over the retrieved clusters and the
+                                  steady zone only (the block top-k workload of
+                                  Vortex 2.A on a wi_build_blocks index)        */
 } wi_decode_params;
 
 /* Byte offsets of the decode workspace regions (for inspection and tests). */
@@ -192,6 +196,22 @@ wi_status wi_build_workspace_size(const wi_kv_cache *kv, int32_t seg_len,
 wi_status wi_build_index(const wi_kv_cache *kv, int32_t seg_len, int32_t cluster_size,
                          int32_t iters, const wi_index *out, void *ws, size_t ws_bytes,
                          wi_stream_t stream);
+
+/*
+ * Build an index of position-contiguous blocks (Vortex summary, section 2.A:
+ * forward_cache builds block centroids; forward_indexer then selects the
+ * top-k blocks and attends).  Inside each segment of seg_len positions,
+ * block j holds positions j*block_size .. (j+1)*block_size - 1 (the last one
+ * may be shorter); its centroid is the mean key and its value sum the sum of
+ * its values, both rounded to the KV dtype; perm is the identity and the K/V
+ * rows are copied to out's pools in position order.  `out` is laid out like
+ * any index, with cluster_size = block_size.  Decode it with
+ * wi_decode_params.exact_only set for the block top-k workload (or without,
+ * to estimate the unselected blocks).  Same workspace as wi_build_index and
+ * the same argument errors (block_size in the cluster_size role).
+ */
+wi_status wi_build_blocks(const wi_kv_cache *kv, int32_t seg_len, int32_t block_size,
+                          const wi_index *out, void *ws, size_t ws_bytes, wi_stream_t stream);
 
 /*
  * Extend a built index to longer sequences (RetroInfer 2.A, Segmented

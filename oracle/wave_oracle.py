@@ -210,6 +210,36 @@ def build_unit(K: np.ndarray, V: np.ndarray, seg_len: int, cluster_size: int, it
                      labels=labels, centroids_exact=C, value_sums_exact=vsum)
 
 
+def build_blocks_unit(K: np.ndarray, V: np.ndarray, seg_len: int, block_size: int,
+                      store: str) -> UnitIndex:
+    """Index of position-contiguous blocks for one (sequence, KV head): inside
+    each segment, block j holds positions j*block_size .. (j+1)*block_size - 1
+    (the last one may be shorter); its summary is the block's mean key (the
+    block centroid of [VX] 2.A forward_cache), its value sum the sum of its
+    values.  Blocks keep position order, so perm is the identity."""
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    T, d = K.shape
+    labels = np.empty(T, dtype=np.int64)
+    base = 0
+    for start, n in segment_spans(T, seg_len):
+        labels[start:start + n] = base + np.arange(n) // block_size
+        base += clusters_in_segment(n, block_size)
+    NC = base
+    counts = np.bincount(labels, minlength=NC)
+    offsets = np.zeros(NC + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    ksum = np.zeros((NC, d))
+    vsum = np.zeros((NC, d))
+    np.add.at(ksum, labels, K)
+    np.add.at(vsum, labels, V)
+    C = ksum / np.maximum(counts, 1)[:, None]
+    perm = np.arange(T, dtype=np.int64)
+    return UnitIndex(centroids=round_stored(C, store), value_sums=round_stored(vsum, store),
+                     offsets=offsets, perm=perm, invperm=perm.copy(), k_perm=K.copy(),
+                     v_perm=V.copy(), labels=labels, centroids_exact=C, value_sums_exact=vsum)
+
+
 def extend_unit(old: UnitIndex, K: np.ndarray, V: np.ndarray, seg_len: int, cluster_size: int,
                 iters: int, store: str) -> UnitIndex:
     """Grow the index `old` of a sequence's first T_old tokens to the longer
@@ -329,7 +359,7 @@ class DecodeTrace:
 
 
 def decode_unit(q: np.ndarray, ix: UnitIndex, n_sink: int, window: int, k: int,
-                selected: Optional[np.ndarray] = None) -> DecodeTrace:
+                selected: Optional[np.ndarray] = None, estimate: bool = True) -> DecodeTrace:
     """One decode step of one KV head's query group ([VX] 2.A forward_indexer).
 
     q: [G][d] query heads of the group (values as fed to the kernel).
@@ -342,6 +372,10 @@ def decode_unit(q: np.ndarray, ix: UnitIndex, n_sink: int, window: int, k: int,
         centroid score, times its mean value);
     (e) the two parts are combined by log-sum-exp.
     `selected` overrides step (b) (used to compare downstream steps on a given set).
+    estimate=False leaves step (d) out: attention over the retrieved blocks and
+    the steady zone only, the block top-k workload ([VX] 2.A: forward_cache
+    builds block centroids, forward_indexer selects the top-k blocks and
+    attends; [VX] results: "block top-k").
     """
     q = np.asarray(q, dtype=np.float64)
     G, d = q.shape
@@ -382,12 +416,12 @@ def decode_unit(q: np.ndarray, ix: UnitIndex, n_sink: int, window: int, k: int,
     exact = zone_stats(s_ex, np.ones(len(ex)), ix.v_perm[ex])
 
     # estimation part: candidates not selected
-    X = np.nonzero(candidate & ~is_sel)[0]
-    estimate = zone_stats(s[:, X], cnt_p[X].astype(np.float64), vsum_p[X])
+    X = np.nonzero(candidate & ~is_sel)[0] if estimate else np.zeros(0, dtype=np.int64)
+    est = zone_stats(s[:, X], cnt_p[X].astype(np.float64), vsum_p[X])
 
-    out, lse = lse_merge([exact, estimate])
+    out, lse = lse_merge([exact, est])
     return DecodeTrace(out=out, lse=lse, selected=sel, scores=s, sel_score=a,
-                       candidate=candidate, k=k, exact=exact, estimate=estimate)
+                       candidate=candidate, k=k, exact=exact, estimate=est)
 
 
 def dense_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray):

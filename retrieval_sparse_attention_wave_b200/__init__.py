@@ -42,7 +42,8 @@ WI_MAX_STEADY = 8192
 WI_DEV_BAD_PAGE, WI_DEV_BAD_SLOT, WI_DEV_BAD_CLUSTER, WI_DEV_BAD_HIST = 0x1, 0x2, 0x4, 0x8
 
 EXPORTED = [
-    "wi_index_clusters", "wi_build_workspace_size", "wi_build_index", "wi_extend_index",
+    "wi_index_clusters", "wi_build_workspace_size", "wi_build_index", "wi_build_blocks",
+    "wi_extend_index",
     "wi_kmeans_assign",
     "wi_decode_workspace_size", "wi_decode_workspace_layout", "wi_decode", "wi_decode_host",
     "wi_decode_stage_count", "wi_decode_stage_name", "wi_read_device_status",
@@ -71,7 +72,7 @@ class WiIndex(C.Structure):
 class WiDecodeParams(C.Structure):
     _fields_ = [("n_q_heads", C.c_int32), ("n_sink", C.c_int32), ("window", C.c_int32),
                 ("topk_clusters", C.c_int32), ("topk_fraction", C.c_double),
-                ("stage_events", C.POINTER(C.c_void_p))]
+                ("stage_events", C.POINTER(C.c_void_p)), ("exact_only", C.c_int32)]
 
 
 class WiDecodeLayout(C.Structure):
@@ -89,6 +90,8 @@ _sig = {
                                           C.POINTER(C.c_size_t)]),
     "wi_build_index": (C.c_int, [C.POINTER(WiKVCache), C.c_int32, C.c_int32, C.c_int32,
                                  C.POINTER(WiIndex), _P, C.c_size_t, _P]),
+    "wi_build_blocks": (C.c_int, [C.POINTER(WiKVCache), C.c_int32, C.c_int32,
+                                  C.POINTER(WiIndex), _P, C.c_size_t, _P]),
     "wi_extend_index": (C.c_int, [C.POINTER(WiIndex), C.POINTER(WiKVCache), C.c_int32,
                                   C.POINTER(WiIndex), _P, C.c_size_t, _P]),
     "wi_kmeans_assign": (C.c_int, [C.POINTER(WiKVCache), C.c_int32, C.c_int32, _P, _P, _P,
@@ -328,6 +331,25 @@ def build_index(kv: KVCache, seg_len: int, cluster_size: int, iters: int,
     return out
 
 
+def build_blocks(kv: KVCache, seg_len: int, block_size: int, out: Optional[WaveIndex] = None,
+                 ws: Optional[torch.Tensor] = None, block_table: Optional[torch.Tensor] = None,
+                 n_pages: Optional[int] = None, stream=None) -> WaveIndex:
+    """Index of position-contiguous blocks of block_size tokens (block
+    centroids and value sums; perm is the identity), laid out like a k-means
+    index with cluster_size = block_size."""
+    if out is None:
+        out = WaveIndex(kv.seq_lens, kv.n_kv_heads, kv.head_dim, kv.k_pool.dtype, kv.page_size,
+                        seg_len, block_size, kv.k_pool.device, block_table, n_pages)
+    need = build_workspace_bytes(kv, seg_len, block_size)
+    if ws is None:
+        ws = workspace(need, kv.k_pool.device)
+    s, o = kv.c_struct(), out.c_struct()
+    _check(_lib.wi_build_blocks(C.byref(s), seg_len, block_size, C.byref(o), _ptr(ws), ws.numel(),
+                                _stream_ptr(stream)), "wi_build_blocks")
+    out._build_ws = ws
+    return out
+
+
 def extend_index(old: WaveIndex, kv: KVCache, iters: int, ws: Optional[torch.Tensor] = None,
                  stream=None) -> WaveIndex:
     """The index of the longer sequences in `kv`, grown from `old` segment by
@@ -374,11 +396,13 @@ class DecodeParams:
     window: int = 64
     topk_clusters: int = -1
     topk_fraction: float = 0.018
+    exact_only: bool = False     # no estimation zone (block top-k workload)
 
     def c_struct(self, events=None) -> WiDecodeParams:
         p = WiDecodeParams()
         p.n_q_heads, p.n_sink, p.window = self.n_q_heads, self.n_sink, self.window
         p.topk_clusters, p.topk_fraction = self.topk_clusters, self.topk_fraction
+        p.exact_only = 1 if self.exact_only else 0
         if events is not None:
             for e in events:
                 if not e.cuda_event:      # torch creates the CUDA event on first record

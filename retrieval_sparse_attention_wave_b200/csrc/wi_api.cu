@@ -108,6 +108,7 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   pl.U = ix->batch * ix->n_kv_heads;
   pl.n_sink = p->n_sink; pl.window = p->window;
   pl.topk_clusters = p->topk_clusters; pl.topk_fraction = p->topk_fraction;
+  pl.exact_only = p->exact_only != 0;
   pl.scale = 1.0f / std::sqrt((float)ix->head_dim);
 
   int max_nc = 0, cap = 1;
@@ -372,6 +373,19 @@ wi_status wi_build_index(const wi_kv_cache* kv, int32_t seg_len, int32_t cluster
   if ((st = check_ws(ws, ws_bytes, pl.total)) != WI_OK) return st;
   const BuildArgs a = build_args(kv, out, ws);
   const cudaError_t e = launch_build(pl, a, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WI_OK : cuda_fail(e);
+}
+
+wi_status wi_build_blocks(const wi_kv_cache* kv, int32_t seg_len, int32_t block_size,
+                          const wi_index* out, void* ws, size_t ws_bytes, wi_stream_t stream) {
+  BuildPlan pl;
+  wi_status st = make_build_plan(kv, seg_len, block_size, pl);
+  if (st != WI_OK) return st;
+  if ((st = check_build_out(kv, seg_len, block_size, out)) != WI_OK) return st;
+  pl.iters = 1;
+  if ((st = check_ws(ws, ws_bytes, pl.total)) != WI_OK) return st;
+  const BuildArgs a = build_args(kv, out, ws);
+  const cudaError_t e = launch_blocks(pl, a, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? WI_OK : cuda_fail(e);
 }
 

@@ -312,6 +312,18 @@ kmeans_update_kernel(const Geo geo, const Pool kin, int S, int cs, const SegFrom
   if (fo.enabled && tid == 0 && start + len == T_) fo.offsets[geo.off_row(b, h) + geo.NC(b)] = T_;
 }
 
+// ------------------------------------------------------- position blocks
+// The block index's assignment: token t of a segment belongs to block
+// t / block_size of that segment (cs plays the block size).
+__global__ void __launch_bounds__(kStreamThreads)
+block_assign_kernel(const Geo geo, int S, int cs, int32_t* __restrict__ assign) {
+  const int u = blockIdx.y, b = u / geo.hkv, h = u - b * geo.hkv;
+  const int T_ = geo.T(b);
+  const int64_t trow = geo.tok_row(b, h);
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T_; t += gridDim.x * blockDim.x)
+    assign[trow + t] = (t % S) / cs;
+}
+
 // ----------------------------------------------------------- extension copy
 // Unit blockIdx.y: the first s0 * S / cs clusters (centroid and value-sum
 // rows, their offsets and the offset after them) and the first s0 * S tokens
@@ -412,6 +424,32 @@ cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s)
       kmeans_update_kernel<T, D><<<dim3(p.nseg_grid, p.U), kUpdThreads, p.update_smem, s>>>(
           p.geo, a.kin, p.S, p.cs, p.sf, cent32, assign, it == p.iters - 1 ? fin : none, status);
     }
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t launch_blocks(const BuildPlan& p, const BuildArgs& a, cudaStream_t s) {
+  uint32_t* status = reinterpret_cast<uint32_t*>(a.ws + p.off_status);
+  float* cent32 = reinterpret_cast<float*>(a.ws + p.off_cent32);
+  int32_t* assign = reinterpret_cast<int32_t*>(a.ws + p.off_assign);
+  return with_build_types(p.dtype, p.D, [&]<typename T, int D>() -> cudaError_t {
+    cudaFuncSetAttribute(kmeans_update_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)p.update_smem);
+    block_assign_kernel<<<dim3(64, p.U), kStreamThreads, 0, s>>>(p.geo, p.S, p.cs, assign);
+    FinalOut fin{};
+    fin.centroids = a.centroids;
+    fin.value_sums = a.value_sums;
+    fin.offsets = a.offsets;
+    fin.perm = a.perm;
+    fin.invperm = a.invperm;
+    fin.labels = a.labels;
+    fin.kout = a.kout;
+    fin.vout = a.vout;
+    fin.pout = Pool{a.kout, a.bt_out, a.n_pages_out, a.max_pages_out, a.page_shift_out};
+    fin.vin = a.vin;
+    fin.enabled = 1;
+    kmeans_update_kernel<T, D><<<dim3(p.nseg_grid, p.U), kUpdThreads, p.update_smem, s>>>(
+        p.geo, a.kin, p.S, p.cs, p.sf, cent32, assign, fin, status);
     return cudaGetLastError();
   });
 }

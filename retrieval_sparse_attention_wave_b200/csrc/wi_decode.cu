@@ -1153,6 +1153,7 @@ struct AttendArgs {
   float* out;
   float* lse;
   float scale;
+  int exact_only;            // no estimation zone: retrieved clusters and steady zone only
 };
 
 template <typename T, int D, int G>
@@ -1243,7 +1244,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
       qa0[ks] = gm < G ? qw[8 * ks + tq] : 0u;
       qa2[ks] = gm < G ? qw[8 * ks + 4 + tq] : 0u;
     }
-    if (role_range) {
+    if (role_range && !A.exact_only) {
       // the range's 256 value-sum rows (index data, independent of the
       // previous kernels): four 64-row tiles, each two 64-column boxes, fill
       // the ring (rows past the last cluster row are zero-filled)
@@ -1258,6 +1259,12 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
           tensor_load_2d(sh + t * 16384 + 8192, &tm_vsum, 64, y0 + 64 * t, &s_vbar);
         }
       }
+    } else {
+      // rows no copy writes keep finite contents (zero weight times a finite row)
+      for (int i = tid; i < 4 * 16384 / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(sh)[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (role_range) {
       const int c0 = (int)blockIdx.x * kRangeW;
       if (c0 + tid < NC) {
         r_o0 = __ldg(off + c0 + tid);
@@ -1271,10 +1278,6 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
           if (r_lp0 + i < kp.max_pages) cp_async4(&s_bt[i], kp.bt + (int64_t)b * kp.max_pages + r_lp0 + i);
         cp_async_commit();
       }
-    } else {
-      // rows no copy writes keep finite contents (zero weight times a finite row)
-      for (int i = tid; i < 4 * 16384 / 16; i += blockDim.x)
-        reinterpret_cast<uint4*>(sh)[i] = make_uint4(0u, 0u, 0u, 0u);
     }
     // the A operands' rows that no head writes stay zero
     for (int i = tid; i < (int)(sizeof(s_P) / 16); i += blockDim.x)
@@ -1611,7 +1614,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     __syncthreads();
     if (af != 0) *afp = 0;  // consumed: clean for the next call
     const bool dense = s_info[6] != 0;
-    const bool est = !dense && s_info[0] < s_info[7] && NC > 0;
+    const bool est = !A.exact_only && !dense && s_info[0] < s_info[7] && NC > 0;
     const uint32_t kstar = (uint32_t)s_info[1];
     const int thr = s_info[2];
     const int cnt = o1 - o0;
@@ -1710,7 +1713,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     };
     auto estimate = [&](int np_) -> int {
       float oe[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      mbar_wait(&s_vbar, 0, status);
+      if (!A.exact_only) mbar_wait(&s_vbar, 0, status);   // (no copies without a zone)
       if (me0 != -INFINITY) est_steps(oe, kRangeW / 32, kRangeW / 16);
       __syncthreads();              // slots 2, 3 are read
       issue_kv(0, np_);
@@ -1811,7 +1814,7 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
     __syncthreads();
     if (af != 0) *afp = 0;  // consumed: clean for the next call
     const bool dense = s_info[6] != 0;
-    const bool est = !dense && s_info[0] < s_info[7] && NC > 0;
+    const bool est = !A.exact_only && !dense && s_info[0] < s_info[7] && NC > 0;
     const uint32_t kstar = (uint32_t)s_info[1];
     const int thr = s_info[2];
     const int cnt = o1 - o0;
@@ -1983,7 +1986,8 @@ wave_attend_kernel(const Geo geo, const T* __restrict__ q, int n_q_heads, const 
   // nothing estimated (dense, or every candidate retrieved) merges the
   // first two groups alone
   const int32_t* I = A.info + (int64_t)u * kInfoInts;
-  const int np = A.n_fold == 0 || (!I[6] && I[0] < I[7] && NC > 0) ? A.n_parts : A.n_rng + A.n_sc;
+  const int np = A.n_fold == 0 || (!A.exact_only && !I[6] && I[0] < I[7] && NC > 0)
+                     ? A.n_parts : A.n_rng + A.n_sc;
   // the parts stream through the ring and the correction rows (contiguous)
   // in batches: one cp.async round per batch, the first batch issued
   // together with the loads of every part's (m, l)
@@ -2272,7 +2276,7 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
     mark(2);
     AttendArgs A{keys, scores, info, aff_of, p.max_nc, aff_start, st_slot, dv, p.cap, a.perm,
                  p.n_sink, p.window, sel, p.sel_words, est_parts, p.n_score_blocks, p.n_rng, p.n_sc,
-                 p.n_fold, p.n_parts, partials, counters, a.out, a.lse, p.scale};
+                 p.n_fold, p.n_parts, partials, counters, a.out, a.lse, p.scale, p.exact_only};
     const size_t smem = decode_attend_smem(p.dtype, D, G, p.n_parts);
     set_smem(wave_attend_kernel<T, D, G>, smem);
     e = launch_ex(wave_attend_kernel<T, D, G>, dim3(p.n_rng + p.n_sc + p.n_fold, p.U), dim3(kStreamThreads),

@@ -19,6 +19,7 @@ constexpr int kFold = 16;             // score-chunk parts folded into one by an
 constexpr int kRangeClusters = 256;   // cluster ids per attend range CTA (one per thread)
 
 struct DecodePlan {
+  int exact_only;          // no estimation zone (block top-k workload)
   Geo geo;
   int dtype, D, G, Hq, U;
   int n_sink, window, topk_clusters;
@@ -105,6 +106,9 @@ size_t decode_attend_smem(int dtype, int D, int G, int n_parts);
 size_t decode_score_smem(int dtype, int D, int G, int sort_pow2, int cap);
 size_t decode_topk_smem(int max_nc, int cap);
 cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s);
+// Position-block index: each token's cluster is its block inside its segment,
+// then one finalizing update pass.
+cudaError_t launch_blocks(const BuildPlan& p, const BuildArgs& a, cudaStream_t s);
 // Copy the part of an old index that an extension keeps (segments below
 // p.sf.s0[b]) into the new index's buffers: centroid and value-sum rows,
 // offsets, perm, invperm and labels.

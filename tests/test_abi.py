@@ -189,6 +189,21 @@ def test_build_validation():
         == W.WI_ERR_INVALID_ARG
 
 
+def test_build_blocks_validation():
+    lib = W.lib()
+    kv = kv_struct()
+    n = C.c_size_t()
+    assert lib.wi_build_workspace_size(C.byref(kv), 1024, 16, C.byref(n)) == W.WI_OK
+    out = index_struct()                       # cluster_size 16
+    assert lib.wi_build_blocks(C.byref(kv), 1024, 32, C.byref(out), FAKE, n.value, None) \
+        == W.WI_ERR_INVALID_ARG                # block size other than the index's
+    alias = index_struct(k_pool=kv.k_pool)
+    assert lib.wi_build_blocks(C.byref(kv), 1024, 16, C.byref(alias), FAKE, n.value, None) \
+        == W.WI_ERR_INVALID_ARG
+    assert lib.wi_build_blocks(C.byref(kv), 1024, 16, C.byref(out), FAKE, 1024, None) \
+        == W.WI_ERR_WORKSPACE
+
+
 def test_extend_validation():
     """wi_extend_index checks every argument before any launch."""
     lib = W.lib()

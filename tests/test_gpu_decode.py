@@ -47,7 +47,8 @@ def check_decode(wl, units, params, *, shuffle_seed=None, page_size=None, ref_de
         NC = len(ix.centroids)
         k = O.k_for(NC, params.topk_clusters, params.topk_fraction)
         qg = qh[b, h * G:(h + 1) * G]
-        tr = O.decode_unit(qg, ix, params.n_sink, params.window, k)
+        est = not params.exact_only
+        tr = O.decode_unit(qg, ix, params.n_sink, params.window, k, estimate=est)
         # (a1) scores
         sc = W.centroid_scores(ws, lay, wx, G, b, h).cpu().numpy().astype(np.float64)
         if not info[u, 6]:
@@ -64,7 +65,8 @@ def check_decode(wl, units, params, *, shuffle_seed=None, page_size=None, ref_de
             kth = np.sort(tr.sel_score[tr.selected])[0]
             assert np.all(np.abs(tr.sel_score[diff] - kth) <= 1e-5 * abs(kth)), \
                 f"unit {(b, h)}: sets differ beyond near-ties"
-            tr = O.decode_unit(qg, ix, params.n_sink, params.window, k, selected=gsel)
+            tr = O.decode_unit(qg, ix, params.n_sink, params.window, k, selected=gsel,
+                               estimate=est)
         # the retrieved clusters' tokens, counted once each
         if info[u, 6]:
             assert int(info[u, 3]) == 0

@@ -176,6 +176,70 @@ def test_extension_equals_build_of_the_longer_sequence(T_old, T_new):
         np.testing.assert_allclose(ext.value_sums_exact, ref.value_sums_exact, atol=1e-12)
 
 
+def test_block_index_is_positional():
+    """Block top-k index ([VX] 2.A block centroids): block j of a segment is
+    positions j*B .. (j+1)*B-1, its summary the mean key; perm is the identity."""
+    rng = np.random.default_rng(12)
+    K, V, _ = mixture(rng, 1300, 8, n_centers=12)
+    ix = O.build_blocks_unit(K, V, seg_len=512, block_size=16, store="f32")
+    assert np.array_equal(ix.perm, np.arange(1300)) and np.array_equal(ix.invperm, ix.perm)
+    spans = O.segment_spans(1300, 512)
+    assert len(ix.centroids) == sum(O.clusters_in_segment(n, 16) for _, n in spans)
+    c = 0
+    for start, n in spans:
+        for j in range(0, n, 16):
+            lo, hi = start + j, start + min(j + 16, n)
+            assert ix.offsets[c] == lo and ix.offsets[c + 1] == hi
+            assert np.all(ix.labels[lo:hi] == c)
+            np.testing.assert_allclose(ix.centroids[c], K[lo:hi].mean(0), atol=1e-13)
+            np.testing.assert_allclose(ix.value_sums[c], V[lo:hi].sum(0), atol=1e-12)
+            c += 1
+
+
+@pytest.mark.parametrize("n_sink,window", [(4, 64), (0, 0)])
+def test_exact_only_with_every_block_is_dense(n_sink, window):
+    """Without the estimation zone, retrieving every block is full attention."""
+    rng = np.random.default_rng(13)
+    K, V, C = mixture(rng, 900, 16, n_centers=10)
+    q = C[:4] + 0.3 * rng.standard_normal((4, 16))
+    ix = O.build_blocks_unit(K, V, seg_len=256, block_size=16, store="f32")
+    tr = O.decode_unit(q, ix, n_sink, window, k=10 ** 6, estimate=False)
+    out, lse = O.dense_attention(q, K, V)
+    np.testing.assert_allclose(tr.out, out, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(tr.lse, lse, rtol=1e-12, atol=1e-12)
+
+
+def test_exact_only_with_no_block_is_steady_attention():
+    """k = 0 and no estimation leaves attention over the sink and window
+    tokens alone."""
+    rng = np.random.default_rng(14)
+    K, V, C = mixture(rng, 700, 16, n_centers=10)
+    q = C[:2] + 0.3 * rng.standard_normal((2, 16))
+    ix = O.build_blocks_unit(K, V, seg_len=256, block_size=16, store="f32")
+    tr = O.decode_unit(q, ix, 4, 32, k=0, estimate=False)
+    st = np.r_[0:4, 700 - 32:700]
+    out, lse = O.dense_attention(q, K[st], V[st])
+    np.testing.assert_allclose(tr.out, out, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(tr.lse, lse, rtol=1e-12, atol=1e-12)
+
+
+def test_exact_only_brute_force():
+    """Exact-only decode equals softmax over the retrieved blocks' tokens
+    (minus steady ones, counted once) plus the steady tokens, by brute force."""
+    rng = np.random.default_rng(15)
+    K, V, C = mixture(rng, 300, 8, n_centers=6)
+    q = C[:2] + 0.3 * rng.standard_normal((2, 8))
+    ix = O.build_blocks_unit(K, V, seg_len=128, block_size=8, store="f32")
+    tr = O.decode_unit(q, ix, 2, 16, k=5, estimate=False)
+    keep = set(range(2)) | set(range(300 - 16, 300))
+    for c in tr.selected:
+        keep |= set(range(ix.offsets[c], ix.offsets[c + 1]))
+    keep = np.array(sorted(keep))
+    out, lse = O.dense_attention(q, K[keep], V[keep])
+    np.testing.assert_allclose(tr.out, out, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(tr.lse, lse, rtol=1e-12, atol=1e-12)
+
+
 # --------------------------------------------------------------- decode pins
 
 def test_steady_positions():

@@ -31,6 +31,15 @@ MUTATIONS = {
     "estimate ignores counts": ("cnt_p[X].astype(np.float64)", "np.ones(len(X))"),
     "bf16 truncation": ("np.rint(x[nz] / quantum)", "np.trunc(x[nz] / quantum)"),
     "value sum not mean": ("C[nz] = sums[nz] / counts[nz, None]", "C[nz] = sums[nz]"),
+    "extension offsets not rebased": ("offsets[nc0 + 1:] = s0 + np.cumsum(counts)",
+                                      "offsets[nc0 + 1:] = np.cumsum(counts)"),
+    "extension keeps a partial segment": (
+        "s0 = (T_old // seg_len) * seg_len                       # first position clustered anew",
+        "s0 = -(-T_old // seg_len) * seg_len"),
+    "block summary is the key sum": ("C = ksum / np.maximum(counts, 1)[:, None]", "C = ksum"),
+    "exact-only keeps the estimate": (
+        "X = np.nonzero(candidate & ~is_sel)[0] if estimate else np.zeros(0, dtype=np.int64)",
+        "X = np.nonzero(candidate & ~is_sel)[0]"),
 }
 
 PINS = [
@@ -46,6 +55,10 @@ PINS = [
     lambda: pins.test_brute_force_tiny(64, 4, 3, 2, 5),
     lambda: pins.test_pure_estimate_golden_two_clusters(),
     lambda: pins.test_group_selection_uses_max_over_heads(),
+    lambda: pins.test_extension_equals_build_of_the_longer_sequence(1500, 2900),
+    lambda: pins.test_block_index_is_positional(),
+    lambda: pins.test_exact_only_with_no_block_is_steady_attention(),
+    lambda: pins.test_exact_only_brute_force(),
 ]
 
 

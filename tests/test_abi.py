@@ -103,6 +103,33 @@ def test_decode_workspace_size_and_layout():
     assert lay.sel_words >= 8 and lay.sel_words % 8 == 0
 
 
+@pytest.mark.parametrize("dtype,d,seq,expect", [
+    # 131072 tokens: 8192 clusters -> 32 range CTAs + 1 steady CTA, 256 bitmap
+    # words; bf16 d = 128 (tensor cores) estimates in the range CTAs: no folds
+    (W.WI_BF16, 128, [131072], dict(n_attend_ctas=33, sel_words=256, n_score_ctas=64)),
+    # fp32: 64 clusters per 32 KB chunk; 32-row tiles, so the 68 steady slots
+    # take two steady CTAs
+    (W.WI_F32, 128, [131072], dict(n_attend_ctas=34, sel_words=256, n_score_ctas=128)),
+    # ragged batch, sized by the longest sequence: 256 clusters -> one range
+    # CTA, one steady CTA, 8 bitmap words, two 128-cluster score chunks
+    (W.WI_BF16, 128, [4096, 300], dict(n_attend_ctas=2, sel_words=8, n_score_ctas=2)),
+])
+def test_decode_plan_shapes(dtype, d, seq, expect):
+    """The launch plan's per-unit CTA counts and bitmap size, from the
+    geometry alone (host logic)."""
+    lay = W.WiDecodeLayout()
+    ix = index_struct(seq=seq, dtype=dtype, head_dim=d, n_pages=16384, max_pages=16384)
+    assert W.lib().wi_decode_workspace_layout(C.byref(ix), C.byref(params()), C.byref(lay)) \
+        == W.WI_OK
+    for k, v in expect.items():
+        assert getattr(lay, k) == v, (k, getattr(lay, k), v)
+    # the exact-only flag changes nothing in the layout
+    lay2 = W.WiDecodeLayout()
+    assert W.lib().wi_decode_workspace_layout(C.byref(ix), C.byref(params(exact_only=1)),
+                                              C.byref(lay2)) == W.WI_OK
+    assert lay2.total_bytes == lay.total_bytes
+
+
 @pytest.mark.parametrize("over,expect", [
     (dict(n_q_heads=0), W.WI_ERR_INVALID_ARG),
     (dict(n_q_heads=31), W.WI_ERR_INVALID_ARG),       # not a multiple of Hkv

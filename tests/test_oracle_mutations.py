@@ -37,6 +37,9 @@ MUTATIONS = {
         "s0 = (T_old // seg_len) * seg_len                       # first position clustered anew",
         "s0 = -(-T_old // seg_len) * seg_len"),
     "block summary is the key sum": ("C = ksum / np.maximum(counts, 1)[:, None]", "C = ksum"),
+    "stochastic draws ignore the seed": ("splitmix64(((seed & 0xFFFFFFFF) << 32) | int(c))",
+                                         "splitmix64(int(c))"),
+    "splitmix64 without its last xor-shift": ("    return z ^ (z >> 31)", "    return z"),
     "exact-only keeps the estimate": (
         "X = np.nonzero(candidate & ~is_sel)[0] if estimate else np.zeros(0, dtype=np.int64)",
         "X = np.nonzero(candidate & ~is_sel)[0]"),
@@ -59,6 +62,8 @@ PINS = [
     lambda: pins.test_block_index_is_positional(),
     lambda: pins.test_exact_only_with_no_block_is_steady_attention(),
     lambda: pins.test_exact_only_brute_force(),
+    lambda: pins.test_splitmix64_published_outputs(),
+    lambda: pins.test_stochastic_topk_samples_the_threshold_bin_uniformly(),
 ]
 
 

@@ -240,6 +240,103 @@ def test_exact_only_brute_force():
     np.testing.assert_allclose(tr.lse, lse, rtol=1e-12, atol=1e-12)
 
 
+# ------------------------------------------------ stochastic radix top-k pins
+
+def test_splitmix64_published_outputs():
+    """The first three SplitMix64 outputs from state 0 (the generator's
+    published known answers: Steele, Lea and Flood 2014, and the reference
+    splitmix64.c seeded with 0); the state advances by the golden-ratio
+    increment between outputs."""
+    gamma = 0x9E3779B97F4A7C15
+    got = [O.splitmix64((i * gamma) & ((1 << 64) - 1)) for i in range(3)]
+    assert got == [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F]
+
+
+def test_ordered_key_preserves_float_order():
+    rng = np.random.default_rng(21)
+    x = np.concatenate([rng.standard_normal(500) * 10.0 ** rng.integers(-30, 30, 500),
+                        [-np.inf, np.inf, -0.0, 0.0, 1e-45, -1e-45]]).astype(np.float32)
+    keys = O.ordered_key32(x)
+    xs = x.astype(np.float64)
+    for i in range(0, len(x), 7):
+        for j in range(0, len(x), 11):
+            if xs[i] < xs[j]:
+                assert keys[i] < keys[j]
+            elif xs[i] > xs[j]:
+                assert keys[i] > keys[j]
+
+
+def stochastic_case(seed, n=400):
+    rng = np.random.default_rng(seed)
+    a = np.round(rng.standard_normal(n), 2)          # duplicates and shared bins
+    cand = rng.random(n) > 0.1
+    return a, cand
+
+
+@pytest.mark.parametrize("k", [0, 1, 17, 100, 359, 10 ** 6])
+def test_stochastic_topk_invariants(k):
+    """k picks (clamped), all candidates; every candidate of a bin above the
+    threshold bin is taken, none below it; the rest come from the bin."""
+    a, cand = stochastic_case(3)
+    sel = O.select_topk_stochastic(a, cand, k, seed=5)
+    n_c = int(cand.sum())
+    assert len(sel) == min(k, n_c) and len(set(sel.tolist())) == len(sel)
+    assert np.all(cand[sel]) and np.all(np.diff(sel) > 0)
+    if 0 < k < n_c:
+        bins = O.ordered_key32(a.astype(np.float32)) >> 21
+        b_star = np.sort(bins[cand])[::-1][k - 1]
+        chosen = np.zeros(len(a), dtype=bool)
+        chosen[sel] = True
+        assert np.all(chosen[cand & (bins > b_star)])
+        assert not np.any(chosen[cand & (bins < b_star)])
+
+
+def test_stochastic_topk_is_exact_when_bins_decide():
+    """Scores whose bins are all distinct leave nothing to sample: the
+    selection is the exact top-k, whatever the seed."""
+    a = 2.0 ** np.arange(-40, 40, 0.5)[::-1]
+    rng = np.random.default_rng(4)
+    rng.shuffle(a)
+    cand = np.ones(len(a), dtype=bool)
+    for k in (1, 5, 33, 100):
+        exact = O.select_topk(a, cand, k)
+        for seed in (0, 1, 99):
+            sel = O.select_topk_stochastic(a, cand, k, seed)
+            assert np.array_equal(sel, exact)
+            assert O.recall(sel, exact) == 1.0
+
+
+def test_stochastic_topk_samples_the_threshold_bin_uniformly():
+    """Ten clear winners and twenty members of one bin: with k = 15 five of
+    the twenty are drawn; over 4000 seeds each is drawn with frequency 1/4
+    (binomial, five sigma), and a fixed seed repeats its draw."""
+    a = np.concatenate([np.arange(10, 20, dtype=np.float64), np.full(20, 1.0)])
+    cand = np.ones(30, dtype=bool)
+    counts = np.zeros(30)
+    for seed in range(4000):
+        sel = O.select_topk_stochastic(a, cand, 15, seed)
+        assert set(range(10)) <= set(sel.tolist())
+        counts[sel] += 1
+    f = counts[10:] / 4000
+    assert np.all(np.abs(f - 0.25) <= 5 * np.sqrt(0.25 * 0.75 / 4000))
+    assert np.array_equal(O.select_topk_stochastic(a, cand, 15, 77),
+                          O.select_topk_stochastic(a, cand, 15, 77))
+
+
+def test_recall_bounds():
+    a, cand = stochastic_case(6)
+    for k in (0, 10, 60):
+        exact = O.select_topk(a, cand, k)
+        sel = O.select_topk_stochastic(a, cand, k, seed=3)
+        r = O.recall(sel, exact)
+        assert 0.0 <= r <= 1.0 and O.recall(exact, exact) == 1.0
+        if k:
+            bins = O.ordered_key32(a.astype(np.float32)) >> 21
+            b_star = np.sort(bins[cand])[::-1][k - 1]
+            m = int((cand & (bins == b_star)).sum())
+            assert r >= (k - m) / k          # only the threshold bin is sampled
+
+
 # --------------------------------------------------------------- decode pins
 
 def test_steady_positions():

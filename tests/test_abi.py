@@ -263,3 +263,28 @@ def test_status_strings():
     for s in range(6):
         assert lib.wi_status_string(s)
     assert lib.wi_read_device_status(None, None, None, 0) == W.WI_ERR_INVALID_ARG
+
+
+def test_selection_bitmap_decoding_on_the_host():
+    """The binding reads the selection bitmap (bit c % 32 of word c / 32 of
+    the unit's words) back into ascending cluster ids."""
+    import types
+
+    import numpy as np
+    import torch
+    lay = types.SimpleNamespace(selected=256, sel_words=16)
+    index = types.SimpleNamespace(n_kv_heads=2)
+    ws = torch.zeros(256 + 4 * 16 * 4, dtype=torch.uint8)
+    words = ws[256:].view(torch.int32)
+    want = {(0, 1): [0, 31, 32, 200, 511], (1, 0): [5, 63, 64, 65]}
+    for (b, h), ids in want.items():
+        u = b * 2 + h
+        for c in ids:
+            w = u * 16 + c // 32
+            words[w] = int(np.int32(np.uint32(int(words[w]) & 0xFFFFFFFF | (1 << (c % 32)))))
+    for (b, h), ids in want.items():
+        got = W.selected_clusters(ws, lay, index, b, h, len(ids))
+        assert got.tolist() == ids
+    assert W.selected_clusters(ws, lay, index, 0, 0, 0).tolist() == []
+    with pytest.raises(RuntimeError):
+        W.selected_clusters(ws, lay, index, 0, 1, 4)

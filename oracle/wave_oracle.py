@@ -35,6 +35,14 @@ Readings where the pages are silent (each is listed in the design doc):
   R-7 centroids and value sums are stored in the KV dtype (round to nearest
       even from the exact mean / sum); decode reads the stored values.
   R-8 softmax scale 1/sqrt(d); no causal mask at decode.
+  R-14 an index grows segment by segment: the whole segments of the old index
+      are kept, a partial last one is clustered again with its new tokens.
+  R-15 a block of the block top-k workload is block_size consecutive
+      positions inside a segment; its summary is the mean key; blocks are
+      scored and selected like clusters; the workload has no estimation zone.
+  R-16 the stochastic top-k ranks by the top 11 bits of the fp32 score's
+      order-preserving key and samples the threshold bin without replacement
+      by a SplitMix64 draw per cluster id.
 
 Parity pins for every function here live in tests/test_oracle_pins.py.
 """

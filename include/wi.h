@@ -176,6 +176,23 @@ wi_status wi_index_clusters(int32_t batch, const int32_t *seq_lens, int32_t seg_
 wi_status wi_build_workspace_size(const wi_kv_cache *kv, int32_t seg_len,
                                   int32_t cluster_size, size_t *bytes);
 
+/* Byte offsets of the build workspace regions (for inspection and tests).
+ * After wi_build_index with `iters` = r, the region at centroids_f32 holds
+ * the fp32 working centroids after round r's update (float [Hkv*sum NC_b][d],
+ * laid out like wi_index.centroids: the correctly rounded means of round r's
+ * assignment, or the previous value for an empty cluster), and the region at
+ * `assign` holds round r's assignment (int32 [Hkv*sum T_b], segment-local
+ * cluster index of each original position, token-indexed like
+ * wi_index.perm).  RetroInfer 2.A, Segmented Clustering.  Host only. */
+typedef struct wi_build_layout {
+  size_t total_bytes;
+  size_t status;          /* uint32 status word (offset 0)                     */
+  size_t centroids_f32;
+  size_t assign;
+} wi_build_layout;
+wi_status wi_build_workspace_layout(const wi_kv_cache *kv, int32_t seg_len,
+                                    int32_t cluster_size, wi_build_layout *layout);
+
 /*
  * Build the wave index (RetroInfer 2.A, Segmented Clustering; Vortex 2.A
  * forward_cache).  For every unit and every segment of seg_len tokens (the
@@ -315,7 +332,10 @@ wi_status wi_decode_host(const void *q_host, const wi_index *idx, const wi_decod
  * first call on a device looks up the array's device address, so make it
  * before any stream capture on that device.  Device-side index checks still
  * skip bad accesses, but their status bits are not readable through this
- * entry point.  q, out, lse: as for wi_decode.
+ * entry point.  The address is cached per CUDA context: after a device reset
+ * the new context looks it up again on its first call.  Argument errors
+ * (null or misaligned q / out / lse, bad index or parameters) are returned
+ * before any CUDA call.  q, out, lse: as for wi_decode.
  */
 #define WI_NOALLOC_SCRATCH_MIB 32
 wi_status wi_decode_noalloc(const void *q, const wi_index *idx, const wi_decode_params *p,

@@ -17,7 +17,7 @@ Sources (page title, section):
         LLMs" (catalog summary): attention sinks and the decoded tail stay
         resident; pages are filled by similarity, not position.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent or leave a step open:
   R-1 k-means distance is squared Euclidean on the raw keys.
   R-2 a segment of n tokens gets ceil(n/cs) centroids, centroid j starts as the
       key at segment position j*cs; `iters` rounds of (assign, update); an

@@ -42,7 +42,8 @@ WI_MAX_STEADY = 8192
 WI_DEV_BAD_PAGE, WI_DEV_BAD_SLOT, WI_DEV_BAD_CLUSTER, WI_DEV_BAD_HIST = 0x1, 0x2, 0x4, 0x8
 
 EXPORTED = [
-    "wi_index_clusters", "wi_build_workspace_size", "wi_build_index", "wi_build_blocks",
+    "wi_index_clusters", "wi_build_workspace_size", "wi_build_workspace_layout",
+    "wi_build_index", "wi_build_blocks",
     "wi_extend_index",
     "wi_kmeans_assign",
     "wi_decode_workspace_size", "wi_decode_workspace_layout", "wi_decode", "wi_decode_host",
@@ -75,6 +76,11 @@ class WiDecodeParams(C.Structure):
                 ("stage_events", C.POINTER(C.c_void_p)), ("exact_only", C.c_int32)]
 
 
+class WiBuildLayout(C.Structure):
+    _fields_ = [("total_bytes", C.c_size_t), ("status", C.c_size_t),
+                ("centroids_f32", C.c_size_t), ("assign", C.c_size_t)]
+
+
 class WiDecodeLayout(C.Structure):
     _fields_ = [("total_bytes", C.c_size_t), ("status", C.c_size_t), ("scores", C.c_size_t),
                 ("keys", C.c_size_t), ("selected", C.c_size_t), ("unit_info", C.c_size_t),
@@ -88,6 +94,8 @@ _sig = {
                                     C.POINTER(C.c_int32), C.POINTER(C.c_int64)]),
     "wi_build_workspace_size": (C.c_int, [C.POINTER(WiKVCache), C.c_int32, C.c_int32,
                                           C.POINTER(C.c_size_t)]),
+    "wi_build_workspace_layout": (C.c_int, [C.POINTER(WiKVCache), C.c_int32, C.c_int32,
+                                            C.POINTER(WiBuildLayout)]),
     "wi_build_index": (C.c_int, [C.POINTER(WiKVCache), C.c_int32, C.c_int32, C.c_int32,
                                  C.POINTER(WiIndex), _P, C.c_size_t, _P]),
     "wi_build_blocks": (C.c_int, [C.POINTER(WiKVCache), C.c_int32, C.c_int32,
@@ -306,6 +314,26 @@ def build_workspace_bytes(kv: KVCache, seg_len: int, cluster_size: int) -> int:
     _check(_lib.wi_build_workspace_size(C.byref(s), seg_len, cluster_size, C.byref(n)),
            "wi_build_workspace_size")
     return n.value
+
+
+def build_layout(kv: KVCache, seg_len: int, cluster_size: int) -> WiBuildLayout:
+    lay = WiBuildLayout()
+    s = kv.c_struct()
+    _check(_lib.wi_build_workspace_layout(C.byref(s), seg_len, cluster_size, C.byref(lay)),
+           "wi_build_workspace_layout")
+    return lay
+
+
+def build_state(kv: KVCache, index: "WaveIndex"):
+    """The fp32 working centroids [Hkv * sum NC_b][d] and the int32 assignment
+    [Hkv * sum T_b] a build left in its workspace (views into it)."""
+    lay = build_layout(kv, index.seg_len, index.cluster_size)
+    ws = index._build_ws
+    ncl = index.n_kv_heads * sum(index.nc)
+    ntok = index.n_kv_heads * sum(index.seq_lens)
+    cent = ws[lay.centroids_f32:lay.centroids_f32 + ncl * index.head_dim * 4].view(torch.float32)
+    asg = ws[lay.assign:lay.assign + ntok * 4].view(torch.int32)
+    return cent.view(ncl, index.head_dim), asg
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:

@@ -361,6 +361,19 @@ wi_status wi_build_workspace_size(const wi_kv_cache* kv, int32_t seg_len, int32_
 }
 
 
+wi_status wi_build_workspace_layout(const wi_kv_cache* kv, int32_t seg_len,
+                                    int32_t cluster_size, wi_build_layout* layout) {
+  if (!layout) return WI_ERR_INVALID_ARG;
+  BuildPlan pl;
+  wi_status st = make_build_plan(kv, seg_len, cluster_size, pl);
+  if (st != WI_OK) return st;
+  layout->total_bytes = pl.total;
+  layout->status = pl.off_status;
+  layout->centroids_f32 = pl.off_cent32;
+  layout->assign = pl.off_assign;
+  return WI_OK;
+}
+
 wi_status wi_build_index(const wi_kv_cache* kv, int32_t seg_len, int32_t cluster_size,
                          int32_t iters, const wi_index* out, void* ws, size_t ws_bytes,
                          wi_stream_t stream) {

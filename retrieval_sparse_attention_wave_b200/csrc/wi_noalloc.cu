@@ -7,6 +7,10 @@
 // memory is owned up front by a fixed arena that hands out no further blocks,
 // and C callers embedded in runtimes that expose no device allocator at all.
 // For them this entry point takes only inputs and outputs.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
 #include <mutex>
 
 #include "wi.h"
@@ -21,33 +25,58 @@ constexpr size_t kScratchBytes = (size_t)WI_NOALLOC_SCRATCH_MIB << 20;
 // loads the library holds it until the process exits.
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
+// Device address of g_scratch per CUDA context.  In host code the name
+// g_scratch is only a host-side stand-in, so the address is looked up once
+// per context with that context current.  Keying by context (not device
+// number) makes a context created after a device reset look the address up
+// again instead of reusing a stale one.
+constexpr int kMaxContexts = 64;
 std::mutex g_mu;
-void* g_ptr[kMaxDevices];  // device address of g_scratch, per device
+CUcontext g_ctx[kMaxContexts];
+void* g_ptr[kMaxContexts];
+int g_n = 0;
 
-// The device address of g_scratch on the current device.  Host code only sees
-// a host-side stand-in under the name g_scratch, so the address is looked up
-// once per device with that device current.
+PFN_cuCtxGetCurrent_v4000 ctx_fn() {
+  static std::once_flag once;
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+  });
+  return fn;
+}
+
 wi_status scratch_ptr(void** out) {
   int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WI_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WI_ERR_CUDA;
+  // make the device's primary context current (a no-op when it already is)
+  if (cudaFree(nullptr) != cudaSuccess) return WI_ERR_CUDA;
+  auto fn = ctx_fn();
+  CUcontext ctx = nullptr;
+  if (!fn || fn(&ctx) != CUDA_SUCCESS || !ctx) return WI_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_scratch);
-    if (e != cudaSuccess || !p) return WI_ERR_CUDA;
-    g_ptr[dev] = p;
-  }
-  *out = g_ptr[dev];
+  for (int i = 0; i < g_n; ++i)
+    if (g_ctx[i] == ctx) { *out = g_ptr[i]; return WI_OK; }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) return WI_ERR_CUDA;
+  if (g_n < kMaxContexts) { g_ctx[g_n] = ctx; g_ptr[g_n] = p; ++g_n; }
+  *out = p;
   return WI_OK;
 }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 }  // namespace
 
 extern "C" wi_status wi_decode_noalloc(const void* q, const wi_index* idx,
                                        const wi_decode_params* p, float* out, float* lse,
                                        wi_stream_t stream) {
+  // every argument error is returned before the first CUDA call
+  if (!q || !out || !aligned(q, 16) || !aligned(out, 4) || (lse && !aligned(lse, 4)))
+    return WI_ERR_INVALID_ARG;
   size_t total = 0, zero_prefix = 0;
   wi_status st = wi::decode_workspace_extent(idx, p, &total, &zero_prefix);
   if (st != WI_OK) return st;

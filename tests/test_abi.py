@@ -288,3 +288,35 @@ def test_selection_bitmap_decoding_on_the_host():
     assert W.selected_clusters(ws, lay, index, 0, 0, 0).tolist() == []
     with pytest.raises(RuntimeError):
         W.selected_clusters(ws, lay, index, 0, 1, 4)
+
+
+def test_noalloc_refuses_on_the_host():
+    """wi_decode_noalloc refuses a decode whose workspace exceeds its fixed
+    scratch, and bad q / out / lse, before any CUDA call: the pointers are
+    never dereferenced."""
+    lib = W.lib()
+    seq = (C.c_int32 * 1)(4_000_000)
+    ix = W.WiIndex()
+    ix.dtype, ix.batch, ix.n_kv_heads, ix.head_dim = W.WI_BF16, 1, 8, 128
+    ix.page_size, ix.seg_len, ix.cluster_size = 16, 8192, 16
+    ix.seq_lens = C.cast(seq, C.POINTER(C.c_int32))
+    for i, f in enumerate(["centroids", "value_sums", "offsets", "perm", "invperm", "labels",
+                           "k_pool", "v_pool", "block_table"]):
+        setattr(ix, f, FAKE + (i + 1) * 0x10000000)
+    ix.n_pages, ix.max_pages = 250_000, 250_000
+    prm = W.DecodeParams(n_q_heads=32).c_struct()
+    n = C.c_size_t()
+    assert lib.wi_decode_workspace_size(C.byref(ix), C.byref(prm), C.byref(n)) == W.WI_OK
+    assert n.value > W.NOALLOC_SCRATCH_MIB << 20
+    assert lib.wi_decode_noalloc(FAKE, C.byref(ix), C.byref(prm), FAKE, None, None) \
+        == W.WI_ERR_WORKSPACE
+    small = index_struct()
+    p = params()
+    assert lib.wi_decode_noalloc(None, C.byref(small), C.byref(p), FAKE, None, None) \
+        == W.WI_ERR_INVALID_ARG
+    assert lib.wi_decode_noalloc(FAKE, C.byref(small), C.byref(p), None, None, None) \
+        == W.WI_ERR_INVALID_ARG
+    assert lib.wi_decode_noalloc(FAKE + 8, C.byref(small), C.byref(p), FAKE, None, None) \
+        == W.WI_ERR_INVALID_ARG
+    assert lib.wi_decode_noalloc(FAKE, C.byref(small), C.byref(p), FAKE, FAKE + 2, None) \
+        == W.WI_ERR_INVALID_ARG

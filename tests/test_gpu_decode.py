@@ -5,8 +5,10 @@ Checked per unit: centroid scores (a1), the retrieved set (a2: identical
 except clusters whose score lies within 1e-5 relative of the k-th), and the
 merged output and lse (a3-a6) within the benchmark spec's tolerance: max|d|/max|ref|
 <= 1e-5 for fp32 inputs, max|d|/rms(ref) <= 2e-2 for bf16 inputs.  A second,
-tighter bound (fp32 accumulation of at most a few thousand terms, see
-the design doc) catches bugs the loose bf16 tolerance would hide.
+tighter bound, 2e-4 of rms(ref), catches bugs the loose bf16 tolerance would
+hide: both sides decode the same stored index values, and the GPU departs
+from the oracle only by fp32 accumulation and the two-term bf16 split of the
+softmax weights (about 2^-17 relative), far below it.
 """
 import math
 

@@ -26,6 +26,10 @@ MUTATIONS = {
     "empty cluster reset": ("C = np.array(C_prev, dtype=np.float64, copy=True)",
                             "C = np.zeros_like(C_prev, dtype=np.float64)"),
     "assign sign flip": ("dist = (X * X).sum(1)[:, None] - 2.0", "dist = (X * X).sum(1)[:, None] + 2.0"),
+    "distance sign flip": ("    return (X * X).sum(1)[:, None] - 2.0 * (X @ C.T)",
+                           "    return (X * X).sum(1)[:, None] + 2.0 * (X @ C.T)"),
+    "distance drops the centroid norm": ("- 2.0 * (X @ C.T) + (C * C).sum(1)[None, :]\n\n\ndef kmeans_update",
+                                         "- 2.0 * (X @ C.T)\n\n\ndef kmeans_update"),
     "merge drops rescale": ("num += f[:, None] * oi", "num += oi"),
     "steady counted twice": ("if not is_steady_pos[ix.perm[slot]]:", "if True:"),
     "estimate ignores counts": ("cnt_p[X].astype(np.float64)", "np.ones(len(X))"),
@@ -48,6 +52,7 @@ MUTATIONS = {
 PINS = [
     lambda: pins.test_round_bf16_matches_torch_on_fp32_inputs(),
     lambda: pins.test_assign_matches_scipy_vq(),
+    lambda: pins.test_distances_match_scipy_cdist_and_a_direct_loop(),
     lambda: pins.test_lloyd_matches_sklearn(),
     lambda: pins.test_kmeans_init_positions_and_empty_cluster_keeps_centroid(),
     lambda: pins.test_steady_positions(),

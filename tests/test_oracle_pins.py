@@ -91,6 +91,24 @@ def test_assign_matches_scipy_vq():
     assert np.array_equal(O.kmeans_assign(X, C), lab)
 
 
+def test_distances_match_scipy_cdist_and_a_direct_loop():
+    """kmeans_distances decides which GPU assignment flips count as near-ties,
+    so it is pinned to scipy's squared Euclidean distance and to the direct
+    per-pair sum of squared differences."""
+    from scipy.spatial.distance import cdist
+    rng = np.random.default_rng(11)
+    X, _, _ = mixture(rng, 400, 24, scale=np.exp(0.5 * rng.standard_normal(24)))
+    C = 2.0 * rng.standard_normal((37, 24))
+    got = O.kmeans_distances(X, C)
+    np.testing.assert_allclose(got, cdist(X, C, "sqeuclidean"), rtol=1e-12, atol=1e-9)
+    for i in (0, 123, 399):
+        for j in (0, 17, 36):
+            direct = sum((X[i, e] - C[j, e]) ** 2 for e in range(24))
+            assert abs(got[i, j] - direct) <= 1e-10 * direct
+    # a point on a centroid is at distance zero from it
+    assert abs(O.kmeans_distances(C[5:6], C)[0, 5]) <= 1e-12 * float((C[5] ** 2).sum())
+
+
 def test_assign_ties_go_to_lower_index():
     X = np.array([[0.0, 0.0], [0.0, 0.0], [2.0, 0.0]])
     C = np.array([[0.0, 1.0], [1.0, 0.0], [-1.0, 0.0], [1.0, 0.0]])

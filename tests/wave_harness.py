@@ -140,3 +140,27 @@ def rel_err(got: np.ndarray, ref: np.ndarray, dtype: torch.dtype) -> float:
 
 
 TOL = {torch.float32: 1e-5, torch.bfloat16: 2e-2}
+
+
+def assert_one_round_moves_are_near_ties(X: np.ndarray, lab_g: np.ndarray, lab_o: np.ndarray,
+                                         seg_len: int, cluster_size: int) -> int:
+    """After one round from the initial centroids, a position whose GPU
+    cluster differs from the oracle's must be a near-tie under those initial
+    centroids: its fp64 distance to the GPU's centroid lies within 1e-5
+    relative of the distance to the oracle's.  lab_g / lab_o are global
+    cluster ids per original position of one unit.  Returns the count."""
+    moved = 0
+    c0 = 0
+    for s, n in O.segment_spans(len(X), seg_len):
+        m = O.clusters_in_segment(n, cluster_size)
+        g, o = lab_g[s:s + n] - c0, lab_o[s:s + n] - c0
+        bad = np.nonzero(g != o)[0]
+        if len(bad):
+            assert g[bad].min() >= 0 and g[bad].max() < m, "moved outside its segment"
+            D = O.kmeans_distances(X[s:s + n][bad], O.kmeans_init(X[s:s + n], cluster_size))
+            dg = D[np.arange(len(bad)), g[bad]]
+            do = D[np.arange(len(bad)), o[bad]]
+            assert np.all(dg <= do * (1 + 1e-5)), "one-round assignment differs beyond near-ties"
+            moved += len(bad)
+        c0 += m
+    return moved

@@ -130,6 +130,10 @@ typedef struct wi_index {
   int32_t max_pages;
 } wi_index;
 
+/* Retrieval-zone selection modes (wi_decode_params.topk_mode). */
+#define WI_TOPK_EXACT   0  /* the k best candidates, lower id first on equal scores */
+#define WI_TOPK_SAMPLED 1  /* Vortex 2.C stochastic radix top-k: see below          */
+
 /* Decode options (query-dependent phase). */
 typedef struct wi_decode_params {
   int32_t n_q_heads;           /* Hq, a multiple of Hkv with G in {1,2,4,8}     */
@@ -144,23 +148,41 @@ typedef struct wi_decode_params {
                                   attention over the retrieved clusters and the
                                   steady zone only (the block top-k workload of
                                   Vortex 2.A on a wi_build_blocks index)        */
+  int32_t topk_mode;           /* WI_TOPK_EXACT or WI_TOPK_SAMPLED.  Sampled
+                                  (Vortex 2.C, early termination by sampling):
+                                  the selection keys are ranked by the top 11
+                                  bits of the fp32 group-max score's
+                                  order-preserving key; every candidate in a bin
+                                  above the bin of the k-th key is retrieved,
+                                  and the rest are drawn from that bin without
+                                  replacement: cluster c draws
+                                  SplitMix64(seed * 2^32 + c) and the smallest
+                                  (draw, c) win                                 */
+  uint32_t seed;               /* draws of WI_TOPK_SAMPLED                      */
+  float *scores_out;           /* optional device float [Hkv*sum NC_b][G]: each
+                                  cluster's score q_g . centroid / sqrt(d) per
+                                  query head (rows laid out like the centroids;
+                                  units attended densely are not written).  It
+                                  costs 4 G bytes of writes per cluster.        */
 } wi_decode_params;
 
 /* Byte offsets of the decode workspace regions (for inspection and tests). */
 typedef struct wi_decode_layout {
   size_t total_bytes;
   size_t status;       /* uint32 status word (offset 0)                           */
-  size_t scores;       /* float [Hkv*sum NC_b][G]: q_h . centroid / sqrt(d)      */
-  size_t keys;         /* uint32 [Hkv*sum NC_b]: order-preserving key of the
-                          group-max score; 0 = not a candidate                   */
-  size_t selected;     /* uint32 [B*Hkv][sel_words]: per unit, bit c % 32 of word
-                          c / 32 is set iff cluster c is retrieved (sel_count
-                          bits; none for a unit attended densely)                 */
-  size_t unit_info;    /* int32 [B*Hkv][8]: {sel_count, thr_key, thr_idx,
-                          sel_tokens, steady, n_affected, dense, candidates}     */
-  int32_t n_attend_ctas; /* exact-attention CTAs per unit                         */
-  int32_t n_score_ctas;  /* score + estimation chunks (CTAs) per unit             */
-  int32_t sel_words;     /* words of `selected` per unit                          */
+  size_t records;      /* uint32 pairs [Hkv*sum NC_b]: {selection key of the
+                          group-max score (order-preserving; 0 = not a
+                          candidate), the cluster's first slot}                  */
+  size_t selected;     /* int32 [Hkv*sum NC_b], rows laid out like the centroids:
+                          the first sel_count entries of a unit's rows are its
+                          retrieved cluster ids, ascending                        */
+  size_t unit_info;    /* int32 [B*Hkv][info_ints]: {sel_count, thr_key, thr_idx,
+                          sel_tokens, steady, n_affected, dense, candidates,
+                          full_rows, partial_rows, non_candidates, no_estimate,
+                          mode, threshold_bin, draw_hi, draw_lo}                  */
+  int32_t n_scan_ctas;   /* streaming CTAs of the scan kernel                     */
+  int32_t n_gather_ctas; /* CTAs of the gather kernel                             */
+  int32_t info_ints;     /* ints per unit record                                  */
 } wi_decode_layout;
 
 /* ------------------------------------------------------------------ sizes */

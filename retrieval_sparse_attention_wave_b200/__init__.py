@@ -40,6 +40,7 @@ WI_MAX_BATCH = 256
 WI_MAX_SEG_LEN = 16384
 WI_MAX_STEADY = 8192
 WI_DEV_BAD_PAGE, WI_DEV_BAD_SLOT, WI_DEV_BAD_CLUSTER, WI_DEV_BAD_HIST = 0x1, 0x2, 0x4, 0x8
+WI_TOPK_EXACT, WI_TOPK_SAMPLED = 0, 1
 
 EXPORTED = [
     "wi_index_clusters", "wi_build_workspace_size", "wi_build_workspace_layout",
@@ -73,7 +74,8 @@ class WiIndex(C.Structure):
 class WiDecodeParams(C.Structure):
     _fields_ = [("n_q_heads", C.c_int32), ("n_sink", C.c_int32), ("window", C.c_int32),
                 ("topk_clusters", C.c_int32), ("topk_fraction", C.c_double),
-                ("stage_events", C.POINTER(C.c_void_p)), ("exact_only", C.c_int32)]
+                ("stage_events", C.POINTER(C.c_void_p)), ("exact_only", C.c_int32),
+                ("topk_mode", C.c_int32), ("seed", C.c_uint32), ("scores_out", C.c_void_p)]
 
 
 class WiBuildLayout(C.Structure):
@@ -82,10 +84,10 @@ class WiBuildLayout(C.Structure):
 
 
 class WiDecodeLayout(C.Structure):
-    _fields_ = [("total_bytes", C.c_size_t), ("status", C.c_size_t), ("scores", C.c_size_t),
-                ("keys", C.c_size_t), ("selected", C.c_size_t), ("unit_info", C.c_size_t),
-                ("n_attend_ctas", C.c_int32), ("n_score_ctas", C.c_int32),
-                ("sel_words", C.c_int32)]
+    _fields_ = [("total_bytes", C.c_size_t), ("status", C.c_size_t), ("records", C.c_size_t),
+                ("selected", C.c_size_t), ("unit_info", C.c_size_t),
+                ("n_scan_ctas", C.c_int32), ("n_gather_ctas", C.c_int32),
+                ("info_ints", C.c_int32)]
 
 
 _P = C.c_void_p
@@ -425,12 +427,20 @@ class DecodeParams:
     topk_clusters: int = -1
     topk_fraction: float = 0.018
     exact_only: bool = False     # no estimation zone (block top-k workload)
+    sampled: bool = False        # stochastic radix top-k (threshold bin sampled)
+    seed: int = 0                # draws of the sampled selection
+    scores_out: Optional[torch.Tensor] = None   # float [Hkv * sum NC_b][G], filled if given
 
     def c_struct(self, events=None) -> WiDecodeParams:
         p = WiDecodeParams()
         p.n_q_heads, p.n_sink, p.window = self.n_q_heads, self.n_sink, self.window
         p.topk_clusters, p.topk_fraction = self.topk_clusters, self.topk_fraction
         p.exact_only = 1 if self.exact_only else 0
+        p.topk_mode = WI_TOPK_SAMPLED if self.sampled else WI_TOPK_EXACT
+        p.seed = int(self.seed) & 0xFFFFFFFF
+        if self.scores_out is not None:
+            assert self.scores_out.dtype == torch.float32 and self.scores_out.is_contiguous()
+            p.scores_out = self.scores_out.data_ptr()
         if events is not None:
             for e in events:
                 if not e.cuda_event:      # torch creates the CUDA event on first record
@@ -522,28 +532,46 @@ def read_device_status(ws: torch.Tensor, stream=None, clear: bool = True) -> int
 # ---------------------------------------------------------------- workspace views
 
 def unit_info(ws: torch.Tensor, layout: WiDecodeLayout, n_units: int) -> torch.Tensor:
-    """Per-unit record {sel_count, thr_key, thr_idx, sel_tokens, steady,
-    n_affected, dense, candidates} from a decode workspace (int32 [U][8])."""
-    return ws[layout.unit_info:layout.unit_info + n_units * 32].view(torch.int32).view(n_units, 8)
+    """Per-unit record from a decode workspace (int32 [U][info_ints]):
+    {sel_count, thr_key, thr_idx, sel_tokens, steady, n_affected, dense,
+    candidates, full_rows, partial_rows, non_candidates, no_estimate, mode,
+    threshold_bin, draw_hi, draw_lo}."""
+    n = layout.info_ints
+    return ws[layout.unit_info:layout.unit_info + n_units * n * 4].view(torch.int32).view(n_units, n)
 
 
 def selected_clusters(ws: torch.Tensor, layout: WiDecodeLayout, index: WaveIndex,
                       b: int, h: int, count: int) -> torch.Tensor:
-    """The retrieved clusters of unit (b, h), ascending, read from the
-    workspace's selection bitmap (`count` of them)."""
-    u = b * index.n_kv_heads + h
-    words = ws[layout.selected:].view(torch.int32)[u * layout.sel_words:(u + 1) * layout.sel_words]
-    bits = (words.to(torch.int64).unsqueeze(1) >> torch.arange(32, device=words.device)) & 1
-    ids = torch.nonzero(bits.flatten()).flatten().to(torch.int32)
-    if len(ids) != count:
-        raise RuntimeError(f"selection bitmap holds {len(ids)} clusters, unit record says {count}")
+    """The retrieved clusters of unit (b, h), ascending: the first `count`
+    entries of the unit's rows of the workspace's selection list (rows laid
+    out like the centroids)."""
+    row = index.cl_row(b, h)
+    if count < 0 or count > index.nc[b]:
+        raise RuntimeError(f"selection count {count} outside [0, {index.nc[b]}]")
+    ids = ws[layout.selected:].view(torch.int32)[row:row + count].clone()
+    if count > 1 and not bool(torch.all(ids[1:] > ids[:-1])):
+        raise RuntimeError("selection list is not ascending")
     return ids
 
 
-def centroid_scores(ws: torch.Tensor, layout: WiDecodeLayout, index: WaveIndex, G: int,
-                    b: int, h: int) -> torch.Tensor:
-    """fp32 scores [NC_b][G] of unit (b, h) from a decode workspace."""
+def selection_keys(ws: torch.Tensor, layout: WiDecodeLayout, index: WaveIndex,
+                   b: int, h: int) -> torch.Tensor:
+    """The order-preserving selection keys of unit (b, h)'s clusters (uint32
+    values in an int64 tensor; 0 = not a candidate)."""
     row = index.cl_row(b, h)
     n = index.nc[b]
-    flat = ws[layout.scores:].view(torch.float32)
-    return flat[row * G:(row + n) * G].view(n, G)
+    rec = ws[layout.records:].view(torch.int32)[2 * row:2 * (row + n)].view(n, 2)
+    return rec[:, 0].to(torch.int64) & 0xFFFFFFFF
+
+
+def scores_buffer(index: WaveIndex, n_q_heads: int) -> torch.Tensor:
+    """A float [Hkv * sum NC_b][G] buffer for DecodeParams.scores_out."""
+    G = n_q_heads // index.n_kv_heads
+    return torch.zeros(index.n_kv_heads * sum(index.nc), G, dtype=torch.float32,
+                       device=index.centroids.device)
+
+
+def centroid_scores(scores: torch.Tensor, index: WaveIndex, b: int, h: int) -> torch.Tensor:
+    """fp32 scores [NC_b][G] of unit (b, h) from a scores_out buffer."""
+    row = index.cl_row(b, h)
+    return scores[row:row + index.nc[b]]

@@ -80,6 +80,9 @@ int64_t n_steady(int64_t T, int64_t n_sink, int64_t window) {
 }
 
 
+// Chunk map of the scan: CTA that takes chunk k of n over N CTAs
+int scan_cta_of(int64_t k, int64_t n, int64_t N) { return (int)(((k + 1) * N - 1) / n); }
+
 wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, DecodePlan& pl) {
   if (!ix || !p) return WI_ERR_INVALID_ARG;
   wi_status st = check_common(ix->dtype, ix->batch, ix->n_kv_heads, ix->head_dim, ix->page_size,
@@ -100,76 +103,129 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   if (p->n_sink < 0 || p->window < 0) return WI_ERR_INVALID_ARG;
   if (p->topk_clusters < 0 && !(p->topk_fraction >= 0.0 && p->topk_fraction <= 1.0))
     return WI_ERR_INVALID_ARG;
+  if (p->topk_mode != WI_TOPK_EXACT && p->topk_mode != WI_TOPK_SAMPLED) return WI_ERR_INVALID_ARG;
+  if (p->scores_out && !aligned(p->scores_out, 4)) return WI_ERR_INVALID_ARG;
 
   std::memset(&pl, 0, sizeof(pl));
   fill_geo(pl.geo, ix->batch, ix->n_kv_heads, ix->head_dim, ix->seq_lens, ix->seg_len,
            ix->cluster_size);
+  const int B = ix->batch, H = ix->n_kv_heads;
   pl.dtype = ix->dtype; pl.D = ix->head_dim; pl.G = G; pl.Hq = p->n_q_heads;
-  pl.U = ix->batch * ix->n_kv_heads;
+  pl.U = B * H;
   pl.n_sink = p->n_sink; pl.window = p->window;
   pl.topk_clusters = p->topk_clusters; pl.topk_fraction = p->topk_fraction;
   pl.exact_only = p->exact_only != 0;
+  pl.mode = p->topk_mode;
+  pl.seed = p->seed;
   pl.scale = 1.0f / std::sqrt((float)ix->head_dim);
 
   int max_nc = 0, cap = 1;
-  for (int b = 0; b < ix->batch; ++b) {
+  bool dense[kMaxBatch];
+  int nst[kMaxBatch];
+  for (int b = 0; b < B; ++b) {
     const int T = ix->seq_lens[b];
     max_nc = std::max(max_nc, pl.geo.NC(b));
-    const int64_t nst = n_steady(T, p->n_sink, p->window);
-    if (nst < T) {  // not attended densely: its steady list is kept
-      if (nst > WI_MAX_STEADY) return WI_ERR_UNSUPPORTED;
-      cap = std::max<int>(cap, (int)nst);
+    const int64_t n = n_steady(T, p->n_sink, p->window);
+    dense[b] = n >= T;
+    nst[b] = (int)std::min<int64_t>(n, T);
+    if (!dense[b]) {   // not attended densely: its steady list is kept
+      if (n > WI_MAX_STEADY) return WI_ERR_UNSUPPORTED;
+      cap = std::max<int>(cap, (int)n);
     }
   }
   pl.max_nc = max_nc;
   pl.cap = cap;
-  pl.sort_pow2 = 1;
-  while (pl.sort_pow2 < cap) pl.sort_pow2 <<= 1;
+  pl.ncl = (int64_t)pl.geo.cl_base[B] * H;
+  pl.ntok = (int64_t)pl.geo.tok_base[B] * H;
 
-  pl.seg_len = ix->seg_len;
-  pl.seg_clusters = ix->seg_len / ix->cluster_size;
-  // score + estimate: one CTA per 32 KB of centroid rows (and their value sums)
-  pl.score_chunk = kScoreChunkBytes / (pl.D * esize(ix->dtype));
-  pl.n_score_blocks = (int)cdiv(max_nc, pl.score_chunk);
-  if (decode_score_smem(pl.dtype, pl.D, G, pl.sort_pow2, cap) > 200 * 1024) return WI_ERR_UNSUPPORTED;
-  // top-k shared memory: exclusion bitmask and the non-candidate list
-  if (decode_topk_smem(max_nc, cap) + 24 * 1024 > 200 * 1024) return WI_ERR_UNSUPPORTED;
-  // attend: range CTAs of kRangeClusters ids, steady CTAs of two 16 KB tiles
-  // of rows
-  const int row_bytes = pl.D * esize(ix->dtype);
-  const int tile_rows = 16384 / row_bytes;
-  pl.n_rng = std::max<int>(1, (int)cdiv(max_nc, kRangeClusters));
-  pl.n_sc = std::max<int>(1, (int)cdiv(cap, 2 * tile_rows));
-  // the tensor-core path (bf16, d = 128) estimates inside the range CTAs;
-  // the CUDA-core path folds the score kernel's chunk parts
-  const bool mma = ix->dtype == WI_BF16 && pl.D == 128;
-  pl.n_fold = mma ? 0 : std::max<int>(1, (int)cdiv(pl.n_score_blocks, kFold));
-  pl.n_parts = pl.n_rng + pl.n_sc + pl.n_fold;
-  if (decode_attend_smem(pl.dtype, pl.D, G, pl.n_parts) + 24 * 1024 > 200 * 1024)
+  // scan: chunks of kTileRows clusters of every unit that is not dense,
+  // contiguous runs of them per CTA, one CTA per SM at most
+  pl.ch_base[0] = 0;
+  for (int b = 0; b < B; ++b) {
+    const int nch = dense[b] ? 0 : (int)cdiv(pl.geo.NC(b), kTileRows);
+    pl.ch_base[b + 1] = pl.ch_base[b] + H * nch;
+  }
+  pl.n_chunks = pl.ch_base[B];
+  pl.n_scan = std::max(1, std::min(pl.n_chunks, kNumSMs));
+  pl.p1max = 1;
+  for (int b = 0; b < B; ++b) {
+    const int nch = (pl.ch_base[b + 1] - pl.ch_base[b]) / H;
+    for (int h = 0; h < H && nch > 0; ++h) {
+      const int64_t k0 = pl.ch_base[b] + (int64_t)h * nch;
+      const int parts = scan_cta_of(k0 + nch - 1, pl.n_chunks, pl.n_scan) -
+                        scan_cta_of(k0, pl.n_chunks, pl.n_scan) + 1;
+      pl.p1max = std::max(pl.p1max, parts);
+    }
+  }
+  // units a scan CTA touches (it runs the tails of those it finishes last)
+  {
+    int b = 0;
+    for (int sc = 0; sc < pl.n_scan && pl.n_chunks > 0; ++sc) {
+      const int64_t k0 = (int64_t)sc * pl.n_chunks / pl.n_scan;
+      const int64_t k1 = (int64_t)(sc + 1) * pl.n_chunks / pl.n_scan;
+      int touched = 0, last_u = -1;
+      for (int64_t k = k0; k < k1; ++k) {
+        while (b + 1 < B && pl.ch_base[b + 1] <= k) ++b;
+        while (b > 0 && pl.ch_base[b] > k) --b;
+        const int per = (pl.ch_base[b + 1] - pl.ch_base[b]) / H;
+        const int u = b * H + (int)((k - pl.ch_base[b]) / per);
+        if (u != last_u) { ++touched; last_u = u; }
+        if (touched > kMaxTailsPerCta) return WI_ERR_UNSUPPORTED;
+        // skip to the unit's last chunk in this CTA's range
+        const int64_t unit_end = pl.ch_base[b] + (int64_t)(u - b * H + 1) * per;
+        k = std::min<int64_t>(k1, unit_end) - 1;
+      }
+    }
+  }
+  const size_t slot = decode_scan_slot_bytes(pl.dtype, pl.D, pl.exact_only);
+  pl.slots = (int)std::max<size_t>(2, std::min<size_t>(4, (size_t)131072 / slot));
+  if (decode_scan_smem(pl.dtype, pl.D, G, pl.slots, pl.exact_only) > 227 * 1024)
     return WI_ERR_UNSUPPORTED;
+  if (decode_gather_smem(pl.dtype, pl.D, G) > 227 * 1024) return WI_ERR_UNSUPPORTED;
+  if (decode_steady_smem(cap) > 96 * 1024) return WI_ERR_UNSUPPORTED;
 
-  const int64_t ncl = (int64_t)pl.geo.cl_base[ix->batch] * ix->n_kv_heads;
-  pl.ncl = ncl;
+  // gather: per sequence, CTAs for the rows the unit is expected to hold
+  // (retrieved tokens at cluster_size each, steady tokens, and the rows taken
+  // out of the estimate), kGatherTiles tiles each; they loop over more
+  const int rpb = kGatherTiles * kTileRows;
+  pl.n2_base[0] = 0;
+  pl.n2max = 1;
+  for (int b = 0; b < B; ++b) {
+    const int T = ix->seq_lens[b], NC = pl.geo.NC(b);
+    int64_t rows;
+    if (dense[b]) {
+      rows = T;
+    } else {
+      const int64_t kr = p->topk_clusters >= 0 ? p->topk_clusters
+                                               : (int64_t)std::ceil(p->topk_fraction * (double)NC);
+      const int64_t k = std::min<int64_t>(std::max<int64_t>(kr, 0), NC);
+      rows = std::min<int64_t>(k * ix->cluster_size, T) + nst[b];
+      if (!pl.exact_only) rows += k + nst[b];
+    }
+    const int n2 = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(rows, rpb), kMaxGatherPerUnit));
+    pl.n2_base[b + 1] = pl.n2_base[b] + H * n2;
+    pl.n2max = std::max(pl.n2max, n2);
+  }
+  pl.n_gather = pl.n2_base[B];
+
   size_t o = 0;
   auto take = [&](size_t bytes) { const size_t r = o; o = align_up(o + bytes, 256); return r; };
+  const size_t PS = (size_t)G * (pl.D + 4) * 4;   // one part: G heads of {m, l, -, -, o[D]}
   pl.off_status = take(256);
-  pl.off_counters = take((size_t)pl.U * 4);
-  pl.off_hist = take((size_t)pl.U * 2048 * 4);      // zeroed after use by the top-k kernel
-  pl.off_aff_of = take((size_t)pl.U * max_nc * 4);  // reset after use by the attend kernel
-  pl.off_scores = take((size_t)ncl * G * 4);
-  pl.off_keys = take((size_t)ncl * 4);
-  pl.sel_words = pl.n_rng * (kRangeClusters / 32);
-  pl.off_sel = take((size_t)pl.U * pl.sel_words * 4);
+  pl.off_cnt1 = take((size_t)pl.U * 4);
+  pl.off_cnt2 = take((size_t)pl.U * 4);
+  pl.off_hist = take((size_t)pl.U * kHistBins * 4);   // zeroed after use by the tails
+  pl.off_rec = take((size_t)pl.ncl * 8);
   pl.off_info = take((size_t)pl.U * kInfoInts * 4);
   pl.off_st_slot = take((size_t)pl.U * cap * 4);
-  pl.off_st_cl = take((size_t)pl.U * cap * 4);
-  pl.off_aff_cl = take((size_t)pl.U * cap * 4);
-  pl.off_aff_start = take((size_t)pl.U * (cap + 1) * 4);
-  pl.off_partials = take((size_t)pl.U * pl.n_parts * G * (pl.D + 4) * 4);
-  pl.off_dv = take((size_t)pl.U * cap * pl.D * 4);
-  pl.off_est = take(mma ? 0 : (size_t)pl.U * pl.n_score_blocks * G * (pl.D + 4) * 4);
-  pl.off_nonc = take((size_t)pl.U * (cap + 1) * 4);
-  const size_t nq = (size_t)ix->batch * p->n_q_heads;
+  pl.off_pc = take((size_t)pl.U * cap * 8);
+  pl.off_nonc = take((size_t)pl.U * cap * 8);
+  pl.off_sel = take((size_t)pl.ncl * 4);
+  pl.off_tok = take((size_t)pl.ntok * 4);
+  pl.off_full = take(((size_t)pl.ncl + (size_t)pl.U * cap) * 8);
+  pl.off_est = take(pl.exact_only ? 0 : (size_t)pl.U * pl.p1max * PS);
+  pl.off_gat = take((size_t)pl.U * pl.n2max * PS);
+  const size_t nq = (size_t)B * p->n_q_heads;
   pl.off_q = take(nq * pl.D * esize(ix->dtype));
   pl.off_out = take(nq * pl.D * 4);
   pl.off_lse = take(nq * 4);
@@ -252,6 +308,7 @@ wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params*
   a.lse = lse;
   a.ws = w;
   a.stage_events = reinterpret_cast<cudaEvent_t*>(p->stage_events);
+  a.scores_out = p->scores_out;
   cudaError_t e = launch_decode(pl, a, s);
   if (e != cudaSuccess) return cuda_fail(e);
   if (host) {
@@ -273,7 +330,7 @@ wi_status decode_workspace_extent(const wi_index* idx, const wi_decode_params* p
   const wi_status st = make_decode_plan(idx, p, pl);
   if (st != WI_OK) return st;
   *total = pl.total;
-  *zero_prefix = pl.off_scores;
+  *zero_prefix = pl.off_rec;
   return WI_OK;
 }
 
@@ -486,13 +543,12 @@ wi_status wi_decode_workspace_layout(const wi_index* idx, const wi_decode_params
   if (st != WI_OK) return st;
   layout->total_bytes = pl.total;
   layout->status = pl.off_status;
-  layout->scores = pl.off_scores;
-  layout->keys = pl.off_keys;
+  layout->records = pl.off_rec;
   layout->selected = pl.off_sel;
   layout->unit_info = pl.off_info;
-  layout->n_attend_ctas = pl.n_rng + pl.n_sc;
-  layout->n_score_ctas = pl.n_score_blocks;
-  layout->sel_words = pl.sel_words;
+  layout->n_scan_ctas = pl.n_scan;
+  layout->n_gather_ctas = pl.n_gather;
+  layout->info_ints = kInfoInts;
   return WI_OK;
 }
 

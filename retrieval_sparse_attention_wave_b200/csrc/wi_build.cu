@@ -14,6 +14,7 @@
 //           permuted pools (one pass over K and V).
 #include <cfloat>
 #include <climits>
+#include <type_traits>
 
 #include "wi_common.cuh"
 #include "wi_plan.h"
@@ -165,6 +166,246 @@ kmeans_assign_kernel(const Geo geo, const Pool kin, int S, int cs, const SegFrom
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       if (ty * 4 + i < ntok) dst[ty * 4 + i] = besti[i];
+  }
+}
+
+// --------------------------------------------- assign on the tensor cores
+// bf16 keys are exact in bf16, so ||k - c||^2 = ||c||^2 - 2 k.c + ||k||^2
+// can take k.c from the tensor cores: the fp32 centroid c is split into
+// three bf16 terms c1 + c2 + c3 (c1 = bf16(c), c2 = bf16(c - c1), c3 =
+// bf16(c - c1 - c2); the rest is below 2^-24 |c|) and k.c1 + k.c2 + k.c3 is
+// accumulated in fp32 on m16n8k16 (the products of two bf16 values are exact
+// in fp32).  A CTA takes kMTok tokens of a segment against all its centroids,
+// kMCen at a time; each warp keeps, per token, the two smallest approximate
+// distances a = ||c||^2 - 2 k.c.
+//
+// The decision is the direct form's: the kernel above computes
+// d = sum_e (k_e - c_e)^2 in fp32 (ascending e, fused multiply-add), and a
+// token whose two best approximate distances are more than delta apart takes
+// the best, since both |a - ||k - c||^2 + ||k||^2 ...| errors are below
+// delta / 2 (see the bound below); any other token re-evaluates the direct
+// form over all the segment's centroids, with the same arithmetic and the
+// same tie rule (lower index), so the assignment equals the direct form's.
+//
+// Error bound: the direct form sums 128 terms, error <= 128 * 2^-24 * d
+// <= 2^-17 (|k|^2 + |c|^2) * 2; the tensor-core form adds at most 384
+// accumulations of products bounded by |k||c| <= (|k|^2 + |c|^2) / 2, each
+// within 2^-23 relative, plus ||c||^2 in fp32 (128 * 2^-24 |c|^2): together
+// below 2^-13 (|k|^2 + |c|^2).  delta = 2^-12 (|k|^2 + max |c|^2) leaves a
+// factor of two.
+constexpr int kMTok = 128, kMCen = 64;
+
+__device__ __forceinline__ int mtile_off(int rows, int r, int c) {   // 16-byte chunk c of row r
+  return (c >> 3) * (rows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+}
+
+template <int D>
+__global__ void __launch_bounds__(256, 2)
+kmeans_assign_mma_kernel(const Geo geo, const Pool kin, int S, int cs, const SegFrom sf,
+                         const float* __restrict__ cent32, int32_t* __restrict__ assign,
+                         uint32_t* status) {
+  using T = __nv_bfloat16;
+  constexpr int CH = D / 8;                     // 16-byte chunks per bf16 row
+  extern __shared__ __align__(1024) unsigned char sh_mma[];
+  unsigned char* sk = sh_mma;                                  // [kMTok][D] bf16, swizzled
+  unsigned char* sc = sk + kMTok * D * 2;                      // 3 x [kMCen][D] bf16 terms
+  float* cn2 = reinterpret_cast<float*>(sc + 3 * kMCen * D * 2);   // [kMCen] |c|^2
+  float* xn2 = cn2 + kMCen;                                    // [kMTok] |k|^2
+  __shared__ float s_cmax2;
+  __shared__ int s_namb;
+  __shared__ int s_amb[kMTok];
+  const int u = blockIdx.z, b = u / geo.hkv, h = u - b * geo.hkv;
+  const int T_ = geo.T(b);
+  const int seg = sf.s0[b] + (int)blockIdx.y, start = seg * S;
+  if (start >= T_) return;
+  const int len = min(S, T_ - start);
+  const int t0 = blockIdx.x * kMTok;
+  if (t0 >= len) return;
+  const int ntok = min(kMTok, len - t0);
+  const int ncl = (len + cs - 1) / cs;
+  const int64_t crow = geo.cl_row(b, h) + (int64_t)seg * (S / cs);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tq = lane & 3;
+
+  // keys of the tile (zero rows past the segment), and their squared norms
+  for (int x = tid; x < kMTok * CH; x += blockDim.x) {
+    const int r = x / CH, c = x - r * CH;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < ntok) {
+      const int64_t ro = pool_row(kin, geo.hkv, D, b, h, start + t0 + r, status);
+      if (ro >= 0) v = ld_stream(reinterpret_cast<const T*>(kin.base) + ro + c * 8);
+    }
+    *reinterpret_cast<uint4*>(sk + mtile_off(kMTok, r, c)) = v;
+  }
+  if (tid == 0) { s_cmax2 = 0.f; s_namb = 0; }
+  __syncthreads();
+  for (int r = warp; r < kMTok; r += 8) {
+    float ss = 0.f;
+    for (int c = lane; c < CH; c += 32) {
+      const uint4 v = *reinterpret_cast<const uint4*>(sk + mtile_off(kMTok, r, c));
+      float xv[8];
+      Elem<T>::unpack(v, xv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(xv[e], xv[e], ss);
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) xn2[r] = ss;
+  }
+  // A fragments of the warp's 16 tokens, all k-steps (kept in registers)
+  uint32_t qa[D / 16][4];
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks)
+    ldsm_x4(qa[ks], sk + mtile_off(kMTok, 16 * warp + (lane & 15), 2 * ks + (lane >> 4)));
+
+  float b1[2] = {INFINITY, INFINITY}, b2[2] = {INFINITY, INFINITY};
+  int i1[2] = {0, 0};
+  for (int cb = 0; cb < ncl; cb += kMCen) {
+    __syncthreads();
+    // the chunk's centroids: three bf16 terms each, and |c|^2 in fp32
+    for (int x = tid; x < kMCen * (D / 8); x += blockDim.x) {
+      const int j = x / (D / 8), c8 = x - j * (D / 8);
+      float v[8];
+      if (cb + j < ncl) {
+        const float4 lo = *reinterpret_cast<const float4*>(cent32 + (crow + cb + j) * D + c8 * 8);
+        const float4 hi = *reinterpret_cast<const float4*>(cent32 + (crow + cb + j) * D + c8 * 8 + 4);
+        v[0] = lo.x; v[1] = lo.y; v[2] = lo.z; v[3] = lo.w;
+        v[4] = hi.x; v[5] = hi.y; v[6] = hi.z; v[7] = hi.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      }
+      uint32_t w[3][4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const __nv_bfloat162 t1 = __floats2bfloat162_rn(v[e], v[e + 1]);
+        const float2 f1 = __bfloat1622float2(t1);
+        const float r0 = v[e] - f1.x, r1 = v[e + 1] - f1.y;
+        const __nv_bfloat162 t2 = __floats2bfloat162_rn(r0, r1);
+        const float2 f2 = __bfloat1622float2(t2);
+        const __nv_bfloat162 t3 = __floats2bfloat162_rn(r0 - f2.x, r1 - f2.y);
+        w[0][e / 2] = *reinterpret_cast<const uint32_t*>(&t1);
+        w[1][e / 2] = *reinterpret_cast<const uint32_t*>(&t2);
+        w[2][e / 2] = *reinterpret_cast<const uint32_t*>(&t3);
+      }
+#pragma unroll
+      for (int t = 0; t < 3; ++t)
+        *reinterpret_cast<uint4*>(sc + t * kMCen * D * 2 + mtile_off(kMCen, j, c8)) =
+            make_uint4(w[t][0], w[t][1], w[t][2], w[t][3]);
+    }
+    for (int j = warp; j < kMCen; j += 8) {
+      float ss = 0.f;
+      if (cb + j < ncl)
+        for (int e = lane; e < D; e += 32) {
+          const float c = cent32[(crow + cb + j) * D + e];
+          ss = fmaf(c, c, ss);
+        }
+      ss = warp_sum(ss);
+      if (lane == 0) {
+        cn2[j] = ss;
+        atomicMax(reinterpret_cast<int*>(&s_cmax2), __float_as_int(ss));   // ss >= 0
+      }
+    }
+    __syncthreads();
+    // k.c for the warp's 16 tokens x the chunk's 64 centroids
+    float acc[kMCen / 8][4];
+#pragma unroll
+    for (int nt = 0; nt < kMCen / 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+      const unsigned char* ct = sc + t * kMCen * D * 2;
+#pragma unroll
+      for (int nt = 0; nt < kMCen / 8; ++nt) {
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ks += 2) {
+          uint32_t bm[4];
+          ldsm_x4(bm, ct + mtile_off(kMCen, 8 * nt + (lane & 7), 2 * ks + (lane >> 3)));
+          mma_bf16_4(acc[nt], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], bm[0], bm[1]);
+          mma_bf16_4(acc[nt], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3],
+                     bm[2], bm[3]);
+        }
+      }
+    }
+    // the two smallest a = |c|^2 - 2 k.c per token (rows g, g + 8), lower
+    // index first on equal values
+#pragma unroll
+    for (int nt = 0; nt < kMCen / 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 8 * nt + 2 * tq + (e & 1);
+        const int tk = e >> 1;
+        if (cb + j < ncl) {
+          const float a = cn2[j] - 2.f * acc[nt][e];
+          if (a < b1[tk]) { b2[tk] = b1[tk]; b1[tk] = a; i1[tk] = cb + j; }
+          else if (a < b2[tk]) b2[tk] = a;
+        }
+      }
+  }
+  // merge over the four lanes that share the tokens
+#pragma unroll
+  for (int tk = 0; tk < 2; ++tk) {
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      const float ob1 = __shfl_xor_sync(0xffffffffu, b1[tk], o);
+      const float ob2 = __shfl_xor_sync(0xffffffffu, b2[tk], o);
+      const int oi1 = __shfl_xor_sync(0xffffffffu, i1[tk], o);
+      if (ob1 < b1[tk] || (ob1 == b1[tk] && oi1 < i1[tk])) {
+        b2[tk] = fminf(b1[tk], ob2);
+        b1[tk] = ob1;
+        i1[tk] = oi1;
+      } else {
+        b2[tk] = fminf(b2[tk], ob1);
+      }
+    }
+  }
+  __syncthreads();
+  const float cmax2 = s_cmax2;
+  int32_t* dst = assign + geo.tok_row(b, h) + start + t0;
+  if (tq == 0) {
+#pragma unroll
+    for (int tk = 0; tk < 2; ++tk) {
+      const int r = 16 * warp + g + 8 * tk;
+      if (r < ntok) {
+        const float delta = ldexpf(xn2[r] + cmax2, -12);
+        if (b2[tk] - b1[tk] > delta) dst[r] = i1[tk];
+        else s_amb[atomicAdd(&s_namb, 1)] = r;
+      }
+    }
+  }
+  __syncthreads();
+  // near the decision boundary: the direct form over every centroid, as the
+  // FMA kernel computes it (fp32, ascending e, lower index on ties)
+  const int namb = s_namb;
+  for (int a = warp; a < namb; a += 8) {
+    const int r = s_amb[a];
+    float best = INFINITY;
+    int bi = 0;
+    for (int j = lane; j < ncl; j += 32) {
+      const float* c = cent32 + (crow + j) * D;
+      float acc = 0.f;
+#pragma unroll 4
+      for (int c8 = 0; c8 < D / 8; ++c8) {
+        float xv[8];
+        Elem<T>::unpack(*reinterpret_cast<const uint4*>(sk + mtile_off(kMTok, r, c8)), xv);
+        const float4 lo = *reinterpret_cast<const float4*>(c + c8 * 8);
+        const float4 hi = *reinterpret_cast<const float4*>(c + c8 * 8 + 4);
+        const float cv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float df = xv[e] - cv[e];
+          acc = fmaf(df, df, acc);
+        }
+      }
+      if (acc < best) { best = acc; bi = j; }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob < best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+    }
+    if (lane == 0) dst[r] = bi;
   }
 }
 
@@ -373,6 +614,32 @@ cudaError_t with_build_types(int dtype, int D, F&& f) {
 }
 
 size_t assign_smem(int D) { return (size_t)D * ((kTok + kPad) + (kCen + kPad)) * sizeof(float); }
+size_t assign_mma_smem(int D) {
+  return (size_t)kMTok * D * 2 + (size_t)3 * kMCen * D * 2 + (size_t)(kMCen + kMTok) * 4;
+}
+
+// One assignment pass over every unit's segments: the tensor-core kernel for
+// bf16 keys, the fp32 direct form otherwise.
+template <typename T, int D>
+cudaError_t launch_assign(const BuildPlan& p, const Pool& kin, const float* cent32,
+                          int32_t* assign, uint32_t* status, cudaStream_t s) {
+  if constexpr (std::is_same_v<T, __nv_bfloat16>) {
+    const size_t smem = assign_mma_smem(D);
+    cudaFuncSetAttribute(kmeans_assign_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    const dim3 grid((p.S + kMTok - 1) / kMTok, p.nseg_grid, p.U);
+    kmeans_assign_mma_kernel<D><<<grid, 256, smem, s>>>(p.geo, kin, p.S, p.cs, p.sf, cent32,
+                                                        assign, status);
+  } else {
+    const size_t smem = assign_smem(D);
+    cudaFuncSetAttribute(kmeans_assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    const dim3 grid((p.S + kTok - 1) / kTok, p.nseg_grid, p.U);
+    kmeans_assign_kernel<T, D><<<grid, 256, smem, s>>>(p.geo, kin, p.S, p.cs, p.sf, cent32,
+                                                       assign, status);
+  }
+  return cudaGetLastError();
+}
 
 }  // namespace
 
@@ -380,13 +647,7 @@ cudaError_t launch_assign_only(const BuildPlan& p, const BuildArgs& a, const flo
                                int32_t* assign, cudaStream_t s) {
   uint32_t* status = reinterpret_cast<uint32_t*>(a.ws + p.off_status);
   return with_build_types(p.dtype, p.D, [&]<typename T, int D>() -> cudaError_t {
-    const size_t smem = assign_smem(D);
-    cudaFuncSetAttribute(kmeans_assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    const dim3 grid((p.S + kTok - 1) / kTok, p.nseg_grid, p.U);
-    kmeans_assign_kernel<T, D><<<grid, 256, smem, s>>>(p.geo, a.kin, p.S, p.cs, p.sf, cent32,
-                                                       assign, status);
-    return cudaGetLastError();
+    return launch_assign<T, D>(p, a.kin, cent32, assign, status, s);
   });
 }
 
@@ -395,9 +656,6 @@ cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s)
   float* cent32 = reinterpret_cast<float*>(a.ws + p.off_cent32);
   int32_t* assign = reinterpret_cast<int32_t*>(a.ws + p.off_assign);
   return with_build_types(p.dtype, p.D, [&]<typename T, int D>() -> cudaError_t {
-    const size_t smem = assign_smem(D);
-    cudaFuncSetAttribute(kmeans_assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
     cudaFuncSetAttribute(kmeans_update_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)p.update_smem);
     if (p.nseg_grid < 1) return cudaSuccess;   // nothing new to cluster
@@ -417,10 +675,9 @@ cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s)
     fin.pout = Pool{a.kout, a.bt_out, a.n_pages_out, a.max_pages_out, a.page_shift_out};
     fin.vin = a.vin;
     fin.enabled = 1;
-    const dim3 agrid((p.S + kTok - 1) / kTok, p.nseg_grid, p.U);
     for (int it = 0; it < p.iters; ++it) {
-      kmeans_assign_kernel<T, D><<<agrid, 256, smem, s>>>(p.geo, a.kin, p.S, p.cs, p.sf, cent32,
-                                                          assign, status);
+      const cudaError_t ea = launch_assign<T, D>(p, a.kin, cent32, assign, status, s);
+      if (ea != cudaSuccess) return ea;
       kmeans_update_kernel<T, D><<<dim3(p.nseg_grid, p.U), kUpdThreads, p.update_smem, s>>>(
           p.geo, a.kin, p.S, p.cs, p.sf, cent32, assign, it == p.iters - 1 ? fin : none, status);
     }

@@ -176,6 +176,16 @@ __device__ __forceinline__ int warp_sum_int(int v) {
   return v;
 }
 
+// Named barrier `id` over the first `n` threads of the CTA (a multiple of 32);
+// id 0 is __syncthreads' barrier.
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Loads of data other CTAs of the same grid wrote (L2, bypassing L1).
+__device__ __forceinline__ int ldcg_i32(const int32_t* p) { return __ldcg(p); }
+__device__ __forceinline__ uint32_t ldcg_u32(const uint32_t* p) { return __ldcg(p); }
+
 // Programmatic dependent launch: let the next kernel in the stream start its
 // prologue now / wait until the previous kernel's results are visible.
 __device__ __forceinline__ void pdl_launch_dependents() {
@@ -281,6 +291,15 @@ __device__ __forceinline__ void mma_bf16_4(float (&d)[4], uint32_t a0, uint32_t 
       " {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// d += a * b, m16n8k8 (bf16 in, fp32 accumulate): a0 rows 0..7 and a1 rows
+// 8..15 of A (k 2t, 2t+1 of thread t % 4), b0 the k-pair of column t / 4
+__device__ __forceinline__ void mma_bf16_k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6},"
+      " {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
 }
 // two floats as a bf16 pair (round to nearest even), low element first
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

@@ -1,0 +1,1646 @@
+#pragma once
+// Decode-step kernels of the wave index (sm_100a), included by the
+// per-type translation units that instantiate them.
+//
+// One decode step is the query-dependent phase of the method (RetroInfer
+// technical summary, section 2.A, items 1-3; Vortex summary, section 2.A
+// forward_indexer).  Three launches, chained with programmatic dependent
+// launch:
+//
+//  K0 steady   one CTA per unit resolves the steady zone (item 1): sink and
+//              window positions -> slots and clusters, sorted by slot; the
+//              clusters left without a non-steady token (not candidates) and
+//              the steady tokens of the other affected clusters.  It runs
+//              beside K1, whose tails are the first to need it.
+//  K1 scan     persistent CTAs stream every cluster's centroid and value-sum
+//              rows once, in tiles of 64 rows brought in by 2-D tensor copies
+//              (one producer warp, a ring of slots, one mbarrier pair per
+//              slot).  Eight consumer warps take 8 rows each: the scores
+//              q . centroid / sqrt(d) of the group's heads (mma.sync, or
+//              packed FMA for fp32), the group-max selection key and its
+//              first radix digit, and ALL the clusters' estimation terms
+//              (item 3) folded into one running softmax part per warp.  The
+//              last CTA to finish a unit runs the unit's exact top-k (item
+//              2; Vortex 2.C Top-K) in its tail and writes the rows the
+//              gather reads.
+//  K2 gather   token-balanced CTAs gather the retrieved clusters' token rows
+//              and the steady rows through the block table and attend them
+//              exactly (items 1 and 2); the same pass takes back out of the
+//              estimate what the estimation zone does not hold (the
+//              retrieved clusters, the clusters left without a candidate
+//              token, and the steady tokens of the other affected clusters).
+//              The last CTA of each unit merges every part by log-sum-exp.
+//
+// The estimation zone is computed as "every cluster minus what the zone
+// leaves out": the same sum over clusters, streamed in the same pass as the
+// centroids instead of after the selection.  A cluster's estimated mass never
+// exceeds the exact mass of its own tokens (Jensen), and those tokens are in
+// the exact part, so the cancellation costs at most a few fp32 ulps of the
+// merged output's denominator.
+#include <cfloat>
+#include <climits>
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <type_traits>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "wi_common.cuh"
+#include "wi_plan.h"
+
+namespace wi {
+
+// ----------------------------------------------------------- chunk map
+// The scan's work: the clusters of every unit that is not attended densely,
+// in chunks of kTileRows; sequence b's units own ch_base[b + 1] - ch_base[b]
+// chunks (Hkv units of equal count).  Scan CTA s takes chunks
+// [s n / N, (s + 1) n / N).
+struct ChunkMap {
+  int32_t ch_base[kMaxBatch + 1];
+  int n_chunks, n_scan, batch, hkv;
+  __device__ __forceinline__ int k0(int s) const { return (int)((int64_t)s * n_chunks / n_scan); }
+  // the scan CTA that takes chunk k
+  __device__ __forceinline__ int cta_of(int k) const {
+    return (int)(((int64_t)(k + 1) * n_scan - 1) / n_chunks);
+  }
+  __device__ __forceinline__ int seq_of(int k) const {
+    int lo = 0, hi = batch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (ch_base[mid] <= k) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  }
+  __device__ __forceinline__ int per_unit(int b) const { return (ch_base[b + 1] - ch_base[b]) / hkv; }
+  __device__ __forceinline__ int first(int b, int h) const { return ch_base[b] + h * per_unit(b); }
+  // scan parts (CTAs) of unit (b, h): the CTAs of its first and last chunk and between
+  __device__ __forceinline__ int parts(int b, int h) const {
+    const int n = per_unit(b);
+    return n == 0 ? 0 : cta_of(first(b, h) + n - 1) - cta_of(first(b, h)) + 1;
+  }
+};
+
+namespace {
+
+constexpr int kHistShift = 21;    // first radix digit: key bits 31..21
+constexpr int kPartStride = 4;    // a softmax part of one head: {m, l, -, -, o[D]}
+
+// ------------------------------------------------------------------ tiles
+// A tile holds kTileRows rows of D elements as NB = D * sizeof(T) / 128
+// boxes of [kTileRows][128 bytes], each 128-byte swizzled: 16-byte chunk c
+// of row r sits at r * 128 + ((c ^ (r & 7)) << 4) of its box.  That is the
+// layout a SWIZZLE_128B tensor copy of a {128-byte, 64-row} box writes, and
+// the layout the gather's cp.async writes; ldmatrix reads it without bank
+// conflicts.
+template <typename T, int D>
+struct TileShape {
+  static constexpr int kRowBytes = D * (int)sizeof(T);
+  static constexpr int NB = kRowBytes / 128;
+  static constexpr int kBoxBytes = kTileRows * 128;
+  static constexpr int kBytes = NB * kBoxBytes;
+  static constexpr int kChunks = kRowBytes / 16;
+  static_assert(kRowBytes % 128 == 0, "rows of a multiple of 128 bytes");
+};
+
+// byte offset of 16-byte chunk c of row r in a tile
+__device__ __forceinline__ int tile_off(int r, int c) {
+  return (c >> 3) * (kTileRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+}
+
+// Multipliers of the 8 rows a warp takes in one step: the row's weight in the
+// numerator (wo) and in the denominator (wl); invalid rows take no part.
+struct RowMult {
+  float wo, wl;
+  int valid;
+};
+
+// ------------------------------------------------- warp softmax accumulators
+// One warp folds rows (a key row and a value row each, with multipliers wo
+// and wl) into a running softmax part of the G query heads:
+//   m = max score, l = sum wl e^(s - m), o = sum wo e^(s - m) value.
+// Scores s = q_g . key / sqrt(d).
+
+// bf16: tensor cores.  Scores on m16n8k16 (A = q, heads in rows 0..7; B = 8
+// key rows by ldmatrix); the weights' two bf16 terms (w = hi + lo to about
+// 2^-17) go in rows 0..7 and 8..15 of one m16n8k8 A operand, built in
+// registers from the score fragments; B = value rows by ldmatrix.trans.
+template <int D, int G>
+struct MmaAcc {
+  static_assert(G <= 8, "at most 8 query heads per KV head (MMA rows 0..7)");
+  uint32_t qa0[D / 16], qa2[D / 16];
+  float m, l;          // head lane / 4: running max, this lane's share of the sum
+  float o[D / 8][4];   // [n-tile][hi pair, lo pair] of output columns 8j + 2(lane % 4)
+
+  __device__ __forceinline__ void load_q(const __nv_bfloat16* q_group) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    const uint32_t* qw = reinterpret_cast<const uint32_t*>(q_group + (g < G ? g : 0) * D);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      qa0[ks] = g < G ? __ldg(qw + 8 * ks + tq) : 0u;
+      qa2[ks] = g < G ? __ldg(qw + 8 * ks + 4 + tq) : 0u;
+    }
+  }
+  __device__ __forceinline__ void reset() {
+    m = -INFINITY;
+    l = 0.f;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[j][e] = 0.f;
+  }
+  // scores of rows r0 + 2t, r0 + 2t + 1 (t = lane % 4) for head lane / 4
+  __device__ __forceinline__ void scores(const unsigned char* ktile, int r0, float scale,
+                                         float& s0, float& s1) const {
+    const int lane = threadIdx.x & 31;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ks += 2) {
+      uint32_t b[4];
+      ldsm_x4(b, ktile + tile_off(r0 + (lane & 7), 2 * ks + (lane >> 3)));
+      mma_bf16(acc, qa0[ks], qa2[ks], b[0], b[1]);
+      mma_bf16(acc, qa0[ks + 1], qa2[ks + 1], b[2], b[3]);
+    }
+    s0 = acc[0] * scale;
+    s1 = acc[1] * scale;
+  }
+  // fold the warp's 8 rows r0 .. r0 + 7: s0 / s1 their scores (as above),
+  // rm the rows' multipliers
+  __device__ __forceinline__ void fold(const unsigned char* vtile, int r0, float s0, float s1,
+                                       const RowMult* rm) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    const RowMult m0 = rm[2 * tq], m1 = rm[2 * tq + 1];
+    const float x0 = (g < G && m0.valid) ? s0 : -INFINITY;
+    const float x1 = (g < G && m1.valid) ? s1 : -INFINITY;
+    float mx = fmaxf(x0, x1);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float mnew = fmaxf(m, mx);
+    const float corr = mnew == -INFINITY ? 1.f : __expf(m - mnew);
+    const float p0 = x0 == -INFINITY ? 0.f : __expf(x0 - mnew);
+    const float p1 = x1 == -INFINITY ? 0.f : __expf(x1 - mnew);
+    l = l * corr + m0.wl * p0 + m1.wl * p1;
+    m = mnew;
+    uint32_t hi, lo;
+    split_bf16(m0.wo * p0, m1.wo * p1, hi, lo);
+#pragma unroll
+    for (int j = 0; j < D / 8; j += 4) {
+      uint32_t b[4];
+      ldsm_x4_t(b, vtile + tile_off(r0 + (lane & 7), j + (lane >> 3)));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[j + i][e] *= corr;
+        mma_bf16_k8(o[j + i], hi, lo, b[i]);
+      }
+    }
+  }
+  // this warp's part -> comb [G][D + 2] = {m, l, o[D]} per head
+  __device__ __forceinline__ void to_smem(float* comb) const {
+    const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    float ls = l;
+    ls += __shfl_xor_sync(0xffffffffu, ls, 1);
+    ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+    if (g < G) {
+      float* row = comb + g * (D + 2);
+#pragma unroll
+      for (int j = 0; j < D / 8; ++j)
+        *reinterpret_cast<float2*>(row + 2 + 8 * j + 2 * tq) =
+            make_float2(o[j][0] + o[j][2], o[j][1] + o[j][3]);
+      if (tq == 0) { row[0] = m; row[1] = ls; }
+    }
+  }
+};
+
+// fp32: packed FMA.  Lane l reads 16-byte chunk l % LPR of row l / LPR (+ RPW
+// per step); dot products are summed over the LPR lanes of a row.
+template <int D, int G>
+struct FmaAcc {
+  static constexpr int LPR = D / 4, RPW = 32 / LPR, NST = 8 / RPW;
+  static_assert(G <= LPR, "group larger than lanes per row");
+  float qv[G][4];
+  float m[G], l[G];
+  float o[G][4];
+
+  __device__ __forceinline__ void load_q(const float* q_group, float scale) {
+    const int sub = (threadIdx.x & 31) % LPR;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(q_group + g * D) + sub);
+      qv[g][0] = v.x * scale; qv[g][1] = v.y * scale; qv[g][2] = v.z * scale; qv[g][3] = v.w * scale;
+    }
+  }
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      m[g] = -INFINITY;
+      l[g] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[g][e] = 0.f;
+    }
+  }
+  __device__ __forceinline__ static float4 chunk(const unsigned char* tile, int r, int c) {
+    return *reinterpret_cast<const float4*>(tile + tile_off(r, c));
+  }
+  // scores of the warp's 8 rows into s [8][G] (shared memory of this warp)
+  __device__ __forceinline__ void scores(const unsigned char* ktile, int r0, float* s) const {
+    const int lane = threadIdx.x & 31, sub = lane % LPR, rs = lane / LPR;
+    const int j = sub / (LPR / G);
+#pragma unroll
+    for (int i = 0; i < NST; ++i) {
+      const int r = RPW * i + rs;
+      const float4 x = chunk(ktile, r0 + r, sub);
+      float a[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float2 t = __ffma2_rn(make_float2(qv[g][0], qv[g][1]), make_float2(x.x, x.y),
+                              make_float2(0.f, 0.f));
+        t = __ffma2_rn(make_float2(qv[g][2], qv[g][3]), make_float2(x.z, x.w), t);
+        a[g] = t.x + t.y;
+      }
+      group_reduce_multi<G, LPR>(a, lane);
+      if (sub % (LPR / G) == 0) s[r * G + j] = a[0];
+    }
+    __syncwarp();
+  }
+  __device__ __forceinline__ void fold(const unsigned char* vtile, int r0, const float* s,
+                                       const RowMult* rm) {
+    const int lane = threadIdx.x & 31, sub = lane % LPR, rs = lane / LPR;
+    float p[8][G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) mx = rm[r].valid ? fmaxf(mx, s[r * G + g]) : mx;
+      const float mnew = fmaxf(m[g], mx);
+      const float corr = mnew == -INFINITY ? 1.f : __expf(m[g] - mnew);
+      float ls = 0.f;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        p[r][g] = rm[r].valid ? __expf(s[r * G + g] - mnew) : 0.f;
+        ls += rm[r].wl * p[r][g];
+      }
+      l[g] = l[g] * corr + ls;
+      m[g] = mnew;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[g][e] *= corr;
+    }
+#pragma unroll
+    for (int i = 0; i < NST; ++i) {
+      const int r = RPW * i + rs;
+      const float4 x = chunk(vtile, r0 + r, sub);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float w = rm[r].wo * p[r][g];
+        float2 a = __ffma2_rn(make_float2(w, w), make_float2(x.x, x.y), make_float2(o[g][0], o[g][1]));
+        float2 b = __ffma2_rn(make_float2(w, w), make_float2(x.z, x.w), make_float2(o[g][2], o[g][3]));
+        o[g][0] = a.x; o[g][1] = a.y; o[g][2] = b.x; o[g][3] = b.y;
+      }
+    }
+    __syncwarp();
+  }
+  __device__ __forceinline__ void to_smem(float* comb) {
+    const int lane = threadIdx.x & 31, sub = lane % LPR, rs = lane / LPR;
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+#pragma unroll
+        for (int ofs = LPR; ofs < 32; ofs <<= 1) o[g][e] += __shfl_xor_sync(0xffffffffu, o[g][e], ofs);
+    if (rs == 0) {
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+        *reinterpret_cast<float4*>(comb + g * (D + 2) + 2 + 4 * sub) =
+            make_float4(o[g][0], o[g][1], o[g][2], o[g][3]);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) { comb[g * (D + 2)] = m[g]; comb[g * (D + 2) + 1] = l[g]; }
+    }
+  }
+};
+
+// Combine the per-warp parts comb [kConsumerWarps][G][D + 2] into one part
+// [G][D + 4] at `part` (threads 0 .. kConsumers - 1).
+template <int D, int G>
+__device__ __forceinline__ void combine_warps(const float* comb, float* part, int tid) {
+  for (int i = tid; i < G * D; i += kConsumers) {
+    const int g = i / D, e = i - g * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * G + g) * (D + 2)]);
+    float O = 0.f, L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float* row = comb + (w * G + g) * (D + 2);
+      const float f = row[0] == -INFINITY ? 0.f : __expf(row[0] - M);
+      O += f * row[2 + e];
+      L += f * row[1];
+    }
+    part[g * (D + kPartStride) + kPartStride + e] = O;
+    if (e == 0) { part[g * (D + kPartStride)] = M; part[g * (D + kPartStride) + 1] = L; }
+  }
+}
+
+// ------------------------------------------------------------- K0 steady
+struct SteadyArgs {
+  const int32_t* invperm;
+  const int32_t* labels;
+  const int32_t* offsets;
+  int n_sink, window, cap;
+  int32_t* info;     // [U][kInfoInts]
+  int32_t* st_slot;  // [U][cap] steady slots, ascending
+  int2* pc;          // [U][cap] (slot, cluster) of steady tokens of candidate clusters
+  int2* nonc;        // [U][cap] (cluster, count) of clusters without a non-steady token
+};
+
+__global__ void __launch_bounds__(256)
+wave_steady_kernel(const Geo geo, const SteadyArgs a, uint32_t* status) {
+  extern __shared__ __align__(16) unsigned long long srt[];   // [npow] sort keys
+  __shared__ int s_runs, s_nonc, s_pc;
+  pdl_launch_dependents();
+  const int u = blockIdx.x, b = u / geo.hkv, h = u - b * geo.hkv;
+  const int Tb = geo.T(b), NC = geo.NC(b);
+  const int ns = min(a.n_sink, Tb);
+  const int wstart = max(Tb - a.window, ns);
+  const int n_st = ns + (Tb - wstart);
+  const int tid = threadIdx.x, lane = tid & 31;
+  int32_t* I = a.info + (int64_t)u * kInfoInts;
+  if (n_st >= Tb) {   // all steady: attended densely, nothing retrieved or estimated
+    if (tid < kInfoInts) {
+      int v = 0;
+      if (tid == kSteady) v = Tb;
+      if (tid == kDense || tid == kNoEstimate) v = 1;
+      if (tid == kThrKey || tid == kThrIdx) v = -1;
+      I[tid] = v;
+    }
+    return;
+  }
+  int npow = 1;
+  while (npow < n_st) npow <<= 1;
+  const int32_t* inv = a.invperm + geo.tok_row(b, h);
+  const int32_t* lab = a.labels + geo.tok_row(b, h);
+  for (int i = tid; i < npow; i += blockDim.x) {
+    unsigned long long k = ~0ull;
+    if (i < n_st) {
+      const int pos = i < ns ? i : wstart + (i - ns);
+      int s = __ldg(inv + pos), c = __ldg(lab + pos);
+      if (s < 0 || s >= Tb) { flag_error(status, WI_DEV_BAD_SLOT); s = Tb; }
+      if (c < 0 || c >= NC) { flag_error(status, WI_DEV_BAD_CLUSTER); c = 0; }
+      k = ((unsigned long long)(uint32_t)s << 32) | (uint32_t)c;
+    }
+    srt[i] = k;
+  }
+  __syncthreads();
+  // bitonic sort by slot (clusters are slot ranges, so this groups them too)
+  for (int k = 2; k <= npow; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < npow; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const bool up = (i & k) == 0;
+          const unsigned long long x = srt[i], y = srt[ixj];
+          if ((x > y) == up) { srt[i] = y; srt[ixj] = x; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  int32_t* slots = a.st_slot + (int64_t)u * a.cap;
+  for (int i = tid; i < n_st; i += blockDim.x) slots[i] = (int32_t)(srt[i] >> 32);
+  // runs of one cluster (clusters are slot ranges, so a cluster's steady
+  // tokens are consecutive): a run's cluster is a candidate iff it keeps a
+  // non-steady member.  Each run's head marks its members (bit 31 of the
+  // key's cluster word, free since cluster ids are below 2^31).
+  const int32_t* off = a.offsets + geo.off_row(b, h);
+  auto cl_of = [&](int i) { return (int)(srt[i] & 0x7fffffffu); };
+  for (int i = tid; i < n_st; i += blockDim.x) {
+    const int c = cl_of(i);
+    if (i == 0 || cl_of(i - 1) != c) {
+      int e = i + 1;
+      while (e < n_st && cl_of(e) == c) ++e;
+      const int full = __ldg(off + c + 1) - __ldg(off + c);
+      if (full - (e - i) > 0)
+        for (int m = i; m < e; ++m) srt[m] |= 0x80000000ull;
+    }
+  }
+  __syncthreads();
+  // in order (warp 0): the non-candidates (cluster, count) and the steady
+  // tokens of candidate clusters (slot, cluster), which the gather takes out
+  // of the estimate unless their cluster is retrieved
+  int2* pc = a.pc + (int64_t)u * a.cap;
+  int2* nonc = a.nonc + (int64_t)u * a.cap;
+  if (tid < 32) {
+    const unsigned lt = (1u << lane) - 1u;
+    int n_runs = 0, n_nc = 0, n_pc = 0;
+    for (int base = 0; base < n_st; base += 32) {
+      const int i = base + lane;
+      const bool in = i < n_st;
+      const int c = in ? cl_of(i) : -1;
+      const bool head = in && (i == 0 || cl_of(i - 1) != c);
+      const bool cand = in && (srt[i] & 0x80000000ull) != 0ull;
+      const unsigned bh = __ballot_sync(0xffffffffu, head);
+      const unsigned bn = __ballot_sync(0xffffffffu, head && !cand);
+      const unsigned bp = __ballot_sync(0xffffffffu, cand);
+      if (head && !cand)
+        nonc[n_nc + __popc(bn & lt)] = make_int2(c, __ldg(off + c + 1) - __ldg(off + c));
+      if (cand) pc[n_pc + __popc(bp & lt)] = make_int2((int)(srt[i] >> 32), c);
+      n_runs += __popc(bh);
+      n_nc += __popc(bn);
+      n_pc += __popc(bp);
+    }
+    if (lane == 0) { s_runs = n_runs; s_nonc = n_nc; s_pc = n_pc; }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    I[kSteady] = n_st;
+    I[kAffected] = s_runs;
+    I[kDense] = 0;
+    I[kPartRows] = s_pc;
+    I[kNonCand] = s_nonc;
+  }
+}
+
+// --------------------------------------------------------------- K1 scan
+struct ScanArgs {
+  const void* q;
+  int Hq;
+  const int32_t* offsets;
+  uint2* rec;            // [ncl] {selection key (0: not a candidate), first slot}
+  int32_t* hist;         // [U][kHistBins] first-digit histogram (zero between calls)
+  int32_t* cnt1;         // [U] arrivals (zero between calls)
+  float* est;            // [U][p1max][G][D + 4] estimation parts
+  int p1max;
+  float* scores_out;     // optional [ncl][G]
+  float scale;
+  int exact_only;
+  // tail
+  int32_t* info;
+  const int2* nonc;
+  int32_t* sel;          // [ncl] retrieved ids (unit rows as the centroids)
+  int32_t* tok;          // [ntok] token slots of the retrieved clusters (unit rows as perm)
+  int2* full;            // [ncl + U cap] (cluster, count) whose estimate is taken back out
+  int cap;
+  int topk_clusters;
+  double topk_fraction;
+  int mode;
+  uint32_t seed;
+  int slots;
+};
+
+// Shared memory of a scan CTA (bytes, after 1024-byte alignment).
+template <typename T, int D, int G>
+struct ScanSmem {
+  using TS = TileShape<T, D>;
+  static constexpr size_t kComb = (size_t)kConsumerWarps * G * (D + 2) * 4;
+  static constexpr size_t kTail = (size_t)kHistBins * 4 + (size_t)kTailCand * 8 + 1024;
+  static constexpr size_t kUnion = kComb > kTail ? kComb : kTail;
+  static constexpr size_t kHist16 = (size_t)kHistBins / 2 * 4;
+  static constexpr size_t kRows = (size_t)kConsumerWarps * 8 * sizeof(RowMult);
+  static constexpr size_t kSc = (size_t)kConsumerWarps * 8 * G * 4;
+  __host__ __device__ static size_t slot_bytes(int exact_only) { return (size_t)TS::kBytes * (exact_only ? 1 : 2); }
+  __host__ __device__ static size_t total(int slots, int exact_only) {
+    return 1024 + slots * slot_bytes(exact_only) + kUnion + kHist16 + kRows + kSc;
+  }
+};
+
+// SplitMix64 (Steele, Lea and Flood 2014): the draw of the sampled selection.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Block-wide helpers over the kConsumers consumer threads (named barrier 1).
+__device__ __forceinline__ void csync() { named_sync(1, kConsumers); }
+
+// inclusive scan of x over the consumers; *total the sum.  sh: 32 ints.
+__device__ __forceinline__ int cscan(int x, int* sh, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[w] = x;
+  csync();
+  if (w == 0) {
+    int s = lane < kConsumerWarps ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < kConsumerWarps) sh[lane] = s;
+  }
+  csync();
+  const int r = x + (w > 0 ? sh[w - 1] : 0);
+  *total = sh[kConsumerWarps - 1];
+  csync();
+  return r;
+}
+
+// inclusive scan of two ints per consumer; *total the sums.  sh: 64 ints.
+__device__ __forceinline__ int2 cscan2(int2 x, int* sh, int2* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ya = __shfl_up_sync(0xffffffffu, x.x, o);
+    const int yb = __shfl_up_sync(0xffffffffu, x.y, o);
+    if (lane >= o) { x.x += ya; x.y += yb; }
+  }
+  if (lane == 31) { sh[w] = x.x; sh[32 + w] = x.y; }
+  csync();
+  if (w == 0) {
+    int a = lane < kConsumerWarps ? sh[lane] : 0, c = lane < kConsumerWarps ? sh[32 + lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ya = __shfl_up_sync(0xffffffffu, a, o);
+      const int yc = __shfl_up_sync(0xffffffffu, c, o);
+      if (lane >= o) { a += ya; c += yc; }
+    }
+    if (lane < kConsumerWarps) { sh[lane] = a; sh[32 + lane] = c; }
+  }
+  csync();
+  const int2 r = make_int2(x.x + (w > 0 ? sh[w - 1] : 0), x.y + (w > 0 ? sh[32 + w - 1] : 0));
+  *total = make_int2(sh[kConsumerWarps - 1], sh[32 + kConsumerWarps - 1]);
+  csync();
+  return r;
+}
+
+// Whether cluster c (selection key `key`, 0 for a non-candidate) is
+// retrieved, given the unit's threshold: exact mode, key > kstar or key ==
+// kstar and c <= thr; sampled mode, a key above the threshold bin, or in it
+// with (SplitMix64(seed 2^32 + c), c) <= (hstar, thr).
+struct Threshold {
+  uint32_t kstar;
+  int thr;
+  int sampled, bin1;
+  uint64_t hstar;
+  uint32_t seed;
+  __device__ __forceinline__ bool picked(uint32_t key, uint32_t c) const {
+    if (key == 0u) return false;
+    if (sampled) {
+      const int bn = (int)(key >> kHistShift);
+      if (bn != bin1) return bn > bin1;
+      const uint64_t d = splitmix64(((uint64_t)seed << 32) | (uint64_t)c);
+      return d < hstar || (d == hstar && (int)c <= thr);
+    }
+    return key > kstar || (key == kstar && (int)c <= thr);
+  }
+};
+
+// Bin of a histogram (bins scanned downwards) that holds the krem-th largest
+// element; *above: the count in the bins above it.  nb bins (<= 2048), each
+// consumer owns nb / kConsumers consecutive bins from the top.
+__device__ __forceinline__ int select_bin(const int* hist, int nb, int krem, int* above, int* sh,
+                                          int* s_ctl) {
+  const int tid = threadIdx.x;
+  const int per = nb / kConsumers;
+  int c[8], s = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = i < per ? hist[nb - 1 - per * tid - i] : 0;
+    s += c[i];
+  }
+  int tot;
+  const int incl = cscan(s, sh, &tot);
+  if (tid == 0) { s_ctl[0] = -1; s_ctl[1] = 0; }
+  csync();
+  int acc = incl - s;
+  if (acc < krem && incl >= krem) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i < per && acc + c[i] >= krem) { s_ctl[0] = nb - 1 - per * tid - i; s_ctl[1] = acc; break; }
+      acc += c[i];
+    }
+  }
+  csync();
+  *above = s_ctl[1];
+  const int r = s_ctl[0];
+  csync();
+  return r;
+}
+
+constexpr int kTailPT = 32;                    // records per consumer per round
+constexpr int kTailRound = kConsumers * kTailPT;
+
+// The tail of unit u (by the last scan CTA to finish it): the exact top-k
+// threshold (kstar, thr) -- cluster c is retrieved iff its key > kstar, or
+// key == kstar and c <= thr (lower id first on equal keys) -- or, in the
+// sampled mode, every key above the threshold bin plus the threshold bin's
+// members with the smallest (SplitMix64(seed 2^32 + c), c) draws; then the
+// retrieved ids, their token slots and the clusters whose estimate the
+// gather takes back out.
+__device__ void scan_tail(const Geo& geo, const ScanArgs& A, int u, unsigned char* sh,
+                          uint32_t* status) {
+  const int b = u / geo.hkv, h = u - b * geo.hkv;
+  const int NC = geo.NC(b), Tb = geo.T(b);
+  const int tid = threadIdx.x;
+  int* s_hist = reinterpret_cast<int*>(sh);                                   // [2048]
+  unsigned long long* s_cand = reinterpret_cast<unsigned long long*>(sh + kHistBins * 4);  // [kTailCand]
+  int* s_sh = reinterpret_cast<int*>(sh + kHistBins * 4 + kTailCand * 8);     // [64]
+  int* s_ctl = s_sh + 64;                                                     // [16]
+  const int64_t row0 = geo.cl_row(b, h);
+  uint2* rec = A.rec + row0;
+  int32_t* I = A.info + (int64_t)u * kInfoInts;
+  int32_t* hg = A.hist + (int64_t)u * kHistBins;
+
+  // round 0's records are loaded first, with the histogram
+  const int n_rounds = (NC + kTailRound - 1) / kTailRound;
+  uint32_t rk[kTailPT];
+  int32_t ro[kTailPT + 1];
+  int loaded = -1;
+  auto load_round = [&](int r) {
+    const int c0 = r * kTailRound + tid * kTailPT;
+#pragma unroll
+    for (int i = 0; i < kTailPT; ++i) {
+      const int c = c0 + i;
+      uint2 v = make_uint2(0u, (uint32_t)Tb);   // past the unit: no key, no tokens
+      if (c < NC) v = __ldcg(rec + c);
+      rk[i] = v.x;
+      ro[i] = (int32_t)v.y;
+    }
+    const int cn = c0 + kTailPT;
+    ro[kTailPT] = cn < NC ? (int32_t)__ldcg(&rec[cn].y) : Tb;
+    loaded = r;
+  };
+  pdl_wait();   // the steady kernel's lists
+  load_round(0);
+  for (int i = tid; i < kHistBins; i += kConsumers) {
+    s_hist[i] = __ldcg(hg + i);
+    hg[i] = 0;   // clean for the next call
+  }
+  const int n_nonc = __ldcg(I + kNonCand);
+  csync();
+  // the clusters left without a non-steady token leave the histogram, and
+  // their keys become 0 (not candidates) for everything that follows
+  const int2* nonc = A.nonc + (int64_t)u * A.cap;
+  for (int j = tid; j < n_nonc; j += kConsumers) {
+    const int c = __ldcg(&nonc[j].x);
+    if (c >= 0 && c < NC) {
+      const uint32_t key = __ldcg(&rec[c].x);
+      if (key) atomicSub(&s_hist[key >> kHistShift], 1);
+      rec[c].x = 0u;
+      // the round-0 registers of its owner are refreshed below
+    }
+  }
+  csync();
+  if (n_nonc > 0) load_round(0);   // see the zeroed keys
+  auto for_rounds = [&](auto&& body) {
+    for (int r = 0; r < n_rounds; ++r) {
+      if (loaded != r) load_round(r);
+      body(r);
+    }
+  };
+  // candidates: the nonzero keys, counted in one pass; the histogram must
+  // hold as many (a stale histogram, left by a failed call, is rebuilt from
+  // the keys)
+  int n_cand = 0, hist_total;
+  for_rounds([&](int) {
+    int s = 0;
+#pragma unroll
+    for (int i = 0; i < kTailPT; ++i) s += rk[i] != 0u;
+    int t;
+    cscan(s, s_sh, &t);
+    n_cand += t;
+  });
+  {
+    int s = 0;
+    for (int i = tid; i < kHistBins; i += kConsumers) s += s_hist[i];
+    cscan(s, s_sh, &hist_total);
+  }
+  if (hist_total != n_cand) {
+    if (tid == 0) flag_error(status, WI_DEV_BAD_HIST);
+    for (int i = tid; i < kHistBins; i += kConsumers) s_hist[i] = 0;
+    csync();
+    for_rounds([&](int) {
+#pragma unroll
+      for (int i = 0; i < kTailPT; ++i)
+        if (rk[i]) atomicAdd(&s_hist[rk[i] >> kHistShift], 1);
+    });
+    csync();
+  }
+  const int k_req = A.topk_clusters >= 0 ? A.topk_clusters
+                                         : (int)ceil(A.topk_fraction * (double)NC);
+  const int k = min(max(k_req, 0), n_cand);
+  uint32_t kstar = 0xFFFFFFFFu;   // nothing retrieved
+  int thr = -1;
+  int bin1 = -1;
+  uint64_t hstar = 0;
+  if (k == n_cand && k > 0) {
+    kstar = 1u;
+    thr = INT_MAX;
+  } else if (k > 0) {
+    int above;
+    bin1 = select_bin(s_hist, kHistBins, k, &above, s_sh, s_ctl);
+    int krem = k - above;
+    const int nb1 = s_hist[bin1];
+    // the threshold bin's members in id order: into shared memory when they
+    // fit; otherwise each refinement pass streams the keys again
+    const bool fits = nb1 <= kTailCand;
+    if (fits) {
+      int base = 0;
+      for_rounds([&](int r) {
+        int s = 0;
+#pragma unroll
+        for (int i = 0; i < kTailPT; ++i) s += rk[i] != 0u && (int)(rk[i] >> kHistShift) == bin1;
+        int t;
+        int pos = base + cscan(s, s_sh, &t) - s;
+#pragma unroll
+        for (int i = 0; i < kTailPT; ++i)
+          if (rk[i] != 0u && (int)(rk[i] >> kHistShift) == bin1) {
+            if (pos < kTailCand)
+              s_cand[pos] = ((unsigned long long)rk[i] << 32) |
+                            (uint32_t)(r * kTailRound + tid * kTailPT + i);
+            ++pos;
+          }
+        base += t;
+      });
+      csync();
+    }
+    if (A.mode == 1) {
+      // sampled: the krem members of the threshold bin with the smallest
+      // (draw, id); streamed or from shared memory, one rank pass
+      // (members are few: the bin holds the k-th key and is a 2^-9 wide
+      // slice of the key range)
+      auto draw = [&](uint32_t c) {
+        return splitmix64(((uint64_t)A.seed << 32) | (uint64_t)c);
+      };
+      if (tid == 0) { s_ctl[2] = -1; }
+      csync();
+      if (fits) {
+        for (int i = tid; i < nb1; i += kConsumers) {
+          const uint32_t ci = (uint32_t)s_cand[i];
+          const uint64_t di = draw(ci);
+          int rank = 0;
+          for (int j = 0; j < nb1; ++j) {
+            const uint32_t cj = (uint32_t)s_cand[j];
+            const uint64_t dj = draw(cj);
+            rank += dj < di || (dj == di && cj < ci);
+          }
+          if (rank == krem - 1) {
+            s_ctl[2] = (int)ci;
+            s_ctl[3] = (int)(uint32_t)(di >> 32);
+            s_ctl[4] = (int)(uint32_t)di;
+          }
+        }
+      } else {
+        // a crowded bin: the krem-th smallest draw by repeated counting is
+        // too slow; take the exact radix refinement of the draws instead:
+        // 64-bit draws ranked by an 11/11/11/11/10/10 digit radix select
+        uint64_t prefix = 0, pmask = 0;
+        int kr = krem;
+        const int shifts[6] = {53, 42, 31, 20, 10, 0};
+        const int bitsv[6] = {11, 11, 11, 11, 10, 10};
+        for (int pass = 0; pass < 6; ++pass) {
+          const int nb = 1 << bitsv[pass];
+          for (int i = tid; i < kHistBins; i += kConsumers) s_hist[i] = 0;
+          csync();
+          for_rounds([&](int r) {
+#pragma unroll
+            for (int i = 0; i < kTailPT; ++i) {
+              if (rk[i] != 0u && (int)(rk[i] >> kHistShift) == bin1) {
+                const uint64_t d = draw((uint32_t)(r * kTailRound + tid * kTailPT + i));
+                if ((d & pmask) == prefix)
+                  atomicAdd(&s_hist[(nb - 1) - (int)((d >> shifts[pass]) & (nb - 1))], 1);
+              }
+            }
+          });
+          csync();
+          // smallest draws first: the histogram is filled reversed so that
+          // select_bin's "largest" is the smallest digit
+          int ab;
+          const int dd = (nb - 1) - select_bin(s_hist, nb == 2048 ? 2048 : 1024, kr, &ab, s_sh, s_ctl);
+          kr -= ab;
+          prefix |= (uint64_t)dd << shifts[pass];
+          pmask |= (uint64_t)(nb - 1) << shifts[pass];
+        }
+        // the kr-th member (in id order) with draw == prefix
+        if (tid == 0) s_ctl[2] = -1;
+        csync();
+        int run = 0;
+        for_rounds([&](int r) {
+          int f = 0, first = -1;
+#pragma unroll
+          for (int i = 0; i < kTailPT; ++i) {
+            const uint32_t c = (uint32_t)(r * kTailRound + tid * kTailPT + i);
+            const bool m = rk[i] != 0u && (int)(rk[i] >> kHistShift) == bin1 && draw(c) == prefix;
+            if (m) { if (first < 0) first = (int)c; ++f; }
+          }
+          int t;
+          const int incl = cscan(f, s_sh, &t);
+          if (f > 0 && run + incl - f < kr && run + incl >= kr) s_ctl[2] = first;
+          run += t;
+        });
+        csync();
+        if (tid == 0) { s_ctl[3] = (int)(uint32_t)(prefix >> 32); s_ctl[4] = (int)(uint32_t)prefix; }
+      }
+      csync();
+      thr = s_ctl[2];
+      hstar = ((uint64_t)(uint32_t)s_ctl[3] << 32) | (uint32_t)s_ctl[4];
+      csync();
+    } else {
+      // exact: refine the threshold bin by the key's lower digits (bits
+      // 20..10, then 9..0), then take the krem-th largest key's ties by id
+      uint32_t prefix = (uint32_t)bin1 << kHistShift, pmask = 0xFFE00000u;
+      const int shifts[2] = {10, 0};
+      const int bitsv[2] = {11, 10};
+      for (int pass = 0; pass < 2; ++pass) {
+        const int nb = 1 << bitsv[pass];
+        for (int i = tid; i < kHistBins; i += kConsumers) s_hist[i] = 0;
+        csync();
+        if (fits) {
+          for (int i = tid; i < nb1; i += kConsumers) {
+            const uint32_t key = (uint32_t)(s_cand[i] >> 32);
+            if ((key & pmask) == prefix) atomicAdd(&s_hist[(key >> shifts[pass]) & (nb - 1)], 1);
+          }
+        } else {
+          for_rounds([&](int) {
+#pragma unroll
+            for (int i = 0; i < kTailPT; ++i)
+              if (rk[i] != 0u && (rk[i] & pmask) == prefix)
+                atomicAdd(&s_hist[(rk[i] >> shifts[pass]) & (nb - 1)], 1);
+          });
+        }
+        csync();
+        int ab;
+        const int dd = select_bin(s_hist, nb == 2048 ? 2048 : 1024, krem, &ab, s_sh, s_ctl);
+        krem -= ab;
+        prefix |= (uint32_t)dd << shifts[pass];
+        pmask |= (uint32_t)(nb - 1) << shifts[pass];
+      }
+      kstar = prefix;
+      // the krem-th member (ascending id) with key == kstar
+      if (tid == 0) s_ctl[2] = -1;
+      csync();
+      if (fits) {
+        for (int i0 = 0; i0 < nb1; i0 += kConsumers) {
+          const int i = i0 + tid;
+          const int f = i < nb1 && (uint32_t)(s_cand[i] >> 32) == kstar;
+          int t;
+          const int incl = cscan(f, s_sh, &t);
+          if (f && incl == krem) s_ctl[2] = (int)(uint32_t)s_cand[i];
+          krem -= t;
+          if (krem <= 0) break;
+        }
+      } else {
+        int run = 0;
+        for_rounds([&](int r) {
+          int f = 0;
+#pragma unroll
+          for (int i = 0; i < kTailPT; ++i) f += rk[i] == kstar;
+          int t;
+          const int incl = cscan(f, s_sh, &t);
+          if (f > 0 && run + incl - f < krem && run + incl >= krem) {
+            int need = krem - (run + incl - f);
+#pragma unroll
+            for (int i = 0; i < kTailPT; ++i)
+              if (rk[i] == kstar && --need == 0) s_ctl[2] = r * kTailRound + tid * kTailPT + i;
+          }
+          run += t;
+        });
+      }
+      csync();
+      thr = s_ctl[2];
+      csync();
+    }
+  }
+  // ---- emit, in id order: retrieved ids, their token slots, and the
+  // clusters taken back out of the estimate (retrieved, then the
+  // non-candidates), unless the estimation zone is empty
+  const bool sampled = A.mode == 1 && k > 0 && k < n_cand;
+  const Threshold th{kstar, thr, sampled ? 1 : 0, bin1, hstar, A.seed};
+  auto picked = [&](uint32_t key, uint32_t c) -> bool { return th.picked(key, c); };
+  const bool no_est = A.exact_only || k == n_cand;
+  int32_t* sel = A.sel + row0;
+  int32_t* tok = A.tok + geo.tok_row(b, h);
+  int2* full = A.full + row0 + (int64_t)u * A.cap;
+  int n_sel = 0, n_tok = 0;
+  if (k > 0) {
+    for_rounds([&](int r) {
+      const int c0 = r * kTailRound + tid * kTailPT;
+      int s = 0, t = 0;
+#pragma unroll
+      for (int i = 0; i < kTailPT; ++i)
+        if (picked(rk[i], (uint32_t)(c0 + i))) { ++s; t += ro[i + 1] - ro[i]; }
+      int2 tot2;
+      const int2 inc = cscan2(make_int2(s, t), s_sh, &tot2);
+      int ps = n_sel + inc.x - s, pt = n_tok + inc.y - t;
+#pragma unroll
+      for (int i = 0; i < kTailPT; ++i) {
+        if (picked(rk[i], (uint32_t)(c0 + i))) {
+          const int cnt = ro[i + 1] - ro[i];
+          sel[ps] = c0 + i;
+          if (!no_est) full[ps] = make_int2(c0 + i, cnt);
+          ++ps;
+          for (int j = 0; j < cnt; ++j) tok[pt + j] = ro[i] + j;
+          pt += cnt;
+        }
+      }
+      n_sel += tot2.x;
+      n_tok += tot2.y;
+    });
+  }
+  int n_full = 0;
+  if (!no_est) {
+    for (int j = tid; j < n_nonc; j += kConsumers) full[n_sel + j] = __ldcg(&nonc[j]);
+    n_full = n_sel + n_nonc;
+  }
+  if (tid == 0) {
+    I[kSelCount] = n_sel;
+    I[kThrKey] = (int32_t)kstar;
+    I[kThrIdx] = thr;
+    I[kSelTokens] = n_tok;
+    I[kCandidates] = n_cand;
+    I[kFullRows] = n_full;
+    I[kNoEstimate] = no_est ? 1 : 0;
+    I[kMode] = sampled ? 1 : 0;
+    I[kSampBin] = bin1;
+    I[kSampHash] = (int32_t)(uint32_t)(hstar >> 32);
+    I[kSampHashLo] = (int32_t)(uint32_t)hstar;
+    A.cnt1[u] = 0;   // clean for the next call
+  }
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kScanThreads, 1)
+wave_scan_kernel(const Geo geo, const ChunkMap cm, const ScanArgs A,
+                 const __grid_constant__ CUtensorMap tm_cent,
+                 const __grid_constant__ CUtensorMap tm_vsum, uint32_t* status) {
+  using TS = TileShape<T, D>;
+  using SM = ScanSmem<T, D, G>;
+  constexpr bool kMma = std::is_same_v<T, __nv_bfloat16>;
+  constexpr int kBoxCols = 128 / (int)sizeof(T);
+  extern __shared__ __align__(16) unsigned char sh_raw[];
+  __shared__ __align__(8) uint64_t s_full[4], s_empty[4];
+  __shared__ int s_last, s_ntails;
+  __shared__ int s_tails[kMaxTailsPerCta];   // units whose last arrival was this CTA's
+  pdl_launch_dependents();
+  unsigned char* sh = align_smem_1024(sh_raw);
+  const int slots = A.slots;
+  const size_t slot_bytes = SM::slot_bytes(A.exact_only);
+  unsigned char* ring = sh;
+  unsigned char* s_union = ring + slots * slot_bytes;
+  uint32_t* hist16 = reinterpret_cast<uint32_t*>(s_union + SM::kUnion);
+  RowMult* s_rows = reinterpret_cast<RowMult*>(reinterpret_cast<unsigned char*>(hist16) + SM::kHist16);
+  float* s_sc = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(s_rows) + SM::kRows);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int s = blockIdx.x;
+  const int k0 = cm.n_chunks > 0 ? cm.k0(s) : 0, k1 = cm.n_chunks > 0 ? cm.k0(s + 1) : 0;
+  const int nk = k1 - k0;
+  struct Chunk { int u, b, h, c0, nrows; int64_t row0; };
+  auto chunk = [&](int k) -> Chunk {
+    Chunk c;
+    c.b = cm.seq_of(k);
+    const int per = cm.per_unit(c.b);
+    const int rel = k - cm.ch_base[c.b];
+    c.h = rel / per;
+    c.c0 = (rel - c.h * per) * kTileRows;
+    c.u = c.b * geo.hkv + c.h;
+    c.nrows = min(kTileRows, geo.NC(c.b) - c.c0);
+    c.row0 = geo.cl_row(c.b, c.h);
+    return c;
+  };
+  if (tid == 0) {
+    for (int i = 0; i < slots; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], kConsumerWarps); }
+    mbar_init_fence();
+  }
+  for (int i = tid; i < kHistBins / 2; i += blockDim.x) hist16[i] = 0u;
+  if (tid == 0) s_ntails = 0;
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ---- producer: chunk i into slot i % slots once the slot is free
+    if (lane == 0) {
+      const uint32_t bytes = (uint32_t)slot_bytes;
+      for (int i = 0; i < nk; ++i) {
+        const int sl = i % slots;
+        if (i >= slots) mbar_wait(&s_empty[sl], (uint32_t)((i / slots - 1) & 1), status);
+        const Chunk c = chunk(k0 + i);
+        const int y = (int)(c.row0 + c.c0);
+        unsigned char* dst = ring + sl * slot_bytes;
+        mbar_arrive_expect(&s_full[sl], bytes);
+#pragma unroll
+        for (int nb = 0; nb < TS::NB; ++nb)
+          tensor_load_2d(dst + nb * TS::kBoxBytes, &tm_cent, nb * kBoxCols, y, &s_full[sl]);
+        if (!A.exact_only) {
+#pragma unroll
+          for (int nb = 0; nb < TS::NB; ++nb)
+            tensor_load_2d(dst + TS::kBytes + nb * TS::kBoxBytes, &tm_vsum, nb * kBoxCols, y,
+                           &s_full[sl]);
+        }
+      }
+      // every copy issued has landed before the CTA may leave (bounded)
+      for (int i = max(0, nk - slots); i < nk; ++i)
+        mbar_wait(&s_full[i % slots], (uint32_t)((i / slots) & 1), status);
+    }
+    pdl_wait();
+    return;
+  }
+
+  // ---- consumers
+  MmaAcc<D, G> macc;
+  FmaAcc<D, G> facc;
+  const int g = lane >> 2, tq = lane & 3;
+  // offsets of the warp's rows, prefetched two chunks ahead: lane l <= 8
+  // holds offsets[c0 + 8 warp + l] of its unit
+  auto load_off = [&](int i) -> int {
+    if (i >= nk || lane > 8) return 0;
+    const Chunk c = chunk(k0 + i);
+    const int cl = c.c0 + 8 * warp + lane;
+    if (cl > geo.NC(c.b)) return 0;
+    return __ldg(A.offsets + geo.off_row(c.b, c.h) + cl);
+  };
+  int off_cur = load_off(0), off_n1 = load_off(1), off_n2 = load_off(2);
+  int cur_u = -1;
+  int since_flush = 0;
+  float* comb = reinterpret_cast<float*>(s_union);
+  RowMult* rm = s_rows + warp * 8;
+  float* sc = s_sc + warp * 8 * G;
+  for (int i = 0; i < nk; ++i) {
+    const Chunk c = chunk(k0 + i);
+    if (c.u != cur_u) {
+      const T* qg = reinterpret_cast<const T*>(A.q) + ((int64_t)c.b * A.Hq + (int64_t)c.h * G) * D;
+      if constexpr (kMma) { macc.load_q(qg); macc.reset(); }
+      else { facc.load_q(qg, A.scale); facc.reset(); }
+      cur_u = c.u;
+    }
+    const int sl = i % slots;
+    const unsigned char* ktile = ring + sl * slot_bytes;
+    const unsigned char* vtile = ktile + TS::kBytes;
+    // rows 8 warp .. 8 warp + 7: counts and first slots from the offsets
+    const int r0 = 8 * warp;
+    __syncwarp();   // the previous chunk's row data is read
+    {
+      const int o_next = __shfl_down_sync(0xffffffffu, off_cur, 1);
+      if (lane < 8) {
+        const int cl = c.c0 + r0 + lane;
+        const int cnt = o_next - off_cur;
+        const bool ok = cl < c.c0 + c.nrows && cnt > 0;
+        rm[lane] = RowMult{1.f, (float)cnt, ok ? 1 : 0};
+      }
+      __syncwarp();
+    }
+    mbar_wait(&s_full[sl], (uint32_t)((i / slots) & 1), status);
+    // scores, keys, histogram, estimation
+    float key_s[2] = {-INFINITY, -INFINITY};   // group max of rows 2tq, 2tq+1 (MMA) / lane's row (FMA)
+    if constexpr (kMma) {
+      float s0, s1;
+      macc.scores(ktile, r0, A.scale, s0, s1);
+      if (A.scores_out && g < G) {
+        const int cl = c.c0 + r0 + 2 * tq;
+        if (cl < c.c0 + c.nrows) A.scores_out[(c.row0 + cl) * G + g] = s0;
+        if (cl + 1 < c.c0 + c.nrows) A.scores_out[(c.row0 + cl + 1) * G + g] = s1;
+      }
+      float m0 = g < G ? s0 : -INFINITY, m1 = g < G ? s1 : -INFINITY;
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+      }
+      key_s[0] = m0;
+      key_s[1] = m1;
+      if (!A.exact_only) macc.fold(vtile, r0, s0, s1, rm);
+    } else {
+      facc.scores(ktile, r0, sc);
+      if (lane < 8) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg) mx = fmaxf(mx, sc[lane * G + gg]);
+        key_s[0] = mx;
+        if (A.scores_out) {
+          const int cl = c.c0 + r0 + lane;
+          if (cl < c.c0 + c.nrows)
+            for (int gg = 0; gg < G; ++gg) A.scores_out[(c.row0 + cl) * G + gg] = sc[lane * G + gg];
+        }
+      }
+      if (!A.exact_only) facc.fold(vtile, r0, sc, rm);
+    }
+    // the slot's last reads are done: release it to the producer
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s_empty[sl]);
+    // keys and the first digit's histogram: MMA lanes 0..3 hold rows 2t and
+    // 2t + 1 (t = lane), FMA lanes 0..7 row lane; each writes the record
+    // {key, first slot} of its rows
+    {
+      const int ra = kMma ? 2 * tq : (lane & 7);
+      const int oa = __shfl_sync(0xffffffffu, off_cur, ra);
+      const int ob = __shfl_sync(0xffffffffu, off_cur, (ra + 1) & 31);
+      const int nkeys = kMma ? (lane < 4 ? 2 : 0) : (lane < 8 ? 1 : 0);
+#pragma unroll
+      for (int kx = 0; kx < 2; ++kx) {
+        if (kx >= nkeys) break;
+        const int r = ra + kx;
+        const int cl = c.c0 + r0 + r;
+        if (cl < c.c0 + c.nrows) {
+          const uint32_t key = rm[r].valid ? ordered_key(key_s[kx]) : 0u;
+          A.rec[c.row0 + cl] = make_uint2(key, (uint32_t)(kx ? ob : oa));
+          if (key) atomicAdd(&hist16[key >> (kHistShift + 1)], 1u << (16 * ((key >> kHistShift) & 1u)));
+        }
+      }
+    }
+    off_cur = off_n1;
+    off_n1 = off_n2;
+    off_n2 = load_off(i + 3);
+    since_flush += kTileRows;
+    // ---- end of the CTA's part of a unit: part, histogram, arrival, tail
+    const bool unit_end = i == nk - 1 || chunk(k0 + i + 1).u != c.u;
+    if (unit_end || since_flush >= 65536 - kTileRows) {
+      csync();
+      int32_t* hg = A.hist + (int64_t)c.u * kHistBins;
+      for (int w = tid; w < kHistBins / 2; w += kConsumers) {
+        const uint32_t v = hist16[w];
+        if (v) {
+          if (v & 0xffffu) atomicAdd(hg + 2 * w, (int)(v & 0xffffu));
+          if (v >> 16) atomicAdd(hg + 2 * w + 1, (int)(v >> 16));
+          hist16[w] = 0u;
+        }
+      }
+      since_flush = 0;
+      csync();   // the words are clear before the next chunk counts into them
+    }
+    if (unit_end) {
+      if (!A.exact_only) {
+        if constexpr (kMma) macc.to_smem(comb + warp * G * (D + 2));
+        else facc.to_smem(comb + warp * G * (D + 2));
+        csync();
+        const int slot = s - cm.cta_of(cm.first(c.b, c.h));
+        float* part = A.est + ((int64_t)c.u * A.p1max + slot) * G * (D + kPartStride);
+        combine_warps<D, G>(comb, part, tid);
+      }
+      __threadfence();
+      csync();
+      if (tid == 0) {
+        const int old = atomicAdd(A.cnt1 + c.u, 1);
+        __threadfence();
+        s_last = old == cm.parts(c.b, c.h) - 1;
+      }
+      csync();
+      if (s_last && tid == 0) s_tails[s_ntails++] = c.u;
+    }
+  }
+  // ---- the tails of the units this CTA finished last (after the loop, so
+  // the accumulators are dead and the tail has the registers)
+  csync();
+  const int nt = s_ntails;
+  for (int t = 0; t < nt; ++t) {
+    scan_tail(geo, A, s_tails[t], s_union, status);
+    csync();
+  }
+  pdl_wait();
+}
+
+// ------------------------------------------------------------- K2 gather
+struct GatherArgs {
+  const void* q;
+  int Hq;
+  Pool kp, vp;
+  const void* centroids;
+  const void* value_sums;
+  const int32_t* perm;
+  const uint2* rec;
+  const int32_t* info;
+  const int32_t* st_slot;
+  const int2* pc;
+  const int32_t* tok;
+  const int2* full;
+  int cap;
+  int n_sink, window;
+  float* est;
+  int p1max;
+  float* gat;            // [U][n2max][G][D + 4]
+  int n2max;
+  int32_t* cnt2;         // [U] arrivals (zero between calls)
+  float* out;
+  float* lse;
+  float scale;
+  uint32_t seed;
+  int32_t n2_base[kMaxBatch + 1];
+};
+
+enum RowKind { kRowNone = 0, kRowToken = 1, kRowSteady = 2, kRowFull = 3, kRowPart = 4 };
+
+template <typename T, int D, int G>
+struct GatherSmem {
+  using TS = TileShape<T, D>;
+  static constexpr int kRowsPerBlock = kGatherTiles * kTileRows;
+  static constexpr size_t kTiles = (size_t)2 * kGatherTiles * TS::kBytes;   // K and V
+  static constexpr size_t kMeta = (size_t)kRowsPerBlock * (8 + 8 + 4 + 4);
+  static constexpr size_t kComb = (size_t)kConsumerWarps * G * (D + 2) * 4;
+  static constexpr size_t kRows = (size_t)kConsumerWarps * 8 * sizeof(RowMult);
+  static constexpr size_t kSc = (size_t)kConsumerWarps * 8 * G * 4;
+  static constexpr size_t kMergeParts = 256;   // parts whose (m, l) are staged per pass
+  static constexpr size_t kMerge = kMergeParts * G * 2 * 4 + (size_t)G * 8;
+  static constexpr size_t kTotal = 1024 + kTiles + kMeta + kComb + kRows + kSc + kMerge;
+};
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kGatherThreads, 2)
+wave_gather_kernel(const Geo geo, const ChunkMap cm, const GatherArgs A, uint32_t* status) {
+  using TS = TileShape<T, D>;
+  using SM = GatherSmem<T, D, G>;
+  constexpr bool kMma = std::is_same_v<T, __nv_bfloat16>;
+  constexpr int RPB = SM::kRowsPerBlock;
+  extern __shared__ __align__(16) unsigned char sh_raw[];
+  __shared__ int s_rec[kInfoInts];
+  __shared__ int s_last;
+  unsigned char* sh = align_smem_1024(sh_raw);
+  unsigned char* tiles = sh;                                   // [K t0][K t1][V t0][V t1]
+  const unsigned char** s_kp = reinterpret_cast<const unsigned char**>(tiles + SM::kTiles);
+  const unsigned char** s_vp = s_kp + RPB;
+  int* s_kind = reinterpret_cast<int*>(s_vp + RPB);
+  int* s_aux = s_kind + RPB;
+  float* comb = reinterpret_cast<float*>(s_aux + RPB);
+  RowMult* s_rows = reinterpret_cast<RowMult*>(reinterpret_cast<unsigned char*>(comb) + SM::kComb);
+  float* s_sc = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(s_rows) + SM::kRows);
+  float* s_merge = s_sc + kConsumerWarps * 8 * G;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // CTA -> (sequence b, KV head h, index j of the unit's n2 CTAs)
+  int b = 0;
+  {
+    int lo = 0, hi = geo.batch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (A.n2_base[mid] <= (int)blockIdx.x) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+  }
+  const int n2 = (A.n2_base[b + 1] - A.n2_base[b]) / geo.hkv;
+  const int rel = (int)blockIdx.x - A.n2_base[b];
+  const int h = rel / n2, j = rel - h * n2;
+  const int u = b * geo.hkv + h;
+  const int Tb = geo.T(b);
+  const int ns = min(A.n_sink, Tb), wstart = max(Tb - A.window, ns);
+  const int64_t row0 = geo.cl_row(b, h), trow = geo.tok_row(b, h);
+  const T* qg = reinterpret_cast<const T*>(A.q) + ((int64_t)b * A.Hq + (int64_t)h * G) * D;
+  MmaAcc<D, G> macc;
+  FmaAcc<D, G> facc;
+  if constexpr (kMma) { macc.load_q(qg); macc.reset(); }
+  else { facc.load_q(qg, A.scale); facc.reset(); }
+
+  pdl_wait();   // the scan's and the steady kernel's results
+  // the unit's record, and (speculatively) the token slots of the first block
+  if (tid < kInfoInts) s_rec[tid] = __ldcg(A.info + (int64_t)u * kInfoInts + tid);
+  int spec = -1;
+  if (tid < RPB && j * RPB + tid < Tb) spec = __ldcg(A.tok + trow + j * RPB + tid);
+  __syncthreads();
+  const bool dense = s_rec[kDense] != 0, no_est = s_rec[kNoEstimate] != 0;
+  const int n_tok = dense ? 0 : s_rec[kSelTokens];
+  const int n_st = s_rec[kSteady];
+  const int n_full = (dense || no_est) ? 0 : s_rec[kFullRows];
+  const int n_pc = (dense || no_est) ? 0 : s_rec[kPartRows];
+  const int R = n_tok + n_st + n_full + n_pc;
+  const Threshold th{(uint32_t)s_rec[kThrKey], s_rec[kThrIdx], s_rec[kMode], s_rec[kSampBin],
+                     ((uint64_t)(uint32_t)s_rec[kSampHash] << 32) | (uint32_t)s_rec[kSampHashLo],
+                     A.seed};
+  const unsigned char* kpool = reinterpret_cast<const unsigned char*>(A.kp.base);
+  const unsigned char* vpool = reinterpret_cast<const unsigned char*>(A.vp.base);
+  const unsigned char* cent = reinterpret_cast<const unsigned char*>(A.centroids);
+  const unsigned char* vsum = reinterpret_cast<const unsigned char*>(A.value_sums);
+  constexpr int RB = TS::kRowBytes;
+
+  for (int blk = j; blk * RPB < R; blk += n2) {
+    const int rb = blk * RPB;
+    // ---- resolve the block's rows: kind, key and value row addresses
+    if (tid < RPB) {
+      const int r = rb + tid;
+      int kind = kRowNone, aux = 0;
+      const unsigned char* kr = nullptr;
+      const unsigned char* vr = nullptr;
+      int slot = -1, c = -1;
+      if (r < R) {
+        if (dense) {
+          slot = r; kind = kRowSteady;
+        } else if (r < n_tok) {
+          slot = blk == j ? spec : __ldcg(A.tok + trow + r);
+          kind = kRowToken;
+        } else if (r < n_tok + n_st) {
+          slot = __ldcg(A.st_slot + (int64_t)u * A.cap + (r - n_tok));
+          kind = kRowSteady;
+        } else if (r < n_tok + n_st + n_full) {
+          const int2 f = __ldcg(A.full + row0 + (int64_t)u * A.cap + (r - n_tok - n_st));
+          c = f.x; aux = f.y; kind = kRowFull;
+        } else {
+          const int2 p = __ldcg(A.pc + (int64_t)u * A.cap + (r - n_tok - n_st - n_full));
+          slot = p.x; c = p.y; kind = kRowPart;
+        }
+      }
+      if (kind == kRowFull || kind == kRowPart) {
+        if (c < 0 || c >= geo.NC(b)) { flag_error(status, WI_DEV_BAD_CLUSTER); kind = kRowNone; }
+        else kr = cent + (row0 + c) * RB;
+      }
+      if (kind == kRowFull) vr = vsum + (row0 + c) * RB;
+      if (kind == kRowToken || kind == kRowSteady || kind == kRowPart) {
+        const int64_t ro = pool_row(A.kp, geo.hkv, D, b, h, slot, status);
+        if (ro < 0) {
+          kind = kRowNone;
+        } else {
+          if (kind != kRowPart) kr = kpool + ro * (int64_t)sizeof(T);
+          vr = vpool + ro * (int64_t)sizeof(T);
+          if (kind == kRowToken) {
+            if (slot >= Tb) { flag_error(status, WI_DEV_BAD_SLOT); kind = kRowNone; }
+            else aux = __ldg(A.perm + trow + slot);
+          } else if (kind == kRowPart) {
+            aux = (int)__ldcg(&A.rec[row0 + c].x);
+          }
+        }
+      }
+      s_kind[tid] = kind;
+      s_aux[tid] = aux;
+      s_kp[tid] = kind == kRowNone ? nullptr : kr;
+      s_vp[tid] = kind == kRowNone ? nullptr : vr;
+      // a partial row's cluster is taken out of the estimate only when it
+      // is not retrieved
+      if (kind == kRowPart) s_aux[tid] = th.picked((uint32_t)aux, (uint32_t)c) ? 1 : 0;
+    }
+    __syncthreads();
+    // ---- gather: every 16-byte chunk of the block's key and value rows
+    for (int x = tid; x < RPB * TS::kChunks * 2; x += blockDim.x) {
+      const int mat = x / (RPB * TS::kChunks);
+      const int rr = (x - mat * RPB * TS::kChunks) / TS::kChunks;
+      const int ch = x - mat * RPB * TS::kChunks - rr * TS::kChunks;
+      const unsigned char* src = mat == 0 ? s_kp[rr] : s_vp[rr];
+      unsigned char* dst = tiles + (size_t)(mat * kGatherTiles + rr / kTileRows) * TS::kBytes +
+                           tile_off(rr % kTileRows, ch);
+      if (src) cp_async16(dst, src + ch * 16);
+      else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    // ---- attend: warp w takes rows 8w .. 8w + 7 of each tile
+#pragma unroll
+    for (int t = 0; t < kGatherTiles; ++t) {
+      const int lr = t * kTileRows + 8 * warp;    // block-local row of the warp's first
+      RowMult* rm = s_rows + warp * 8;
+      if (lane < 8) {
+        const int q = lr + lane;
+        const int kind = s_kind[q];
+        RowMult m{0.f, 0.f, 0};
+        if (kind == kRowToken) {
+          const int pos = s_aux[q];
+          const bool st = pos < ns || pos >= wstart;
+          m = st ? RowMult{0.f, 0.f, 0} : RowMult{1.f, 1.f, 1};
+        } else if (kind == kRowSteady) {
+          m = RowMult{1.f, 1.f, 1};
+        } else if (kind == kRowFull) {
+          m = RowMult{-1.f, -(float)s_aux[q], 1};
+        } else if (kind == kRowPart) {
+          m = s_aux[q] ? RowMult{0.f, 0.f, 0} : RowMult{-1.f, -1.f, 1};
+        }
+        rm[lane] = m;
+      }
+      __syncwarp();
+      const unsigned char* kt = tiles + (size_t)t * TS::kBytes;
+      const unsigned char* vt = tiles + (size_t)(kGatherTiles + t) * TS::kBytes;
+      if constexpr (kMma) {
+        float s0, s1;
+        macc.scores(kt, 8 * warp, A.scale, s0, s1);
+        macc.fold(vt, 8 * warp, s0, s1, rm);
+      } else {
+        float* sc = s_sc + warp * 8 * G;
+        facc.scores(kt, 8 * warp, sc);
+        facc.fold(vt, 8 * warp, sc, rm);
+      }
+      __syncwarp();
+    }
+    __syncthreads();   // tiles and row data are read before the next block
+  }
+  // ---- this CTA's part, then the unit's merge by its last CTA
+  if constexpr (kMma) macc.to_smem(comb + warp * G * (D + 2));
+  else facc.to_smem(comb + warp * G * (D + 2));
+  __syncthreads();
+  float* part = A.gat + ((int64_t)u * A.n2max + j) * G * (D + kPartStride);
+  combine_warps<D, G>(comb, part, tid);
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int old = atomicAdd(A.cnt2 + u, 1);
+    __threadfence();
+    s_last = old == n2 - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  // parts: the scan's (unless the estimation zone is empty), then the gather's
+  const int np1 = no_est ? 0 : cm.parts(b, h);
+  const int np = np1 + n2;
+  auto part_ptr = [&](int p) -> const float* {
+    return p < np1 ? A.est + ((int64_t)u * A.p1max + p) * G * (D + kPartStride)
+                   : A.gat + ((int64_t)u * A.n2max + (p - np1)) * G * (D + kPartStride);
+  };
+  float* s_f = s_merge;                             // [kMergeParts][G] (m, l) then factor
+  float* s_M = s_merge + SM::kMergeParts * G * 2;   // [G] max, [G] denominator
+  float* s_L = s_M + G;
+  for (int x = tid; x < np * G; x += blockDim.x) {
+    const int p = x / G, gg = x - p * G;
+    const float* pp = part_ptr(p) + gg * (D + kPartStride);
+    s_f[2 * x] = __ldcg(pp);
+    s_f[2 * x + 1] = __ldcg(pp + 1);
+  }
+  __syncthreads();
+  if (warp < G) {   // warp g: head g's max, the parts' factors, the denominator
+    float M = -INFINITY;
+    for (int p = lane; p < np; p += 32) M = fmaxf(M, s_f[2 * (p * G + warp)]);
+    M = warp_max(M);
+    float L = 0.f;
+    for (int p = lane; p < np; p += 32) {
+      const float mp = s_f[2 * (p * G + warp)];
+      const float f = mp == -INFINITY ? 0.f : expf(mp - M);
+      L += f * s_f[2 * (p * G + warp) + 1];
+      s_f[2 * (p * G + warp)] = f;
+    }
+    L = warp_sum(L);
+    if (lane == 0) { s_M[warp] = M; s_L[warp] = L; }
+  }
+  __syncthreads();
+  for (int i = tid; i < G * D; i += blockDim.x) {
+    const int gg = i / D, e = i - gg * D;
+    float O = 0.f;
+    for (int p = 0; p < np; ++p) {
+      const float f = s_f[2 * (p * G + gg)];
+      if (f != 0.f) O += f * __ldcg(part_ptr(p) + gg * (D + kPartStride) + kPartStride + e);
+    }
+    const float L = s_L[gg];
+    const int64_t qh = (int64_t)b * A.Hq + (int64_t)h * G + gg;
+    A.out[qh * D + e] = L > 0.f ? O / L : 0.f;
+    if (e == 0 && A.lse) A.lse[qh] = L > 0.f ? s_M[gg] + logf(L) : -INFINITY;
+  }
+  if (tid == 0) A.cnt2[u] = 0;   // clean for the next call
+}
+
+}  // namespace
+}  // namespace wi
+
+
+namespace wi {
+namespace {
+
+template <typename Kern, typename... Args>
+cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                      Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library); null when unavailable
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// rows x D matrix of bf16 or fp32, boxes of 64 rows x 128 bytes, 128-byte swizzle
+bool encode_rows(CUtensorMap* tm, const void* base, int64_t rows, int D, int dtype) {
+  auto fn = encode_fn();
+  if (!fn || rows <= 0) return false;
+  const int es = dtype == WI_BF16 ? 2 : 4;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * es};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / es), (cuuint32_t)kTileRows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(tm, dtype == WI_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+            2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Dynamic shared memory limit, and the full shared-memory carveout for every
+// decode kernel (kernels that overlap under programmatic dependent launch
+// then never need the SM's L1 / shared split reconfigured between them).
+template <typename Kern>
+void set_smem(Kern kern, size_t bytes) {
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                       (int)cudaSharedmemCarveoutMaxShared);
+}
+
+int pow2_at_least(int n) {
+  int p = 1;
+  while (p < n) p <<= 1;
+  return p;
+}
+
+}  // namespace
+
+// K1 and K2 of one decode for key type T, head size D and group size G (the
+// steady kernel, which does not depend on them, is launched by the caller).
+template <typename T, int D, int G>
+cudaError_t launch_decode_typed(const DecodePlan& p, const DecodeArgs& a, const ChunkMap& cm,
+                                cudaStream_t s) {
+  unsigned char* ws = a.ws;
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + p.off_status);
+  cudaEvent_t* ev = a.stage_events;
+  const bool pdl = ev == nullptr;
+  auto mark = [&](int i) { if (ev) cudaEventRecord(ev[i], s); };
+  int32_t* info = reinterpret_cast<int32_t*>(ws + p.off_info);
+  int32_t* st_slot = reinterpret_cast<int32_t*>(ws + p.off_st_slot);
+  int2* pc = reinterpret_cast<int2*>(ws + p.off_pc);
+  int2* nonc = reinterpret_cast<int2*>(ws + p.off_nonc);
+  // K1: scan + tails
+  CUtensorMap tmc, tmv;
+  std::memset(&tmc, 0, sizeof(tmc));
+  std::memset(&tmv, 0, sizeof(tmv));
+  if (!encode_rows(&tmc, a.centroids, p.ncl, D, p.dtype) ||
+      !encode_rows(&tmv, a.value_sums, p.ncl, D, p.dtype))
+    return cudaErrorInvalidValue;
+  ScanArgs A{};
+  A.q = a.q;
+  A.Hq = p.Hq;
+  A.offsets = a.offsets;
+  A.rec = reinterpret_cast<uint2*>(ws + p.off_rec);
+  A.hist = reinterpret_cast<int32_t*>(ws + p.off_hist);
+  A.cnt1 = reinterpret_cast<int32_t*>(ws + p.off_cnt1);
+  A.est = reinterpret_cast<float*>(ws + p.off_est);
+  A.p1max = std::max(1, p.p1max);
+  A.scores_out = a.scores_out;
+  A.scale = p.scale;
+  A.exact_only = p.exact_only;
+  A.info = info;
+  A.nonc = nonc;
+  A.sel = reinterpret_cast<int32_t*>(ws + p.off_sel);
+  A.tok = reinterpret_cast<int32_t*>(ws + p.off_tok);
+  A.full = reinterpret_cast<int2*>(ws + p.off_full);
+  A.cap = p.cap;
+  A.topk_clusters = p.topk_clusters;
+  A.topk_fraction = p.topk_fraction;
+  A.mode = p.mode;
+  A.seed = p.seed;
+  A.slots = p.slots;
+  const size_t scan_smem = ScanSmem<T, D, G>::total(p.slots, p.exact_only);
+  set_smem(wave_scan_kernel<T, D, G>, scan_smem);
+  mark(1);
+  cudaError_t e1 = launch_ex(wave_scan_kernel<T, D, G>, dim3(std::max(1, p.n_scan)),
+                             dim3(kScanThreads), scan_smem, s, pdl, p.geo, cm, A, tmc, tmv,
+                             status);
+  if (e1 != cudaSuccess) return e1;
+  // K2: gather, exact attention, estimate corrections, merge
+  GatherArgs B{};
+  B.q = a.q;
+  B.Hq = p.Hq;
+  B.kp = a.kp;
+  B.vp = a.vp;
+  B.centroids = a.centroids;
+  B.value_sums = a.value_sums;
+  B.perm = a.perm;
+  B.rec = A.rec;
+  B.info = info;
+  B.st_slot = st_slot;
+  B.pc = pc;
+  B.tok = A.tok;
+  B.full = A.full;
+  B.cap = p.cap;
+  B.n_sink = p.n_sink;
+  B.window = p.window;
+  B.est = A.est;
+  B.p1max = A.p1max;
+  B.gat = reinterpret_cast<float*>(ws + p.off_gat);
+  B.n2max = p.n2max;
+  B.cnt2 = reinterpret_cast<int32_t*>(ws + p.off_cnt2);
+  B.out = a.out;
+  B.lse = a.lse;
+  B.scale = p.scale;
+  B.seed = p.seed;
+  std::memcpy(B.n2_base, p.n2_base, sizeof(B.n2_base));
+  const size_t g_smem = GatherSmem<T, D, G>::kTotal;
+  set_smem(wave_gather_kernel<T, D, G>, g_smem);
+  mark(2);
+  cudaError_t e2 = launch_ex(wave_gather_kernel<T, D, G>, dim3(p.n_gather), dim3(kGatherThreads),
+                             g_smem, s, pdl, p.geo, cm, B, status);
+  if (e2 != cudaSuccess) return e2;
+  mark(3);
+  return cudaGetLastError();
+}
+
+#define WI_DECODE_INSTANTIATE(T, D)                                                          \
+  template cudaError_t launch_decode_typed<T, D, 1>(const DecodePlan&, const DecodeArgs&,    \
+                                                    const ChunkMap&, cudaStream_t);          \
+  template cudaError_t launch_decode_typed<T, D, 2>(const DecodePlan&, const DecodeArgs&,    \
+                                                    const ChunkMap&, cudaStream_t);          \
+  template cudaError_t launch_decode_typed<T, D, 4>(const DecodePlan&, const DecodeArgs&,    \
+                                                    const ChunkMap&, cudaStream_t);          \
+  template cudaError_t launch_decode_typed<T, D, 8>(const DecodePlan&, const DecodeArgs&,    \
+                                                    const ChunkMap&, cudaStream_t);
+
+}  // namespace wi

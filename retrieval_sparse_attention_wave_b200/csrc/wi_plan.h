@@ -9,42 +9,69 @@
 
 namespace wi {
 
-constexpr int kStreamThreads = 256;   // streaming kernels: 8 warps
-constexpr int kTopkThreads = 512;     // one CTA per unit
-constexpr int kAttendTile = 64;       // tokens per exact-attention tile
-constexpr int kInfoInts = 8;          // per-unit info record (see wi_decode_layout)
+constexpr int kStreamThreads = 256;   // build kernels: 8 warps
 constexpr int kNumSMs = 148;          // B200
-constexpr int kScoreChunkBytes = 32768;  // centroid bytes (and as many value-sum bytes) per score CTA
-constexpr int kFold = 16;             // score-chunk parts folded into one by an attend fold CTA
-constexpr int kRangeClusters = 256;   // cluster ids per attend range CTA (one per thread)
+
+// Decode kernels.  A tile is 64 rows (centroid / value-sum rows in the scan,
+// gathered key / value rows in the gather); each of 8 consumer warps takes 8.
+constexpr int kTileRows = 64;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = 32 * kConsumerWarps;   // 256 consumer threads
+constexpr int kScanThreads = kConsumers + 32;     // + one producer warp
+constexpr int kGatherThreads = kConsumers;
+constexpr int kGatherTiles = 2;                   // tiles per gather block (128 rows)
+constexpr int kInfoInts = 16;                     // per-unit record (see wi_decode_layout)
+constexpr int kHistBins = 2048;                   // first radix digit: key bits 31..21
+constexpr int kTailCand = 1024;                   // threshold-bin members refined in shared memory
+constexpr int kMaxGatherPerUnit = 64;             // gather CTAs per unit (they loop beyond)
+constexpr int kMaxTailsPerCta = 64;               // units one scan CTA may touch
+
+// Per-unit record fields (int32 [U][kInfoInts]).
+enum UnitField {
+  kSelCount = 0,   // retrieved clusters (tail)
+  kThrKey = 1,     // k-th key, 0xFFFFFFFF when nothing is retrieved (tail)
+  kThrIdx = 2,     // largest id taken at the k-th key (tail)
+  kSelTokens = 3,  // token rows of the retrieved clusters (tail)
+  kSteady = 4,     // steady slots (steady kernel; T_b for a dense unit)
+  kAffected = 5,   // clusters holding a steady token (steady kernel)
+  kDense = 6,      // 1: attended densely (steady kernel)
+  kCandidates = 7, // candidate clusters (tail)
+  kFullRows = 8,   // clusters whose estimate is taken back out (tail)
+  kPartRows = 9,   // steady tokens of candidate clusters (steady kernel)
+  kNonCand = 10,   // clusters left without a non-steady token (steady kernel)
+  kNoEstimate = 11,// 1: the estimation zone is empty (tail)
+  kMode = 12,      // selection mode (0 exact, 1 sampled threshold bin)
+  kSampBin = 13,   // sampled mode: the threshold bin
+  kSampHash = 14,  // sampled mode: high 32 bits of the last draw taken ...
+  kSampHashLo = 15 // ... and its low 32 bits (the id is kThrIdx)
+};
 
 struct DecodePlan {
   int exact_only;          // no estimation zone (block top-k workload)
+  int mode;                // 0 exact top-k, 1 sampled threshold bin
+  uint32_t seed;           // draws of the sampled mode
   Geo geo;
   int dtype, D, G, Hq, U;
   int n_sink, window, topk_clusters;
   double topk_fraction;
-  int max_nc;
-  int64_t ncl;               // centroid rows of the index (Hkv * sum NC_b)
-  int seg_len, seg_clusters;  // segment length and clusters per full segment
-  int score_chunk, n_score_blocks;   // clusters per score CTA, score CTAs per unit
-  int cap;                 // steady-list capacity per unit (>= 1)
-  int sort_pow2;           // shared-memory sort size for the steady list
-  int n_rng;               // attend range CTAs per unit (kRangeW cluster ids each)
-  int n_sc;                // attend steady CTAs per unit (two tiles of steady slots each)
-  int n_fold;              // fold CTAs per unit (kFold score parts each)
-  int n_parts;             // n_rng + n_sc + n_fold softmax parts per (unit, head)
   float scale;             // 1/sqrt(d)
-  // workspace byte offsets; [0, off_scores) must be zero before the first call
-  size_t off_status, off_counters, off_hist, off_aff_of;
-  size_t off_scores, off_keys, off_sel, off_info;
-  int sel_words;           // selection bitmap words per unit (kRangeClusters / 32 per range CTA)
-  size_t off_st_slot, off_st_cl, off_aff_cl, off_aff_start, off_partials;
-  size_t off_dv, off_est, off_nonc;
-  size_t off_q, off_out, off_lse;
+  int max_nc;
+  int cap;                 // steady slots per unit (>= 1)
+  int64_t ncl;             // centroid rows of the index (Hkv * sum NC_b)
+  int64_t ntok;            // token rows of the index (Hkv * sum T_b)
+  // scan (K1): chunks of kTileRows clusters of the units that are not dense
+  int32_t ch_base[kMaxBatch + 1];   // chunk prefix over sequences (Hkv chunks-per-unit each)
+  int n_chunks, n_scan, p1max;      // total chunks, scan CTAs, parts per unit at most
+  int slots;                        // ring slots per scan CTA
+  // gather (K2): per sequence n2_b CTAs per unit
+  int32_t n2_base[kMaxBatch + 1];   // CTA prefix over sequences (Hkv * n2_b each)
+  int n_gather, n2max;
+  // workspace byte offsets; [0, off_rec) must be zero before the first call
+  size_t off_status, off_cnt1, off_cnt2, off_hist;
+  size_t off_rec, off_info, off_st_slot, off_pc, off_nonc, off_sel, off_tok, off_full;
+  size_t off_est, off_gat, off_q, off_out, off_lse;
   size_t total;
 };
-
 // First segment each sequence's build kernels process (all zero for a full
 // build; an index extension starts at the old index's first incomplete one).
 struct SegFrom {
@@ -76,6 +103,7 @@ struct DecodeArgs {
   float* lse;
   unsigned char* ws;
   cudaEvent_t* stage_events;
+  float* scores_out;       // optional [ncl][G] per-head centroid scores
 };
 
 struct BuildArgs {
@@ -102,9 +130,11 @@ extern const char* const kDecodeStageNames[kDecodeStages];
 cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 wi_status decode_workspace_extent(const wi_index* idx, const wi_decode_params* p, size_t* total,
                                   size_t* zero_prefix);
-size_t decode_attend_smem(int dtype, int D, int G, int n_parts);
-size_t decode_score_smem(int dtype, int D, int G, int sort_pow2, int cap);
-size_t decode_topk_smem(int max_nc, int cap);
+// shared memory of the decode kernels (host plan checks)
+size_t decode_scan_smem(int dtype, int D, int G, int slots, int exact_only);
+size_t decode_gather_smem(int dtype, int D, int G);
+size_t decode_steady_smem(int cap);
+size_t decode_scan_slot_bytes(int dtype, int D, int exact_only);
 cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s);
 // Position-block index: each token's cluster is its block inside its segment,
 // then one finalizing update pass.

@@ -28,7 +28,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_stage_names():
-    assert W.stage_names() == ["score", "topk", "attend"]
+    assert W.stage_names() == ["steady", "scan", "gather"]
     assert W.lib().wi_decode_stage_name(99) is None
 
 
@@ -98,36 +98,37 @@ def test_decode_workspace_size_and_layout():
     assert W.lib().wi_decode_workspace_layout(C.byref(index_struct()), C.byref(params()),
                                               C.byref(lay)) == W.WI_OK
     assert lay.total_bytes == n and lay.status == 0
-    assert 0 < lay.scores < lay.keys < lay.selected < lay.unit_info < n
-    assert lay.n_attend_ctas >= 2 and lay.n_score_ctas >= 1
-    assert lay.sel_words >= 8 and lay.sel_words % 8 == 0
+    assert 0 < lay.records < lay.selected < n and 0 < lay.unit_info < n
+    assert lay.n_scan_ctas >= 1 and lay.n_gather_ctas >= 8 and lay.info_ints == 16
 
 
 @pytest.mark.parametrize("dtype,d,seq,expect", [
-    # 131072 tokens: 8192 clusters -> 32 range CTAs + 1 steady CTA, 256 bitmap
-    # words; bf16 d = 128 (tensor cores) estimates in the range CTAs: no folds
-    (W.WI_BF16, 128, [131072], dict(n_attend_ctas=33, sel_words=256, n_score_ctas=64)),
-    # fp32: 64 clusters per 32 KB chunk; 32-row tiles, so the 68 steady slots
-    # take two steady CTAs
-    (W.WI_F32, 128, [131072], dict(n_attend_ctas=34, sel_words=256, n_score_ctas=128)),
-    # ragged batch, sized by the longest sequence: 256 clusters -> one range
-    # CTA, one steady CTA, 8 bitmap words, two 128-cluster score chunks
-    (W.WI_BF16, 128, [4096, 300], dict(n_attend_ctas=2, sel_words=8, n_score_ctas=2)),
+    # 131072 tokens, 8 KV heads: 8192 clusters per head -> 128 chunks of 64,
+    # 1024 chunks on 148 streaming CTAs; k = ceil(0.018 * 8192) = 148, so a
+    # head expects 148 * 16 retrieved + 68 steady + 148 + 68 correction rows
+    # = 2652 rows -> 21 gather CTAs of 128 rows per head
+    (W.WI_BF16, 128, [131072], dict(n_scan_ctas=148, n_gather_ctas=168)),
+    # fp32: the same chunking (64-row tiles whatever the row size)
+    (W.WI_F32, 128, [131072], dict(n_scan_ctas=148, n_gather_ctas=168)),
+    # ragged batch: 256 clusters (4 chunks) and 19 clusters (1 chunk) per
+    # head -> 40 chunks, 40 CTAs; 221 and 153 expected rows -> 2 + 2 gather
+    # CTAs per head
+    (W.WI_BF16, 128, [4096, 300], dict(n_scan_ctas=40, n_gather_ctas=32)),
 ])
 def test_decode_plan_shapes(dtype, d, seq, expect):
-    """The launch plan's per-unit CTA counts and bitmap size, from the
-    geometry alone (host logic)."""
+    """The launch plan's CTA counts, from the geometry alone (host logic)."""
     lay = W.WiDecodeLayout()
     ix = index_struct(seq=seq, dtype=dtype, head_dim=d, n_pages=16384, max_pages=16384)
     assert W.lib().wi_decode_workspace_layout(C.byref(ix), C.byref(params()), C.byref(lay)) \
         == W.WI_OK
     for k, v in expect.items():
         assert getattr(lay, k) == v, (k, getattr(lay, k), v)
-    # the exact-only flag changes nothing in the layout
+    # the exact-only workload keeps no estimation parts and fewer rows
     lay2 = W.WiDecodeLayout()
     assert W.lib().wi_decode_workspace_layout(C.byref(ix), C.byref(params(exact_only=1)),
                                               C.byref(lay2)) == W.WI_OK
-    assert lay2.total_bytes == lay.total_bytes
+    assert lay2.total_bytes < lay.total_bytes
+    assert lay2.n_gather_ctas <= lay.n_gather_ctas
 
 
 @pytest.mark.parametrize("over,expect", [
@@ -140,6 +141,9 @@ def test_decode_plan_shapes(dtype, d, seq, expect):
     (dict(topk_clusters=-1, topk_fraction=1.5), W.WI_ERR_INVALID_ARG),
     (dict(n_sink=5000, window=5000), W.WI_OK),        # all steady (dense) is legal
     (dict(n_sink=8000, window=192), W.WI_OK),         # exactly WI_MAX_STEADY
+    (dict(topk_mode=1, seed=7), W.WI_OK),              # sampled threshold bin
+    (dict(topk_mode=2), W.WI_ERR_INVALID_ARG),         # no such selection mode
+    (dict(scores_out=FAKE + 2), W.WI_ERR_INVALID_ARG),  # misaligned score buffer
 ])
 def test_decode_param_validation(over, expect):
     st, _ = ws_size(index_struct(seq=[10000]), params(**over))
@@ -265,29 +269,29 @@ def test_status_strings():
     assert lib.wi_read_device_status(None, None, None, 0) == W.WI_ERR_INVALID_ARG
 
 
-def test_selection_bitmap_decoding_on_the_host():
-    """The binding reads the selection bitmap (bit c % 32 of word c / 32 of
-    the unit's words) back into ascending cluster ids."""
+def test_selection_list_decoding_on_the_host():
+    """The binding reads a unit's retrieved ids from its rows of the
+    selection list (laid out like the centroids) and checks them."""
     import types
 
-    import numpy as np
     import torch
-    lay = types.SimpleNamespace(selected=256, sel_words=16)
-    index = types.SimpleNamespace(n_kv_heads=2)
-    ws = torch.zeros(256 + 4 * 16 * 4, dtype=torch.uint8)
-    words = ws[256:].view(torch.int32)
-    want = {(0, 1): [0, 31, 32, 200, 511], (1, 0): [5, 63, 64, 65]}
-    for (b, h), ids in want.items():
-        u = b * 2 + h
-        for c in ids:
-            w = u * 16 + c // 32
-            words[w] = int(np.int32(np.uint32(int(words[w]) & 0xFFFFFFFF | (1 << (c % 32)))))
-    for (b, h), ids in want.items():
-        got = W.selected_clusters(ws, lay, index, b, h, len(ids))
-        assert got.tolist() == ids
+    lay = types.SimpleNamespace(selected=256)
+    index = types.SimpleNamespace(n_kv_heads=2, nc=[10, 7],
+                                  cl_row=lambda b, h: 2 * sum([10, 7][:b]) + h * [10, 7][b])
+    ws = torch.zeros(256 + 4 * 34, dtype=torch.uint8)
+    ids = ws[256:].view(torch.int32)
+    want = {(0, 1): [0, 3, 9], (1, 0): [2, 5, 6]}
+    for (b, h), xs in want.items():
+        r = index.cl_row(b, h)
+        ids[r:r + len(xs)] = torch.tensor(xs, dtype=torch.int32)
+    for (b, h), xs in want.items():
+        assert W.selected_clusters(ws, lay, index, b, h, len(xs)).tolist() == xs
     assert W.selected_clusters(ws, lay, index, 0, 0, 0).tolist() == []
+    with pytest.raises(RuntimeError):       # more than the unit's clusters
+        W.selected_clusters(ws, lay, index, 1, 0, 8)
+    ids[index.cl_row(1, 0)] = 9             # not ascending
     with pytest.raises(RuntimeError):
-        W.selected_clusters(ws, lay, index, 0, 1, 4)
+        W.selected_clusters(ws, lay, index, 1, 0, 3)
 
 
 def test_noalloc_refuses_on_the_host():

@@ -32,6 +32,7 @@ def check_decode(wl, units, params, *, shuffle_seed=None, page_size=None, ref_de
     H.upload_index(wx, units)
     q = wl.q.to(DEV)
     ws = W.decode_workspace(wx, params)
+    params.scores_out = W.scores_buffer(wx, wl.n_q_heads)
     out, lse = W.decode(q, wx, params, ws=ws)
     torch.cuda.synchronize()
     assert W.read_device_status(ws) == 0
@@ -52,7 +53,7 @@ def check_decode(wl, units, params, *, shuffle_seed=None, page_size=None, ref_de
         est = not params.exact_only
         tr = O.decode_unit(qg, ix, params.n_sink, params.window, k, estimate=est)
         # (a1) scores
-        sc = W.centroid_scores(ws, lay, wx, G, b, h).cpu().numpy().astype(np.float64)
+        sc = W.centroid_scores(params.scores_out, wx, b, h).cpu().numpy().astype(np.float64)
         if not info[u, 6]:
             smax = np.max(np.abs(tr.scores))
             assert np.max(np.abs(sc - tr.scores.T)) <= 1e-5 * max(smax, 1.0)

@@ -11,9 +11,11 @@ namespace wi {
 
 const char* const kDecodeStageNames[kDecodeStages] = {"steady", "scan", "gather"};
 
-template <typename T, int D, int G>
-cudaError_t launch_decode_typed(const DecodePlan& p, const DecodeArgs& a, const ChunkMap& cm,
-                                cudaStream_t s);
+// compiled one key type and head size per file
+WI_DECODE_EXTERN(__nv_bfloat16, 128)
+WI_DECODE_EXTERN(__nv_bfloat16, 64)
+WI_DECODE_EXTERN(float, 128)
+WI_DECODE_EXTERN(float, 64)
 
 namespace {
 

@@ -635,7 +635,7 @@ constexpr int kTailRound = kConsumers * kTailPT;
 // members with the smallest (SplitMix64(seed 2^32 + c), c) draws; then the
 // retrieved ids, their token slots and the clusters whose estimate the
 // gather takes back out.
-__device__ void scan_tail(const Geo& geo, const ScanArgs& A, int u, unsigned char* sh,
+__device__ __noinline__ void scan_tail(const Geo& geo, const ScanArgs& A, int u, unsigned char* sh,
                           uint32_t* status) {
   const int b = u / geo.hkv, h = u - b * geo.hkv;
   const int NC = geo.NC(b), Tb = geo.T(b);
@@ -1642,5 +1642,15 @@ cudaError_t launch_decode_typed(const DecodePlan& p, const DecodeArgs& a, const 
                                                     const ChunkMap&, cudaStream_t);          \
   template cudaError_t launch_decode_typed<T, D, 8>(const DecodePlan&, const DecodeArgs&,    \
                                                     const ChunkMap&, cudaStream_t);
+
+#define WI_DECODE_EXTERN(T, D)                                                               \
+  extern template cudaError_t launch_decode_typed<T, D, 1>(const DecodePlan&, const DecodeArgs&, \
+                                                           const ChunkMap&, cudaStream_t);       \
+  extern template cudaError_t launch_decode_typed<T, D, 2>(const DecodePlan&, const DecodeArgs&, \
+                                                           const ChunkMap&, cudaStream_t);       \
+  extern template cudaError_t launch_decode_typed<T, D, 4>(const DecodePlan&, const DecodeArgs&, \
+                                                           const ChunkMap&, cudaStream_t);       \
+  extern template cudaError_t launch_decode_typed<T, D, 8>(const DecodePlan&, const DecodeArgs&, \
+                                                           const ChunkMap&, cudaStream_t);
 
 }  // namespace wi

@@ -79,6 +79,13 @@ typedef enum wi_dtype { WI_F32 = 0, WI_BF16 = 1 } wi_dtype;
                                     after a failed call); recomputed, result valid */
 #define WI_DEV_TIMEOUT     0x10u /* a bounded wait for an asynchronous copy gave
                                     up; the call's results are not valid        */
+#define WI_DEV_CANCELLATION 0x20u /* the estimate taken back out (retrieved and
+                                    non-candidate clusters, steady tokens) was
+                                    more than 16x the output's softmax
+                                    denominator, so the estimation zone lost its
+                                    precision: the index's centroids are not the
+                                    means of their members (every index the
+                                    build calls write is); results not valid    */
 
 /*
  * Paged KV cache in original token order (the build input).

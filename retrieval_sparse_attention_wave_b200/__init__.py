@@ -40,6 +40,7 @@ WI_MAX_BATCH = 256
 WI_MAX_SEG_LEN = 16384
 WI_MAX_STEADY = 8192
 WI_DEV_BAD_PAGE, WI_DEV_BAD_SLOT, WI_DEV_BAD_CLUSTER, WI_DEV_BAD_HIST = 0x1, 0x2, 0x4, 0x8
+WI_DEV_TIMEOUT, WI_DEV_CANCELLATION = 0x10, 0x20
 WI_TOPK_EXACT, WI_TOPK_SAMPLED = 0, 1
 
 EXPORTED = [

@@ -86,7 +86,8 @@ struct ChunkMap {
 namespace {
 
 constexpr int kHistShift = 21;    // first radix digit: key bits 31..21
-constexpr int kPartStride = 4;    // a softmax part of one head: {m, l, -, -, o[D]}
+constexpr float kCancelRatio = 16.f;   // taken-out mass / merged denominator flagged above this
+constexpr int kPartStride = 4;    // a softmax part of one head: {m, l, ln, -, o[D]}
 
 // ------------------------------------------------------------------ tiles
 // A tile holds kTileRows rows of D elements as NB = D * sizeof(T) / 128
@@ -132,6 +133,7 @@ struct MmaAcc {
   static_assert(G <= 8, "at most 8 query heads per KV head (MMA rows 0..7)");
   uint32_t qa0[D / 16], qa2[D / 16];
   float m, l;          // head lane / 4: running max, this lane's share of the sum
+  float ln;            // this lane's share of the rows with negative weight, as magnitudes
   float o[D / 8][4];   // [n-tile][hi pair, lo pair] of output columns 8j + 2(lane % 4)
 
   __device__ __forceinline__ void load_q(const __nv_bfloat16* q_group) {
@@ -146,6 +148,7 @@ struct MmaAcc {
   __device__ __forceinline__ void reset() {
     m = -INFINITY;
     l = 0.f;
+    ln = 0.f;
 #pragma unroll
     for (int j = 0; j < D / 8; ++j)
 #pragma unroll
@@ -182,6 +185,7 @@ struct MmaAcc {
     const float p0 = x0 == -INFINITY ? 0.f : __expf(x0 - mnew);
     const float p1 = x1 == -INFINITY ? 0.f : __expf(x1 - mnew);
     l = l * corr + m0.wl * p0 + m1.wl * p1;
+    ln = ln * corr + fmaxf(-m0.wl, 0.f) * p0 + fmaxf(-m1.wl, 0.f) * p1;
     m = mnew;
     uint32_t hi, lo;
     split_bf16(m0.wo * p0, m1.wo * p1, hi, lo);
@@ -197,19 +201,21 @@ struct MmaAcc {
       }
     }
   }
-  // this warp's part -> comb [G][D + 2] = {m, l, o[D]} per head
+  // this warp's part -> comb [G][D + 4] = {m, l, ln, -, o[D]} per head
   __device__ __forceinline__ void to_smem(float* comb) const {
     const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-    float ls = l;
+    float ls = l, lns = ln;
     ls += __shfl_xor_sync(0xffffffffu, ls, 1);
     ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+    lns += __shfl_xor_sync(0xffffffffu, lns, 1);
+    lns += __shfl_xor_sync(0xffffffffu, lns, 2);
     if (g < G) {
-      float* row = comb + g * (D + 2);
+      float* row = comb + g * (D + kPartStride);
 #pragma unroll
       for (int j = 0; j < D / 8; ++j)
-        *reinterpret_cast<float2*>(row + 2 + 8 * j + 2 * tq) =
+        *reinterpret_cast<float2*>(row + kPartStride + 8 * j + 2 * tq) =
             make_float2(o[j][0] + o[j][2], o[j][1] + o[j][3]);
-      if (tq == 0) { row[0] = m; row[1] = ls; }
+      if (tq == 0) { row[0] = m; row[1] = ls; row[2] = lns; }
     }
   }
 };
@@ -221,7 +227,7 @@ struct FmaAcc {
   static constexpr int LPR = D / 4, RPW = 32 / LPR, NST = 8 / RPW;
   static_assert(G <= LPR, "group larger than lanes per row");
   float qv[G][4];
-  float m[G], l[G];
+  float m[G], l[G], ln[G];
   float o[G][4];
 
   __device__ __forceinline__ void load_q(const float* q_group, float scale) {
@@ -237,6 +243,7 @@ struct FmaAcc {
     for (int g = 0; g < G; ++g) {
       m[g] = -INFINITY;
       l[g] = 0.f;
+      ln[g] = 0.f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[g][e] = 0.f;
     }
@@ -276,13 +283,15 @@ struct FmaAcc {
       for (int r = 0; r < 8; ++r) mx = rm[r].valid ? fmaxf(mx, s[r * G + g]) : mx;
       const float mnew = fmaxf(m[g], mx);
       const float corr = mnew == -INFINITY ? 1.f : __expf(m[g] - mnew);
-      float ls = 0.f;
+      float ls = 0.f, lns = 0.f;
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         p[r][g] = rm[r].valid ? __expf(s[r * G + g] - mnew) : 0.f;
         ls += rm[r].wl * p[r][g];
+        lns += fmaxf(-rm[r].wl, 0.f) * p[r][g];
       }
       l[g] = l[g] * corr + ls;
+      ln[g] = ln[g] * corr + lns;
       m[g] = mnew;
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[g][e] *= corr;
@@ -309,20 +318,26 @@ struct FmaAcc {
       for (int e = 0; e < 4; ++e)
 #pragma unroll
         for (int ofs = LPR; ofs < 32; ofs <<= 1) o[g][e] += __shfl_xor_sync(0xffffffffu, o[g][e], ofs);
-    if (rs == 0) {
+    if (rs == 0) {   // rows of D + 4 floats: 8-byte aligned pairs
 #pragma unroll
-      for (int g = 0; g < G; ++g)
-        *reinterpret_cast<float4*>(comb + g * (D + 2) + 2 + 4 * sub) =
-            make_float4(o[g][0], o[g][1], o[g][2], o[g][3]);
+      for (int g = 0; g < G; ++g) {
+        float2* p = reinterpret_cast<float2*>(comb + g * (D + kPartStride) + kPartStride + 4 * sub);
+        p[0] = make_float2(o[g][0], o[g][1]);
+        p[1] = make_float2(o[g][2], o[g][3]);
+      }
     }
     if (lane == 0) {
 #pragma unroll
-      for (int g = 0; g < G; ++g) { comb[g * (D + 2)] = m[g]; comb[g * (D + 2) + 1] = l[g]; }
+      for (int g = 0; g < G; ++g) {
+        comb[g * (D + kPartStride)] = m[g];
+        comb[g * (D + kPartStride) + 1] = l[g];
+        comb[g * (D + kPartStride) + 2] = ln[g];
+      }
     }
   }
 };
 
-// Combine the per-warp parts comb [kConsumerWarps][G][D + 2] into one part
+// Combine the per-warp parts comb [kConsumerWarps][G][D + 4] into one part
 // [G][D + 4] at `part` (threads 0 .. kConsumers - 1).
 template <int D, int G>
 __device__ __forceinline__ void combine_warps(const float* comb, float* part, int tid) {
@@ -330,17 +345,22 @@ __device__ __forceinline__ void combine_warps(const float* comb, float* part, in
     const int g = i / D, e = i - g * D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * G + g) * (D + 2)]);
-    float O = 0.f, L = 0.f;
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * G + g) * (D + kPartStride)]);
+    float O = 0.f, L = 0.f, LN = 0.f;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
-      const float* row = comb + (w * G + g) * (D + 2);
+      const float* row = comb + (w * G + g) * (D + kPartStride);
       const float f = row[0] == -INFINITY ? 0.f : __expf(row[0] - M);
-      O += f * row[2 + e];
+      O += f * row[kPartStride + e];
       L += f * row[1];
+      LN += f * row[2];
     }
     part[g * (D + kPartStride) + kPartStride + e] = O;
-    if (e == 0) { part[g * (D + kPartStride)] = M; part[g * (D + kPartStride) + 1] = L; }
+    if (e == 0) {
+      part[g * (D + kPartStride)] = M;
+      part[g * (D + kPartStride) + 1] = L;
+      part[g * (D + kPartStride) + 2] = LN;
+    }
   }
 }
 
@@ -394,6 +414,19 @@ wave_steady_kernel(const Geo geo, const SteadyArgs a, uint32_t* status) {
     srt[i] = k;
   }
   __syncthreads();
+  if (n_st <= (int)blockDim.x) {
+    // short lists (the usual 68): each key's rank among all, one step
+    const unsigned long long mine = tid < n_st ? srt[tid] : 0ull;
+    int rank = 0;
+    if (tid < n_st)
+      for (int j = 0; j < n_st; ++j) {
+        const unsigned long long x = srt[j];
+        rank += x < mine || (x == mine && j < tid);   // equal keys only on a bad slot
+      }
+    __syncthreads();
+    if (tid < n_st) srt[rank] = mine;
+    __syncthreads();
+  } else {
   // bitonic sort by slot (clusters are slot ranges, so this groups them too)
   for (int k = 2; k <= npow; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
@@ -407,6 +440,7 @@ wave_steady_kernel(const Geo geo, const SteadyArgs a, uint32_t* status) {
       }
       __syncthreads();
     }
+  }
   }
   int32_t* slots = a.st_slot + (int64_t)u * a.cap;
   for (int i = tid; i < n_st; i += blockDim.x) slots[i] = (int32_t)(srt[i] >> 32);
@@ -490,19 +524,32 @@ struct ScanArgs {
   int slots;
 };
 
+constexpr int kTailPT = 32;                    // records per consumer per round
+constexpr int kTailRound = kConsumers * kTailPT;
+// A round's records (and one more, for the last one's count) sit in shared
+// memory with one pad slot per 32, so a consumer's run of 32 consecutive
+// records falls on distinct banks.
+__device__ __forceinline__ int rpad(int i) { return i + (i >> 5); }
+constexpr size_t kTailRecBytes = (size_t)(kTailRound + 1 + kTailRound / 32 + 1) * 8;
+
 // Shared memory of a scan CTA (bytes, after 1024-byte alignment).
 template <typename T, int D, int G>
 struct ScanSmem {
   using TS = TileShape<T, D>;
-  static constexpr size_t kComb = (size_t)kConsumerWarps * G * (D + 2) * 4;
+  static constexpr size_t kComb = (size_t)kConsumerWarps * G * (D + kPartStride) * 4;
   static constexpr size_t kTail = (size_t)kHistBins * 4 + (size_t)kTailCand * 8 + 1024;
   static constexpr size_t kUnion = kComb > kTail ? kComb : kTail;
   static constexpr size_t kHist16 = (size_t)kHistBins / 2 * 4;
   static constexpr size_t kRows = (size_t)kConsumerWarps * 8 * sizeof(RowMult);
   static constexpr size_t kSc = (size_t)kConsumerWarps * 8 * G * 4;
   __host__ __device__ static size_t slot_bytes(int exact_only) { return (size_t)TS::kBytes * (exact_only ? 1 : 2); }
+  // the ring, which the tails reuse for their records once the chunks are done
+  __host__ __device__ static size_t ring_bytes(int slots, int exact_only) {
+    const size_t r = slots * slot_bytes(exact_only);
+    return r > kTailRecBytes ? r : (kTailRecBytes + 1023) / 1024 * 1024;
+  }
   __host__ __device__ static size_t total(int slots, int exact_only) {
-    return 1024 + slots * slot_bytes(exact_only) + kUnion + kHist16 + kRows + kSc;
+    return 1024 + ring_bytes(slots, exact_only) + kUnion + kHist16 + kRows + kSc;
   }
 };
 
@@ -625,8 +672,13 @@ __device__ __forceinline__ int select_bin(const int* hist, int nb, int krem, int
   return r;
 }
 
-constexpr int kTailPT = 32;                    // records per consumer per round
-constexpr int kTailRound = kConsumers * kTailPT;
+
+// The unit's geometry, passed to the tail as scalars (the 2 KB Geo would be
+// copied to local memory for a call).
+struct TailUnit {
+  int u, NC, Tb;
+  int64_t row0, trow;
+};
 
 // The tail of unit u (by the last scan CTA to finish it): the exact top-k
 // threshold (kstar, thr) -- cluster c is retrieved iff its key > kstar, or
@@ -635,75 +687,87 @@ constexpr int kTailRound = kConsumers * kTailPT;
 // members with the smallest (SplitMix64(seed 2^32 + c), c) draws; then the
 // retrieved ids, their token slots and the clusters whose estimate the
 // gather takes back out.
-__device__ __noinline__ void scan_tail(const Geo& geo, const ScanArgs& A, int u, unsigned char* sh,
-                          uint32_t* status) {
-  const int b = u / geo.hkv, h = u - b * geo.hkv;
-  const int NC = geo.NC(b), Tb = geo.T(b);
+//
+// Its passes are rolled loops over the records in shared memory.
+__device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, unsigned char* sh,
+                                       uint2* srec, uint32_t* status) {
+  const int u = tu.u, NC = tu.NC, Tb = tu.Tb;
   const int tid = threadIdx.x;
   int* s_hist = reinterpret_cast<int*>(sh);                                   // [2048]
   unsigned long long* s_cand = reinterpret_cast<unsigned long long*>(sh + kHistBins * 4);  // [kTailCand]
   int* s_sh = reinterpret_cast<int*>(sh + kHistBins * 4 + kTailCand * 8);     // [64]
   int* s_ctl = s_sh + 64;                                                     // [16]
-  const int64_t row0 = geo.cl_row(b, h);
+  const int64_t row0 = tu.row0;
   uint2* rec = A.rec + row0;
   int32_t* I = A.info + (int64_t)u * kInfoInts;
   int32_t* hg = A.hist + (int64_t)u * kHistBins;
-
-  // round 0's records are loaded first, with the histogram
   const int n_rounds = (NC + kTailRound - 1) / kTailRound;
-  uint32_t rk[kTailPT];
-  int32_t ro[kTailPT + 1];
   int loaded = -1;
+  // round r's records r R .. r R + R into shared memory (L2 loads, all in
+  // flight together); past the unit: no key, count 0
   auto load_round = [&](int r) {
-    const int c0 = r * kTailRound + tid * kTailPT;
+    const int c0 = r * kTailRound;
+    uint2 v[(kTailRound + kConsumers) / kConsumers];
 #pragma unroll
-    for (int i = 0; i < kTailPT; ++i) {
-      const int c = c0 + i;
-      uint2 v = make_uint2(0u, (uint32_t)Tb);   // past the unit: no key, no tokens
-      if (c < NC) v = __ldcg(rec + c);
-      rk[i] = v.x;
-      ro[i] = (int32_t)v.y;
+    for (int j = 0; j < (kTailRound + kConsumers) / kConsumers; ++j) {
+      const int i = tid + j * kConsumers, c = c0 + i;
+      v[j] = make_uint2(0u, (uint32_t)Tb);
+      if (i <= kTailRound && c < NC) v[j] = __ldcg(rec + c);
     }
-    const int cn = c0 + kTailPT;
-    ro[kTailPT] = cn < NC ? (int32_t)__ldcg(&rec[cn].y) : Tb;
+    csync();   // the previous round's readers are done
+#pragma unroll
+    for (int j = 0; j < (kTailRound + kConsumers) / kConsumers; ++j) {
+      const int i = tid + j * kConsumers;
+      if (i <= kTailRound) srec[rpad(i)] = v[j];
+    }
+    csync();
     loaded = r;
   };
-  pdl_wait();   // the steady kernel's lists
-  load_round(0);
-  for (int i = tid; i < kHistBins; i += kConsumers) {
-    s_hist[i] = __ldcg(hg + i);
-    hg[i] = 0;   // clean for the next call
-  }
-  const int n_nonc = __ldcg(I + kNonCand);
-  csync();
-  // the clusters left without a non-steady token leave the histogram, and
-  // their keys become 0 (not candidates) for everything that follows
-  const int2* nonc = A.nonc + (int64_t)u * A.cap;
-  for (int j = tid; j < n_nonc; j += kConsumers) {
-    const int c = __ldcg(&nonc[j].x);
-    if (c >= 0 && c < NC) {
-      const uint32_t key = __ldcg(&rec[c].x);
-      if (key) atomicSub(&s_hist[key >> kHistShift], 1);
-      rec[c].x = 0u;
-      // the round-0 registers of its owner are refreshed below
-    }
-  }
-  csync();
-  if (n_nonc > 0) load_round(0);   // see the zeroed keys
+  auto key_at = [&](int i) { return srec[rpad(tid * kTailPT + i)].x; };
+  auto cnt_at = [&](int i) {
+    return (int)srec[rpad(tid * kTailPT + i + 1)].y - (int)srec[rpad(tid * kTailPT + i)].y;
+  };
   auto for_rounds = [&](auto&& body) {
     for (int r = 0; r < n_rounds; ++r) {
       if (loaded != r) load_round(r);
       body(r);
     }
   };
+
+  pdl_wait();   // the steady kernel's lists
+  {
+    int hv[kHistBins / kConsumers];
+#pragma unroll
+    for (int j = 0; j < kHistBins / kConsumers; ++j) hv[j] = __ldcg(hg + tid + j * kConsumers);
+#pragma unroll
+    for (int j = 0; j < kHistBins / kConsumers; ++j) {
+      s_hist[tid + j * kConsumers] = hv[j];
+      hg[tid + j * kConsumers] = 0;   // clean for the next call
+    }
+  }
+  const int n_nonc = __ldcg(I + kNonCand);
+  // the clusters left without a non-steady token leave the histogram, and
+  // their keys become 0 (not candidates) before the records are read
+  const int2* nonc = A.nonc + (int64_t)u * A.cap;
+  csync();
+  for (int j = tid; j < n_nonc; j += kConsumers) {
+    const int c = __ldcg(&nonc[j].x);
+    if (c >= 0 && c < NC) {
+      const uint32_t key = __ldcg(&rec[c].x);
+      if (key) atomicSub(&s_hist[key >> kHistShift], 1);
+      __stcg(&rec[c].x, 0u);
+    }
+  }
+  __threadfence_block();
+  csync();
   // candidates: the nonzero keys, counted in one pass; the histogram must
   // hold as many (a stale histogram, left by a failed call, is rebuilt from
   // the keys)
   int n_cand = 0, hist_total;
   for_rounds([&](int) {
     int s = 0;
-#pragma unroll
-    for (int i = 0; i < kTailPT; ++i) s += rk[i] != 0u;
+#pragma unroll 1
+    for (int i = 0; i < kTailPT; ++i) s += key_at(i) != 0u;
     int t;
     cscan(s, s_sh, &t);
     n_cand += t;
@@ -718,9 +782,11 @@ __device__ __noinline__ void scan_tail(const Geo& geo, const ScanArgs& A, int u,
     for (int i = tid; i < kHistBins; i += kConsumers) s_hist[i] = 0;
     csync();
     for_rounds([&](int) {
-#pragma unroll
-      for (int i = 0; i < kTailPT; ++i)
-        if (rk[i]) atomicAdd(&s_hist[rk[i] >> kHistShift], 1);
+#pragma unroll 1
+      for (int i = 0; i < kTailPT; ++i) {
+        const uint32_t key = key_at(i);
+        if (key) atomicAdd(&s_hist[key >> kHistShift], 1);
+      }
     });
     csync();
   }
@@ -731,6 +797,7 @@ __device__ __noinline__ void scan_tail(const Geo& geo, const ScanArgs& A, int u,
   int thr = -1;
   int bin1 = -1;
   uint64_t hstar = 0;
+  auto draw = [&](uint32_t c) { return splitmix64(((uint64_t)A.seed << 32) | (uint64_t)c); };
   if (k == n_cand && k > 0) {
     kstar = 1u;
     thr = INT_MAX;
@@ -740,43 +807,47 @@ __device__ __noinline__ void scan_tail(const Geo& geo, const ScanArgs& A, int u,
     int krem = k - above;
     const int nb1 = s_hist[bin1];
     // the threshold bin's members in id order: into shared memory when they
-    // fit; otherwise each refinement pass streams the keys again
+    // fit; otherwise each refinement pass streams the records again
     const bool fits = nb1 <= kTailCand;
     if (fits) {
       int base = 0;
       for_rounds([&](int r) {
         int s = 0;
-#pragma unroll
-        for (int i = 0; i < kTailPT; ++i) s += rk[i] != 0u && (int)(rk[i] >> kHistShift) == bin1;
+#pragma unroll 1
+        for (int i = 0; i < kTailPT; ++i) {
+          const uint32_t key = key_at(i);
+          s += key != 0u && (int)(key >> kHistShift) == bin1;
+        }
         int t;
         int pos = base + cscan(s, s_sh, &t) - s;
-#pragma unroll
-        for (int i = 0; i < kTailPT; ++i)
-          if (rk[i] != 0u && (int)(rk[i] >> kHistShift) == bin1) {
+#pragma unroll 1
+        for (int i = 0; i < kTailPT && s > 0; ++i) {
+          const uint32_t key = key_at(i);
+          if (key != 0u && (int)(key >> kHistShift) == bin1) {
             if (pos < kTailCand)
-              s_cand[pos] = ((unsigned long long)rk[i] << 32) |
+              s_cand[pos] = ((unsigned long long)key << 32) |
                             (uint32_t)(r * kTailRound + tid * kTailPT + i);
             ++pos;
+            --s;
           }
+        }
         base += t;
       });
       csync();
     }
+    // (members: the bin holding the k-th key is a 2^-9 wide slice of the
+    // key range, so it normally holds a few dozen clusters)
     if (A.mode == 1) {
       // sampled: the krem members of the threshold bin with the smallest
-      // (draw, id); streamed or from shared memory, one rank pass
-      // (members are few: the bin holds the k-th key and is a 2^-9 wide
-      // slice of the key range)
-      auto draw = [&](uint32_t c) {
-        return splitmix64(((uint64_t)A.seed << 32) | (uint64_t)c);
-      };
-      if (tid == 0) { s_ctl[2] = -1; }
+      // (draw, id)
+      if (tid == 0) s_ctl[2] = -1;
       csync();
       if (fits) {
         for (int i = tid; i < nb1; i += kConsumers) {
           const uint32_t ci = (uint32_t)s_cand[i];
           const uint64_t di = draw(ci);
           int rank = 0;
+#pragma unroll 1
           for (int j = 0; j < nb1; ++j) {
             const uint32_t cj = (uint32_t)s_cand[j];
             const uint64_t dj = draw(cj);
@@ -789,47 +860,49 @@ __device__ __noinline__ void scan_tail(const Geo& geo, const ScanArgs& A, int u,
           }
         }
       } else {
-        // a crowded bin: the krem-th smallest draw by repeated counting is
-        // too slow; take the exact radix refinement of the draws instead:
-        // 64-bit draws ranked by an 11/11/11/11/10/10 digit radix select
+        // a crowded bin: an exact radix select of the 64-bit draws
+        // (11/11/11/11/10/10-bit digits, smallest first), then ties in id order
         uint64_t prefix = 0, pmask = 0;
         int kr = krem;
-        const int shifts[6] = {53, 42, 31, 20, 10, 0};
-        const int bitsv[6] = {11, 11, 11, 11, 10, 10};
+#pragma unroll 1
         for (int pass = 0; pass < 6; ++pass) {
-          const int nb = 1 << bitsv[pass];
+          const int sh_ = pass < 4 ? 53 - 11 * pass : (pass == 4 ? 10 : 0);
+          const int nb = pass < 4 ? 2048 : 1024;
           for (int i = tid; i < kHistBins; i += kConsumers) s_hist[i] = 0;
           csync();
           for_rounds([&](int r) {
-#pragma unroll
+#pragma unroll 1
             for (int i = 0; i < kTailPT; ++i) {
-              if (rk[i] != 0u && (int)(rk[i] >> kHistShift) == bin1) {
+              const uint32_t key = key_at(i);
+              if (key != 0u && (int)(key >> kHistShift) == bin1) {
                 const uint64_t d = draw((uint32_t)(r * kTailRound + tid * kTailPT + i));
                 if ((d & pmask) == prefix)
-                  atomicAdd(&s_hist[(nb - 1) - (int)((d >> shifts[pass]) & (nb - 1))], 1);
+                  atomicAdd(&s_hist[(nb - 1) - (int)((d >> sh_) & (uint64_t)(nb - 1))], 1);
               }
             }
           });
           csync();
-          // smallest draws first: the histogram is filled reversed so that
-          // select_bin's "largest" is the smallest digit
+          // the histogram is filled reversed, so select_bin's largest bin is
+          // the smallest digit
           int ab;
-          const int dd = (nb - 1) - select_bin(s_hist, nb == 2048 ? 2048 : 1024, kr, &ab, s_sh, s_ctl);
+          const int dd = (nb - 1) - select_bin(s_hist, nb, kr, &ab, s_sh, s_ctl);
           kr -= ab;
-          prefix |= (uint64_t)dd << shifts[pass];
-          pmask |= (uint64_t)(nb - 1) << shifts[pass];
+          prefix |= (uint64_t)dd << sh_;
+          pmask |= (uint64_t)(nb - 1) << sh_;
         }
-        // the kr-th member (in id order) with draw == prefix
         if (tid == 0) s_ctl[2] = -1;
         csync();
         int run = 0;
         for_rounds([&](int r) {
           int f = 0, first = -1;
-#pragma unroll
+#pragma unroll 1
           for (int i = 0; i < kTailPT; ++i) {
             const uint32_t c = (uint32_t)(r * kTailRound + tid * kTailPT + i);
-            const bool m = rk[i] != 0u && (int)(rk[i] >> kHistShift) == bin1 && draw(c) == prefix;
-            if (m) { if (first < 0) first = (int)c; ++f; }
+            const uint32_t key = key_at(i);
+            if (key != 0u && (int)(key >> kHistShift) == bin1 && draw(c) == prefix) {
+              if (first < 0) first = (int)c;
+              ++f;
+            }
           }
           int t;
           const int incl = cscan(f, s_sh, &t);
@@ -844,34 +917,36 @@ __device__ __noinline__ void scan_tail(const Geo& geo, const ScanArgs& A, int u,
       hstar = ((uint64_t)(uint32_t)s_ctl[3] << 32) | (uint32_t)s_ctl[4];
       csync();
     } else {
-      // exact: refine the threshold bin by the key's lower digits (bits
-      // 20..10, then 9..0), then take the krem-th largest key's ties by id
+      // exact: refine the threshold bin by the key's bits 20..10, then
+      // 9..0, then take the krem-th largest key's ties in id order
       uint32_t prefix = (uint32_t)bin1 << kHistShift, pmask = 0xFFE00000u;
-      const int shifts[2] = {10, 0};
-      const int bitsv[2] = {11, 10};
+#pragma unroll 1
       for (int pass = 0; pass < 2; ++pass) {
-        const int nb = 1 << bitsv[pass];
+        const int sh_ = pass == 0 ? 10 : 0;
+        const int nb = pass == 0 ? 2048 : 1024;
         for (int i = tid; i < kHistBins; i += kConsumers) s_hist[i] = 0;
         csync();
         if (fits) {
           for (int i = tid; i < nb1; i += kConsumers) {
             const uint32_t key = (uint32_t)(s_cand[i] >> 32);
-            if ((key & pmask) == prefix) atomicAdd(&s_hist[(key >> shifts[pass]) & (nb - 1)], 1);
+            if ((key & pmask) == prefix) atomicAdd(&s_hist[(key >> sh_) & (nb - 1)], 1);
           }
         } else {
           for_rounds([&](int) {
-#pragma unroll
-            for (int i = 0; i < kTailPT; ++i)
-              if (rk[i] != 0u && (rk[i] & pmask) == prefix)
-                atomicAdd(&s_hist[(rk[i] >> shifts[pass]) & (nb - 1)], 1);
+#pragma unroll 1
+            for (int i = 0; i < kTailPT; ++i) {
+              const uint32_t key = key_at(i);
+              if (key != 0u && (key & pmask) == prefix)
+                atomicAdd(&s_hist[(key >> sh_) & (nb - 1)], 1);
+            }
           });
         }
         csync();
         int ab;
-        const int dd = select_bin(s_hist, nb == 2048 ? 2048 : 1024, krem, &ab, s_sh, s_ctl);
+        const int dd = select_bin(s_hist, nb, krem, &ab, s_sh, s_ctl);
         krem -= ab;
-        prefix |= (uint32_t)dd << shifts[pass];
-        pmask |= (uint32_t)(nb - 1) << shifts[pass];
+        prefix |= (uint32_t)dd << sh_;
+        pmask |= (uint32_t)(nb - 1) << sh_;
       }
       kstar = prefix;
       // the krem-th member (ascending id) with key == kstar
@@ -891,15 +966,15 @@ __device__ __noinline__ void scan_tail(const Geo& geo, const ScanArgs& A, int u,
         int run = 0;
         for_rounds([&](int r) {
           int f = 0;
-#pragma unroll
-          for (int i = 0; i < kTailPT; ++i) f += rk[i] == kstar;
+#pragma unroll 1
+          for (int i = 0; i < kTailPT; ++i) f += key_at(i) == kstar;
           int t;
           const int incl = cscan(f, s_sh, &t);
           if (f > 0 && run + incl - f < krem && run + incl >= krem) {
             int need = krem - (run + incl - f);
-#pragma unroll
+#pragma unroll 1
             for (int i = 0; i < kTailPT; ++i)
-              if (rk[i] == kstar && --need == 0) s_ctl[2] = r * kTailRound + tid * kTailPT + i;
+              if (key_at(i) == kstar && --need == 0) s_ctl[2] = r * kTailRound + tid * kTailPT + i;
           }
           run += t;
         });
@@ -914,30 +989,32 @@ __device__ __noinline__ void scan_tail(const Geo& geo, const ScanArgs& A, int u,
   // non-candidates), unless the estimation zone is empty
   const bool sampled = A.mode == 1 && k > 0 && k < n_cand;
   const Threshold th{kstar, thr, sampled ? 1 : 0, bin1, hstar, A.seed};
-  auto picked = [&](uint32_t key, uint32_t c) -> bool { return th.picked(key, c); };
   const bool no_est = A.exact_only || k == n_cand;
   int32_t* sel = A.sel + row0;
-  int32_t* tok = A.tok + geo.tok_row(b, h);
+  int32_t* tok = A.tok + tu.trow;
   int2* full = A.full + row0 + (int64_t)u * A.cap;
   int n_sel = 0, n_tok = 0;
   if (k > 0) {
     for_rounds([&](int r) {
       const int c0 = r * kTailRound + tid * kTailPT;
       int s = 0, t = 0;
-#pragma unroll
+#pragma unroll 1
       for (int i = 0; i < kTailPT; ++i)
-        if (picked(rk[i], (uint32_t)(c0 + i))) { ++s; t += ro[i + 1] - ro[i]; }
+        if (th.picked(key_at(i), (uint32_t)(c0 + i))) { ++s; t += cnt_at(i); }
       int2 tot2;
       const int2 inc = cscan2(make_int2(s, t), s_sh, &tot2);
       int ps = n_sel + inc.x - s, pt = n_tok + inc.y - t;
-#pragma unroll
-      for (int i = 0; i < kTailPT; ++i) {
-        if (picked(rk[i], (uint32_t)(c0 + i))) {
-          const int cnt = ro[i + 1] - ro[i];
+#pragma unroll 1
+      for (int i = 0; i < kTailPT && s > 0; ++i) {
+        if (th.picked(key_at(i), (uint32_t)(c0 + i))) {
+          const int cnt = cnt_at(i);
+          const int o0 = (int)srec[rpad(tid * kTailPT + i)].y;
           sel[ps] = c0 + i;
           if (!no_est) full[ps] = make_int2(c0 + i, cnt);
           ++ps;
-          for (int j = 0; j < cnt; ++j) tok[pt + j] = ro[i] + j;
+          --s;
+#pragma unroll 1
+          for (int j = 0; j < cnt; ++j) tok[pt + j] = o0 + j;
           pt += cnt;
         }
       }
@@ -968,7 +1045,8 @@ __device__ __noinline__ void scan_tail(const Geo& geo, const ScanArgs& A, int u,
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kScanThreads, 1)
-wave_scan_kernel(const Geo geo, const ChunkMap cm, const ScanArgs A,
+wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkMap cm,
+                 const __grid_constant__ ScanArgs A,
                  const __grid_constant__ CUtensorMap tm_cent,
                  const __grid_constant__ CUtensorMap tm_vsum, uint32_t* status) {
   using TS = TileShape<T, D>;
@@ -984,7 +1062,7 @@ wave_scan_kernel(const Geo geo, const ChunkMap cm, const ScanArgs A,
   const int slots = A.slots;
   const size_t slot_bytes = SM::slot_bytes(A.exact_only);
   unsigned char* ring = sh;
-  unsigned char* s_union = ring + slots * slot_bytes;
+  unsigned char* s_union = ring + SM::ring_bytes(slots, A.exact_only);
   uint32_t* hist16 = reinterpret_cast<uint32_t*>(s_union + SM::kUnion);
   RowMult* s_rows = reinterpret_cast<RowMult*>(reinterpret_cast<unsigned char*>(hist16) + SM::kHist16);
   float* s_sc = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(s_rows) + SM::kRows);
@@ -1165,8 +1243,8 @@ wave_scan_kernel(const Geo geo, const ChunkMap cm, const ScanArgs A,
     }
     if (unit_end) {
       if (!A.exact_only) {
-        if constexpr (kMma) macc.to_smem(comb + warp * G * (D + 2));
-        else facc.to_smem(comb + warp * G * (D + 2));
+        if constexpr (kMma) macc.to_smem(comb + warp * G * (D + kPartStride));
+        else facc.to_smem(comb + warp * G * (D + kPartStride));
         csync();
         const int slot = s - cm.cta_of(cm.first(c.b, c.h));
         float* part = A.est + ((int64_t)c.u * A.p1max + slot) * G * (D + kPartStride);
@@ -1188,7 +1266,9 @@ wave_scan_kernel(const Geo geo, const ChunkMap cm, const ScanArgs A,
   csync();
   const int nt = s_ntails;
   for (int t = 0; t < nt; ++t) {
-    scan_tail(geo, A, s_tails[t], s_union, status);
+    const int u = s_tails[t], b = u / geo.hkv, h = u - b * geo.hkv;
+    const TailUnit tu{u, geo.NC(b), geo.T(b), geo.cl_row(b, h), geo.tok_row(b, h)};
+    scan_tail(tu, A, s_union, reinterpret_cast<uint2*>(ring), status);
     csync();
   }
   pdl_wait();
@@ -1230,17 +1310,20 @@ struct GatherSmem {
   static constexpr int kRowsPerBlock = kGatherTiles * kTileRows;
   static constexpr size_t kTiles = (size_t)2 * kGatherTiles * TS::kBytes;   // K and V
   static constexpr size_t kMeta = (size_t)kRowsPerBlock * (8 + 8 + 4 + 4);
-  static constexpr size_t kComb = (size_t)kConsumerWarps * G * (D + 2) * 4;
+  static constexpr size_t kComb = (size_t)kConsumerWarps * G * (D + kPartStride) * 4;
   static constexpr size_t kRows = (size_t)kConsumerWarps * 8 * sizeof(RowMult);
   static constexpr size_t kSc = (size_t)kConsumerWarps * 8 * G * 4;
-  static constexpr size_t kMergeParts = 256;   // parts whose (m, l) are staged per pass
-  static constexpr size_t kMerge = kMergeParts * G * 2 * 4 + (size_t)G * 8;
-  static constexpr size_t kTotal = 1024 + kTiles + kMeta + kComb + kRows + kSc + kMerge;
+  static constexpr size_t kMergeParts = kMaxGatherPerUnit;   // parts a unit's merge reads
+  static constexpr size_t kMerge = (kMergeParts * G * 3 * 4 + (size_t)G * 8 + 15) / 16 * 16;
+  static constexpr size_t kPart = (size_t)G * (D + kPartStride) * 4;   // s_part, s_pre
+  static constexpr size_t kTotal = 1024 + kTiles + kMeta + kComb + kRows + kSc + kMerge +
+                                   2 * kPart + (size_t)G * 8;
 };
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kGatherThreads, 2)
-wave_gather_kernel(const Geo geo, const ChunkMap cm, const GatherArgs A, uint32_t* status) {
+wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkMap cm,
+                   const __grid_constant__ GatherArgs A, uint32_t* status) {
   using TS = TileShape<T, D>;
   using SM = GatherSmem<T, D, G>;
   constexpr bool kMma = std::is_same_v<T, __nv_bfloat16>;
@@ -1258,6 +1341,9 @@ wave_gather_kernel(const Geo geo, const ChunkMap cm, const GatherArgs A, uint32_
   RowMult* s_rows = reinterpret_cast<RowMult*>(reinterpret_cast<unsigned char*>(comb) + SM::kComb);
   float* s_sc = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(s_rows) + SM::kRows);
   float* s_merge = s_sc + kConsumerWarps * 8 * G;
+  float* s_part = s_merge + SM::kMerge / 4;                  // [G][D + 4] this CTA's part
+  float* s_pre = s_part + SM::kPart / 4;                     // [G][D + 4] a prefetched scan part
+  float* s_fac = s_pre + SM::kPart / 4;                      // [G][2] fold factors
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   // CTA -> (sequence b, KV head h, index j of the unit's n2 CTAs)
@@ -1290,6 +1376,15 @@ wave_gather_kernel(const Geo geo, const ChunkMap cm, const GatherArgs A, uint32_
   if (tid < RPB && j * RPB + tid < Tb) spec = __ldcg(A.tok + trow + j * RPB + tid);
   __syncthreads();
   const bool dense = s_rec[kDense] != 0, no_est = s_rec[kNoEstimate] != 0;
+  // the scan's estimation parts this CTA folds into its own (p = j, j + n2,
+  // ...): the first one's copies go out now, to land during the gather
+  const int np1 = no_est ? 0 : cm.parts(b, h);
+  if (np1 > j) {
+    const float* src = A.est + ((int64_t)u * A.p1max + j) * G * (D + kPartStride);
+    for (int x = tid; x < G * (D + kPartStride) / 4; x += blockDim.x)
+      cp_async16(s_pre + 4 * x, src + 4 * x);
+    cp_async_commit();
+  }
   const int n_tok = dense ? 0 : s_rec[kSelTokens];
   const int n_st = s_rec[kSteady];
   const int n_full = (dense || no_est) ? 0 : s_rec[kFullRows];
@@ -1374,7 +1469,7 @@ wave_gather_kernel(const Geo geo, const ChunkMap cm, const GatherArgs A, uint32_
     cp_async_wait<0>();
     __syncthreads();
     // ---- attend: warp w takes rows 8w .. 8w + 7 of each tile
-#pragma unroll
+#pragma unroll 1
     for (int t = 0; t < kGatherTiles; ++t) {
       const int lr = t * kTileRows + 8 * warp;    // block-local row of the warp's first
       RowMult* rm = s_rows + warp * 8;
@@ -1411,12 +1506,43 @@ wave_gather_kernel(const Geo geo, const ChunkMap cm, const GatherArgs A, uint32_
     }
     __syncthreads();   // tiles and row data are read before the next block
   }
-  // ---- this CTA's part, then the unit's merge by its last CTA
-  if constexpr (kMma) macc.to_smem(comb + warp * G * (D + 2));
-  else facc.to_smem(comb + warp * G * (D + 2));
+  // ---- this CTA's part (its rows, plus its share of the scan's estimation
+  // parts: p = j, j + n2, ...), then the unit's merge by its last CTA
+  if constexpr (kMma) macc.to_smem(comb + warp * G * (D + kPartStride));
+  else facc.to_smem(comb + warp * G * (D + kPartStride));
   __syncthreads();
+  combine_warps<D, G>(comb, s_part, tid);
+  __syncthreads();
+  auto fold_part = [&](const float* src) {   // s_part <- s_part (+) src (shared or global)
+    if (tid < G) {
+      const float ma = s_part[tid * (D + kPartStride)], mb = src[tid * (D + kPartStride)];
+      const float M = fmaxf(ma, mb);
+      const float fa = ma == -INFINITY ? 0.f : expf(ma - M);
+      const float fb = mb == -INFINITY ? 0.f : expf(mb - M);
+      s_fac[2 * tid] = fa;
+      s_fac[2 * tid + 1] = fb;
+      float* row = s_part + tid * (D + kPartStride);
+      row[0] = M;
+      row[1] = row[1] * fa + src[tid * (D + kPartStride) + 1] * fb;
+      row[2] = row[2] * fa + src[tid * (D + kPartStride) + 2] * fb;
+    }
+    __syncthreads();
+    for (int i = tid; i < G * D; i += blockDim.x) {
+      const int gg = i / D, e = i - gg * D;
+      float* o = s_part + gg * (D + kPartStride) + kPartStride + e;
+      *o = *o * s_fac[2 * gg] + src[gg * (D + kPartStride) + kPartStride + e] * s_fac[2 * gg + 1];
+    }
+    __syncthreads();
+  };
+  if (np1 > j) {
+    cp_async_wait<0>();   // the prefetched part (its copies were issued after the grid wait)
+    __syncthreads();
+    fold_part(s_pre);
+    for (int p = j + n2; p < np1; p += n2)
+      fold_part(A.est + ((int64_t)u * A.p1max + p) * G * (D + kPartStride));
+  }
   float* part = A.gat + ((int64_t)u * A.n2max + j) * G * (D + kPartStride);
-  combine_warps<D, G>(comb, part, tid);
+  for (int i = tid; i < G * (D + kPartStride); i += blockDim.x) part[i] = s_part[i];
   __threadfence();
   __syncthreads();
   if (tid == 0) {
@@ -1426,49 +1552,83 @@ wave_gather_kernel(const Geo geo, const ChunkMap cm, const GatherArgs A, uint32_
   }
   __syncthreads();
   if (!s_last) return;
-  // parts: the scan's (unless the estimation zone is empty), then the gather's
-  const int np1 = no_est ? 0 : cm.parts(b, h);
-  const int np = np1 + n2;
+  // the merge of the unit's n2 parts: their (m, l, ln) first, then their
+  // outputs, staged in shared memory by asynchronous copies in batches of
+  // the tile area's size
+  const int np = n2;
   auto part_ptr = [&](int p) -> const float* {
-    return p < np1 ? A.est + ((int64_t)u * A.p1max + p) * G * (D + kPartStride)
-                   : A.gat + ((int64_t)u * A.n2max + (p - np1)) * G * (D + kPartStride);
+    return A.gat + ((int64_t)u * A.n2max + p) * G * (D + kPartStride);
   };
-  float* s_f = s_merge;                             // [kMergeParts][G] (m, l) then factor
-  float* s_M = s_merge + SM::kMergeParts * G * 2;   // [G] max, [G] denominator
+  float* s_f = s_merge;                             // [kMergeParts][G] (m then factor, l, ln)
+  float* s_M = s_merge + SM::kMergeParts * G * 3;   // [G] max, [G] denominator
   float* s_L = s_M + G;
   for (int x = tid; x < np * G; x += blockDim.x) {
     const int p = x / G, gg = x - p * G;
     const float* pp = part_ptr(p) + gg * (D + kPartStride);
-    s_f[2 * x] = __ldcg(pp);
-    s_f[2 * x + 1] = __ldcg(pp + 1);
+    s_f[3 * x] = __ldcg(pp);
+    s_f[3 * x + 1] = __ldcg(pp + 1);
+    s_f[3 * x + 2] = __ldcg(pp + 2);
   }
   __syncthreads();
   if (warp < G) {   // warp g: head g's max, the parts' factors, the denominator
     float M = -INFINITY;
-    for (int p = lane; p < np; p += 32) M = fmaxf(M, s_f[2 * (p * G + warp)]);
+    for (int p = lane; p < np; p += 32) M = fmaxf(M, s_f[3 * (p * G + warp)]);
     M = warp_max(M);
-    float L = 0.f;
+    float L = 0.f, LN = 0.f;
     for (int p = lane; p < np; p += 32) {
-      const float mp = s_f[2 * (p * G + warp)];
+      const float mp = s_f[3 * (p * G + warp)];
       const float f = mp == -INFINITY ? 0.f : expf(mp - M);
-      L += f * s_f[2 * (p * G + warp) + 1];
-      s_f[2 * (p * G + warp)] = f;
+      L += f * s_f[3 * (p * G + warp) + 1];
+      LN += f * s_f[3 * (p * G + warp) + 2];
+      s_f[3 * (p * G + warp)] = f;
     }
     L = warp_sum(L);
-    if (lane == 0) { s_M[warp] = M; s_L[warp] = L; }
-  }
-  __syncthreads();
-  for (int i = tid; i < G * D; i += blockDim.x) {
-    const int gg = i / D, e = i - gg * D;
-    float O = 0.f;
-    for (int p = 0; p < np; ++p) {
-      const float f = s_f[2 * (p * G + gg)];
-      if (f != 0.f) O += f * __ldcg(part_ptr(p) + gg * (D + kPartStride) + kPartStride + e);
+    LN = warp_sum(LN);
+    if (lane == 0) {
+      s_M[warp] = M;
+      s_L[warp] = L;
+      // the estimate is "every cluster minus what the zone leaves out": the
+      // mass taken back out stays within the merged denominator when every
+      // centroid is the mean of its members (Jensen); far above it, the
+      // difference has lost its precision, and the call says so
+      if (LN > kCancelRatio * fmaxf(L, 0.f)) flag_error(status, WI_DEV_CANCELLATION);
     }
-    const float L = s_L[gg];
-    const int64_t qh = (int64_t)b * A.Hq + (int64_t)h * G + gg;
-    A.out[qh * D + e] = L > 0.f ? O / L : 0.f;
-    if (e == 0 && A.lse) A.lse[qh] = L > 0.f ? s_M[gg] + logf(L) : -INFINITY;
+  }
+  constexpr int kPS = G * (D + kPartStride);          // floats per part
+  constexpr int PB = (int)(SM::kTiles / (kPS * 4));   // parts per staged batch
+  float* stage = reinterpret_cast<float*>(tiles);
+  constexpr int kOut = (G * D + kGatherThreads - 1) / kGatherThreads;
+  float O[kOut];
+#pragma unroll
+  for (int k = 0; k < kOut; ++k) O[k] = 0.f;
+  for (int p0 = 0; p0 < np; p0 += PB) {
+    const int nb = min(PB, np - p0);
+    __syncthreads();   // the previous batch (and the factors) are read
+    for (int x = tid; x < nb * kPS / 4; x += blockDim.x)
+      cp_async16(stage + 4 * x, part_ptr(p0) + 4 * x);   // parts of a unit are contiguous
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kOut; ++k) {
+      const int i = tid + k * kGatherThreads;
+      if (i < G * D) {
+        const int gg = i / D, e = i - gg * D;
+        for (int p = 0; p < nb; ++p)
+          O[k] += s_f[3 * ((p0 + p) * G + gg)] * stage[p * kPS + gg * (D + kPartStride) + kPartStride + e];
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kOut; ++k) {
+    const int i = tid + k * kGatherThreads;
+    if (i < G * D) {
+      const int gg = i / D, e = i - gg * D;
+      const float L = s_L[gg];
+      const int64_t qh = (int64_t)b * A.Hq + (int64_t)h * G + gg;
+      A.out[qh * D + e] = L > 0.f ? O[k] / L : 0.f;
+      if (e == 0 && A.lse) A.lse[qh] = L > 0.f ? s_M[gg] + logf(L) : -INFINITY;
+    }
   }
   if (tid == 0) A.cnt2[u] = 0;   // clean for the next call
 }

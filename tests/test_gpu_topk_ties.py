@@ -2,15 +2,22 @@
 threshold (Vortex summary, section 2.C Top-K; reading R-6: equal scores go
 to the lower cluster id).
 
-The index is a block index (position blocks, perm the identity) whose
-centroids are then overwritten with multiples a_j * u of one vector u, the
-group's first query head: every query head of the group scores cluster j as
-a_j * (q_g . u) / sqrt(d), so clusters with the same a_j score exactly
-alike, in fp32 on the GPU as in fp64 in the oracle, and a larger a_j always
-scores higher.  Each case places the k-th score inside a run of exactly equal
-scores; the retrieved set must then equal the oracle's exactly, with no
-near-tie slack.  The clusters whose members all lie in the steady window get
-the highest a_j of all: they are not candidates and must not be retrieved.
+The index is a block index (position blocks, perm the identity) of keys
+that are multiples a_j * u of one vector u, the group's first query head,
+the same for every token of block j, so block j's centroid is a_j * u too:
+every query head of the group scores cluster j as a_j * (q_g . u) / sqrt(d),
+so clusters with the same a_j score exactly alike, in fp32 on the GPU as in
+fp64 in the oracle, and a larger a_j always scores higher.  Each case places
+the k-th score inside a run of exactly equal scores; the retrieved set must
+then equal the oracle's exactly, with no near-tie slack.  The clusters whose
+members all lie in the steady window get the highest a_j of all: they are
+not candidates and must not be retrieved.
+
+The last test overwrites the centroids of such an index with values that are
+not their members' means: the decode takes its estimation zone as "every
+cluster minus what the zone leaves out", which stays precise only while a
+cluster's estimated mass is bounded by its members' exact mass (Jensen, true
+of every built index), and must report the violation in its status word.
 """
 import numpy as np
 import pytest
@@ -25,10 +32,12 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def tied_index(n_top, n_tied, seed):
+def tied_index(n_top, n_tied, seed, consistent=True):
     """One sequence of 65536 tokens, 2 KV heads, G = 4, d = 128, blocks of 16
-    (4096 clusters per head).  Clusters 0..n_top-1 (spread over the ids) get
-    distinct high scores, n_tied others one shared score, the rest a low one."""
+    (4096 clusters per head).  n_top clusters (spread over the ids) get
+    distinct high scores, n_tied others one shared score, the rest a low one.
+    consistent: the keys of block j are all a_j * u (so its centroid is the
+    mean of its keys); otherwise only the centroids are a_j * u."""
     wl = WI.mixture_workload("ties", seq_lens=[65536], n_q_heads=8, n_kv_heads=2, head_dim=128,
                              n_centers=64, seg_len=1024, cluster_size=16, iters=1,
                              topk_clusters=148, seed=seed, device=DEV)
@@ -38,8 +47,7 @@ def tied_index(n_top, n_tied, seed):
     rng = np.random.default_rng(seed)
     units = {}
     for h in range(2):
-        ix = O.build_blocks_unit(keys[0][h], vals[0][h], wl.seg_len, wl.cluster_size, "bf16")
-        NC = len(ix.centroids)
+        NC = 65536 // wl.cluster_size
         u = qh[0, 4 * h]                              # bf16 values of the group's first head
         assert np.max(qh[0, 4 * h:4 * h + 4] @ u) > 0
         ids = rng.permutation(NC - 4)                 # the last 4 blocks are all steady
@@ -47,7 +55,13 @@ def tied_index(n_top, n_tied, seed):
         a[ids[:n_top]] = 2.0 + np.arange(n_top) / 64.0    # above the tied run
         a[ids[n_top:n_top + n_tied]] = 1.0
         a[NC - 4:] = 4.0                              # best scores, but not candidates
-        ix.centroids = O.round_bf16(a[:, None] * u[None, :])
+        cent = O.round_bf16(a[:, None] * u[None, :])
+        K = np.repeat(cent, wl.cluster_size, axis=0) if consistent else keys[0][h]
+        ix = O.build_blocks_unit(K, vals[0][h], wl.seg_len, wl.cluster_size, "bf16")
+        if consistent:
+            assert np.array_equal(ix.centroids, cent)
+        else:
+            ix.centroids = cent
         units[(0, h)] = ix
     H.upload_index(wx, units)
     return wl, wx, units
@@ -75,3 +89,13 @@ def test_ties_at_the_kth_score_go_to_the_lower_id(n_top, n_tied):
         assert H.rel_err(og, tr.out, wl.dtype) <= 2e-4
         np.testing.assert_allclose(lse[0, 4 * h:4 * h + 4].cpu().numpy(), tr.lse, rtol=2e-6,
                                    atol=2e-5)
+
+
+def test_centroids_far_from_their_members_are_reported():
+    wl, wx, units = tied_index(100, 60, seed=5, consistent=False)
+    p = H.params_of(wl)
+    ws = W.decode_workspace(wx, p)
+    W.decode(wl.q.to(DEV), wx, p, ws=ws)
+    flags = W.read_device_status(ws)
+    assert flags & W.WI_DEV_CANCELLATION
+    assert not flags & ~W.WI_DEV_CANCELLATION

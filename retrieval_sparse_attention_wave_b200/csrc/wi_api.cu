@@ -177,8 +177,10 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
       }
     }
   }
-  const size_t slot = decode_scan_slot_bytes(pl.dtype, pl.D, pl.exact_only);
-  pl.slots = (int)std::max<size_t>(2, std::min<size_t>(4, (size_t)131072 / slot));
+  // ring slots: tile(s) plus the side area (offsets box, queries); about
+  // 144 KB of them, 2 to 4
+  const size_t slot = decode_scan_slot_bytes(pl.dtype, pl.D, G, pl.exact_only);
+  pl.slots = (int)std::max<size_t>(2, std::min<size_t>(4, (size_t)147456 / slot));
   if (decode_scan_smem(pl.dtype, pl.D, G, pl.slots, pl.exact_only) > 227 * 1024)
     return WI_ERR_UNSUPPORTED;
   if (decode_gather_smem(pl.dtype, pl.D, G) > 227 * 1024) return WI_ERR_UNSUPPORTED;

@@ -261,6 +261,15 @@ __device__ __forceinline__ void tensor_load_2d(void* smem, const void* tmap, int
       "r"(smem_addr(bar)) : "memory");
 }
 
+// 1-D tiled bulk copy through a tensor map (box at element coordinate x;
+// x * element size a multiple of 16 bytes)
+__device__ __forceinline__ void tensor_load_1d(void* smem, const void* tmap, int x, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2}], [%3];" ::"r"(smem_addr(smem)), "l"(tmap), "r"(x), "r"(smem_addr(bar))
+      : "memory");
+}
+
 // ---- warp-level bf16 tensor-core fragments (m16n8k16, fp32 accumulate)
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* smem) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"

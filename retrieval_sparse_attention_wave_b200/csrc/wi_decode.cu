@@ -51,9 +51,13 @@ size_t decode_scan_smem(int dtype, int D, int G, int slots, int exact_only) {
   return r;
 }
 
-size_t decode_scan_slot_bytes(int dtype, int D, int exact_only) {
-  const size_t tile = (size_t)kTileRows * D * (dtype == WI_BF16 ? 2 : 4);
-  return tile * (exact_only ? 1 : 2);
+size_t decode_scan_slot_bytes(int dtype, int D, int G, int exact_only) {
+  size_t r = 0;
+  with_types(dtype, D, G, [&]<typename T, int DD, int GG>() -> cudaError_t {
+    r = ScanSmem<T, DD, GG>::tile_bytes(exact_only) + ScanSmem<T, DD, GG>::kSide;
+    return cudaSuccess;
+  });
+  return r;
 }
 
 size_t decode_gather_smem(int dtype, int D, int G) {

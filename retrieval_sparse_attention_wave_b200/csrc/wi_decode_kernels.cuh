@@ -141,8 +141,8 @@ struct MmaAcc {
     const uint32_t* qw = reinterpret_cast<const uint32_t*>(q_group + (g < G ? g : 0) * D);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
-      qa0[ks] = g < G ? __ldg(qw + 8 * ks + tq) : 0u;
-      qa2[ks] = g < G ? __ldg(qw + 8 * ks + 4 + tq) : 0u;
+      qa0[ks] = g < G ? qw[8 * ks + tq] : 0u;
+      qa2[ks] = g < G ? qw[8 * ks + 4 + tq] : 0u;
     }
   }
   __device__ __forceinline__ void reset() {
@@ -234,7 +234,7 @@ struct FmaAcc {
     const int sub = (threadIdx.x & 31) % LPR;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(q_group + g * D) + sub);
+      const float4 v = reinterpret_cast<const float4*>(q_group + g * D)[sub];
       qv[g][0] = v.x * scale; qv[g][1] = v.y * scale; qv[g][2] = v.z * scale; qv[g][3] = v.w * scale;
     }
   }
@@ -501,7 +501,6 @@ wave_steady_kernel(const Geo geo, const SteadyArgs a, uint32_t* status) {
 struct ScanArgs {
   const void* q;
   int Hq;
-  const int32_t* offsets;
   uint2* rec;            // [ncl] {selection key (0: not a candidate), first slot}
   int32_t* hist;         // [U][kHistBins] first-digit histogram (zero between calls)
   int32_t* cnt1;         // [U] arrivals (zero between calls)
@@ -524,32 +523,89 @@ struct ScanArgs {
   int slots;
 };
 
-constexpr int kTailPT = 32;                    // records per consumer per round
-constexpr int kTailRound = kConsumers * kTailPT;
-// A round's records (and one more, for the last one's count) sit in shared
-// memory with one pad slot per 32, so a consumer's run of 32 consecutive
-// records falls on distinct banks.
-__device__ __forceinline__ int rpad(int i) { return i + (i >> 5); }
-constexpr size_t kTailRecBytes = (size_t)(kTailRound + 1 + kTailRound / 32 + 1) * 8;
+// A chunk's offsets arrive as one 1-D tensor box of kOffBox int32 that starts
+// at the entry of the chunk's first cluster rounded down to a multiple of 4
+// (16 bytes): the chunk's kTileRows + 1 entries sit at box index
+// (first entry) % 4.
+constexpr int kOffBox = 72;
+constexpr int kOffArea = 512;   // bytes of a slot's side area before its queries
 
-// Shared memory of a scan CTA (bytes, after 1024-byte alignment).
+// Position of a scan chunk: its unit and first cluster.  Consecutive chunks
+// of one unit advance by kTileRows clusters; the kernel parameters are read
+// again only when a chunk starts another unit.
+struct ChunkPos {
+  int k;            // chunk index
+  int b, h, u;
+  int c0, nrows;    // first cluster in the unit, rows in the chunk
+  int NC;           // clusters of the unit
+  int kend;         // one past the unit's last chunk
+  int64_t row0;     // centroid row of the unit's cluster 0
+  int64_t orow;     // offsets entry of the unit's cluster 0
+};
+__device__ __forceinline__ void chunk_seek(ChunkPos& p, const Geo& geo, const ChunkMap& cm, int k) {
+  p.k = k;
+  p.b = cm.seq_of(k);
+  const int per = cm.per_unit(p.b);
+  const int rel = k - cm.ch_base[p.b];
+  p.h = rel / per;
+  p.c0 = (rel - p.h * per) * kTileRows;
+  p.u = p.b * geo.hkv + p.h;
+  p.NC = geo.NC(p.b);
+  p.kend = cm.ch_base[p.b] + (p.h + 1) * per;
+  p.row0 = geo.cl_row(p.b, p.h);
+  p.orow = geo.off_row(p.b, p.h);
+  p.nrows = min(kTileRows, p.NC - p.c0);
+}
+__device__ __forceinline__ void chunk_next(ChunkPos& p, const Geo& geo, const ChunkMap& cm) {
+  if (p.k + 1 < p.kend) {
+    ++p.k;
+    p.c0 += kTileRows;
+    p.nrows = min(kTileRows, p.NC - p.c0);
+  } else {
+    chunk_seek(p, geo, cm, p.k + 1);
+  }
+}
+
+constexpr int kTailSteps = 32;                       // records per consumer lane and round
+constexpr int kTailRound = kConsumers * kTailSteps;  // 8192 records per round
+constexpr int kTailDraws = 256;                      // threshold bins ranked member by member
+// a round of records (and the next one) staged in shared memory, one pad
+// record per 32 (the ring, once the chunks are done)
+constexpr size_t kTailStage = ((size_t)(kTailRound + kTailRound / 32 + 2) * 8 + 1023) / 1024 * 1024;
+// the ring keeps the slots' side areas (tensor-copy destinations) 128-byte
+// aligned and the tiles 1024-byte aligned
+static_assert(kTailStage % 1024 == 0, "record stage must keep the ring 1024-byte aligned");
+
+// Shared memory of a scan CTA (bytes, after 1024-byte alignment): the ring of
+// tiles (also the tail's record stage), each slot's side area (offsets box,
+// the unit's queries), and a union of the per-warp softmax parts and the
+// tail's work areas.
 template <typename T, int D, int G>
 struct ScanSmem {
   using TS = TileShape<T, D>;
+  static constexpr size_t kQBytes = (size_t)G * D * sizeof(T);
+  static constexpr size_t kSide = kOffArea + (kQBytes + 127) / 128 * 128;
+  static_assert(kSide % 128 == 0 && TS::kBytes % 1024 == 0, "slot areas keep tensor-copy alignment");
   static constexpr size_t kComb = (size_t)kConsumerWarps * G * (D + kPartStride) * 4;
-  static constexpr size_t kTail = (size_t)kHistBins * 4 + (size_t)kTailCand * 8 + 1024;
+  // tail: histogram, threshold-bin members, their draws, scan scratch and
+  // control words
+  static constexpr size_t kTailHist = 0;
+  static constexpr size_t kTailCandOff = kTailHist + (size_t)kHistBins * 4;
+  static constexpr size_t kTailDrawOff = kTailCandOff + (size_t)kTailCand * 8;
+  static constexpr size_t kTailShOff = kTailDrawOff + (size_t)kTailDraws * 8;
+  static constexpr size_t kTail = kTailShOff + 512;
   static constexpr size_t kUnion = kComb > kTail ? kComb : kTail;
   static constexpr size_t kHist16 = (size_t)kHistBins / 2 * 4;
   static constexpr size_t kRows = (size_t)kConsumerWarps * 8 * sizeof(RowMult);
   static constexpr size_t kSc = (size_t)kConsumerWarps * 8 * G * 4;
-  __host__ __device__ static size_t slot_bytes(int exact_only) { return (size_t)TS::kBytes * (exact_only ? 1 : 2); }
-  // the ring, which the tails reuse for their records once the chunks are done
+  __host__ __device__ static size_t tile_bytes(int exact_only) { return (size_t)TS::kBytes * (exact_only ? 1 : 2); }
   __host__ __device__ static size_t ring_bytes(int slots, int exact_only) {
-    const size_t r = slots * slot_bytes(exact_only);
-    return r > kTailRecBytes ? r : (kTailRecBytes + 1023) / 1024 * 1024;
+    const size_t r = slots * tile_bytes(exact_only);
+    return r > kTailStage ? r : kTailStage;
   }
+  __host__ __device__ static size_t side_bytes(int slots) { return slots * kSide; }
   __host__ __device__ static size_t total(int slots, int exact_only) {
-    return 1024 + ring_bytes(slots, exact_only) + kUnion + kHist16 + kRows + kSc;
+    return 1024 + ring_bytes(slots, exact_only) + side_bytes(slots) + kUnion + kHist16 + kRows + kSc;
   }
 };
 
@@ -590,32 +646,23 @@ __device__ __forceinline__ int cscan(int x, int* sh, int* total) {
   return r;
 }
 
-// inclusive scan of two ints per consumer; *total the sums.  sh: 64 ints.
-__device__ __forceinline__ int2 cscan2(int2 x, int* sh, int2* total) {
+// Exclusive prefix over the consumer warps of a warp-uniform pair of values;
+// *total the sums.  sh: 16 ints.
+__device__ __forceinline__ int2 wscan2(int2 v, int* sh, int2* total) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int ya = __shfl_up_sync(0xffffffffu, x.x, o);
-    const int yb = __shfl_up_sync(0xffffffffu, x.y, o);
-    if (lane >= o) { x.x += ya; x.y += yb; }
-  }
-  if (lane == 31) { sh[w] = x.x; sh[32 + w] = x.y; }
+  if (lane == 0) { sh[w] = v.x; sh[8 + w] = v.y; }
   csync();
-  if (w == 0) {
-    int a = lane < kConsumerWarps ? sh[lane] : 0, c = lane < kConsumerWarps ? sh[32 + lane] : 0;
+  int2 base = make_int2(0, 0), t = make_int2(0, 0);
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int ya = __shfl_up_sync(0xffffffffu, a, o);
-      const int yc = __shfl_up_sync(0xffffffffu, c, o);
-      if (lane >= o) { a += ya; c += yc; }
-    }
-    if (lane < kConsumerWarps) { sh[lane] = a; sh[32 + lane] = c; }
+  for (int i = 0; i < kConsumerWarps; ++i) {
+    const int a = sh[i], c = sh[8 + i];
+    if (i < w) { base.x += a; base.y += c; }
+    t.x += a;
+    t.y += c;
   }
   csync();
-  const int2 r = make_int2(x.x + (w > 0 ? sh[w - 1] : 0), x.y + (w > 0 ? sh[32 + w - 1] : 0));
-  *total = make_int2(sh[kConsumerWarps - 1], sh[32 + kConsumerWarps - 1]);
-  csync();
-  return r;
+  *total = t;
+  return base;
 }
 
 // Whether cluster c (selection key `key`, 0 for a non-candidate) is
@@ -672,13 +719,57 @@ __device__ __forceinline__ int select_bin(const int* hist, int nb, int krem, int
   return r;
 }
 
-
 // The unit's geometry, passed to the tail as scalars (the 2 KB Geo would be
 // copied to local memory for a call).
 struct TailUnit {
   int u, NC, Tb;
   int64_t row0, trow;
 };
+
+// Records of a round as staged in shared memory: record i (round-relative)
+// at i + i / 32, so consumer thread t reads its 32 consecutive records
+// 32 t .. 32 t + 31 without bank conflicts.
+__device__ __forceinline__ int rpad(int i) { return i + (i >> 5); }
+
+// Stage round r of a unit's records in shared memory (record r kTailRound +
+// i; past the unit: key 0, first slot T_b; and the record after the round,
+// for the last count).  Loads of 8 records per thread are in flight at once.
+__device__ __forceinline__ void stage_round(const uint2* rec, int NC, int Tb, int r, uint2* stage) {
+  const int tid = threadIdx.x;
+  const int c0 = r * kTailRound;
+  csync();   // the previous round's readers are done
+#pragma unroll 1
+  for (int q0 = 0; q0 < kTailSteps; q0 += 8) {
+    uint2 v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int c = c0 + tid + (q0 + q) * kConsumers;
+      v[q] = c < NC ? __ldcg(rec + c) : make_uint2(0u, (uint32_t)Tb);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) stage[rpad(tid + (q0 + q) * kConsumers)] = v[q];
+  }
+  if (tid == 0)
+    stage[rpad(kTailRound)] =
+        make_uint2(0u, c0 + kTailRound < NC ? __ldcg(&rec[c0 + kTailRound].y) : (uint32_t)Tb);
+  csync();
+}
+
+// Exclusive prefix over the consumer threads of a pair of values (thread
+// order); *total the sums.  sh: 16 ints.
+__device__ __forceinline__ int2 cscan2_excl(int2 v, int* sh, int2* total) {
+  const int lane = threadIdx.x & 31;
+  int2 x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ya = __shfl_up_sync(0xffffffffu, x.x, o);
+    const int yb = __shfl_up_sync(0xffffffffu, x.y, o);
+    if (lane >= o) { x.x += ya; x.y += yb; }
+  }
+  const int2 wtot = make_int2(__shfl_sync(0xffffffffu, x.x, 31), __shfl_sync(0xffffffffu, x.y, 31));
+  const int2 wb = wscan2(wtot, sh, total);
+  return make_int2(wb.x + x.x - v.x, wb.y + x.y - v.y);
+}
 
 // The tail of unit u (by the last scan CTA to finish it): the exact top-k
 // threshold (kstar, thr) -- cluster c is retrieved iff its key > kstar, or
@@ -688,106 +779,101 @@ struct TailUnit {
 // retrieved ids, their token slots and the clusters whose estimate the
 // gather takes back out.
 //
-// Its passes are rolled loops over the records in shared memory.
+// A round of kTailRound records at a time is staged in shared memory, and
+// consumer thread t walks records 32 t .. 32 t + 31, so thread order is id
+// order: every pass is one short loop per thread and one block-wide prefix
+// sum.  The tail runs once per unit on one CTA: its cost is its chains of
+// dependent shuffles and shared loads and the fetch of its instructions, so
+// its loops stay rolled and its code small.
 __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, unsigned char* sh,
-                                       uint2* srec, uint32_t* status) {
+                                          unsigned char* stage_bytes, size_t cand_off,
+                                          size_t draw_off, size_t sh_off, uint32_t* status) {
   const int u = tu.u, NC = tu.NC, Tb = tu.Tb;
   const int tid = threadIdx.x;
-  int* s_hist = reinterpret_cast<int*>(sh);                                   // [2048]
-  unsigned long long* s_cand = reinterpret_cast<unsigned long long*>(sh + kHistBins * 4);  // [kTailCand]
-  int* s_sh = reinterpret_cast<int*>(sh + kHistBins * 4 + kTailCand * 8);     // [64]
-  int* s_ctl = s_sh + 64;                                                     // [16]
-  const int64_t row0 = tu.row0;
-  uint2* rec = A.rec + row0;
+  int* s_hist = reinterpret_cast<int*>(sh);                                         // [2048]
+  unsigned long long* s_cand = reinterpret_cast<unsigned long long*>(sh + cand_off); // [kTailCand]
+  unsigned long long* s_draw = reinterpret_cast<unsigned long long*>(sh + draw_off); // [kTailDraws]
+  int* s_sh = reinterpret_cast<int*>(sh + sh_off);                                   // [64]
+  int* s_ctl = s_sh + 64;                                                             // [16]
+  uint2* stage = reinterpret_cast<uint2*>(stage_bytes);
+  uint2* rec = A.rec + tu.row0;
   int32_t* I = A.info + (int64_t)u * kInfoInts;
   int32_t* hg = A.hist + (int64_t)u * kHistBins;
+  const int2* nonc = A.nonc + (int64_t)u * A.cap;
   const int n_rounds = (NC + kTailRound - 1) / kTailRound;
+  auto draw = [&](uint32_t c) { return splitmix64(((uint64_t)A.seed << 32) | (uint64_t)c); };
   int loaded = -1;
-  // round r's records r R .. r R + R into shared memory (L2 loads, all in
-  // flight together); past the unit: no key, count 0
-  auto load_round = [&](int r) {
-    const int c0 = r * kTailRound;
-    uint2 v[(kTailRound + kConsumers) / kConsumers];
-#pragma unroll
-    for (int j = 0; j < (kTailRound + kConsumers) / kConsumers; ++j) {
-      const int i = tid + j * kConsumers, c = c0 + i;
-      v[j] = make_uint2(0u, (uint32_t)Tb);
-      if (i <= kTailRound && c < NC) v[j] = __ldcg(rec + c);
-    }
-    csync();   // the previous round's readers are done
-#pragma unroll
-    for (int j = 0; j < (kTailRound + kConsumers) / kConsumers; ++j) {
-      const int i = tid + j * kConsumers;
-      if (i <= kTailRound) srec[rpad(i)] = v[j];
-    }
-    csync();
-    loaded = r;
-  };
-  auto key_at = [&](int i) { return srec[rpad(tid * kTailPT + i)].x; };
-  auto cnt_at = [&](int i) {
-    return (int)srec[rpad(tid * kTailPT + i + 1)].y - (int)srec[rpad(tid * kTailPT + i)].y;
-  };
-  auto for_rounds = [&](auto&& body) {
-    for (int r = 0; r < n_rounds; ++r) {
-      if (loaded != r) load_round(r);
-      body(r);
+  auto get_round = [&](int r) {
+    if (loaded != r) {
+      stage_round(rec, NC, Tb, r, stage);
+      loaded = r;
     }
   };
+  // this thread's record j of the staged round, and its member count
+  auto key_of = [&](int j) { return stage[rpad(kTailSteps * tid + j)].x; };
+  auto cnt_of = [&](int j) {
+    return (int)(stage[rpad(kTailSteps * tid + j + 1)].y - stage[rpad(kTailSteps * tid + j)].y);
+  };
+  auto id_of = [&](int r, int j) { return (uint32_t)(r * kTailRound + kTailSteps * tid + j); };
 
   pdl_wait();   // the steady kernel's lists
-  {
-    int hv[kHistBins / kConsumers];
-#pragma unroll
-    for (int j = 0; j < kHistBins / kConsumers; ++j) hv[j] = __ldcg(hg + tid + j * kConsumers);
-#pragma unroll
-    for (int j = 0; j < kHistBins / kConsumers; ++j) {
-      s_hist[tid + j * kConsumers] = hv[j];
-      hg[tid + j * kConsumers] = 0;   // clean for the next call
-    }
-  }
+  // ---- the histogram, the non-candidate count and round 0 in one round trip
+  const int4 h0 = __ldcg(reinterpret_cast<const int4*>(hg) + tid);
+  const int4 h1 = __ldcg(reinterpret_cast<const int4*>(hg) + kConsumers + tid);
   const int n_nonc = __ldcg(I + kNonCand);
-  // the clusters left without a non-steady token leave the histogram, and
-  // their keys become 0 (not candidates) before the records are read
-  const int2* nonc = A.nonc + (int64_t)u * A.cap;
+  get_round(0);
+  reinterpret_cast<int4*>(s_hist)[tid] = h0;
+  reinterpret_cast<int4*>(s_hist)[kConsumers + tid] = h1;
+  reinterpret_cast<int4*>(hg)[tid] = make_int4(0, 0, 0, 0);               // clean for the next call
+  reinterpret_cast<int4*>(hg)[kConsumers + tid] = make_int4(0, 0, 0, 0);
   csync();
-  for (int j = tid; j < n_nonc; j += kConsumers) {
-    const int c = __ldcg(&nonc[j].x);
-    if (c >= 0 && c < NC) {
-      const uint32_t key = __ldcg(&rec[c].x);
-      if (key) atomicSub(&s_hist[key >> kHistShift], 1);
-      __stcg(&rec[c].x, 0u);
+  // the clusters left without a non-steady token are not candidates: their
+  // keys leave the histogram and become 0 (in the records; the round is
+  // staged again), once, at the round's first staging
+  auto apply_nonc = [&](int r) {
+    for (int j = tid; j < n_nonc; j += kConsumers) {
+      const int c = __ldcg(&nonc[j].x), i = c - r * kTailRound;
+      if (i >= 0 && i < kTailRound && c < NC) {
+        const uint32_t key = stage[rpad(i)].x;
+        if (key) {
+          atomicSub(&s_hist[key >> kHistShift], 1);
+          __stcg(&rec[c].x, 0u);
+        }
+      }
     }
+    csync();       // the cleared keys are visible before the round is staged again
+    loaded = -1;
+    get_round(r);
+  };
+  if (n_nonc > 0) apply_nonc(0);
+
+  // ---- candidates: the nonzero keys; the histogram must hold as many (a
+  // stale one, left by a failed call, is rebuilt)
+  int cand = 0;
+  for (int r = 0; r < n_rounds; ++r) {
+    if (loaded != r) {
+      get_round(r);
+      if (n_nonc > 0) apply_nonc(r);
+    }
+#pragma unroll 4
+    for (int j = 0; j < kTailSteps; ++j) cand += key_of(j) != 0u;
   }
-  __threadfence_block();
-  csync();
-  // candidates: the nonzero keys, counted in one pass; the histogram must
-  // hold as many (a stale histogram, left by a failed call, is rebuilt from
-  // the keys)
-  int n_cand = 0, hist_total;
-  for_rounds([&](int) {
-    int s = 0;
-#pragma unroll 1
-    for (int i = 0; i < kTailPT; ++i) s += key_at(i) != 0u;
-    int t;
-    cscan(s, s_sh, &t);
-    n_cand += t;
-  });
-  {
-    int s = 0;
-    for (int i = tid; i < kHistBins; i += kConsumers) s += s_hist[i];
-    cscan(s, s_sh, &hist_total);
-  }
-  if (hist_total != n_cand) {
+  int hs = 0;
+#pragma unroll
+  for (int i = 0; i < kHistBins / kConsumers; ++i) hs += s_hist[tid * (kHistBins / kConsumers) + i];
+  int2 tot2;
+  wscan2(make_int2(warp_sum_int(cand), warp_sum_int(hs)), s_sh, &tot2);
+  const int n_cand = tot2.x;
+  if (tot2.y != n_cand) {
     if (tid == 0) flag_error(status, WI_DEV_BAD_HIST);
     for (int i = tid; i < kHistBins; i += kConsumers) s_hist[i] = 0;
     csync();
-    for_rounds([&](int) {
-#pragma unroll 1
-      for (int i = 0; i < kTailPT; ++i) {
-        const uint32_t key = key_at(i);
-        if (key) atomicAdd(&s_hist[key >> kHistShift], 1);
-      }
-    });
+    for (int r = 0; r < n_rounds; ++r) {
+      get_round(r);
+#pragma unroll 4
+      for (int j = 0; j < kTailSteps; ++j)
+        if (key_of(j)) atomicAdd(&s_hist[key_of(j) >> kHistShift], 1);
+    }
     csync();
   }
   const int k_req = A.topk_clusters >= 0 ? A.topk_clusters
@@ -797,7 +883,30 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
   int thr = -1;
   int bin1 = -1;
   uint64_t hstar = 0;
-  auto draw = [&](uint32_t c) { return splitmix64(((uint64_t)A.seed << 32) | (uint64_t)c); };
+
+  // the kth (1-based) record in id order that satisfies pred(key, id)
+  auto ordered_pick = [&](auto&& pred, int kth) -> int {
+    if (tid == 0) s_ctl[2] = -1;
+    int run = 0;
+    for (int r = 0; r < n_rounds; ++r) {
+      get_round(r);
+      uint32_t m = 0u;
+#pragma unroll 4
+      for (int j = 0; j < kTailSteps; ++j) m |= pred(key_of(j), id_of(r, j)) ? 1u << j : 0u;
+      int2 t2;
+      const int before = run + cscan2_excl(make_int2(__popc(m), 0), s_sh, &t2).x;
+      if (before < kth && before + __popc(m) >= kth) {
+        for (int n = kth - before; n > 1; --n) m &= m - 1u;   // drop the first n - 1 set bits
+        s_ctl[2] = (int)id_of(r, __ffs(m) - 1);
+      }
+      run += t2.x;
+    }
+    csync();
+    const int id = s_ctl[2];
+    csync();
+    return id;
+  };
+
   if (k == n_cand && k > 0) {
     kstar = 1u;
     thr = INT_MAX;
@@ -806,62 +915,76 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
     bin1 = select_bin(s_hist, kHistBins, k, &above, s_sh, s_ctl);
     int krem = k - above;
     const int nb1 = s_hist[bin1];
-    // the threshold bin's members in id order: into shared memory when they
-    // fit; otherwise each refinement pass streams the records again
+    csync();   // read by all before the radix passes reuse the histogram
+    // the threshold bin's members (key, id) when they fit; otherwise each
+    // refinement pass reads the records again
     const bool fits = nb1 <= kTailCand;
     if (fits) {
-      int base = 0;
-      for_rounds([&](int r) {
-        int s = 0;
-#pragma unroll 1
-        for (int i = 0; i < kTailPT; ++i) {
-          const uint32_t key = key_at(i);
-          s += key != 0u && (int)(key >> kHistShift) == bin1;
+      int run = 0;
+      for (int r = 0; r < n_rounds; ++r) {
+        get_round(r);
+        uint32_t m = 0u;
+#pragma unroll 4
+        for (int j = 0; j < kTailSteps; ++j)
+          m |= (key_of(j) != 0u && (int)(key_of(j) >> kHistShift) == bin1) ? 1u << j : 0u;
+        int2 t2;
+        int pos = run + cscan2_excl(make_int2(__popc(m), 0), s_sh, &t2).x;
+        while (m) {
+          const int j = __ffs(m) - 1;
+          m &= m - 1u;
+          const uint2 x = stage[rpad(kTailSteps * tid + j)];
+          if (pos < kTailCand) s_cand[pos] = ((unsigned long long)x.x << 32) | id_of(r, j);
+          ++pos;
         }
-        int t;
-        int pos = base + cscan(s, s_sh, &t) - s;
-#pragma unroll 1
-        for (int i = 0; i < kTailPT && s > 0; ++i) {
-          const uint32_t key = key_at(i);
-          if (key != 0u && (int)(key >> kHistShift) == bin1) {
-            if (pos < kTailCand)
-              s_cand[pos] = ((unsigned long long)key << 32) |
-                            (uint32_t)(r * kTailRound + tid * kTailPT + i);
-            ++pos;
-            --s;
-          }
-        }
-        base += t;
-      });
+        run += t2.x;
+      }
       csync();
     }
-    // (members: the bin holding the k-th key is a 2^-9 wide slice of the
-    // key range, so it normally holds a few dozen clusters)
+    auto cand_key = [&](int i) { return (uint32_t)(s_cand[i] >> 32); };
+    auto cand_id = [&](int i) { return (uint32_t)s_cand[i]; };
+    // a radix pass over the members (or, when they did not fit, over the
+    // records of the threshold bin): count(x) takes each one's value
+    auto over_members = [&](auto&& count) {
+      if (fits) {
+        for (int i = tid; i < nb1; i += kConsumers) count(cand_key(i), cand_id(i));
+      } else {
+        for (int r = 0; r < n_rounds; ++r) {
+          get_round(r);
+#pragma unroll 4
+          for (int j = 0; j < kTailSteps; ++j)
+            if (key_of(j) != 0u && (int)(key_of(j) >> kHistShift) == bin1) count(key_of(j), id_of(r, j));
+        }
+      }
+    };
     if (A.mode == 1) {
       // sampled: the krem members of the threshold bin with the smallest
       // (draw, id)
-      if (tid == 0) s_ctl[2] = -1;
-      csync();
-      if (fits) {
-        for (int i = tid; i < nb1; i += kConsumers) {
-          const uint32_t ci = (uint32_t)s_cand[i];
-          const uint64_t di = draw(ci);
+      if (fits && nb1 <= kTailDraws) {
+        if (tid < nb1) s_draw[tid] = draw(cand_id(tid));
+        if (tid == 0) s_ctl[2] = -1;
+        csync();
+        if (tid < nb1) {
+          const uint64_t dm = s_draw[tid];
+          const uint32_t im = cand_id(tid);
           int rank = 0;
-#pragma unroll 1
+#pragma unroll 8
           for (int j = 0; j < nb1; ++j) {
-            const uint32_t cj = (uint32_t)s_cand[j];
-            const uint64_t dj = draw(cj);
-            rank += dj < di || (dj == di && cj < ci);
+            const uint64_t dj = s_draw[j];
+            rank += dj < dm || (dj == dm && cand_id(j) < im);
           }
           if (rank == krem - 1) {
-            s_ctl[2] = (int)ci;
-            s_ctl[3] = (int)(uint32_t)(di >> 32);
-            s_ctl[4] = (int)(uint32_t)di;
+            s_ctl[2] = (int)im;
+            s_ctl[3] = (int)(uint32_t)(dm >> 32);
+            s_ctl[4] = (int)(uint32_t)dm;
           }
         }
+        csync();
+        thr = s_ctl[2];
+        hstar = ((uint64_t)(uint32_t)s_ctl[3] << 32) | (uint32_t)s_ctl[4];
+        csync();
       } else {
-        // a crowded bin: an exact radix select of the 64-bit draws
-        // (11/11/11/11/10/10-bit digits, smallest first), then ties in id order
+        // an exact radix select of the 64-bit draws (11/11/11/11/10/10-bit
+        // digits, smallest first), then the ties in id order
         uint64_t prefix = 0, pmask = 0;
         int kr = krem;
 #pragma unroll 1
@@ -870,16 +993,10 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
           const int nb = pass < 4 ? 2048 : 1024;
           for (int i = tid; i < kHistBins; i += kConsumers) s_hist[i] = 0;
           csync();
-          for_rounds([&](int r) {
-#pragma unroll 1
-            for (int i = 0; i < kTailPT; ++i) {
-              const uint32_t key = key_at(i);
-              if (key != 0u && (int)(key >> kHistShift) == bin1) {
-                const uint64_t d = draw((uint32_t)(r * kTailRound + tid * kTailPT + i));
-                if ((d & pmask) == prefix)
-                  atomicAdd(&s_hist[(nb - 1) - (int)((d >> sh_) & (uint64_t)(nb - 1))], 1);
-              }
-            }
+          over_members([&](uint32_t, uint32_t id) {
+            const uint64_t d = draw(id);
+            if ((d & pmask) == prefix)
+              atomicAdd(&s_hist[(nb - 1) - (int)((d >> sh_) & (uint64_t)(nb - 1))], 1);
           });
           csync();
           // the histogram is filled reversed, so select_bin's largest bin is
@@ -890,98 +1007,87 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
           prefix |= (uint64_t)dd << sh_;
           pmask |= (uint64_t)(nb - 1) << sh_;
         }
+        hstar = prefix;
+        if (fits) {
+          // the kr-th smallest id among the members drawing hstar
+          if (tid == 0) s_ctl[2] = -1;
+          csync();
+          for (int i = tid; i < nb1; i += kConsumers) {
+            const uint32_t ci = cand_id(i);
+            if (draw(ci) != hstar) continue;
+            int rank = 0;
+            for (int j = 0; j < nb1; ++j) {
+              const uint32_t cj = cand_id(j);
+              rank += cj < ci && draw(cj) == hstar;
+            }
+            if (rank == kr - 1) s_ctl[2] = (int)ci;
+          }
+          csync();
+          thr = s_ctl[2];
+          csync();
+        } else {
+          thr = ordered_pick([&](uint32_t key, uint32_t id) {
+            return key != 0u && (int)(key >> kHistShift) == bin1 && draw(id) == hstar;
+          }, kr);
+        }
+      }
+    } else {
+      // exact: the krem-th largest (key, -id) of the threshold bin
+      if (fits && nb1 <= kTailDraws) {
         if (tid == 0) s_ctl[2] = -1;
         csync();
-        int run = 0;
-        for_rounds([&](int r) {
-          int f = 0, first = -1;
-#pragma unroll 1
-          for (int i = 0; i < kTailPT; ++i) {
-            const uint32_t c = (uint32_t)(r * kTailRound + tid * kTailPT + i);
-            const uint32_t key = key_at(i);
-            if (key != 0u && (int)(key >> kHistShift) == bin1 && draw(c) == prefix) {
-              if (first < 0) first = (int)c;
-              ++f;
-            }
+        if (tid < nb1) {
+          const uint32_t km = cand_key(tid), im = cand_id(tid);
+          int rank = 0;
+#pragma unroll 8
+          for (int j = 0; j < nb1; ++j) {
+            const unsigned long long cj = s_cand[j];
+            const uint32_t kj = (uint32_t)(cj >> 32);
+            rank += kj > km || (kj == km && (uint32_t)cj < im);
           }
-          int t;
-          const int incl = cscan(f, s_sh, &t);
-          if (f > 0 && run + incl - f < kr && run + incl >= kr) s_ctl[2] = first;
-          run += t;
-        });
-        csync();
-        if (tid == 0) { s_ctl[3] = (int)(uint32_t)(prefix >> 32); s_ctl[4] = (int)(uint32_t)prefix; }
-      }
-      csync();
-      thr = s_ctl[2];
-      hstar = ((uint64_t)(uint32_t)s_ctl[3] << 32) | (uint32_t)s_ctl[4];
-      csync();
-    } else {
-      // exact: refine the threshold bin by the key's bits 20..10, then
-      // 9..0, then take the krem-th largest key's ties in id order
-      uint32_t prefix = (uint32_t)bin1 << kHistShift, pmask = 0xFFE00000u;
-#pragma unroll 1
-      for (int pass = 0; pass < 2; ++pass) {
-        const int sh_ = pass == 0 ? 10 : 0;
-        const int nb = pass == 0 ? 2048 : 1024;
-        for (int i = tid; i < kHistBins; i += kConsumers) s_hist[i] = 0;
-        csync();
-        if (fits) {
-          for (int i = tid; i < nb1; i += kConsumers) {
-            const uint32_t key = (uint32_t)(s_cand[i] >> 32);
-            if ((key & pmask) == prefix) atomicAdd(&s_hist[(key >> sh_) & (nb - 1)], 1);
-          }
-        } else {
-          for_rounds([&](int) {
-#pragma unroll 1
-            for (int i = 0; i < kTailPT; ++i) {
-              const uint32_t key = key_at(i);
-              if (key != 0u && (key & pmask) == prefix)
-                atomicAdd(&s_hist[(key >> sh_) & (nb - 1)], 1);
-            }
-          });
+          if (rank == krem - 1) { s_ctl[2] = (int)im; s_ctl[3] = (int)km; }
         }
         csync();
-        int ab;
-        const int dd = select_bin(s_hist, nb, krem, &ab, s_sh, s_ctl);
-        krem -= ab;
-        prefix |= (uint32_t)dd << sh_;
-        pmask |= (uint32_t)(nb - 1) << sh_;
-      }
-      kstar = prefix;
-      // the krem-th member (ascending id) with key == kstar
-      if (tid == 0) s_ctl[2] = -1;
-      csync();
-      if (fits) {
-        for (int i0 = 0; i0 < nb1; i0 += kConsumers) {
-          const int i = i0 + tid;
-          const int f = i < nb1 && (uint32_t)(s_cand[i] >> 32) == kstar;
-          int t;
-          const int incl = cscan(f, s_sh, &t);
-          if (f && incl == krem) s_ctl[2] = (int)(uint32_t)s_cand[i];
-          krem -= t;
-          if (krem <= 0) break;
-        }
+        thr = s_ctl[2];
+        kstar = (uint32_t)s_ctl[3];
+        csync();
       } else {
-        int run = 0;
-        for_rounds([&](int r) {
-          int f = 0;
+        // refine by the key's bits 20..10, then 9..0, then the ties in id order
+        uint32_t prefix = (uint32_t)bin1 << kHistShift, pmask = 0xFFE00000u;
 #pragma unroll 1
-          for (int i = 0; i < kTailPT; ++i) f += key_at(i) == kstar;
-          int t;
-          const int incl = cscan(f, s_sh, &t);
-          if (f > 0 && run + incl - f < krem && run + incl >= krem) {
-            int need = krem - (run + incl - f);
-#pragma unroll 1
-            for (int i = 0; i < kTailPT; ++i)
-              if (key_at(i) == kstar && --need == 0) s_ctl[2] = r * kTailRound + tid * kTailPT + i;
+        for (int pass = 0; pass < 2; ++pass) {
+          const int sh_ = pass == 0 ? 10 : 0;
+          const int nb = pass == 0 ? 2048 : 1024;
+          for (int i = tid; i < kHistBins; i += kConsumers) s_hist[i] = 0;
+          csync();
+          over_members([&](uint32_t key, uint32_t) {
+            if ((key & pmask) == prefix) atomicAdd(&s_hist[(key >> sh_) & (nb - 1)], 1);
+          });
+          csync();
+          int ab;
+          const int dd = select_bin(s_hist, nb, krem, &ab, s_sh, s_ctl);
+          krem -= ab;
+          prefix |= (uint32_t)dd << sh_;
+          pmask |= (uint32_t)(nb - 1) << sh_;
+        }
+        kstar = prefix;
+        if (fits) {
+          if (tid == 0) s_ctl[2] = -1;
+          csync();
+          for (int i = tid; i < nb1; i += kConsumers) {
+            if (cand_key(i) != kstar) continue;
+            const uint32_t ci = cand_id(i);
+            int rank = 0;
+            for (int j = 0; j < nb1; ++j) rank += cand_key(j) == kstar && cand_id(j) < ci;
+            if (rank == krem - 1) s_ctl[2] = (int)ci;
           }
-          run += t;
-        });
+          csync();
+          thr = s_ctl[2];
+          csync();
+        } else {
+          thr = ordered_pick([&](uint32_t key, uint32_t) { return key == kstar; }, krem);
+        }
       }
-      csync();
-      thr = s_ctl[2];
-      csync();
     }
   }
   // ---- emit, in id order: retrieved ids, their token slots, and the
@@ -990,37 +1096,59 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
   const bool sampled = A.mode == 1 && k > 0 && k < n_cand;
   const Threshold th{kstar, thr, sampled ? 1 : 0, bin1, hstar, A.seed};
   const bool no_est = A.exact_only || k == n_cand;
-  int32_t* sel = A.sel + row0;
+  int32_t* sel = A.sel + tu.row0;
   int32_t* tok = A.tok + tu.trow;
-  int2* full = A.full + row0 + (int64_t)u * A.cap;
+  int2* full = A.full + tu.row0 + (int64_t)u * A.cap;
   int n_sel = 0, n_tok = 0;
+  // retrieved clusters as {token position, first slot, count}, for the
+  // expansion of their token slots (the members' area, free by now)
+  int4* s_pick = reinterpret_cast<int4*>(s_cand);
+  constexpr int kPickCap = kTailCand / 2;
   if (k > 0) {
-    for_rounds([&](int r) {
-      const int c0 = r * kTailRound + tid * kTailPT;
-      int s = 0, t = 0;
-#pragma unroll 1
-      for (int i = 0; i < kTailPT; ++i)
-        if (th.picked(key_at(i), (uint32_t)(c0 + i))) { ++s; t += cnt_at(i); }
-      int2 tot2;
-      const int2 inc = cscan2(make_int2(s, t), s_sh, &tot2);
-      int ps = n_sel + inc.x - s, pt = n_tok + inc.y - t;
-#pragma unroll 1
-      for (int i = 0; i < kTailPT && s > 0; ++i) {
-        if (th.picked(key_at(i), (uint32_t)(c0 + i))) {
-          const int cnt = cnt_at(i);
-          const int o0 = (int)srec[rpad(tid * kTailPT + i)].y;
-          sel[ps] = c0 + i;
-          if (!no_est) full[ps] = make_int2(c0 + i, cnt);
-          ++ps;
-          --s;
-#pragma unroll 1
-          for (int j = 0; j < cnt; ++j) tok[pt + j] = o0 + j;
-          pt += cnt;
-        }
+    for (int r = 0; r < n_rounds; ++r) {
+      get_round(r);
+      uint32_t pm = 0u;
+      int pt = 0;
+#pragma unroll 4
+      for (int j = 0; j < kTailSteps; ++j) {
+        const bool p = th.picked(key_of(j), id_of(r, j));
+        pm |= p ? 1u << j : 0u;
+        pt += p ? cnt_of(j) : 0;
       }
-      n_sel += tot2.x;
-      n_tok += tot2.y;
-    });
+      int2 tot;
+      const int2 ex = cscan2_excl(make_int2(__popc(pm), pt), s_sh, &tot);
+      for (int e0 = 0; e0 < tot.x; e0 += kPickCap) {
+        int e = ex.x, tpos = n_tok + ex.y;
+        uint32_t m = pm;
+        while (m) {
+          const int j = __ffs(m) - 1;
+          m &= m - 1u;
+          const uint2 x = stage[rpad(kTailSteps * tid + j)];
+          const int cnt = (int)(stage[rpad(kTailSteps * tid + j + 1)].y - x.y);
+          const int id = (int)id_of(r, j);
+          if (e0 == 0) {
+            sel[n_sel + e] = id;
+            if (!no_est) full[n_sel + e] = make_int2(id, cnt);
+          }
+          if (e >= e0 && e < e0 + kPickCap) s_pick[e - e0] = make_int4(tpos, (int)x.y, cnt, 0);
+          ++e;
+          tpos += cnt;
+        }
+        csync();
+        // token slots: warp w expands picks w, w + 8, ..., one coalesced run each
+        const int np = min(kPickCap, tot.x - e0);
+        const int lane = tid & 31, w = tid >> 5;
+#pragma unroll 4
+        for (int q = w; q < np; q += kConsumerWarps) {
+          const int4 pk = s_pick[q];
+          if (lane < pk.z) tok[pk.x + lane] = pk.y + lane;
+          for (int x = lane + 32; x < pk.z; x += 32) tok[pk.x + x] = pk.y + x;
+        }
+        csync();
+      }
+      n_sel += tot.x;
+      n_tok += tot.y;
+    }
   }
   int n_full = 0;
   if (!no_est) {
@@ -1048,21 +1176,23 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkMap cm,
                  const __grid_constant__ ScanArgs A,
                  const __grid_constant__ CUtensorMap tm_cent,
-                 const __grid_constant__ CUtensorMap tm_vsum, uint32_t* status) {
+                 const __grid_constant__ CUtensorMap tm_vsum,
+                 const __grid_constant__ CUtensorMap tm_off, uint32_t* status) {
   using TS = TileShape<T, D>;
   using SM = ScanSmem<T, D, G>;
   constexpr bool kMma = std::is_same_v<T, __nv_bfloat16>;
   constexpr int kBoxCols = 128 / (int)sizeof(T);
   extern __shared__ __align__(16) unsigned char sh_raw[];
   __shared__ __align__(8) uint64_t s_full[4], s_empty[4];
-  __shared__ int s_last, s_ntails;
+  __shared__ int s_ntails;
   __shared__ int s_tails[kMaxTailsPerCta];   // units whose last arrival was this CTA's
   pdl_launch_dependents();
   unsigned char* sh = align_smem_1024(sh_raw);
   const int slots = A.slots;
-  const size_t slot_bytes = SM::slot_bytes(A.exact_only);
+  const size_t tile_bytes = SM::tile_bytes(A.exact_only);
   unsigned char* ring = sh;
-  unsigned char* s_union = ring + SM::ring_bytes(slots, A.exact_only);
+  unsigned char* side0 = ring + SM::ring_bytes(slots, A.exact_only);
+  unsigned char* s_union = side0 + SM::side_bytes(slots);
   uint32_t* hist16 = reinterpret_cast<uint32_t*>(s_union + SM::kUnion);
   RowMult* s_rows = reinterpret_cast<RowMult*>(reinterpret_cast<unsigned char*>(hist16) + SM::kHist16);
   float* s_sc = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(s_rows) + SM::kRows);
@@ -1070,19 +1200,6 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
   const int s = blockIdx.x;
   const int k0 = cm.n_chunks > 0 ? cm.k0(s) : 0, k1 = cm.n_chunks > 0 ? cm.k0(s + 1) : 0;
   const int nk = k1 - k0;
-  struct Chunk { int u, b, h, c0, nrows; int64_t row0; };
-  auto chunk = [&](int k) -> Chunk {
-    Chunk c;
-    c.b = cm.seq_of(k);
-    const int per = cm.per_unit(c.b);
-    const int rel = k - cm.ch_base[c.b];
-    c.h = rel / per;
-    c.c0 = (rel - c.h * per) * kTileRows;
-    c.u = c.b * geo.hkv + c.h;
-    c.nrows = min(kTileRows, geo.NC(c.b) - c.c0);
-    c.row0 = geo.cl_row(c.b, c.h);
-    return c;
-  };
   if (tid == 0) {
     for (int i = 0; i < slots; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], kConsumerWarps); }
     mbar_init_fence();
@@ -1092,15 +1209,23 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
   __syncthreads();
 
   if (warp == kConsumerWarps) {
-    // ---- producer: chunk i into slot i % slots once the slot is free
-    if (lane == 0) {
-      const uint32_t bytes = (uint32_t)slot_bytes;
+    // ---- producer: chunk i into slot i % slots once the slot is free: its
+    // key (and value-sum) tile, its offsets box, and the unit's queries when
+    // the chunk starts a unit
+    if (lane == 0 && nk > 0) {
+      ChunkPos p;
+      chunk_seek(p, geo, cm, k0);
+      int prev_u = -1;
       for (int i = 0; i < nk; ++i) {
         const int sl = i % slots;
         if (i >= slots) mbar_wait(&s_empty[sl], (uint32_t)((i / slots - 1) & 1), status);
-        const Chunk c = chunk(k0 + i);
-        const int y = (int)(c.row0 + c.c0);
-        unsigned char* dst = ring + sl * slot_bytes;
+        if (i > 0) chunk_next(p, geo, cm);
+        const bool new_u = p.u != prev_u;
+        prev_u = p.u;
+        const int y = (int)(p.row0 + p.c0);
+        unsigned char* dst = ring + sl * tile_bytes;
+        unsigned char* side = side0 + sl * SM::kSide;
+        const uint32_t bytes = (uint32_t)tile_bytes + kOffBox * 4 + (new_u ? (uint32_t)SM::kQBytes : 0u);
         mbar_arrive_expect(&s_full[sl], bytes);
 #pragma unroll
         for (int nb = 0; nb < TS::NB; ++nb)
@@ -1110,6 +1235,12 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
           for (int nb = 0; nb < TS::NB; ++nb)
             tensor_load_2d(dst + TS::kBytes + nb * TS::kBoxBytes, &tm_vsum, nb * kBoxCols, y,
                            &s_full[sl]);
+        }
+        tensor_load_1d(side, &tm_off, (int)((p.orow + p.c0) & ~(int64_t)3), &s_full[sl]);
+        if (new_u) {
+          const unsigned char* qsrc = reinterpret_cast<const unsigned char*>(A.q) +
+                                      ((int64_t)p.b * A.Hq + (int64_t)p.h * G) * D * (int64_t)sizeof(T);
+          bulk_load(side + kOffArea, qsrc, (uint32_t)SM::kQBytes, &s_full[sl]);
         }
       }
       // every copy issued has landed before the CTA may leave (bounded)
@@ -1124,47 +1255,48 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
   MmaAcc<D, G> macc;
   FmaAcc<D, G> facc;
   const int g = lane >> 2, tq = lane & 3;
-  // offsets of the warp's rows, prefetched two chunks ahead: lane l <= 8
-  // holds offsets[c0 + 8 warp + l] of its unit
-  auto load_off = [&](int i) -> int {
-    if (i >= nk || lane > 8) return 0;
-    const Chunk c = chunk(k0 + i);
-    const int cl = c.c0 + 8 * warp + lane;
-    if (cl > geo.NC(c.b)) return 0;
-    return __ldg(A.offsets + geo.off_row(c.b, c.h) + cl);
-  };
-  int off_cur = load_off(0), off_n1 = load_off(1), off_n2 = load_off(2);
-  int cur_u = -1;
+  ChunkPos c;
+  if (nk > 0) chunk_seek(c, geo, cm, k0);
+  int cur_u = -1, u_slot = 0, u_parts = 1;
   int since_flush = 0;
   float* comb = reinterpret_cast<float*>(s_union);
   RowMult* rm = s_rows + warp * 8;
   float* sc = s_sc + warp * 8 * G;
+  const int r0 = 8 * warp;   // the warp's rows of every chunk
   for (int i = 0; i < nk; ++i) {
-    const Chunk c = chunk(k0 + i);
-    if (c.u != cur_u) {
-      const T* qg = reinterpret_cast<const T*>(A.q) + ((int64_t)c.b * A.Hq + (int64_t)c.h * G) * D;
-      if constexpr (kMma) { macc.load_q(qg); macc.reset(); }
-      else { facc.load_q(qg, A.scale); facc.reset(); }
-      cur_u = c.u;
-    }
+    if (i > 0) chunk_next(c, geo, cm);
     const int sl = i % slots;
-    const unsigned char* ktile = ring + sl * slot_bytes;
+    const unsigned char* ktile = ring + sl * tile_bytes;
     const unsigned char* vtile = ktile + TS::kBytes;
-    // rows 8 warp .. 8 warp + 7: counts and first slots from the offsets
-    const int r0 = 8 * warp;
+    const unsigned char* side = side0 + sl * SM::kSide;
+    const bool new_u = c.u != cur_u;
+    if (new_u) {
+      // this CTA's part index among the unit's scan CTAs, and their number
+      cur_u = c.u;
+      const int cf = cm.cta_of(c.kend - cm.per_unit(c.b));
+      u_slot = s - cf;
+      u_parts = cm.cta_of(c.kend - 1) - cf + 1;
+    }
     __syncwarp();   // the previous chunk's row data is read
+    mbar_wait(&s_full[sl], (uint32_t)((i / slots) & 1), status);
+    if (new_u) {
+      const T* qs = reinterpret_cast<const T*>(side + kOffArea);
+      if constexpr (kMma) { macc.load_q(qs); macc.reset(); }
+      else { facc.load_q(qs, A.scale); facc.reset(); }
+    }
+    // rows r0 .. r0 + 7: counts and first slots from the chunk's offsets
+    const int32_t* offs = reinterpret_cast<const int32_t*>(side) + (int)((c.orow + c.c0) & 3);
+    const int off_l = lane <= 8 ? offs[r0 + lane] : 0;
     {
-      const int o_next = __shfl_down_sync(0xffffffffu, off_cur, 1);
+      const int o_next = __shfl_down_sync(0xffffffffu, off_l, 1);
       if (lane < 8) {
-        const int cl = c.c0 + r0 + lane;
-        const int cnt = o_next - off_cur;
-        const bool ok = cl < c.c0 + c.nrows && cnt > 0;
+        const int cnt = o_next - off_l;
+        const bool ok = r0 + lane < c.nrows && cnt > 0;
         rm[lane] = RowMult{1.f, (float)cnt, ok ? 1 : 0};
       }
       __syncwarp();
     }
-    mbar_wait(&s_full[sl], (uint32_t)((i / slots) & 1), status);
-    // scores, keys, histogram, estimation
+    // scores, keys, estimation
     float key_s[2] = {-INFINITY, -INFINITY};   // group max of rows 2tq, 2tq+1 (MMA) / lane's row (FMA)
     if constexpr (kMma) {
       float s0, s1;
@@ -1201,41 +1333,34 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
     // the slot's last reads are done: release it to the producer
     __syncwarp();
     if (lane == 0) mbar_arrive(&s_empty[sl]);
-    // keys and the first digit's histogram: MMA lanes 0..3 hold rows 2t and
-    // 2t + 1 (t = lane), FMA lanes 0..7 row lane; each writes the record
-    // {key, first slot} of its rows
+    // the records {key, first slot} of the warp's 8 rows (lanes 0..7, one
+    // 64-byte store) and the first digit's histogram
     {
-      const int ra = kMma ? 2 * tq : (lane & 7);
-      const int oa = __shfl_sync(0xffffffffu, off_cur, ra);
-      const int ob = __shfl_sync(0xffffffffu, off_cur, (ra + 1) & 31);
-      const int nkeys = kMma ? (lane < 4 ? 2 : 0) : (lane < 8 ? 1 : 0);
-#pragma unroll
-      for (int kx = 0; kx < 2; ++kx) {
-        if (kx >= nkeys) break;
-        const int r = ra + kx;
-        const int cl = c.c0 + r0 + r;
-        if (cl < c.c0 + c.nrows) {
-          const uint32_t key = rm[r].valid ? ordered_key(key_s[kx]) : 0u;
-          A.rec[c.row0 + cl] = make_uint2(key, (uint32_t)(kx ? ob : oa));
-          if (key) atomicAdd(&hist16[key >> (kHistShift + 1)], 1u << (16 * ((key >> kHistShift) & 1u)));
-        }
+      float kv = key_s[0];
+      if constexpr (kMma) {
+        // MMA lane t (t < 4) holds the keys of rows 2t and 2t + 1
+        const float ka = __shfl_sync(0xffffffffu, key_s[0], (lane >> 1) & 3);
+        const float kb = __shfl_sync(0xffffffffu, key_s[1], (lane >> 1) & 3);
+        kv = (lane & 1) ? kb : ka;
+      }
+      if (lane < 8 && r0 + lane < c.nrows) {
+        const uint32_t key = rm[lane].valid ? ordered_key(kv) : 0u;
+        A.rec[c.row0 + c.c0 + r0 + lane] = make_uint2(key, (uint32_t)off_l);
+        if (key) atomicAdd(&hist16[key >> (kHistShift + 1)], 1u << (16 * ((key >> kHistShift) & 1u)));
       }
     }
-    off_cur = off_n1;
-    off_n1 = off_n2;
-    off_n2 = load_off(i + 3);
     since_flush += kTileRows;
-    // ---- end of the CTA's part of a unit: part, histogram, arrival, tail
-    const bool unit_end = i == nk - 1 || chunk(k0 + i + 1).u != c.u;
+    // ---- end of the CTA's part of a unit: histogram, part, arrival
+    const bool unit_end = i == nk - 1 || c.k + 1 == c.kend;
     if (unit_end || since_flush >= 65536 - kTileRows) {
       csync();
       int32_t* hg = A.hist + (int64_t)c.u * kHistBins;
-      for (int w = tid; w < kHistBins / 2; w += kConsumers) {
-        const uint32_t v = hist16[w];
+      for (int wd = tid; wd < kHistBins / 2; wd += kConsumers) {
+        const uint32_t v = hist16[wd];
         if (v) {
-          if (v & 0xffffu) atomicAdd(hg + 2 * w, (int)(v & 0xffffu));
-          if (v >> 16) atomicAdd(hg + 2 * w + 1, (int)(v >> 16));
-          hist16[w] = 0u;
+          if (v & 0xffffu) atomicAdd(hg + 2 * wd, (int)(v & 0xffffu));
+          if (v >> 16) atomicAdd(hg + 2 * wd + 1, (int)(v >> 16));
+          hist16[wd] = 0u;
         }
       }
       since_flush = 0;
@@ -1246,19 +1371,20 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
         if constexpr (kMma) macc.to_smem(comb + warp * G * (D + kPartStride));
         else facc.to_smem(comb + warp * G * (D + kPartStride));
         csync();
-        const int slot = s - cm.cta_of(cm.first(c.b, c.h));
-        float* part = A.est + ((int64_t)c.u * A.p1max + slot) * G * (D + kPartStride);
+        float* part = A.est + ((int64_t)c.u * A.p1max + u_slot) * G * (D + kPartStride);
         combine_warps<D, G>(comb, part, tid);
       }
-      __threadfence();
+      // every thread's records, histogram counts and part are written before
+      // the barrier; one fenced arrival publishes them (a cumulative fence)
       csync();
       if (tid == 0) {
-        const int old = atomicAdd(A.cnt1 + c.u, 1);
         __threadfence();
-        s_last = old == cm.parts(c.b, c.h) - 1;
+        const int old = atomicAdd(A.cnt1 + c.u, 1);
+        if (old == u_parts - 1) {
+          __threadfence();
+          s_tails[s_ntails++] = c.u;
+        }
       }
-      csync();
-      if (s_last && tid == 0) s_tails[s_ntails++] = c.u;
     }
   }
   // ---- the tails of the units this CTA finished last (after the loop, so
@@ -1268,7 +1394,7 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
   for (int t = 0; t < nt; ++t) {
     const int u = s_tails[t], b = u / geo.hkv, h = u - b * geo.hkv;
     const TailUnit tu{u, geo.NC(b), geo.T(b), geo.cl_row(b, h), geo.tok_row(b, h)};
-    scan_tail(tu, A, s_union, reinterpret_cast<uint2*>(ring), status);
+    scan_tail(tu, A, s_union, ring, SM::kTailCandOff, SM::kTailDrawOff, SM::kTailShOff, status);
     csync();
   }
   pdl_wait();
@@ -1686,6 +1812,19 @@ bool encode_rows(CUtensorMap* tm, const void* base, int64_t rows, int D, int dty
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// the offsets array as a 1-D int32 tensor, boxes of kOffBox entries
+bool encode_offsets(CUtensorMap* tm, const int32_t* base, int64_t n) {
+  auto fn = encode_fn();
+  if (!fn || n <= 0) return false;
+  const cuuint64_t dims[1] = {(cuuint64_t)n};
+  const cuuint64_t strides[1] = {4};   // unused for one dimension
+  const cuuint32_t box[1] = {(cuuint32_t)kOffBox};
+  const cuuint32_t estr[1] = {1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_INT32, 1, const_cast<int32_t*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Dynamic shared memory limit, and the full shared-memory carveout for every
 // decode kernel (kernels that overlap under programmatic dependent launch
 // then never need the SM's L1 / shared split reconfigured between them).
@@ -1719,16 +1858,17 @@ cudaError_t launch_decode_typed(const DecodePlan& p, const DecodeArgs& a, const 
   int2* pc = reinterpret_cast<int2*>(ws + p.off_pc);
   int2* nonc = reinterpret_cast<int2*>(ws + p.off_nonc);
   // K1: scan + tails
-  CUtensorMap tmc, tmv;
+  CUtensorMap tmc, tmv, tmo;
   std::memset(&tmc, 0, sizeof(tmc));
   std::memset(&tmv, 0, sizeof(tmv));
+  std::memset(&tmo, 0, sizeof(tmo));
+  const int64_t n_off = ((int64_t)p.geo.cl_base[p.geo.batch] + p.geo.batch) * p.geo.hkv;
   if (!encode_rows(&tmc, a.centroids, p.ncl, D, p.dtype) ||
-      !encode_rows(&tmv, a.value_sums, p.ncl, D, p.dtype))
+      !encode_rows(&tmv, a.value_sums, p.ncl, D, p.dtype) || !encode_offsets(&tmo, a.offsets, n_off))
     return cudaErrorInvalidValue;
   ScanArgs A{};
   A.q = a.q;
   A.Hq = p.Hq;
-  A.offsets = a.offsets;
   A.rec = reinterpret_cast<uint2*>(ws + p.off_rec);
   A.hist = reinterpret_cast<int32_t*>(ws + p.off_hist);
   A.cnt1 = reinterpret_cast<int32_t*>(ws + p.off_cnt1);
@@ -1753,7 +1893,7 @@ cudaError_t launch_decode_typed(const DecodePlan& p, const DecodeArgs& a, const 
   mark(1);
   cudaError_t e1 = launch_ex(wave_scan_kernel<T, D, G>, dim3(std::max(1, p.n_scan)),
                              dim3(kScanThreads), scan_smem, s, pdl, p.geo, cm, A, tmc, tmv,
-                             status);
+                             tmo, status);
   if (e1 != cudaSuccess) return e1;
   // K2: gather, exact attention, estimate corrections, merge
   GatherArgs B{};

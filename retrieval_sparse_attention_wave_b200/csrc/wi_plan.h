@@ -134,7 +134,7 @@ wi_status decode_workspace_extent(const wi_index* idx, const wi_decode_params* p
 size_t decode_scan_smem(int dtype, int D, int G, int slots, int exact_only);
 size_t decode_gather_smem(int dtype, int D, int G);
 size_t decode_steady_smem(int cap);
-size_t decode_scan_slot_bytes(int dtype, int D, int exact_only);
+size_t decode_scan_slot_bytes(int dtype, int D, int G, int exact_only);
 cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s);
 // Position-block index: each token's cluster is its block inside its segment,
 // then one finalizing update pass.

@@ -204,6 +204,10 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
       rows = std::min<int64_t>(k * ix->cluster_size, T) + nst[b];
       if (!pl.exact_only) rows += k + nst[b];
     }
+    // a quarter more than expected: retrieved clusters run larger than the
+    // average cluster, and a CTA that loops over a second block holds up the
+    // unit's merge
+    rows += rows / 4;
     const int n2 = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(rows, rpb), kMaxGatherPerUnit));
     pl.n2_base[b + 1] = pl.n2_base[b] + H * n2;
     pl.n2max = std::max(pl.n2max, n2);
@@ -224,7 +228,7 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   pl.off_nonc = take((size_t)pl.U * cap * 8);
   pl.off_sel = take((size_t)pl.ncl * 4);
   pl.off_tok = take((size_t)pl.ntok * 4);
-  pl.off_full = take(((size_t)pl.ncl + (size_t)pl.U * cap) * 8);
+  pl.off_selinfo = take((size_t)pl.ncl * 16);
   pl.off_est = take(pl.exact_only ? 0 : (size_t)pl.U * pl.p1max * PS);
   pl.off_gat = take((size_t)pl.U * pl.n2max * PS);
   const size_t nq = (size_t)B * p->n_q_heads;

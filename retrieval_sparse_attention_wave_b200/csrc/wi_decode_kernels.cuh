@@ -512,9 +512,10 @@ struct ScanArgs {
   // tail
   int32_t* info;
   const int2* nonc;
-  int32_t* sel;          // [ncl] retrieved ids (unit rows as the centroids)
-  int32_t* tok;          // [ntok] token slots of the retrieved clusters (unit rows as perm)
-  int2* full;            // [ncl + U cap] (cluster, count) whose estimate is taken back out
+  int32_t* sel;          // [ncl] retrieved ids, ascending (unit rows as the centroids)
+  int4* selinfo;         // [ncl] retrieved {id, first slot, count, first token row}
+  int32_t* blkf;         // [ntok] per block of kGatherRows token rows: its first retrieved
+                         // cluster (unit rows as perm)
   int cap;
   int topk_clusters;
   double topk_fraction;
@@ -809,11 +810,9 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
       loaded = r;
     }
   };
-  // this thread's record j of the staged round, and its member count
+  // this thread's record j of the staged round
   auto key_of = [&](int j) { return stage[rpad(kTailSteps * tid + j)].x; };
-  auto cnt_of = [&](int j) {
-    return (int)(stage[rpad(kTailSteps * tid + j + 1)].y - stage[rpad(kTailSteps * tid + j)].y);
-  };
+
   auto id_of = [&](int r, int j) { return (uint32_t)(r * kTailRound + kTailSteps * tid + j); };
 
   pdl_wait();   // the steady kernel's lists
@@ -1090,71 +1089,66 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
       }
     }
   }
-  // ---- emit, in id order: retrieved ids, their token slots, and the
-  // clusters taken back out of the estimate (retrieved, then the
-  // non-candidates), unless the estimation zone is empty
+  // ---- emit, in id order: the retrieved clusters {id, first slot, count,
+  // first token row} (the gather's token rows are theirs, concatenated; the
+  // clusters taken back out of the estimate are they and the
+  // non-candidates), and for every block of kGatherRows token rows the first
+  // retrieved cluster that overlaps it
   const bool sampled = A.mode == 1 && k > 0 && k < n_cand;
   const Threshold th{kstar, thr, sampled ? 1 : 0, bin1, hstar, A.seed};
   const bool no_est = A.exact_only || k == n_cand;
   int32_t* sel = A.sel + tu.row0;
-  int32_t* tok = A.tok + tu.trow;
-  int2* full = A.full + tu.row0 + (int64_t)u * A.cap;
+  int4* selinfo = A.selinfo + tu.row0;
+  int32_t* blkf = A.blkf + tu.trow;
   int n_sel = 0, n_tok = 0;
-  // retrieved clusters as {token position, first slot, count}, for the
-  // expansion of their token slots (the members' area, free by now)
-  int4* s_pick = reinterpret_cast<int4*>(s_cand);
-  constexpr int kPickCap = kTailCand / 2;
   if (k > 0) {
     for (int r = 0; r < n_rounds; ++r) {
       get_round(r);
+      // (the mode test out of the loop; each record's count without a
+      // branch, from its first slot and the next record's)
       uint32_t pm = 0u;
       int pt = 0;
+      const int rb = kTailSteps * tid;
+      if (!th.sampled) {
 #pragma unroll 4
-      for (int j = 0; j < kTailSteps; ++j) {
-        const bool p = th.picked(key_of(j), id_of(r, j));
-        pm |= p ? 1u << j : 0u;
-        pt += p ? cnt_of(j) : 0;
+        for (int j = 0; j < kTailSteps; ++j) {
+          const uint2 x = stage[rpad(rb + j)];
+          const uint32_t nx = stage[rpad(rb + j + 1)].y;
+          const bool p = x.x != 0u && (x.x > th.kstar || (x.x == th.kstar && (int)id_of(r, j) <= th.thr));
+          pm |= (uint32_t)p << j;
+          pt += p ? (int)(nx - x.y) : 0;
+        }
+      } else {
+#pragma unroll 4
+        for (int j = 0; j < kTailSteps; ++j) {
+          const uint2 x = stage[rpad(rb + j)];
+          const uint32_t nx = stage[rpad(rb + j + 1)].y;
+          const bool p = th.picked(x.x, id_of(r, j));
+          pm |= (uint32_t)p << j;
+          pt += p ? (int)(nx - x.y) : 0;
+        }
       }
       int2 tot;
       const int2 ex = cscan2_excl(make_int2(__popc(pm), pt), s_sh, &tot);
-      for (int e0 = 0; e0 < tot.x; e0 += kPickCap) {
-        int e = ex.x, tpos = n_tok + ex.y;
-        uint32_t m = pm;
-        while (m) {
-          const int j = __ffs(m) - 1;
-          m &= m - 1u;
-          const uint2 x = stage[rpad(kTailSteps * tid + j)];
-          const int cnt = (int)(stage[rpad(kTailSteps * tid + j + 1)].y - x.y);
-          const int id = (int)id_of(r, j);
-          if (e0 == 0) {
-            sel[n_sel + e] = id;
-            if (!no_est) full[n_sel + e] = make_int2(id, cnt);
-          }
-          if (e >= e0 && e < e0 + kPickCap) s_pick[e - e0] = make_int4(tpos, (int)x.y, cnt, 0);
-          ++e;
-          tpos += cnt;
-        }
-        csync();
-        // token slots: warp w expands picks w, w + 8, ..., one coalesced run each
-        const int np = min(kPickCap, tot.x - e0);
-        const int lane = tid & 31, w = tid >> 5;
-#pragma unroll 4
-        for (int q = w; q < np; q += kConsumerWarps) {
-          const int4 pk = s_pick[q];
-          if (lane < pk.z) tok[pk.x + lane] = pk.y + lane;
-          for (int x = lane + 32; x < pk.z; x += 32) tok[pk.x + x] = pk.y + x;
-        }
-        csync();
+      int e = n_sel + ex.x, tpos = n_tok + ex.y;
+      while (pm) {
+        const int j = __ffs(pm) - 1;
+        pm &= pm - 1u;
+        const uint2 x = stage[rpad(rb + j)];
+        const int cnt = (int)(stage[rpad(rb + j + 1)].y - x.y);
+        const int id = (int)id_of(r, j);
+        sel[e] = id;
+        selinfo[e] = make_int4(id, (int)x.y, cnt, tpos);
+        for (int bk = (tpos + kGatherRows - 1) / kGatherRows; bk * kGatherRows < tpos + cnt; ++bk)
+          blkf[bk] = e;
+        ++e;
+        tpos += cnt;
       }
       n_sel += tot.x;
       n_tok += tot.y;
     }
   }
-  int n_full = 0;
-  if (!no_est) {
-    for (int j = tid; j < n_nonc; j += kConsumers) full[n_sel + j] = __ldcg(&nonc[j]);
-    n_full = n_sel + n_nonc;
-  }
+  const int n_full = no_est ? 0 : n_sel + n_nonc;
   if (tid == 0) {
     I[kSelCount] = n_sel;
     I[kThrKey] = (int32_t)kstar;
@@ -1412,8 +1406,9 @@ struct GatherArgs {
   const int32_t* info;
   const int32_t* st_slot;
   const int2* pc;
-  const int32_t* tok;
-  const int2* full;
+  const int4* selinfo;   // retrieved {id, first slot, count, first token row}
+  const int32_t* blkf;   // per block of token rows: its first retrieved cluster
+  const int2* nonc;      // (cluster, count) of the non-candidates
   int cap;
   int n_sink, window;
   float* est;
@@ -1457,6 +1452,8 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
   extern __shared__ __align__(16) unsigned char sh_raw[];
   __shared__ int s_rec[kInfoInts];
   __shared__ int s_last;
+  __shared__ int s_bf[2];                  // first retrieved clusters of the CTA's first block and the next
+  __shared__ int s_slot[kGatherRows];      // token slots of the block's token rows
   unsigned char* sh = align_smem_1024(sh_raw);
   unsigned char* tiles = sh;                                   // [K t0][K t1][V t0][V t1]
   const unsigned char** s_kp = reinterpret_cast<const unsigned char**>(tiles + SM::kTiles);
@@ -1496,10 +1493,13 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
   else { facc.load_q(qg, A.scale); facc.reset(); }
 
   pdl_wait();   // the scan's and the steady kernel's results
-  // the unit's record, and (speculatively) the token slots of the first block
+  // the unit's record, and (speculatively) where the first block's token
+  // rows start among the retrieved clusters
   if (tid < kInfoInts) s_rec[tid] = __ldcg(A.info + (int64_t)u * kInfoInts + tid);
-  int spec = -1;
-  if (tid < RPB && j * RPB + tid < Tb) spec = __ldcg(A.tok + trow + j * RPB + tid);
+  if (tid == 32 || tid == 33) {
+    const int bk = j + tid - 32;
+    s_bf[tid - 32] = bk < Tb ? __ldcg(A.blkf + trow + bk) : 0;
+  }
   __syncthreads();
   const bool dense = s_rec[kDense] != 0, no_est = s_rec[kNoEstimate] != 0;
   // the scan's estimation parts this CTA folds into its own (p = j, j + n2,
@@ -1511,6 +1511,7 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
       cp_async16(s_pre + 4 * x, src + 4 * x);
     cp_async_commit();
   }
+  const int n_sel = dense ? 0 : s_rec[kSelCount];
   const int n_tok = dense ? 0 : s_rec[kSelTokens];
   const int n_st = s_rec[kSteady];
   const int n_full = (dense || no_est) ? 0 : s_rec[kFullRows];
@@ -1527,6 +1528,26 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
 
   for (int blk = j; blk * RPB < R; blk += n2) {
     const int rb = blk * RPB;
+    // ---- the block's token rows: the slots of the retrieved clusters that
+    // overlap it (at most RPB + 1 of them), filled in by their records
+    if (rb < n_tok) {
+      int s_lo = blk == j ? s_bf[0] : __ldcg(A.blkf + trow + blk);
+      int s_hi = rb + RPB >= n_tok ? n_sel - 1
+                                   : (blk == j ? s_bf[1] : __ldcg(A.blkf + trow + blk + 1));
+      if (s_lo < 0 || s_hi >= n_sel || s_hi < s_lo || s_hi - s_lo > RPB) {
+        if (tid == 0) flag_error(status, WI_DEV_BAD_CLUSTER);
+        s_lo = 0;
+        s_hi = -1;
+      }
+      if (tid < RPB) s_slot[tid] = -1;
+      __syncthreads();
+      for (int e = tid; e <= s_hi - s_lo; e += blockDim.x) {
+        const int4 si = __ldcg(A.selinfo + row0 + s_lo + e);   // {id, first slot, count, first row}
+        const int r0 = max(si.w, rb), r1 = min(min(si.w + si.z, rb + RPB), n_tok);
+        for (int r = r0; r < r1; ++r) s_slot[r - rb] = si.y + (r - si.w);
+      }
+      __syncthreads();
+    }
     // ---- resolve the block's rows: kind, key and value row addresses
     if (tid < RPB) {
       const int r = rb + tid;
@@ -1538,14 +1559,21 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
         if (dense) {
           slot = r; kind = kRowSteady;
         } else if (r < n_tok) {
-          slot = blk == j ? spec : __ldcg(A.tok + trow + r);
+          slot = s_slot[tid];
           kind = kRowToken;
         } else if (r < n_tok + n_st) {
           slot = __ldcg(A.st_slot + (int64_t)u * A.cap + (r - n_tok));
           kind = kRowSteady;
         } else if (r < n_tok + n_st + n_full) {
-          const int2 f = __ldcg(A.full + row0 + (int64_t)u * A.cap + (r - n_tok - n_st));
-          c = f.x; aux = f.y; kind = kRowFull;
+          const int f = r - n_tok - n_st;   // retrieved clusters, then the non-candidates
+          if (f < n_sel) {
+            const int4 si = __ldcg(A.selinfo + row0 + f);
+            c = si.x; aux = si.z;
+          } else {
+            const int2 nc = __ldcg(A.nonc + (int64_t)u * A.cap + (f - n_sel));
+            c = nc.x; aux = nc.y;
+          }
+          kind = kRowFull;
         } else {
           const int2 p = __ldcg(A.pc + (int64_t)u * A.cap + (r - n_tok - n_st - n_full));
           slot = p.x; c = p.y; kind = kRowPart;
@@ -1880,8 +1908,8 @@ cudaError_t launch_decode_typed(const DecodePlan& p, const DecodeArgs& a, const 
   A.info = info;
   A.nonc = nonc;
   A.sel = reinterpret_cast<int32_t*>(ws + p.off_sel);
-  A.tok = reinterpret_cast<int32_t*>(ws + p.off_tok);
-  A.full = reinterpret_cast<int2*>(ws + p.off_full);
+  A.blkf = reinterpret_cast<int32_t*>(ws + p.off_tok);
+  A.selinfo = reinterpret_cast<int4*>(ws + p.off_selinfo);
   A.cap = p.cap;
   A.topk_clusters = p.topk_clusters;
   A.topk_fraction = p.topk_fraction;
@@ -1908,8 +1936,9 @@ cudaError_t launch_decode_typed(const DecodePlan& p, const DecodeArgs& a, const 
   B.info = info;
   B.st_slot = st_slot;
   B.pc = pc;
-  B.tok = A.tok;
-  B.full = A.full;
+  B.blkf = A.blkf;
+  B.selinfo = A.selinfo;
+  B.nonc = nonc;
   B.cap = p.cap;
   B.n_sink = p.n_sink;
   B.window = p.window;

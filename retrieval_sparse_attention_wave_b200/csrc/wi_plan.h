@@ -20,6 +20,7 @@ constexpr int kConsumers = 32 * kConsumerWarps;   // 256 consumer threads
 constexpr int kScanThreads = kConsumers + 32;     // + one producer warp
 constexpr int kGatherThreads = kConsumers;
 constexpr int kGatherTiles = 2;                   // tiles per gather block (128 rows)
+constexpr int kGatherRows = kGatherTiles * kTileRows;   // rows per gather block
 constexpr int kInfoInts = 16;                     // per-unit record (see wi_decode_layout)
 constexpr int kHistBins = 2048;                   // first radix digit: key bits 31..21
 constexpr int kTailCand = 1024;                   // threshold-bin members refined in shared memory
@@ -68,7 +69,7 @@ struct DecodePlan {
   int n_gather, n2max;
   // workspace byte offsets; [0, off_rec) must be zero before the first call
   size_t off_status, off_cnt1, off_cnt2, off_hist;
-  size_t off_rec, off_info, off_st_slot, off_pc, off_nonc, off_sel, off_tok, off_full;
+  size_t off_rec, off_info, off_st_slot, off_pc, off_nonc, off_sel, off_tok, off_selinfo;
   size_t off_est, off_gat, off_q, off_out, off_lse;
   size_t total;
 };

@@ -1245,109 +1245,126 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
     return;
   }
 
-  // ---- consumers
+  // ---- consumers: an outer loop over the units of the CTA's range, a
+  // tight inner loop over a unit's chunks (slot and phase kept as counters)
   MmaAcc<D, G> macc;
   FmaAcc<D, G> facc;
   const int g = lane >> 2, tq = lane & 3;
-  ChunkPos c;
-  if (nk > 0) chunk_seek(c, geo, cm, k0);
-  int cur_u = -1, u_slot = 0, u_parts = 1;
   int since_flush = 0;
   float* comb = reinterpret_cast<float*>(s_union);
   RowMult* rm = s_rows + warp * 8;
   float* sc = s_sc + warp * 8 * G;
   const int r0 = 8 * warp;   // the warp's rows of every chunk
-  for (int i = 0; i < nk; ++i) {
-    if (i > 0) chunk_next(c, geo, cm);
-    const int sl = i % slots;
-    const unsigned char* ktile = ring + sl * tile_bytes;
-    const unsigned char* vtile = ktile + TS::kBytes;
-    const unsigned char* side = side0 + sl * SM::kSide;
-    const bool new_u = c.u != cur_u;
-    if (new_u) {
-      // this CTA's part index among the unit's scan CTAs, and their number
-      cur_u = c.u;
-      const int cf = cm.cta_of(c.kend - cm.per_unit(c.b));
-      u_slot = s - cf;
-      u_parts = cm.cta_of(c.kend - 1) - cf + 1;
-    }
-    __syncwarp();   // the previous chunk's row data is read
-    mbar_wait(&s_full[sl], (uint32_t)((i / slots) & 1), status);
-    if (new_u) {
-      const T* qs = reinterpret_cast<const T*>(side + kOffArea);
-      if constexpr (kMma) { macc.load_q(qs); macc.reset(); }
-      else { facc.load_q(qs, A.scale); facc.reset(); }
-    }
-    // rows r0 .. r0 + 7: counts and first slots from the chunk's offsets
-    const int32_t* offs = reinterpret_cast<const int32_t*>(side) + (int)((c.orow + c.c0) & 3);
-    const int off_l = lane <= 8 ? offs[r0 + lane] : 0;
-    {
-      const int o_next = __shfl_down_sync(0xffffffffu, off_l, 1);
-      if (lane < 8) {
-        const int cnt = o_next - off_l;
-        const bool ok = r0 + lane < c.nrows && cnt > 0;
-        rm[lane] = RowMult{1.f, (float)cnt, ok ? 1 : 0};
+  int sl = 0;
+  uint32_t ph = 0u;
+  for (int i = 0; i < nk;) {
+    ChunkPos c;
+    chunk_seek(c, geo, cm, k0 + i);
+    const int n_here = min(nk - i, c.kend - c.k);   // the unit's chunks in this CTA
+    // this CTA's part index among the unit's scan CTAs, and their number
+    const int cf = cm.cta_of(c.kend - cm.per_unit(c.b));
+    const int u_slot = s - cf;
+    const int u_parts = cm.cta_of(c.kend - 1) - cf + 1;
+    for (int ii = 0; ii < n_here; ++ii) {
+      const unsigned char* ktile = ring + sl * tile_bytes;
+      const unsigned char* vtile = ktile + TS::kBytes;
+      const unsigned char* side = side0 + sl * SM::kSide;
+      __syncwarp();   // the previous chunk's row data is read
+      mbar_wait(&s_full[sl], ph, status);
+      if (ii == 0) {
+        const T* qs = reinterpret_cast<const T*>(side + kOffArea);
+        if constexpr (kMma) { macc.load_q(qs); macc.reset(); }
+        else { facc.load_q(qs, A.scale); facc.reset(); }
       }
+      // rows r0 .. r0 + 7: counts and first slots from the chunk's offsets
+      const int32_t* offs = reinterpret_cast<const int32_t*>(side) + (int)((c.orow + c.c0) & 3);
+      const int off_l = lane <= 8 ? offs[r0 + lane] : 0;
+      {
+        const int o_next = __shfl_down_sync(0xffffffffu, off_l, 1);
+        if (lane < 8) {
+          const int cnt = o_next - off_l;
+          const bool ok = r0 + lane < c.nrows && cnt > 0;
+          rm[lane] = RowMult{1.f, (float)cnt, ok ? 1 : 0};
+        }
+        __syncwarp();
+      }
+      // scores, keys, estimation
+      float key_s[2] = {-INFINITY, -INFINITY};   // group max of rows 2tq, 2tq+1 (MMA) / lane's row (FMA)
+      if constexpr (kMma) {
+        float s0, s1;
+        macc.scores(ktile, r0, A.scale, s0, s1);
+        if (A.scores_out && g < G) {
+          const int cl = c.c0 + r0 + 2 * tq;
+          if (cl < c.c0 + c.nrows) A.scores_out[(c.row0 + cl) * G + g] = s0;
+          if (cl + 1 < c.c0 + c.nrows) A.scores_out[(c.row0 + cl + 1) * G + g] = s1;
+        }
+        float m0 = g < G ? s0 : -INFINITY, m1 = g < G ? s1 : -INFINITY;
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+          m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+        }
+        key_s[0] = m0;
+        key_s[1] = m1;
+        if (!A.exact_only) macc.fold(vtile, r0, s0, s1, rm);
+      } else {
+        facc.scores(ktile, r0, sc);
+        if (lane < 8) {
+          float mx = -INFINITY;
+#pragma unroll
+          for (int gg = 0; gg < G; ++gg) mx = fmaxf(mx, sc[lane * G + gg]);
+          key_s[0] = mx;
+          if (A.scores_out) {
+            const int cl = c.c0 + r0 + lane;
+            if (cl < c.c0 + c.nrows)
+              for (int gg = 0; gg < G; ++gg) A.scores_out[(c.row0 + cl) * G + gg] = sc[lane * G + gg];
+          }
+        }
+        if (!A.exact_only) facc.fold(vtile, r0, sc, rm);
+      }
+      // the slot's last reads are done: release it to the producer
       __syncwarp();
-    }
-    // scores, keys, estimation
-    float key_s[2] = {-INFINITY, -INFINITY};   // group max of rows 2tq, 2tq+1 (MMA) / lane's row (FMA)
-    if constexpr (kMma) {
-      float s0, s1;
-      macc.scores(ktile, r0, A.scale, s0, s1);
-      if (A.scores_out && g < G) {
-        const int cl = c.c0 + r0 + 2 * tq;
-        if (cl < c.c0 + c.nrows) A.scores_out[(c.row0 + cl) * G + g] = s0;
-        if (cl + 1 < c.c0 + c.nrows) A.scores_out[(c.row0 + cl + 1) * G + g] = s1;
-      }
-      float m0 = g < G ? s0 : -INFINITY, m1 = g < G ? s1 : -INFINITY;
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
-        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
-      }
-      key_s[0] = m0;
-      key_s[1] = m1;
-      if (!A.exact_only) macc.fold(vtile, r0, s0, s1, rm);
-    } else {
-      facc.scores(ktile, r0, sc);
-      if (lane < 8) {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int gg = 0; gg < G; ++gg) mx = fmaxf(mx, sc[lane * G + gg]);
-        key_s[0] = mx;
-        if (A.scores_out) {
-          const int cl = c.c0 + r0 + lane;
-          if (cl < c.c0 + c.nrows)
-            for (int gg = 0; gg < G; ++gg) A.scores_out[(c.row0 + cl) * G + gg] = sc[lane * G + gg];
+      if (lane == 0) mbar_arrive(&s_empty[sl]);
+      if (++sl == slots) { sl = 0; ph ^= 1u; }
+      // the records {key, first slot} of the warp's 8 rows (lanes 0..7, one
+      // 64-byte store) and the first digit's histogram
+      {
+        float kv = key_s[0];
+        if constexpr (kMma) {
+          // MMA lane t (t < 4) holds the keys of rows 2t and 2t + 1
+          const float ka = __shfl_sync(0xffffffffu, key_s[0], (lane >> 1) & 3);
+          const float kb = __shfl_sync(0xffffffffu, key_s[1], (lane >> 1) & 3);
+          kv = (lane & 1) ? kb : ka;
+        }
+        if (lane < 8 && r0 + lane < c.nrows) {
+          const uint32_t key = rm[lane].valid ? ordered_key(kv) : 0u;
+          A.rec[c.row0 + c.c0 + r0 + lane] = make_uint2(key, (uint32_t)off_l);
+          if (key) atomicAdd(&hist16[key >> (kHistShift + 1)], 1u << (16 * ((key >> kHistShift) & 1u)));
         }
       }
-      if (!A.exact_only) facc.fold(vtile, r0, sc, rm);
+      since_flush += kTileRows;
+      if (since_flush >= 65536 - kTileRows && ii + 1 < n_here) {
+        // 16-bit counters near overflow inside a long unit: flush them now
+        csync();
+        int32_t* hg = A.hist + (int64_t)c.u * kHistBins;
+        for (int wd = tid; wd < kHistBins / 2; wd += kConsumers) {
+          const uint32_t v = hist16[wd];
+          if (v) {
+            if (v & 0xffffu) atomicAdd(hg + 2 * wd, (int)(v & 0xffffu));
+            if (v >> 16) atomicAdd(hg + 2 * wd + 1, (int)(v >> 16));
+            hist16[wd] = 0u;
+          }
+        }
+        since_flush = 0;
+        csync();
+      }
+      c.c0 += kTileRows;
+      c.nrows = min(kTileRows, c.NC - c.c0);
     }
-    // the slot's last reads are done: release it to the producer
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&s_empty[sl]);
-    // the records {key, first slot} of the warp's 8 rows (lanes 0..7, one
-    // 64-byte store) and the first digit's histogram
+    i += n_here;
+    // ---- end of the CTA's part of the unit: histogram, part, arrival
+    csync();
     {
-      float kv = key_s[0];
-      if constexpr (kMma) {
-        // MMA lane t (t < 4) holds the keys of rows 2t and 2t + 1
-        const float ka = __shfl_sync(0xffffffffu, key_s[0], (lane >> 1) & 3);
-        const float kb = __shfl_sync(0xffffffffu, key_s[1], (lane >> 1) & 3);
-        kv = (lane & 1) ? kb : ka;
-      }
-      if (lane < 8 && r0 + lane < c.nrows) {
-        const uint32_t key = rm[lane].valid ? ordered_key(kv) : 0u;
-        A.rec[c.row0 + c.c0 + r0 + lane] = make_uint2(key, (uint32_t)off_l);
-        if (key) atomicAdd(&hist16[key >> (kHistShift + 1)], 1u << (16 * ((key >> kHistShift) & 1u)));
-      }
-    }
-    since_flush += kTileRows;
-    // ---- end of the CTA's part of a unit: histogram, part, arrival
-    const bool unit_end = i == nk - 1 || c.k + 1 == c.kend;
-    if (unit_end || since_flush >= 65536 - kTileRows) {
-      csync();
       int32_t* hg = A.hist + (int64_t)c.u * kHistBins;
       for (int wd = tid; wd < kHistBins / 2; wd += kConsumers) {
         const uint32_t v = hist16[wd];
@@ -1358,26 +1375,24 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
         }
       }
       since_flush = 0;
-      csync();   // the words are clear before the next chunk counts into them
     }
-    if (unit_end) {
-      if (!A.exact_only) {
-        if constexpr (kMma) macc.to_smem(comb + warp * G * (D + kPartStride));
-        else facc.to_smem(comb + warp * G * (D + kPartStride));
-        csync();
-        float* part = A.est + ((int64_t)c.u * A.p1max + u_slot) * G * (D + kPartStride);
-        combine_warps<D, G>(comb, part, tid);
-      }
-      // every thread's records, histogram counts and part are written before
-      // the barrier; one fenced arrival publishes them (a cumulative fence)
+    csync();   // the words are clear before the next unit counts into them
+    if (!A.exact_only) {
+      if constexpr (kMma) macc.to_smem(comb + warp * G * (D + kPartStride));
+      else facc.to_smem(comb + warp * G * (D + kPartStride));
       csync();
-      if (tid == 0) {
+      float* part = A.est + ((int64_t)c.u * A.p1max + u_slot) * G * (D + kPartStride);
+      combine_warps<D, G>(comb, part, tid);
+    }
+    // every thread's records, histogram counts and part are written before
+    // the barrier; one fenced arrival publishes them (a cumulative fence)
+    csync();
+    if (tid == 0) {
+      __threadfence();
+      const int old = atomicAdd(A.cnt1 + c.u, 1);
+      if (old == u_parts - 1) {
         __threadfence();
-        const int old = atomicAdd(A.cnt1 + c.u, 1);
-        if (old == u_parts - 1) {
-          __threadfence();
-          s_tails[s_ntails++] = c.u;
-        }
+        s_tails[s_ntails++] = c.u;
       }
     }
   }

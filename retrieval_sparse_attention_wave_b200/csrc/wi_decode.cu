@@ -86,7 +86,9 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
   SteadyArgs sa{a.invperm, a.labels, a.offsets, p.n_sink, p.window, p.cap,
                 reinterpret_cast<int32_t*>(ws + p.off_info),
                 reinterpret_cast<int32_t*>(ws + p.off_st_slot),
-                reinterpret_cast<int2*>(ws + p.off_pc), reinterpret_cast<int2*>(ws + p.off_nonc)};
+                reinterpret_cast<int2*>(ws + p.off_pc), reinterpret_cast<int2*>(ws + p.off_nonc),
+                reinterpret_cast<int32_t*>(ws + p.off_hist), reinterpret_cast<int32_t*>(ws + p.off_cnt1),
+                reinterpret_cast<int32_t*>(ws + p.off_cnt2)};
   const size_t st_smem = decode_steady_smem(p.cap);
   set_smem(wave_steady_kernel, st_smem);
   const cudaError_t e = launch_ex(wave_steady_kernel, dim3(p.U), dim3(256), st_smem, s, false,

@@ -374,6 +374,9 @@ struct SteadyArgs {
   int32_t* st_slot;  // [U][cap] steady slots, ascending
   int2* pc;          // [U][cap] (slot, cluster) of steady tokens of candidate clusters
   int2* nonc;        // [U][cap] (cluster, count) of clusters without a non-steady token
+  int32_t* hist;     // [U][kHistBins] the scan's first-digit histograms, cleared here
+  int32_t* cnt1;     // [U] the scan's arrivals, cleared here
+  int32_t* cnt2;     // [U] the gather's arrivals, cleared here
 };
 
 __global__ void __launch_bounds__(256)
@@ -388,6 +391,11 @@ wave_steady_kernel(const Geo geo, const SteadyArgs a, uint32_t* status) {
   const int n_st = ns + (Tb - wstart);
   const int tid = threadIdx.x, lane = tid & 31;
   int32_t* I = a.info + (int64_t)u * kInfoInts;
+  // this call's counters start from zero whatever an earlier call left (the
+  // scan and the gather touch them only after this kernel has finished)
+  for (int i = tid; i < kHistBins / 4; i += blockDim.x)
+    reinterpret_cast<int4*>(a.hist + (int64_t)u * kHistBins)[i] = make_int4(0, 0, 0, 0);
+  if (tid == 0) { a.cnt1[u] = 0; a.cnt2[u] = 0; }
   if (n_st >= Tb) {   // all steady: attended densely, nothing retrieved or estimated
     if (tid < kInfoInts) {
       int v = 0;
@@ -823,58 +831,33 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
   get_round(0);
   reinterpret_cast<int4*>(s_hist)[tid] = h0;
   reinterpret_cast<int4*>(s_hist)[kConsumers + tid] = h1;
-  reinterpret_cast<int4*>(hg)[tid] = make_int4(0, 0, 0, 0);               // clean for the next call
-  reinterpret_cast<int4*>(hg)[kConsumers + tid] = make_int4(0, 0, 0, 0);
   csync();
   // the clusters left without a non-steady token are not candidates: their
-  // keys leave the histogram and become 0 (in the records; the round is
-  // staged again), once, at the round's first staging
-  auto apply_nonc = [&](int r) {
+  // keys leave the histogram and become 0 in the records (round 0 is staged
+  // again)
+  if (n_nonc > 0) {
     for (int j = tid; j < n_nonc; j += kConsumers) {
-      const int c = __ldcg(&nonc[j].x), i = c - r * kTailRound;
-      if (i >= 0 && i < kTailRound && c < NC) {
-        const uint32_t key = stage[rpad(i)].x;
+      const int c = __ldcg(&nonc[j].x);
+      if (c >= 0 && c < NC) {
+        const uint32_t key = __ldcg(&rec[c].x);
         if (key) {
           atomicSub(&s_hist[key >> kHistShift], 1);
           __stcg(&rec[c].x, 0u);
         }
       }
     }
-    csync();       // the cleared keys are visible before the round is staged again
+    csync();   // the cleared keys are visible before the round is staged again
     loaded = -1;
-    get_round(r);
-  };
-  if (n_nonc > 0) apply_nonc(0);
-
-  // ---- candidates: the nonzero keys; the histogram must hold as many (a
-  // stale one, left by a failed call, is rebuilt)
-  int cand = 0;
-  for (int r = 0; r < n_rounds; ++r) {
-    if (loaded != r) {
-      get_round(r);
-      if (n_nonc > 0) apply_nonc(r);
-    }
-#pragma unroll 4
-    for (int j = 0; j < kTailSteps; ++j) cand += key_of(j) != 0u;
+    get_round(0);
   }
+  // ---- candidates: the histogram's total (the steady kernel cleared it, and
+  // the threshold bin's member count is checked against it below)
   int hs = 0;
 #pragma unroll
   for (int i = 0; i < kHistBins / kConsumers; ++i) hs += s_hist[tid * (kHistBins / kConsumers) + i];
   int2 tot2;
-  wscan2(make_int2(warp_sum_int(cand), warp_sum_int(hs)), s_sh, &tot2);
+  wscan2(make_int2(warp_sum_int(hs), 0), s_sh, &tot2);
   const int n_cand = tot2.x;
-  if (tot2.y != n_cand) {
-    if (tid == 0) flag_error(status, WI_DEV_BAD_HIST);
-    for (int i = tid; i < kHistBins; i += kConsumers) s_hist[i] = 0;
-    csync();
-    for (int r = 0; r < n_rounds; ++r) {
-      get_round(r);
-#pragma unroll 4
-      for (int j = 0; j < kTailSteps; ++j)
-        if (key_of(j)) atomicAdd(&s_hist[key_of(j) >> kHistShift], 1);
-    }
-    csync();
-  }
   const int k_req = A.topk_clusters >= 0 ? A.topk_clusters
                                          : (int)ceil(A.topk_fraction * (double)NC);
   const int k = min(max(k_req, 0), n_cand);
@@ -882,6 +865,10 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
   int thr = -1;
   int bin1 = -1;
   uint64_t hstar = 0;
+  // a single round: this thread's records above the threshold bin and in it
+  // (masks), and the tokens above it, from the member pass
+  uint32_t am = 0u, bm1 = 0u;
+  int atok = 0;
 
   // the kth (1-based) record in id order that satisfies pred(key, id)
   auto ordered_pick = [&](auto&& pred, int kth) -> int {
@@ -918,25 +905,39 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
     // the threshold bin's members (key, id) when they fit; otherwise each
     // refinement pass reads the records again
     const bool fits = nb1 <= kTailCand;
-    if (fits) {
+    if (fits || n_rounds == 1) {
       int run = 0;
+      const int rb = kTailSteps * tid;
       for (int r = 0; r < n_rounds; ++r) {
         get_round(r);
         uint32_t m = 0u;
 #pragma unroll 4
-        for (int j = 0; j < kTailSteps; ++j)
-          m |= (key_of(j) != 0u && (int)(key_of(j) >> kHistShift) == bin1) ? 1u << j : 0u;
+        for (int j = 0; j < kTailSteps; ++j) {
+          const uint2 x = stage[rpad(rb + j)];
+          const uint32_t nx = stage[rpad(rb + j + 1)].y;
+          const int bn = (int)(x.x >> kHistShift);
+          const bool in = x.x != 0u && bn == bin1, up = x.x != 0u && bn > bin1;
+          m |= (uint32_t)in << j;
+          am |= (uint32_t)up << j;
+          atok += up ? (int)(nx - x.y) : 0;
+        }
+        bm1 = m;
         int2 t2;
         int pos = run + cscan2_excl(make_int2(__popc(m), 0), s_sh, &t2).x;
-        while (m) {
-          const int j = __ffs(m) - 1;
-          m &= m - 1u;
-          const uint2 x = stage[rpad(kTailSteps * tid + j)];
-          if (pos < kTailCand) s_cand[pos] = ((unsigned long long)x.x << 32) | id_of(r, j);
-          ++pos;
+        if (fits) {
+          while (m) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1u;
+            const uint2 x = stage[rpad(rb + j)];
+            if (pos < kTailCand) s_cand[pos] = ((unsigned long long)x.x << 32) | id_of(r, j);
+            ++pos;
+          }
         }
         run += t2.x;
       }
+      // the members counted must be the histogram's (its bins were cleared by
+      // the steady kernel; a mismatch says the workspace was disturbed)
+      if (tid == 0 && run != nb1) flag_error(status, WI_DEV_BAD_HIST);
       csync();
     }
     auto cand_key = [&](int i) { return (uint32_t)(s_cand[i] >> 32); };
@@ -1109,7 +1110,22 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
       uint32_t pm = 0u;
       int pt = 0;
       const int rb = kTailSteps * tid;
-      if (!th.sampled) {
+      if (n_rounds == 1 && bin1 >= 0) {
+        // a single round: the records above the threshold bin, and the bin's
+        // members that the threshold keeps (masks from the member pass)
+        pm = am;
+        pt = atok;
+        uint32_t mm = bm1;
+        while (mm) {
+          const int j = __ffs(mm) - 1;
+          mm &= mm - 1u;
+          const uint2 x = stage[rpad(rb + j)];
+          if (th.picked(x.x, id_of(r, j))) {
+            pm |= 1u << j;
+            pt += (int)(stage[rpad(rb + j + 1)].y - x.y);
+          }
+        }
+      } else if (!th.sampled) {
 #pragma unroll 4
         for (int j = 0; j < kTailSteps; ++j) {
           const uint2 x = stage[rpad(rb + j)];
@@ -1345,6 +1361,7 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
       since_flush += kTileRows;
       if (since_flush >= 65536 - kTileRows && ii + 1 < n_here) {
         // 16-bit counters near overflow inside a long unit: flush them now
+        pdl_wait();   // (the steady kernel has cleared the histograms)
         csync();
         int32_t* hg = A.hist + (int64_t)c.u * kHistBins;
         for (int wd = tid; wd < kHistBins / 2; wd += kConsumers) {
@@ -1363,6 +1380,7 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
     }
     i += n_here;
     // ---- end of the CTA's part of the unit: histogram, part, arrival
+    pdl_wait();   // the steady kernel has cleared the histograms and counters
     csync();
     {
       int32_t* hg = A.hist + (int64_t)c.u * kHistBins;

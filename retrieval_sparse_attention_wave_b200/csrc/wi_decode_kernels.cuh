@@ -1514,7 +1514,9 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
   }
   const int n2 = (A.n2_base[b + 1] - A.n2_base[b]) / geo.hkv;
   const int rel = (int)blockIdx.x - A.n2_base[b];
-  const int h = rel / n2, j = rel - h * n2;
+  // index j of the unit's CTAs major: the CTAs that launch first (one per SM)
+  // are the ones whose blocks are full
+  const int j = rel / geo.hkv, h = rel - j * geo.hkv;
   const int u = b * geo.hkv + h;
   const int Tb = geo.T(b);
   const int ns = min(A.n_sink, Tb), wstart = max(Tb - A.window, ns);
@@ -1781,8 +1783,8 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
       if (LN > kCancelRatio * fmaxf(L, 0.f)) flag_error(status, WI_DEV_CANCELLATION);
     }
   }
-  constexpr int kPS = G * (D + kPartStride);          // floats per part
-  constexpr int PB = (int)(SM::kTiles / (kPS * 4));   // parts per staged batch
+  constexpr int kPO = G * D;                          // staged floats per part: its outputs
+  constexpr int PB = (int)(SM::kTiles / (kPO * 4));   // parts per staged batch
   float* stage = reinterpret_cast<float*>(tiles);
   constexpr int kOut = (G * D + kGatherThreads - 1) / kGatherThreads;
   float O[kOut];
@@ -1791,8 +1793,12 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
   for (int p0 = 0; p0 < np; p0 += PB) {
     const int nb = min(PB, np - p0);
     __syncthreads();   // the previous batch (and the factors) are read
-    for (int x = tid; x < nb * kPS / 4; x += blockDim.x)
-      cp_async16(stage + 4 * x, part_ptr(p0) + 4 * x);   // parts of a unit are contiguous
+    for (int x = tid; x < nb * kPO / 4; x += blockDim.x) {
+      const int pp = x / (kPO / 4), rem = x - pp * (kPO / 4);
+      const int gg = rem / (D / 4), c4 = rem - gg * (D / 4);
+      cp_async16(stage + pp * kPO + gg * D + 4 * c4,
+                 part_ptr(p0 + pp) + gg * (D + kPartStride) + kPartStride + 4 * c4);
+    }
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
@@ -1802,7 +1808,7 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
       if (i < G * D) {
         const int gg = i / D, e = i - gg * D;
         for (int p = 0; p < nb; ++p)
-          O[k] += s_f[3 * ((p0 + p) * G + gg)] * stage[p * kPS + gg * (D + kPartStride) + kPartStride + e];
+          O[k] += s_f[3 * ((p0 + p) * G + gg)] * stage[p * kPO + gg * D + e];
       }
     }
   }

@@ -106,13 +106,13 @@ def test_decode_workspace_size_and_layout():
     # 131072 tokens, 8 KV heads: 8192 clusters per head -> 128 chunks of 64,
     # 1024 chunks on 148 streaming CTAs; k = ceil(0.018 * 8192) = 148, so a
     # head expects 148 * 16 retrieved + 68 steady + 148 + 68 correction rows
-    # = 2652 rows, plus a quarter: 3315 -> 26 gather CTAs of 128 rows per head
-    (W.WI_BF16, 128, [131072], dict(n_scan_ctas=148, n_gather_ctas=208)),
+    # = 2652 rows, plus half: 3978 -> 32 gather CTAs of 128 rows per head
+    (W.WI_BF16, 128, [131072], dict(n_scan_ctas=148, n_gather_ctas=256)),
     # fp32: the same chunking (64-row tiles whatever the row size)
-    (W.WI_F32, 128, [131072], dict(n_scan_ctas=148, n_gather_ctas=208)),
+    (W.WI_F32, 128, [131072], dict(n_scan_ctas=148, n_gather_ctas=256)),
     # ragged batch: 256 clusters (4 chunks) and 19 clusters (1 chunk) per
-    # head -> 40 chunks, 40 CTAs; 221 and 153 expected rows, plus a quarter
-    # (276, 191) -> 3 + 2 gather CTAs per head
+    # head -> 40 chunks, 40 CTAs; 221 and 153 expected rows, plus half
+    # (331, 229) -> 3 + 2 gather CTAs per head
     (W.WI_BF16, 128, [4096, 300], dict(n_scan_ctas=40, n_gather_ctas=40)),
 ])
 def test_decode_plan_shapes(dtype, d, seq, expect):

@@ -42,7 +42,10 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
+#include <utility>
 #include <type_traits>
 
 #include <cuda.h>
@@ -1895,11 +1898,47 @@ bool encode_offsets(CUtensorMap* tm, const int32_t* base, int64_t n) {
 // Dynamic shared memory limit, and the full shared-memory carveout for every
 // decode kernel (kernels that overlap under programmatic dependent launch
 // then never need the SM's L1 / shared split reconfigured between them).
+// The attributes are set once per device and kernel, raised when a call
+// needs more (each setting is a driver call on the decode's launch path).
 template <typename Kern>
 void set_smem(Kern kern, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, size_t> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  size_t& have = done[{dev, reinterpret_cast<const void*>(kern)}];
+  if (have >= bytes && have != 0) return;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                        (int)cudaSharedmemCarveoutMaxShared);
+  have = bytes;
+}
+
+// Tensor maps of recent calls' buffers, by (device, base, extent, row size,
+// type); a map describes the buffer only, so a hit is always valid.
+struct MapKey {
+  int dev, dtype, D;
+  const void* base;
+  int64_t n;
+  bool operator<(const MapKey& o) const {
+    return std::tie(dev, dtype, D, base, n) < std::tie(o.dev, o.dtype, o.D, o.base, o.n);
+  }
+};
+template <typename Encode>
+bool cached_map(CUtensorMap* tm, const MapKey& key, Encode&& encode) {
+  static std::mutex mu;
+  static std::map<MapKey, CUtensorMap> maps;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = maps.find(key);
+    if (it != maps.end()) { *tm = it->second; return true; }
+  }
+  if (!encode(tm)) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (maps.size() >= 64) maps.clear();
+  maps[key] = *tm;
+  return true;
 }
 
 int pow2_at_least(int n) {
@@ -1930,8 +1969,15 @@ cudaError_t launch_decode_typed(const DecodePlan& p, const DecodeArgs& a, const 
   std::memset(&tmv, 0, sizeof(tmv));
   std::memset(&tmo, 0, sizeof(tmo));
   const int64_t n_off = ((int64_t)p.geo.cl_base[p.geo.batch] + p.geo.batch) * p.geo.hkv;
-  if (!encode_rows(&tmc, a.centroids, p.ncl, D, p.dtype) ||
-      !encode_rows(&tmv, a.value_sums, p.ncl, D, p.dtype) || !encode_offsets(&tmo, a.offsets, n_off))
+  int dev = 0;
+  cudaGetDevice(&dev);
+  auto rows_map = [&](CUtensorMap* tm, const void* base) {
+    return cached_map(tm, MapKey{dev, p.dtype, D, base, p.ncl},
+                      [&](CUtensorMap* t) { return encode_rows(t, base, p.ncl, D, p.dtype); });
+  };
+  if (!rows_map(&tmc, a.centroids) || !rows_map(&tmv, a.value_sums) ||
+      !cached_map(&tmo, MapKey{dev, -1, 0, a.offsets, n_off},
+                  [&](CUtensorMap* t) { return encode_offsets(t, a.offsets, n_off); }))
     return cudaErrorInvalidValue;
   ScanArgs A{};
   A.q = a.q;

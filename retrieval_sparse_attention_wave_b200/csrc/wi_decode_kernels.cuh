@@ -1735,22 +1735,37 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
   }
   float* part = A.gat + ((int64_t)u * A.n2max + j) * G * (D + kPartStride);
   for (int i = tid; i < G * (D + kPartStride); i += blockDim.x) part[i] = s_part[i];
-  __threadfence();
+  // every thread's part is written before the barrier; one fenced arrival
+  // publishes it (a cumulative fence)
   __syncthreads();
   if (tid == 0) {
-    const int old = atomicAdd(A.cnt2 + u, 1);
     __threadfence();
+    const int old = atomicAdd(A.cnt2 + u, 1);
+    if (old == n2 - 1) __threadfence();
     s_last = old == n2 - 1;
   }
   __syncthreads();
   if (!s_last) return;
-  // the merge of the unit's n2 parts: their (m, l, ln) first, then their
-  // outputs, staged in shared memory by asynchronous copies in batches of
-  // the tile area's size
+  // the merge of the unit's n2 parts: their outputs are staged in shared
+  // memory by asynchronous copies (the first batch issued now, beside the
+  // loads of their (m, l, ln)), in batches of the tile area's size
   const int np = n2;
   auto part_ptr = [&](int p) -> const float* {
     return A.gat + ((int64_t)u * A.n2max + p) * G * (D + kPartStride);
   };
+  constexpr int kPO = G * D;                          // staged floats per part: its outputs
+  constexpr int PB = (int)(SM::kTiles / (kPO * 4));   // parts per staged batch
+  float* stage = reinterpret_cast<float*>(tiles);
+  auto stage_batch = [&](int p0, int nb) {
+    for (int x = tid; x < nb * kPO / 4; x += blockDim.x) {
+      const int pp = x / (kPO / 4), rem = x - pp * (kPO / 4);
+      const int gg = rem / (D / 4), c4 = rem - gg * (D / 4);
+      cp_async16(stage + pp * kPO + gg * D + 4 * c4,
+                 part_ptr(p0 + pp) + gg * (D + kPartStride) + kPartStride + 4 * c4);
+    }
+    cp_async_commit();
+  };
+  stage_batch(0, min(PB, np));
   float* s_f = s_merge;                             // [kMergeParts][G] (m then factor, l, ln)
   float* s_M = s_merge + SM::kMergeParts * G * 3;   // [G] max, [G] denominator
   float* s_L = s_M + G;
@@ -1786,23 +1801,16 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
       if (LN > kCancelRatio * fmaxf(L, 0.f)) flag_error(status, WI_DEV_CANCELLATION);
     }
   }
-  constexpr int kPO = G * D;                          // staged floats per part: its outputs
-  constexpr int PB = (int)(SM::kTiles / (kPO * 4));   // parts per staged batch
-  float* stage = reinterpret_cast<float*>(tiles);
   constexpr int kOut = (G * D + kGatherThreads - 1) / kGatherThreads;
   float O[kOut];
 #pragma unroll
   for (int k = 0; k < kOut; ++k) O[k] = 0.f;
   for (int p0 = 0; p0 < np; p0 += PB) {
     const int nb = min(PB, np - p0);
-    __syncthreads();   // the previous batch (and the factors) are read
-    for (int x = tid; x < nb * kPO / 4; x += blockDim.x) {
-      const int pp = x / (kPO / 4), rem = x - pp * (kPO / 4);
-      const int gg = rem / (D / 4), c4 = rem - gg * (D / 4);
-      cp_async16(stage + pp * kPO + gg * D + 4 * c4,
-                 part_ptr(p0 + pp) + gg * (D + kPartStride) + kPartStride + 4 * c4);
+    if (p0 > 0) {
+      __syncthreads();   // the previous batch is read
+      stage_batch(p0, nb);
     }
-    cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
 #pragma unroll

@@ -269,6 +269,14 @@ wi_status make_build_plan(const wi_kv_cache* kv, int S, int cs, BuildPlan& pl) {
   pl.off_status = take(256);
   pl.off_cent32 = take((size_t)ncl * pl.D * 4);
   pl.off_assign = take((size_t)ntok * 4);
+  // bf16 keys: per (unit, segment), the two bf16 terms of each chunk of
+  // 128 centroids as operand tiles, and the centroids' squared norms
+  pl.nch = (int)cdiv(pl.max_ncl_seg, 128);
+  const size_t nchunks = (size_t)pl.U * max_nseg * pl.nch;
+  if (pl.dtype == WI_BF16) {
+    pl.off_cimg = take(nchunks * 2 * 128 * pl.D * 2);
+    pl.off_cn2 = take(nchunks * 128 * 4);
+  }
   pl.total = o;
   return WI_OK;
 }

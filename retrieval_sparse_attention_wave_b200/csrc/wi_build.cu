@@ -6,7 +6,9 @@
 //   init    centroid j of a segment = key at segment position j*cs
 //   assign  argmin_j sum_e (k_e - c_je)^2 in fp32 (direct form, no
 //           ||k||^2 - 2k.c + ||c||^2 cancellation), ties to the lower j;
-//           64 tokens x 64 centroids per tile, 4x4 outputs per thread
+//           fp32 keys: 64 tokens x 64 centroids per tile, 4x4 outputs per
+//           thread; bf16 keys: k.c on the tcgen05 tensor cores, the direct
+//           form wherever the two best are too close to call
 //   update  per (unit, segment): stable counting sort of the tokens by
 //           cluster, fp64 sums in ascending position, mean = sum / count;
 //           on the last round it also writes offsets, perm, invperm, labels, the
@@ -18,6 +20,7 @@
 
 #include "wi_common.cuh"
 #include "wi_plan.h"
+#include "wi_umma.cuh"
 
 namespace wi {
 namespace {
@@ -171,213 +174,312 @@ kmeans_assign_kernel(const Geo geo, const Pool kin, int S, int cs, const SegFrom
 
 // --------------------------------------------- assign on the tensor cores
 // bf16 keys are exact in bf16, so ||k - c||^2 = ||c||^2 - 2 k.c + ||k||^2
-// can take k.c from the tensor cores: the fp32 centroid c is split into
-// three bf16 terms c1 + c2 + c3 (c1 = bf16(c), c2 = bf16(c - c1), c3 =
-// bf16(c - c1 - c2); the rest is below 2^-24 |c|) and k.c1 + k.c2 + k.c3 is
-// accumulated in fp32 on m16n8k16 (the products of two bf16 values are exact
-// in fp32).  A CTA takes kMTok tokens of a segment against all its centroids,
-// kMCen at a time; each warp keeps, per token, the two smallest approximate
-// distances a = ||c||^2 - 2 k.c.
+// can take k.c from the tensor cores: the fp32 centroid c is split into two
+// bf16 terms c1 + c2 (c1 = bf16(c), c2 = bf16(c - c1); the rest is below
+// 2^-18 |c| elementwise) and k.c1 + k.c2 is accumulated in fp32 by tcgen05
+// MMAs in tensor memory (the products of two bf16 values are exact in fp32).
 //
-// The decision is the direct form's: the kernel above computes
+// kmeans_split_kernel writes, once per round, every segment's centroids as
+// the two terms' operand tiles (kUCen centroids x D, the MMA's K-major
+// 128-byte-swizzled layout, one tile per (chunk of kUCen centroids, term);
+// zero rows pad a segment's last chunk) and their ||c||^2 in fp32.
+// kmeans_assign_umma_kernel takes kUTok tokens of a segment (the MMA's M)
+// against every chunk of its centroids (the MMA's N): one warp streams the
+// chunks' term tiles into a ring of shared-memory stages with bulk copies,
+// one thread issues the MMAs (A = the keys, staged once; B = a term tile;
+// both terms of a chunk accumulate into the chunk's kUCen columns of tensor
+// memory, kUSlots chunks in flight), and four warps read each finished chunk
+// back, one token row per thread, keeping each token's two smallest
+// approximate distances a = ||c||^2 - 2 k.c.  Two CTAs share an SM, so one's
+// loads and read-back overlap the other's MMAs.
+//
+// The decision is the direct form's: the FMA kernel above computes
 // d = sum_e (k_e - c_e)^2 in fp32 (ascending e, fused multiply-add), and a
 // token whose two best approximate distances are more than delta apart takes
-// the best, since both |a - ||k - c||^2 + ||k||^2 ...| errors are below
-// delta / 2 (see the bound below); any other token re-evaluates the direct
-// form over all the segment's centroids, with the same arithmetic and the
-// same tie rule (lower index), so the assignment equals the direct form's.
+// the best, since both |a - ||k - c||^2 + ||k||^2| errors are below
+// delta / 2 (see the bound below); any other token (ties included)
+// re-evaluates the direct form over all the segment's centroids, with the
+// same arithmetic and the same tie rule (lower index), so the assignment
+// equals the direct form's.
 //
-// Error bound: the direct form sums 128 terms, error <= 128 * 2^-24 * d
-// <= 2^-17 (|k|^2 + |c|^2) * 2; the tensor-core form adds at most 384
-// accumulations of products bounded by |k||c| <= (|k|^2 + |c|^2) / 2, each
-// within 2^-23 relative, plus ||c||^2 in fp32 (128 * 2^-24 |c|^2): together
+// Error bound, with |k.c| <= |k||c| <= (|k|^2 + |c|^2) / 2: the direct form
+// sums D <= 128 terms, error <= 128 * 2^-24 * d <= 2^-16 (|k|^2 + |c|^2).
+// The tensor-core sum adds 2 D <= 256 exact products, in whatever order,
+// each addition within 2^-23 relative even if the accumulator truncates, so
+// 2 k.c is off by at most 2 * 256 * 2^-23 (|k|^2 + |c|^2) / 2 =
+// 2^-15 (|k|^2 + |c|^2); the split leaves 2 * 2^-18 |k||c| <=
+// 2^-18 (|k|^2 + |c|^2); ||c||^2 in fp32 adds 128 * 2^-24 |c|^2: together
 // below 2^-13 (|k|^2 + |c|^2).  delta = 2^-12 (|k|^2 + max |c|^2) leaves a
 // factor of two.
-constexpr int kMTok = 128, kMCen = 64;
+constexpr int kUTok = 128;      // tokens per CTA: the MMA's M, one tensor-memory lane each
+constexpr int kUCen = 128;      // centroids per chunk: the MMA's N
+constexpr int kUTerms = 2;      // bf16 terms per centroid
+constexpr int kUStages = 2;     // term tiles in flight
+constexpr int kUSlots = 2;      // chunks accumulating at once: kUSlots * kUCen columns
+constexpr int kUThreads = 192;  // warps 0..3 read the accumulators, 4 loads, 5 issues the MMAs
 
-__device__ __forceinline__ int mtile_off(int rows, int r, int c) {   // 16-byte chunk c of row r
+// byte offset of 16-byte chunk c of row r in a K-major, 128-byte-swizzled
+// operand tile of `rows` rows: K blocks of 64 bf16, each rows x 128 bytes
+__host__ __device__ __forceinline__ int mtile_off(int rows, int r, int c) {
   return (c >> 3) * (rows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
 }
 
+// first chunk of (unit u, segment seg) among the operand tiles and norms
+__host__ __device__ __forceinline__ int64_t cimg_chunk0(int u, int seg, int max_nseg, int nch) {
+  return ((int64_t)u * max_nseg + seg) * nch;
+}
+
 template <int D>
-__global__ void __launch_bounds__(256, 2)
-kmeans_assign_mma_kernel(const Geo geo, const Pool kin, int S, int cs, const SegFrom sf,
-                         const float* __restrict__ cent32, int32_t* __restrict__ assign,
-                         uint32_t* status) {
-  using T = __nv_bfloat16;
-  constexpr int CH = D / 8;                     // 16-byte chunks per bf16 row
-  extern __shared__ __align__(1024) unsigned char sh_mma[];
-  unsigned char* sk = sh_mma;                                  // [kMTok][D] bf16, swizzled
-  unsigned char* sc = sk + kMTok * D * 2;                      // 3 x [kMCen][D] bf16 terms
-  float* cn2 = reinterpret_cast<float*>(sc + 3 * kMCen * D * 2);   // [kMCen] |c|^2
-  float* xn2 = cn2 + kMCen;                                    // [kMTok] |k|^2
-  __shared__ float s_cmax2;
-  __shared__ int s_namb;
-  __shared__ int s_amb[kMTok];
+__global__ void __launch_bounds__(256)
+kmeans_split_kernel(const Geo geo, int S, int cs, const SegFrom sf, int max_nseg, int nch,
+                    const float* __restrict__ cent32, unsigned char* __restrict__ cimg,
+                    float* __restrict__ cn2) {
+  constexpr int CH = D / 8;                 // 16-byte chunks of a bf16 row
+  constexpr int CPB = 256 / CH;             // centroids per block
+  static_assert(kUCen % CPB == 0, "blocks tile a chunk");
+  constexpr size_t kTile = (size_t)kUCen * D * 2;
   const int u = blockIdx.z, b = u / geo.hkv, h = u - b * geo.hkv;
   const int T_ = geo.T(b);
   const int seg = sf.s0[b] + (int)blockIdx.y, start = seg * S;
   if (start >= T_) return;
   const int len = min(S, T_ - start);
-  const int t0 = blockIdx.x * kMTok;
-  if (t0 >= len) return;
-  const int ntok = min(kMTok, len - t0);
   const int ncl = (len + cs - 1) / cs;
+  const int j = blockIdx.x * CPB + (int)threadIdx.x / CH, c8 = (int)threadIdx.x % CH;
   const int64_t crow = geo.cl_row(b, h) + (int64_t)seg * (S / cs);
+  float v[8];
+  if (j < ncl) {
+    const float4 lo = *reinterpret_cast<const float4*>(cent32 + (crow + j) * D + c8 * 8);
+    const float4 hi = *reinterpret_cast<const float4*>(cent32 + (crow + j) * D + c8 * 8 + 4);
+    v[0] = lo.x; v[1] = lo.y; v[2] = lo.z; v[3] = lo.w;
+    v[4] = hi.x; v[5] = hi.y; v[6] = hi.z; v[7] = hi.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = 0.f;
+  }
+  uint32_t w[kUTerms][4];
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) split_bf16(v[e], v[e + 1], w[0][e / 2], w[1][e / 2]);
+  const int64_t ch0 = cimg_chunk0(u, seg, max_nseg, nch);
+  unsigned char* tiles = cimg + (ch0 + j / kUCen) * kUTerms * kTile;
+#pragma unroll
+  for (int t = 0; t < kUTerms; ++t)
+    *reinterpret_cast<uint4*>(tiles + t * kTile + mtile_off(kUCen, j % kUCen, c8)) =
+        make_uint4(w[t][0], w[t][1], w[t][2], w[t][3]);
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+#pragma unroll
+  for (int o = 1; o < CH; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (c8 == 0) cn2[ch0 * kUCen + j] = ss;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kUThreads, 2)
+kmeans_assign_umma_kernel(const Geo geo, const Pool kin, int S, int cs, const SegFrom sf,
+                          int max_nseg, int nch, const unsigned char* __restrict__ cimg,
+                          const float* __restrict__ cn2, const float* __restrict__ cent32,
+                          int32_t* __restrict__ assign, uint32_t* status) {
+  using T = __nv_bfloat16;
+  constexpr int CH = D / 8;                                // 16-byte chunks per bf16 row
+  constexpr uint32_t kTile = (uint32_t)kUCen * D * 2;      // a term tile (and the key tile)
+  static_assert(kUTok == kUCen, "A and B tiles share their K-block stride");
+  constexpr uint32_t kKBlock = (uint32_t)kUCen * 128;      // bytes between K blocks of 64 bf16
+  constexpr uint32_t kIdesc = umma_idesc_bf16_f32<kUTok, kUCen>();
+  constexpr int kRowsPerPass = kUThreads / CH;             // key rows staged per pass
+  constexpr int kPasses = (kUTok + kRowsPerPass - 1) / kRowsPerPass;
+  extern __shared__ unsigned char sh_umma_raw[];
+  unsigned char* sk = align_smem_1024(sh_umma_raw);        // keys [kUTok][D], swizzled
+  unsigned char* stg = sk + kTile;                         // kUStages term tiles
+  __shared__ __align__(8) uint64_t s_full[kUStages], s_empty[kUStages];
+  __shared__ __align__(8) uint64_t s_accf[kUSlots], s_acce[kUSlots], s_done;
+  __shared__ __align__(16) float s_cn2[kUSlots][kUCen];   // the chunks' ||c||^2 (+inf past the segment)
+  __shared__ uint32_t s_tmem;
+  __shared__ float s_cmax2;
+  __shared__ int s_namb;
+  __shared__ int s_amb[kUTok];
+  const int u = blockIdx.z, b = u / geo.hkv, h = u - b * geo.hkv;
+  const int T_ = geo.T(b);
+  const int seg = sf.s0[b] + (int)blockIdx.y, start = seg * S;
+  if (start >= T_) return;
+  const int len = min(S, T_ - start);
+  const int t0 = blockIdx.x * kUTok;
+  if (t0 >= len) return;
+  const int ntok = min(kUTok, len - t0);
+  const int ncl = (len + cs - 1) / cs;
+  const int nchs = (ncl + kUCen - 1) / kUCen;              // this segment's chunks
+  const int nst = kUTerms * nchs;                          // term tiles
+  const int64_t crow = geo.cl_row(b, h) + (int64_t)seg * (S / cs);
+  const int64_t ch0 = cimg_chunk0(u, seg, max_nseg, nch);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, tq = lane & 3;
+  const uint32_t ncols = nchs == 1 ? (uint32_t)kUCen : (uint32_t)(kUSlots * kUCen);
 
-  // keys of the tile (zero rows past the segment), and their squared norms
-  for (int x = tid; x < kMTok * CH; x += blockDim.x) {
-    const int r = x / CH, c = x - r * CH;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < ntok) {
-      const int64_t ro = pool_row(kin, geo.hkv, D, b, h, start + t0 + r, status);
-      if (ro >= 0) v = ld_stream(reinterpret_cast<const T*>(kin.base) + ro + c * 8);
+  if (tid == 0) {
+    for (int i = 0; i < kUStages; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 1);
     }
-    *reinterpret_cast<uint4*>(sk + mtile_off(kMTok, r, c)) = v;
+    for (int i = 0; i < kUSlots; ++i) {
+      mbar_init(&s_accf[i], 1);
+      mbar_init(&s_acce[i], 4);
+    }
+    mbar_init(&s_done, 1);
+    mbar_init_fence();
+    s_cmax2 = 0.f;
+    s_namb = 0;
   }
-  if (tid == 0) { s_cmax2 = 0.f; s_namb = 0; }
+  if (warp == 5) tmem_alloc(&s_tmem, ncols);
+  tc_fence_before();
   __syncthreads();
-  for (int r = warp; r < kMTok; r += 8) {
-    float ss = 0.f;
-    for (int c = lane; c < CH; c += 32) {
-      const uint4 v = *reinterpret_cast<const uint4*>(sk + mtile_off(kMTok, r, c));
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  // the first term tiles go out before the keys are staged
+  const int npre = min(nst, kUStages);
+  if (warp == 4 && lane == 0)
+    for (int i = 0; i < npre; ++i) {
+      mbar_arrive_expect(&s_full[i], kTile);
+      bulk_load(stg + (size_t)i * kTile, cimg + (size_t)(ch0 * kUTerms + i) * kTile, kTile, &s_full[i]);
+    }
+  // the keys (zero rows past the segment), every row's page looked up
+  // before any copy is issued; read by the MMAs through the async proxy
+  {
+    const int c = tid % CH;
+    int64_t ro[kPasses];
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+      const int r = tid / CH + p * kRowsPerPass;
+      ro[p] = r < ntok ? pool_row(kin, geo.hkv, D, b, h, start + t0 + r, status) : -1;
+    }
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+      const int r = tid / CH + p * kRowsPerPass;
+      if (r < kUTok) {
+        unsigned char* dst = sk + mtile_off(kUTok, r, c);
+        if (ro[p] >= 0) cp_async16(dst, reinterpret_cast<const T*>(kin.base) + ro[p] + c * 8);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    cp_async_commit();
+    float m = 0.f;   // the largest ||c||^2 of the segment (norms are >= 0)
+    for (int j = tid; j < ncl; j += kUThreads) m = fmaxf(m, __ldg(cn2 + ch0 * kUCen + j));
+    atomicMax(reinterpret_cast<int*>(&s_cmax2), __float_as_int(m));
+    cp_async_wait<0>();
+  }
+  fence_proxy_async();
+  __syncthreads();
+
+  if (warp == 4) {
+    // ---- loads: term tile i = kUTerms c + t of chunk c into stage i % kUStages
+    if (lane == 0) {
+      int issued = npre;
+      for (int i = npre; i < nst; ++i) {
+        const int s = i % kUStages;
+        if (!mbar_wait(&s_empty[s], (uint32_t)((i / kUStages) - 1) & 1u, status)) break;
+        mbar_arrive_expect(&s_full[s], kTile);
+        bulk_load(stg + (size_t)s * kTile, cimg + (size_t)(ch0 * kUTerms + i) * kTile, kTile, &s_full[s]);
+        issued = i + 1;
+      }
+      // no copy is left in flight when the CTA ends
+      for (int i = max(0, issued - kUStages); i < issued; ++i)
+        mbar_wait(&s_full[i % kUStages], (uint32_t)(i / kUStages) & 1u, status);
+    }
+  } else if (warp == 5) {
+    // ---- MMAs: chunk c into columns (c % kUSlots) kUCen .., once the
+    // accumulators read back from them are free
+    if (lane == 0) {
+      const uint32_t a0 = smem_addr(sk);
+      for (int c = 0; c < nchs; ++c) {
+        const int slot = c % kUSlots;
+        if (c >= kUSlots && !mbar_wait(&s_acce[slot], (uint32_t)((c / kUSlots) - 1) & 1u, status)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int t = 0; t < kUTerms && ok; ++t) {
+          const int i = kUTerms * c + t, s = i % kUStages;
+          ok = mbar_wait(&s_full[s], (uint32_t)(i / kUStages) & 1u, status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t b0 = smem_addr(stg + (size_t)s * kTile);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {   // K = 16 per MMA: 32 bytes of each row
+            const uint32_t ko = (uint32_t)(k >> 2) * kKBlock + (uint32_t)(k & 3) * 32u;
+            umma_bf16(tmem + (uint32_t)(slot * kUCen), umma_desc_sw128(a0 + ko),
+                      umma_desc_sw128(b0 + ko), kIdesc, (t | k) != 0);
+          }
+          umma_commit(&s_empty[s]);   // the stage is free once these MMAs are done
+        }
+        if (!ok) break;
+        umma_commit(&s_accf[slot]);
+      }
+      // every MMA issued has completed before the columns are released
+      umma_commit(&s_done);
+      mbar_wait(&s_done, 0u, status);
+    }
+  } else {
+    // ---- accumulators: token row r = 32 warp + lane, lane r of tensor memory
+    const int r = 32 * warp + lane;
+    float xn2 = 0.f;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
       float xv[8];
-      Elem<T>::unpack(v, xv);
+      Elem<T>::unpack(*reinterpret_cast<const uint4*>(sk + mtile_off(kUTok, r, c)), xv);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(xv[e], xv[e], ss);
+      for (int e = 0; e < 8; ++e) xn2 = fmaf(xv[e], xv[e], xn2);
     }
-    ss = warp_sum(ss);
-    if (lane == 0) xn2[r] = ss;
-  }
-  // A fragments of the warp's 16 tokens, all k-steps (kept in registers)
-  uint32_t qa[D / 16][4];
-#pragma unroll
-  for (int ks = 0; ks < D / 16; ++ks)
-    ldsm_x4(qa[ks], sk + mtile_off(kMTok, 16 * warp + (lane & 15), 2 * ks + (lane >> 4)));
-
-  float b1[2] = {INFINITY, INFINITY}, b2[2] = {INFINITY, INFINITY};
-  int i1[2] = {0, 0};
-  for (int cb = 0; cb < ncl; cb += kMCen) {
-    __syncthreads();
-    // the chunk's centroids: three bf16 terms each, and |c|^2 in fp32
-    for (int x = tid; x < kMCen * (D / 8); x += blockDim.x) {
-      const int j = x / (D / 8), c8 = x - j * (D / 8);
-      float v[8];
-      if (cb + j < ncl) {
-        const float4 lo = *reinterpret_cast<const float4*>(cent32 + (crow + cb + j) * D + c8 * 8);
-        const float4 hi = *reinterpret_cast<const float4*>(cent32 + (crow + cb + j) * D + c8 * 8 + 4);
-        v[0] = lo.x; v[1] = lo.y; v[2] = lo.z; v[3] = lo.w;
-        v[4] = hi.x; v[5] = hi.y; v[6] = hi.z; v[7] = hi.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+    // b1 <= b2: the two smallest a, i1: the index of b1 (equal values make
+    // b2 == b1 and send the token to the direct form)
+    float b1 = INFINITY, b2 = INFINITY;
+    int i1 = 0;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+    for (int c = 0; c < nchs; ++c) {
+      const int slot = c % kUSlots;
+      {
+        const int j = c * kUCen + r;
+        s_cn2[slot][r] = j < ncl ? __ldg(cn2 + ch0 * kUCen + j) : INFINITY;
       }
-      uint32_t w[3][4];
+      named_sync(1, 128);   // the chunk's norms (every reader of chunk c - kUSlots is past it)
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_accf[slot], (uint32_t)(c / kUSlots) & 1u, status));
+      tc_fence_after();
+      if (ok) {
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const __nv_bfloat162 t1 = __floats2bfloat162_rn(v[e], v[e + 1]);
-        const float2 f1 = __bfloat1622float2(t1);
-        const float r0 = v[e] - f1.x, r1 = v[e + 1] - f1.y;
-        const __nv_bfloat162 t2 = __floats2bfloat162_rn(r0, r1);
-        const float2 f2 = __bfloat1622float2(t2);
-        const __nv_bfloat162 t3 = __floats2bfloat162_rn(r0 - f2.x, r1 - f2.y);
-        w[0][e / 2] = *reinterpret_cast<const uint32_t*>(&t1);
-        w[1][e / 2] = *reinterpret_cast<const uint32_t*>(&t2);
-        w[2][e / 2] = *reinterpret_cast<const uint32_t*>(&t3);
-      }
+        for (int q = 0; q < kUCen / 32; ++q) {
+          float v[32];
+          tmem_ld32(lane_base + (uint32_t)(slot * kUCen + 32 * q), v);
 #pragma unroll
-      for (int t = 0; t < 3; ++t)
-        *reinterpret_cast<uint4*>(sc + t * kMCen * D * 2 + mtile_off(kMCen, j, c8)) =
-            make_uint4(w[t][0], w[t][1], w[t][2], w[t][3]);
-    }
-    for (int j = warp; j < kMCen; j += 8) {
-      float ss = 0.f;
-      if (cb + j < ncl)
-        for (int e = lane; e < D; e += 32) {
-          const float c = cent32[(crow + cb + j) * D + e];
-          ss = fmaf(c, c, ss);
-        }
-      ss = warp_sum(ss);
-      if (lane == 0) {
-        cn2[j] = ss;
-        atomicMax(reinterpret_cast<int*>(&s_cmax2), __float_as_int(ss));   // ss >= 0
-      }
-    }
-    __syncthreads();
-    // k.c for the warp's 16 tokens x the chunk's 64 centroids
-    float acc[kMCen / 8][4];
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 n4 = *reinterpret_cast<const float4*>(&s_cn2[slot][32 * q + 4 * e4]);
+            const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
 #pragma unroll
-    for (int nt = 0; nt < kMCen / 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-#pragma unroll
-    for (int t = 0; t < 3; ++t) {
-      const unsigned char* ct = sc + t * kMCen * D * 2;
-#pragma unroll
-      for (int nt = 0; nt < kMCen / 8; ++nt) {
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ks += 2) {
-          uint32_t bm[4];
-          ldsm_x4(bm, ct + mtile_off(kMCen, 8 * nt + (lane & 7), 2 * ks + (lane >> 3)));
-          mma_bf16_4(acc[nt], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], bm[0], bm[1]);
-          mma_bf16_4(acc[nt], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3],
-                     bm[2], bm[3]);
+            for (int e = 0; e < 4; ++e) {
+              const float a = fmaf(-2.f, v[4 * e4 + e], nn[e]);
+              i1 = a < b1 ? c * kUCen + 32 * q + 4 * e4 + e : i1;
+              b2 = fminf(b2, fmaxf(b1, a));
+              b1 = fminf(b1, a);
+            }
+          }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_acce[slot]);
     }
-    // the two smallest a = |c|^2 - 2 k.c per token (rows g, g + 8), lower
-    // index first on equal values
-#pragma unroll
-    for (int nt = 0; nt < kMCen / 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = 8 * nt + 2 * tq + (e & 1);
-        const int tk = e >> 1;
-        if (cb + j < ncl) {
-          const float a = cn2[j] - 2.f * acc[nt][e];
-          if (a < b1[tk]) { b2[tk] = b1[tk]; b1[tk] = a; i1[tk] = cb + j; }
-          else if (a < b2[tk]) b2[tk] = a;
-        }
-      }
-  }
-  // merge over the four lanes that share the tokens
-#pragma unroll
-  for (int tk = 0; tk < 2; ++tk) {
-#pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-      const float ob1 = __shfl_xor_sync(0xffffffffu, b1[tk], o);
-      const float ob2 = __shfl_xor_sync(0xffffffffu, b2[tk], o);
-      const int oi1 = __shfl_xor_sync(0xffffffffu, i1[tk], o);
-      if (ob1 < b1[tk] || (ob1 == b1[tk] && oi1 < i1[tk])) {
-        b2[tk] = fminf(b1[tk], ob2);
-        b1[tk] = ob1;
-        i1[tk] = oi1;
-      } else {
-        b2[tk] = fminf(b2[tk], ob1);
-      }
+    int32_t* dst = assign + geo.tok_row(b, h) + start + t0;
+    if (r < ntok) {
+      const float delta = ldexpf(xn2 + s_cmax2, -12);
+      if (b2 - b1 > delta) dst[r] = i1;
+      else s_amb[atomicAdd(&s_namb, 1)] = r;
     }
   }
+  tc_fence_before();
   __syncthreads();
-  const float cmax2 = s_cmax2;
-  int32_t* dst = assign + geo.tok_row(b, h) + start + t0;
-  if (tq == 0) {
-#pragma unroll
-    for (int tk = 0; tk < 2; ++tk) {
-      const int r = 16 * warp + g + 8 * tk;
-      if (r < ntok) {
-        const float delta = ldexpf(xn2[r] + cmax2, -12);
-        if (b2[tk] - b1[tk] > delta) dst[r] = i1[tk];
-        else s_amb[atomicAdd(&s_namb, 1)] = r;
-      }
-    }
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, ncols);
   }
-  __syncthreads();
   // near the decision boundary: the direct form over every centroid, as the
   // FMA kernel computes it (fp32, ascending e, lower index on ties)
+  int32_t* dst = assign + geo.tok_row(b, h) + start + t0;
   const int namb = s_namb;
-  for (int a = warp; a < namb; a += 8) {
+  for (int a = warp; a < namb; a += kUThreads / 32) {
     const int r = s_amb[a];
     float best = INFINITY;
     int bi = 0;
@@ -385,9 +487,9 @@ kmeans_assign_mma_kernel(const Geo geo, const Pool kin, int S, int cs, const Seg
       const float* c = cent32 + (crow + j) * D;
       float acc = 0.f;
 #pragma unroll 4
-      for (int c8 = 0; c8 < D / 8; ++c8) {
+      for (int c8 = 0; c8 < CH; ++c8) {
         float xv[8];
-        Elem<T>::unpack(*reinterpret_cast<const uint4*>(sk + mtile_off(kMTok, r, c8)), xv);
+        Elem<T>::unpack(*reinterpret_cast<const uint4*>(sk + mtile_off(kUTok, r, c8)), xv);
         const float4 lo = *reinterpret_cast<const float4*>(c + c8 * 8);
         const float4 hi = *reinterpret_cast<const float4*>(c + c8 * 8 + 4);
         const float cv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
@@ -614,22 +716,25 @@ cudaError_t with_build_types(int dtype, int D, F&& f) {
 }
 
 size_t assign_smem(int D) { return (size_t)D * ((kTok + kPad) + (kCen + kPad)) * sizeof(float); }
-size_t assign_mma_smem(int D) {
-  return (size_t)kMTok * D * 2 + (size_t)3 * kMCen * D * 2 + (size_t)(kMCen + kMTok) * 4;
-}
+size_t assign_umma_smem(int D) { return 1024 + (size_t)(1 + kUStages) * kUCen * D * 2; }
 
-// One assignment pass over every unit's segments: the tensor-core kernel for
-// bf16 keys, the fp32 direct form otherwise.
+// One assignment pass over every unit's segments: the tensor-core kernels
+// for bf16 keys (the centroids' operand tiles, then the assignment), the
+// fp32 direct form otherwise.
 template <typename T, int D>
 cudaError_t launch_assign(const BuildPlan& p, const Pool& kin, const float* cent32,
-                          int32_t* assign, uint32_t* status, cudaStream_t s) {
+                          int32_t* assign, unsigned char* ws, uint32_t* status, cudaStream_t s) {
   if constexpr (std::is_same_v<T, __nv_bfloat16>) {
-    const size_t smem = assign_mma_smem(D);
-    cudaFuncSetAttribute(kmeans_assign_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    unsigned char* cimg = ws + p.off_cimg;
+    float* cn2 = reinterpret_cast<float*>(ws + p.off_cn2);
+    kmeans_split_kernel<D><<<dim3(p.nch * kUCen / (256 / (D / 8)), p.nseg_grid, p.U), 256, 0, s>>>(
+        p.geo, p.S, p.cs, p.sf, p.max_nseg, p.nch, cent32, cimg, cn2);
+    const size_t smem = assign_umma_smem(D);
+    cudaFuncSetAttribute(kmeans_assign_umma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    const dim3 grid((p.S + kMTok - 1) / kMTok, p.nseg_grid, p.U);
-    kmeans_assign_mma_kernel<D><<<grid, 256, smem, s>>>(p.geo, kin, p.S, p.cs, p.sf, cent32,
-                                                        assign, status);
+    const dim3 grid((p.S + kUTok - 1) / kUTok, p.nseg_grid, p.U);
+    kmeans_assign_umma_kernel<D><<<grid, kUThreads, smem, s>>>(
+        p.geo, kin, p.S, p.cs, p.sf, p.max_nseg, p.nch, cimg, cn2, cent32, assign, status);
   } else {
     const size_t smem = assign_smem(D);
     cudaFuncSetAttribute(kmeans_assign_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -647,7 +752,7 @@ cudaError_t launch_assign_only(const BuildPlan& p, const BuildArgs& a, const flo
                                int32_t* assign, cudaStream_t s) {
   uint32_t* status = reinterpret_cast<uint32_t*>(a.ws + p.off_status);
   return with_build_types(p.dtype, p.D, [&]<typename T, int D>() -> cudaError_t {
-    return launch_assign<T, D>(p, a.kin, cent32, assign, status, s);
+    return launch_assign<T, D>(p, a.kin, cent32, assign, a.ws, status, s);
   });
 }
 
@@ -676,7 +781,7 @@ cudaError_t launch_build(const BuildPlan& p, const BuildArgs& a, cudaStream_t s)
     fin.vin = a.vin;
     fin.enabled = 1;
     for (int it = 0; it < p.iters; ++it) {
-      const cudaError_t ea = launch_assign<T, D>(p, a.kin, cent32, assign, status, s);
+      const cudaError_t ea = launch_assign<T, D>(p, a.kin, cent32, assign, a.ws, status, s);
       if (ea != cudaSuccess) return ea;
       kmeans_update_kernel<T, D><<<dim3(p.nseg_grid, p.U), kUpdThreads, p.update_smem, s>>>(
           p.geo, a.kin, p.S, p.cs, p.sf, cent32, assign, it == p.iters - 1 ? fin : none, status);

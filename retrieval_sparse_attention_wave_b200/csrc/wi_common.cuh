@@ -83,6 +83,11 @@ __device__ __forceinline__ int64_t pool_row_pg(const Pool& p, int hkv, int d, in
   return ((((int64_t)pg * hkv + h) << p.page_shift) + row) * d;
 }
 
+// Hint: bring the 128-byte line holding ptr into L2.
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
+
 // 16-byte streaming load (read-only path, no L1 allocation).
 __device__ __forceinline__ uint4 ld_stream(const void* ptr) {
   uint4 r;

@@ -1529,6 +1529,11 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
   FmaAcc<D, G> facc;
   if constexpr (kMma) { macc.load_q(qg); macc.reset(); }
   else { facc.load_q(qg, A.scale); facc.reset(); }
+  // while the scan finishes: the sequence's block table into L2 (by the
+  // first CTA of each sequence; the token rows' page lookups hit it there)
+  if (rel == 0)
+    for (int i = 32 * tid; i < A.kp.max_pages; i += 32 * kGatherThreads)
+      prefetch_l2(A.kp.bt + (int64_t)b * A.kp.max_pages + i);
 
   pdl_wait();   // the scan's and the steady kernel's results
   // the unit's record, and (speculatively) where the first block's token
@@ -1586,10 +1591,14 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
       }
       __syncthreads();
     }
-    // ---- resolve the block's rows: kind, key and value row addresses
+    // ---- resolve the block's rows: kind, key and value row addresses (the
+    // token rows' positions and the partial rows' cluster keys, which only
+    // the attention needs, are loaded once the rows' copies are out)
+    int kind = kRowNone, aux = 0;
+    const int32_t* auxp = nullptr;
+    int auxc = -1;
     if (tid < RPB) {
       const int r = rb + tid;
-      int kind = kRowNone, aux = 0;
       const unsigned char* kr = nullptr;
       const unsigned char* vr = nullptr;
       int slot = -1, c = -1;
@@ -1631,9 +1640,10 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
           vr = vpool + ro * (int64_t)sizeof(T);
           if (kind == kRowToken) {
             if (slot >= Tb) { flag_error(status, WI_DEV_BAD_SLOT); kind = kRowNone; }
-            else aux = __ldg(A.perm + trow + slot);
+            else auxp = A.perm + trow + slot;
           } else if (kind == kRowPart) {
-            aux = (int)__ldcg(&A.rec[row0 + c].x);
+            auxp = reinterpret_cast<const int32_t*>(&A.rec[row0 + c].x);
+            auxc = c;
           }
         }
       }
@@ -1641,9 +1651,6 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
       s_aux[tid] = aux;
       s_kp[tid] = kind == kRowNone ? nullptr : kr;
       s_vp[tid] = kind == kRowNone ? nullptr : vr;
-      // a partial row's cluster is taken out of the estimate only when it
-      // is not retrieved
-      if (kind == kRowPart) s_aux[tid] = th.picked((uint32_t)aux, (uint32_t)c) ? 1 : 0;
     }
     __syncthreads();
     // ---- gather: every 16-byte chunk of the block's key and value rows
@@ -1658,6 +1665,13 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
       else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
     }
     cp_async_commit();
+    if (kind == kRowToken) {
+      s_aux[tid] = __ldg(auxp);   // the token's position in the sequence
+    } else if (kind == kRowPart) {
+      // a partial row's cluster is taken out of the estimate only when it
+      // is not retrieved
+      s_aux[tid] = th.picked(__ldcg(reinterpret_cast<const uint32_t*>(auxp)), (uint32_t)auxc) ? 1 : 0;
+    }
     cp_async_wait<0>();
     __syncthreads();
     // ---- attend: warp w takes rows 8w .. 8w + 7 of each tile

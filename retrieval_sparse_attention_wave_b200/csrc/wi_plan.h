@@ -86,7 +86,9 @@ struct BuildPlan {
   SegFrom sf;              // first segment per sequence
   int nseg_grid;           // max over sequences of (segments - first segment)
   size_t update_smem;
+  int nch;                 // chunks of 128 centroids per segment (tensor-core assignment)
   size_t off_status, off_cent32, off_assign;
+  size_t off_cimg, off_cn2;  // bf16 keys: the centroids' operand tiles and squared norms
   size_t total;
 };
 

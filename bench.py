@@ -36,8 +36,7 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse-decode µs/step/layer + achieved HBM GB/s (% of roofline), 128K–1M ctx"
 UNIT = "us/step/layer"
 FALLBACK_HBM_GBS = 6650.0
-# FP32 CUDA-core peak for the build's assignment (148 SMs x 128 lanes x 2 flop x 1.965 GHz)
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+FALLBACK_BF16_TFLOPS = 1590.0   # dense bf16 tensor-core burst (cuBLAS) on this part
 
 
 def measured_peaks():
@@ -46,7 +45,7 @@ def measured_peaks():
         with open(p) as f:
             d = json.load(f)
         return d, "measured"
-    return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS}, "fallback"
 
 
 def kernel_source_sha256() -> str:
@@ -244,6 +243,25 @@ def build_workload(cfg, dev, seed):
     return wl, kv, wx, bt_out, n_out, b0.elapsed_time(b1)
 
 
+def assign_round_us(W, wl, kv, wx, reps=10):
+    """One k-means assignment round over every segment (the build's hot
+    kernel pair), through the public assignment call, against the built
+    index's fp32 centroids: mean of `reps` event-timed calls after a warm-up."""
+    cent, _ = W.build_state(kv, wx)
+    cent = cent.clone()
+    ws = torch.empty(W.build_workspace_bytes(kv, wl.seg_len, wl.cluster_size), dtype=torch.uint8,
+                     device=cent.device)
+    W.kmeans_assign(kv, wl.seg_len, wl.cluster_size, cent, ws=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        W.kmeans_assign(kv, wl.seg_len, wl.cluster_size, cent, ws=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / reps
+
+
 class DecodeTimer:
     """Timed decode steps of one workload: R layer replicas of the index
     (R x step bytes > 2 x L2, so each step reads from HBM), one CUDA graph per
@@ -391,6 +409,7 @@ def run_wave(args, rank, world, local_rank):
 
     if args.decode_only:
         return run_decode_only(args, W, wl, kv, wx, dev, build_ms)
+    assign_us = assign_round_us(W, wl, kv, wx)
     # index extension: each sequence's last seg_len tokens arrive later (as a
     # decode appends them); the index of the shorter sequences grows to the
     # full ones, timed with events, and must equal the full build
@@ -551,7 +570,18 @@ def run_wave(args, rank, world, local_rank):
                 "d2h_bytes_per_step": int(out_h.numel() * 4 + lse_h.numel() * 4)},
         "build": {"ms": build_ms, "iters": wl.iters, "assign_tflop": assign_flop / 1e12,
                   "assign_tflops_achieved": assign_flop / (build_ms * 1e-3) / 1e12,
-                  "bound": "alu", "peak_tflops": FP32_ALU_TFLOPS},
+                  "assign_round_us": assign_us,
+                  # one assignment round (split + tensor-core kernel) against
+                  # the bf16 peak: the tensor cores do two bf16 terms per
+                  # centroid, twice the round's distance flops
+                  "assign_roofline": {
+                      "bound": "tensor",
+                      "achieved": 2 * assign_flop / wl.iters / (assign_us * 1e-6) / 1e12,
+                      "peak": float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)),
+                      "unit": "TFLOP/s",
+                      "frac": 2 * assign_flop / wl.iters / (assign_us * 1e-6) / 1e12
+                              / float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)),
+                      "peak_kind": peak_kind}},
         "block_topk": {"us_per_step": block_us, "wave_us_per_step_same_protocol": wave_flushed_us,
                        "note": "exact attention over the top blocks of cluster_size tokens "
                                "and the steady zone, no estimation; one graph per step, "

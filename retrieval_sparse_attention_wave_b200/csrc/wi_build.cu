@@ -513,6 +513,7 @@ kmeans_assign_umma_kernel(const Geo geo, const Pool kin, int S, int cs, const Se
 
 // ----------------------------------------------------------------- update
 constexpr int kUpdThreads = 512;
+constexpr int kUpdBatch = 8;   // cluster members whose rows are in flight together
 
 struct FinalOut {
   void* centroids;
@@ -603,32 +604,56 @@ kmeans_update_kernel(const Geo geo, const Pool kin, int S, int cs, const SegFrom
     double ks[R::EPL], vs[R::EPL];
 #pragma unroll
     for (int e = 0; e < R::EPL; ++e) { ks[e] = 0.0; vs[e] = 0.0; }
-    for (int m = m0; m < m1; ++m) {
-      const int p = start + s_mem[m];
-      const int64_t ro = pool_row(kin, geo.hkv, D, b, h, p, status);
-      if (ro < 0) continue;
-      const uint4 kraw = ld_stream(kb + ro);
-      float x[R::EPL];
-      Elem<T>::unpack(kraw, x);
+    // kUpdBatch members at a time: their pages looked up and their rows
+    // loaded together, then summed in ascending position order
+    for (int mb = m0; mb < m1; mb += kUpdBatch) {
+      int p[kUpdBatch];
+      int64_t ro[kUpdBatch];
+      uint4 kraw[kUpdBatch];
 #pragma unroll
-      for (int e = 0; e < R::EPL; ++e) ks[e] += (double)x[e];
+      for (int q = 0; q < kUpdBatch; ++q) {
+        p[q] = mb + q < m1 ? start + s_mem[mb + q] : -1;
+        ro[q] = p[q] >= 0 ? pool_row(kin, geo.hkv, D, b, h, p[q], status) : -1;
+      }
+#pragma unroll
+      for (int q = 0; q < kUpdBatch; ++q) kraw[q] = ro[q] >= 0 ? ld_stream(kb + ro[q]) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int q = 0; q < kUpdBatch; ++q) {
+        if (ro[q] < 0) continue;
+        float x[R::EPL];
+        Elem<T>::unpack(kraw[q], x);
+#pragma unroll
+        for (int e = 0; e < R::EPL; ++e) ks[e] += (double)x[e];
+      }
       if (fo.enabled) {
-        const int slot = start + m;
-        const int64_t vo = pool_row(fo.vin, geo.hkv, D, b, h, p, status);
-        const int64_t oo = pool_row(fo.pout, geo.hkv, D, b, h, slot, status);
-        uint4 vraw = make_uint4(0, 0, 0, 0);
-        if (vo >= 0) vraw = ld_stream(reinterpret_cast<const T*>(fo.vin.base) + vo + sub * R::EPL);
-        Elem<T>::unpack(vraw, x);
+        int64_t vo[kUpdBatch], oo[kUpdBatch];
+        uint4 vraw[kUpdBatch];
 #pragma unroll
-        for (int e = 0; e < R::EPL; ++e) vs[e] += (double)x[e];
-        if (oo >= 0) {
-          *reinterpret_cast<uint4*>(reinterpret_cast<T*>(fo.kout) + oo + sub * R::EPL) = kraw;
-          *reinterpret_cast<uint4*>(reinterpret_cast<T*>(fo.vout) + oo + sub * R::EPL) = vraw;
+        for (int q = 0; q < kUpdBatch; ++q) {
+          vo[q] = ro[q] >= 0 ? pool_row(fo.vin, geo.hkv, D, b, h, p[q], status) : -1;
+          oo[q] = ro[q] >= 0 ? pool_row(fo.pout, geo.hkv, D, b, h, start + mb + q, status) : -1;
         }
-        if (sub == 0) {
-          fo.perm[trow + slot] = p;
-          fo.invperm[trow + p] = slot;
-          fo.labels[trow + p] = seg * (S / cs) + j;
+#pragma unroll
+        for (int q = 0; q < kUpdBatch; ++q)
+          vraw[q] = vo[q] >= 0 ? ld_stream(reinterpret_cast<const T*>(fo.vin.base) + vo[q] + sub * R::EPL)
+                               : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int q = 0; q < kUpdBatch; ++q) {
+          if (ro[q] < 0) continue;
+          const int slot = start + mb + q;
+          float x[R::EPL];
+          Elem<T>::unpack(vraw[q], x);
+#pragma unroll
+          for (int e = 0; e < R::EPL; ++e) vs[e] += (double)x[e];
+          if (oo[q] >= 0) {
+            *reinterpret_cast<uint4*>(reinterpret_cast<T*>(fo.kout) + oo[q] + sub * R::EPL) = kraw[q];
+            *reinterpret_cast<uint4*>(reinterpret_cast<T*>(fo.vout) + oo[q] + sub * R::EPL) = vraw[q];
+          }
+          if (sub == 0) {
+            fo.perm[trow + slot] = p[q];
+            fo.invperm[trow + p[q]] = slot;
+            fo.labels[trow + p[q]] = seg * (S / cs) + j;
+          }
         }
       }
     }

@@ -81,7 +81,6 @@ int64_t n_steady(int64_t T, int64_t n_sink, int64_t window) {
 
 
 // Chunk map of the scan: CTA that takes chunk k of n over N CTAs
-int scan_cta_of(int64_t k, int64_t n, int64_t N) { return (int)(((k + 1) * N - 1) / n); }
 
 wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, DecodePlan& pl) {
   if (!ix || !p) return WI_ERR_INVALID_ARG;
@@ -147,34 +146,20 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   }
   pl.n_chunks = pl.ch_base[B];
   pl.n_scan = std::max(1, std::min(pl.n_chunks, kNumSMs));
+  if ((int64_t)pl.n_chunks * pl.n_scan >= ((int64_t)1 << 32)) return WI_ERR_UNSUPPORTED;   // ChunkMap arithmetic
+  const ChunkMap cm = chunk_map(pl);
   pl.p1max = 1;
-  for (int b = 0; b < B; ++b) {
-    const int nch = (pl.ch_base[b + 1] - pl.ch_base[b]) / H;
-    for (int h = 0; h < H && nch > 0; ++h) {
-      const int64_t k0 = pl.ch_base[b] + (int64_t)h * nch;
-      const int parts = scan_cta_of(k0 + nch - 1, pl.n_chunks, pl.n_scan) -
-                        scan_cta_of(k0, pl.n_chunks, pl.n_scan) + 1;
-      pl.p1max = std::max(pl.p1max, parts);
-    }
-  }
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H && cm.per_unit(b) > 0; ++h) pl.p1max = std::max(pl.p1max, cm.parts(b, h));
   // units a scan CTA touches (it runs the tails of those it finishes last)
-  {
-    int b = 0;
-    for (int sc = 0; sc < pl.n_scan && pl.n_chunks > 0; ++sc) {
-      const int64_t k0 = (int64_t)sc * pl.n_chunks / pl.n_scan;
-      const int64_t k1 = (int64_t)(sc + 1) * pl.n_chunks / pl.n_scan;
-      int touched = 0, last_u = -1;
-      for (int64_t k = k0; k < k1; ++k) {
-        while (b + 1 < B && pl.ch_base[b + 1] <= k) ++b;
-        while (b > 0 && pl.ch_base[b] > k) --b;
-        const int per = (pl.ch_base[b + 1] - pl.ch_base[b]) / H;
-        const int u = b * H + (int)((k - pl.ch_base[b]) / per);
-        if (u != last_u) { ++touched; last_u = u; }
-        if (touched > kMaxTailsPerCta) return WI_ERR_UNSUPPORTED;
-        // skip to the unit's last chunk in this CTA's range
-        const int64_t unit_end = pl.ch_base[b] + (int64_t)(u - b * H + 1) * per;
-        k = std::min<int64_t>(k1, unit_end) - 1;
-      }
+  for (int sc = 0; sc < pl.n_scan && pl.n_chunks > 0; ++sc) {
+    const int k0 = cm.k0(sc), k1 = cm.k0(sc + 1);
+    int touched = 0;
+    for (int k = k0; k < k1;) {
+      const int b = cm.seq_of(k), per = cm.per_unit(b);
+      const int h = (k - cm.ch_base[b]) / per;
+      if (++touched > kMaxTailsPerCta) return WI_ERR_UNSUPPORTED;
+      k = std::min(k1, cm.first(b, h) + per);   // past the unit's last chunk in this CTA's range
     }
   }
   // ring slots: tile(s) plus the side area (offsets box, queries); about

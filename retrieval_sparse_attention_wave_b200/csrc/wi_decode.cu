@@ -76,12 +76,7 @@ cudaError_t launch_decode(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + p.off_status);
   cudaEvent_t* ev = a.stage_events;
   if (ev) cudaEventRecord(ev[0], s);
-  ChunkMap cm;
-  std::memcpy(cm.ch_base, p.ch_base, sizeof(cm.ch_base));
-  cm.n_chunks = p.n_chunks;
-  cm.n_scan = std::max(1, p.n_scan);
-  cm.batch = p.geo.batch;
-  cm.hkv = p.geo.hkv;
+  const ChunkMap cm = chunk_map(p);
   // K0: steady zone (a normal launch: everything before it in the stream is done)
   SteadyArgs sa{a.invperm, a.labels, a.offsets, p.n_sink, p.window, p.cap,
                 reinterpret_cast<int32_t*>(ws + p.off_info),

@@ -56,36 +56,6 @@
 
 namespace wi {
 
-// ----------------------------------------------------------- chunk map
-// The scan's work: the clusters of every unit that is not attended densely,
-// in chunks of kTileRows; sequence b's units own ch_base[b + 1] - ch_base[b]
-// chunks (Hkv units of equal count).  Scan CTA s takes chunks
-// [s n / N, (s + 1) n / N).
-struct ChunkMap {
-  int32_t ch_base[kMaxBatch + 1];
-  int n_chunks, n_scan, batch, hkv;
-  __device__ __forceinline__ int k0(int s) const { return (int)((int64_t)s * n_chunks / n_scan); }
-  // the scan CTA that takes chunk k
-  __device__ __forceinline__ int cta_of(int k) const {
-    return (int)(((int64_t)(k + 1) * n_scan - 1) / n_chunks);
-  }
-  __device__ __forceinline__ int seq_of(int k) const {
-    int lo = 0, hi = batch - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (ch_base[mid] <= k) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-  }
-  __device__ __forceinline__ int per_unit(int b) const { return (ch_base[b + 1] - ch_base[b]) / hkv; }
-  __device__ __forceinline__ int first(int b, int h) const { return ch_base[b] + h * per_unit(b); }
-  // scan parts (CTAs) of unit (b, h): the CTAs of its first and last chunk and between
-  __device__ __forceinline__ int parts(int b, int h) const {
-    const int n = per_unit(b);
-    return n == 0 ? 0 : cta_of(first(b, h) + n - 1) - cta_of(first(b, h)) + 1;
-  }
-};
-
 namespace {
 
 constexpr int kHistShift = 21;    // first radix digit: key bits 31..21
@@ -1535,6 +1505,8 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
     for (int i = 32 * tid; i < A.kp.max_pages; i += 32 * kGatherThreads)
       prefetch_l2(A.kp.bt + (int64_t)b * A.kp.max_pages + i);
 
+  const int np_scan = cm.parts(b, h);   // the scan's parts of the unit
+
   pdl_wait();   // the scan's and the steady kernel's results
   // the unit's record, and (speculatively) where the first block's token
   // rows start among the retrieved clusters
@@ -1547,7 +1519,7 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
   const bool dense = s_rec[kDense] != 0, no_est = s_rec[kNoEstimate] != 0;
   // the scan's estimation parts this CTA folds into its own (p = j, j + n2,
   // ...): the first one's copies go out now, to land during the gather
-  const int np1 = no_est ? 0 : cm.parts(b, h);
+  const int np1 = no_est ? 0 : np_scan;
   if (np1 > j) {
     const float* src = A.est + ((int64_t)u * A.p1max + j) * G * (D + kPartStride);
     for (int x = tid; x < G * (D + kPartStride) / 4; x += blockDim.x)

@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cstring>
 
 #include "wi_common.cuh"
 
@@ -26,6 +27,40 @@ constexpr int kHistBins = 2048;                   // first radix digit: key bits
 constexpr int kTailCand = 1024;                   // threshold-bin members refined in shared memory
 constexpr int kMaxGatherPerUnit = 64;             // gather CTAs per unit (they loop beyond)
 constexpr int kMaxTailsPerCta = 64;               // units one scan CTA may touch
+
+// The scan's work: the clusters of every unit that is not attended densely,
+// in chunks of kTileRows; sequence b's units own ch_base[b + 1] - ch_base[b]
+// chunks (Hkv units of equal count).  Scan CTA s takes chunks
+// [s n / N, (s + 1) n / N).  (32-bit unsigned arithmetic: the plan keeps
+// n * N below 2^32.)
+struct ChunkMap {
+  int32_t ch_base[kMaxBatch + 1];
+  int n_chunks, n_scan, batch, hkv;
+  __host__ __device__ __forceinline__ int k0(int s) const {
+    return (int)((uint32_t)s * (uint32_t)n_chunks / (uint32_t)n_scan);
+  }
+  // the scan CTA that takes chunk k
+  __host__ __device__ __forceinline__ int cta_of(int k) const {
+    return (int)(((uint32_t)(k + 1) * (uint32_t)n_scan - 1u) / (uint32_t)n_chunks);
+  }
+  __host__ __device__ __forceinline__ int seq_of(int k) const {
+    int lo = 0, hi = batch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (ch_base[mid] <= k) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  }
+  __host__ __device__ __forceinline__ int per_unit(int b) const {
+    return (int)((uint32_t)(ch_base[b + 1] - ch_base[b]) / (uint32_t)hkv);
+  }
+  __host__ __device__ __forceinline__ int first(int b, int h) const { return ch_base[b] + h * per_unit(b); }
+  // scan parts (CTAs) of unit (b, h): the CTAs of its first and last chunk and between
+  __host__ __device__ __forceinline__ int parts(int b, int h) const {
+    const int n = per_unit(b);
+    return n == 0 ? 0 : cta_of(first(b, h) + n - 1) - cta_of(first(b, h)) + 1;
+  }
+};
 
 // Per-unit record fields (int32 [U][kInfoInts]).
 enum UnitField {
@@ -73,6 +108,17 @@ struct DecodePlan {
   size_t off_est, off_gat, off_q, off_out, off_lse;
   size_t total;
 };
+
+// The scan's chunk map of a plan.
+inline ChunkMap chunk_map(const DecodePlan& p) {
+  ChunkMap cm;
+  std::memcpy(cm.ch_base, p.ch_base, sizeof(cm.ch_base));
+  cm.n_chunks = p.n_chunks;
+  cm.n_scan = p.n_scan > 0 ? p.n_scan : 1;
+  cm.batch = p.geo.batch;
+  cm.hkv = p.geo.hkv;
+  return cm;
+}
 // First segment each sequence's build kernels process (all zero for a full
 // build; an index extension starts at the old index's first incomplete one).
 struct SegFrom {

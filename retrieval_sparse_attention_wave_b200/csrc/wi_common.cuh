@@ -187,6 +187,11 @@ __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// Arrive at named barrier `id` (n threads in all) without waiting.
+__device__ __forceinline__ void named_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 // Loads of data other CTAs of the same grid wrote (L2, bypassing L1).
 __device__ __forceinline__ int ldcg_i32(const int32_t* p) { return __ldcg(p); }
 __device__ __forceinline__ uint32_t ldcg_u32(const uint32_t* p) { return __ldcg(p); }

@@ -337,6 +337,48 @@ __device__ __forceinline__ void combine_warps(const float* comb, float* part, in
   }
 }
 
+// combine_warps by one warp: lane l takes columns 4 l .. 4 l + 3 of every
+// head, each lane computing the heads' maxima and the warps' factors itself
+// (broadcast reads).
+template <int D, int G>
+__device__ __forceinline__ void combine_warps_1w(const float* comb, float* part, int lane) {
+  static_assert(D <= 128, "4 columns per lane");
+  constexpr int RS = D + kPartStride;
+  const int c = 4 * lane;
+#pragma unroll 1
+  for (int g = 0; g < G; ++g) {
+    float mw[kConsumerWarps];
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      mw[w] = comb[(w * G + g) * RS];
+      M = fmaxf(M, mw[w]);
+    }
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    float L = 0.f, LN = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float* row = comb + (w * G + g) * RS;
+      const float f = mw[w] == -INFINITY ? 0.f : __expf(mw[w] - M);
+      L = fmaf(f, row[1], L);
+      LN = fmaf(f, row[2], LN);
+      if (c < D) {
+        const float4 x = *reinterpret_cast<const float4*>(row + kPartStride + c);
+        o.x = fmaf(f, x.x, o.x);
+        o.y = fmaf(f, x.y, o.y);
+        o.z = fmaf(f, x.z, o.z);
+        o.w = fmaf(f, x.w, o.w);
+      }
+    }
+    if (c < D) *reinterpret_cast<float4*>(part + g * RS + kPartStride + c) = o;
+    if (lane == 0) {
+      part[g * RS] = M;
+      part[g * RS + 1] = L;
+      part[g * RS + 2] = LN;
+    }
+  }
+}
+
 // ------------------------------------------------------------- K0 steady
 struct SteadyArgs {
   const int32_t* invperm;
@@ -576,7 +618,6 @@ struct ScanSmem {
   static constexpr size_t kTailDrawOff = kTailCandOff + (size_t)kTailCand * 8;
   static constexpr size_t kTailShOff = kTailDrawOff + (size_t)kTailDraws * 8;
   static constexpr size_t kTail = kTailShOff + 512;
-  static constexpr size_t kUnion = kComb > kTail ? kComb : kTail;
   static constexpr size_t kHist16 = (size_t)kHistBins / 2 * 4;
   static constexpr size_t kRows = (size_t)kConsumerWarps * 8 * sizeof(RowMult);
   static constexpr size_t kSc = (size_t)kConsumerWarps * 8 * G * 4;
@@ -587,7 +628,7 @@ struct ScanSmem {
   }
   __host__ __device__ static size_t side_bytes(int slots) { return slots * kSide; }
   __host__ __device__ static size_t total(int slots, int exact_only) {
-    return 1024 + ring_bytes(slots, exact_only) + side_bytes(slots) + kUnion + kHist16 + kRows + kSc;
+    return 1024 + ring_bytes(slots, exact_only) + side_bytes(slots) + kTail + kComb + kHist16 + kRows + kSc;
   }
 };
 
@@ -1169,14 +1210,16 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
   __shared__ __align__(8) uint64_t s_full[4], s_empty[4];
   __shared__ int s_ntails;
   __shared__ int s_tails[kMaxTailsPerCta];   // units whose last arrival was this CTA's
+  __shared__ float* s_last_part;             // the CTA's last unit's estimation part
   pdl_launch_dependents();
   unsigned char* sh = align_smem_1024(sh_raw);
   const int slots = A.slots;
   const size_t tile_bytes = SM::tile_bytes(A.exact_only);
   unsigned char* ring = sh;
   unsigned char* side0 = ring + SM::ring_bytes(slots, A.exact_only);
-  unsigned char* s_union = side0 + SM::side_bytes(slots);
-  uint32_t* hist16 = reinterpret_cast<uint32_t*>(s_union + SM::kUnion);
+  unsigned char* s_tail = side0 + SM::side_bytes(slots);
+  float* comb = reinterpret_cast<float*>(s_tail + SM::kTail);   // per-warp softmax parts
+  uint32_t* hist16 = reinterpret_cast<uint32_t*>(reinterpret_cast<unsigned char*>(comb) + SM::kComb);
   RowMult* s_rows = reinterpret_cast<RowMult*>(reinterpret_cast<unsigned char*>(hist16) + SM::kHist16);
   float* s_sc = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(s_rows) + SM::kRows);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1230,6 +1273,13 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
       for (int i = max(0, nk - slots); i < nk; ++i)
         mbar_wait(&s_full[i % slots], (uint32_t)((i / slots) & 1), status);
     }
+    // the CTA's last estimation part, combined while the consumers run the
+    // tails (barrier 2: the consumers' warp parts are in shared memory)
+    if (!A.exact_only && nk > 0) {
+      __syncwarp();
+      named_sync(2, kScanThreads);
+      combine_warps_1w<D, G>(comb, s_last_part, lane);
+    }
     pdl_wait();
     return;
   }
@@ -1240,7 +1290,6 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
   FmaAcc<D, G> facc;
   const int g = lane >> 2, tq = lane & 3;
   int since_flush = 0;
-  float* comb = reinterpret_cast<float*>(s_union);
   RowMult* rm = s_rows + warp * 8;
   float* sc = s_sc + warp * 8 * G;
   const int r0 = 8 * warp;   // the warp's rows of every chunk
@@ -1352,7 +1401,7 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
       c.nrows = min(kTileRows, c.NC - c.c0);
     }
     i += n_here;
-    // ---- end of the CTA's part of the unit: histogram, part, arrival
+    // ---- end of the CTA's part of the unit: histogram, arrival, part
     pdl_wait();   // the steady kernel has cleared the histograms and counters
     csync();
     {
@@ -1367,23 +1416,31 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
       }
       since_flush = 0;
     }
-    csync();   // the words are clear before the next unit counts into them
-    if (!A.exact_only) {
-      if constexpr (kMma) macc.to_smem(comb + warp * G * (D + kPartStride));
-      else facc.to_smem(comb + warp * G * (D + kPartStride));
-      csync();
-      float* part = A.est + ((int64_t)c.u * A.p1max + u_slot) * G * (D + kPartStride);
-      combine_warps<D, G>(comb, part, tid);
-    }
-    // every thread's records, histogram counts and part are written before
-    // the barrier; one fenced arrival publishes them (a cumulative fence)
-    csync();
+    // every thread's records and histogram counts are written before the
+    // barrier; one fenced arrival publishes them (a cumulative fence)
+    csync();   // (and the words are clear before the next unit counts into them)
     if (tid == 0) {
       __threadfence();
       const int old = atomicAdd(A.cnt1 + c.u, 1);
       if (old == u_parts - 1) {
         __threadfence();
         s_tails[s_ntails++] = c.u;
+      }
+    }
+    // the estimation part is the gather's, read once the scan has completed:
+    // the warps' parts are combined after the arrival, the CTA's last unit's
+    // by the producer warp while the consumers run the tails
+    if (!A.exact_only) {
+      if constexpr (kMma) macc.to_smem(comb + warp * G * (D + kPartStride));
+      else facc.to_smem(comb + warp * G * (D + kPartStride));
+      csync();
+      float* part = A.est + ((int64_t)c.u * A.p1max + u_slot) * G * (D + kPartStride);
+      if (i < nk) {
+        combine_warps<D, G>(comb, part, tid);
+        csync();   // the parts are read before the next unit writes them
+      } else {
+        if (tid == 0) s_last_part = part;
+        named_arrive(2, kScanThreads);   // the producer warp combines it
       }
     }
   }
@@ -1394,7 +1451,7 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
   for (int t = 0; t < nt; ++t) {
     const int u = s_tails[t], b = u / geo.hkv, h = u - b * geo.hkv;
     const TailUnit tu{u, geo.NC(b), geo.T(b), geo.cl_row(b, h), geo.tok_row(b, h)};
-    scan_tail(tu, A, s_union, ring, SM::kTailCandOff, SM::kTailDrawOff, SM::kTailShOff, status);
+    scan_tail(tu, A, s_tail, ring, SM::kTailCandOff, SM::kTailDrawOff, SM::kTailShOff, status);
     csync();
   }
   pdl_wait();

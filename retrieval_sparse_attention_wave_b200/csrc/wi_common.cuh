@@ -187,6 +187,15 @@ __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// Release / acquire fence at GPU scope: the writes this thread has made or
+// observed (a CTA barrier before it included) are visible GPU-wide before
+// its later writes (a counter it then increments); for the thread that
+// reads the last increment, the others' published writes are visible after
+// it.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 // Arrive at named barrier `id` (n threads in all) without waiting.
 __device__ __forceinline__ void named_arrive(int id, int n) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");

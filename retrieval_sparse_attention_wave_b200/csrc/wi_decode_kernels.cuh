@@ -1420,10 +1420,10 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
     // barrier; one fenced arrival publishes them (a cumulative fence)
     csync();   // (and the words are clear before the next unit counts into them)
     if (tid == 0) {
-      __threadfence();
+      fence_acq_rel_gpu();
       const int old = atomicAdd(A.cnt1 + c.u, 1);
       if (old == u_parts - 1) {
-        __threadfence();
+        fence_acq_rel_gpu();
         s_tails[s_ntails++] = c.u;
       }
     }
@@ -1782,9 +1782,9 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
   // publishes it (a cumulative fence)
   __syncthreads();
   if (tid == 0) {
-    __threadfence();
+    fence_acq_rel_gpu();
     const int old = atomicAdd(A.cnt2 + u, 1);
-    if (old == n2 - 1) __threadfence();
+    if (old == n2 - 1) fence_acq_rel_gpu();
     s_last = old == n2 - 1;
   }
   __syncthreads();

@@ -313,27 +313,37 @@ struct FmaAcc {
 // Combine the per-warp parts comb [kConsumerWarps][G][D + 4] into one part
 // [G][D + 4] at `part` (threads 0 .. kConsumers - 1).
 template <int D, int G>
-__device__ __forceinline__ void combine_warps(const float* comb, float* part, int tid) {
-  for (int i = tid; i < G * D; i += kConsumers) {
-    const int g = i / D, e = i - g * D;
+__device__ __forceinline__ void combine_warps(float* comb, float* part, int tid) {
+  constexpr int RS = D + kPartStride;
+  // each head's maximum, denominators and the warps' factors (kept in each
+  // row's spare word 3) by one thread per head
+  if (tid < G) {
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * G + g) * (D + kPartStride)]);
-    float O = 0.f, L = 0.f, LN = 0.f;
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * G + tid) * RS]);
+    float L = 0.f, LN = 0.f;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
-      const float* row = comb + (w * G + g) * (D + kPartStride);
+      float* row = comb + (w * G + tid) * RS;
       const float f = row[0] == -INFINITY ? 0.f : __expf(row[0] - M);
-      O += f * row[kPartStride + e];
+      row[3] = f;
       L += f * row[1];
       LN += f * row[2];
     }
-    part[g * (D + kPartStride) + kPartStride + e] = O;
-    if (e == 0) {
-      part[g * (D + kPartStride)] = M;
-      part[g * (D + kPartStride) + 1] = L;
-      part[g * (D + kPartStride) + 2] = LN;
+    part[tid * RS] = M;
+    part[tid * RS + 1] = L;
+    part[tid * RS + 2] = LN;
+  }
+  named_sync(1, kConsumers);   // the consumer threads (all of the gather's)
+  for (int i = tid; i < G * D; i += kConsumers) {
+    const int g = i / D, e = i - g * D;
+    float O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float* row = comb + (w * G + g) * RS;
+      O += row[3] * row[kPartStride + e];
     }
+    part[g * RS + kPartStride + e] = O;
   }
 }
 

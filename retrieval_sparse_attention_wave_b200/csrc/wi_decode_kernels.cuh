@@ -84,6 +84,20 @@ __device__ __forceinline__ int tile_off(int r, int c) {
   return (c >> 3) * (kTileRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
 }
 
+// Tile layouts the accumulators read: the scan's (the swizzled boxes above,
+// as its tensor copies write them) and the gather's (whole rows of RB bytes,
+// RB + 16 apart, as its row copies write them: the pad puts the same 16-byte
+// chunk of eight consecutive rows in eight distinct groups of four banks).
+struct SwzTile {
+  __device__ static __forceinline__ int off(int r, int c) { return tile_off(r, c); }
+};
+template <int RB>
+struct PadTile {
+  static constexpr int kStride = RB + 16;
+  static constexpr int kBytes = kTileRows * kStride;
+  __device__ static __forceinline__ int off(int r, int c) { return r * kStride + c * 16; }
+};
+
 // Multipliers of the 8 rows a warp takes in one step: the row's weight in the
 // numerator (wo) and in the denominator (wl); invalid rows take no part.
 struct RowMult {
@@ -128,6 +142,7 @@ struct MmaAcc {
       for (int e = 0; e < 4; ++e) o[j][e] = 0.f;
   }
   // scores of rows r0 + 2t, r0 + 2t + 1 (t = lane % 4) for head lane / 4
+  template <class Lay = SwzTile>
   __device__ __forceinline__ void scores(const unsigned char* ktile, int r0, float scale,
                                          float& s0, float& s1) const {
     const int lane = threadIdx.x & 31;
@@ -135,7 +150,7 @@ struct MmaAcc {
 #pragma unroll
     for (int ks = 0; ks < D / 16; ks += 2) {
       uint32_t b[4];
-      ldsm_x4(b, ktile + tile_off(r0 + (lane & 7), 2 * ks + (lane >> 3)));
+      ldsm_x4(b, ktile + Lay::off(r0 + (lane & 7), 2 * ks + (lane >> 3)));
       mma_bf16(acc, qa0[ks], qa2[ks], b[0], b[1]);
       mma_bf16(acc, qa0[ks + 1], qa2[ks + 1], b[2], b[3]);
     }
@@ -144,6 +159,7 @@ struct MmaAcc {
   }
   // fold the warp's 8 rows r0 .. r0 + 7: s0 / s1 their scores (as above),
   // rm the rows' multipliers
+  template <class Lay = SwzTile>
   __device__ __forceinline__ void fold(const unsigned char* vtile, int r0, float s0, float s1,
                                        const RowMult* rm) {
     const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
@@ -165,7 +181,7 @@ struct MmaAcc {
 #pragma unroll
     for (int j = 0; j < D / 8; j += 4) {
       uint32_t b[4];
-      ldsm_x4_t(b, vtile + tile_off(r0 + (lane & 7), j + (lane >> 3)));
+      ldsm_x4_t(b, vtile + Lay::off(r0 + (lane & 7), j + (lane >> 3)));
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
 #pragma unroll
@@ -221,17 +237,19 @@ struct FmaAcc {
       for (int e = 0; e < 4; ++e) o[g][e] = 0.f;
     }
   }
+  template <class Lay>
   __device__ __forceinline__ static float4 chunk(const unsigned char* tile, int r, int c) {
-    return *reinterpret_cast<const float4*>(tile + tile_off(r, c));
+    return *reinterpret_cast<const float4*>(tile + Lay::off(r, c));
   }
   // scores of the warp's 8 rows into s [8][G] (shared memory of this warp)
+  template <class Lay = SwzTile>
   __device__ __forceinline__ void scores(const unsigned char* ktile, int r0, float* s) const {
     const int lane = threadIdx.x & 31, sub = lane % LPR, rs = lane / LPR;
     const int j = sub / (LPR / G);
 #pragma unroll
     for (int i = 0; i < NST; ++i) {
       const int r = RPW * i + rs;
-      const float4 x = chunk(ktile, r0 + r, sub);
+      const float4 x = chunk<Lay>(ktile, r0 + r, sub);
       float a[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -245,6 +263,7 @@ struct FmaAcc {
     }
     __syncwarp();
   }
+  template <class Lay = SwzTile>
   __device__ __forceinline__ void fold(const unsigned char* vtile, int r0, const float* s,
                                        const RowMult* rm) {
     const int lane = threadIdx.x & 31, sub = lane % LPR, rs = lane / LPR;
@@ -272,7 +291,7 @@ struct FmaAcc {
 #pragma unroll
     for (int i = 0; i < NST; ++i) {
       const int r = RPW * i + rs;
-      const float4 x = chunk(vtile, r0 + r, sub);
+      const float4 x = chunk<Lay>(vtile, r0 + r, sub);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float w = rm[r].wo * p[r][g];
@@ -1501,8 +1520,9 @@ enum RowKind { kRowNone = 0, kRowToken = 1, kRowSteady = 2, kRowFull = 3, kRowPa
 template <typename T, int D, int G>
 struct GatherSmem {
   using TS = TileShape<T, D>;
+  using GT = PadTile<TS::kRowBytes>;   // the gather's tile layout
   static constexpr int kRowsPerBlock = kGatherTiles * kTileRows;
-  static constexpr size_t kTiles = (size_t)2 * kGatherTiles * TS::kBytes;   // K and V
+  static constexpr size_t kTiles = (size_t)2 * kGatherTiles * GT::kBytes;   // K and V
   static constexpr size_t kMeta = (size_t)kRowsPerBlock * (8 + 8 + 4 + 4);
   static constexpr size_t kComb = (size_t)kConsumerWarps * G * (D + kPartStride) * 4;
   static constexpr size_t kRows = (size_t)kConsumerWarps * 8 * sizeof(RowMult);
@@ -1520,13 +1540,16 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
                    const __grid_constant__ GatherArgs A, uint32_t* status) {
   using TS = TileShape<T, D>;
   using SM = GatherSmem<T, D, G>;
+  using GT = typename SM::GT;
   constexpr bool kMma = std::is_same_v<T, __nv_bfloat16>;
   constexpr int RPB = SM::kRowsPerBlock;
+  static_assert(kGatherThreads == 2 * RPB, "one thread per row of K and of V");
   extern __shared__ __align__(16) unsigned char sh_raw[];
   __shared__ int s_rec[kInfoInts];
   __shared__ int s_last;
   __shared__ int s_bf[2];                  // first retrieved clusters of the CTA's first block and the next
   __shared__ int s_slot[kGatherRows];      // token slots of the block's token rows
+  __shared__ __align__(8) uint64_t s_gbar; // the block's row copies
   unsigned char* sh = align_smem_1024(sh_raw);
   unsigned char* tiles = sh;                                   // [K t0][K t1][V t0][V t1]
   const unsigned char** s_kp = reinterpret_cast<const unsigned char**>(tiles + SM::kTiles);
@@ -1573,6 +1596,12 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
       prefetch_l2(A.kp.bt + (int64_t)b * A.kp.max_pages + i);
 
   const int np_scan = cm.parts(b, h);   // the scan's parts of the unit
+
+  if (tid == 0) {
+    mbar_init(&s_gbar, 1);
+    mbar_init_fence();
+  }
+  uint32_t gphase = 0u;
 
   pdl_wait();   // the scan's and the steady kernel's results
   // the unit's record, and (speculatively) where the first block's token
@@ -1691,19 +1720,24 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
       s_kp[tid] = kind == kRowNone ? nullptr : kr;
       s_vp[tid] = kind == kRowNone ? nullptr : vr;
     }
-    __syncthreads();
-    // ---- gather: every 16-byte chunk of the block's key and value rows
-    for (int x = tid; x < RPB * TS::kChunks * 2; x += blockDim.x) {
-      const int mat = x / (RPB * TS::kChunks);
-      const int rr = (x - mat * RPB * TS::kChunks) / TS::kChunks;
-      const int ch = x - mat * RPB * TS::kChunks - rr * TS::kChunks;
+    const int nrows = __syncthreads_count(tid < RPB && kind != kRowNone);
+    // ---- gather: each key and value row by one bulk copy (thread t: row
+    // t % RPB of K or V), all completing on one barrier; rows past the
+    // block's are zero
+    if (tid == 0) mbar_arrive_expect(&s_gbar, (uint32_t)(2 * nrows * TS::kRowBytes));
+    {
+      const int mat = tid / RPB, rr = tid - mat * RPB;
       const unsigned char* src = mat == 0 ? s_kp[rr] : s_vp[rr];
-      unsigned char* dst = tiles + (size_t)(mat * kGatherTiles + rr / kTileRows) * TS::kBytes +
-                           tile_off(rr % kTileRows, ch);
-      if (src) cp_async16(dst, src + ch * 16);
-      else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+      unsigned char* dst = tiles + (size_t)(mat * kGatherTiles + rr / kTileRows) * GT::kBytes +
+                           GT::off(rr % kTileRows, 0);
+      if (src) {
+        bulk_load(dst, src, TS::kRowBytes, &s_gbar);
+      } else {
+#pragma unroll
+        for (int ch = 0; ch < TS::kChunks; ++ch)
+          reinterpret_cast<uint4*>(dst)[ch] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
-    cp_async_commit();
     if (kind == kRowToken) {
       s_aux[tid] = __ldg(auxp);   // the token's position in the sequence
     } else if (kind == kRowPart) {
@@ -1711,8 +1745,9 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
       // is not retrieved
       s_aux[tid] = th.picked(__ldcg(reinterpret_cast<const uint32_t*>(auxp)), (uint32_t)auxc) ? 1 : 0;
     }
-    cp_async_wait<0>();
-    __syncthreads();
+    mbar_wait(&s_gbar, gphase, status);
+    gphase ^= 1u;
+    __syncthreads();   // (the zero rows)
     // ---- attend: warp w takes rows 8w .. 8w + 7 of each tile
 #pragma unroll 1
     for (int t = 0; t < kGatherTiles; ++t) {
@@ -1736,20 +1771,21 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
         rm[lane] = m;
       }
       __syncwarp();
-      const unsigned char* kt = tiles + (size_t)t * TS::kBytes;
-      const unsigned char* vt = tiles + (size_t)(kGatherTiles + t) * TS::kBytes;
+      const unsigned char* kt = tiles + (size_t)t * GT::kBytes;
+      const unsigned char* vt = tiles + (size_t)(kGatherTiles + t) * GT::kBytes;
       if constexpr (kMma) {
         float s0, s1;
-        macc.scores(kt, 8 * warp, A.scale, s0, s1);
-        macc.fold(vt, 8 * warp, s0, s1, rm);
+        macc.template scores<GT>(kt, 8 * warp, A.scale, s0, s1);
+        macc.template fold<GT>(vt, 8 * warp, s0, s1, rm);
       } else {
         float* sc = s_sc + warp * 8 * G;
-        facc.scores(kt, 8 * warp, sc);
-        facc.fold(vt, 8 * warp, sc, rm);
+        facc.template scores<GT>(kt, 8 * warp, sc);
+        facc.template fold<GT>(vt, 8 * warp, sc, rm);
       }
       __syncwarp();
     }
-    __syncthreads();   // tiles and row data are read before the next block
+    fence_proxy_async();   // the tiles' reads and zero rows before the next block's copies
+    __syncthreads();       // tiles and row data are read before the next block
   }
   // ---- this CTA's part (its rows, plus its share of the scan's estimation
   // parts: p = j, j + n2, ...), then the unit's merge by its last CTA

@@ -789,18 +789,16 @@ __device__ __forceinline__ int rpad(int i) { return i + (i >> 5); }
 __device__ __forceinline__ void stage_round(const uint2* rec, int NC, int Tb, int r, uint2* stage) {
   const int tid = threadIdx.x;
   const int c0 = r * kTailRound;
-  csync();   // the previous round's readers are done
-#pragma unroll 1
-  for (int q0 = 0; q0 < kTailSteps; q0 += 8) {
-    uint2 v[8];
+  // (every thread's loads in flight together: one round trip)
+  uint2 v[kTailSteps];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int c = c0 + tid + (q0 + q) * kConsumers;
-      v[q] = c < NC ? __ldcg(rec + c) : make_uint2(0u, (uint32_t)Tb);
-    }
-#pragma unroll
-    for (int q = 0; q < 8; ++q) stage[rpad(tid + (q0 + q) * kConsumers)] = v[q];
+  for (int q = 0; q < kTailSteps; ++q) {
+    const int c = c0 + tid + q * kConsumers;
+    v[q] = c < NC ? __ldcg(rec + c) : make_uint2(0u, (uint32_t)Tb);
   }
+  csync();   // the previous round's readers are done
+#pragma unroll
+  for (int q = 0; q < kTailSteps; ++q) stage[rpad(tid + q * kConsumers)] = v[q];
   if (tid == 0)
     stage[rpad(kTailRound)] =
         make_uint2(0u, c0 + kTailRound < NC ? __ldcg(&rec[c0 + kTailRound].y) : (uint32_t)Tb);
@@ -871,27 +869,27 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
   const int4 h0 = __ldcg(reinterpret_cast<const int4*>(hg) + tid);
   const int4 h1 = __ldcg(reinterpret_cast<const int4*>(hg) + kConsumers + tid);
   const int n_nonc = __ldcg(I + kNonCand);
+  const int nc_first = tid < A.cap ? __ldcg(&nonc[tid].x) : -1;   // (read before the count is known)
   get_round(0);
   reinterpret_cast<int4*>(s_hist)[tid] = h0;
   reinterpret_cast<int4*>(s_hist)[kConsumers + tid] = h1;
   csync();
   // the clusters left without a non-steady token are not candidates: their
-  // keys leave the histogram and become 0 in the records (round 0 is staged
-  // again)
+  // keys leave the histogram and become 0 in the records (and in the staged
+  // round 0)
   if (n_nonc > 0) {
     for (int j = tid; j < n_nonc; j += kConsumers) {
-      const int c = __ldcg(&nonc[j].x);
+      const int c = j == tid ? nc_first : __ldcg(&nonc[j].x);
       if (c >= 0 && c < NC) {
-        const uint32_t key = __ldcg(&rec[c].x);
+        const uint32_t key = c < kTailRound ? stage[rpad(c)].x : __ldcg(&rec[c].x);
         if (key) {
           atomicSub(&s_hist[key >> kHistShift], 1);
+          if (c < kTailRound) stage[rpad(c)].x = 0u;
           __stcg(&rec[c].x, 0u);
         }
       }
     }
-    csync();   // the cleared keys are visible before the round is staged again
-    loaded = -1;
-    get_round(0);
+    csync();   // the cleared keys and counts are visible to every thread
   }
   // ---- candidates: the histogram's total (the steady kernel cleared it, and
   // the threshold bin's member count is checked against it below)

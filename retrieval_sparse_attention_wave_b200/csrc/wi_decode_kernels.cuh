@@ -952,15 +952,16 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
       for (int r = 0; r < n_rounds; ++r) {
         get_round(r);
         uint32_t m = 0u;
+        uint2 x = stage[rpad(rb)];   // each record read once: the next one's first slot ends it
 #pragma unroll 4
         for (int j = 0; j < kTailSteps; ++j) {
-          const uint2 x = stage[rpad(rb + j)];
-          const uint32_t nx = stage[rpad(rb + j + 1)].y;
+          const uint2 xn = stage[rpad(rb + j + 1)];
           const int bn = (int)(x.x >> kHistShift);
           const bool in = x.x != 0u && bn == bin1, up = x.x != 0u && bn > bin1;
           m |= (uint32_t)in << j;
           am |= (uint32_t)up << j;
-          atok += up ? (int)(nx - x.y) : 0;
+          atok += up ? (int)(xn.y - x.y) : 0;
+          x = xn;
         }
         bm1 = m;
         int2 t2;
@@ -1075,18 +1076,28 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
     } else {
       // exact: the krem-th largest (key, -id) of the threshold bin
       if (fits && nb1 <= kTailDraws) {
+        // (key, -id) as one 64-bit value (key high, the id's complement low):
+        // a member's rank is the count of larger values, one comparison each
+        unsigned long long* s_kv = s_draw;
+        if (tid < nb1) {
+          const unsigned long long cm_ = s_cand[tid];
+          s_kv[tid] = (cm_ & 0xFFFFFFFF00000000ull) | (uint32_t)~(uint32_t)cm_;
+        }
         if (tid == 0) s_ctl[2] = -1;
         csync();
         if (tid < nb1) {
-          const uint32_t km = cand_key(tid), im = cand_id(tid);
+          const unsigned long long me = s_kv[tid];
           int rank = 0;
-#pragma unroll 8
-          for (int j = 0; j < nb1; ++j) {
-            const unsigned long long cj = s_cand[j];
-            const uint32_t kj = (uint32_t)(cj >> 32);
-            rank += kj > km || (kj == km && (uint32_t)cj < im);
+#pragma unroll 4
+          for (int j = 0; j + 1 < nb1; j += 2) {
+            const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(s_kv + j);
+            rank += (v.x > me) + (v.y > me);
           }
-          if (rank == krem - 1) { s_ctl[2] = (int)im; s_ctl[3] = (int)km; }
+          if (nb1 & 1) rank += s_kv[nb1 - 1] > me;
+          if (rank == krem - 1) {
+            s_ctl[2] = (int)~(uint32_t)me;
+            s_ctl[3] = (int)(uint32_t)(me >> 32);
+          }
         }
         csync();
         thr = s_ctl[2];

@@ -892,13 +892,18 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
     csync();   // the cleared keys and counts are visible to every thread
   }
   // ---- candidates: the histogram's total (the steady kernel cleared it, and
-  // the threshold bin's member count is checked against it below)
-  int hs = 0;
+  // the threshold bin's member count is checked against it below), and a
+  // prefix over its bins from the top down (thread t: bins 2047 - 8 t ..
+  // 2040 - 8 t), from which the threshold bin is read once k is known
+  constexpr int kBpt = kHistBins / kConsumers;
+  int hc[kBpt], hs = 0;
 #pragma unroll
-  for (int i = 0; i < kHistBins / kConsumers; ++i) hs += s_hist[tid * (kHistBins / kConsumers) + i];
-  int2 tot2;
-  wscan2(make_int2(warp_sum_int(hs), 0), s_sh, &tot2);
-  const int n_cand = tot2.x;
+  for (int i = 0; i < kBpt; ++i) {
+    hc[i] = s_hist[kHistBins - 1 - kBpt * tid - i];
+    hs += hc[i];
+  }
+  int n_cand;
+  const int h_incl = cscan(hs, s_sh, &n_cand);
   const int k_req = A.topk_clusters >= 0 ? A.topk_clusters
                                          : (int)ceil(A.topk_fraction * (double)NC);
   const int k = min(max(k_req, 0), n_cand);
@@ -938,8 +943,24 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
     kstar = 1u;
     thr = INT_MAX;
   } else if (k > 0) {
-    int above;
-    bin1 = select_bin(s_hist, kHistBins, k, &above, s_sh, s_ctl);
+    // the bin holding the k-th largest key: exactly one thread's bins do
+    {
+      int acc = h_incl - hs;
+      if (acc < k && h_incl >= k) {
+#pragma unroll
+        for (int i = 0; i < kBpt; ++i) {
+          if (acc + hc[i] >= k) {
+            s_ctl[0] = kHistBins - 1 - kBpt * tid - i;
+            s_ctl[1] = acc;
+            break;
+          }
+          acc += hc[i];
+        }
+      }
+    }
+    csync();
+    bin1 = s_ctl[0];
+    const int above = s_ctl[1];
     int krem = k - above;
     const int nb1 = s_hist[bin1];
     csync();   // read by all before the radix passes reuse the histogram

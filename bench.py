@@ -467,7 +467,9 @@ def run_wave(args, rank, world, local_rank):
     lse_h = torch.empty(wl.batch, wl.n_q_heads, dtype=torch.float32).pin_memory()
     n_e2e = max(10, min(args.steps, 200))
     with torch.cuda.stream(stream):
-        for i in range(3):
+        # warm-up: every replica's call seen twice (the library captures a
+        # call's copies and kernels into a graph the second time it sees it)
+        for i in range(max(3, 2 * T.R)):
             W.decode_host(q_h, T.reps[i % T.R], params, out_h, lse_h, T.ws, stream=stream)
         stream.synchronize()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

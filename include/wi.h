@@ -339,6 +339,12 @@ wi_status wi_decode(const void *q, const wi_index *idx, const wi_decode_params *
  * valid until the stream reaches the copies; use pinned memory for
  * asynchronous copies.  Needs the workspace size wi_decode_workspace_size
  * reports (it includes the staging area).
+ * With pinned host buffers on a stream other than the legacy default one,
+ * and no stage events or score output, the second call with the same
+ * pointers, sizes and options captures the call's copies and kernels into a
+ * CUDA graph, and later such calls launch that graph (the library keeps the
+ * 16 most recently used); the result is the same.  A call on a stream that
+ * is being captured enqueues its work into that capture instead.
  */
 wi_status wi_decode_host(const void *q_host, const wi_index *idx, const wi_decode_params *p,
                          float *out_host, float *lse_host, void *ws, size_t ws_bytes,

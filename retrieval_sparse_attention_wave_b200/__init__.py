@@ -286,6 +286,13 @@ class WaveIndex:
         return self.n_kv_heads * sum(self.seq_lens[:b]) + h * self.seq_lens[b]
 
     def c_struct(self) -> WiIndex:
+        # the marshalled struct is kept while the buffers it points at are
+        # the same (a decode per layer and step marshals the same index)
+        bufs = (self.centroids, self.value_sums, self.offsets, self.perm, self.invperm,
+                self.labels, self.k_pool, self.v_pool, self.block_table)
+        sig = tuple(t.data_ptr() for t in bufs) + (self.k_pool.shape[0], self.block_table.shape[1])
+        if getattr(self, "_cs_sig", None) == sig:
+            return self._cs
         s = WiIndex()
         s.dtype = _dtype_code(self.dtype)
         s.batch = len(self.seq_lens)
@@ -306,6 +313,7 @@ class WaveIndex:
         s.n_pages = self.k_pool.shape[0]
         s.block_table = self.block_table.data_ptr()
         s.max_pages = self.block_table.shape[1]
+        self._cs, self._cs_sig = s, sig
         return s
 
 
@@ -433,6 +441,11 @@ class DecodeParams:
     scores_out: Optional[torch.Tensor] = None   # float [Hkv * sum NC_b][G], filled if given
 
     def c_struct(self, events=None) -> WiDecodeParams:
+        sig = (self.n_q_heads, self.n_sink, self.window, self.topk_clusters, self.topk_fraction,
+               self.exact_only, self.sampled, self.seed)
+        plain = events is None and self.scores_out is None
+        if plain and getattr(self, "_cs_sig", None) == sig:
+            return self._cs
         p = WiDecodeParams()
         p.n_q_heads, p.n_sink, p.window = self.n_q_heads, self.n_sink, self.window
         p.topk_clusters, p.topk_fraction = self.topk_clusters, self.topk_fraction
@@ -449,6 +462,8 @@ class DecodeParams:
             arr = (C.c_void_p * len(events))(*[e.cuda_event for e in events])
             p.stage_events = C.cast(arr, C.POINTER(C.c_void_p))
             p._keep = arr
+        if plain:
+            self._cs, self._cs_sig = p, sig
         return p
 
 

@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <map>
+#include <vector>
 #include <algorithm>
 #include <mutex>
 
@@ -270,6 +272,58 @@ Pool make_pool(const void* base, const int32_t* bt, int64_t n_pages, int max_pag
   return Pool{base, bt, n_pages, max_pages, ilog2(page)};
 }
 
+// Host-buffer decodes replayed from CUDA graphs: the copy of q in, the
+// decode's kernels and the copies of out and lse back, captured once a call
+// with the same key (every pointer, size and option the launches bake in)
+// is seen a second time, then launched as one graph.  A call on the legacy
+// default stream, on a stream that is being captured, with pageable host
+// buffers or with stage events or score output enqueues its work directly.
+struct HostGraphs {
+  std::mutex mu;
+  struct Entry {
+    cudaGraphExec_t exec;
+    uint64_t used;
+  };
+  std::map<std::vector<int64_t>, Entry> graphs;
+  std::map<std::vector<int64_t>, int> seen;
+  uint64_t tick = 0;
+};
+HostGraphs& host_graphs() {
+  static HostGraphs* g = new HostGraphs;   // (left to the process's exit)
+  return *g;
+}
+constexpr size_t kMaxHostGraphs = 16;
+
+bool host_pinned(const void* ptr) {
+  if (!ptr) return true;
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeHost;
+}
+
+std::vector<int64_t> host_graph_key(const wi_index* ix, const wi_decode_params* p, const void* ws,
+                                    size_t ws_bytes, const void* q_host, const float* out_host,
+                                    const float* lse_host) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  auto ptr = [](const void* x) { return (int64_t)reinterpret_cast<intptr_t>(x); };
+  double frac = p->topk_fraction;
+  int64_t frac_bits = 0;
+  std::memcpy(&frac_bits, &frac, sizeof(frac_bits));
+  std::vector<int64_t> k = {dev, ptr(ws), (int64_t)ws_bytes, ptr(q_host), ptr(out_host),
+                            ptr(lse_host), ix->dtype, ix->batch, ix->n_kv_heads, ix->head_dim,
+                            ix->page_size, ix->seg_len, ix->cluster_size, ptr(ix->centroids),
+                            ptr(ix->value_sums), ptr(ix->offsets), ptr(ix->perm), ptr(ix->invperm),
+                            ptr(ix->labels), ptr(ix->k_pool), ptr(ix->v_pool), ix->n_pages,
+                            ptr(ix->block_table), ix->max_pages, p->n_q_heads, p->n_sink, p->window,
+                            p->topk_clusters, frac_bits, p->exact_only, p->topk_mode, p->seed};
+  for (int b = 0; b < ix->batch; ++b) k.push_back(ix->seq_lens[b]);
+  return k;
+}
+
 wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params* p, float* out,
                       float* lse, void* ws, size_t ws_bytes, cudaStream_t s, const void* q_host,
                       float* out_host, float* lse_host) {
@@ -290,9 +344,6 @@ wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params*
     q = w + pl.off_q;
     out = reinterpret_cast<float*>(w + pl.off_out);
     lse = lse_host ? reinterpret_cast<float*>(w + pl.off_lse) : nullptr;
-    cudaError_t e = cudaMemcpyAsync(const_cast<void*>(q), q_host, nq * pl.D * esize(ix->dtype),
-                                    cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return cuda_fail(e);
   }
   DecodeArgs a{};
   a.q = q;
@@ -309,14 +360,73 @@ wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params*
   a.ws = w;
   a.stage_events = reinterpret_cast<cudaEvent_t*>(p->stage_events);
   a.scores_out = p->scores_out;
-  cudaError_t e = launch_decode(pl, a, s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (host) {
-    e = cudaMemcpyAsync(out_host, out, nq * pl.D * 4, cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess && lse_host) e = cudaMemcpyAsync(lse_host, lse, nq * 4, cudaMemcpyDeviceToHost, s);
-    if (e != cudaSuccess) return cuda_fail(e);
+  // the call's work on the stream: copies of the host buffers around the kernels
+  auto enqueue = [&]() -> cudaError_t {
+    cudaError_t e = cudaSuccess;
+    if (host)
+      e = cudaMemcpyAsync(const_cast<void*>(q), q_host, nq * pl.D * esize(ix->dtype),
+                          cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = launch_decode(pl, a, s);
+    if (e == cudaSuccess && host) {
+      e = cudaMemcpyAsync(out_host, out, nq * pl.D * 4, cudaMemcpyDeviceToHost, s);
+      if (e == cudaSuccess && lse_host)
+        e = cudaMemcpyAsync(lse_host, lse, nq * 4, cudaMemcpyDeviceToHost, s);
+    }
+    return e;
+  };
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  const bool graphable = host && s != nullptr && s != cudaStreamLegacy && !p->stage_events &&
+                         !p->scores_out && cudaStreamIsCapturing(s, &cap) == cudaSuccess &&
+                         cap == cudaStreamCaptureStatusNone && host_pinned(q_host) &&
+                         host_pinned(out_host) && host_pinned(lse_host);
+  if (graphable) {
+    HostGraphs& hg = host_graphs();
+    const std::vector<int64_t> key = host_graph_key(ix, p, ws, ws_bytes, q_host, out_host, lse_host);
+    cudaGraphExec_t exec = nullptr;
+    bool capture = false;
+    {
+      std::lock_guard<std::mutex> lock(hg.mu);
+      auto it = hg.graphs.find(key);
+      if (it != hg.graphs.end()) {
+        exec = it->second.exec;
+        it->second.used = ++hg.tick;
+      } else {
+        if (hg.seen.size() >= 1024) hg.seen.clear();
+        capture = ++hg.seen[key] >= 2;
+      }
+    }
+    if (!exec && capture) {
+      cudaGraph_t graph = nullptr;
+      cudaError_t e = cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal);
+      if (e == cudaSuccess) {
+        const cudaError_t e1 = enqueue();
+        e = cudaStreamEndCapture(s, &graph);
+        if (e == cudaSuccess) e = e1;
+      }
+      if (e == cudaSuccess && graph) e = cudaGraphInstantiate(&exec, graph, 0);
+      if (graph) cudaGraphDestroy(graph);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        exec = nullptr;   // (this call enqueues its work directly)
+      } else {
+        std::lock_guard<std::mutex> lock(hg.mu);
+        if (hg.graphs.size() >= kMaxHostGraphs) {   // the least recently used leaves
+          auto lru = hg.graphs.begin();
+          for (auto it = hg.graphs.begin(); it != hg.graphs.end(); ++it)
+            if (it->second.used < lru->second.used) lru = it;
+          cudaGraphExecDestroy(lru->second.exec);
+          hg.graphs.erase(lru);
+        }
+        hg.graphs[key] = HostGraphs::Entry{exec, ++hg.tick};
+      }
+    }
+    if (exec) {
+      const cudaError_t e = cudaGraphLaunch(exec, s);
+      return e == cudaSuccess ? WI_OK : cuda_fail(e);
+    }
   }
-  return WI_OK;
+  const cudaError_t e = enqueue();
+  return e == cudaSuccess ? WI_OK : cuda_fail(e);
 }
 
 }  // namespace

@@ -189,6 +189,34 @@ def test_decode_host_buffers_match_device_call(base):
     assert torch.equal(out_h, out_d.cpu()) and torch.equal(lse_h, lse_d.cpu())
 
 
+def test_decode_host_graph_replays_match(base):
+    """Repeated host-buffer calls with the same buffers on a side stream: the
+    second captures a graph of the copies and kernels, the later ones replay
+    it; every call's output equals the device call's, also after q changes
+    (the graph copies the host buffer's current contents)."""
+    wl, units = base
+    p = H.params_of(wl)
+    wx = H.empty_index(wl, DEV)
+    H.upload_index(wx, units)
+    ws = W.decode_workspace(wx, p)
+    q2 = (wl.q.float() * 0.5).to(wl.q.dtype)
+    ref = [W.decode(x.to(DEV), wx, p, ws=ws) for x in (wl.q, q2)]
+    torch.cuda.synchronize()
+    qh = wl.q.cpu().pin_memory()
+    out_h = torch.empty(ref[0][0].shape, dtype=torch.float32).pin_memory()
+    lse_h = torch.empty(ref[0][1].shape, dtype=torch.float32).pin_memory()
+    st = torch.cuda.Stream()
+    for i in range(5):
+        src = wl.q if i < 3 else q2
+        qh.copy_(src)
+        out_h.zero_()
+        W.decode_host(qh, wx, p, out_h, lse_h, ws, stream=st)
+        st.synchronize()
+        o, l = ref[0] if i < 3 else ref[1]
+        assert torch.equal(out_h, o.cpu()) and torch.equal(lse_h, l.cpu()), i
+    assert W.read_device_status(ws) == 0
+
+
 def test_repeat_runs_are_bit_identical(base):
     wl, units = base
     p = H.params_of(wl)

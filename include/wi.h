@@ -343,8 +343,9 @@ wi_status wi_decode(const void *q, const wi_index *idx, const wi_decode_params *
  * and no stage events or score output, the second call with the same
  * pointers, sizes and options captures the call's copies and kernels into a
  * CUDA graph, and later such calls launch that graph (the library keeps the
- * 16 most recently used); the result is the same.  A call on a stream that
- * is being captured enqueues its work into that capture instead.
+ * 16 most recently used, keyed by the current CUDA context's unique id, so a
+ * device reset never reuses one); the result is the same.  A call on a
+ * stream that is being captured enqueues its work into that capture instead.
  */
 wi_status wi_decode_host(const void *q_host, const wi_index *idx, const wi_decode_params *p,
                          float *out_host, float *lse_host, void *ws, size_t ws_bytes,

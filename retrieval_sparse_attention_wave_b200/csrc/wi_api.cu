@@ -9,6 +9,9 @@
 #include <algorithm>
 #include <mutex>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "wi.h"
 #include "wi_common.cuh"
 #include "wi_plan.h"
@@ -304,16 +307,38 @@ bool host_pinned(const void* ptr) {
   return at.type == cudaMemoryTypeHost;
 }
 
-std::vector<int64_t> host_graph_key(const wi_index* ix, const wi_decode_params* p, const void* ws,
-                                    size_t ws_bytes, const void* q_host, const float* out_host,
-                                    const float* lse_host) {
-  int dev = 0;
-  cudaGetDevice(&dev);
+// The current context's id (unique for the process's life, so a graph of a
+// context that a device reset destroyed is never handed to its successor);
+// 0 when it cannot be read (the call then enqueues its work directly).
+unsigned long long current_context_id() {
+  static std::once_flag once;
+  static PFN_cuCtxGetCurrent_v4000 get_ctx = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_ctx = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_ctx || !get_id || get_ctx(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+std::vector<int64_t> host_graph_key(unsigned long long ctx_id, const wi_index* ix,
+                                    const wi_decode_params* p, const void* ws, size_t ws_bytes,
+                                    const void* q_host, const float* out_host, const float* lse_host) {
   auto ptr = [](const void* x) { return (int64_t)reinterpret_cast<intptr_t>(x); };
   double frac = p->topk_fraction;
   int64_t frac_bits = 0;
   std::memcpy(&frac_bits, &frac, sizeof(frac_bits));
-  std::vector<int64_t> k = {dev, ptr(ws), (int64_t)ws_bytes, ptr(q_host), ptr(out_host),
+  std::vector<int64_t> k = {(int64_t)ctx_id, ptr(ws), (int64_t)ws_bytes, ptr(q_host), ptr(out_host),
                             ptr(lse_host), ix->dtype, ix->batch, ix->n_kv_heads, ix->head_dim,
                             ix->page_size, ix->seg_len, ix->cluster_size, ptr(ix->centroids),
                             ptr(ix->value_sums), ptr(ix->offsets), ptr(ix->perm), ptr(ix->invperm),
@@ -379,9 +404,11 @@ wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params*
                          !p->scores_out && cudaStreamIsCapturing(s, &cap) == cudaSuccess &&
                          cap == cudaStreamCaptureStatusNone && host_pinned(q_host) &&
                          host_pinned(out_host) && host_pinned(lse_host);
-  if (graphable) {
+  const unsigned long long ctx_id = graphable ? current_context_id() : 0;
+  if (graphable && ctx_id != 0) {
     HostGraphs& hg = host_graphs();
-    const std::vector<int64_t> key = host_graph_key(ix, p, ws, ws_bytes, q_host, out_host, lse_host);
+    const std::vector<int64_t> key =
+        host_graph_key(ctx_id, ix, p, ws, ws_bytes, q_host, out_host, lse_host);
     cudaGraphExec_t exec = nullptr;
     bool capture = false;
     {

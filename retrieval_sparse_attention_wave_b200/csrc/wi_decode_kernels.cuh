@@ -24,8 +24,9 @@
 //              2; Vortex 2.C Top-K) in its tail and writes the rows the
 //              gather reads.
 //  K2 gather   token-balanced CTAs gather the retrieved clusters' token rows
-//              and the steady rows through the block table and attend them
-//              exactly (items 1 and 2); the same pass takes back out of the
+//              and the steady rows through the block table (one bulk copy a
+//              row) and attend them exactly (items 1 and 2); the same pass
+//              takes back out of the
 //              estimate what the estimation zone does not hold (the
 //              retrieved clusters, the clusters left without a candidate
 //              token, and the steady tokens of the other affected clusters).
@@ -66,9 +67,9 @@ constexpr int kPartStride = 4;    // a softmax part of one head: {m, l, ln, -, o
 // A tile holds kTileRows rows of D elements as NB = D * sizeof(T) / 128
 // boxes of [kTileRows][128 bytes], each 128-byte swizzled: 16-byte chunk c
 // of row r sits at r * 128 + ((c ^ (r & 7)) << 4) of its box.  That is the
-// layout a SWIZZLE_128B tensor copy of a {128-byte, 64-row} box writes, and
-// the layout the gather's cp.async writes; ldmatrix reads it without bank
-// conflicts.
+// layout a SWIZZLE_128B tensor copy of a {128-byte, 64-row} box writes (the
+// scan's tiles); ldmatrix reads it without bank conflicts.  The gather's
+// tiles hold whole rows instead (PadTile below).
 template <typename T, int D>
 struct TileShape {
   static constexpr int kRowBytes = D * (int)sizeof(T);

@@ -575,6 +575,8 @@ struct ScanArgs {
   int mode;
   uint32_t seed;
   int slots;
+  int mid_ok;      // a second part buffer fits: a CTA whose chunks span units hands its
+                   // first unit's arrival to the producer warp
 };
 
 // A chunk's offsets arrive as one 1-D tensor box of kOffBox int32 that starts
@@ -657,8 +659,10 @@ struct ScanSmem {
     return r > kTailStage ? r : kTailStage;
   }
   __host__ __device__ static size_t side_bytes(int slots) { return slots * kSide; }
-  __host__ __device__ static size_t total(int slots, int exact_only) {
-    return 1024 + ring_bytes(slots, exact_only) + side_bytes(slots) + kTail + kComb + kHist16 + kRows + kSc;
+  // (mid: room for a second unit's warp parts, see ScanArgs::mid_ok)
+  __host__ __device__ static size_t total(int slots, int exact_only, int mid = 0) {
+    return 1024 + ring_bytes(slots, exact_only) + side_bytes(slots) + kTail + (mid ? 2 : 1) * kComb +
+           kHist16 + kRows + kSc;
   }
 };
 
@@ -1271,6 +1275,11 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
   __shared__ int s_ntails;
   __shared__ int s_tails[kMaxTailsPerCta];   // units whose last arrival was this CTA's
   __shared__ float* s_last_part;             // the CTA's last unit's estimation part
+  // the hand-off of the first unit's arrival to the producer warp, when the
+  // CTA's chunks span more than one unit
+  __shared__ __align__(8) uint64_t s_mid_full, s_mid_done;
+  __shared__ float* s_mid_part;
+  __shared__ int s_mid_u, s_mid_parts;
   pdl_launch_dependents();
   unsigned char* sh = align_smem_1024(sh_raw);
   const int slots = A.slots;
@@ -1279,15 +1288,28 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
   unsigned char* side0 = ring + SM::ring_bytes(slots, A.exact_only);
   unsigned char* s_tail = side0 + SM::side_bytes(slots);
   float* comb = reinterpret_cast<float*>(s_tail + SM::kTail);   // per-warp softmax parts
-  uint32_t* hist16 = reinterpret_cast<uint32_t*>(reinterpret_cast<unsigned char*>(comb) + SM::kComb);
+  float* comb2 = comb + SM::kComb / 4;                          // (of the first of two units)
+  uint32_t* hist16 = reinterpret_cast<uint32_t*>(reinterpret_cast<unsigned char*>(comb) +
+                                                 SM::kComb * (A.mid_ok ? 2 : 1));
   RowMult* s_rows = reinterpret_cast<RowMult*>(reinterpret_cast<unsigned char*>(hist16) + SM::kHist16);
   float* s_sc = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(s_rows) + SM::kRows);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int s = blockIdx.x;
   const int k0 = cm.n_chunks > 0 ? cm.k0(s) : 0, k1 = cm.n_chunks > 0 ? cm.k0(s + 1) : 0;
   const int nk = k1 - k0;
+  // chunks of the CTA's first unit; `mid`: more follow (the first unit's
+  // arrival is then the producer warp's)
+  int n1 = 0;
+  if (nk > 0) {
+    ChunkPos p1;
+    chunk_seek(p1, geo, cm, k0);
+    n1 = min(nk, p1.kend - p1.k);
+  }
+  const bool mid = A.mid_ok && n1 < nk;
   if (tid == 0) {
     for (int i = 0; i < slots; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], kConsumerWarps); }
+    mbar_init(&s_mid_full, 1);
+    mbar_init(&s_mid_done, 1);
     mbar_init_fence();
   }
   for (int i = tid; i < kHistBins / 2; i += blockDim.x) hist16[i] = 0u;
@@ -1299,12 +1321,26 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
     // key (and value-sum) tile, its offsets box, and the unit's queries when
     // the chunk starts a unit
     if (lane == 0 && nk > 0) {
+      // the first unit's arrival, once the consumers have flushed its
+      // histogram counts (they hand it over on s_mid_full)
+      auto mid_arrival = [&]() {
+        mbar_wait(&s_mid_full, 0u, status);
+        fence_acq_rel_gpu();
+        const int old = atomicAdd(A.cnt1 + s_mid_u, 1);
+        if (old == s_mid_parts - 1) {
+          fence_acq_rel_gpu();
+          s_tails[atomicAdd(&s_ntails, 1)] = s_mid_u;
+        }
+        mbar_arrive(&s_mid_done);
+      };
+      const int i_mid = n1 - 1 + slots;   // the first issue that needs the first unit's last slot
       ChunkPos p;
       chunk_seek(p, geo, cm, k0);
       int prev_u = -1;
       for (int i = 0; i < nk; ++i) {
         const int sl = i % slots;
         if (i >= slots) mbar_wait(&s_empty[sl], (uint32_t)((i / slots - 1) & 1), status);
+        if (mid && i == i_mid) mid_arrival();
         if (i > 0) chunk_next(p, geo, cm);
         const bool new_u = p.u != prev_u;
         prev_u = p.u;
@@ -1329,6 +1365,7 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
           bulk_load(side + kOffArea, qsrc, (uint32_t)SM::kQBytes, &s_full[sl]);
         }
       }
+      if (mid && i_mid >= nk) mid_arrival();
       // every copy issued has landed before the CTA may leave (bounded)
       for (int i = max(0, nk - slots); i < nk; ++i)
         mbar_wait(&s_full[i % slots], (uint32_t)((i / slots) & 1), status);
@@ -1339,6 +1376,7 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
       __syncwarp();
       named_sync(2, kScanThreads);
       combine_warps_1w<D, G>(comb, s_last_part, lane);
+      if (mid) combine_warps_1w<D, G>(comb2, s_mid_part, lane);
     }
     pdl_wait();
     return;
@@ -1479,12 +1517,29 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
     // every thread's records and histogram counts are written before the
     // barrier; one fenced arrival publishes them (a cumulative fence)
     csync();   // (and the words are clear before the next unit counts into them)
+    float* const part = A.est + ((int64_t)c.u * A.p1max + u_slot) * G * (D + kPartStride);
+    if (mid && i == n1) {
+      // the first of several units: its warps' parts wait in comb2 and the
+      // producer warp arrives for it (and combines the parts at the end)
+      if (!A.exact_only) {
+        if constexpr (kMma) macc.to_smem(comb2 + warp * G * (D + kPartStride));
+        else facc.to_smem(comb2 + warp * G * (D + kPartStride));
+      }
+      csync();
+      if (tid == 0) {
+        s_mid_part = part;
+        s_mid_u = c.u;
+        s_mid_parts = u_parts;
+        mbar_arrive(&s_mid_full);
+      }
+      continue;
+    }
     if (tid == 0) {
       fence_acq_rel_gpu();
       const int old = atomicAdd(A.cnt1 + c.u, 1);
       if (old == u_parts - 1) {
         fence_acq_rel_gpu();
-        s_tails[s_ntails++] = c.u;
+        s_tails[atomicAdd(&s_ntails, 1)] = c.u;
       }
     }
     // the estimation part is the gather's, read once the scan has completed:
@@ -1494,7 +1549,6 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
       if constexpr (kMma) macc.to_smem(comb + warp * G * (D + kPartStride));
       else facc.to_smem(comb + warp * G * (D + kPartStride));
       csync();
-      float* part = A.est + ((int64_t)c.u * A.p1max + u_slot) * G * (D + kPartStride);
       if (i < nk) {
         combine_warps<D, G>(comb, part, tid);
         csync();   // the parts are read before the next unit writes them
@@ -1506,6 +1560,7 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
   }
   // ---- the tails of the units this CTA finished last (after the loop, so
   // the accumulators are dead and the tail has the registers)
+  if (mid) mbar_wait(&s_mid_done, 0u, status);   // the producer's arrival for the first unit
   csync();
   const int nt = s_ntails;
   for (int t = 0; t < nt; ++t) {
@@ -2129,7 +2184,8 @@ cudaError_t launch_decode_typed(const DecodePlan& p, const DecodeArgs& a, const 
   A.mode = p.mode;
   A.seed = p.seed;
   A.slots = p.slots;
-  const size_t scan_smem = ScanSmem<T, D, G>::total(p.slots, p.exact_only);
+  A.mid_ok = ScanSmem<T, D, G>::total(p.slots, p.exact_only, 1) <= (size_t)227 * 1024 ? 1 : 0;
+  const size_t scan_smem = ScanSmem<T, D, G>::total(p.slots, p.exact_only, A.mid_ok);
   set_smem(wave_scan_kernel<T, D, G>, scan_smem);
   mark(1);
   cudaError_t e1 = launch_ex(wave_scan_kernel<T, D, G>, dim3(std::max(1, p.n_scan)),

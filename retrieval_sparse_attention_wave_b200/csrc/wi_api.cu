@@ -151,7 +151,11 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   }
   pl.n_chunks = pl.ch_base[B];
   pl.n_scan = std::max(1, std::min(pl.n_chunks, kNumSMs));
-  if ((int64_t)pl.n_chunks * pl.n_scan >= ((int64_t)1 << 32)) return WI_ERR_UNSUPPORTED;   // ChunkMap arithmetic
+  if ((int64_t)5 * pl.n_chunks * pl.n_scan >= ((int64_t)1 << 32)) return WI_ERR_UNSUPPORTED;   // ChunkMap arithmetic
+  // the scan CTAs launched last share their SMs with the steady kernel's U
+  // CTAs until those end: a lighter share for them, when there are chunks
+  // enough for every CTA to keep one
+  pl.n_late = pl.n_chunks >= 2 * pl.n_scan ? std::min(pl.U, pl.n_scan / 4) : 0;
   const ChunkMap cm = chunk_map(pl);
   pl.p1max = 1;
   for (int b = 0; b < B; ++b)

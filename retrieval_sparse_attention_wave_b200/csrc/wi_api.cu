@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <tuple>
 #include <vector>
 #include <algorithm>
 #include <mutex>
@@ -87,6 +88,146 @@ int64_t n_steady(int64_t T, int64_t n_sink, int64_t window) {
 
 // Chunk map of the scan: CTA that takes chunk k of n over N CTAs
 
+// The scan CTAs' chunk runs (pl.k0s).  The last `late` CTAs are launched
+// beside the steady kernel's U CTAs and start once those have left their
+// SMs: they take a share of weight 3 against 5 (when there are chunks enough
+// for every CTA to keep one).  With up to 32 units (and no more units than
+// CTAs) the runs are unit-aligned: unit u gets c_u CTAs of its own, its
+// chunks split over them by weight, and the c_u are moved one at a time
+// from the unit that loses least to the unit with the latest predicted
+// finish (a CTA's predicted finish, in chunk times: its share of its unit's
+// chunks, plus 3 for a late CTA) while the latest finish drops, so no CTA
+// ends one unit and starts another in the middle of its run.  Otherwise CTA
+// s takes chunks [n W(s) / W(N), n W(s + 1) / W(N)), W the prefix of the
+// weights.  The runs are kept by geometry.
+void balance_scan(DecodePlan& pl) {
+  const int n = pl.n_chunks, N = pl.n_scan, H = pl.geo.hkv, B = pl.geo.batch;
+  pl.k0s[0] = 0;
+  for (int s = 1; s <= kNumSMs; ++s) pl.k0s[s] = n;
+  if (n <= 0) return;
+  const int late = n >= 2 * N ? std::min(pl.U, N / 4) : 0;
+  auto weighted = [&]() {
+    const int a = N - late;
+    auto ws = [&](int s) -> uint64_t { return s <= a ? 5ull * s : 5ull * a + 3ull * (uint64_t)(s - a); };
+    for (int s = 0; s <= N; ++s) pl.k0s[s] = (int32_t)((uint64_t)n * ws(s) / ws(N));
+  };
+  std::vector<int> uf, um;   // the units with chunks: first chunk, chunks
+  for (int b = 0; b < B; ++b) {
+    const int per = (pl.ch_base[b + 1] - pl.ch_base[b]) / H;
+    for (int h = 0; h < H && per > 0; ++h) {
+      uf.push_back(pl.ch_base[b] + h * per);
+      um.push_back(per);
+    }
+  }
+  const int Uu = (int)uf.size();
+  if (Uu == 0 || Uu > 32 || Uu > N) {
+    weighted();
+    return;
+  }
+  using Key = std::tuple<std::vector<int32_t>, int, int, int>;
+  static std::mutex mu;
+  static std::map<Key, std::vector<int32_t>> memo;
+  Key key{std::vector<int32_t>(pl.ch_base, pl.ch_base + B + 1), H, N, late};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = memo.find(key);
+    if (it != memo.end()) {
+      std::copy(it->second.begin(), it->second.end(), pl.k0s);
+      return;
+    }
+  }
+  // CTAs per unit, first in proportion to its chunks
+  std::vector<int> c(Uu);
+  int sum = 0;
+  for (int i = 0; i < Uu; ++i) {
+    c[i] = std::max(1, (int)std::lround((double)N * um[i] / n));
+    sum += c[i];
+  }
+  while (sum > N) {
+    int i = 0;
+    for (int j = 1; j < Uu; ++j) if (c[j] > c[i]) i = j;
+    --c[i];
+    --sum;
+  }
+  while (sum < N) {
+    int i = 0;
+    for (int j = 1; j < Uu; ++j) if ((double)um[j] / c[j] > (double)um[i] / c[i]) i = j;
+    ++c[i];
+    ++sum;
+  }
+  // each unit's late CTAs (the last `late` of all), its predicted finish,
+  // and whether every CTA keeps a chunk
+  std::vector<double> cost(Uu);
+  auto evaluate = [&](const std::vector<int>& cc, double* worst) {
+    int F = 0;
+    *worst = 0.0;
+    bool ok = true;
+    for (int i = 0; i < Uu; ++i) {
+      const int nl = std::max(0, std::min(F + cc[i], N) - std::max(F, N - late));
+      const int nn = cc[i] - nl;
+      const double W = 5.0 * nn + 3.0 * nl;
+      double r = 0.0;
+      if (nn > 0) r = um[i] * 5.0 / W;
+      if (nl > 0) r = std::max(r, 3.0 + um[i] * 3.0 / W);
+      cost[i] = r;
+      *worst = std::max(*worst, r);
+      if (cc[i] > um[i] || (nl > 0 && um[i] * 3.0 / W < 1.0) || (nn > 0 && um[i] * 5.0 / W < 1.0))
+        ok = false;
+      F += cc[i];
+    }
+    return ok;
+  };
+  double worst;
+  if (!evaluate(c, &worst)) {
+    weighted();
+    return;
+  }
+  for (int it = 0; it < 8 * N; ++it) {
+    int imax = 0;
+    for (int i = 1; i < Uu; ++i) if (cost[i] > cost[imax]) imax = i;
+    double best = worst;
+    int bj = -1;
+    for (int j = 0; j < Uu; ++j) {
+      if (j == imax || c[j] <= 1) continue;
+      std::vector<int> c2 = c;
+      --c2[j];
+      ++c2[imax];
+      double w2;
+      if (evaluate(c2, &w2) && w2 < best - 1e-9) {
+        best = w2;
+        bj = j;
+      }
+    }
+    if (bj < 0) break;
+    --c[bj];
+    ++c[imax];
+    evaluate(c, &worst);
+  }
+  std::vector<int32_t> tab(N + 1);
+  int s = 0;
+  for (int i = 0; i < Uu; ++i) {
+    const int F = s;
+    uint64_t W = 0;
+    for (int j = 0; j < c[i]; ++j) W += F + j >= N - late ? 3 : 5;
+    uint64_t acc = 0;
+    for (int j = 0; j < c[i]; ++j) {
+      tab[s++] = uf[i] + (int32_t)((uint64_t)um[i] * acc / W);
+      acc += F + j >= N - late ? 3 : 5;
+    }
+  }
+  tab[N] = n;
+  bool ok = s == N && tab[0] == 0;
+  for (int t = 0; t < N && ok; ++t) ok = tab[t] < tab[t + 1];
+  if (!ok) {
+    weighted();
+    return;
+  }
+  std::copy(tab.begin(), tab.end(), pl.k0s);
+  std::lock_guard<std::mutex> lock(mu);
+  if (memo.size() >= 256) memo.clear();
+  memo[key] = tab;
+}
+
 wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, DecodePlan& pl) {
   if (!ix || !p) return WI_ERR_INVALID_ARG;
   wi_status st = check_common(ix->dtype, ix->batch, ix->n_kv_heads, ix->head_dim, ix->page_size,
@@ -151,11 +292,7 @@ wi_status make_decode_plan(const wi_index* ix, const wi_decode_params* p, Decode
   }
   pl.n_chunks = pl.ch_base[B];
   pl.n_scan = std::max(1, std::min(pl.n_chunks, kNumSMs));
-  if ((int64_t)5 * pl.n_chunks * pl.n_scan >= ((int64_t)1 << 32)) return WI_ERR_UNSUPPORTED;   // ChunkMap arithmetic
-  // the scan CTAs launched last share their SMs with the steady kernel's U
-  // CTAs until those end: a lighter share for them, when there are chunks
-  // enough for every CTA to keep one
-  pl.n_late = pl.n_chunks >= 2 * pl.n_scan ? std::min(pl.U, pl.n_scan / 4) : 0;
+  balance_scan(pl);
   const ChunkMap cm = chunk_map(pl);
   pl.p1max = 1;
   for (int b = 0; b < B; ++b)

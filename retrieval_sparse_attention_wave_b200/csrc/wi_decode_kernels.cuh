@@ -1275,6 +1275,7 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
   __shared__ int s_ntails;
   __shared__ int s_tails[kMaxTailsPerCta];   // units whose last arrival was this CTA's
   __shared__ float* s_last_part;             // the CTA's last unit's estimation part
+  __shared__ int32_t s_k0s[kNumSMs + 1];     // the scan CTAs' first chunks
   // the hand-off of the first unit's arrival to the producer warp, when the
   // CTA's chunks span more than one unit
   __shared__ __align__(8) uint64_t s_mid_full, s_mid_done;
@@ -1313,6 +1314,7 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
     mbar_init_fence();
   }
   for (int i = tid; i < kHistBins / 2; i += blockDim.x) hist16[i] = 0u;
+  for (int i = tid; i <= cm.n_scan; i += blockDim.x) s_k0s[i] = cm.k0s[i];
   if (tid == 0) s_ntails = 0;
   __syncthreads();
 
@@ -1398,9 +1400,9 @@ wave_scan_kernel(const __grid_constant__ Geo geo, const __grid_constant__ ChunkM
     chunk_seek(c, geo, cm, k0 + i);
     const int n_here = min(nk - i, c.kend - c.k);   // the unit's chunks in this CTA
     // this CTA's part index among the unit's scan CTAs, and their number
-    const int cf = cm.cta_of(c.kend - cm.per_unit(c.b));
+    const int cf = ChunkMap::cta_in(s_k0s, cm.n_scan, c.kend - cm.per_unit(c.b));
     const int u_slot = s - cf;
-    const int u_parts = cm.cta_of(c.kend - 1) - cf + 1;
+    const int u_parts = ChunkMap::cta_in(s_k0s, cm.n_scan, c.kend - 1) - cf + 1;
     for (int ii = 0; ii < n_here; ++ii) {
       const unsigned char* ktile = ring + sl * tile_bytes;
       const unsigned char* vtile = ktile + TS::kBytes;
@@ -1681,7 +1683,10 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
     for (int i = 32 * tid; i < A.kp.max_pages; i += 32 * kGatherThreads)
       prefetch_l2(A.kp.bt + (int64_t)b * A.kp.max_pages + i);
 
-  const int np_scan = cm.parts(b, h);   // the scan's parts of the unit
+  // the scan's parts of the unit: the scan CTAs whose chunks meet its own
+  const int u_first = cm.first(b, h), u_end = u_first + cm.per_unit(b);
+  const int np_scan = __syncthreads_count(tid < cm.n_scan && cm.k0s[tid] < u_end &&
+                                          cm.k0s[tid + 1] > u_first);
 
   if (tid == 0) {
     mbar_init(&s_gbar, 1);

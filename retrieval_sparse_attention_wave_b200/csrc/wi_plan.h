@@ -31,29 +31,23 @@ constexpr int kMaxTailsPerCta = 64;               // units one scan CTA may touc
 // The scan's work: the clusters of every unit that is not attended densely,
 // in chunks of kTileRows; sequence b's units own ch_base[b + 1] - ch_base[b]
 // chunks (Hkv units of equal count).  Scan CTA s takes the chunks
-// [k0(s), k0(s + 1)), a share of weight 5, except the last n_late CTAs,
-// which take weight 3: they are launched last and start once the steady
-// kernel's CTAs have left their SMs.  (32-bit unsigned arithmetic: the plan
-// keeps 5 n_chunks n_scan below 2^32, and sets n_late only when every CTA
-// then keeps a chunk at least.)
+// [k0s[s], k0s[s + 1]): contiguous runs in order, at least one chunk each,
+// sized on the host (balance_scan in the plan).
 struct ChunkMap {
   int32_t ch_base[kMaxBatch + 1];
   int n_chunks, n_scan, batch, hkv;
-  int n_late;
-  // weight of CTAs [0, s)
-  __host__ __device__ __forceinline__ uint32_t wsum(int s) const {
-    const int a = n_scan - n_late;
-    return s <= a ? 5u * (uint32_t)s : 5u * (uint32_t)a + 3u * (uint32_t)(s - a);
+  int32_t k0s[kNumSMs + 1];
+  __host__ __device__ __forceinline__ int k0(int s) const { return k0s[s]; }
+  // the CTA of chunk k in a table of first chunks (the last s with tab[s] <= k)
+  __host__ __device__ __forceinline__ static int cta_in(const int32_t* tab, int n_scan, int k) {
+    int lo = 0, hi = n_scan - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (tab[mid] <= k) lo = mid; else hi = mid - 1;
+    }
+    return lo;
   }
-  __host__ __device__ __forceinline__ int k0(int s) const {
-    return (int)((uint32_t)n_chunks * wsum(s) / wsum(n_scan));
-  }
-  // the scan CTA that takes chunk k: the last s with k0(s) <= k
-  __host__ __device__ __forceinline__ int cta_of(int k) const {
-    const uint32_t n = (uint32_t)n_chunks, a = (uint32_t)(n_scan - n_late);
-    const uint32_t t = (uint32_t)(k + 1) * wsum(n_scan) - 1u;
-    return t < 5u * n * a ? (int)(t / (5u * n)) : (int)(a + (t - 5u * n * a) / (3u * n));
-  }
+  __host__ __device__ __forceinline__ int cta_of(int k) const { return cta_in(k0s, n_scan, k); }
   __host__ __device__ __forceinline__ int seq_of(int k) const {
     int lo = 0, hi = batch - 1;
     while (lo < hi) {
@@ -109,7 +103,7 @@ struct DecodePlan {
   // scan (K1): chunks of kTileRows clusters of the units that are not dense
   int32_t ch_base[kMaxBatch + 1];   // chunk prefix over sequences (Hkv chunks-per-unit each)
   int n_chunks, n_scan, p1max;      // total chunks, scan CTAs, parts per unit at most
-  int n_late;                       // scan CTAs of the lighter share (ChunkMap)
+  int32_t k0s[kNumSMs + 1];         // first chunk of each scan CTA (ChunkMap)
   int slots;                        // ring slots per scan CTA
   // gather (K2): per sequence n2_b CTAs per unit
   int32_t n2_base[kMaxBatch + 1];   // CTA prefix over sequences (Hkv * n2_b each)
@@ -129,7 +123,7 @@ inline ChunkMap chunk_map(const DecodePlan& p) {
   cm.n_scan = p.n_scan > 0 ? p.n_scan : 1;
   cm.batch = p.geo.batch;
   cm.hkv = p.geo.hkv;
-  cm.n_late = p.n_late;
+  std::memcpy(cm.k0s, p.k0s, sizeof(cm.k0s));
   return cm;
 }
 // First segment each sequence's build kernels process (all zero for a full

@@ -333,18 +333,27 @@ struct FmaAcc {
 // Combine the per-warp parts comb [kConsumerWarps][G][D + 4] into one part
 // [G][D + 4] at `part` (threads 0 .. kConsumers - 1).
 template <int D, int G>
-__device__ __forceinline__ void combine_warps(float* comb, float* part, int tid) {
+__device__ __forceinline__ void combine_warps(float* comb, float* part, int tid, float* pre = nullptr) {
   constexpr int RS = D + kPartStride;
   // each head's maximum, denominators and the warps' factors (kept in each
-  // row's spare word 3) by one thread per head
+  // row's spare word 3) by one thread per head; `pre` (shared memory, the
+  // same rows), when given, is one more part to fold in
   if (tid < G) {
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * G + tid) * RS]);
+    if (pre) M = fmaxf(M, pre[tid * RS]);
     float L = 0.f, LN = 0.f;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
       float* row = comb + (w * G + tid) * RS;
+      const float f = row[0] == -INFINITY ? 0.f : __expf(row[0] - M);
+      row[3] = f;
+      L += f * row[1];
+      LN += f * row[2];
+    }
+    if (pre) {
+      float* row = pre + tid * RS;
       const float f = row[0] == -INFINITY ? 0.f : __expf(row[0] - M);
       row[3] = f;
       L += f * row[1];
@@ -363,6 +372,7 @@ __device__ __forceinline__ void combine_warps(float* comb, float* part, int tid)
       const float* row = comb + (w * G + g) * RS;
       O += row[3] * row[kPartStride + e];
     }
+    if (pre) O += pre[g * RS + 3] * pre[g * RS + kPartStride + e];
     part[g * RS + kPartStride + e] = O;
   }
 }
@@ -1882,9 +1892,14 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
   // parts: p = j, j + n2, ...), then the unit's merge by its last CTA
   if constexpr (kMma) macc.to_smem(comb + warp * G * (D + kPartStride));
   else facc.to_smem(comb + warp * G * (D + kPartStride));
+  const bool has_pre = np1 > j;               // the scan part prefetched into s_pre
+  const bool extra = j + n2 < np1;            // more scan parts than the unit's CTAs
+  if (has_pre) cp_async_wait<0>();
   __syncthreads();
-  combine_warps<D, G>(comb, s_part, tid);
-  __syncthreads();
+  float* part = A.gat + ((int64_t)u * A.n2max + j) * G * (D + kPartStride);
+  // the warps' parts and the prefetched scan part in one combine, straight
+  // into the published part (through s_part when more scan parts follow)
+  combine_warps<D, G>(comb, extra ? s_part : part, tid, has_pre ? s_pre : nullptr);
   auto fold_part = [&](const float* src) {   // s_part <- s_part (+) src (shared or global)
     if (tid < G) {
       const float ma = s_part[tid * (D + kPartStride)], mb = src[tid * (D + kPartStride)];
@@ -1906,15 +1921,12 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
     }
     __syncthreads();
   };
-  if (np1 > j) {
-    cp_async_wait<0>();   // the prefetched part (its copies were issued after the grid wait)
+  if (extra) {
     __syncthreads();
-    fold_part(s_pre);
     for (int p = j + n2; p < np1; p += n2)
       fold_part(A.est + ((int64_t)u * A.p1max + p) * G * (D + kPartStride));
+    for (int i = tid; i < G * (D + kPartStride); i += blockDim.x) part[i] = s_part[i];
   }
-  float* part = A.gat + ((int64_t)u * A.n2max + j) * G * (D + kPartStride);
-  for (int i = tid; i < G * (D + kPartStride); i += blockDim.x) part[i] = s_part[i];
   // every thread's part is written before the barrier; one fenced arrival
   // publishes it (a cumulative fence)
   __syncthreads();

@@ -1648,8 +1648,6 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
   __shared__ int s_bf[2];                  // first retrieved clusters of the CTA's first block and the next
   __shared__ int s_slot[kGatherRows];      // token slots of the block's token rows
   __shared__ __align__(8) uint64_t s_gbar; // the block's row copies
-  constexpr int kWin = 64, kWinLead = 16;  // records read with the unit's (see below)
-  __shared__ int4 s_win[kWin];
   unsigned char* sh = align_smem_1024(sh_raw);
   unsigned char* tiles = sh;                                   // [K t0][K t1][V t0][V t1]
   const unsigned char** s_kp = reinterpret_cast<const unsigned char**>(tiles + SM::kTiles);
@@ -1714,15 +1712,6 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
     const int bk = j + tid - 32;
     s_bf[tid - 32] = bk < Tb ? __ldcg(A.blkf + trow + bk) : 0;
   }
-  // and the records of the retrieved clusters around the one expected to
-  // start the first block (its rows at the unit's mean cluster size): read
-  // from here when they cover the block, from L2 otherwise
-  const int NCb = geo.NC(b);
-  const int w0 = max(0, (int)((float)(j * RPB) * ((float)NCb / (float)max(Tb, 1))) - kWinLead);
-  if (tid >= 64 && tid < 64 + kWin) {
-    const int e = w0 + tid - 64;
-    s_win[tid - 64] = e < NCb ? __ldcg(A.selinfo + row0 + e) : make_int4(0, 0, 0, 0);
-  }
   __syncthreads();
   const bool dense = s_rec[kDense] != 0, no_est = s_rec[kNoEstimate] != 0;
   // the scan's estimation parts this CTA folds into its own (p = j, j + n2,
@@ -1765,8 +1754,7 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
       if (tid < RPB) s_slot[tid] = -1;
       __syncthreads();
       for (int e = tid; e <= s_hi - s_lo; e += blockDim.x) {
-        const int c = s_lo + e;   // {id, first slot, count, first row}
-        const int4 si = (blk == j && c >= w0 && c < w0 + kWin) ? s_win[c - w0] : __ldcg(A.selinfo + row0 + c);
+        const int4 si = __ldcg(A.selinfo + row0 + s_lo + e);   // {id, first slot, count, first row}
         const int r0 = max(si.w, rb), r1 = min(min(si.w + si.z, rb + RPB), n_tok);
         for (int r = r0; r < r1; ++r) s_slot[r - rb] = si.y + (r - si.w);
       }

@@ -1938,35 +1938,50 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
   }
   __syncthreads();
   if (!s_last) return;
-  // the merge of the unit's n2 parts: their outputs are staged in shared
-  // memory by asynchronous copies (the first batch issued now, beside the
-  // loads of their (m, l, ln)), in batches of the tile area's size
+  // the merge of the unit's n2 parts.  Every part's (m, l, ln) is loaded
+  // first; then each thread's share of the parts' outputs (a 16-byte column,
+  // the threads forming kS slices of the parts) is loaded straight into
+  // registers, landing while the heads' maxima and the parts' factors form
   const int np = n2;
   auto part_ptr = [&](int p) -> const float* {
     return A.gat + ((int64_t)u * A.n2max + p) * G * (D + kPartStride);
   };
-  constexpr int kPO = G * D;                          // staged floats per part: its outputs
-  constexpr int PB = (int)(SM::kTiles / (kPO * 4));   // parts per staged batch
-  float* stage = reinterpret_cast<float*>(tiles);
-  auto stage_batch = [&](int p0, int nb) {
-    for (int x = tid; x < nb * kPO / 4; x += blockDim.x) {
-      const int pp = x / (kPO / 4), rem = x - pp * (kPO / 4);
-      const int gg = rem / (D / 4), c4 = rem - gg * (D / 4);
-      cp_async16(stage + pp * kPO + gg * D + 4 * c4,
-                 part_ptr(p0 + pp) + gg * (D + kPartStride) + kPartStride + 4 * c4);
-    }
-    cp_async_commit();
+  constexpr int C4 = G * D / 4;                     // 16-byte columns of a part's outputs
+  static_assert(kGatherThreads % C4 == 0, "the columns tile the CTA");
+  constexpr int kS = kGatherThreads / C4;           // part slices
+  constexpr int kB = 16;                            // parts a thread holds in registers
+  constexpr int kF = (kMaxGatherPerUnit * G + kGatherThreads - 1) / kGatherThreads;
+  const int c4 = tid % C4, sl = tid / C4;
+  const int gq = c4 / (D / 4), e4 = c4 - gq * (D / 4);   // the column's head and offset
+  const int64_t qh = (int64_t)b * A.Hq + (int64_t)h * G + gq;
+  float* outp = A.out + qh * D + 4 * e4;
+  float* lsep = A.lse;
+  asm volatile("" : "+l"(outp), "+l"(lsep));   // the parameters are read now, off the tail
+  auto col = [&](int p) {
+    return __ldcg(reinterpret_cast<const float4*>(part_ptr(p) + gq * (D + kPartStride) + kPartStride) + e4);
   };
-  stage_batch(0, min(PB, np));
+  float4 fm[kF];
+#pragma unroll
+  for (int k = 0; k < kF; ++k) {
+    const int x = tid + k * kGatherThreads;
+    if (x < np * G)
+      fm[k] = __ldcg(reinterpret_cast<const float4*>(part_ptr(x / G) + (x % G) * (D + kPartStride)));
+  }
+  float4 ov[kB];
+#pragma unroll
+  for (int i = 0; i < kB; ++i)
+    if (sl + i * kS < np) ov[i] = col(sl + i * kS);
   float* s_f = s_merge;                             // [kMergeParts][G] (m then factor, l, ln)
   float* s_M = s_merge + SM::kMergeParts * G * 3;   // [G] max, [G] denominator
   float* s_L = s_M + G;
-  for (int x = tid; x < np * G; x += blockDim.x) {
-    const int p = x / G, gg = x - p * G;
-    const float* pp = part_ptr(p) + gg * (D + kPartStride);
-    s_f[3 * x] = __ldcg(pp);
-    s_f[3 * x + 1] = __ldcg(pp + 1);
-    s_f[3 * x + 2] = __ldcg(pp + 2);
+#pragma unroll
+  for (int k = 0; k < kF; ++k) {
+    const int x = tid + k * kGatherThreads;
+    if (x < np * G) {
+      s_f[3 * x] = fm[k].x;
+      s_f[3 * x + 1] = fm[k].y;
+      s_f[3 * x + 2] = fm[k].z;
+    }
   }
   __syncthreads();
   if (warp < G) {   // warp g: head g's max, the parts' factors, the denominator
@@ -1993,38 +2008,49 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
       if (LN > kCancelRatio * fmaxf(L, 0.f)) flag_error(status, WI_DEV_CANCELLATION);
     }
   }
-  constexpr int kOut = (G * D + kGatherThreads - 1) / kGatherThreads;
-  float O[kOut];
+  __syncthreads();
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto fold = [&](int p0) {
 #pragma unroll
-  for (int k = 0; k < kOut; ++k) O[k] = 0.f;
-  for (int p0 = 0; p0 < np; p0 += PB) {
-    const int nb = min(PB, np - p0);
-    if (p0 > 0) {
-      __syncthreads();   // the previous batch is read
-      stage_batch(p0, nb);
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < kOut; ++k) {
-      const int i = tid + k * kGatherThreads;
-      if (i < G * D) {
-        const int gg = i / D, e = i - gg * D;
-        for (int p = 0; p < nb; ++p)
-          O[k] += s_f[3 * ((p0 + p) * G + gg)] * stage[p * kPO + gg * D + e];
+    for (int i = 0; i < kB; ++i) {
+      const int p = p0 + sl + i * kS;
+      if (p < np) {
+        const float f = s_f[3 * (p * G + gq)];
+        o.x += f * ov[i].x;
+        o.y += f * ov[i].y;
+        o.z += f * ov[i].z;
+        o.w += f * ov[i].w;
       }
     }
-  }
+  };
+  fold(0);
+  for (int p0 = kB * kS; p0 < np; p0 += kB * kS) {   // parts beyond the registers' batch
 #pragma unroll
-  for (int k = 0; k < kOut; ++k) {
-    const int i = tid + k * kGatherThreads;
-    if (i < G * D) {
-      const int gg = i / D, e = i - gg * D;
-      const float L = s_L[gg];
-      const int64_t qh = (int64_t)b * A.Hq + (int64_t)h * G + gg;
-      A.out[qh * D + e] = L > 0.f ? O[k] / L : 0.f;
-      if (e == 0 && A.lse) A.lse[qh] = L > 0.f ? s_M[gg] + logf(L) : -INFINITY;
-    }
+    for (int i = 0; i < kB; ++i)
+      if (p0 + sl + i * kS < np) ov[i] = col(p0 + sl + i * kS);
+    fold(p0);
+  }
+  if constexpr (kS > 1) {   // the slices' sums (the tile area is free by now)
+    float4* red = reinterpret_cast<float4*>(tiles);
+    if (sl > 0) red[(sl - 1) * C4 + c4] = o;
+    __syncthreads();
+    if (sl == 0)
+#pragma unroll
+      for (int k = 1; k < kS; ++k) {
+        const float4 r = red[(k - 1) * C4 + c4];
+        o.x += r.x;
+        o.y += r.y;
+        o.z += r.z;
+        o.w += r.w;
+      }
+  }
+  if (sl == 0) {
+    const float L = s_L[gq];
+    outp[0] = L > 0.f ? o.x / L : 0.f;
+    outp[1] = L > 0.f ? o.y / L : 0.f;
+    outp[2] = L > 0.f ? o.z / L : 0.f;
+    outp[3] = L > 0.f ? o.w / L : 0.f;
+    if (e4 == 0 && lsep) lsep[qh] = L > 0.f ? s_M[gq] + logf(L) : -INFINITY;
   }
   if (tid == 0) A.cnt2[u] = 0;   // clean for the next call
 }

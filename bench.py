@@ -569,7 +569,10 @@ def run_wave(args, rank, world, local_rank):
         "gpu_launches": nst * args.steps,
         "e2e": {"value": e2e_us, "unit": UNIT,
                 "h2d_bytes_per_step": int(q_h.numel() * q_h.element_size()),
-                "d2h_bytes_per_step": int(out_h.numel() * 4 + lse_h.numel() * 4)},
+                "d2h_bytes_per_step": int(out_h.numel() * 4 + lse_h.numel() * 4),
+                "path": "wi_decode_host: q copied host to device; out and lse written by the "
+                        "kernels into the pinned, device-mapped host buffers; a synchronise "
+                        "per step"},
         "build": {"ms": build_ms, "iters": wl.iters, "assign_tflop": assign_flop / 1e12,
                   "assign_tflops_achieved": assign_flop / (build_ms * 1e-3) / 1e12,
                   "assign_round_us": assign_us,

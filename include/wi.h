@@ -335,9 +335,12 @@ wi_status wi_decode(const void *q, const wi_index *idx, const wi_decode_params *
 /*
  * wi_decode with host buffers: copies q (host [B][Hq][d], KV dtype) into the
  * workspace, decodes, and copies out (host float [B][Hq][d]) and lse (host
- * float [B][Hq], nullable) back, all on `stream`.  The host buffers must stay
- * valid until the stream reaches the copies; use pinned memory for
- * asynchronous copies.  Needs the workspace size wi_decode_workspace_size
+ * float [B][Hq], nullable) back, all on `stream`.  When out (and lse, if
+ * given) are pinned, device-mapped host memory (as cudaHostAlloc returns on
+ * a unified-address system), the kernels write them directly through their
+ * device addresses instead, and they are complete once the stream passes
+ * the call.  The host buffers must stay valid until the stream has passed
+ * the call; use pinned memory for asynchronous copies.  Needs the workspace size wi_decode_workspace_size
  * reports (it includes the staging area).
  * With pinned host buffers on a stream other than the legacy default one,
  * and no stage events or score output, the second call with the same

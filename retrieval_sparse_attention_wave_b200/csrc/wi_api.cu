@@ -438,6 +438,17 @@ HostGraphs& host_graphs() {
 }
 constexpr size_t kMaxHostGraphs = 16;
 
+// The device address of a pinned, device-mapped host buffer, else null.
+void* mapped_device_ptr(const void* ptr) {
+  if (!ptr) return nullptr;
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
 bool host_pinned(const void* ptr) {
   if (!ptr) return true;
   cudaPointerAttributes at{};
@@ -506,10 +517,22 @@ wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params*
   if ((st = check_ws(ws, ws_bytes, pl.total)) != WI_OK) return st;
   unsigned char* w = static_cast<unsigned char*>(ws);
   const size_t nq = (size_t)ix->batch * p->n_q_heads;
+  // out and lse: written by the kernels straight into the caller's host
+  // buffers when both are pinned and device-mapped, else into the
+  // workspace and copied back
+  bool direct_out = false;
   if (host) {
     q = w + pl.off_q;
-    out = reinterpret_cast<float*>(w + pl.off_out);
-    lse = lse_host ? reinterpret_cast<float*>(w + pl.off_lse) : nullptr;
+    float* out_dev = static_cast<float*>(mapped_device_ptr(out_host));
+    float* lse_dev = static_cast<float*>(mapped_device_ptr(lse_host));
+    direct_out = out_dev && (!lse_host || lse_dev);
+    if (direct_out) {
+      out = out_dev;
+      lse = lse_dev;
+    } else {
+      out = reinterpret_cast<float*>(w + pl.off_out);
+      lse = lse_host ? reinterpret_cast<float*>(w + pl.off_lse) : nullptr;
+    }
   }
   DecodeArgs a{};
   a.q = q;
@@ -533,7 +556,7 @@ wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params*
       e = cudaMemcpyAsync(const_cast<void*>(q), q_host, nq * pl.D * esize(ix->dtype),
                           cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) e = launch_decode(pl, a, s);
-    if (e == cudaSuccess && host) {
+    if (e == cudaSuccess && host && !direct_out) {
       e = cudaMemcpyAsync(out_host, out, nq * pl.D * 4, cudaMemcpyDeviceToHost, s);
       if (e == cudaSuccess && lse_host)
         e = cudaMemcpyAsync(lse_host, lse, nq * 4, cudaMemcpyDeviceToHost, s);
@@ -548,8 +571,8 @@ wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params*
   const unsigned long long ctx_id = graphable ? current_context_id() : 0;
   if (graphable && ctx_id != 0) {
     HostGraphs& hg = host_graphs();
-    const std::vector<int64_t> key =
-        host_graph_key(ctx_id, ix, p, ws, ws_bytes, q_host, out_host, lse_host);
+    std::vector<int64_t> key = host_graph_key(ctx_id, ix, p, ws, ws_bytes, q_host, out_host, lse_host);
+    key.push_back(direct_out ? 1 : 0);
     cudaGraphExec_t exec = nullptr;
     bool capture = false;
     {

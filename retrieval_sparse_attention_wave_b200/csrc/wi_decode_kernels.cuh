@@ -2046,10 +2046,18 @@ wave_gather_kernel(const __grid_constant__ Geo geo, const __grid_constant__ Chun
   }
   if (sl == 0) {
     const float L = s_L[gq];
-    outp[0] = L > 0.f ? o.x / L : 0.f;
-    outp[1] = L > 0.f ? o.y / L : 0.f;
-    outp[2] = L > 0.f ? o.z / L : 0.f;
-    outp[3] = L > 0.f ? o.w / L : 0.f;
+    const float4 r = make_float4(L > 0.f ? o.x / L : 0.f, L > 0.f ? o.y / L : 0.f, L > 0.f ? o.z / L : 0.f,
+                                 L > 0.f ? o.w / L : 0.f);
+    // one 16-byte store where the output allows it (whole lines, also when
+    // the output is the caller's mapped host buffer)
+    if ((reinterpret_cast<uintptr_t>(outp) & 15) == 0) {
+      *reinterpret_cast<float4*>(outp) = r;
+    } else {
+      outp[0] = r.x;
+      outp[1] = r.y;
+      outp[2] = r.z;
+      outp[3] = r.w;
+    }
     if (e4 == 0 && lsep) lsep[qh] = L > 0.f ? s_M[gq] + logf(L) : -INFINITY;
   }
   if (tid == 0) A.cnt2[u] = 0;   // clean for the next call

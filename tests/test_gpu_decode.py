@@ -189,6 +189,37 @@ def test_decode_host_buffers_match_device_call(base):
     assert torch.equal(out_h, out_d.cpu()) and torch.equal(lse_h, lse_d.cpu())
 
 
+def test_decode_host_pageable_and_unaligned_outputs(base):
+    """Pageable host buffers take the copy path; pinned outputs that are
+    only 4-byte aligned are written directly, by scalar stores.  Both give
+    the device call's result bit for bit."""
+    wl, units = base
+    p = H.params_of(wl)
+    wx = H.empty_index(wl, DEV)
+    H.upload_index(wx, units)
+    ws = W.decode_workspace(wx, p)
+    out_d, lse_d = W.decode(wl.q.to(DEV), wx, p, ws=ws)
+    torch.cuda.synchronize()
+    n, m = out_d.numel(), lse_d.numel()
+    out_h = torch.full(out_d.shape, float("nan"), dtype=torch.float32)
+    lse_h = torch.full(lse_d.shape, float("nan"), dtype=torch.float32)
+    W.decode_host(wl.q.cpu(), wx, p, out_h, lse_h, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h, out_d.cpu()) and torch.equal(lse_h, lse_d.cpu())
+    buf = torch.full((n + m + 2,), float("nan"), dtype=torch.float32).pin_memory()
+    out_u = buf[1:1 + n].view(out_d.shape)          # 4 bytes past a 16-byte boundary
+    lse_u = buf[1 + n:1 + n + m].view(lse_d.shape)
+    W.decode_host(wl.q.cpu().pin_memory(), wx, p, out_u, lse_u, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out_u, out_d.cpu()) and torch.equal(lse_u, lse_d.cpu())
+    assert torch.isnan(buf[0]) and torch.isnan(buf[-1])   # nothing written outside
+    out_x = torch.full((n + 1,), float("nan"), dtype=torch.float32, device=DEV)[1:].view(out_d.shape)
+    W.decode(wl.q.to(DEV), wx, p, out=out_x, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out_x, out_d)
+    assert W.read_device_status(ws) == 0
+
+
 def test_decode_host_graph_replays_match(base):
     """Repeated host-buffer calls with the same buffers on a side stream: the
     second captures a graph of the copies and kernels, the later ones replay

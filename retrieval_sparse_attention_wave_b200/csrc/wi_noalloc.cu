@@ -27,26 +27,36 @@ static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 // Device address of g_scratch per CUDA context.  In host code the name
 // g_scratch is only a host-side stand-in, so the address is looked up once
-// per context with that context current.  Keying by context (not device
-// number) makes a context created after a device reset look the address up
+// per context with that context current.  Keying by the context's unique id
+// (not the device number, nor the context handle, which a context created
+// after a device reset may reuse) makes such a context look the address up
 // again instead of reusing a stale one.
 constexpr int kMaxContexts = 64;
 std::mutex g_mu;
-CUcontext g_ctx[kMaxContexts];
+unsigned long long g_ctx[kMaxContexts];
 void* g_ptr[kMaxContexts];
 int g_n = 0;
 
-PFN_cuCtxGetCurrent_v4000 ctx_fn() {
+// The current context's unique id, or 0 when it cannot be read.
+unsigned long long current_ctx_id() {
   static std::once_flag once;
-  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static PFN_cuCtxGetCurrent_v4000 get_ctx = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
   std::call_once(once, [] {
     void* f = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+      get_ctx = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
   });
-  return fn;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_ctx || !get_id || get_ctx(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
 }
 
 wi_status scratch_ptr(void** out) {
@@ -54,9 +64,8 @@ wi_status scratch_ptr(void** out) {
   if (cudaGetDevice(&dev) != cudaSuccess) return WI_ERR_CUDA;
   // make the device's primary context current (a no-op when it already is)
   if (cudaFree(nullptr) != cudaSuccess) return WI_ERR_CUDA;
-  auto fn = ctx_fn();
-  CUcontext ctx = nullptr;
-  if (!fn || fn(&ctx) != CUDA_SUCCESS || !ctx) return WI_ERR_CUDA;
+  const unsigned long long ctx = current_ctx_id();
+  if (ctx == 0) return WI_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
   for (int i = 0; i < g_n; ++i)
     if (g_ctx[i] == ctx) { *out = g_ptr[i]; return WI_OK; }

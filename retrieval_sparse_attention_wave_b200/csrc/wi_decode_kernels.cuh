@@ -635,6 +635,7 @@ __device__ __forceinline__ void chunk_next(ChunkPos& p, const Geo& geo, const Ch
 constexpr int kTailSteps = 32;                       // records per consumer lane and round
 constexpr int kTailRound = kConsumers * kTailSteps;  // 8192 records per round
 constexpr int kTailDraws = 256;                      // threshold bins ranked member by member
+static_assert(kTailDraws % 16 == 0 && kTailDraws <= kConsumers, "the rank rounds read 16 values; a thread per value");
 // a round of records (and the next one) staged in shared memory, one pad
 // record per 32 (the ring, once the chunks are done)
 constexpr size_t kTailStage = ((size_t)(kTailRound + kTailRound / 32 + 2) * 8 + 1023) / 1024 * 1024;
@@ -1114,22 +1115,29 @@ __device__ __forceinline__ void scan_tail(const TailUnit tu, const ScanArgs& A, 
       if (fits && nb1 <= kTailDraws) {
         // (key, -id) as one 64-bit value (key high, the id's complement low):
         // a member's rank is the count of larger values, one comparison each
+        // Padded with zeros (below every member, whose key is nonzero) to a
+        // multiple of 16, read 16 values a round with all loads in flight.
         unsigned long long* s_kv = s_draw;
+        const int nbp = (nb1 + 15) & ~15;   // <= kTailDraws, a multiple of 16
         if (tid < nb1) {
           const unsigned long long cm_ = s_cand[tid];
           s_kv[tid] = (cm_ & 0xFFFFFFFF00000000ull) | (uint32_t)~(uint32_t)cm_;
+        } else if (tid < nbp) {
+          s_kv[tid] = 0ull;
         }
         if (tid == 0) s_ctl[2] = -1;
         csync();
         if (tid < nb1) {
           const unsigned long long me = s_kv[tid];
           int rank = 0;
-#pragma unroll 4
-          for (int j = 0; j + 1 < nb1; j += 2) {
-            const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(s_kv + j);
-            rank += (v.x > me) + (v.y > me);
+#pragma unroll 1
+          for (int j = 0; j < nbp; j += 16) {
+            ulonglong2 v[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) v[t] = *reinterpret_cast<const ulonglong2*>(s_kv + j + 2 * t);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) rank += (v[t].x > me) + (v[t].y > me);
           }
-          if (nb1 & 1) rank += s_kv[nb1 - 1] > me;
           if (rank == krem - 1) {
             s_ctl[2] = (int)~(uint32_t)me;
             s_ctl[3] = (int)(uint32_t)(me >> 32);

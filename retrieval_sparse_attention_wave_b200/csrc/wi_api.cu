@@ -521,11 +521,13 @@ wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params*
   // buffers when both are pinned and device-mapped, else into the
   // workspace and copied back
   bool direct_out = false;
+  bool outs_pinned = false;   // out_host and lse_host (if given) pinned and mapped
   if (host) {
     q = w + pl.off_q;
     float* out_dev = static_cast<float*>(mapped_device_ptr(out_host));
     float* lse_dev = static_cast<float*>(mapped_device_ptr(lse_host));
     direct_out = out_dev && (!lse_host || lse_dev);
+    outs_pinned = direct_out;
     if (direct_out) {
       out = out_dev;
       lse = lse_dev;
@@ -566,8 +568,7 @@ wi_status decode_impl(const void* q, const wi_index* ix, const wi_decode_params*
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   const bool graphable = host && s != nullptr && s != cudaStreamLegacy && !p->stage_events &&
                          !p->scores_out && cudaStreamIsCapturing(s, &cap) == cudaSuccess &&
-                         cap == cudaStreamCaptureStatusNone && host_pinned(q_host) &&
-                         host_pinned(out_host) && host_pinned(lse_host);
+                         cap == cudaStreamCaptureStatusNone && host_pinned(q_host) && outs_pinned;
   const unsigned long long ctx_id = graphable ? current_context_id() : 0;
   if (graphable && ctx_id != 0) {
     HostGraphs& hg = host_graphs();
